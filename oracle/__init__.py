@@ -1,0 +1,5 @@
+"""fp64 CPU oracle of the DART layer -- test infrastructure only.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The CUDA library never does.
+"""

@@ -1,0 +1,386 @@
+/*
+ * dart_oracle.c -- plain, slow, fp64 CPU oracle for the DART layer.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may call, link or
+ * load this file: it exists so that tests/, the smoke check and the CPU
+ * baseline leg of the benchmark can compare the CUDA library against an
+ * obviously-correct restatement of the method.  It shares no code, header,
+ * table or constant with the CUDA library.
+ *
+ * What it computes, and where the pages define it:
+ *
+ *  - The selective-SSM recurrence of Mamba-2 (the SSD view, Eq. (4), cited by
+ *    the Pith review of DART, "Axiom & Free-Parameter Ledger", to Dao & Gu,
+ *    "Transformers are SSMs", 2024):
+ *        H_t = exp(dt_t * A_h) * H_{t-1} + dt_t * B_t x_t^T      (N x P)
+ *        y_t = H_t^T C_t                                         (P)
+ *    run token by token, never chunked.  The state read at token t already
+ *    includes token t.
+ *
+ *  - The chunk state contribution dH[c] in R^{N x P}: the part of the
+ *    chunk-boundary state that chunk c itself contributes (Pith review, "What
+ *    carries the argument"; referee major comment 3 on Eq. (8): "the
+ *    contribution at the chunk boundary").  Computed with a second accumulator
+ *    that restarts from zero at the first token of every chunk and follows
+ *    the same update rule; at the chunk's last token it equals dH[c], and H at
+ *    that token is the boundary state states[c].
+ *
+ *  - State-memory attention (Pith review, "Core claim" and "What carries the
+ *    argument"; referee report summary; SMA Eqs. (5)-(10)): for token t in
+ *    chunk k(t) = t / S and every earlier chunk c < k(t),
+ *        value  v_{t,c} = C_t^T dH[c]              (read from the left, P)
+ *        key    k_{t,c} = dH[c] E_t                (value axis contracted, N)
+ *        score  s_{t,c} = Q_t . k_{t,c} / sqrt(N)
+ *    then a softmax over c and o_t = sum_c p_{t,c} v_{t,c}.  Memories are the
+ *    raw dH[c] with no inter-chunk decay (referee major comment 3).  A token
+ *    in chunk 0 has no memory and gets o_t = 0.
+ *
+ *  - The gated residual y_t = y_ssd_t + g * o_t with one scalar g (Pith
+ *    review, "Core claim": a zero-initialised scalar gate added to the SSM
+ *    output).
+ *
+ *  - One decode step: the same per-token rules for a single new token against
+ *    a cache of completed chunk memories; when the token closes its chunk the
+ *    running contribution is appended to the cache after the token's output
+ *    is formed (DART abstract; Pith review "If this is right": the
+ *    length-dependent inference cache is the set of chunk memories).
+ *
+ * Readings where the pages are silent: mask c < k(t) (strict), scale 1/sqrt(N),
+ * exp(dt*A) discretisation with input dt*B x^T, no D skip, ngroups = 1 (B and C
+ * shared by all heads), o_t = 0 with no memory.
+ *
+ * Layouts (row-major, last index fastest):
+ *   x[B,L,H,P] dt[B,L,H] A[H] Bm[B,L,N] Cm[B,L,N] Q[B,L,H,N] E[B,L,H,P]
+ *   y[B,L,H,P] dH[B,H,C,N,P] states[B,H,C,N,P] init_state[B,H,N,P]
+ * Inputs are float (bf16 inputs are exact in float); all arithmetic and every
+ * output is double.
+ *
+ * Parallelism: independent (batch, head) problems are split over pthreads;
+ * inside one problem the arithmetic runs in the order written above.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+typedef struct {
+    int batch, seqlen, nheads, headdim, dstate, chunk;
+} oracle_dims;
+
+/* ------------------------------------------------------------------ */
+/* a tiny work splitter over (batch, head) problems                    */
+/* ------------------------------------------------------------------ */
+typedef void (*unit_fn)(void* ctx, int unit);
+
+typedef struct {
+    unit_fn fn;
+    void* ctx;
+    int nunits, stride, first;
+} worker_arg;
+
+static void* worker_main(void* p) {
+    worker_arg* w = (worker_arg*)p;
+    for (int u = w->first; u < w->nunits; u += w->stride) w->fn(w->ctx, u);
+    return NULL;
+}
+
+static void run_units(unit_fn fn, void* ctx, int nunits, int nthreads) {
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > nunits) nthreads = nunits;
+    if (nthreads <= 1) {
+        for (int u = 0; u < nunits; ++u) fn(ctx, u);
+        return;
+    }
+    pthread_t* th = (pthread_t*)malloc(sizeof(pthread_t) * (size_t)nthreads);
+    worker_arg* wa = (worker_arg*)malloc(sizeof(worker_arg) * (size_t)nthreads);
+    for (int i = 0; i < nthreads; ++i) {
+        wa[i].fn = fn; wa[i].ctx = ctx; wa[i].nunits = nunits;
+        wa[i].stride = nthreads; wa[i].first = i;
+        pthread_create(&th[i], NULL, worker_main, &wa[i]);
+    }
+    for (int i = 0; i < nthreads; ++i) pthread_join(th[i], NULL);
+    free(th);
+    free(wa);
+}
+
+/* ------------------------------------------------------------------ */
+/* 1 + 2: token-by-token recurrence, chunk contributions, boundary states */
+/* ------------------------------------------------------------------ */
+typedef struct {
+    const oracle_dims* d;
+    const float *x, *dt, *A, *Bm, *Cm;
+    const double* init_state;
+    double *y, *dH, *states;
+} scan_ctx;
+
+static void scan_unit(void* vctx, int unit) {
+    scan_ctx* c = (scan_ctx*)vctx;
+    const oracle_dims* d = c->d;
+    const int L = d->seqlen, H = d->nheads, P = d->headdim, N = d->dstate, S = d->chunk;
+    const int nchunks = L / S;
+    const int b = unit / H, h = unit % H;
+    double* Hs = (double*)calloc((size_t)N * P, sizeof(double)); /* recurrent state  */
+    double* D = (double*)calloc((size_t)N * P, sizeof(double));  /* chunk contribution */
+    if (c->init_state) {
+        const double* h0 = c->init_state + ((size_t)b * H + h) * N * P;
+        for (int i = 0; i < N * P; ++i) Hs[i] = h0[i];
+    }
+    const double Ah = (double)c->A[h];
+    for (int t = 0; t < L; ++t) {
+        const double dtt = (double)c->dt[((size_t)b * L + t) * H + h];
+        const double decay = exp(dtt * Ah);
+        const float* Bt = c->Bm + ((size_t)b * L + t) * N;
+        const float* Ct = c->Cm + ((size_t)b * L + t) * N;
+        const float* xt = c->x + (((size_t)b * L + t) * H + h) * P;
+        if (t % S == 0) memset(D, 0, sizeof(double) * (size_t)N * P);
+        for (int n = 0; n < N; ++n) {
+            for (int p = 0; p < P; ++p) {
+                const double inp = dtt * (double)Bt[n] * (double)xt[p];
+                Hs[n * P + p] = decay * Hs[n * P + p] + inp;
+                D[n * P + p] = decay * D[n * P + p] + inp;
+            }
+        }
+        double* yt = c->y + (((size_t)b * L + t) * H + h) * P;
+        for (int p = 0; p < P; ++p) {
+            double acc = 0.0;
+            for (int n = 0; n < N; ++n) acc += (double)Ct[n] * Hs[n * P + p];
+            yt[p] = acc;
+        }
+        if (t % S == S - 1) {
+            const int ck = t / S;
+            const size_t off = (((size_t)b * H + h) * nchunks + ck) * (size_t)N * P;
+            if (c->dH) memcpy(c->dH + off, D, sizeof(double) * (size_t)N * P);
+            if (c->states) memcpy(c->states + off, Hs, sizeof(double) * (size_t)N * P);
+        }
+    }
+    free(Hs);
+    free(D);
+}
+
+/* Returns 0 on success, -1 on a shape it does not accept. */
+int oracle_ssd_scan(const oracle_dims* d, const float* x, const float* dt, const float* A,
+                    const float* Bm, const float* Cm, const double* init_state,
+                    double* y_ssd, double* dH, double* states, int nthreads) {
+    if (!d || d->chunk <= 0 || d->seqlen % d->chunk != 0) return -1;
+    scan_ctx c = {d, x, dt, A, Bm, Cm, init_state, y_ssd, dH, states};
+    run_units(scan_unit, &c, d->batch * d->nheads, nthreads);
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* 3 + 4: state-memory attention, naive per (t, c), and the gate        */
+/* ------------------------------------------------------------------ */
+typedef struct {
+    const oracle_dims* d;
+    const float *Q, *E, *Cm;
+    const double* dH;
+    double g;
+    const double* y_ssd; /* nullable; indexed like the output rows */
+    double* o;           /* nullable: raw readout o_t              */
+    double* y;           /* nullable: y_ssd + g * o_t              */
+    double* scores;      /* nullable: [B,H,L,C], NaN where masked   */
+    const int* tokens;   /* nullable: sample of token positions     */
+    int ntok;
+} sma_ctx;
+
+static void sma_unit(void* vctx, int unit) {
+    sma_ctx* c = (sma_ctx*)vctx;
+    const oracle_dims* d = c->d;
+    const int L = d->seqlen, H = d->nheads, P = d->headdim, N = d->dstate, S = d->chunk;
+    const int nchunks = L / S;
+    const int b = unit / H, h = unit % H;
+    const int nrows = c->tokens ? c->ntok : L;
+    double* key = (double*)malloc(sizeof(double) * (size_t)N);
+    double* val = (double*)malloc(sizeof(double) * (size_t)nchunks * P);
+    double* sc = (double*)malloc(sizeof(double) * (size_t)nchunks);
+    double* o = (double*)malloc(sizeof(double) * (size_t)P);
+    const double inv_sqrt_n = 1.0 / sqrt((double)N);
+    for (int r = 0; r < nrows; ++r) {
+        const int t = c->tokens ? c->tokens[r] : r;
+        const int k = t / S; /* chunk holding t; memories are c < k */
+        const float* Qt = c->Q + (((size_t)b * L + t) * H + h) * N;
+        const float* Et = c->E + (((size_t)b * L + t) * H + h) * P;
+        const float* Ct = c->Cm + ((size_t)b * L + t) * N;
+        for (int cc = 0; cc < k; ++cc) {
+            const double* M = c->dH + (((size_t)b * H + h) * nchunks + cc) * (size_t)N * P;
+            /* key = dH[c] E_t */
+            for (int n = 0; n < N; ++n) {
+                double acc = 0.0;
+                for (int p = 0; p < P; ++p) acc += M[n * P + p] * (double)Et[p];
+                key[n] = acc;
+            }
+            /* value = C_t^T dH[c] */
+            for (int p = 0; p < P; ++p) {
+                double acc = 0.0;
+                for (int n = 0; n < N; ++n) acc += (double)Ct[n] * M[n * P + p];
+                val[(size_t)cc * P + p] = acc;
+            }
+            /* score = Q_t . key / sqrt(N) */
+            double s = 0.0;
+            for (int n = 0; n < N; ++n) s += (double)Qt[n] * key[n];
+            sc[cc] = s * inv_sqrt_n;
+        }
+        /* softmax over the k memories, then the weighted sum of values */
+        for (int p = 0; p < P; ++p) o[p] = 0.0;
+        if (k > 0) {
+            double m = sc[0];
+            for (int cc = 1; cc < k; ++cc) if (sc[cc] > m) m = sc[cc];
+            double z = 0.0;
+            for (int cc = 0; cc < k; ++cc) z += exp(sc[cc] - m);
+            for (int cc = 0; cc < k; ++cc) {
+                const double w = exp(sc[cc] - m) / z;
+                for (int p = 0; p < P; ++p) o[p] += w * val[(size_t)cc * P + p];
+            }
+        }
+        const size_t row = (((size_t)b * nrows + r) * H + h) * P;
+        if (c->o) for (int p = 0; p < P; ++p) c->o[row + p] = o[p];
+        if (c->y) {
+            for (int p = 0; p < P; ++p) {
+                const double base = c->y_ssd ? c->y_ssd[row + p] : 0.0;
+                c->y[row + p] = base + c->g * o[p];
+            }
+        }
+        if (c->scores) {
+            double* srow = c->scores + (((size_t)b * H + h) * nrows + r) * nchunks;
+            for (int cc = 0; cc < nchunks; ++cc) srow[cc] = cc < k ? sc[cc] : NAN;
+        }
+    }
+    free(key);
+    free(val);
+    free(sc);
+    free(o);
+}
+
+/*
+ * Q[B,L,H,N], E[B,L,H,P], Cm[B,L,N] float; dH[B,H,C,N,P] double.
+ * With tokens == NULL every position is computed and the outputs are
+ * [B,L,H,P]; otherwise only the ntok listed positions, outputs [B,ntok,H,P]
+ * (and y_ssd, when given, is read with that same compact indexing).
+ */
+int oracle_sma(const oracle_dims* d, const float* Q, const float* E, const float* Cm,
+               const double* dH, double g, const double* y_ssd, double* o, double* y,
+               double* scores, const int* tokens, int ntok, int nthreads) {
+    if (!d || d->chunk <= 0 || d->seqlen % d->chunk != 0) return -1;
+    if (tokens) {
+        for (int i = 0; i < ntok; ++i)
+            if (tokens[i] < 0 || tokens[i] >= d->seqlen) return -1;
+    }
+    sma_ctx c = {d, Q, E, Cm, dH, g, y_ssd, o, y, scores, tokens, ntok};
+    run_units(sma_unit, &c, d->batch * d->nheads, nthreads);
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* 5: one decode step against the cache of completed chunk memories     */
+/* ------------------------------------------------------------------ */
+typedef struct {
+    const oracle_dims* d; /* batch = number of sequences; seqlen unused */
+    int cmax;
+    const float *x, *dt, *A, *Bm, *Cm, *Q, *E;
+    double g;
+    double *state, *dHcur, *cache;
+    const int *nchunks, *pos;
+    double* y;
+} dec_ctx;
+
+static void decode_unit(void* vctx, int unit) {
+    dec_ctx* c = (dec_ctx*)vctx;
+    const oracle_dims* d = c->d;
+    const int H = d->nheads, P = d->headdim, N = d->dstate, S = d->chunk;
+    const int b = unit / H, h = unit % H;
+    const int nmem = c->nchunks[b];
+    const size_t bh = (size_t)b * H + h;
+    double* Hs = c->state + bh * N * P;
+    double* D = c->dHcur + bh * N * P;
+    const float* xt = c->x + bh * P;
+    const float* Bt = c->Bm + (size_t)b * N;
+    const float* Ct = c->Cm + (size_t)b * N;
+    const float* Qt = c->Q + bh * N;
+    const float* Et = c->E + bh * P;
+    const double dtt = (double)c->dt[bh];
+    const double decay = exp(dtt * (double)c->A[h]);
+    /* recurrence and running chunk contribution, including this token */
+    for (int n = 0; n < N; ++n)
+        for (int p = 0; p < P; ++p) {
+            const double inp = dtt * (double)Bt[n] * (double)xt[p];
+            Hs[n * P + p] = decay * Hs[n * P + p] + inp;
+            D[n * P + p] = decay * D[n * P + p] + inp;
+        }
+    double* yt = c->y + bh * P;
+    for (int p = 0; p < P; ++p) {
+        double acc = 0.0;
+        for (int n = 0; n < N; ++n) acc += (double)Ct[n] * Hs[n * P + p];
+        yt[p] = acc;
+    }
+    /* SMA over the nmem completed chunks */
+    if (nmem > 0) {
+        const double inv_sqrt_n = 1.0 / sqrt((double)N);
+        double* sc = (double*)malloc(sizeof(double) * (size_t)nmem);
+        double* val = (double*)malloc(sizeof(double) * (size_t)nmem * P);
+        double* key = (double*)malloc(sizeof(double) * (size_t)N);
+        for (int cc = 0; cc < nmem; ++cc) {
+            const double* M = c->cache + (bh * (size_t)c->cmax + cc) * (size_t)N * P;
+            for (int n = 0; n < N; ++n) {
+                double acc = 0.0;
+                for (int p = 0; p < P; ++p) acc += M[n * P + p] * (double)Et[p];
+                key[n] = acc;
+            }
+            for (int p = 0; p < P; ++p) {
+                double acc = 0.0;
+                for (int n = 0; n < N; ++n) acc += (double)Ct[n] * M[n * P + p];
+                val[(size_t)cc * P + p] = acc;
+            }
+            double s = 0.0;
+            for (int n = 0; n < N; ++n) s += (double)Qt[n] * key[n];
+            sc[cc] = s * inv_sqrt_n;
+        }
+        double m = sc[0];
+        for (int cc = 1; cc < nmem; ++cc) if (sc[cc] > m) m = sc[cc];
+        double z = 0.0;
+        for (int cc = 0; cc < nmem; ++cc) z += exp(sc[cc] - m);
+        for (int p = 0; p < P; ++p) {
+            double acc = 0.0;
+            for (int cc = 0; cc < nmem; ++cc) acc += exp(sc[cc] - m) / z * val[(size_t)cc * P + p];
+            yt[p] += c->g * acc;
+        }
+        free(sc);
+        free(val);
+        free(key);
+    }
+    /* the token that closes its chunk appends the finished contribution */
+    if (c->pos[b] == S - 1) {
+        double* slot = c->cache + (bh * (size_t)c->cmax + nmem) * (size_t)N * P;
+        memcpy(slot, D, sizeof(double) * (size_t)N * P);
+        memset(D, 0, sizeof(double) * (size_t)N * P);
+    }
+}
+
+/*
+ * x[Bs,H,P] dt[Bs,H] A[H] Bm[Bs,N] Cm[Bs,N] Q[Bs,H,N] E[Bs,H,P] (float);
+ * state, dH_cur [Bs,H,N,P], cache [Bs,H,cmax,N,P], y [Bs,H,P] (double);
+ * nchunks[Bs], pos[Bs] in/out.  Returns -1 (and changes nothing) when an
+ * append would overflow the cache or a counter is out of range.
+ */
+int oracle_decode_step(const oracle_dims* d, int cmax, const float* x, const float* dt,
+                       const float* A, const float* Bm, const float* Cm, const float* Q,
+                       const float* E, double g, double* state, double* dH_cur, double* cache,
+                       int* nchunks, int* pos, double* y, int nthreads) {
+    if (!d || d->chunk <= 0) return -1;
+    for (int b = 0; b < d->batch; ++b) {
+        if (nchunks[b] < 0 || nchunks[b] > cmax) return -1;
+        if (pos[b] < 0 || pos[b] >= d->chunk) return -1;
+        if (pos[b] == d->chunk - 1 && nchunks[b] >= cmax) return -1;
+    }
+    dec_ctx c = {d, cmax, x, dt, A, Bm, Cm, Q, E, g, state, dH_cur, cache, nchunks, pos, y};
+    run_units(decode_unit, &c, d->batch * d->nheads, nthreads);
+    for (int b = 0; b < d->batch; ++b) {
+        if (pos[b] == d->chunk - 1) {
+            nchunks[b] += 1;
+            pos[b] = 0;
+        } else {
+            pos[b] += 1;
+        }
+    }
+    return 0;
+}

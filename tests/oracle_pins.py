@@ -1,0 +1,337 @@
+"""Pins of the fp64 oracle to facts other than the oracle itself.
+
+Each ``pin_*`` function takes an ``oracle.dart_oracle.Oracle`` and raises
+AssertionError when the oracle disagrees with a closed form, an identity of
+the method, a textbook routine on explicitly materialised keys/values, or the
+pages' worked example.  ``test_oracle_pins.py`` runs them on the real oracle;
+``test_oracle_mutants.py`` runs them on deliberately broken builds and checks
+that every planted mistake trips at least one.
+
+Citations are to the pages' own sections: the Pith review of DART ("Core
+claim", "What carries the argument", referee major comment 3 on Eq. (8),
+circularity check on Eq. (14)), the DART abstract, and the paper-daily
+summary's worked example.
+"""
+from __future__ import annotations
+
+import os
+
+import numpy as np
+import torch
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _rand_layer(seed, Bz, L, H, P, N, dt_scale=0.3, a_max=2.0):
+    r = np.random.default_rng(seed)
+    return dict(
+        x=r.standard_normal((Bz, L, H, P)).astype(np.float32),
+        dt=(r.uniform(0.05, 1.0, (Bz, L, H)) * dt_scale).astype(np.float32),
+        A=(-r.uniform(0.1, a_max, (H,))).astype(np.float32),
+        Bm=(r.standard_normal((Bz, L, N)) / np.sqrt(N)).astype(np.float32),
+        Cm=(r.standard_normal((Bz, L, N)) / np.sqrt(N)).astype(np.float32),
+        Q=r.standard_normal((Bz, L, H, N)).astype(np.float32),
+        E=(r.standard_normal((Bz, L, H, P)) / np.sqrt(P)).astype(np.float32),
+    )
+
+
+def _log_decay(dt, A):
+    """a[b,t,h] = dt * A_h (the per-token log-decay, as float64)."""
+    return dt.astype(np.float64) * A.astype(np.float64)[None, None, :]
+
+
+def _close(a, b, tol, what):
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    err = np.max(np.abs(a - b)) if a.size else 0.0
+    scale = max(np.max(np.abs(b)) if b.size else 0.0, 1e-300)
+    assert err <= tol * max(scale, 1.0), f"{what}: max|err| {err:.3e} (scale {scale:.3e})"
+
+
+# ----------------------------------------------------------------------------
+# recurrence
+# ----------------------------------------------------------------------------
+def pin_closed_form_single_token(orc):
+    """A single non-zero input token s: with the recurrence
+    H_t = exp(dt_t A) H_{t-1} + dt_t B_t x_t^T, the state for t >= s is
+    exp(sum_{r=s+1..t} dt_r A) dt_s B_s x_s^T and y_t = H_t^T C_t; before s
+    everything is zero.  The chunk holding s owns the whole contribution."""
+    Bz, L, H, P, N, S = 1, 24, 2, 3, 5, 8
+    inp = _rand_layer(1, Bz, L, H, P, N)
+    s = 10
+    x = np.zeros_like(inp["x"])
+    x[0, s] = inp["x"][0, s]
+    y, dH, st = orc.ssd_scan(x, inp["dt"], inp["A"], inp["Bm"], inp["Cm"], S)
+    a = _log_decay(inp["dt"], inp["A"])[0]  # [L,H]
+    for h in range(H):
+        outer = inp["dt"][0, s, h] * np.outer(inp["Bm"][0, s].astype(np.float64),
+                                              x[0, s, h].astype(np.float64))
+        for t in range(L):
+            if t < s:
+                expect_y = np.zeros(P)
+            else:
+                Ht = np.exp(a[s + 1:t + 1, h].sum()) * outer
+                expect_y = Ht.T @ inp["Cm"][0, t].astype(np.float64)
+            _close(y[0, t, h], expect_y, 1e-12, f"y[t={t},h={h}]")
+        for c in range(L // S):
+            e = c * S + S - 1
+            exp_dh = np.exp(a[s + 1:e + 1, h].sum()) * outer if c == s // S else np.zeros((N, P))
+            _close(dH[0, h, c], exp_dh, 1e-12, f"dH[c={c}]")
+            exp_st = np.exp(a[s + 1:e + 1, h].sum()) * outer if e >= s else np.zeros((N, P))
+            _close(st[0, h, c], exp_st, 1e-12, f"states[c={c}]")
+
+
+def pin_quadratic_form(orc):
+    """The SSD (structured masked attention) form of Mamba-2 -- Eq. (4) of the
+    SSD view the Pith review cites: y_t = sum_{s<=t} (C_t . B_s)
+    exp(sum_{r=s+1..t} a_r) dt_s x_s, plus exp(sum_{r<=t} a_r) C_t^T H_init.
+    Written here as an explicit double loop over (t, s)."""
+    Bz, L, H, P, N, S = 2, 32, 3, 4, 6, 8
+    inp = _rand_layer(2, Bz, L, H, P, N)
+    r = np.random.default_rng(22)
+    h0 = r.standard_normal((Bz, H, N, P))
+    y, _, _ = orc.ssd_scan(inp["x"], inp["dt"], inp["A"], inp["Bm"], inp["Cm"], S, init_state=h0)
+    a = _log_decay(inp["dt"], inp["A"])
+    cum = np.cumsum(a, axis=1)  # inclusive prefix sums over t
+    Bm, Cm, x, dt = (inp[k].astype(np.float64) for k in ("Bm", "Cm", "x", "dt"))
+    expect = np.zeros_like(y)
+    for b in range(Bz):
+        for h in range(H):
+            for t in range(L):
+                acc = np.exp(cum[b, t, h]) * (h0[b, h].T @ Cm[b, t])
+                for s in range(t + 1):
+                    w = (Cm[b, t] @ Bm[b, s]) * np.exp(cum[b, t, h] - cum[b, s, h]) * dt[b, s, h]
+                    acc = acc + w * x[b, s, h]
+                expect[b, t, h] = acc
+    _close(y, expect, 1e-11, "y_ssd vs quadratic form")
+
+
+def pin_chunk_memory_definition(orc):
+    """dH[c] is what chunk c contributes to the state at its own last token
+    e(c) (Pith review, "What carries the argument"; referee comment 3 on
+    Eq. (8)): sum_{s in c} exp(sum_{r=s+1..e(c)} a_r) dt_s B_s x_s^T.  The
+    boundary states obey states[c] = exp(sum_{r in c} a_r) states[c-1] + dH[c]
+    and the final state is the decayed sum of all chunk memories."""
+    Bz, L, H, P, N, S = 1, 40, 2, 3, 4, 8
+    inp = _rand_layer(3, Bz, L, H, P, N)
+    _, dH, st = orc.ssd_scan(inp["x"], inp["dt"], inp["A"], inp["Bm"], inp["Cm"], S)
+    a = _log_decay(inp["dt"], inp["A"])[0]
+    Bm, x, dt = inp["Bm"][0].astype(np.float64), inp["x"][0].astype(np.float64), inp["dt"][0]
+    C = L // S
+    for h in range(H):
+        for c in range(C):
+            e = c * S + S - 1
+            m = np.zeros((N, P))
+            for s in range(c * S, e + 1):
+                m += np.exp(a[s + 1:e + 1, h].sum()) * dt[s, h] * np.outer(Bm[s], x[s, h])
+            _close(dH[0, h, c], m, 1e-12, f"dH[h={h},c={c}]")
+            prev = st[0, h, c - 1] if c else np.zeros((N, P))
+            _close(st[0, h, c], np.exp(a[c * S:e + 1, h].sum()) * prev + dH[0, h, c], 1e-12,
+                   "states recursion")
+        final = sum(np.exp(a[c * S + S:, h].sum()) * dH[0, h, c] for c in range(C))
+        _close(st[0, h, C - 1], final, 1e-12, "final state = decayed sum of dH")
+
+
+def pin_init_state_continuation(orc):
+    """Running the recurrence over L1 + L2 tokens equals running L1 tokens and
+    continuing L2 tokens from the boundary state (the recurrence is Markov in
+    H).  Chunk memories of the continued part are unaffected by the carried
+    state."""
+    Bz, L, H, P, N, S = 1, 32, 2, 4, 4, 8
+    inp = _rand_layer(4, Bz, L, H, P, N)
+    keys = ("x", "dt", "Bm", "Cm")
+    y, dH, st = orc.ssd_scan(inp["x"], inp["dt"], inp["A"], inp["Bm"], inp["Cm"], S)
+    first = {k: inp[k][:, :16] for k in keys}
+    second = {k: inp[k][:, 16:] for k in keys}
+    y1, _, st1 = orc.ssd_scan(first["x"], first["dt"], inp["A"], first["Bm"], first["Cm"], S)
+    y2, dH2, st2 = orc.ssd_scan(second["x"], second["dt"], inp["A"], second["Bm"], second["Cm"], S,
+                                init_state=st1[:, :, -1])
+    _close(np.concatenate([y1, y2], 1), y, 1e-12, "continued y")
+    _close(dH2, dH[:, :, 2:], 1e-12, "continued dH")
+    _close(st2, st[:, :, 2:], 1e-12, "continued states")
+
+
+# ----------------------------------------------------------------------------
+# state-memory attention
+# ----------------------------------------------------------------------------
+def pin_single_prior_chunk(orc):
+    """A token of chunk 1 sees exactly one memory, so its softmax weight is 1
+    and o_t = C_t^T dH[0] whatever Q and E are (Pith review, "Core claim":
+    value = C_t dH[c]; mask c < chunk(t))."""
+    Bz, L, H, P, N, S = 1, 16, 2, 5, 3, 8
+    inp = _rand_layer(5, Bz, L, H, P, N)
+    dH = np.random.default_rng(55).standard_normal((Bz, H, 2, N, P))
+    r = orc.sma(inp["Q"], inp["E"], inp["Cm"], dH, S, g=1.0)
+    for h in range(H):
+        for t in range(S, 2 * S):
+            _close(r["o"][0, t, h], inp["Cm"][0, t].astype(np.float64) @ dH[0, h, 0], 1e-13,
+                   f"o[t={t}]")
+        assert np.all(r["o"][0, :S, h] == 0.0), "chunk 0 has no memory"
+
+
+def pin_bruteforce_attention(orc):
+    """Materialise, per token, the key matrix K_t[c] = (dH[c] E_t)^T and value
+    matrix V_t[c] = C_t^T dH[c] over c < chunk(t), then call torch's
+    scaled-dot-product attention (a textbook softmax(q K^T / sqrt(N)) V)."""
+    Bz, L, H, P, N, S = 2, 48, 2, 5, 7, 8
+    inp = _rand_layer(6, Bz, L, H, P, N)
+    dH = np.random.default_rng(66).standard_normal((Bz, H, L // S, N, P))
+    g = 0.75
+    ys = np.random.default_rng(67).standard_normal((Bz, L, H, P))
+    r = orc.sma(inp["Q"], inp["E"], inp["Cm"], dH, S, g=g, y_ssd=ys)
+    Q = torch.from_numpy(inp["Q"].astype(np.float64))
+    E = torch.from_numpy(inp["E"].astype(np.float64))
+    Cm = torch.from_numpy(inp["Cm"].astype(np.float64))
+    M = torch.from_numpy(dH)
+    for b in range(Bz):
+        for h in range(H):
+            for t in range(L):
+                k = t // S
+                if k == 0:
+                    expect = torch.zeros(P, dtype=torch.float64)
+                else:
+                    Kt = torch.einsum("cnp,p->cn", M[b, h, :k], E[b, t, h])       # [k, N]
+                    Vt = torch.einsum("n,cnp->cp", Cm[b, t], M[b, h, :k])         # [k, P]
+                    expect = torch.nn.functional.scaled_dot_product_attention(
+                        Q[b, t, h][None, None, None, :], Kt[None, None], Vt[None, None])[0, 0, 0]
+                _close(r["o"][b, t, h], expect.numpy(), 1e-12, f"o[b={b},t={t},h={h}]")
+                _close(r["y"][b, t, h], ys[b, t, h] + g * expect.numpy(), 1e-12, "gated y")
+
+
+def pin_worked_example(orc):
+    """The paper-daily summary's L=8, S=4, N=2 example, finished in DART's
+    terms (tests/golden/worked_example.txt)."""
+    vals = {}
+    with open(os.path.join(GOLDEN, "worked_example.txt")) as f:
+        for line in f:
+            line = line.split("#", 1)[0].split()
+            if line:
+                vals[line[0]] = [float(v) for v in line[1:]]
+    L, S, N, P = (int(vals[k][0]) for k in ("L", "S", "N", "P"))
+    g = vals["g"][0]
+    q = np.array(vals["q"], np.float32)
+    x = np.zeros((1, L, 1, P), np.float32)
+    Bm = np.zeros((1, L, N), np.float32)
+    x[0, 0, 0, 0] = Bm[0, 0, 0] = 1.0
+    x[0, 1, 0, 1] = Bm[0, 1, 1] = 1.0
+    Cm = np.zeros((1, L, N), np.float32)
+    Cm[0, :, 0] = 1.0
+    E = np.zeros((1, L, 1, P), np.float32)
+    E[0, :, 0, 0] = 1.0
+    Q = np.broadcast_to(q, (1, L, 1, N)).copy()
+    dt = np.ones((1, L, 1), np.float32)
+    A = np.zeros((1,), np.float32)
+    y_ssd, dH, _ = orc.ssd_scan(x, dt, A, Bm, Cm, S)
+    np.testing.assert_allclose(dH[0, 0, 0].ravel(), vals["dH_c0"], atol=1e-15)
+    r = orc.sma(Q, E, Cm, dH, S, g=g, y_ssd=y_ssd, want_scores=True)
+    np.testing.assert_allclose(r["scores"][0, 0, 4, 0], vals["score_t4_c0"][0], rtol=1e-14)
+    for t in range(L):
+        np.testing.assert_allclose(r["y"][0, t, 0], vals[f"y_t{t}"], atol=1e-14)
+
+
+def pin_gate_zero(orc):
+    """g = 0 removes the SMA branch (Pith review, "If this is right": the
+    SMA-removal ablation gives Mamba-2): y equals y_ssd exactly."""
+    Bz, L, H, P, N, S = 1, 32, 2, 4, 6, 8
+    inp = _rand_layer(7, Bz, L, H, P, N)
+    r = orc.layer_forward(inp["x"], inp["dt"], inp["A"], inp["Bm"], inp["Cm"], inp["Q"], inp["E"],
+                          S, g=0.0)
+    assert np.array_equal(r["y"], r["y_ssd"])
+    assert np.any(r["o"] != 0.0)
+
+
+def pin_one_hot_mask(orc):
+    """One-hot memories dH[c] = (c+1) e_0 e_0^T with a query that makes the
+    score grow steeply with c: the softmax is a one-hot on the last allowed
+    chunk, so o_t[0] = chunk(t) * C_t[0].  An off-by-one in the causal mask
+    (c < chunk(t)) moves the value by a whole chunk."""
+    Bz, L, H, P, N, S = 1, 48, 1, 3, 4, 8
+    C = L // S
+    dH = np.zeros((Bz, H, C, N, P))
+    for c in range(C):
+        dH[0, 0, c, 0, 0] = c + 1.0
+    Q = np.zeros((Bz, L, H, N), np.float32)
+    Q[..., 0] = 400.0
+    E = np.zeros((Bz, L, H, P), np.float32)
+    E[..., 0] = 1.0
+    Cm = np.random.default_rng(8).uniform(0.5, 1.5, (Bz, L, N)).astype(np.float32)
+    r = orc.sma(Q, E, Cm, dH, S, g=1.0)
+    for t in range(L):
+        k = t // S
+        expect = k * float(Cm[0, t, 0]) if k else 0.0
+        assert abs(r["o"][0, t, 0, 0] - expect) < 1e-9 * max(1.0, expect), (t, r["o"][0, t, 0, 0], expect)
+        assert np.all(r["o"][0, t, 0, 1:] == 0.0)
+
+
+def pin_sampled_rows(orc):
+    """Computing a sample of token positions gives the same rows as the full
+    computation (the sample path is what the large-size parity tests use)."""
+    Bz, L, H, P, N, S = 2, 40, 2, 3, 5, 8
+    inp = _rand_layer(9, Bz, L, H, P, N)
+    dH = np.random.default_rng(99).standard_normal((Bz, H, L // S, N, P))
+    full = orc.sma(inp["Q"], inp["E"], inp["Cm"], dH, S, g=0.3)
+    tok = [0, 7, 8, 15, 16, 39, 22]
+    part = orc.sma(inp["Q"], inp["E"], inp["Cm"], dH, S, g=0.3, tokens=tok)
+    assert np.array_equal(part["o"], full["o"][:, tok])
+
+
+# ----------------------------------------------------------------------------
+# decode
+# ----------------------------------------------------------------------------
+def pin_decode_matches_prefill(orc):
+    """Forward over L + S tokens equals forward over L tokens followed by S
+    single-token decode steps against the cache of chunk memories (DART
+    abstract: the inference cache is the chunk state memories), including the
+    append when the last token closes its chunk."""
+    Bz, L, H, P, N, S = 2, 24, 2, 4, 5, 8
+    T = L + S
+    inp = _rand_layer(10, Bz, T, H, P, N)
+    g = 0.6
+    full = orc.layer_forward(inp["x"], inp["dt"], inp["A"], inp["Bm"], inp["Cm"], inp["Q"],
+                             inp["E"], S, g)
+    pre = orc.layer_forward(*(inp[k][:, :L] if k != "A" else inp[k]
+                              for k in ("x", "dt", "A", "Bm", "Cm", "Q", "E")), S, g)
+    cmax = L // S + 2
+    cache = np.zeros((Bz, H, cmax, N, P))
+    cache[:, :, :L // S] = pre["dH"]
+    state = np.ascontiguousarray(pre["states"][:, :, -1])
+    dcur = np.zeros((Bz, H, N, P))
+    nch = np.full((Bz,), L // S, np.int32)
+    pos = np.zeros((Bz,), np.int32)
+    for t in range(L, T):
+        y = orc.decode_step(inp["x"][:, t], inp["dt"][:, t], inp["A"], inp["Bm"][:, t],
+                            inp["Cm"][:, t], inp["Q"][:, t], inp["E"][:, t], g, state, dcur,
+                            cache, nch, pos, S)
+        _close(y, full["y"][:, t], 1e-12, f"decode y at t={t}")
+    assert np.all(nch == L // S + 1) and np.all(pos == 0)
+    _close(cache[:, :, L // S], full["dH"][:, :, L // S], 1e-12, "appended memory")
+    assert np.all(dcur == 0.0)
+    _close(state, full["states"][:, :, -1], 1e-12, "decode state")
+
+
+def pin_cache_ratio(orc):
+    """Eq. (14) (Pith review, circularity check): per head the DART cache is
+    M N P elements (M = L/S chunk memories) against 2 L P for a token-level
+    attention cache, a ratio of N/(2S): 0.25 at S=256, N=128 (the abstract's
+    75% saving).  Checked on the shapes of the 128-memory decode cache."""
+    del orc
+    L, S, N, P = 32768, 256, 128, 64
+    dart = (L // S) * N * P
+    attn = 2 * L * P
+    assert dart / attn == N / (2 * S) == 0.25
+
+
+ALL_PINS = [
+    pin_closed_form_single_token,
+    pin_quadratic_form,
+    pin_chunk_memory_definition,
+    pin_init_state_continuation,
+    pin_single_prior_chunk,
+    pin_bruteforce_attention,
+    pin_worked_example,
+    pin_gate_zero,
+    pin_one_hot_mask,
+    pin_sampled_rows,
+    pin_decode_matches_prefill,
+    pin_cache_ratio,
+]
