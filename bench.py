@@ -1,0 +1,503 @@
+#!/usr/bin/env python
+"""Throughput of the DART layer hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl dart|reference]
+
+Headline workload: the bf16 layer forward at training length (B=2, L=8192,
+H=32, P=64, N=128, S=256; 16384 tokens per step), inputs resident in HBM.  A
+step is one `dart_ssd_chunk_scan` + one `dart_sma_forward` (scan, chunk
+memories, state-memory attention, gated residual).  Beside it the decode
+workload (64 sequences x 128 cached chunk memories, 256 consecutive steps with
+the append on the last) is timed as its own region and reported under
+"decode".  Rank 0 prints one JSON line.
+
+Timing: CUDA events on the launching stream, W untimed warm-up steps, K timed
+steps between a barrier + device synchronisation on both sides, max over
+ranks.  Per-step inputs (272 MiB) exceed the 126 MB L2, so no flush is needed
+between steps.  The roofline fraction is the SMA kernel's algorithmic rate
+over the measured peak in MEASURED_PEAKS.json.
+
+--impl reference times the fp64 CPU oracle (the only reference there is) on
+a bounded sample of the same workload, on this host's cores.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from mamba_ssd_state_b200 import synth  # noqa: E402
+
+FWD = synth.TRAIN_L8K
+DEC = synth.DECODE_64x32K
+METRIC = "DART layer fwd tokens/s at L=8K (% BF16 peak); decode tokens/s (% HBM BW)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "sm_max_mhz": 1965.0}
+SMS = 148
+FP32_LANES_PER_SM = 128
+
+
+def parse():
+    p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=("dart", "reference"), default="dart")
+    p.add_argument("--no-decode", action="store_true", help="skip the decode region")
+    p.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end region")
+    p.add_argument("--no-cpu-baseline", action="store_true", help="skip timing the oracle")
+    p.add_argument("--decode-steps", type=int, default=DEC.nsteps)
+    return p.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS if k in d}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work (only what the method needs: masked pairs excluded)
+# ---------------------------------------------------------------------------
+def sma_flops(s: synth.LayerShape) -> float:
+    """4*N*P per valid (token, earlier chunk) pair per head: 2NP for Q^T dH and
+    2NP for C^T dH.  Pairs per (b, h): S * C(C-1)/2."""
+    C = s.nchunks
+    return 4.0 * s.dstate * s.headdim * s.chunk * C * (C - 1) / 2 * s.batch * s.nheads
+
+
+def ssd_flops(s: synth.LayerShape) -> float:
+    """Lower-triangular C B^T once per chunk (ngroups = 1), the causal intra
+    block per (chunk, head), the chunk memory per (chunk, head) and the
+    inter-chunk output per (chunk >= 1, head)."""
+    S, N, P, C, H, B = s.chunk, s.dstate, s.headdim, s.nchunks, s.nheads, s.batch
+    per_b = C * S * (S + 1) * N + C * H * S * (S + 1) * P + C * H * 2 * S * N * P + (C - 1) * H * 2 * S * N * P
+    return float(B * per_b)
+
+
+def decode_bytes(d: synth.DecodeShape, n: int, append: bool) -> float:
+    """Bytes one decode step must move: every cached memory once, the float32
+    state and running contribution read and written, the token inputs, the
+    output, and the appended memory when the step closes a chunk."""
+    esz = 2 if d.dtype == "bf16" else 4
+    per_sh = n * d.dstate * d.headdim * esz + 4 * d.dstate * d.headdim * 4
+    per_sh += (2 * d.headdim + d.dstate) * esz + 4 + d.headdim * 4
+    per_seq = d.nheads * per_sh + 2 * d.dstate * esz
+    total = d.nseq * per_seq
+    if append:
+        total += d.nseq * d.nheads * d.dstate * d.headdim * esz
+    return float(total)
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows),
+                "power_w_max": max((float(r[3]) for r in rows if r[3].replace(".", "").isdigit()), default=None)}
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (one process per GPU; weak scaling, no data-path collective)
+# ---------------------------------------------------------------------------
+class Dist:
+    def __init__(self):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+        if self.world > 1:
+            import torch.distributed as dist
+            backend = "nccl" if torch.cuda.is_available() else "gloo"
+            if backend == "nccl":
+                torch.cuda.set_device(self.local)
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+            self.pg = dist
+
+    def barrier(self):
+        if self.pg:
+            if torch.cuda.is_available():
+                self.pg.barrier(device_ids=[self.local])
+            else:
+                self.pg.barrier()
+
+    def max(self, v: float) -> float:
+        if not self.pg:
+            return v
+        dev = torch.device("cuda", self.local) if torch.cuda.is_available() else torch.device("cpu")
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            self.pg.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------
+# GPU regions
+# ---------------------------------------------------------------------------
+def forward_region(args, dist, dart):
+    dev = torch.device("cuda", torch.cuda.current_device())
+    inp = synth.layer_inputs(FWD, seed=dist.rank)
+    d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    B, L, H, P, N, S = FWD.batch, FWD.seqlen, FWD.nheads, FWD.headdim, FWD.dstate, FWD.chunk
+    C = L // S
+    y = torch.empty((B, L, H, P), device=dev, dtype=torch.float32)
+    dH = torch.empty((B, H, C, N, P), device=dev, dtype=torch.bfloat16)
+    states = torch.empty((B, H, C, N, P), device=dev, dtype=torch.float32)
+    ws = torch.empty(max(16, dart.scan_workspace_bytes(B, L, H, P, N, S, torch.bfloat16)), device=dev,
+                     dtype=torch.uint8)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        dart.dart_ssd_chunk_scan(d["x"], d["dt"], d["A"], d["Bm"], d["Cm"], S, y_ssd=y, dH=dH, states=states,
+                                 workspace=ws)
+        if ev:
+            ev[1].record(stream)
+        dart.dart_sma_forward(d["Q"], d["E"], d["Cm"], dH, S, d["g"], y, out=y)
+        if ev:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    dart.dart_sync_status()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(dev.index)
+    clocks.start()
+    time.sleep(0.25)
+    dist.barrier()
+    torch.cuda.synchronize()
+    n0 = dart.launch_count()
+    start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    end.record(stream)
+    torch.cuda.synchronize()
+    n1 = dart.launch_count()
+    dist.barrier()
+    clk = clocks.stop()
+    dart.dart_sync_status()
+    ms = start.elapsed_time(end)
+    scan_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    sma_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    return {"ms_total": ms, "scan_ms": scan_ms, "sma_ms": sma_ms, "launches": n1 - n0, "clocks": clk,
+            "inputs": inp}
+
+
+def e2e_region(args, dist, dart, inp):
+    """Same workload through the public call with host (pinned) buffers: the
+    inputs are copied host->device and y device->host inside every step."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    host = {k: (v.pin_memory() if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    B, L, H, P, N, S = FWD.batch, FWD.seqlen, FWD.nheads, FWD.headdim, FWD.dstate, FWD.chunk
+    C = L // S
+    bufs = {"y": torch.empty((B, L, H, P), device=dev, dtype=torch.float32),
+            "dH": torch.empty((B, H, C, N, P), device=dev, dtype=torch.bfloat16),
+            "states": torch.empty((B, H, C, N, P), device=dev, dtype=torch.float32),
+            "workspace": torch.empty(max(16, dart.scan_workspace_bytes(B, L, H, P, N, S, torch.bfloat16)),
+                                     device=dev, dtype=torch.uint8)}
+    h2d = sum(v.numel() * v.element_size() for k, v in host.items() if isinstance(v, torch.Tensor))
+    d2h = B * L * H * P * 4
+    stream = torch.cuda.current_stream()
+
+    def step():
+        out = dart.layer_forward(host["x"], host["dt"], host["A"], host["Bm"], host["Cm"], host["Q"],
+                                 host["E"], S, host["g"], outputs=("y",), buffers=bufs)
+        return out["y"]
+
+    for _ in range(max(1, min(args.warmup, 3))):
+        step()
+    torch.cuda.synchronize()
+    k = max(1, min(args.steps, 10))
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist.barrier()
+    torch.cuda.synchronize()
+    start.record(stream)
+    for _ in range(k):
+        step()
+    end.record(stream)
+    torch.cuda.synchronize()
+    dist.barrier()
+    ms = dist.max(start.elapsed_time(end))
+    return {"value": dist.world * B * L * k / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": k,
+            "path": "dart.layer_forward on pinned host inputs, y returned to host"}
+
+
+def decode_region(args, dist, dart, peaks):
+    dev = torch.device("cuda", torch.cuda.current_device())
+    init = synth.decode_initial(DEC, seed=dist.rank)
+    work = {k: v.to(dev) for k, v in init.items()}
+    saved = {k: v.clone() for k, v in work.items()}
+    A = synth.decode_A(DEC, seed=dist.rank).to(dev)
+    # the cache holds one free slot: at most S steps (one append) per run
+    nsteps = max(1, min(args.decode_steps, DEC.chunk * (DEC.cmax - DEC.ncached)))
+    toks = [synth.decode_tokens(DEC, s, seed=dist.rank) for s in range(nsteps)]
+    toks = [{k: v.to(dev) for k, v in t.items()} for t in toks]
+    y = torch.empty((DEC.nseq, DEC.nheads, DEC.headdim), device=dev, dtype=torch.float32)
+    ws = torch.empty(max(16, dart.decode_workspace_bytes(DEC.nseq, DEC.nheads, DEC.headdim, DEC.dstate,
+                                                         DEC.chunk, DEC.cmax, torch.bfloat16)),
+                     device=dev, dtype=torch.uint8)
+    stream = torch.cuda.current_stream()
+
+    def step(s, ev=None):
+        t = toks[s]
+        if ev:
+            ev[0].record(stream)
+        dart.dart_decode_step(t["x"], t["dt"], A, t["Bm"], t["Cm"], t["Q"], t["E"], DEC.g, work["state"],
+                              work["dH_cur"], work["cache"], work["nchunks"], work["pos"], DEC.chunk, y=y,
+                              workspace=ws)
+        if ev:
+            ev[1].record(stream)
+
+    for s in range(min(args.warmup, nsteps)):
+        step(s)
+    dart.dart_sync_status()
+    for k in work:
+        work[k].copy_(saved[k])
+    del saved
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(nsteps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(dev.index)
+    clocks.start()
+    time.sleep(0.25)
+    dist.barrier()
+    torch.cuda.synchronize()
+    n0 = dart.launch_count()
+    start.record(stream)
+    for s in range(nsteps):
+        step(s, evs[s])
+    end.record(stream)
+    torch.cuda.synchronize()
+    n1 = dart.launch_count()
+    dist.barrier()
+    clk = clocks.stop()
+    dart.dart_sync_status()
+    ms = dist.max(start.elapsed_time(end))
+    per = [e[0].elapsed_time(e[1]) for e in evs]
+    # step s starts at pos = s % S with ncached + s // S memories; pos = S-1 appends
+    total_bytes = sum(decode_bytes(DEC, DEC.ncached + s // DEC.chunk, s % DEC.chunk == DEC.chunk - 1)
+                      for s in range(nsteps))
+    bytes_step = total_bytes / nsteps
+    step_ms = statistics.mean(per)
+    achieved = bytes_step / (step_ms / 1e3) / 1e9
+    return {
+        "value": dist.world * DEC.nseq * nsteps / (ms / 1e3), "unit": "tokens/s",
+        "ms_per_step": ms / nsteps, "steps": nsteps, "launches": n1 - n0, "clocks": clk,
+        "config": {"workload": "decode_64seq_128mem", "nseq": DEC.nseq, "nheads": DEC.nheads,
+                   "headdim": DEC.headdim, "dstate": DEC.dstate, "chunk": DEC.chunk,
+                   "cached_chunks": DEC.ncached, "context": DEC.ncached * DEC.chunk,
+                   "l2": "cache 4.3 GB per step >> 126 MB L2"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                     "kernel": "dart_decode_step (decode_partial + decode_combine + decode_advance)",
+                     "bytes_per_step": bytes_step},
+    }
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle
+# ---------------------------------------------------------------------------
+def oracle_sample(inp, heads, nthreads):
+    from oracle import dart_oracle
+
+    orc = dart_oracle.Oracle(nthreads=nthreads)
+    f = {}
+    for k, v in inp.items():
+        if not isinstance(v, torch.Tensor):
+            f[k] = v
+            continue
+        a = v.float().numpy()
+        if k in ("x", "dt", "Q", "E"):
+            a = a[:1][:, :, heads]
+        elif k in ("Bm", "Cm"):
+            a = a[:1]
+        elif k == "A":
+            a = a[heads]
+        f[k] = np.ascontiguousarray(a)
+    t0 = time.perf_counter()
+    orc.layer_forward(f["x"], f["dt"], f["A"], f["Bm"], f["Cm"], f["Q"], f["E"], FWD.chunk, f["g"])
+    sec = time.perf_counter() - t0
+    tokens = FWD.seqlen * len(heads) / FWD.nheads  # full-layer token equivalents
+    return tokens / sec, sec
+
+
+def cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(inp):
+    nthreads = cores()
+    nh = min(FWD.nheads, max(1, 3 * nthreads))
+    heads = list(range(nh))
+    value, sec = oracle_sample(inp, heads, nthreads)
+    return {"value": value, "unit": "tokens/s", "cores": min(nthreads, nh), "kind": "oracle",
+            "sample": f"batch 0 of 2, heads 0..{nh - 1} of {FWD.nheads}, all {FWD.seqlen} tokens "
+                      f"(fp64 scan + SMA + gate, {sec:.1f} s); tokens/s counted as full-layer tokens "
+                      f"({FWD.seqlen} x {nh}/{FWD.nheads})"}
+
+
+def run_reference(args, dist):
+    """The reference arm: the fp64 oracle on this host's cores, one bounded
+    sample of the forward workload per step."""
+    if dist.rank != 0:
+        return
+    inp = synth.layer_inputs(FWD, seed=0)
+    nthreads = cores()
+    heads = list(range(min(FWD.nheads, nthreads)))
+    for _ in range(args.warmup):
+        oracle_sample(inp, heads, nthreads)
+    secs = []
+    for _ in range(args.steps):
+        _, s = oracle_sample(inp, heads, nthreads)
+        secs.append(s)
+    total = sum(secs)
+    tokens = FWD.seqlen * len(heads) / FWD.nheads * args.steps
+    value = tokens / total
+    sample = (f"per step: batch 0, heads 0..{len(heads) - 1} of {FWD.nheads}, all {FWD.seqlen} tokens; "
+              f"full-layer token equivalents")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": "dart_layer_fwd_L8k", "batch": FWD.batch,
+                                            "seqlen": FWD.seqlen, "nheads": FWD.nheads,
+                                            "headdim": FWD.headdim, "dstate": FWD.dstate, "chunk": FWD.chunk},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": min(nthreads, len(heads)),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+def main():
+    args = parse()
+    dist = Dist()
+    try:
+        if args.impl == "reference":
+            run_reference(args, dist)
+            return
+        from mamba_ssd_state_b200 import build as dart_build
+        from mamba_ssd_state_b200 import dart
+
+        if dist.rank == 0 or dist.world == 1:
+            dart_build.build()
+        dist.barrier()
+        if not torch.cuda.is_available():
+            raise SystemExit("bench.py needs a CUDA device")
+        torch.cuda.set_device(dist.local)
+        peaks, peak_src = load_peaks()
+
+        fwd = forward_region(args, dist, dart)
+        ms = dist.max(fwd["ms_total"])
+        tokens = FWD.batch * FWD.seqlen
+        value = dist.world * tokens * args.steps / (ms / 1e3)
+        impl = dart.sma_impl(FWD.dstate, FWD.headdim, FWD.chunk, torch.bfloat16)
+        f_sma = sma_flops(FWD)
+        f_ssd = ssd_flops(FWD)
+        sma_tflops = f_sma / (fwd["sma_ms"] / 1e3) / 1e12
+        if impl == "sma_tcgen05":
+            roof = {"bound": "tensor", "achieved": sma_tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                    "frac": sma_tflops / peaks["bf16_tflops"]}
+            peak_note = f"bf16_tflops ({peak_src})"
+        else:
+            alu_peak = SMS * FP32_LANES_PER_SM * 2 * peaks["sm_max_mhz"] * 1e6 / 1e12
+            roof = {"bound": "alu", "achieved": sma_tflops, "peak": alu_peak, "unit": "TFLOP/s",
+                    "frac": sma_tflops / alu_peak}
+            peak_note = "fp32 FMA peak: 148 SMs x 128 lanes x 2 flop x sm_max_mhz"
+        roof.update({"traffic": None, "kernel": impl, "flop_per_launch": f_sma, "peak_source": peak_note})
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": dist.world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "dart_layer_fwd_L8k", "batch": FWD.batch, "seqlen": FWD.seqlen,
+                       "nheads": FWD.nheads, "headdim": FWD.headdim, "dstate": FWD.dstate, "chunk": FWD.chunk,
+                       "ngroups": 1, "parallelism": f"dp{dist.world}",
+                       "l2": "inputs larger than L2 (272 MiB per step)"},
+            "gpu_launches": fwd["launches"],
+            "clocks": fwd["clocks"],
+            "roofline": roof,
+            "fwd_breakdown": {"scan_ms": fwd["scan_ms"], "sma_ms": fwd["sma_ms"],
+                              "sma_gflop": f_sma / 1e9, "ssd_gflop": f_ssd / 1e9,
+                              "layer_tflops": (f_sma + f_ssd) / (ms / args.steps / 1e3) / 1e12,
+                              "layer_frac_bf16_peak": (f_sma + f_ssd) / (ms / args.steps / 1e3) / 1e12
+                              / peaks["bf16_tflops"]},
+        }
+        if not args.no_e2e:
+            line["e2e"] = e2e_region(args, dist, dart, fwd["inputs"])
+        if not args.no_decode:
+            dec = decode_region(args, dist, dart, peaks)
+            line["decode"] = dec
+            line["gpu_launches"] += dec["launches"]
+        if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(fwd["inputs"])
+        if dist.rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        dist.close()
+
+
+if __name__ == "__main__":
+    main()

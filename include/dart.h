@@ -1,0 +1,196 @@
+/*
+ * dart.h -- C ABI of libdart.so, the sm_100a implementation of the DART layer
+ * hot path ("DART: Decoded Attention over Recurrent States for Efficient
+ * Long-Context Sequence Modeling").
+ *
+ * Three compute entry points, one per stage of the layer:
+ *   dart_ssd_chunk_scan  Mamba-2 SSD chunked scan that also writes out every
+ *                        chunk's state contribution dH[c] (the chunk memory);
+ *   dart_sma_forward     state-memory attention over those memories plus the
+ *                        gated residual;
+ *   dart_decode_step     one new token per sequence against the cache of
+ *                        chunk memories and the recurrent state.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Notation: B batch, L sequence length, H heads, P head dimension (value
+ *   axis), N state size (key axis), S chunk size, C = L / S chunks.  B and C
+ *   projections are shared by all heads (ngroups = 1).
+ * - Every tensor is dense, row-major (last index fastest), on the CUDA device
+ *   that is current for the calling thread, and 16-byte aligned.  Layouts:
+ *     x[B,L,H,P]  dt[B,L,H]  A[H]  Bm[B,L,N]  Cm[B,L,N]  Q[B,L,H,N]
+ *     E[B,L,H,P]  y[B,L,H,P]  dH[B,H,C,N,P]  states[B,H,C,N,P]
+ * - dtype selects the element type of x, Bm, Cm, Q, E and of the chunk
+ *   memories dH / the decode cache: DART_F32 (float) or DART_BF16
+ *   (__nv_bfloat16).  dt, A, y, states, the decode state and dH_cur are
+ *   always float.  Accumulation is always float.
+ * - Ownership: the caller allocates and owns every buffer, including the
+ *   optional workspace; the library keeps no device memory of its own apart
+ *   from one status word per device.
+ * - Execution: calls enqueue kernels on `stream` (a cudaStream_t; NULL is the
+ *   legacy default stream) and return without synchronising.  Arguments are
+ *   validated on the host before anything is enqueued; a rejected call
+ *   enqueues nothing and returns DART_ERR_INVALID_ARG or
+ *   DART_ERR_UNSUPPORTED, with a message in dart_last_error().  Conditions
+ *   only the device can see (a decode counter out of range, a bounded wait
+ *   that gave up) are latched in the device status word and reported by
+ *   dart_sync_status().  Nothing traps.
+ * - Thread safety: calls may be made from several host threads; each thread
+ *   has its own dart_last_error() message.
+ */
+#ifndef DART_H_
+#define DART_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    DART_OK = 0,
+    DART_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad size, bad counter */
+    DART_ERR_UNSUPPORTED = 2,  /* valid but not compiled: (N, P, S, dtype) combination */
+    DART_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed */
+    DART_ERR_TIMEOUT = 4,      /* a bounded device-side wait gave up */
+    DART_ERR_DEVICE = 5        /* the device flagged bad state (e.g. decode cache full) */
+} dart_status;
+
+typedef enum { DART_F32 = 0, DART_BF16 = 1 } dart_dtype;
+
+typedef struct {
+    int batch;    /* B (decode: number of sequences) */
+    int seqlen;   /* L, a multiple of chunk (ignored by dart_decode_step) */
+    int nheads;   /* H */
+    int headdim;  /* P, the value axis */
+    int dstate;   /* N, the key axis */
+    int chunk;    /* S */
+    int ngroups;  /* must be 1: B and C shared by all heads */
+} dart_dims;
+
+/*
+ * Workspace for dart_ssd_chunk_scan: B*H*C floats (the per-chunk sum of
+ * log-decays).  Pass at least this many bytes, 16-byte aligned.
+ */
+size_t dart_ssd_chunk_scan_workspace_bytes(const dart_dims* dims, dart_dtype dtype);
+
+/*
+ * Mamba-2 SSD chunked scan with retained chunk memories.
+ *
+ * Computes, per batch b and head h (Mamba-2 "Transformers are SSMs" SSD view,
+ * Eq. (4), which the DART pages build on; Pith review of DART, "What carries
+ * the argument"):
+ *   recurrence   H_t = exp(dt_t A_h) H_{t-1} + dt_t B_t x_t^T,  H_{-1} = init
+ *   output       y_ssd_t = H_t^T C_t   (the state already includes token t)
+ *   memory       dH[c] = sum_{s in chunk c} exp(sum_{r=s+1}^{e(c)} dt_r A_h)
+ *                         dt_s B_s x_s^T    (what chunk c adds to the state at
+ *                         its last token e(c); no decay beyond e(c))
+ *   boundary     states[c] = H_{e(c)}
+ * evaluated chunk-wise (intra-chunk quadratic block + inter-chunk state
+ * passing), not token by token.
+ *
+ *   x, Bm, Cm     dtype inputs; dt, A float inputs (dt > 0 after softplus,
+ *                 A < 0 per head).
+ *   init_state    nullable float [B,H,N,P]; NULL means zero.
+ *   y_ssd         float [B,L,H,P] output.
+ *   dH            dtype [B,H,C,N,P] output (rounded to nearest-even for bf16).
+ *   states        float [B,H,C,N,P] output.
+ *   workspace     device scratch of dart_ssd_chunk_scan_workspace_bytes().
+ * Requires L % S == 0, ngroups == 1, and (N, P, S, dtype) in the compiled set
+ * (see dart_supported()).
+ */
+dart_status dart_ssd_chunk_scan(const dart_dims* dims, dart_dtype dtype,
+                                const void* x, const float* dt, const float* A,
+                                const void* Bm, const void* Cm, const float* init_state,
+                                float* y_ssd, void* dH, float* states,
+                                void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * State-memory attention with the gated residual (Pith review of DART, "Core
+ * claim" and "What carries the argument"; SMA Eqs. (5)-(10)).  For token t in
+ * chunk k(t) = t / S and each chunk c < k(t):
+ *   value  v_{t,c} = C_t^T dH[c]            (P)
+ *   key    k_{t,c} = dH[c] E_t              (N)
+ *   score  s_{t,c} = Q_t . k_{t,c} / sqrt(N)
+ *   o_t = sum_c softmax_c(s_{t,c}) v_{t,c};   o_t = 0 when k(t) == 0.
+ * Memories are used as stored, without inter-chunk decay (referee comment 3
+ * on Eq. (8)).
+ *   out = y_ssd + g * o   when y_ssd != NULL (the DART layer output), else
+ *   out = o               (the raw readout).
+ *   Q[B,L,H,N], E[B,L,H,P], Cm[B,L,N], dH[B,H,C,N,P]: dtype inputs.
+ *   y_ssd: nullable float [B,L,H,P]; out: float [B,L,H,P] (may alias y_ssd).
+ */
+dart_status dart_sma_forward(const dart_dims* dims, dart_dtype dtype,
+                             const void* Q, const void* E, const void* Cm, const void* dH,
+                             float g, const float* y_ssd, float* out, void* stream);
+
+/*
+ * Workspace for dart_decode_step: per (sequence, head, split) partial softmax
+ * statistics and partial outputs.  Pass at least this many bytes.
+ */
+size_t dart_decode_step_workspace_bytes(const dart_dims* dims, dart_dtype dtype, int cmax);
+
+/*
+ * One decode step for dims->batch sequences (DART abstract and Pith review
+ * "If this is right": the length-dependent inference cache is the set of
+ * chunk memories).  Per sequence b and head h, with n = n_chunks[b] completed
+ * memories and pos = pos[b] the index of the incoming token inside its chunk:
+ *   a = exp(dt A_h);  state = a state + dt B x^T;  dH_cur = a dH_cur + dt B x^T
+ *   y = state^T C + g * SMA(Q, E, C; dH_cache[b,h,0..n-1])
+ *   if pos == S-1:  dH_cache[b,h,n] = dH_cur (rounded to dtype);
+ *                   dH_cur = 0;  n_chunks[b] = n + 1;  pos[b] = 0
+ *   else            pos[b] = pos + 1
+ *   x_t[B,H,P], B_t[B,N], C_t[B,N], Q_t[B,H,N], E_t[B,H,P]: dtype inputs;
+ *   dt_t[B,H], A[H]: float inputs.
+ *   state, dH_cur: float [B,H,N,P], in/out.
+ *   dH_cache: dtype [B,H,cmax,N,P], in/out (slots >= n are not read).
+ *   n_chunks, pos: int32 [B] device arrays, in/out.
+ *   y: float [B,H,P] output.
+ * A sequence whose counters are out of range (n > cmax, pos outside [0,S),
+ * or an append with n == cmax) produces no output update for that sequence,
+ * leaves its state untouched and latches DART_ERR_DEVICE.
+ */
+dart_status dart_decode_step(const dart_dims* dims, dart_dtype dtype,
+                             const void* x_t, const float* dt_t, const float* A,
+                             const void* B_t, const void* C_t, const void* Q_t, const void* E_t,
+                             float g, float* state, float* dH_cur, void* dH_cache, int cmax,
+                             int* n_chunks, int* pos, float* y,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * 1 when (dstate N, headdim P, chunk S, dtype) is compiled in, else 0.
+ */
+int dart_supported(int dstate, int headdim, int chunk, dart_dtype dtype);
+
+/*
+ * Name of the kernel dart_sma_forward dispatches to for this shape and dtype
+ * ("sma_simt" on CUDA cores, "sma_tcgen05" on the tensor cores), or "" when
+ * the combination is not compiled.  The string is static.
+ */
+const char* dart_sma_impl(int dstate, int headdim, int chunk, dart_dtype dtype);
+
+/*
+ * Synchronises `stream`, then returns and clears the device status word of
+ * the current device: DART_OK, DART_ERR_TIMEOUT or DART_ERR_DEVICE (or
+ * DART_ERR_CUDA if the synchronisation itself failed).
+ */
+dart_status dart_sync_status(void* stream);
+
+/* Message describing the last failure on the calling host thread ("" if none). */
+const char* dart_last_error(void);
+
+/* ABI version, bumped on any signature change. */
+int dart_abi_version(void);
+
+/*
+ * Number of CUDA kernels this library has enqueued since it was loaded
+ * (process-wide, all devices and threads).  Lets a caller count the launches
+ * inside a region without a profiler.
+ */
+unsigned long long dart_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DART_H_ */

@@ -1,0 +1,203 @@
+// dart_abi.cu -- the extern "C" surface declared in include/dart.h:
+// host-side validation, workspace sizing, dispatch to the kernel families and
+// the device status word.
+#include <atomic>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "dart_common.cuh"
+
+namespace dart {
+__device__ int g_status = 0;
+
+namespace {
+std::atomic<unsigned long long> g_launches{0};
+}  // namespace
+
+void count_launches(int n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
+}  // namespace dart
+
+namespace {
+
+// Device address of the status word on the current device (looked up once
+// per device; the lookup is idempotent, so a race only repeats it).
+int* status_word() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    static int* cache[64] = {};
+    if (!cache[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, dart::g_status) != cudaSuccess) return nullptr;
+        cache[dev] = static_cast<int*>(p);
+    }
+    return cache[dev];
+}
+
+thread_local char t_err[512] = "";
+
+dart_status fail(dart_status st, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(t_err, sizeof(t_err), fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+dart_status cuda_fail(cudaError_t e, const char* where) {
+    return fail(DART_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+#define DART_REQUIRE_PTR(p)                                                           \
+    do {                                                                              \
+        if (!(p)) return fail(DART_ERR_INVALID_ARG, "%s: null pointer", #p);          \
+        if (!aligned16(p)) return fail(DART_ERR_INVALID_ARG, "%s: not 16-byte aligned", #p); \
+    } while (0)
+
+#define DART_OPTIONAL_PTR(p)                                                          \
+    do {                                                                              \
+        if ((p) && !aligned16(p))                                                     \
+            return fail(DART_ERR_INVALID_ARG, "%s: not 16-byte aligned", #p);         \
+    } while (0)
+
+dart_status check_common(const dart_dims* d, dart_dtype dt, bool need_seqlen) {
+    if (!d) return fail(DART_ERR_INVALID_ARG, "dims: null pointer");
+    if (dt != DART_F32 && dt != DART_BF16) return fail(DART_ERR_INVALID_ARG, "dtype: unknown value %d", (int)dt);
+    if (d->batch < 1 || d->nheads < 1 || d->headdim < 1 || d->dstate < 1 || d->chunk < 1)
+        return fail(DART_ERR_INVALID_ARG, "dims: batch, nheads, headdim, dstate and chunk must be >= 1");
+    if (d->ngroups != 1) return fail(DART_ERR_UNSUPPORTED, "ngroups = %d: only 1 (B, C shared by all heads)", d->ngroups);
+    if (need_seqlen) {
+        if (d->seqlen < 1) return fail(DART_ERR_INVALID_ARG, "dims: seqlen must be >= 1");
+        if (d->seqlen % d->chunk != 0)
+            return fail(DART_ERR_UNSUPPORTED, "seqlen %d is not a multiple of chunk %d", d->seqlen, d->chunk);
+    }
+    if (d->batch > 65535 || d->nheads > 65535)
+        return fail(DART_ERR_UNSUPPORTED, "batch and nheads must be <= 65535");
+    return DART_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int dart_abi_version(void) { return 1; }
+
+unsigned long long dart_launch_count(void) { return dart::g_launches.load(std::memory_order_relaxed); }
+
+const char* dart_last_error(void) { return t_err; }
+
+int dart_supported(int dstate, int headdim, int chunk, dart_dtype dtype) {
+    if (dtype != DART_F32 && dtype != DART_BF16) return 0;
+    return dart::ssd_scan_supported(dstate, headdim, chunk, dtype) &&
+           dart::sma_supported(dstate, headdim, chunk, dtype) &&
+           dart::decode_supported(dstate, headdim, chunk, dtype);
+}
+
+const char* dart_sma_impl(int dstate, int headdim, int chunk, dart_dtype dtype) {
+    if ((dtype != DART_F32 && dtype != DART_BF16) || !dart::sma_supported(dstate, headdim, chunk, dtype))
+        return "";
+    return dart::sma_impl_name(dstate, headdim, chunk, dtype);
+}
+
+size_t dart_ssd_chunk_scan_workspace_bytes(const dart_dims* d, dart_dtype) {
+    if (!d || d->chunk < 1) return 0;
+    const size_t C = (size_t)(d->seqlen / d->chunk);
+    return sizeof(float) * (size_t)d->batch * (size_t)d->nheads * C;
+}
+
+dart_status dart_ssd_chunk_scan(const dart_dims* d, dart_dtype dtype, const void* x, const float* dt,
+                                const float* A, const void* Bm, const void* Cm, const float* init_state,
+                                float* y_ssd, void* dH, float* states, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+    t_err[0] = 0;
+    dart_status st = check_common(d, dtype, true);
+    if (st != DART_OK) return st;
+    if (!dart::ssd_scan_supported(d->dstate, d->headdim, d->chunk, dtype))
+        return fail(DART_ERR_UNSUPPORTED, "dart_ssd_chunk_scan: (N=%d, P=%d, S=%d) not compiled",
+                    d->dstate, d->headdim, d->chunk);
+    DART_REQUIRE_PTR(x); DART_REQUIRE_PTR(dt); DART_REQUIRE_PTR(A); DART_REQUIRE_PTR(Bm);
+    DART_REQUIRE_PTR(Cm); DART_OPTIONAL_PTR(init_state); DART_REQUIRE_PTR(y_ssd);
+    DART_REQUIRE_PTR(dH); DART_REQUIRE_PTR(states); DART_REQUIRE_PTR(workspace);
+    if (workspace_bytes < dart_ssd_chunk_scan_workspace_bytes(d, dtype))
+        return fail(DART_ERR_INVALID_ARG, "workspace: %zu bytes, need %zu", workspace_bytes,
+                    dart_ssd_chunk_scan_workspace_bytes(d, dtype));
+    dart::ScanArgs a{d->batch, d->seqlen, d->nheads, d->headdim, d->dstate, d->chunk,
+                     x, dt, A, Bm, Cm, init_state, y_ssd, dH, states, static_cast<float*>(workspace)};
+    cudaError_t e = dart::launch_ssd_scan(a, dtype, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "dart_ssd_chunk_scan launch");
+    return DART_OK;
+}
+
+dart_status dart_sma_forward(const dart_dims* d, dart_dtype dtype, const void* Q, const void* E,
+                             const void* Cm, const void* dH, float g, const float* y_ssd, float* out,
+                             void* stream) {
+    t_err[0] = 0;
+    dart_status st = check_common(d, dtype, true);
+    if (st != DART_OK) return st;
+    if (!dart::sma_supported(d->dstate, d->headdim, d->chunk, dtype))
+        return fail(DART_ERR_UNSUPPORTED, "dart_sma_forward: (N=%d, P=%d, S=%d) not compiled",
+                    d->dstate, d->headdim, d->chunk);
+    DART_REQUIRE_PTR(Q); DART_REQUIRE_PTR(E); DART_REQUIRE_PTR(Cm); DART_REQUIRE_PTR(dH);
+    DART_OPTIONAL_PTR(y_ssd); DART_REQUIRE_PTR(out);
+    dart::SmaArgs a{d->batch, d->seqlen, d->nheads, d->headdim, d->dstate, d->chunk,
+                    Q, E, Cm, dH, g, y_ssd, out};
+    cudaError_t e = dart::launch_sma(a, dtype, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "dart_sma_forward launch");
+    return DART_OK;
+}
+
+size_t dart_decode_step_workspace_bytes(const dart_dims* d, dart_dtype, int cmax) {
+    if (!d || cmax < 0) return 0;
+    const size_t ns = (size_t)dart::decode_num_splits(d->batch, d->nheads, cmax);
+    return sizeof(float) * (size_t)d->batch * (size_t)d->nheads * ns * (2 + 2 * (size_t)d->headdim);
+}
+
+dart_status dart_decode_step(const dart_dims* d, dart_dtype dtype, const void* x_t, const float* dt_t,
+                             const float* A, const void* B_t, const void* C_t, const void* Q_t,
+                             const void* E_t, float g, float* state, float* dH_cur, void* dH_cache,
+                             int cmax, int* n_chunks, int* pos, float* y, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+    t_err[0] = 0;
+    dart_status st = check_common(d, dtype, false);
+    if (st != DART_OK) return st;
+    if (!dart::decode_supported(d->dstate, d->headdim, d->chunk, dtype))
+        return fail(DART_ERR_UNSUPPORTED, "dart_decode_step: (N=%d, P=%d) not compiled", d->dstate, d->headdim);
+    if (cmax < 1) return fail(DART_ERR_INVALID_ARG, "cmax must be >= 1");
+    DART_REQUIRE_PTR(x_t); DART_REQUIRE_PTR(dt_t); DART_REQUIRE_PTR(A); DART_REQUIRE_PTR(B_t);
+    DART_REQUIRE_PTR(C_t); DART_REQUIRE_PTR(Q_t); DART_REQUIRE_PTR(E_t); DART_REQUIRE_PTR(state);
+    DART_REQUIRE_PTR(dH_cur); DART_REQUIRE_PTR(dH_cache); DART_REQUIRE_PTR(n_chunks);
+    DART_REQUIRE_PTR(pos); DART_REQUIRE_PTR(y); DART_REQUIRE_PTR(workspace);
+    if (workspace_bytes < dart_decode_step_workspace_bytes(d, dtype, cmax))
+        return fail(DART_ERR_INVALID_ARG, "workspace: %zu bytes, need %zu", workspace_bytes,
+                    dart_decode_step_workspace_bytes(d, dtype, cmax));
+    dart::DecodeArgs a{d->batch, d->nheads, d->headdim, d->dstate, d->chunk, cmax,
+                       dart::decode_num_splits(d->batch, d->nheads, cmax),
+                       x_t, dt_t, A, B_t, C_t, Q_t, E_t, g, state, dH_cur, dH_cache,
+                       n_chunks, pos, y, static_cast<float*>(workspace), status_word()};
+    if (!a.status) return fail(DART_ERR_CUDA, "dart_decode_step: no device status word");
+    cudaError_t e = dart::launch_decode(a, dtype, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "dart_decode_step launch");
+    return DART_OK;
+}
+
+dart_status dart_sync_status(void* stream) {
+    t_err[0] = 0;
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "dart_sync_status: stream synchronize");
+    int flags = 0;
+    e = cudaMemcpyFromSymbol(&flags, dart::g_status, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e, "dart_sync_status: read status");
+    if (flags) {
+        const int zero = 0;
+        e = cudaMemcpyToSymbol(dart::g_status, &zero, sizeof(int));
+        if (e != cudaSuccess) return cuda_fail(e, "dart_sync_status: clear status");
+    }
+    if (flags & dart::kStatusTimeout) return fail(DART_ERR_TIMEOUT, "a bounded device wait gave up");
+    if (flags & dart::kStatusDevice)
+        return fail(DART_ERR_DEVICE, "device flagged bad state (decode counters out of range or cache full)");
+    return DART_OK;
+}
+
+}  // extern "C"

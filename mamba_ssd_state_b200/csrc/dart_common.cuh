@@ -1,0 +1,133 @@
+// dart_common.cuh -- small device helpers shared by the DART kernels.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/dart.h"
+
+namespace dart {
+
+// Device status word bits (latched by kernels, read by dart_sync_status).
+enum : int {
+    kStatusTimeout = 1,   // a bounded wait gave up
+    kStatusDevice = 2,    // bad device-side state (decode counters / cache full)
+};
+
+// The status word lives in dart_abi.cu (one per device); kernels receive its
+// device address and set bits with atomicOr.
+__device__ __forceinline__ void flag_status(int* status, int bits) { atomicOr(status, bits); }
+
+// ---------------------------------------------------------------------------
+// element conversion
+// ---------------------------------------------------------------------------
+template <typename T> struct Elem;
+template <> struct Elem<float> {
+    static __device__ __forceinline__ float to_f(float v) { return v; }
+    static __device__ __forceinline__ float from_f(float v) { return v; }
+};
+template <> struct Elem<__nv_bfloat16> {
+    static __device__ __forceinline__ float to_f(__nv_bfloat16 v) { return __bfloat162float(v); }
+    static __device__ __forceinline__ __nv_bfloat16 from_f(float v) { return __float2bfloat16_rn(v); }
+};
+
+template <typename T> __device__ __forceinline__ float ldf(const T* p) { return Elem<T>::to_f(*p); }
+
+// 16-byte vector of T unpacked to floats: 4 floats or 8 bf16.
+template <typename T> struct Vec16;
+template <> struct Vec16<float> {
+    static constexpr int kN = 4;
+    static __device__ __forceinline__ void load(const float* p, float* out) {
+        float4 v = *reinterpret_cast<const float4*>(p);
+        out[0] = v.x; out[1] = v.y; out[2] = v.z; out[3] = v.w;
+    }
+    static __device__ __forceinline__ void load_nc(const float* p, float* out) {
+        float4 v = __ldg(reinterpret_cast<const float4*>(p));
+        out[0] = v.x; out[1] = v.y; out[2] = v.z; out[3] = v.w;
+    }
+    static __device__ __forceinline__ void store(float* p, const float* in) {
+        *reinterpret_cast<float4*>(p) = make_float4(in[0], in[1], in[2], in[3]);
+    }
+};
+template <> struct Vec16<__nv_bfloat16> {
+    static constexpr int kN = 8;
+    static __device__ __forceinline__ void unpack(uint4 v, float* out) {
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            out[2 * i] = __uint_as_float(w[i] << 16);
+            out[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+        }
+    }
+    static __device__ __forceinline__ void load(const __nv_bfloat16* p, float* out) {
+        unpack(*reinterpret_cast<const uint4*>(p), out);
+    }
+    static __device__ __forceinline__ void load_nc(const __nv_bfloat16* p, float* out) {
+        unpack(__ldg(reinterpret_cast<const uint4*>(p)), out);
+    }
+    static __device__ __forceinline__ void store(__nv_bfloat16* p, const float* in) {
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            __nv_bfloat162 h = __floats2bfloat162_rn(in[2 * i], in[2 * i + 1]);
+            w[i] = *reinterpret_cast<uint32_t*>(&h);
+        }
+        *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+};
+
+// Streaming 16-byte load that does not allocate in L1 (read-once data).
+__device__ __forceinline__ uint4 ld_stream_u4(const void* p) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// log2(e): the softmax runs in base 2 on scores pre-multiplied by it.
+constexpr float kLog2e = 1.4426950408889634f;
+
+}  // namespace dart
+
+// Host-side launch helpers implemented per kernel family.
+namespace dart {
+struct ScanArgs {
+    int B, L, H, P, N, S;
+    const void* x; const float* dt; const float* A; const void* Bm; const void* Cm;
+    const float* init_state;
+    float* y; void* dH; float* states; float* asum;  // asum: [B,H,C] workspace
+};
+struct SmaArgs {
+    int B, L, H, P, N, S;
+    const void* Q; const void* E; const void* Cm; const void* dH;
+    float g; const float* y_ssd; float* out;
+};
+struct DecodeArgs {
+    int B, H, P, N, S, cmax, nsplit;
+    const void* x; const float* dt; const float* A; const void* Bm; const void* Cm;
+    const void* Q; const void* E; float g;
+    float* state; float* dHcur; void* cache; int* nchunks; int* pos; float* y;
+    float* part;  // [B,H,nsplit,2+2P] workspace
+    int* status;  // device status word
+};
+
+// Counts one kernel launch (see dart_launch_count).
+void count_launches(int n);
+
+cudaError_t launch_ssd_scan(const ScanArgs& a, dart_dtype dt, cudaStream_t st);
+cudaError_t launch_sma(const SmaArgs& a, dart_dtype dt, cudaStream_t st);
+cudaError_t launch_decode(const DecodeArgs& a, dart_dtype dt, cudaStream_t st);
+bool ssd_scan_supported(int N, int P, int S, dart_dtype dt);
+bool sma_supported(int N, int P, int S, dart_dtype dt);
+const char* sma_impl_name(int N, int P, int S, dart_dtype dt);
+bool decode_supported(int N, int P, int S, dart_dtype dt);
+int decode_num_splits(int B, int H, int cmax);
+}  // namespace dart

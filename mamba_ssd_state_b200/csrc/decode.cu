@@ -1,0 +1,268 @@
+// decode.cu -- one DART decode step: recurrent update, SSM readout and
+// state-memory attention over the cache of chunk memories.
+//
+// The cache is the length-dependent part of DART's inference state (DART
+// abstract; Pith review, "If this is right": N/(2S) of a token-level KV cache,
+// Eq. (14)).  A step streams every cached memory once, so the kernel is bound
+// by HBM bandwidth: each warp reads whole memories with coalesced 16-byte
+// non-allocating loads and reduces with warp shuffles; nothing goes through
+// shared memory on the streaming path.
+//
+// decode_partial  grid (split, h, b), 4 warps.  Split j owns
+//   - rows [j*N/ns, (j+1)*N/ns) of the state and of dH_cur: updates them,
+//     appends them to the cache when the token closes its chunk, and forms
+//     their part of y_ssd = state^T C;
+//   - cached memories c in [j*cps, (j+1)*cps) with c < n: per memory
+//     v = C^T dH[c], s = (Q^T dH[c]) . E / sqrt(N), merged into one online
+//     softmax per block.
+//   Writes (m, l, o[P], y_ssd part[P]) for the split to the workspace.
+// decode_combine  grid (h, b): merges the splits, y = y_ssd + g * o.
+// decode_advance  one thread per sequence: advances (n_chunks, pos) after
+//   every block of the step has read them.
+#include "dart_common.cuh"
+
+namespace dart {
+namespace {
+
+constexpr int kWarps = 4;
+constexpr int kThreads = 32 * kWarps;
+constexpr int kChunksPerSplit = 16;
+
+struct SeqCounters {
+    int n, pos;
+    bool ok, append;
+};
+
+__device__ __forceinline__ SeqCounters read_counters(const DecodeArgs& a, int b) {
+    SeqCounters s;
+    s.n = a.nchunks[b];
+    s.pos = a.pos[b];
+    s.ok = s.n >= 0 && s.n <= a.cmax && s.pos >= 0 && s.pos < a.S;
+    s.append = s.ok && s.pos == a.S - 1;
+    if (s.append && s.n >= a.cmax) s.ok = false;
+    return s;
+}
+
+template <typename T, int N, int P>
+__global__ void __launch_bounds__(kThreads) decode_partial_kernel(DecodeArgs a) {
+    constexpr int VEC = Vec16<T>::kN;        // elements per 16-byte load
+    constexpr int LPR = P / VEC;             // lanes per memory row
+    constexpr int RPW = 32 / LPR;            // rows per warp load
+    static_assert(32 % LPR == 0 && N % RPW == 0, "unsupported (N, P) for decode");
+    constexpr int STRIDE = 2 + 2 * P;
+
+    const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int ns = gridDim.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const SeqCounters sc = read_counters(a, b);
+    float* part = a.part + (((size_t)b * a.H + h) * ns + split) * STRIDE;
+    if (!sc.ok) {
+        if (split == 0 && h == 0 && tid == 0) flag_status(a.status, kStatusDevice);
+        return;
+    }
+    __shared__ float q_s[N], c_s[N], x_s[P];
+    __shared__ float red_m[kWarps], red_l[kWarps], red_o[kWarps][P];
+    __shared__ float ypart[kThreads];
+
+    const size_t bh = (size_t)b * a.H + h;
+    const T* xt = static_cast<const T*>(a.x) + bh * P;
+    const T* Bt = static_cast<const T*>(a.Bm) + (size_t)b * N;
+    const T* Ct = static_cast<const T*>(a.Cm) + (size_t)b * N;
+    const T* Qt = static_cast<const T*>(a.Q) + bh * N;
+    const T* Et = static_cast<const T*>(a.E) + bh * P;
+    const float qscale = kLog2e * rsqrtf((float)N);
+    for (int i = tid; i < N; i += kThreads) {
+        q_s[i] = qscale * ldf(Qt + i);
+        c_s[i] = ldf(Ct + i);
+    }
+    for (int i = tid; i < P; i += kThreads) x_s[i] = ldf(xt + i);
+    __syncthreads();
+
+    // ---- recurrent update of this split's rows --------------------------
+    {
+        const float dt = a.dt[bh];
+        const float decay = expf(dt * a.A[h]);
+        const int r0 = split * N / ns, r1 = (split + 1) * N / ns;
+        float* st = a.state + bh * N * P;
+        float* dc = a.dHcur + bh * N * P;
+        T* slot = static_cast<T*>(a.cache) + (bh * a.cmax + sc.n) * (size_t)N * P;
+        float yp = 0.f;  // thread owns column p = tid % P when P divides kThreads
+        for (int i = r0 * P + tid; i < r1 * P; i += kThreads) {
+            const int n = i / P, p = i % P;
+            const float inp = dt * ldf(Bt + n) * x_s[p];
+            const float hv = fmaf(decay, st[i], inp);
+            const float dv = fmaf(decay, dc[i], inp);
+            st[i] = hv;
+            if (sc.append) {
+                slot[i] = Elem<T>::from_f(dv);
+                dc[i] = 0.f;
+            } else {
+                dc[i] = dv;
+            }
+            yp = fmaf(c_s[n], hv, yp);
+        }
+        ypart[tid] = yp;
+    }
+
+    // ---- state-memory attention over this split's cached chunks ----------
+    const int lrow = lane / LPR;             // row inside a warp load
+    const int pcol = (lane % LPR) * VEC;     // first column of this lane
+    float ev[VEC];
+    {
+        float tmp[VEC];
+#pragma unroll
+        for (int j = 0; j < VEC; ++j) tmp[j] = ldf(Et + pcol + j);
+#pragma unroll
+        for (int j = 0; j < VEC; ++j) ev[j] = tmp[j];
+    }
+    float m = -INFINITY, l = 0.f, o[VEC];
+#pragma unroll
+    for (int j = 0; j < VEC; ++j) o[j] = 0.f;
+    const int c_begin = split * kChunksPerSplit;
+    const int c_end = min(sc.n, c_begin + kChunksPerSplit);
+    const T* cache = static_cast<const T*>(a.cache) + bh * a.cmax * (size_t)N * P;
+    for (int c = c_begin + warp; c < c_end; c += kWarps) {
+        const T* mem = cache + (size_t)c * N * P + (size_t)lrow * P + pcol;
+        float v[VEC], s = 0.f;
+#pragma unroll
+        for (int j = 0; j < VEC; ++j) v[j] = 0.f;
+        constexpr int ITER = N / RPW;
+        constexpr int UNROLL = ITER < 8 ? ITER : 8;
+#pragma unroll
+        for (int i0 = 0; i0 < ITER; i0 += UNROLL) {
+            uint4 raw[UNROLL];
+#pragma unroll
+            for (int u = 0; u < UNROLL; ++u) raw[u] = ld_stream_u4(mem + (size_t)(i0 + u) * RPW * P);
+#pragma unroll
+            for (int u = 0; u < UNROLL; ++u) {
+                const int n = lrow + (i0 + u) * RPW;
+                float mv[VEC];
+                if constexpr (VEC == 8) {
+                    Vec16<__nv_bfloat16>::unpack(raw[u], mv);
+                } else {
+                    mv[0] = __uint_as_float(raw[u].x); mv[1] = __uint_as_float(raw[u].y);
+                    mv[2] = __uint_as_float(raw[u].z); mv[3] = __uint_as_float(raw[u].w);
+                }
+                float rd = 0.f;
+#pragma unroll
+                for (int j = 0; j < VEC; ++j) {
+                    v[j] = fmaf(c_s[n], mv[j], v[j]);
+                    rd = fmaf(mv[j], ev[j], rd);
+                }
+                s = fmaf(q_s[n], rd, s);
+            }
+        }
+        // v: sum over lanes holding the same columns; s: sum over the warp
+#pragma unroll
+        for (int off = LPR; off < 32; off <<= 1)
+#pragma unroll
+            for (int j = 0; j < VEC; ++j) v[j] += __shfl_xor_sync(0xffffffffu, v[j], off);
+        s = warp_sum(s);
+        const float mnew = fmaxf(m, s);
+        const float alpha = exp2f(m - mnew);
+        const float w = exp2f(s - mnew);
+        l = l * alpha + w;
+#pragma unroll
+        for (int j = 0; j < VEC; ++j) o[j] = fmaf(o[j], alpha, w * v[j]);
+        m = mnew;
+    }
+    if (lane == 0) { red_m[warp] = m; red_l[warp] = l; }
+    if (lrow == 0) {
+#pragma unroll
+        for (int j = 0; j < VEC; ++j) red_o[warp][pcol + j] = o[j];
+    }
+    __syncthreads();
+    if (tid < P) {
+        float mm = -INFINITY;
+        for (int w = 0; w < kWarps; ++w) mm = fmaxf(mm, red_m[w]);
+        float ll = 0.f, oo = 0.f;
+        if (mm != -INFINITY) {
+            for (int w = 0; w < kWarps; ++w) {
+                const float f = exp2f(red_m[w] - mm);
+                ll = fmaf(red_l[w], f, ll);
+                oo = fmaf(red_o[w][tid], f, oo);
+            }
+        }
+        float yp = 0.f;
+        for (int i = tid; i < kThreads; i += P) yp += ypart[i];
+        if (tid == 0) { part[0] = mm; part[1] = ll; }
+        part[2 + tid] = oo;
+        part[2 + P + tid] = yp;
+    }
+}
+
+template <int P>
+__global__ void __launch_bounds__(P) decode_combine_kernel(DecodeArgs a) {
+    constexpr int STRIDE = 2 + 2 * P;
+    const int h = blockIdx.x, b = blockIdx.y, p = threadIdx.x;
+    const SeqCounters sc = read_counters(a, b);
+    if (!sc.ok) return;
+    const int ns = a.nsplit;
+    const float* part = a.part + ((size_t)b * a.H + h) * ns * STRIDE;
+    float mm = -INFINITY;
+    for (int j = 0; j < ns; ++j) mm = fmaxf(mm, part[j * STRIDE]);
+    float l = 0.f, o = 0.f, y = 0.f;
+    for (int j = 0; j < ns; ++j) {
+        const float* pj = part + j * STRIDE;
+        if (mm != -INFINITY) {
+            const float f = exp2f(pj[0] - mm);
+            l = fmaf(pj[1], f, l);
+            o = fmaf(pj[2 + p], f, o);
+        }
+        y += pj[2 + P + p];
+    }
+    const float oo = l > 0.f ? o / l : 0.f;
+    a.y[((size_t)b * a.H + h) * P + p] = fmaf(a.g, oo, y);
+}
+
+// Advances the per-sequence counters once every head has read them.
+__global__ void decode_advance_kernel(DecodeArgs a) {
+    const int b = blockIdx.x * blockDim.x + threadIdx.x;
+    if (b >= a.B) return;
+    const SeqCounters sc = read_counters(a, b);
+    if (!sc.ok) return;
+    if (sc.append) {
+        a.nchunks[b] = sc.n + 1;
+        a.pos[b] = 0;
+    } else {
+        a.pos[b] = sc.pos + 1;
+    }
+}
+
+template <typename T, int N, int P>
+cudaError_t run(const DecodeArgs& a, cudaStream_t st) {
+    decode_partial_kernel<T, N, P><<<dim3(a.nsplit, a.H, a.B), kThreads, 0, st>>>(a);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    decode_combine_kernel<P><<<dim3(a.H, a.B), P, 0, st>>>(a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    decode_advance_kernel<<<(a.B + 127) / 128, 128, 0, st>>>(a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    count_launches(3);
+    return cudaSuccess;
+}
+
+}  // namespace
+
+int decode_num_splits(int, int, int cmax) {
+    const int ns = (cmax + kChunksPerSplit - 1) / kChunksPerSplit;
+    return ns < 1 ? 1 : ns;
+}
+
+bool decode_supported(int N, int P, int S, dart_dtype) {
+    const bool np = (N == 16 && P == 16) || (N == 64 && P == 64) || (N == 128 && P == 64);
+    return np && S >= 1;
+}
+
+cudaError_t launch_decode(const DecodeArgs& a, dart_dtype dt, cudaStream_t st) {
+#define DART_DEC_CASE(NN, PP)                                                       \
+    if (a.N == NN && a.P == PP)                                                     \
+        return dt == DART_F32 ? run<float, NN, PP>(a, st) : run<__nv_bfloat16, NN, PP>(a, st);
+    DART_DEC_CASE(16, 16)
+    DART_DEC_CASE(64, 64)
+    DART_DEC_CASE(128, 64)
+#undef DART_DEC_CASE
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace dart

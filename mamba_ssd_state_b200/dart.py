@@ -1,0 +1,295 @@
+"""Python binding of libdart.so (argument marshalling only).
+
+Every computation runs in the library's CUDA kernels; this module checks
+tensor shapes/dtypes, allocates outputs and workspaces with PyTorch (device
+memory and streams are PyTorch's), and passes raw pointers plus the current
+CUDA stream to the C ABI declared in ``include/dart.h``.  The functions carry
+the C names.  Inputs given as CPU tensors are copied to the device first and
+the results copied back (the host-buffer path), so the same calls serve
+device-resident and host-resident data.
+
+There is no fallback: if the library is missing or no CUDA device is present
+the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIBRARY = os.path.join(_HERE, "libdart.so")
+
+DART_OK, DART_ERR_INVALID_ARG, DART_ERR_UNSUPPORTED, DART_ERR_CUDA, DART_ERR_TIMEOUT, DART_ERR_DEVICE = range(6)
+DART_F32, DART_BF16 = 0, 1
+_STATUS = {0: "DART_OK", 1: "DART_ERR_INVALID_ARG", 2: "DART_ERR_UNSUPPORTED", 3: "DART_ERR_CUDA",
+           4: "DART_ERR_TIMEOUT", 5: "DART_ERR_DEVICE"}
+
+# every symbol include/dart.h declares
+EXPORTS = ("dart_ssd_chunk_scan_workspace_bytes", "dart_ssd_chunk_scan", "dart_sma_forward",
+           "dart_decode_step_workspace_bytes", "dart_decode_step", "dart_supported",
+           "dart_sync_status", "dart_last_error", "dart_abi_version", "dart_launch_count",
+           "dart_sma_impl")
+
+
+class DartError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{_STATUS.get(status, status)}: {message}")
+        self.status = status
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in
+                ("batch", "seqlen", "nheads", "headdim", "dstate", "chunk", "ngroups")]
+
+
+_P = ctypes.c_void_p
+_lib = None
+
+
+def load(path: str = LIBRARY) -> ctypes.CDLL:
+    """Load libdart.so (raises OSError if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise OSError(f"{path} not found: build it with `python -m mamba_ssd_state_b200.build`")
+    lib = ctypes.CDLL(path)
+    D = ctypes.POINTER(Dims)
+    lib.dart_ssd_chunk_scan_workspace_bytes.restype = ctypes.c_size_t
+    lib.dart_ssd_chunk_scan_workspace_bytes.argtypes = [D, ctypes.c_int]
+    lib.dart_ssd_chunk_scan.restype = ctypes.c_int
+    lib.dart_ssd_chunk_scan.argtypes = [D, ctypes.c_int] + [_P] * 10 + [ctypes.c_size_t, _P]
+    lib.dart_sma_forward.restype = ctypes.c_int
+    lib.dart_sma_forward.argtypes = [D, ctypes.c_int] + [_P] * 4 + [ctypes.c_float, _P, _P, _P]
+    lib.dart_decode_step_workspace_bytes.restype = ctypes.c_size_t
+    lib.dart_decode_step_workspace_bytes.argtypes = [D, ctypes.c_int, ctypes.c_int]
+    lib.dart_decode_step.restype = ctypes.c_int
+    lib.dart_decode_step.argtypes = ([D, ctypes.c_int] + [_P] * 7 + [ctypes.c_float] + [_P] * 3
+                                     + [ctypes.c_int] + [_P] * 4 + [ctypes.c_size_t, _P])
+    lib.dart_supported.restype = ctypes.c_int
+    lib.dart_supported.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int]
+    lib.dart_sync_status.restype = ctypes.c_int
+    lib.dart_sync_status.argtypes = [_P]
+    lib.dart_last_error.restype = ctypes.c_char_p
+    lib.dart_last_error.argtypes = []
+    lib.dart_abi_version.restype = ctypes.c_int
+    lib.dart_abi_version.argtypes = []
+    lib.dart_launch_count.restype = ctypes.c_ulonglong
+    lib.dart_launch_count.argtypes = []
+    lib.dart_sma_impl.restype = ctypes.c_char_p
+    lib.dart_sma_impl.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int]
+    _lib = lib
+    return lib
+
+
+def _check(rc: int):
+    if rc != DART_OK:
+        raise DartError(rc, load().dart_last_error().decode())
+
+
+def _dtype_code(t: torch.dtype) -> int:
+    if t == torch.float32:
+        return DART_F32
+    if t == torch.bfloat16:
+        return DART_BF16
+    raise TypeError(f"unsupported dtype {t}; use float32 or bfloat16")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream() -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _dev(t: Optional[torch.Tensor], device, dtype=None) -> Optional[torch.Tensor]:
+    """Contiguous tensor on `device` (copying host tensors there)."""
+    if t is None:
+        return None
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"expected {dtype}, got {t.dtype}")
+    if t.device != device:
+        t = t.to(device, non_blocking=True)
+    return t.contiguous()
+
+
+def _device_of(*ts) -> torch.device:
+    for t in ts:
+        if isinstance(t, torch.Tensor) and t.is_cuda:
+            return t.device
+    if not torch.cuda.is_available():
+        raise RuntimeError("dart: no CUDA device available (there is no CPU path)")
+    return torch.device("cuda", torch.cuda.current_device())
+
+
+def _shape(name, t, shape):
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def supported(dstate: int, headdim: int, chunk: int, dtype: torch.dtype) -> bool:
+    return bool(load().dart_supported(dstate, headdim, chunk, _dtype_code(dtype)))
+
+
+def abi_version() -> int:
+    return load().dart_abi_version()
+
+
+def sma_impl(dstate: int, headdim: int, chunk: int, dtype: torch.dtype) -> str:
+    """Which SMA kernel the library dispatches to for this shape/dtype."""
+    return load().dart_sma_impl(dstate, headdim, chunk, _dtype_code(dtype)).decode()
+
+
+def launch_count() -> int:
+    """Kernels the library has enqueued so far in this process."""
+    return int(load().dart_launch_count())
+
+
+# ---------------------------------------------------------------------------
+def dart_ssd_chunk_scan(x, dt, A, Bm, Cm, chunk: int, init_state=None, *, y_ssd=None, dH=None,
+                        states=None, workspace=None):
+    """SSD chunked scan keeping the chunk memories.
+
+    x[B,L,H,P], Bm/Cm[B,L,N] (float32 or bfloat16), dt[B,L,H] and A[H] float32,
+    init_state optional float32 [B,H,N,P].  Returns (y_ssd float32 [B,L,H,P],
+    dH [B,H,C,N,P] in x's dtype, states float32 [B,H,C,N,P]).  Optional
+    preallocated outputs/workspace avoid allocation in timed loops."""
+    lib = load()
+    host = not x.is_cuda
+    dev = _device_of(x, dt, A, Bm, Cm)
+    x, Bm, Cm = (_dev(v, dev, x.dtype) for v in (x, Bm, Cm))
+    dt, A = _dev(dt, dev, torch.float32), _dev(A, dev, torch.float32)
+    init_state = _dev(init_state, dev, torch.float32)
+    Bsz, L, H, P = x.shape
+    N = Bm.shape[-1]
+    _shape("dt", dt, (Bsz, L, H)); _shape("A", A, (H,)); _shape("Bm", Bm, (Bsz, L, N))
+    _shape("Cm", Cm, (Bsz, L, N))
+    if init_state is not None:
+        _shape("init_state", init_state, (Bsz, H, N, P))
+    if L % chunk:
+        raise ValueError(f"seqlen {L} is not a multiple of chunk {chunk}")
+    C = L // chunk
+    dims = Dims(Bsz, L, H, P, N, chunk, 1)
+    code = _dtype_code(x.dtype)
+    if y_ssd is None:
+        y_ssd = torch.empty((Bsz, L, H, P), device=dev, dtype=torch.float32)
+    if dH is None:
+        dH = torch.empty((Bsz, H, C, N, P), device=dev, dtype=x.dtype)
+    if states is None:
+        states = torch.empty((Bsz, H, C, N, P), device=dev, dtype=torch.float32)
+    wsb = lib.dart_ssd_chunk_scan_workspace_bytes(ctypes.byref(dims), code)
+    if workspace is None:
+        workspace = torch.empty(max(16, wsb), device=dev, dtype=torch.uint8)
+    with torch.cuda.device(dev):
+        _check(lib.dart_ssd_chunk_scan(ctypes.byref(dims), code, _ptr(x), _ptr(dt), _ptr(A), _ptr(Bm),
+                                       _ptr(Cm), _ptr(init_state), _ptr(y_ssd), _ptr(dH), _ptr(states),
+                                       _ptr(workspace), workspace.numel(), _stream()))
+    if host:
+        return y_ssd.cpu(), dH.cpu(), states.cpu()
+    return y_ssd, dH, states
+
+
+def dart_sma_forward(Q, E, Cm, dH, chunk: int, g: float, y_ssd=None, *, out=None):
+    """State-memory attention plus gated residual: returns float32 [B,L,H,P]
+    equal to y_ssd + g*o (or o when y_ssd is None)."""
+    lib = load()
+    host = not Q.is_cuda
+    dev = _device_of(Q, E, Cm, dH)
+    Q, E, Cm, dH = (_dev(v, dev, Q.dtype) for v in (Q, E, Cm, dH))
+    y_ssd = _dev(y_ssd, dev, torch.float32)
+    Bsz, L, H, N = Q.shape
+    P = E.shape[-1]
+    if L % chunk:
+        raise ValueError(f"seqlen {L} is not a multiple of chunk {chunk}")
+    C = L // chunk
+    _shape("E", E, (Bsz, L, H, P)); _shape("Cm", Cm, (Bsz, L, N)); _shape("dH", dH, (Bsz, H, C, N, P))
+    if y_ssd is not None:
+        _shape("y_ssd", y_ssd, (Bsz, L, H, P))
+    if out is None:
+        out = torch.empty((Bsz, L, H, P), device=dev, dtype=torch.float32)
+    dims = Dims(Bsz, L, H, P, N, chunk, 1)
+    with torch.cuda.device(dev):
+        _check(lib.dart_sma_forward(ctypes.byref(dims), _dtype_code(Q.dtype), _ptr(Q), _ptr(E), _ptr(Cm),
+                                    _ptr(dH), float(g), _ptr(y_ssd), _ptr(out), _stream()))
+    return out.cpu() if host else out
+
+
+def layer_forward(x, dt, A, Bm, Cm, Q, E, chunk: int, g: float, init_state=None, *,
+                  outputs=("y", "dH", "states"), buffers: Optional[dict] = None):
+    """The DART layer forward: scan, then SMA with the gated residual written
+    in place over y_ssd.  Returns a dict with the requested `outputs` among
+    y, dH, states.  With host (CPU) inputs the inputs are copied to the
+    current device and only the requested outputs are copied back.
+    `buffers` may hold preallocated device tensors y, dH, states, workspace."""
+    host = not x.is_cuda
+    dev = _device_of(x)
+    args = [_dev(v, dev) for v in (x, dt, A, Bm, Cm, Q, E)]
+    init_state = _dev(init_state, dev)
+    b = buffers or {}
+    y, dH, states = dart_ssd_chunk_scan(*args[:5], chunk, init_state, y_ssd=b.get("y"), dH=b.get("dH"),
+                                        states=b.get("states"), workspace=b.get("workspace"))
+    dart_sma_forward(args[5], args[6], args[4], dH, chunk, g, y, out=y)
+    res = {"y": y, "dH": dH, "states": states}
+    if host:
+        return {k: res[k].cpu() for k in outputs}
+    return {k: res[k] for k in outputs}
+
+
+def dart_decode_step(x, dt, A, Bm, Cm, Q, E, g: float, state, dH_cur, cache, nchunks, pos,
+                     chunk: int, *, y=None, workspace=None):
+    """One decode step for every sequence.  x[Bs,H,P], Bm/Cm[Bs,N],
+    Q[Bs,H,N], E[Bs,H,P] (cache dtype), dt[Bs,H], A[H] float32; state and
+    dH_cur float32 [Bs,H,N,P], cache [Bs,H,cmax,N,P], nchunks/pos int32 [Bs]
+    are device tensors updated in place.  Returns y float32 [Bs,H,P]."""
+    lib = load()
+    for name, t in (("state", state), ("dH_cur", dH_cur), ("cache", cache), ("nchunks", nchunks),
+                    ("pos", pos)):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor (updated in place)")
+    dev = cache.device
+    host = not x.is_cuda
+    x, Bm, Cm, Q, E = (_dev(v, dev, cache.dtype) for v in (x, Bm, Cm, Q, E))
+    dt, A = _dev(dt, dev, torch.float32), _dev(A, dev, torch.float32)
+    Bs, H, P = x.shape
+    N = Bm.shape[-1]
+    cmax = cache.shape[2]
+    _shape("state", state, (Bs, H, N, P)); _shape("dH_cur", dH_cur, (Bs, H, N, P))
+    _shape("cache", cache, (Bs, H, cmax, N, P)); _shape("Q", Q, (Bs, H, N)); _shape("E", E, (Bs, H, P))
+    _shape("dt", dt, (Bs, H)); _shape("Cm", Cm, (Bs, N))
+    if state.dtype != torch.float32 or dH_cur.dtype != torch.float32:
+        raise TypeError("state and dH_cur must be float32")
+    if nchunks.dtype != torch.int32 or pos.dtype != torch.int32:
+        raise TypeError("nchunks and pos must be int32")
+    dims = Dims(Bs, 0, H, P, N, chunk, 1)
+    code = _dtype_code(cache.dtype)
+    if y is None:
+        y = torch.empty((Bs, H, P), device=dev, dtype=torch.float32)
+    wsb = lib.dart_decode_step_workspace_bytes(ctypes.byref(dims), code, cmax)
+    if workspace is None:
+        workspace = torch.empty(max(16, wsb), device=dev, dtype=torch.uint8)
+    with torch.cuda.device(dev):
+        _check(lib.dart_decode_step(ctypes.byref(dims), code, _ptr(x), _ptr(dt), _ptr(A), _ptr(Bm), _ptr(Cm),
+                                    _ptr(Q), _ptr(E), float(g), _ptr(state), _ptr(dH_cur), _ptr(cache),
+                                    cmax, _ptr(nchunks), _ptr(pos), _ptr(y), _ptr(workspace),
+                                    workspace.numel(), _stream()))
+    return y.cpu() if host else y
+
+
+def decode_workspace_bytes(nseq, nheads, headdim, dstate, chunk, cmax, dtype) -> int:
+    dims = Dims(nseq, 0, nheads, headdim, dstate, chunk, 1)
+    return load().dart_decode_step_workspace_bytes(ctypes.byref(dims), _dtype_code(dtype), cmax)
+
+
+def scan_workspace_bytes(batch, seqlen, nheads, headdim, dstate, chunk, dtype) -> int:
+    dims = Dims(batch, seqlen, nheads, headdim, dstate, chunk, 1)
+    return load().dart_ssd_chunk_scan_workspace_bytes(ctypes.byref(dims), _dtype_code(dtype))
+
+
+def dart_sync_status(stream: Optional[torch.cuda.Stream] = None):
+    """Synchronise the stream and raise DartError if a kernel latched an error."""
+    s = stream or torch.cuda.current_stream()
+    _check(load().dart_sync_status(ctypes.c_void_p(s.cuda_stream)))

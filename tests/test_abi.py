@@ -1,0 +1,127 @@
+"""The C-ABI library builds, loads and exports every symbol include/dart.h
+declares; host-side validation rejects bad arguments before touching the GPU.
+CPU only: no call here reaches a kernel launch."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from mamba_ssd_state_b200 import build, dart
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dart.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return dart.load()
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(dart_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for want in ("dart_ssd_chunk_scan", "dart_sma_forward", "dart_decode_step", "dart_sync_status"):
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared():
+        assert hasattr(lib, name), f"{name} declared in dart.h but not exported"
+    assert set(dart.EXPORTS) <= set(_declared())
+
+
+def test_abi_version(lib):
+    assert lib.dart_abi_version() == 1
+
+
+def test_supported_set(lib):
+    assert dart.supported(128, 64, 256, torch.bfloat16)
+    assert dart.supported(16, 16, 64, torch.float32)
+    assert not dart.supported(96, 64, 256, torch.bfloat16)
+    assert not dart.supported(128, 64, 100, torch.bfloat16)
+
+
+FAKE = ctypes.c_void_p(0x10000)       # 16-byte aligned, never dereferenced on the host
+MISALIGNED = ctypes.c_void_p(0x10004)
+
+
+def _scan(lib, dims, dtype=dart.DART_BF16, x=FAKE, ws_bytes=1 << 20):
+    return lib.dart_ssd_chunk_scan(ctypes.byref(dims), dtype, x, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE,
+                                   FAKE, FAKE, ws_bytes, None)
+
+
+def test_scan_rejects_ragged_seqlen(lib):
+    rc = _scan(lib, dart.Dims(1, 300, 2, 64, 128, 256, 1))
+    assert rc == dart.DART_ERR_UNSUPPORTED
+    assert b"multiple of chunk" in lib.dart_last_error()
+
+
+def test_scan_rejects_ngroups(lib):
+    assert _scan(lib, dart.Dims(1, 256, 2, 64, 128, 256, 2)) == dart.DART_ERR_UNSUPPORTED
+
+
+def test_scan_rejects_uncompiled_shape(lib):
+    assert _scan(lib, dart.Dims(1, 256, 2, 64, 96, 256, 1)) == dart.DART_ERR_UNSUPPORTED
+
+
+def test_scan_rejects_null_and_misaligned(lib):
+    d = dart.Dims(1, 256, 2, 64, 128, 256, 1)
+    assert _scan(lib, d, x=None) == dart.DART_ERR_INVALID_ARG
+    assert b"null" in lib.dart_last_error()
+    assert _scan(lib, d, x=MISALIGNED) == dart.DART_ERR_INVALID_ARG
+    assert b"aligned" in lib.dart_last_error()
+
+
+def test_scan_rejects_small_workspace(lib):
+    d = dart.Dims(2, 512, 4, 64, 128, 256, 1)
+    need = lib.dart_ssd_chunk_scan_workspace_bytes(ctypes.byref(d), dart.DART_BF16)
+    assert need == 4 * 2 * 4 * 2
+    assert _scan(lib, d, ws_bytes=need - 1) == dart.DART_ERR_INVALID_ARG
+
+
+def test_scan_rejects_bad_dtype_and_dims(lib):
+    assert _scan(lib, dart.Dims(1, 256, 2, 64, 128, 256, 1), dtype=7) == dart.DART_ERR_INVALID_ARG
+    assert _scan(lib, dart.Dims(0, 256, 2, 64, 128, 256, 1)) == dart.DART_ERR_INVALID_ARG
+    assert lib.dart_ssd_chunk_scan(None, 1, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE,
+                                   16, None) == dart.DART_ERR_INVALID_ARG
+
+
+def test_sma_rejects_bad_args(lib):
+    d = dart.Dims(1, 512, 2, 64, 128, 256, 1)
+    rc = lib.dart_sma_forward(ctypes.byref(d), dart.DART_BF16, FAKE, None, FAKE, FAKE, 0.5, None, FAKE, None)
+    assert rc == dart.DART_ERR_INVALID_ARG
+    d.seqlen = 500
+    rc = lib.dart_sma_forward(ctypes.byref(d), dart.DART_BF16, FAKE, FAKE, FAKE, FAKE, 0.5, None, FAKE, None)
+    assert rc == dart.DART_ERR_UNSUPPORTED
+
+
+def test_decode_rejects_bad_args(lib):
+    d = dart.Dims(4, 0, 2, 64, 128, 256, 1)
+    ws = lib.dart_decode_step_workspace_bytes(ctypes.byref(d), dart.DART_BF16, 9)
+    assert ws > 0
+
+    def call(cmax=9, state=FAKE, ws_bytes=ws):
+        return lib.dart_decode_step(ctypes.byref(d), dart.DART_BF16, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                    0.5, state, FAKE, FAKE, cmax, FAKE, FAKE, FAKE, FAKE, ws_bytes, None)
+
+    assert call(cmax=0) == dart.DART_ERR_INVALID_ARG
+    assert call(state=None) == dart.DART_ERR_INVALID_ARG
+    assert call(ws_bytes=ws - 4) == dart.DART_ERR_INVALID_ARG
+
+
+def test_binding_fails_loudly_without_cuda(lib):
+    if torch.cuda.is_available():
+        pytest.skip("a CUDA device is present")
+    x = torch.zeros(1, 256, 1, 64, dtype=torch.bfloat16)
+    with pytest.raises(RuntimeError):
+        dart.dart_ssd_chunk_scan(x, torch.zeros(1, 256, 1), torch.zeros(1),
+                                 torch.zeros(1, 256, 128, dtype=torch.bfloat16),
+                                 torch.zeros(1, 256, 128, dtype=torch.bfloat16), 256)

@@ -1,0 +1,159 @@
+"""GPU parity of the decode step against the oracle, prefill/decode
+consistency on the GPU, and the device-side error path."""
+import numpy as np
+import pytest
+import torch
+
+from mamba_ssd_state_b200 import build, dart, synth
+from mamba_ssd_state_b200.synth import DecodeShape, LayerShape
+from oracle import dart_oracle
+from tests.parity import TOL, assert_close, oracle_inputs, to_device
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def orc():
+    return dart_oracle.get()
+
+
+@pytest.fixture(scope="module", autouse=True)
+def lib():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    build.build()
+    return dart.load()
+
+
+def _oracle_state(init):
+    return {"cache": init["cache"].double().numpy().copy(), "state": init["state"].double().numpy().copy(),
+            "dH_cur": init["dH_cur"].double().numpy().copy(), "nchunks": init["nchunks"].numpy().copy(),
+            "pos": init["pos"].numpy().copy()}
+
+
+def _run_decode(orc, shape, init, steps, seqs_for_oracle, seed=0, check_every=1):
+    """Run `steps` decode steps on the GPU for every sequence and in the
+    oracle for `seqs_for_oracle`; compare y each checked step and the final
+    state, running contribution, cache and counters."""
+    tol = TOL[synth.torch_dtype(shape.dtype)]
+    A = synth.decode_A(shape, seed)
+    g = shape.g
+    dev = {k: v.cuda() for k, v in init.items()}
+    sub = {k: v[seqs_for_oracle] for k, v in init.items()}
+    ref = _oracle_state(sub)
+    worst = 0.0
+    for step in range(steps):
+        tok = synth.decode_tokens(shape, step, seed)
+        y = dart.dart_decode_step(tok["x"].cuda(), tok["dt"].cuda(), A.cuda(), tok["Bm"].cuda(), tok["Cm"].cuda(),
+                                  tok["Q"].cuda(), tok["E"].cuda(), g, dev["state"], dev["dH_cur"],
+                                  dev["cache"], dev["nchunks"], dev["pos"], shape.chunk)
+        t = oracle_inputs({k: v[seqs_for_oracle] for k, v in tok.items()})
+        yr = orc.decode_step(t["x"], t["dt"], A.numpy(), t["Bm"], t["Cm"], t["Q"], t["E"], g, ref["state"],
+                             ref["dH_cur"], ref["cache"], ref["nchunks"], ref["pos"], shape.chunk)
+        if step % check_every == 0 or step == steps - 1:
+            worst = max(worst, assert_close(f"y step {step}", y[seqs_for_oracle], yr, tol))
+    dart.dart_sync_status()
+    assert np.array_equal(dev["nchunks"].cpu().numpy()[seqs_for_oracle], ref["nchunks"])
+    assert np.array_equal(dev["pos"].cpu().numpy()[seqs_for_oracle], ref["pos"])
+    assert_close("state", dev["state"][seqs_for_oracle], ref["state"], tol)
+    assert_close("dH_cur", dev["dH_cur"][seqs_for_oracle], ref["dH_cur"], tol)
+    got_cache = dev["cache"][seqs_for_oracle]
+    for i in range(len(seqs_for_oracle)):
+        n = int(ref["nchunks"][i])
+        assert_close(f"cache of sequence {seqs_for_oracle[i]}", got_cache[i, :, :n], ref["cache"][i, :, :n], tol)
+    return dev, ref, worst
+
+
+def _small_init(shape, nchunks, pos, seed):
+    init = synth.decode_initial(shape, seed)
+    init["nchunks"] = torch.tensor(nchunks, dtype=torch.int32)
+    init["pos"] = torch.tensor(pos, dtype=torch.int32)
+    # a non-zero running contribution for sequences that start mid-chunk
+    r = np.random.default_rng(seed)
+    for b, p in enumerate(pos):
+        if p > 0:
+            init["dH_cur"][b] = torch.from_numpy(r.standard_normal(init["dH_cur"][b].shape).astype(np.float32) * 0.05)
+    # slots past nchunks hold garbage that must never be read
+    for b, n in enumerate(nchunks):
+        init["cache"][b, :, n:] = 1e4
+    return init
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_decode_small_with_appends(orc, dtype):
+    """Three sequences at different counters, chunk size 4: appends happen at
+    different steps, one sequence starts with an empty cache."""
+    shape = DecodeShape(3, 2, 64, 128, 4, 7, 7, 9, dtype)
+    init = _small_init(shape, [2, 0, 3], [0, 2, 3], seed=1)
+    _run_decode(orc, shape, init, shape.nsteps, [0, 1, 2])
+
+
+def test_decode_tiny_fp32_dims(orc):
+    shape = DecodeShape(2, 2, 16, 16, 8, 5, 5, 12, "f32")
+    init = _small_init(shape, [1, 3], [5, 0], seed=2)
+    _run_decode(orc, shape, init, shape.nsteps, [0, 1])
+
+
+def test_decode_config_sampled(orc):
+    """64 sequences with 128 cached memories each (context 32768 at S=256),
+    256 steps with the append on the last one; the oracle follows sequences 0
+    and 63."""
+    shape = synth.DECODE_64x32K
+    init = synth.decode_initial(shape, seed=0)
+    dev, ref, _ = _run_decode(orc, shape, init, shape.nsteps, [0, 63], check_every=15)
+    assert np.all(ref["nchunks"] == 129) and np.all(ref["pos"] == 0)
+    assert int(dev["nchunks"].min()) == 129
+
+
+def test_prefill_then_decode_matches_longer_prefill():
+    """forward(L + S) on the GPU equals forward(L) followed by S decode steps
+    fed from its dH and final boundary state, including the append."""
+    S = 256
+    shape = LayerShape(2, 4 * S, 3, 64, 128, S, "bf16", "loguniform")
+    inp = synth.layer_inputs(shape, seed=20)
+    d = to_device(inp)
+    L = 3 * S
+    full = dart.layer_forward(d["x"], d["dt"], d["A"], d["Bm"], d["Cm"], d["Q"], d["E"], S, d["g"])
+    pre = dart.layer_forward(*(d[k][:, :L] if k != "A" else d[k] for k in ("x", "dt", "A", "Bm", "Cm", "Q", "E")),
+                             S, d["g"])
+    B, H, N, P = 2, 3, 128, 64
+    cmax = 5
+    cache = torch.zeros(B, H, cmax, N, P, dtype=torch.bfloat16, device="cuda")
+    cache[:, :, :3] = pre["dH"]
+    state = pre["states"][:, :, -1].contiguous()
+    dcur = torch.zeros_like(state)
+    nch = torch.full((B,), 3, dtype=torch.int32, device="cuda")
+    pos = torch.zeros(B, dtype=torch.int32, device="cuda")
+    ys = []
+    for t in range(L, L + S):
+        ys.append(dart.dart_decode_step(d["x"][:, t], d["dt"][:, t], d["A"], d["Bm"][:, t], d["Cm"][:, t],
+                                        d["Q"][:, t], d["E"][:, t], d["g"], state, dcur, cache, nch, pos, S))
+    dart.dart_sync_status()
+    y_dec = torch.stack(ys, 1)
+    assert_close("decode vs prefill y", y_dec, full["y"][:, L:].cpu().numpy(), 2e-2)
+    assert torch.all(nch == 4) and torch.all(pos == 0)
+    assert_close("appended memory", cache[:, :, 3].float(), full["dH"][:, :, 3].float().cpu().numpy(), 2e-2)
+    assert_close("state", state, full["states"][:, :, -1].cpu().numpy(), 2e-2)
+
+
+def test_decode_bad_counters_are_flagged():
+    """A sequence with pos outside [0, S) or a full cache is skipped and the
+    device status reports DART_ERR_DEVICE; the other sequences advance."""
+    shape = DecodeShape(3, 2, 64, 128, 4, 2, 3, 1, "bf16")
+    init = synth.decode_initial(shape, seed=3)
+    init["pos"] = torch.tensor([0, 7, 3], dtype=torch.int32)      # seq 1: pos out of range
+    init["nchunks"] = torch.tensor([2, 2, 3], dtype=torch.int32)  # seq 2: append into a full cache
+    dev = {k: v.cuda() for k, v in init.items()}
+    st0 = dev["state"].clone()
+    tok = synth.decode_tokens(shape, 0, 3)
+    A = synth.decode_A(shape, 3)
+    dart.dart_decode_step(tok["x"].cuda(), tok["dt"].cuda(), A.cuda(), tok["Bm"].cuda(), tok["Cm"].cuda(),
+                          tok["Q"].cuda(), tok["E"].cuda(), 0.5, dev["state"], dev["dH_cur"], dev["cache"],
+                          dev["nchunks"], dev["pos"], shape.chunk)
+    with pytest.raises(dart.DartError) as ei:
+        dart.dart_sync_status()
+    assert ei.value.status == dart.DART_ERR_DEVICE
+    assert torch.equal(dev["state"][1:], st0[1:])
+    assert not torch.equal(dev["state"][0], st0[0])
+    assert dev["pos"].tolist() == [1, 7, 3] and dev["nchunks"].tolist() == [2, 2, 3]
+    dart.dart_sync_status()  # the status word was cleared by the read
