@@ -142,7 +142,8 @@ dart_status dart_sma_forward(const dart_dims* d, dart_dtype dtype, const void* Q
     DART_REQUIRE_PTR(Q); DART_REQUIRE_PTR(E); DART_REQUIRE_PTR(Cm); DART_REQUIRE_PTR(dH);
     DART_OPTIONAL_PTR(y_ssd); DART_REQUIRE_PTR(out);
     dart::SmaArgs a{d->batch, d->seqlen, d->nheads, d->headdim, d->dstate, d->chunk,
-                    Q, E, Cm, dH, g, y_ssd, out};
+                    Q, E, Cm, dH, g, y_ssd, out, status_word()};
+    if (!a.status) return fail(DART_ERR_CUDA, "dart_sma_forward: no device status word");
     cudaError_t e = dart::launch_sma(a, dtype, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "dart_sma_forward launch");
     return DART_OK;

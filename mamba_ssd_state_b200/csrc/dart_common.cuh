@@ -109,6 +109,7 @@ struct SmaArgs {
     int B, L, H, P, N, S;
     const void* Q; const void* E; const void* Cm; const void* dH;
     float g; const float* y_ssd; float* out;
+    int* status;  // device status word
 };
 struct DecodeArgs {
     int B, H, P, N, S, cmax, nsplit;
@@ -127,6 +128,8 @@ cudaError_t launch_sma(const SmaArgs& a, dart_dtype dt, cudaStream_t st);
 cudaError_t launch_decode(const DecodeArgs& a, dart_dtype dt, cudaStream_t st);
 bool ssd_scan_supported(int N, int P, int S, dart_dtype dt);
 bool sma_supported(int N, int P, int S, dart_dtype dt);
+bool sma_tc_applicable(int N, int P, int S, dart_dtype dt);
+cudaError_t launch_sma_tc(const SmaArgs& a, cudaStream_t st);
 const char* sma_impl_name(int N, int P, int S, dart_dtype dt);
 bool decode_supported(int N, int P, int S, dart_dtype dt);
 int decode_num_splits(int B, int H, int cmax);

@@ -119,9 +119,12 @@ bool sma_supported(int N, int P, int S, dart_dtype) {
     return np && (S == 64 || S == 128 || S == 256);
 }
 
-const char* sma_impl_name(int, int, int, dart_dtype) { return "sma_simt"; }
+const char* sma_impl_name(int N, int P, int S, dart_dtype dt) {
+    return sma_tc_applicable(N, P, S, dt) ? "sma_tcgen05" : "sma_simt";
+}
 
 cudaError_t launch_sma(const SmaArgs& a, dart_dtype dt, cudaStream_t st) {
+    if (sma_tc_applicable(a.N, a.P, a.S, dt)) return launch_sma_tc(a, st);
 #define DART_SMA_CASE(NN, PP)                                                       \
     if (a.N == NN && a.P == PP)                                                     \
         return dt == DART_F32 ? run<float, NN, PP>(a, st) : run<__nv_bfloat16, NN, PP>(a, st);

@@ -1,0 +1,369 @@
+// sma_tc.cu -- state-memory attention on the 5th-generation tensor cores.
+//
+// What it computes (Pith review of DART, "Core claim" / "What carries the
+// argument"; SMA Eqs. (5)-(10)): for token t in chunk k(t) and each earlier
+// chunk memory c < k(t),
+//   U_{t,c} = Q_t^T dH[c]  (P),   V_{t,c} = C_t^T dH[c]  (P),
+//   s_{t,c} = U_{t,c} . E_t / sqrt(N)   (= Q_t . (dH[c] E_t) / sqrt(N)),
+//   o_t = sum_c softmax_c(s) V_{t,c},   out = y_ssd + g o_t.
+//
+// Why this shape: the only dense contractions are [Q_T; C_T] x dH[c]; the
+// "PV" step is per token and per chunk (every token decodes its own value),
+// so it is element-wise work on CUDA cores, not a second GEMM.  One CTA owns
+// a tile of 128 query tokens of one (b, h), all inside chunk k:
+//   A operands  Q_T, C_T   128 x 128 bf16, K-major, loaded once per tile;
+//   B operand   4 chunk memories side by side, 128 (K = N) x 256 (4 x P),
+//               MN-major exactly as stored in HBM, streamed by TMA;
+//   D           U (TMEM columns 0..255) and V (columns 256..511), fp32.
+// Each batch of 4 memories costs two M=128, N=256, K=128 MMAs.  The epilogue
+// warps read U as soon as it lands (scores, online softmax) and hand the U
+// columns back while the V MMA runs, then read V (value accumulation) while
+// the next batch's U MMA runs, so the tensor pipe never waits for them.
+//
+// Roles (192 threads): warp 0 issues TMA, warp 1 allocates TMEM and issues
+// tcgen05.mma, warps 2-5 (one per TMEM lane quadrant) run the softmax and
+// write the output.  The grid is persistent: CTA i takes tiles i, i+G, ...
+// of a list ordered from the most memories to the fewest, so the triangular
+// work spreads evenly.
+#include <cuda_bf16.h>
+#include <string.h>
+
+#include "dart_common.cuh"
+#include "sm100.cuh"
+#include "tensor_map.h"
+
+namespace dart {
+namespace {
+
+using namespace sm100;
+
+constexpr int kN = 128, kP = 64;   // compiled shape
+constexpr int kBQ = 128;           // query tokens per tile (MMA M)
+constexpr int kCB = 4;             // chunk memories per MMA (N = 4 * P = 256)
+constexpr int kNB = 2;             // stages of the memory ring
+constexpr uint32_t kHalfA = 128 * 64 * 2;        // 128 rows x 64 bf16 (one swizzle panel)
+constexpr uint32_t kMemBytes = kN * kP * 2;       // one chunk memory, 16 KB
+constexpr uint32_t kOffQ = 0;
+constexpr uint32_t kOffC = 2 * kHalfA;
+constexpr uint32_t kOffB = 4 * kHalfA;
+constexpr uint32_t kStageBytes = kCB * kMemBytes;
+constexpr uint32_t kOffBar = kOffB + kNB * kStageBytes;
+constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;  // + barriers, + alignment slack
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColV = 256;
+
+enum Bar { Q_FULL = 0, Q_FREE, C_FULL, C_FREE, U_FULL, U_EMPTY, V_FULL, V_EMPTY, B_FULL0, B_EMPTY0 = B_FULL0 + kNB,
+           NUM_BARS = B_EMPTY0 + kNB };
+
+struct SmaTcParams {
+    CUtensorMap tmap_q;  // Q viewed as dims (N, B*L, H)
+    CUtensorMap tmap_c;  // Cm viewed as dims (N, B*L)
+    CUtensorMap tmap_h;  // dH viewed as dims (P, B*H*C*N)
+    const __nv_bfloat16* E;
+    const float* y_ssd;
+    float* out;
+    float g;
+    int B, L, H, S, C;
+    int tiles_per_chunk, total_tiles;
+    int* status;
+};
+
+struct Tile {
+    int b, h, k, t0;
+};
+
+// Tile list ordered by decreasing chunk index (most memories first).
+__device__ __forceinline__ Tile decode_tile(const SmaTcParams& p, int i) {
+    const int per_k = p.B * p.H * p.tiles_per_chunk;
+    Tile t;
+    t.k = p.C - 1 - i / per_k;
+    const int r = i % per_k;
+    const int sub = r % p.tiles_per_chunk;
+    const int bh = r / p.tiles_per_chunk;
+    t.b = bh / p.H;
+    t.h = bh % p.H;
+    t.t0 = t.k * p.S + sub * kBQ;
+    return t;
+}
+
+__device__ __forceinline__ void load_row_bf16(const __nv_bfloat16* src, float* dst) {
+#pragma unroll
+    for (int i = 0; i < kP / 8; ++i) {
+        float tmp[8];
+        Vec16<__nv_bfloat16>::load(src + 8 * i, tmp);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) dst[8 * i + j] = tmp[j];
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 1) sma_tc_kernel(const __grid_constant__ SmaTcParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + kOffBar + NUM_BARS * 8);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+    auto bar = [&](int i) -> uint32_t { return sbase + kOffBar + 8u * (uint32_t)i; };
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar(Q_FULL), 1);
+        mbar_init(bar(Q_FREE), 1);
+        mbar_init(bar(C_FULL), 1);
+        mbar_init(bar(C_FREE), 1);
+        mbar_init(bar(U_FULL), 1);
+        mbar_init(bar(U_EMPTY), 4);
+        mbar_init(bar(V_FULL), 1);
+        mbar_init(bar(V_EMPTY), 4);
+        for (int s = 0; s < kNB; ++s) {
+            mbar_init(bar(B_FULL0 + s), 1);
+            mbar_init(bar(B_EMPTY0 + s), 1);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&p.tmap_q);
+        tma_prefetch_desc(&p.tmap_c);
+        tma_prefetch_desc(&p.tmap_h);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_holder), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA
+        if (lane == 0) {
+            uint32_t q_ph = 0, c_ph = 0;
+            int it_b = 0;
+            for (int i = blockIdx.x; i < p.total_tiles; i += gridDim.x) {
+                const Tile t = decode_tile(p, i);
+                if (t.k == 0) continue;
+                const int row = t.b * p.L + t.t0;
+                if (!mbar_wait(bar(Q_FREE), q_ph ^ 1, abort_flag, p.status)) break;
+                mbar_expect_tx(bar(Q_FULL), 2 * kHalfA);
+                tma_load_3d(sbase + kOffQ, &p.tmap_q, bar(Q_FULL), 0, row, t.h);
+                tma_load_3d(sbase + kOffQ + kHalfA, &p.tmap_q, bar(Q_FULL), 64, row, t.h);
+                q_ph ^= 1;
+                if (!mbar_wait(bar(C_FREE), c_ph ^ 1, abort_flag, p.status)) break;
+                mbar_expect_tx(bar(C_FULL), 2 * kHalfA);
+                tma_load_2d(sbase + kOffC, &p.tmap_c, bar(C_FULL), 0, row);
+                tma_load_2d(sbase + kOffC + kHalfA, &p.tmap_c, bar(C_FULL), 64, row);
+                c_ph ^= 1;
+                const int nbatch = (t.k + kCB - 1) / kCB;
+                bool ok = true;
+                for (int j = 0; j < nbatch && ok; ++j, ++it_b) {
+                    const int nv = min(kCB, t.k - kCB * j);
+                    const int s = it_b % kNB;
+                    const uint32_t ph = (uint32_t)(it_b / kNB) & 1u;
+                    if (!mbar_wait(bar(B_EMPTY0 + s), ph ^ 1, abort_flag, p.status)) { ok = false; break; }
+                    mbar_expect_tx(bar(B_FULL0 + s), (uint32_t)nv * kMemBytes);
+                    const int mem_row = ((t.b * p.H + t.h) * p.C + kCB * j) * kN;
+                    for (int q = 0; q < nv; ++q)
+                        tma_load_2d(sbase + kOffB + (uint32_t)s * kStageBytes + (uint32_t)q * kMemBytes, &p.tmap_h,
+                                    bar(B_FULL0 + s), 0, mem_row + q * kN);
+                }
+                if (!ok) break;
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA
+        if (lane == 0) {
+            uint32_t q_ph = 0, c_ph = 0;
+            int it_b = 0, it_u = 0;
+            bool ok = true;
+            for (int i = blockIdx.x; i < p.total_tiles && ok; i += gridDim.x) {
+                const Tile t = decode_tile(p, i);
+                if (t.k == 0) continue;
+                if (!mbar_wait(bar(Q_FULL), q_ph, abort_flag, p.status)) break;
+                q_ph ^= 1;
+                tc_fence_after();
+                const int nbatch = (t.k + kCB - 1) / kCB;
+                for (int j = 0; j < nbatch; ++j, ++it_b, ++it_u) {
+                    const int nv = min(kCB, t.k - kCB * j);
+                    const int s = it_b % kNB;
+                    const uint32_t ph = (uint32_t)(it_b / kNB) & 1u;
+                    const uint32_t idesc = idesc_bf16_f32(kBQ, kP * nv, false, true);
+                    const uint32_t b_base = sbase + kOffB + (uint32_t)s * kStageBytes;
+                    if (!mbar_wait(bar(B_FULL0 + s), ph, abort_flag, p.status)) { ok = false; break; }
+                    if (!mbar_wait(bar(U_EMPTY), ((uint32_t)it_u & 1u) ^ 1u, abort_flag, p.status)) { ok = false; break; }
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < kN / 16; ++kk) {
+                        const uint64_t ad = smem_desc_sw128(sbase + kOffQ + (uint32_t)(kk >> 2) * kHalfA + (uint32_t)(kk & 3) * 32, 16, 1024);
+                        const uint64_t bd = smem_desc_sw128(b_base + (uint32_t)kk * 2048, kMemBytes, 1024);
+                        mma_f16_ss(tmem, ad, bd, idesc, kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(bar(U_FULL));
+                    if (j == nbatch - 1) mma_commit(bar(Q_FREE));
+                    if (j == 0) {
+                        if (!mbar_wait(bar(C_FULL), c_ph, abort_flag, p.status)) { ok = false; break; }
+                        c_ph ^= 1;
+                    }
+                    if (!mbar_wait(bar(V_EMPTY), ((uint32_t)it_u & 1u) ^ 1u, abort_flag, p.status)) { ok = false; break; }
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < kN / 16; ++kk) {
+                        const uint64_t ad = smem_desc_sw128(sbase + kOffC + (uint32_t)(kk >> 2) * kHalfA + (uint32_t)(kk & 3) * 32, 16, 1024);
+                        const uint64_t bd = smem_desc_sw128(b_base + (uint32_t)kk * 2048, kMemBytes, 1024);
+                        mma_f16_ss(tmem + kColV, ad, bd, idesc, kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(bar(V_FULL));
+                    mma_commit(bar(B_EMPTY0 + s));
+                    if (j == nbatch - 1) mma_commit(bar(C_FREE));
+                }
+            }
+        }
+    } else {
+        // ------------------------------------------------------- epilogue
+        const int quad = warp & 3;                 // TMEM lane quadrant of this warp
+        const int row = quad * 32 + lane;          // token row inside the tile
+        const uint32_t t_lane = tmem + ((uint32_t)(quad * 32) << 16);
+        const float sscale = kLog2e * rsqrtf((float)kN);
+        int it_u = 0;
+        for (int i = blockIdx.x; i < p.total_tiles; i += gridDim.x) {
+            const Tile t = decode_tile(p, i);
+            const size_t tok = (size_t)t.b * p.L + t.t0 + row;
+            float* orow = p.out + (tok * p.H + t.h) * kP;
+            const float* yrow = p.y_ssd ? p.y_ssd + (tok * p.H + t.h) * kP : nullptr;
+            float o[kP];
+#pragma unroll
+            for (int j = 0; j < kP; ++j) o[j] = 0.f;
+            float l = 0.f;
+            bool ok = true;
+            if (t.k > 0) {
+                float e[kP];
+                load_row_bf16(p.E + (tok * p.H + t.h) * kP, e);
+                float m = -INFINITY;
+                const int nbatch = (t.k + kCB - 1) / kCB;
+                for (int j = 0; j < nbatch; ++j, ++it_u) {
+                    const int nv = min(kCB, t.k - kCB * j);
+                    const uint32_t ph = (uint32_t)it_u & 1u;
+                    if (!mbar_wait_warp(bar(U_FULL), ph, abort_flag, p.status)) { ok = false; break; }
+                    tc_fence_after();
+                    float sc[kCB];
+#pragma unroll
+                    for (int c = 0; c < kCB; ++c) {
+                        sc[c] = -INFINITY;
+                        if (c < nv) {
+                            float u[kP];
+                            tmem_ld_32x32b_x32(t_lane + (uint32_t)(c * kP), u);
+                            tmem_ld_32x32b_x32(t_lane + (uint32_t)(c * kP + 32), u + 32);
+                            tmem_ld_wait();
+                            float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+                            for (int q = 0; q < kP; q += 2) {
+                                acc0 = fmaf(u[q], e[q], acc0);
+                                acc1 = fmaf(u[q + 1], e[q + 1], acc1);
+                            }
+                            sc[c] = (acc0 + acc1) * sscale;
+                        }
+                    }
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar(U_EMPTY));
+                    float mnew = m;
+#pragma unroll
+                    for (int c = 0; c < kCB; ++c) mnew = fmaxf(mnew, sc[c]);
+                    const float alpha = exp2f(m - mnew);
+                    float w[kCB];
+#pragma unroll
+                    for (int c = 0; c < kCB; ++c) w[c] = c < nv ? exp2f(sc[c] - mnew) : 0.f;
+                    l = l * alpha + (w[0] + w[1]) + (w[2] + w[3]);
+                    m = mnew;
+#pragma unroll
+                    for (int q = 0; q < kP; ++q) o[q] *= alpha;
+                    if (!mbar_wait_warp(bar(V_FULL), ph, abort_flag, p.status)) { ok = false; break; }
+                    tc_fence_after();
+#pragma unroll
+                    for (int c = 0; c < kCB; ++c) {
+                        if (c < nv) {
+                            float v[kP];
+                            tmem_ld_32x32b_x32(t_lane + kColV + (uint32_t)(c * kP), v);
+                            tmem_ld_32x32b_x32(t_lane + kColV + (uint32_t)(c * kP + 32), v + 32);
+                            tmem_ld_wait();
+#pragma unroll
+                            for (int q = 0; q < kP; ++q) o[q] = fmaf(w[c], v[q], o[q]);
+                        }
+                    }
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar(V_EMPTY));
+                }
+            }
+            if (!ok) break;
+            const float inv = t.k > 0 ? 1.f / l : 0.f;
+#pragma unroll
+            for (int q = 0; q < kP; q += 4) {
+                float4 r = make_float4(o[q] * inv, o[q + 1] * inv, o[q + 2] * inv, o[q + 3] * inv);
+                if (yrow) {
+                    const float4 yv = *reinterpret_cast<const float4*>(yrow + q);
+                    r = make_float4(fmaf(p.g, r.x, yv.x), fmaf(p.g, r.y, yv.y), fmaf(p.g, r.z, yv.z),
+                                    fmaf(p.g, r.w, yv.w));
+                }
+                *reinterpret_cast<float4*>(orow + q) = r;
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+}  // namespace
+
+bool sma_tc_applicable(int N, int P, int S, dart_dtype dt) {
+    return dt == DART_BF16 && N == kN && P == kP && S % kBQ == 0;
+}
+
+cudaError_t launch_sma_tc(const SmaArgs& a, cudaStream_t st) {
+    SmaTcParams p;
+    memset(&p, 0, sizeof(p));
+    const int C = a.L / a.S;
+    {
+        const uint64_t dims[3] = {(uint64_t)kN, (uint64_t)a.B * a.L, (uint64_t)a.H};
+        const uint64_t strides[2] = {(uint64_t)a.H * kN * 2, (uint64_t)kN * 2};
+        const uint32_t box[3] = {64, kBQ, 1};
+        if (!encode_tile_map_bf16(&p.tmap_q, 3, a.Q, dims, strides, box)) return cudaErrorInvalidValue;
+    }
+    {
+        const uint64_t dims[2] = {(uint64_t)kN, (uint64_t)a.B * a.L};
+        const uint64_t strides[1] = {(uint64_t)kN * 2};
+        const uint32_t box[2] = {64, kBQ};
+        if (!encode_tile_map_bf16(&p.tmap_c, 2, a.Cm, dims, strides, box)) return cudaErrorInvalidValue;
+    }
+    {
+        const uint64_t dims[2] = {(uint64_t)kP, (uint64_t)a.B * a.H * C * kN};
+        const uint64_t strides[1] = {(uint64_t)kP * 2};
+        const uint32_t box[2] = {kP, kN};
+        if (!encode_tile_map_bf16(&p.tmap_h, 2, a.dH, dims, strides, box)) return cudaErrorInvalidValue;
+    }
+    p.E = static_cast<const __nv_bfloat16*>(a.E);
+    p.y_ssd = a.y_ssd;
+    p.out = a.out;
+    p.g = a.g;
+    p.B = a.B; p.L = a.L; p.H = a.H; p.S = a.S; p.C = C;
+    p.tiles_per_chunk = a.S / kBQ;
+    p.total_tiles = C * a.B * a.H * p.tiles_per_chunk;
+    p.status = a.status;
+    const int sms = sm_count();
+    if (sms <= 0) return cudaErrorInvalidDevice;
+    const int grid = p.total_tiles < sms ? p.total_tiles : sms;
+    cudaError_t e = cudaFuncSetAttribute(sma_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    sma_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    count_launches(1);
+    return cudaSuccess;
+}
+
+}  // namespace dart

@@ -80,6 +80,20 @@ def test_fp32_N64_P64_S64(orc):
     check_full(orc, shape, synth.layer_inputs(shape, seed=3), TOL[torch.float32])
 
 
+def test_bf16_N64_P64_cuda_core_path(orc):
+    """bf16 at a shape the tensor-core kernel does not cover (N=64) runs the
+    CUDA-core SMA kernel; same tolerance."""
+    assert dart.sma_impl(64, 64, 128, torch.bfloat16) == "sma_simt"
+    shape = LayerShape(2, 5 * 128, 2, 64, 64, 128, "bf16", "loguniform")
+    check_full(orc, shape, synth.layer_inputs(shape, seed=31), TOL[torch.bfloat16])
+
+
+def test_dispatch_uses_tensor_cores_for_the_layer_shape():
+    assert dart.sma_impl(128, 64, 256, torch.bfloat16) == "sma_tcgen05"
+    assert dart.sma_impl(128, 64, 128, torch.bfloat16) == "sma_tcgen05"
+    assert dart.sma_impl(128, 64, 256, torch.float32) == "sma_simt"
+
+
 def test_layer_L2k_config_full(orc):
     """B=4, L=2048, H=32, P=64, N=128, S=256 (the Mamba-2-370M layer shape)."""
     inp = synth.layer_inputs(synth.LAYER_L2K, seed=0)
