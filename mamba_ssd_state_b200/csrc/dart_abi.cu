@@ -50,6 +50,10 @@ dart_status cuda_fail(cudaError_t e, const char* where) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Workspace of the scan: per-chunk decay sums (float), padded to 256 bytes,
+// followed on the tensor-core path by the bf16 state entering each chunk.
+size_t scan_asum_bytes(size_t bhc) { return (bhc * sizeof(float) + 255) & ~size_t(255); }
+
 #define DART_REQUIRE_PTR(p)                                                           \
     do {                                                                              \
         if (!(p)) return fail(DART_ERR_INVALID_ARG, "%s: null pointer", #p);          \
@@ -101,10 +105,14 @@ const char* dart_sma_impl(int dstate, int headdim, int chunk, dart_dtype dtype) 
     return dart::sma_impl_name(dstate, headdim, chunk, dtype);
 }
 
-size_t dart_ssd_chunk_scan_workspace_bytes(const dart_dims* d, dart_dtype) {
+size_t dart_ssd_chunk_scan_workspace_bytes(const dart_dims* d, dart_dtype dtype) {
     if (!d || d->chunk < 1) return 0;
     const size_t C = (size_t)(d->seqlen / d->chunk);
-    return sizeof(float) * (size_t)d->batch * (size_t)d->nheads * C;
+    const size_t bhc = (size_t)d->batch * (size_t)d->nheads * C;
+    size_t bytes = scan_asum_bytes(bhc);
+    if (dart::ssd_scan_tc_applicable(d->dstate, d->headdim, d->chunk, dtype))
+        bytes += bhc * (size_t)d->dstate * (size_t)d->headdim * 2;  // bf16 state entering each chunk
+    return bytes;
 }
 
 dart_status dart_ssd_chunk_scan(const dart_dims* d, dart_dtype dtype, const void* x, const float* dt,
@@ -123,8 +131,11 @@ dart_status dart_ssd_chunk_scan(const dart_dims* d, dart_dtype dtype, const void
     if (workspace_bytes < dart_ssd_chunk_scan_workspace_bytes(d, dtype))
         return fail(DART_ERR_INVALID_ARG, "workspace: %zu bytes, need %zu", workspace_bytes,
                     dart_ssd_chunk_scan_workspace_bytes(d, dtype));
+    const size_t bhc = (size_t)d->batch * (size_t)d->nheads * (size_t)(d->seqlen / d->chunk);
     dart::ScanArgs a{d->batch, d->seqlen, d->nheads, d->headdim, d->dstate, d->chunk,
-                     x, dt, A, Bm, Cm, init_state, y_ssd, dH, states, static_cast<float*>(workspace)};
+                     x, dt, A, Bm, Cm, init_state, y_ssd, dH, states, static_cast<float*>(workspace),
+                     static_cast<char*>(workspace) + scan_asum_bytes(bhc), status_word()};
+    if (!a.status) return fail(DART_ERR_CUDA, "dart_ssd_chunk_scan: no device status word");
     cudaError_t e = dart::launch_ssd_scan(a, dtype, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "dart_ssd_chunk_scan launch");
     return DART_OK;

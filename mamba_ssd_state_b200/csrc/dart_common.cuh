@@ -104,6 +104,8 @@ struct ScanArgs {
     const void* x; const float* dt; const float* A; const void* Bm; const void* Cm;
     const float* init_state;
     float* y; void* dH; float* states; float* asum;  // asum: [B,H,C] workspace
+    void* hin;    // tensor-core path: bf16 state entering each chunk [B,H,C,N,P] (workspace)
+    int* status;  // device status word
 };
 struct SmaArgs {
     int B, L, H, P, N, S;
@@ -127,6 +129,8 @@ cudaError_t launch_ssd_scan(const ScanArgs& a, dart_dtype dt, cudaStream_t st);
 cudaError_t launch_sma(const SmaArgs& a, dart_dtype dt, cudaStream_t st);
 cudaError_t launch_decode(const DecodeArgs& a, dart_dtype dt, cudaStream_t st);
 bool ssd_scan_supported(int N, int P, int S, dart_dtype dt);
+bool ssd_scan_tc_applicable(int N, int P, int S, dart_dtype dt);
+cudaError_t launch_ssd_scan_tc(const ScanArgs& a, cudaStream_t st);
 bool sma_supported(int N, int P, int S, dart_dtype dt);
 bool sma_tc_applicable(int N, int P, int S, dart_dtype dt);
 cudaError_t launch_sma_tc(const SmaArgs& a, cudaStream_t st);

@@ -259,6 +259,7 @@ bool ssd_scan_supported(int N, int P, int S, dart_dtype) {
 }
 
 cudaError_t launch_ssd_scan(const ScanArgs& a, dart_dtype dt, cudaStream_t st) {
+    if (ssd_scan_tc_applicable(a.N, a.P, a.S, dt)) return launch_ssd_scan_tc(a, st);
 #define DART_SCAN_CASE(NN, PP)                                                      \
     if (a.N == NN && a.P == PP)                                                     \
         return dt == DART_F32 ? run<float, NN, PP>(a, st) : run<__nv_bfloat16, NN, PP>(a, st);

@@ -1,0 +1,682 @@
+// ssd_scan_tc.cu -- the SSD chunked scan with retained chunk memories on the
+// 5th-generation tensor cores (bf16 inputs, N = 128, P = 64, S in {128, 256}).
+//
+// Same three stages as the CUDA-core scan (Mamba-2 SSD chunked scan as used by
+// DART: "Transformers are SSMs" SSD view, Eq. (4); Pith review of DART, "What
+// carries the argument" for the retained chunk contribution dH[c]):
+//
+//  chunk_state_tc  one CTA per (b, c, group of heads).  The chunk's B tile
+//      (S x N) is loaded once and shared by every head of the group (B is the
+//      same for all heads, ngroups = 1).  Per head the x tile (S x P) is
+//      scaled in shared memory by w_s = exp(Acum_e - Acum_s) dt_s and
+//        dH[c] = B^T (w o x)      (M = N = 128, N_mma = P = 64, K = S)
+//      runs on the tensor core.  Writes dH (bf16), its fp32 value into
+//      `states` (consumed in place by state_pass) and Asum[c] = Acum_e.
+//  state_pass_tc   states[c] = exp(Asum[c]) states[c-1] + dH[c] in place,
+//      sequential in c; also writes the bf16 state entering each chunk,
+//      hin[c] = bf16(states[c-1]) (hin[0] = init_state or 0), the operand of
+//      the inter-chunk output product.
+//  chunk_output_tc one CTA per (b, c, half of the chunk's rows, group of
+//      heads).  G = C B^T for the half's rows (128 x KS, KS = 128 (half+1))
+//      is computed once into TMEM and shared by the heads of the group.  Per
+//      head the worker warps build P[t,s] = G[t,s] exp(Acum_t - Acum_s)
+//      (s <= t, else 0) in bf16 straight from TMEM into shared memory, scale
+//      the x tile by dt, and the tensor core computes
+//        Y_diag = P (dt o x)          (K = KS)
+//        Y_off  = C hin[c]            (K = N)
+//      y = Y_diag + exp(Acum_t) Y_off.
+//
+// Decay factors: exp(Acum_t - Acum_s) = exp(Acum_t - Acum_r) exp(Acum_r -
+// Acum_s) with r the first token of the 32-token column block holding s; both
+// factors stay inside float range (the second is at most exp(32 |a|max)), so
+// only one exponential per (row, block) and one per column are needed.
+#include <cuda_bf16.h>
+#include <string.h>
+
+#include "dart_common.cuh"
+#include "sm100.cuh"
+#include "tensor_map.h"
+
+namespace dart {
+namespace {
+
+using namespace sm100;
+
+constexpr int kN = 128, kP = 64;
+constexpr uint32_t kRowBytes = 128;                  // one 64-element bf16 row of a swizzle panel
+constexpr uint32_t kBox = 128 * kRowBytes;           // a 128-row TMA box, 16 KB
+
+struct ScanTcParams {
+    CUtensorMap tmap_x;    // x  as (P, B*L, H), box (64, 128, 1)
+    CUtensorMap tmap_b;    // Bm as (N, B*L),    box (64, 128)
+    CUtensorMap tmap_c;    // Cm as (N, B*L),    box (64, 128)
+    CUtensorMap tmap_hin;  // hin as (P, B*H*C*N), box (64, 128)
+    const float* dt;
+    const float* A;
+    const float* init_state;
+    __nv_bfloat16* dH;
+    float* states;
+    float* asum;
+    __nv_bfloat16* hin;
+    float* y;
+    int B, L, H, S, C, HG;
+    int* status;
+};
+
+// Inclusive prefix sum over `n` values held one or two per thread by
+// `nthreads` threads (n <= 2 * nthreads, nthreads a multiple of 32).
+// v0/v1 are this thread's values for elements 2*i, 2*i+1 (pair mode) or
+// element i (single mode, v1 ignored).  Returns the inclusive prefix of each.
+template <bool kPair>
+__device__ __forceinline__ void block_scan(float& v0, float& v1, int i, int nthreads, float* warp_tot, int bar_id) {
+    const int lane = i & 31, w = i >> 5;
+    float local = kPair ? v0 + v1 : v0;
+    float incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const float up = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += up;
+    }
+    if (lane == 31) warp_tot[w] = incl;
+    named_bar_sync(bar_id, nthreads);
+    float base = 0.f;
+    for (int j = 0; j < w; ++j) base += warp_tot[j];
+    const float excl = base + incl - local;
+    if (kPair) {
+        v0 = excl + v0;
+        v1 = v0 + v1;
+    } else {
+        v0 = excl + v0;
+    }
+}
+
+// ===========================================================================
+// chunk_state_tc
+// ===========================================================================
+namespace cs {
+constexpr int kThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 workers
+enum Bar { B_FULL = 0, X_FULL0, X_EMPTY0 = X_FULL0 + 2, W_READY0 = X_EMPTY0 + 2, ACC_FULL0 = W_READY0 + 2,
+           ACC_EMPTY0 = ACC_FULL0 + 2, NUM_BARS = ACC_EMPTY0 + 2 };
+
+template <int S>
+struct Layout {
+    static constexpr uint32_t kOffB = 0;                        // 2 panels x S rows
+    static constexpr uint32_t kOffX = 2 * S * kRowBytes;        // 2 buffers x S rows
+    static constexpr uint32_t kXBytes = S * kRowBytes;
+    static constexpr uint32_t kOffF = kOffX + 2 * kXBytes;      // w[S] floats + 8 warp totals
+    static constexpr uint32_t kOffBar = kOffF + (S + 8) * 4;
+    static constexpr uint32_t kBytes = kOffBar + NUM_BARS * 8 + 16 + 1024;
+};
+
+template <int S>
+__global__ void __launch_bounds__(kThreads, 1) chunk_state_tc_kernel(const __grid_constant__ ScanTcParams p) {
+    using Ly = Layout<S>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    float* w_s = reinterpret_cast<float*>(smem + Ly::kOffF);
+    float* warp_tot = w_s + S;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Ly::kOffBar + NUM_BARS * 8);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+    auto bar = [&](int i) -> uint32_t { return sbase + Ly::kOffBar + 8u * (uint32_t)i; };
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    const int ngroups = p.H / p.HG;
+    const int hg = blockIdx.x % ngroups;
+    const int c = (blockIdx.x / ngroups) % p.C;
+    const int b = blockIdx.x / (ngroups * p.C);
+    const int row0 = b * p.L + c * S;  // first token of the chunk in the (B*L) row space
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar(B_FULL), 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(bar(X_FULL0 + s), 1);
+            mbar_init(bar(X_EMPTY0 + s), 1);
+            mbar_init(bar(W_READY0 + s), 4);
+            mbar_init(bar(ACC_FULL0 + s), 1);
+            mbar_init(bar(ACC_EMPTY0 + s), 4);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_holder), 128);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            tma_prefetch_desc(&p.tmap_x);
+            tma_prefetch_desc(&p.tmap_b);
+            mbar_expect_tx(bar(B_FULL), 2 * S * kRowBytes);
+            for (int pnl = 0; pnl < 2; ++pnl)
+                for (int r = 0; r < S / 128; ++r)
+                    tma_load_2d(sbase + Ly::kOffB + (uint32_t)pnl * S * kRowBytes + (uint32_t)r * kBox, &p.tmap_b,
+                                bar(B_FULL), 64 * pnl, row0 + 128 * r);
+            for (int i = 0; i < p.HG; ++i) {
+                const int xs = i & 1;
+                const uint32_t ph = (uint32_t)(i >> 1) & 1u;
+                if (!mbar_wait(bar(X_EMPTY0 + xs), ph ^ 1u, abort_flag, p.status)) break;
+                mbar_expect_tx(bar(X_FULL0 + xs), Ly::kXBytes);
+                for (int r = 0; r < S / 128; ++r)
+                    tma_load_3d(sbase + Ly::kOffX + (uint32_t)xs * Ly::kXBytes + (uint32_t)r * kBox, &p.tmap_x,
+                                bar(X_FULL0 + xs), 0, row0 + 128 * r, hg * p.HG + i);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // D[n, p] = sum_s B[s, n] W[s, p]: A = B^T (MN-major, M = n over two
+            // 64-wide panels), B = W (MN-major), K = s.
+            const uint32_t idesc = idesc_bf16_f32(128, kP, true, true);
+            bool ok = mbar_wait(bar(B_FULL), 0, abort_flag, p.status);
+            for (int i = 0; i < p.HG && ok; ++i) {
+                const int xs = i & 1, a = i & 1;
+                const uint32_t ph = (uint32_t)(i >> 1) & 1u;
+                if (!mbar_wait(bar(W_READY0 + xs), ph, abort_flag, p.status)) break;
+                if (!mbar_wait(bar(ACC_EMPTY0 + a), ph ^ 1u, abort_flag, p.status)) break;
+                tc_fence_after();
+                const uint32_t xbase = sbase + Ly::kOffX + (uint32_t)xs * Ly::kXBytes;
+#pragma unroll 4
+                for (int kk = 0; kk < S / 16; ++kk) {
+                    const uint64_t ad = smem_desc_sw128(sbase + Ly::kOffB + (uint32_t)kk * 2048, S * kRowBytes, 1024);
+                    const uint64_t bd = smem_desc_sw128(xbase + (uint32_t)kk * 2048, 8192, 1024);
+                    mma_f16_ss(tmem + (uint32_t)a * 64, ad, bd, idesc, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(bar(ACC_FULL0 + a));
+                mma_commit(bar(X_EMPTY0 + xs));
+            }
+        }
+    } else {
+        // ---------------------------------------------------------- workers
+        const int wi = threadIdx.x - 64;            // 0..127
+        const int quad = warp & 3;
+        const int nrow = quad * 32 + lane;          // TMEM lane = state row n
+        const uint32_t t_lane = tmem + ((uint32_t)(quad * 32) << 16);
+        auto epilogue = [&](int i) -> bool {
+            const int a = i & 1;
+            const uint32_t ph = (uint32_t)(i >> 1) & 1u;
+            if (!mbar_wait_warp(bar(ACC_FULL0 + a), ph, abort_flag, p.status)) return false;
+            tc_fence_after();
+            float v[kP];
+            tmem_ld_32x32b_x32(t_lane + (uint32_t)a * 64, v);
+            tmem_ld_32x32b_x32(t_lane + (uint32_t)a * 64 + 32, v + 32);
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(ACC_EMPTY0 + a));
+            const int h = hg * p.HG + i;
+            const size_t off = ((((size_t)b * p.H + h) * p.C + c) * kN + nrow) * kP;
+#pragma unroll
+            for (int q = 0; q < kP; q += 8) {
+                Vec16<__nv_bfloat16>::store(p.dH + off + q, v + q);
+                *reinterpret_cast<float4*>(p.states + off + q) = make_float4(v[q], v[q + 1], v[q + 2], v[q + 3]);
+                *reinterpret_cast<float4*>(p.states + off + q + 4) =
+                    make_float4(v[q + 4], v[q + 5], v[q + 6], v[q + 7]);
+            }
+            return true;
+        };
+        bool ok = true;
+        for (int i = 0; i < p.HG && ok; ++i) {
+            const int h = hg * p.HG + i;
+            const float Ah = p.A[h];
+            if (i > 0) named_bar_sync(1, 128);  // w_s of the previous head fully consumed
+            // per-token log-decay prefix and the memory weights w_s
+            float d0, d1 = 0.f, a0, a1 = 0.f;
+            const float* dtp = p.dt + ((size_t)row0) * p.H + h;
+            if (S == 256) {
+                d0 = dtp[(size_t)(2 * wi) * p.H];
+                d1 = dtp[(size_t)(2 * wi + 1) * p.H];
+                a0 = d0 * Ah;
+                a1 = d1 * Ah;
+                block_scan<true>(a0, a1, wi, 128, warp_tot, 2);
+            } else {
+                d0 = dtp[(size_t)wi * p.H];
+                a0 = d0 * Ah;
+                block_scan<false>(a0, a1, wi, 128, warp_tot, 2);
+            }
+            // total over the chunk: the last thread's inclusive value
+            if (wi == 127) warp_tot[4] = (S == 256) ? a1 : a0;
+            named_bar_sync(1, 128);
+            const float aend = warp_tot[4];
+            if (S == 256) {
+                w_s[2 * wi] = expf(aend - a0) * d0;
+                w_s[2 * wi + 1] = expf(aend - a1) * d1;
+            } else {
+                w_s[wi] = expf(aend - a0) * d0;
+            }
+            if (wi == 0) p.asum[((size_t)b * p.H + h) * p.C + c] = aend;
+            named_bar_sync(1, 128);
+            // scale the x tile in place: row s of the panel times w_s
+            const int xs = i & 1;
+            const uint32_t ph = (uint32_t)(i >> 1) & 1u;
+            if (!mbar_wait_warp(bar(X_FULL0 + xs), ph, abort_flag, p.status)) { ok = false; break; }
+            uint8_t* xb = smem + Ly::kOffX + (uint32_t)xs * Ly::kXBytes;
+            for (int k = wi; k < S * 8; k += 128) {
+                uint4* ptr = reinterpret_cast<uint4*>(xb + (size_t)k * 16);
+                float f[8];
+                Vec16<__nv_bfloat16>::unpack(*ptr, f);
+                const float ws = w_s[k >> 3];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) f[j] *= ws;
+                Vec16<__nv_bfloat16>::store(reinterpret_cast<__nv_bfloat16*>(ptr), f);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(W_READY0 + xs));
+            if (i > 0 && !epilogue(i - 1)) { ok = false; break; }
+        }
+        if (ok) epilogue(p.HG - 1);
+        (void)warp_tot;
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 128);
+    }
+}
+}  // namespace cs
+
+// ===========================================================================
+// state_pass_tc (CUDA cores; memory-bound)
+// ===========================================================================
+__global__ void __launch_bounds__(256) state_pass_tc_kernel(const __grid_constant__ ScanTcParams p) {
+    constexpr int NP = kN * kP;
+    const int h = blockIdx.y, b = blockIdx.z;
+    const int e4 = (blockIdx.x * blockDim.x + threadIdx.x) * 4;  // 4 consecutive elements
+    if (e4 >= NP) return;
+    const size_t bh = (size_t)b * p.H + h;
+    float4 prev = p.init_state ? *reinterpret_cast<const float4*>(p.init_state + bh * NP + e4)
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+    float* st = p.states + bh * (size_t)p.C * NP + e4;
+    __nv_bfloat16* hin = p.hin + bh * (size_t)p.C * NP + e4;
+    const float* asum = p.asum + bh * p.C;
+    for (int c = 0; c < p.C; ++c) {
+        __nv_bfloat162 lo = __floats2bfloat162_rn(prev.x, prev.y), hi = __floats2bfloat162_rn(prev.z, prev.w);
+        uint2 pk;
+        pk.x = *reinterpret_cast<uint32_t*>(&lo);
+        pk.y = *reinterpret_cast<uint32_t*>(&hi);
+        *reinterpret_cast<uint2*>(hin + (size_t)c * NP) = pk;
+        const float dec = expf(asum[c]);
+        const float4 d = *reinterpret_cast<const float4*>(st + (size_t)c * NP);
+        prev = make_float4(fmaf(dec, prev.x, d.x), fmaf(dec, prev.y, d.y), fmaf(dec, prev.z, d.z),
+                           fmaf(dec, prev.w, d.w));
+        *reinterpret_cast<float4*>(st + (size_t)c * NP) = prev;
+    }
+}
+
+// ===========================================================================
+// chunk_output_tc
+// ===========================================================================
+namespace co {
+constexpr int kWorkers = 256;
+constexpr int kThreads = 64 + kWorkers;  // warp 0 TMA, warp 1 MMA, warps 2-9 workers
+enum Bar { IN_FULL = 0, G_FULL, X_FULL0, X_FREE0 = X_FULL0 + 2, READY, P_FREE, ACC_FULL0, ACC_EMPTY0 = ACC_FULL0 + 2,
+           NUM_BARS = ACC_EMPTY0 + 2 };
+constexpr uint32_t kOffC = 0;                          // C rows: 2 panels x 128 rows (32 KB)
+constexpr uint32_t kOffBP = 2 * kBox;                  // B rows (2 panels x KS rows), later P (KS/64 panels x 128 rows)
+constexpr uint32_t kOffX = kOffBP + 4 * kBox;          // 2 buffers x (256 rows x 128 B)
+constexpr uint32_t kXBytes = 2 * kBox;
+constexpr uint32_t kOffHp = kOffX + 2 * kXBytes;       // 2 buffers x 128 rows (16 KB)
+constexpr uint32_t kOffF = kOffHp + 2 * kBox;          // a2[256], colf[256], dts[256], warp totals[16]
+constexpr uint32_t kOffBar = kOffF + (3 * 256 + 16) * 4;
+constexpr uint32_t kBytes = kOffBar + NUM_BARS * 8 + 16 + 1024;
+constexpr uint32_t kColDiag = 256, kColOff = 384;
+
+__global__ void __launch_bounds__(kThreads, 1) chunk_output_tc_kernel(const __grid_constant__ ScanTcParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    float* a2 = reinterpret_cast<float*>(smem + kOffF);   // log2(e) * Acum over the chunk
+    float* colf = a2 + 256;
+    float* dts = colf + 256;
+    float* warp_tot = dts + 256;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + kOffBar + NUM_BARS * 8);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+    auto bar = [&](int i) -> uint32_t { return sbase + kOffBar + 8u * (uint32_t)i; };
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    // CTA -> (b, c, half, head group); the heavier second halves come first
+    const int S = p.S;
+    const int R = S / 128;
+    const int ngroups = p.H / p.HG;
+    int idx = blockIdx.x;
+    const int per_half = p.B * p.C * ngroups;
+    const int half = (R - 1) - idx / per_half;
+    idx %= per_half;
+    const int hg = idx % ngroups;
+    const int c = (idx / ngroups) % p.C;
+    const int b = idx / (ngroups * p.C);
+    const int KS = 128 * (half + 1);               // source tokens this half depends on
+    const int row0 = b * p.L + c * S;              // first token of the chunk
+    const bool has_off = (c > 0) || (p.init_state != nullptr);
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar(IN_FULL), 1);
+        mbar_init(bar(G_FULL), 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(bar(X_FULL0 + s), 1);
+            mbar_init(bar(X_FREE0 + s), 1);
+            mbar_init(bar(ACC_FULL0 + s), 1);
+            mbar_init(bar(ACC_EMPTY0 + s), kWorkers / 32);
+        }
+        mbar_init(bar(READY), kWorkers / 32);
+        mbar_init(bar(P_FREE), 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_holder), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            tma_prefetch_desc(&p.tmap_x);
+            tma_prefetch_desc(&p.tmap_b);
+            tma_prefetch_desc(&p.tmap_c);
+            tma_prefetch_desc(&p.tmap_hin);
+            // C rows of this half (A of G and of Y_off) and B rows 0..KS-1 (B of G)
+            mbar_expect_tx(bar(IN_FULL), 2 * kBox + 2 * (uint32_t)KS * kRowBytes);
+            for (int pnl = 0; pnl < 2; ++pnl) {
+                tma_load_2d(sbase + kOffC + (uint32_t)pnl * kBox, &p.tmap_c, bar(IN_FULL), 64 * pnl,
+                            row0 + 128 * half);
+                for (int r = 0; r < KS / 128; ++r)
+                    tma_load_2d(sbase + kOffBP + (uint32_t)pnl * KS * kRowBytes + (uint32_t)r * kBox, &p.tmap_b,
+                                bar(IN_FULL), 64 * pnl, row0 + 128 * r);
+            }
+            for (int i = 0; i < p.HG; ++i) {
+                const int xs = i & 1;
+                const uint32_t ph = (uint32_t)(i >> 1) & 1u;
+                const int h = hg * p.HG + i;
+                if (!mbar_wait(bar(X_FREE0 + xs), ph ^ 1u, abort_flag, p.status)) break;
+                const uint32_t bytes = (uint32_t)KS * kRowBytes + (has_off ? kBox : 0u);
+                mbar_expect_tx(bar(X_FULL0 + xs), bytes);
+                for (int r = 0; r < KS / 128; ++r)
+                    tma_load_3d(sbase + kOffX + (uint32_t)xs * kXBytes + (uint32_t)r * kBox, &p.tmap_x,
+                                bar(X_FULL0 + xs), 0, row0 + 128 * r, h);
+                if (has_off)
+                    tma_load_2d(sbase + kOffHp + (uint32_t)xs * kBox, &p.tmap_hin, bar(X_FULL0 + xs), 0,
+                                ((b * p.H + h) * p.C + c) * kN);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            bool ok = mbar_wait(bar(IN_FULL), 0, abort_flag, p.status);
+            if (ok) {
+                // G[t, s] = sum_n C[t, n] B[s, n]: both K-major, K = N.
+                tc_fence_after();
+                const uint32_t idesc_g = idesc_bf16_f32(128, KS, false, false);
+#pragma unroll
+                for (int kk = 0; kk < kN / 16; ++kk) {
+                    const uint32_t koff = (uint32_t)(kk & 3) * 32;   // 16 K-elements inside a panel
+                    const uint64_t ad = smem_desc_sw128(sbase + kOffC + (uint32_t)(kk >> 2) * kBox + koff, 16, 1024);
+                    const uint64_t bd = smem_desc_sw128(
+                        sbase + kOffBP + (uint32_t)(kk >> 2) * (uint32_t)KS * kRowBytes + koff, 16, 1024);
+                    mma_f16_ss(tmem, ad, bd, idesc_g, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(bar(G_FULL));
+            }
+            const uint32_t idesc_y = idesc_bf16_f32(128, kP, false, true);
+            for (int i = 0; i < p.HG && ok; ++i) {
+                const int xs = i & 1, a = i & 1;
+                const uint32_t ph = (uint32_t)(i >> 1) & 1u;
+                if (!mbar_wait(bar(READY), (uint32_t)i & 1u, abort_flag, p.status)) break;
+                if (!mbar_wait(bar(ACC_EMPTY0 + a), ph ^ 1u, abort_flag, p.status)) break;
+                tc_fence_after();
+                // Y_diag = P (dt o x): A = P (K-major, K = s), B = x (MN-major)
+                const uint32_t xbase = sbase + kOffX + (uint32_t)xs * kXBytes;
+                for (int kk = 0; kk < KS / 16; ++kk) {
+                    const uint64_t ad = smem_desc_sw128(sbase + kOffBP + (uint32_t)(kk >> 2) * kBox + (uint32_t)(kk & 3) * 32,
+                                                        16, 1024);
+                    const uint64_t bd = smem_desc_sw128(xbase + (uint32_t)kk * 2048, 8192, 1024);
+                    mma_f16_ss(tmem + kColDiag + (uint32_t)a * 64, ad, bd, idesc_y, kk > 0 ? 1u : 0u);
+                }
+                if (has_off) {
+                    // Y_off = C hin[c]: A = C rows (K-major, K = n), B = hin (MN-major)
+                    const uint32_t hbase = sbase + kOffHp + (uint32_t)xs * kBox;
+#pragma unroll
+                    for (int kk = 0; kk < kN / 16; ++kk) {
+                        const uint64_t ad = smem_desc_sw128(
+                            sbase + kOffC + (uint32_t)(kk >> 2) * kBox + (uint32_t)(kk & 3) * 32, 16, 1024);
+                        const uint64_t bd = smem_desc_sw128(hbase + (uint32_t)kk * 2048, 8192, 1024);
+                        mma_f16_ss(tmem + kColOff + (uint32_t)a * 64, ad, bd, idesc_y, kk > 0 ? 1u : 0u);
+                    }
+                }
+                mma_commit(bar(ACC_FULL0 + a));
+                mma_commit(bar(X_FREE0 + xs));
+                mma_commit(bar(P_FREE));
+            }
+        }
+    } else {
+        // ---------------------------------------------------------- workers
+        const int wi = threadIdx.x - 64;                 // 0..255
+        const int wk = warp - 2;                         // 0..7
+        const int quad = warp & 3;                       // TMEM lane quadrant
+        const int colhalf = wk >> 2;                     // which half of the columns
+        const int trow = quad * 32 + lane;               // row inside the half (TMEM lane)
+        const int t = 128 * half + trow;                 // chunk-local token of this row
+        const uint32_t t_lane = tmem + ((uint32_t)(quad * 32) << 16);
+        const int nblk = KS / 32;                        // 32-column blocks of P
+        const int blk0 = colhalf * (nblk / 2), blk1 = blk0 + nblk / 2;
+        float row_scale_prev = 0.f;
+        auto epilogue = [&](int i, float row_scale) -> bool {
+            const int a = i & 1;
+            const uint32_t ph = (uint32_t)(i >> 1) & 1u;
+            if (!mbar_wait_warp(bar(ACC_FULL0 + a), ph, abort_flag, p.status)) return false;
+            tc_fence_after();
+            float yd[32], yo[32];
+            tmem_ld_32x32b_x32(t_lane + kColDiag + (uint32_t)a * 64 + (uint32_t)colhalf * 32, yd);
+            if (has_off) tmem_ld_32x32b_x32(t_lane + kColOff + (uint32_t)a * 64 + (uint32_t)colhalf * 32, yo);
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(ACC_EMPTY0 + a));
+            const int h = hg * p.HG + i;
+            float* yrow = p.y + (((size_t)row0 + t) * p.H + h) * kP + colhalf * 32;
+#pragma unroll
+            for (int q = 0; q < 32; q += 4) {
+                float4 r = make_float4(yd[q], yd[q + 1], yd[q + 2], yd[q + 3]);
+                if (has_off) {
+                    r.x = fmaf(row_scale, yo[q], r.x);
+                    r.y = fmaf(row_scale, yo[q + 1], r.y);
+                    r.z = fmaf(row_scale, yo[q + 2], r.z);
+                    r.w = fmaf(row_scale, yo[q + 3], r.w);
+                }
+                *reinterpret_cast<float4*>(yrow + q) = r;
+            }
+            return true;
+        };
+        bool ok = true;
+        for (int i = 0; i < p.HG && ok; ++i) {
+            const int h = hg * p.HG + i;
+            const float Ah = p.A[h] * kLog2e;
+            if (i > 0) named_bar_sync(1, kWorkers);      // a2 / colf / dts of the previous head consumed
+            // log2-domain prefix of the decay over the chunk's first KS tokens
+            float d0 = 0.f, v0 = 0.f, v1 = 0.f;
+            if (wi < KS) {
+                d0 = p.dt[((size_t)row0 + wi) * p.H + h];
+                v0 = d0 * Ah;
+            }
+            block_scan<false>(v0, v1, wi, kWorkers, warp_tot, 2);
+            if (wi < KS) {
+                a2[wi] = v0;
+                dts[wi] = d0;
+            }
+            named_bar_sync(1, kWorkers);
+            if (wi < KS) colf[wi] = exp2f(a2[wi & ~31] - a2[wi]);
+            const float a2t = a2[t];
+            const float row_scale = exp2f(a2t);          // exp(Acum_t): decay from the chunk start
+            named_bar_sync(1, kWorkers);
+            // scale x rows by dt in place
+            const int xs = i & 1;
+            const uint32_t ph = (uint32_t)(i >> 1) & 1u;
+            if (!mbar_wait_warp(bar(X_FULL0 + xs), ph, abort_flag, p.status)) { ok = false; break; }
+            uint8_t* xb = smem + kOffX + (uint32_t)xs * kXBytes;
+            for (int k = wi; k < KS * 8; k += kWorkers) {
+                uint4* ptr = reinterpret_cast<uint4*>(xb + (size_t)k * 16);
+                float f[8];
+                Vec16<__nv_bfloat16>::unpack(*ptr, f);
+                const float ds = dts[k >> 3];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) f[j] *= ds;
+                Vec16<__nv_bfloat16>::store(reinterpret_cast<__nv_bfloat16*>(ptr), f);
+            }
+            // P may be written once G (first head) or the previous head's MMA has consumed the buffer
+            if (i == 0) {
+                if (!mbar_wait_warp(bar(G_FULL), 0, abort_flag, p.status)) { ok = false; break; }
+            } else {
+                if (!mbar_wait_warp(bar(P_FREE), (uint32_t)(i - 1) & 1u, abort_flag, p.status)) { ok = false; break; }
+            }
+            tc_fence_after();
+            // P[t, s] = G[t, s] * exp(Acum_t - Acum_r) * exp(Acum_r - Acum_s), s <= t
+            const int warp_tmax = 128 * half + 32 * quad + 31;   // last row of this warp
+            for (int j = blk0; j < blk1; ++j) {
+                const int s0 = 32 * j;
+                uint32_t packed[16];
+                float g[32];
+                const bool warp_needs = s0 <= warp_tmax;            // warp-uniform
+                if (warp_needs) {
+                    tmem_ld_32x32b_x32(t_lane + (uint32_t)s0, g);
+                    tmem_ld_wait();
+                }
+                if (warp_needs && s0 <= t) {
+                    const float rf = exp2f(a2t - a2[s0]);
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) {
+                        const int sa = s0 + 2 * q, sb = sa + 1;
+                        const float va = sa <= t ? g[2 * q] * rf * colf[sa] : 0.f;
+                        const float vb = sb <= t ? g[2 * q + 1] * rf * colf[sb] : 0.f;
+                        __nv_bfloat162 pr = __floats2bfloat162_rn(va, vb);
+                        packed[q] = *reinterpret_cast<uint32_t*>(&pr);
+                    }
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) packed[q] = 0u;
+                }
+                // row trow of panel j/2, 16-byte chunks (j%2)*4 .. +3, 128-byte swizzle
+                uint8_t* prow = smem + kOffBP + (uint32_t)(j >> 1) * kBox + (uint32_t)trow * kRowBytes;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int ch = ((j & 1) * 4 + u) ^ (trow & 7);
+                    *reinterpret_cast<uint4*>(prow + ch * 16) =
+                        make_uint4(packed[4 * u], packed[4 * u + 1], packed[4 * u + 2], packed[4 * u + 3]);
+                }
+            }
+            tc_fence_before();
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(READY));
+            if (i > 0 && !epilogue(i - 1, row_scale_prev)) { ok = false; break; }
+            row_scale_prev = row_scale;
+        }
+        if (ok) epilogue(p.HG - 1, row_scale_prev);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+}  // namespace co
+
+bool make_maps(const ScanArgs& a, ScanTcParams& p) {
+    const uint64_t BL = (uint64_t)a.B * a.L;
+    const int C = a.L / a.S;
+    {
+        const uint64_t dims[3] = {(uint64_t)kP, BL, (uint64_t)a.H};
+        const uint64_t strides[2] = {(uint64_t)a.H * kP * 2, (uint64_t)kP * 2};
+        const uint32_t box[3] = {64, 128, 1};
+        if (!encode_tile_map_bf16(&p.tmap_x, 3, a.x, dims, strides, box)) return false;
+    }
+    {
+        const uint64_t dims[2] = {(uint64_t)kN, BL};
+        const uint64_t strides[1] = {(uint64_t)kN * 2};
+        const uint32_t box[2] = {64, 128};
+        if (!encode_tile_map_bf16(&p.tmap_b, 2, a.Bm, dims, strides, box)) return false;
+        if (!encode_tile_map_bf16(&p.tmap_c, 2, a.Cm, dims, strides, box)) return false;
+    }
+    {
+        const uint64_t dims[2] = {(uint64_t)kP, (uint64_t)a.B * a.H * C * kN};
+        const uint64_t strides[1] = {(uint64_t)kP * 2};
+        const uint32_t box[2] = {64, 128};
+        if (!encode_tile_map_bf16(&p.tmap_hin, 2, a.hin, dims, strides, box)) return false;
+    }
+    return true;
+}
+
+int pick_group(int H, int want) {
+    int g = want < H ? want : H;
+    while (H % g) --g;
+    return g;
+}
+
+}  // namespace
+
+bool ssd_scan_tc_applicable(int N, int P, int S, dart_dtype dt) {
+    return dt == DART_BF16 && N == kN && P == kP && (S == 128 || S == 256);
+}
+
+cudaError_t launch_ssd_scan_tc(const ScanArgs& a, cudaStream_t st) {
+    ScanTcParams p;
+    memset(&p, 0, sizeof(p));
+    if (!make_maps(a, p)) return cudaErrorInvalidValue;
+    p.dt = a.dt;
+    p.A = a.A;
+    p.init_state = a.init_state;
+    p.dH = static_cast<__nv_bfloat16*>(a.dH);
+    p.states = a.states;
+    p.asum = a.asum;
+    p.hin = static_cast<__nv_bfloat16*>(a.hin);
+    p.y = a.y;
+    p.B = a.B; p.L = a.L; p.H = a.H; p.S = a.S; p.C = a.L / a.S;
+    p.status = a.status;
+    cudaError_t e;
+    // 1. chunk memories
+    p.HG = pick_group(a.H, 8);
+    {
+        const int grid = a.B * p.C * (a.H / p.HG);
+        if (a.S == 256) {
+            auto k = cs::chunk_state_tc_kernel<256>;
+            const uint32_t smem = cs::Layout<256>::kBytes;
+            if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+                return e;
+            k<<<grid, cs::kThreads, smem, st>>>(p);
+        } else {
+            auto k = cs::chunk_state_tc_kernel<128>;
+            const uint32_t smem = cs::Layout<128>::kBytes;
+            if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+                return e;
+            k<<<grid, cs::kThreads, smem, st>>>(p);
+        }
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    // 2. state passing
+    state_pass_tc_kernel<<<dim3(kN * kP / 4 / 256, a.H, a.B), 256, 0, st>>>(p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    // 3. outputs
+    p.HG = pick_group(a.H, 16);
+    {
+        const int grid = a.B * p.C * (a.H / p.HG) * (a.S / 128);
+        if ((e = cudaFuncSetAttribute(co::chunk_output_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)co::kBytes)) != cudaSuccess)
+            return e;
+        co::chunk_output_tc_kernel<<<grid, co::kThreads, co::kBytes, st>>>(p);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    count_launches(3);
+    return cudaSuccess;
+}
+
+}  // namespace dart
