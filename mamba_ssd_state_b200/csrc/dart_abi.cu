@@ -9,7 +9,9 @@
 #include "dart_common.cuh"
 
 namespace dart {
-__device__ int g_status = 0;
+// [0]: status flags; [1]: (kernel id << 8 | wait site) of the first bounded
+// wait that gave up, 0 if none.
+__device__ int g_status[2] = {0, 0};
 
 namespace {
 std::atomic<unsigned long long> g_launches{0};
@@ -198,16 +200,18 @@ dart_status dart_sync_status(void* stream) {
     t_err[0] = 0;
     cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "dart_sync_status: stream synchronize");
-    int flags = 0;
-    e = cudaMemcpyFromSymbol(&flags, dart::g_status, sizeof(int));
+    int words[2] = {0, 0};
+    e = cudaMemcpyFromSymbol(words, dart::g_status, sizeof(words));
     if (e != cudaSuccess) return cuda_fail(e, "dart_sync_status: read status");
-    if (flags) {
-        const int zero = 0;
-        e = cudaMemcpyToSymbol(dart::g_status, &zero, sizeof(int));
+    if (words[0] || words[1]) {
+        const int zero[2] = {0, 0};
+        e = cudaMemcpyToSymbol(dart::g_status, zero, sizeof(zero));
         if (e != cudaSuccess) return cuda_fail(e, "dart_sync_status: clear status");
     }
-    if (flags & dart::kStatusTimeout) return fail(DART_ERR_TIMEOUT, "a bounded device wait gave up");
-    if (flags & dart::kStatusDevice)
+    if (words[0] & dart::kStatusTimeout)
+        return fail(DART_ERR_TIMEOUT, "a bounded device wait gave up (kernel %d, wait site %d)", words[1] >> 8,
+                    words[1] & 0xff);
+    if (words[0] & dart::kStatusDevice)
         return fail(DART_ERR_DEVICE, "device flagged bad state (decode counters out of range or cache full)");
     return DART_OK;
 }

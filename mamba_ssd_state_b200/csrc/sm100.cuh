@@ -3,8 +3,12 @@
 // tcgen05.mma / commit / ld, and the shared-memory matrix descriptors.
 //
 // Every wait is bounded: a wait that has not completed after kWaitLimitNs
-// latches the timeout bit in the device status word, raises the CTA's abort
-// flag and returns false, so that no kernel can spin forever.
+// (or kWaitIterCap polls) latches the timeout bit in the device status word,
+// records where it gave up, raises the CTA's abort flag and returns false,
+// so that no kernel can spin forever.  Kernels built on these waits keep
+// every block-level barrier reachable after an abort: role loops run on
+// whole warps, and warps that share named barriers never leave the barrier
+// sequence early.
 #pragma once
 
 #include <cuda.h>
@@ -56,18 +60,32 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// What a wait needs besides the barrier: the CTA's abort flag (shared
+// memory), the device status words ([0] flags, [1] first timeout site) and a
+// kernel id that, with the call site, identifies a wait that gave up.
+struct WaitCtx {
+    volatile int* abort_flag;
+    int* status;
+    int kernel_id;
+};
+
+constexpr uint32_t kWaitIterCap = 1u << 26;  // second bound, independent of the timer
+
 // Waits until the phase with the given parity has completed.  Returns false
-// (after flagging) if the wait gave up or another role already aborted.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* status) {
+// at once if the CTA already aborted; returns false after flagging (timeout
+// bit, first timeout site, CTA abort flag) if the wait passed its limit.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCtx& w, int site) {
+    if (*w.abort_flag) return false;
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = global_ns();
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((i & 63u) == 0) {
-            if (*abort_flag) return false;
-            if (global_ns() - t0 > kWaitLimitNs) {
-                *abort_flag = 1;
-                flag_status(status, kStatusTimeout);
+            if (*w.abort_flag) return false;
+            if (global_ns() - t0 > kWaitLimitNs || i >= kWaitIterCap) {
+                *w.abort_flag = 1;
+                flag_status(w.status, kStatusTimeout);
+                atomicCAS(w.status + 1, 0, (w.kernel_id << 8) | site);
                 return false;
             }
         }
@@ -77,10 +95,9 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 // Warp-uniform wait: lane 0 polls, the verdict is broadcast, and the warp
 // reconverges, so that the .sync.aligned tcgen05 instructions that follow
 // are always reached by all 32 lanes together.
-__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                               int* status) {
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, const WaitCtx& w, int site) {
     int ok = 0;
-    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort_flag, status) ? 1 : 0;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, w, site) ? 1 : 0;
     ok = __shfl_sync(0xffffffffu, ok, 0);
     __syncwarp();
     return ok != 0;

@@ -136,63 +136,70 @@ __global__ void __launch_bounds__(kThreads, 1) sma_tc_kernel(const __grid_consta
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
 
+    const WaitCtx wc{abort_flag, p.status, 1};
     if (warp == 0) {
         // ------------------------------------------------------------ TMA
-        if (lane == 0) {
-            uint32_t q_ph = 0, c_ph = 0;
-            int it_b = 0;
-            for (int i = blockIdx.x; i < p.total_tiles; i += gridDim.x) {
-                const Tile t = decode_tile(p, i);
-                if (t.k == 0) continue;
-                const int row = t.b * p.L + t.t0;
-                if (!mbar_wait(bar(Q_FREE), q_ph ^ 1, abort_flag, p.status)) break;
+        // The whole warp walks the schedule; lane 0 issues the copies.
+        uint32_t q_ph = 0, c_ph = 0;
+        int it_b = 0;
+        bool ok = true;
+        for (int i = blockIdx.x; i < p.total_tiles && ok; i += gridDim.x) {
+            const Tile t = decode_tile(p, i);
+            if (t.k == 0) continue;
+            const int row = t.b * p.L + t.t0;
+            if (!(ok = mbar_wait_warp(bar(Q_FREE), q_ph ^ 1, wc, 1))) break;
+            if (lane == 0) {
                 mbar_expect_tx(bar(Q_FULL), 2 * kHalfA);
                 tma_load_3d(sbase + kOffQ, &p.tmap_q, bar(Q_FULL), 0, row, t.h);
                 tma_load_3d(sbase + kOffQ + kHalfA, &p.tmap_q, bar(Q_FULL), 64, row, t.h);
-                q_ph ^= 1;
-                if (!mbar_wait(bar(C_FREE), c_ph ^ 1, abort_flag, p.status)) break;
+            }
+            q_ph ^= 1;
+            if (!(ok = mbar_wait_warp(bar(C_FREE), c_ph ^ 1, wc, 2))) break;
+            if (lane == 0) {
                 mbar_expect_tx(bar(C_FULL), 2 * kHalfA);
                 tma_load_2d(sbase + kOffC, &p.tmap_c, bar(C_FULL), 0, row);
                 tma_load_2d(sbase + kOffC + kHalfA, &p.tmap_c, bar(C_FULL), 64, row);
-                c_ph ^= 1;
-                const int nbatch = (t.k + kCB - 1) / kCB;
-                bool ok = true;
-                for (int j = 0; j < nbatch && ok; ++j, ++it_b) {
-                    const int nv = min(kCB, t.k - kCB * j);
-                    const int s = it_b % kNB;
-                    const uint32_t ph = (uint32_t)(it_b / kNB) & 1u;
-                    if (!mbar_wait(bar(B_EMPTY0 + s), ph ^ 1, abort_flag, p.status)) { ok = false; break; }
+            }
+            c_ph ^= 1;
+            const int nbatch = (t.k + kCB - 1) / kCB;
+            for (int j = 0; j < nbatch; ++j, ++it_b) {
+                const int nv = min(kCB, t.k - kCB * j);
+                const int s = it_b % kNB;
+                const uint32_t ph = (uint32_t)(it_b / kNB) & 1u;
+                if (!(ok = mbar_wait_warp(bar(B_EMPTY0 + s), ph ^ 1, wc, 3))) break;
+                if (lane == 0) {
                     mbar_expect_tx(bar(B_FULL0 + s), (uint32_t)nv * kMemBytes);
                     const int mem_row = ((t.b * p.H + t.h) * p.C + kCB * j) * kN;
                     for (int q = 0; q < nv; ++q)
                         tma_load_2d(sbase + kOffB + (uint32_t)s * kStageBytes + (uint32_t)q * kMemBytes, &p.tmap_h,
                                     bar(B_FULL0 + s), 0, mem_row + q * kN);
                 }
-                if (!ok) break;
             }
+            __syncwarp();
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA
-        if (lane == 0) {
-            uint32_t q_ph = 0, c_ph = 0;
-            int it_b = 0, it_u = 0;
-            bool ok = true;
-            for (int i = blockIdx.x; i < p.total_tiles && ok; i += gridDim.x) {
-                const Tile t = decode_tile(p, i);
-                if (t.k == 0) continue;
-                if (!mbar_wait(bar(Q_FULL), q_ph, abort_flag, p.status)) break;
-                q_ph ^= 1;
+        // The whole warp walks the schedule; lane 0 issues the MMAs.
+        uint32_t q_ph = 0, c_ph = 0;
+        int it_b = 0, it_u = 0;
+        bool ok = true;
+        for (int i = blockIdx.x; i < p.total_tiles && ok; i += gridDim.x) {
+            const Tile t = decode_tile(p, i);
+            if (t.k == 0) continue;
+            if (!(ok = mbar_wait_warp(bar(Q_FULL), q_ph, wc, 4))) break;
+            q_ph ^= 1;
+            tc_fence_after();
+            const int nbatch = (t.k + kCB - 1) / kCB;
+            for (int j = 0; j < nbatch; ++j, ++it_b, ++it_u) {
+                const int nv = min(kCB, t.k - kCB * j);
+                const int s = it_b % kNB;
+                const uint32_t ph = (uint32_t)(it_b / kNB) & 1u;
+                const uint32_t idesc = idesc_bf16_f32(kBQ, kP * nv, false, true);
+                const uint32_t b_base = sbase + kOffB + (uint32_t)s * kStageBytes;
+                if (!(ok = mbar_wait_warp(bar(B_FULL0 + s), ph, wc, 5))) break;
+                if (!(ok = mbar_wait_warp(bar(U_EMPTY), ((uint32_t)it_u & 1u) ^ 1u, wc, 6))) break;
                 tc_fence_after();
-                const int nbatch = (t.k + kCB - 1) / kCB;
-                for (int j = 0; j < nbatch; ++j, ++it_b, ++it_u) {
-                    const int nv = min(kCB, t.k - kCB * j);
-                    const int s = it_b % kNB;
-                    const uint32_t ph = (uint32_t)(it_b / kNB) & 1u;
-                    const uint32_t idesc = idesc_bf16_f32(kBQ, kP * nv, false, true);
-                    const uint32_t b_base = sbase + kOffB + (uint32_t)s * kStageBytes;
-                    if (!mbar_wait(bar(B_FULL0 + s), ph, abort_flag, p.status)) { ok = false; break; }
-                    if (!mbar_wait(bar(U_EMPTY), ((uint32_t)it_u & 1u) ^ 1u, abort_flag, p.status)) { ok = false; break; }
-                    tc_fence_after();
+                if (lane == 0) {
 #pragma unroll
                     for (int kk = 0; kk < kN / 16; ++kk) {
                         const uint64_t ad = smem_desc_sw128(sbase + kOffQ + (uint32_t)(kk >> 2) * kHalfA + (uint32_t)(kk & 3) * 32, 16, 1024);
@@ -201,12 +208,15 @@ __global__ void __launch_bounds__(kThreads, 1) sma_tc_kernel(const __grid_consta
                     }
                     mma_commit(bar(U_FULL));
                     if (j == nbatch - 1) mma_commit(bar(Q_FREE));
-                    if (j == 0) {
-                        if (!mbar_wait(bar(C_FULL), c_ph, abort_flag, p.status)) { ok = false; break; }
-                        c_ph ^= 1;
-                    }
-                    if (!mbar_wait(bar(V_EMPTY), ((uint32_t)it_u & 1u) ^ 1u, abort_flag, p.status)) { ok = false; break; }
-                    tc_fence_after();
+                }
+                __syncwarp();
+                if (j == 0) {
+                    if (!(ok = mbar_wait_warp(bar(C_FULL), c_ph, wc, 7))) break;
+                    c_ph ^= 1;
+                }
+                if (!(ok = mbar_wait_warp(bar(V_EMPTY), ((uint32_t)it_u & 1u) ^ 1u, wc, 8))) break;
+                tc_fence_after();
+                if (lane == 0) {
 #pragma unroll
                     for (int kk = 0; kk < kN / 16; ++kk) {
                         const uint64_t ad = smem_desc_sw128(sbase + kOffC + (uint32_t)(kk >> 2) * kHalfA + (uint32_t)(kk & 3) * 32, 16, 1024);
@@ -217,6 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1) sma_tc_kernel(const __grid_consta
                     mma_commit(bar(B_EMPTY0 + s));
                     if (j == nbatch - 1) mma_commit(bar(C_FREE));
                 }
+                __syncwarp();
             }
         }
     } else {
@@ -244,7 +255,7 @@ __global__ void __launch_bounds__(kThreads, 1) sma_tc_kernel(const __grid_consta
                 for (int j = 0; j < nbatch; ++j, ++it_u) {
                     const int nv = min(kCB, t.k - kCB * j);
                     const uint32_t ph = (uint32_t)it_u & 1u;
-                    if (!mbar_wait_warp(bar(U_FULL), ph, abort_flag, p.status)) { ok = false; break; }
+                    if (!mbar_wait_warp(bar(U_FULL), ph, wc, 9)) { ok = false; break; }
                     tc_fence_after();
                     float sc[kCB];
 #pragma unroll
@@ -278,7 +289,7 @@ __global__ void __launch_bounds__(kThreads, 1) sma_tc_kernel(const __grid_consta
                     m = mnew;
 #pragma unroll
                     for (int q = 0; q < kP; ++q) o[q] *= alpha;
-                    if (!mbar_wait_warp(bar(V_FULL), ph, abort_flag, p.status)) { ok = false; break; }
+                    if (!mbar_wait_warp(bar(V_FULL), ph, wc, 10)) { ok = false; break; }
                     tc_fence_after();
 #pragma unroll
                     for (int c = 0; c < kCB; ++c) {

@@ -148,7 +148,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_state_tc_kernel(const __gri
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
 
+    const WaitCtx wc{abort_flag, p.status, 2};
     if (warp == 0) {
+        // TMA: the whole warp walks the heads, lane 0 issues
         if (lane == 0) {
             tma_prefetch_desc(&p.tmap_x);
             tma_prefetch_desc(&p.tmap_b);
@@ -157,28 +159,32 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_state_tc_kernel(const __gri
                 for (int r = 0; r < S / 128; ++r)
                     tma_load_2d(sbase + Ly::kOffB + (uint32_t)pnl * S * kRowBytes + (uint32_t)r * kBox, &p.tmap_b,
                                 bar(B_FULL), 64 * pnl, row0 + 128 * r);
-            for (int i = 0; i < p.HG; ++i) {
-                const int xs = i & 1;
-                const uint32_t ph = (uint32_t)(i >> 1) & 1u;
-                if (!mbar_wait(bar(X_EMPTY0 + xs), ph ^ 1u, abort_flag, p.status)) break;
+        }
+        __syncwarp();
+        for (int i = 0; i < p.HG; ++i) {
+            const int xs = i & 1;
+            const uint32_t ph = (uint32_t)(i >> 1) & 1u;
+            if (!mbar_wait_warp(bar(X_EMPTY0 + xs), ph ^ 1u, wc, 1)) break;
+            if (lane == 0) {
                 mbar_expect_tx(bar(X_FULL0 + xs), Ly::kXBytes);
                 for (int r = 0; r < S / 128; ++r)
                     tma_load_3d(sbase + Ly::kOffX + (uint32_t)xs * Ly::kXBytes + (uint32_t)r * kBox, &p.tmap_x,
                                 bar(X_FULL0 + xs), 0, row0 + 128 * r, hg * p.HG + i);
             }
+            __syncwarp();
         }
     } else if (warp == 1) {
-        if (lane == 0) {
-            // D[n, p] = sum_s B[s, n] W[s, p]: A = B^T (MN-major, M = n over two
-            // 64-wide panels), B = W (MN-major), K = s.
-            const uint32_t idesc = idesc_bf16_f32(128, kP, true, true);
-            bool ok = mbar_wait(bar(B_FULL), 0, abort_flag, p.status);
-            for (int i = 0; i < p.HG && ok; ++i) {
-                const int xs = i & 1, a = i & 1;
-                const uint32_t ph = (uint32_t)(i >> 1) & 1u;
-                if (!mbar_wait(bar(W_READY0 + xs), ph, abort_flag, p.status)) break;
-                if (!mbar_wait(bar(ACC_EMPTY0 + a), ph ^ 1u, abort_flag, p.status)) break;
-                tc_fence_after();
+        // MMA: D[n, p] = sum_s B[s, n] W[s, p]: A = B^T (MN-major, M = n over
+        // two 64-wide panels), B = W (MN-major), K = s.  Lane 0 issues.
+        const uint32_t idesc = idesc_bf16_f32(128, kP, true, true);
+        bool ok = mbar_wait_warp(bar(B_FULL), 0, wc, 2);
+        for (int i = 0; i < p.HG && ok; ++i) {
+            const int xs = i & 1, a = i & 1;
+            const uint32_t ph = (uint32_t)(i >> 1) & 1u;
+            if (!(ok = mbar_wait_warp(bar(W_READY0 + xs), ph, wc, 3))) break;
+            if (!(ok = mbar_wait_warp(bar(ACC_EMPTY0 + a), ph ^ 1u, wc, 4))) break;
+            tc_fence_after();
+            if (lane == 0) {
                 const uint32_t xbase = sbase + Ly::kOffX + (uint32_t)xs * Ly::kXBytes;
 #pragma unroll 4
                 for (int kk = 0; kk < S / 16; ++kk) {
@@ -189,9 +195,13 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_state_tc_kernel(const __gri
                 mma_commit(bar(ACC_FULL0 + a));
                 mma_commit(bar(X_EMPTY0 + xs));
             }
+            __syncwarp();
         }
     } else {
         // ---------------------------------------------------------- workers
+        // Every worker warp executes the same sequence of named barriers for
+        // every head, also after a failed wait (it then skips the work), so
+        // no warp can be left waiting at a barrier the others never reach.
         const int wi = threadIdx.x - 64;            // 0..127
         const int quad = warp & 3;
         const int nrow = quad * 32 + lane;          // TMEM lane = state row n
@@ -199,7 +209,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_state_tc_kernel(const __gri
         auto epilogue = [&](int i) -> bool {
             const int a = i & 1;
             const uint32_t ph = (uint32_t)(i >> 1) & 1u;
-            if (!mbar_wait_warp(bar(ACC_FULL0 + a), ph, abort_flag, p.status)) return false;
+            if (!mbar_wait_warp(bar(ACC_FULL0 + a), ph, wc, 5)) return false;
             tc_fence_after();
             float v[kP];
             tmem_ld_32x32b_x32(t_lane + (uint32_t)a * 64, v);
@@ -220,7 +230,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_state_tc_kernel(const __gri
             return true;
         };
         bool ok = true;
-        for (int i = 0; i < p.HG && ok; ++i) {
+        for (int i = 0; i < p.HG; ++i) {
             const int h = hg * p.HG + i;
             const float Ah = p.A[h];
             if (i > 0) named_bar_sync(1, 128);  // w_s of the previous head fully consumed
@@ -253,24 +263,25 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_state_tc_kernel(const __gri
             // scale the x tile in place: row s of the panel times w_s
             const int xs = i & 1;
             const uint32_t ph = (uint32_t)(i >> 1) & 1u;
-            if (!mbar_wait_warp(bar(X_FULL0 + xs), ph, abort_flag, p.status)) { ok = false; break; }
-            uint8_t* xb = smem + Ly::kOffX + (uint32_t)xs * Ly::kXBytes;
-            for (int k = wi; k < S * 8; k += 128) {
-                uint4* ptr = reinterpret_cast<uint4*>(xb + (size_t)k * 16);
-                float f[8];
-                Vec16<__nv_bfloat16>::unpack(*ptr, f);
-                const float ws = w_s[k >> 3];
+            if (ok) ok = mbar_wait_warp(bar(X_FULL0 + xs), ph, wc, 6);
+            if (ok) {
+                uint8_t* xb = smem + Ly::kOffX + (uint32_t)xs * Ly::kXBytes;
+                for (int k = wi; k < S * 8; k += 128) {
+                    uint4* ptr = reinterpret_cast<uint4*>(xb + (size_t)k * 16);
+                    float f[8];
+                    Vec16<__nv_bfloat16>::unpack(*ptr, f);
+                    const float ws = w_s[k >> 3];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) f[j] *= ws;
-                Vec16<__nv_bfloat16>::store(reinterpret_cast<__nv_bfloat16*>(ptr), f);
+                    for (int j = 0; j < 8; ++j) f[j] *= ws;
+                    Vec16<__nv_bfloat16>::store(reinterpret_cast<__nv_bfloat16*>(ptr), f);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(W_READY0 + xs));
             }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(W_READY0 + xs));
-            if (i > 0 && !epilogue(i - 1)) { ok = false; break; }
+            if (ok && i > 0) ok = epilogue(i - 1);
         }
         if (ok) epilogue(p.HG - 1);
-        (void)warp_tot;
     }
 
     tc_fence_before();
@@ -379,7 +390,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_output_tc_kernel(const __gr
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
 
+    const WaitCtx wc{abort_flag, p.status, 3};
     if (warp == 0) {
+        // TMA: the whole warp walks the heads, lane 0 issues
         if (lane == 0) {
             tma_prefetch_desc(&p.tmap_x);
             tma_prefetch_desc(&p.tmap_b);
@@ -394,11 +407,14 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_output_tc_kernel(const __gr
                     tma_load_2d(sbase + kOffBP + (uint32_t)pnl * KS * kRowBytes + (uint32_t)r * kBox, &p.tmap_b,
                                 bar(IN_FULL), 64 * pnl, row0 + 128 * r);
             }
-            for (int i = 0; i < p.HG; ++i) {
-                const int xs = i & 1;
-                const uint32_t ph = (uint32_t)(i >> 1) & 1u;
-                const int h = hg * p.HG + i;
-                if (!mbar_wait(bar(X_FREE0 + xs), ph ^ 1u, abort_flag, p.status)) break;
+        }
+        __syncwarp();
+        for (int i = 0; i < p.HG; ++i) {
+            const int xs = i & 1;
+            const uint32_t ph = (uint32_t)(i >> 1) & 1u;
+            const int h = hg * p.HG + i;
+            if (!mbar_wait_warp(bar(X_FREE0 + xs), ph ^ 1u, wc, 1)) break;
+            if (lane == 0) {
                 const uint32_t bytes = (uint32_t)KS * kRowBytes + (has_off ? kBox : 0u);
                 mbar_expect_tx(bar(X_FULL0 + xs), bytes);
                 for (int r = 0; r < KS / 128; ++r)
@@ -408,13 +424,15 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_output_tc_kernel(const __gr
                     tma_load_2d(sbase + kOffHp + (uint32_t)xs * kBox, &p.tmap_hin, bar(X_FULL0 + xs), 0,
                                 ((b * p.H + h) * p.C + c) * kN);
             }
+            __syncwarp();
         }
     } else if (warp == 1) {
-        if (lane == 0) {
-            bool ok = mbar_wait(bar(IN_FULL), 0, abort_flag, p.status);
-            if (ok) {
-                // G[t, s] = sum_n C[t, n] B[s, n]: both K-major, K = N.
-                tc_fence_after();
+        // MMA: lane 0 issues, the whole warp walks the heads
+        bool ok = mbar_wait_warp(bar(IN_FULL), 0, wc, 2);
+        if (ok) {
+            // G[t, s] = sum_n C[t, n] B[s, n]: both K-major, K = N.
+            tc_fence_after();
+            if (lane == 0) {
                 const uint32_t idesc_g = idesc_bf16_f32(128, KS, false, false);
 #pragma unroll
                 for (int kk = 0; kk < kN / 16; ++kk) {
@@ -426,18 +444,21 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_output_tc_kernel(const __gr
                 }
                 mma_commit(bar(G_FULL));
             }
-            const uint32_t idesc_y = idesc_bf16_f32(128, kP, false, true);
-            for (int i = 0; i < p.HG && ok; ++i) {
-                const int xs = i & 1, a = i & 1;
-                const uint32_t ph = (uint32_t)(i >> 1) & 1u;
-                if (!mbar_wait(bar(READY), (uint32_t)i & 1u, abort_flag, p.status)) break;
-                if (!mbar_wait(bar(ACC_EMPTY0 + a), ph ^ 1u, abort_flag, p.status)) break;
-                tc_fence_after();
+            __syncwarp();
+        }
+        const uint32_t idesc_y = idesc_bf16_f32(128, kP, false, true);
+        for (int i = 0; i < p.HG && ok; ++i) {
+            const int xs = i & 1, a = i & 1;
+            const uint32_t ph = (uint32_t)(i >> 1) & 1u;
+            if (!(ok = mbar_wait_warp(bar(READY), (uint32_t)i & 1u, wc, 3))) break;
+            if (!(ok = mbar_wait_warp(bar(ACC_EMPTY0 + a), ph ^ 1u, wc, 4))) break;
+            tc_fence_after();
+            if (lane == 0) {
                 // Y_diag = P (dt o x): A = P (K-major, K = s), B = x (MN-major)
                 const uint32_t xbase = sbase + kOffX + (uint32_t)xs * kXBytes;
                 for (int kk = 0; kk < KS / 16; ++kk) {
-                    const uint64_t ad = smem_desc_sw128(sbase + kOffBP + (uint32_t)(kk >> 2) * kBox + (uint32_t)(kk & 3) * 32,
-                                                        16, 1024);
+                    const uint64_t ad = smem_desc_sw128(
+                        sbase + kOffBP + (uint32_t)(kk >> 2) * kBox + (uint32_t)(kk & 3) * 32, 16, 1024);
                     const uint64_t bd = smem_desc_sw128(xbase + (uint32_t)kk * 2048, 8192, 1024);
                     mma_f16_ss(tmem + kColDiag + (uint32_t)a * 64, ad, bd, idesc_y, kk > 0 ? 1u : 0u);
                 }
@@ -456,6 +477,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_output_tc_kernel(const __gr
                 mma_commit(bar(X_FREE0 + xs));
                 mma_commit(bar(P_FREE));
             }
+            __syncwarp();
         }
     } else {
         // ---------------------------------------------------------- workers
@@ -472,7 +494,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_output_tc_kernel(const __gr
         auto epilogue = [&](int i, float row_scale) -> bool {
             const int a = i & 1;
             const uint32_t ph = (uint32_t)(i >> 1) & 1u;
-            if (!mbar_wait_warp(bar(ACC_FULL0 + a), ph, abort_flag, p.status)) return false;
+            if (!mbar_wait_warp(bar(ACC_FULL0 + a), ph, wc, 8)) return false;
             tc_fence_after();
             float yd[32], yo[32];
             tmem_ld_32x32b_x32(t_lane + kColDiag + (uint32_t)a * 64 + (uint32_t)colhalf * 32, yd);
@@ -496,8 +518,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_output_tc_kernel(const __gr
             }
             return true;
         };
+        // Every worker warp executes the same named barriers for every head,
+        // also after a failed wait (it then skips the work).
         bool ok = true;
-        for (int i = 0; i < p.HG && ok; ++i) {
+        for (int i = 0; i < p.HG; ++i) {
             const int h = hg * p.HG + i;
             const float Ah = p.A[h] * kLog2e;
             if (i > 0) named_bar_sync(1, kWorkers);      // a2 / colf / dts of the previous head consumed
@@ -520,7 +544,11 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_output_tc_kernel(const __gr
             // scale x rows by dt in place
             const int xs = i & 1;
             const uint32_t ph = (uint32_t)(i >> 1) & 1u;
-            if (!mbar_wait_warp(bar(X_FULL0 + xs), ph, abort_flag, p.status)) { ok = false; break; }
+            if (ok) ok = mbar_wait_warp(bar(X_FULL0 + xs), ph, wc, 5);
+            // P may be written once G (first head) or the previous head's MMA has consumed the buffer
+            if (ok) ok = (i == 0) ? mbar_wait_warp(bar(G_FULL), 0, wc, 6)
+                                  : mbar_wait_warp(bar(P_FREE), (uint32_t)(i - 1) & 1u, wc, 7);
+            if (!ok) continue;
             uint8_t* xb = smem + kOffX + (uint32_t)xs * kXBytes;
             for (int k = wi; k < KS * 8; k += kWorkers) {
                 uint4* ptr = reinterpret_cast<uint4*>(xb + (size_t)k * 16);
@@ -530,12 +558,6 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_output_tc_kernel(const __gr
 #pragma unroll
                 for (int j = 0; j < 8; ++j) f[j] *= ds;
                 Vec16<__nv_bfloat16>::store(reinterpret_cast<__nv_bfloat16*>(ptr), f);
-            }
-            // P may be written once G (first head) or the previous head's MMA has consumed the buffer
-            if (i == 0) {
-                if (!mbar_wait_warp(bar(G_FULL), 0, abort_flag, p.status)) { ok = false; break; }
-            } else {
-                if (!mbar_wait_warp(bar(P_FREE), (uint32_t)(i - 1) & 1u, abort_flag, p.status)) { ok = false; break; }
             }
             tc_fence_after();
             // P[t, s] = G[t, s] * exp(Acum_t - Acum_r) * exp(Acum_r - Acum_s), s <= t
@@ -576,7 +598,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_output_tc_kernel(const __gr
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(READY));
-            if (i > 0 && !epilogue(i - 1, row_scale_prev)) { ok = false; break; }
+            if (i > 0) ok = epilogue(i - 1, row_scale_prev);
             row_scale_prev = row_scale;
         }
         if (ok) epilogue(p.HG - 1, row_scale_prev);
