@@ -327,8 +327,12 @@ __global__ void __launch_bounds__(256) state_pass_tc_kernel(const __grid_constan
 namespace co {
 constexpr int kWorkers = 256;
 constexpr int kThreads = 64 + kWorkers;  // warp 0 TMA, warp 1 MMA, warps 2-9 workers
-enum Bar { IN_FULL = 0, G_FULL, X_FULL0, X_FREE0 = X_FULL0 + 2, READY, P_FREE, ACC_FULL0, ACC_EMPTY0 = ACC_FULL0 + 2,
-           NUM_BARS = ACC_EMPTY0 + 2 };
+// Barrier slots; the two-deep rings take two consecutive slots each.
+enum Bar { IN_FULL = 0, G_FULL = 1, X_FULL0 = 2, X_FREE0 = 4, READY = 6, P_FREE = 7, ACC_FULL0 = 8,
+           ACC_EMPTY0 = 10, NUM_BARS = 12 };
+static_assert(X_FREE0 >= X_FULL0 + 2 && READY >= X_FREE0 + 2 && ACC_EMPTY0 >= ACC_FULL0 + 2 &&
+                  NUM_BARS >= ACC_EMPTY0 + 2 && P_FREE != READY && ACC_FULL0 > P_FREE,
+              "barrier slots overlap");
 constexpr uint32_t kOffC = 0;                          // C rows: 2 panels x 128 rows (32 KB)
 constexpr uint32_t kOffBP = 2 * kBox;                  // B rows (2 panels x KS rows), later P (KS/64 panels x 128 rows)
 constexpr uint32_t kOffX = kOffBP + 4 * kBox;          // 2 buffers x (256 rows x 128 B)

@@ -70,6 +70,14 @@ def test_bf16_ragged_chunks_several_tiles(orc):
     check_full(orc, shape, synth.layer_inputs(shape, seed=1), TOL[torch.bfloat16])
 
 
+def test_bf16_many_heads_per_group(orc):
+    """16 and 32 heads: the scan kernels walk many heads per CTA, so every
+    double-buffered stage is reused several times; every head is compared."""
+    for H, seed in ((16, 41), (32, 42)):
+        shape = LayerShape(1, 3 * 256, H, 64, 128, 256, "bf16", "loguniform")
+        check_full(orc, shape, synth.layer_inputs(shape, seed=seed), TOL[torch.bfloat16])
+
+
 def test_bf16_two_batches_S128(orc):
     shape = LayerShape(2, 5 * 128, 2, 64, 128, 128, "bf16", "loguniform")
     check_full(orc, shape, synth.layer_inputs(shape, seed=2), TOL[torch.bfloat16])
