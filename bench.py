@@ -59,6 +59,8 @@ def parse():
     p.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end region")
     p.add_argument("--no-cpu-baseline", action="store_true", help="skip timing the oracle")
     p.add_argument("--decode-steps", type=int, default=DEC.nsteps)
+    p.add_argument("--reference-heads", type=int, default=0,
+                   help="heads per reference-arm step (default: one per host core, at most 32)")
     return p.parse_args()
 
 
@@ -400,14 +402,17 @@ def cpu_baseline(inp):
                       f"({FWD.seqlen} x {nh}/{FWD.nheads})"}
 
 
-def run_reference(args, dist):
+def run_reference(args):
     """The reference arm: the fp64 oracle on this host's cores, one bounded
-    sample of the forward workload per step."""
-    if dist.rank != 0:
+    sample of the forward workload per step.  CPU only; under torchrun rank
+    0 alone runs it and the other ranks exit without work (no process group
+    is created)."""
+    if int(os.environ.get("RANK", "0")) != 0:
         return
     inp = synth.layer_inputs(FWD, seed=0)
     nthreads = cores()
-    heads = list(range(min(FWD.nheads, nthreads)))
+    nh = args.reference_heads if args.reference_heads > 0 else nthreads
+    heads = list(range(min(FWD.nheads, nh)))
     for _ in range(args.warmup):
         oracle_sample(inp, heads, nthreads)
     secs = []
@@ -434,11 +439,11 @@ def run_reference(args, dist):
 # ---------------------------------------------------------------------------
 def main():
     args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+        return
     dist = Dist()
     try:
-        if args.impl == "reference":
-            run_reference(args, dist)
-            return
         from mamba_ssd_state_b200 import build as dart_build
         from mamba_ssd_state_b200 import dart
 
