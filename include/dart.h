@@ -158,6 +158,36 @@ dart_status dart_decode_step(const dart_dims* dims, dart_dtype dtype,
                              void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * dart_decode_step for callers that cannot allocate device memory.  The
+ * paper has no counterpart: this is an interface for embedding the decode
+ * step where cudaMalloc is not available to the caller -- for example a host
+ * runtime that owns all device memory and hands out only preallocated
+ * tensors, or a serving loop that must not call into the allocator (which
+ * may synchronise the device) between steps.
+ *
+ * Same arguments, computation and device-side error behaviour as
+ * dart_decode_step, without the workspace: the per-(sequence, head, split)
+ * partial results live in a 16 MiB array that the library keeps in static
+ * device memory, one per device that loads the library, held until the
+ * process exits.  The caller still passes every input and output.
+ *   - Limit: dart_decode_step_workspace_bytes(dims, dtype, cmax) must be at
+ *     most 16 MiB (16777216 bytes); larger batches are rejected with
+ *     DART_ERR_UNSUPPORTED and a message giving both sizes.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture.
+ *   - Every call shares the one array: calls that overlap on the GPU (on
+ *     different streams, or from several threads without ordering) race.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ */
+dart_status dart_decode_step_noalloc(const dart_dims* dims, dart_dtype dtype,
+                                     const void* x_t, const float* dt_t, const float* A,
+                                     const void* B_t, const void* C_t, const void* Q_t,
+                                     const void* E_t, float g, float* state, float* dH_cur,
+                                     void* dH_cache, int cmax, int* n_chunks, int* pos, float* y,
+                                     void* stream);
+
+/*
  * 1 when (dstate N, headdim P, chunk S, dtype) is compiled in, else 0.
  */
 int dart_supported(int dstate, int headdim, int chunk, dart_dtype dtype);

@@ -196,6 +196,44 @@ dart_status dart_decode_step(const dart_dims* d, dart_dtype dtype, const void* x
     return DART_OK;
 }
 
+// The decode step for callers that cannot allocate device memory: the split
+// partials go to the library's fixed static scratch (decode.cu) instead of a
+// caller workspace.  Validation matches dart_decode_step, plus the scratch
+// size limit; no allocation of any kind happens here.
+dart_status dart_decode_step_noalloc(const dart_dims* d, dart_dtype dtype, const void* x_t, const float* dt_t,
+                                     const float* A, const void* B_t, const void* C_t, const void* Q_t,
+                                     const void* E_t, float g, float* state, float* dH_cur, void* dH_cache,
+                                     int cmax, int* n_chunks, int* pos, float* y, void* stream) {
+    t_err[0] = 0;
+    dart_status st = check_common(d, dtype, false);
+    if (st != DART_OK) return st;
+    if (!dart::decode_supported(d->dstate, d->headdim, d->chunk, dtype))
+        return fail(DART_ERR_UNSUPPORTED, "dart_decode_step_noalloc: (N=%d, P=%d) not compiled", d->dstate,
+                    d->headdim);
+    if (cmax < 1) return fail(DART_ERR_INVALID_ARG, "cmax must be >= 1");
+    DART_REQUIRE_PTR(x_t); DART_REQUIRE_PTR(dt_t); DART_REQUIRE_PTR(A); DART_REQUIRE_PTR(B_t);
+    DART_REQUIRE_PTR(C_t); DART_REQUIRE_PTR(Q_t); DART_REQUIRE_PTR(E_t); DART_REQUIRE_PTR(state);
+    DART_REQUIRE_PTR(dH_cur); DART_REQUIRE_PTR(dH_cache); DART_REQUIRE_PTR(n_chunks);
+    DART_REQUIRE_PTR(pos); DART_REQUIRE_PTR(y);
+    const size_t need = dart_decode_step_workspace_bytes(d, dtype, cmax);
+    if (need > dart::kNoAllocScratchBytes)
+        return fail(DART_ERR_UNSUPPORTED,
+                    "dart_decode_step_noalloc: this batch needs %zu bytes of scratch, more than the fixed %zu; "
+                    "use dart_decode_step with a workspace or fewer sequences / a smaller cmax",
+                    need, dart::kNoAllocScratchBytes);
+    void* scratch = nullptr;
+    cudaError_t e = dart::noalloc_scratch(&scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "dart_decode_step_noalloc: static scratch address");
+    dart::DecodeArgs a{d->batch, d->nheads, d->headdim, d->dstate, d->chunk, cmax,
+                       dart::decode_num_splits(d->batch, d->nheads, cmax),
+                       x_t, dt_t, A, B_t, C_t, Q_t, E_t, g, state, dH_cur, dH_cache,
+                       n_chunks, pos, y, static_cast<float*>(scratch), status_word()};
+    if (!a.status) return fail(DART_ERR_CUDA, "dart_decode_step_noalloc: no device status word");
+    e = dart::launch_decode(a, dtype, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "dart_decode_step_noalloc launch");
+    return DART_OK;
+}
+
 dart_status dart_sync_status(void* stream) {
     t_err[0] = 0;
     cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));

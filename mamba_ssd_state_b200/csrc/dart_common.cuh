@@ -137,4 +137,9 @@ cudaError_t launch_sma_tc(const SmaArgs& a, cudaStream_t st);
 const char* sma_impl_name(int N, int P, int S, dart_dtype dt);
 bool decode_supported(int N, int P, int S, dart_dtype dt);
 int decode_num_splits(int B, int H, int cmax);
+
+// dart_decode_step_noalloc: size of the library-owned static scratch, and its
+// device address on the current device (set up on the first call per device).
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;
+cudaError_t noalloc_scratch(void** out);
 }  // namespace dart

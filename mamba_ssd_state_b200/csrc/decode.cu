@@ -265,4 +265,37 @@ cudaError_t launch_decode(const DecodeArgs& a, dart_dtype dt, cudaStream_t st) {
     return cudaErrorInvalidValue;
 }
 
+// ---------------------------------------------------------------------------
+// Fixed scratch for dart_decode_step_noalloc.
+//
+// Callers that cannot allocate device memory get the decode step's split
+// partials in this file-scope array instead of a workspace they pass in.  It
+// exists once per device that loads the library and lives until the process
+// exits.  Every call shares it and it keeps the last call's contents; the
+// decode kernels write every slot they later read, so nothing needs clearing.
+// Calls that overlap on the GPU (different streams, or different threads
+// without ordering) race on it.
+//
+// On the host `g_noalloc_scratch` names a host-side stand-in, not the device
+// array, so kernels are given the address cudaGetSymbolAddress reports for
+// the current device.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+cudaError_t noalloc_scratch(void** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    static void* cache[64] = {};  // looked up once per device; a racing lookup only repeats it
+    if (!cache[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        cache[dev] = p;
+    }
+    *out = cache[dev];
+    return cudaSuccess;
+}
+
 }  // namespace dart

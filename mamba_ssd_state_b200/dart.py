@@ -31,7 +31,7 @@ _STATUS = {0: "DART_OK", 1: "DART_ERR_INVALID_ARG", 2: "DART_ERR_UNSUPPORTED", 3
 EXPORTS = ("dart_ssd_chunk_scan_workspace_bytes", "dart_ssd_chunk_scan", "dart_sma_forward",
            "dart_decode_step_workspace_bytes", "dart_decode_step", "dart_supported",
            "dart_sync_status", "dart_last_error", "dart_abi_version", "dart_launch_count",
-           "dart_sma_impl")
+           "dart_sma_impl", "dart_decode_step_noalloc")
 
 
 class DartError(RuntimeError):
@@ -81,6 +81,9 @@ def load(path: str = LIBRARY) -> ctypes.CDLL:
     lib.dart_launch_count.argtypes = []
     lib.dart_sma_impl.restype = ctypes.c_char_p
     lib.dart_sma_impl.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int]
+    lib.dart_decode_step_noalloc.restype = ctypes.c_int
+    lib.dart_decode_step_noalloc.argtypes = ([D, ctypes.c_int] + [_P] * 7 + [ctypes.c_float] + [_P] * 3
+                                             + [ctypes.c_int] + [_P] * 4)
     _lib = lib
     return lib
 
@@ -277,6 +280,35 @@ def dart_decode_step(x, dt, A, Bm, Cm, Q, E, g: float, state, dH_cur, cache, nch
                                     cmax, _ptr(nchunks), _ptr(pos), _ptr(y), _ptr(workspace),
                                     workspace.numel(), _stream()))
     return y.cpu() if host else y
+
+
+def dart_decode_step_noalloc(x, dt, A, Bm, Cm, Q, E, g: float, state, dH_cur, cache, nchunks, pos,
+                             chunk: int, *, y=None):
+    """dart_decode_step for callers that cannot allocate device memory: the
+    library keeps the step's scratch in a fixed 16 MiB static device array
+    instead of a caller workspace (see include/dart.h for its limits).  All
+    tensors must already be on the device; `y` may be preallocated so that the
+    call allocates nothing at all.  Calls overlapping on the GPU race on the
+    shared scratch."""
+    lib = load()
+    for name, t in (("x", x), ("dt", dt), ("A", A), ("Bm", Bm), ("Cm", Cm), ("Q", Q), ("E", E),
+                    ("state", state), ("dH_cur", dH_cur), ("cache", cache), ("nchunks", nchunks), ("pos", pos)):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    Bs, H, P = x.shape
+    N = Bm.shape[-1]
+    cmax = cache.shape[2]
+    _shape("state", state, (Bs, H, N, P)); _shape("dH_cur", dH_cur, (Bs, H, N, P))
+    _shape("cache", cache, (Bs, H, cmax, N, P))
+    if y is None:
+        y = torch.empty((Bs, H, P), device=cache.device, dtype=torch.float32)
+    dims = Dims(Bs, 0, H, P, N, chunk, 1)
+    with torch.cuda.device(cache.device):
+        _check(lib.dart_decode_step_noalloc(ctypes.byref(dims), _dtype_code(cache.dtype), _ptr(x), _ptr(dt),
+                                            _ptr(A), _ptr(Bm), _ptr(Cm), _ptr(Q), _ptr(E), float(g), _ptr(state),
+                                            _ptr(dH_cur), _ptr(cache), cmax, _ptr(nchunks), _ptr(pos), _ptr(y),
+                                            _stream()))
+    return y
 
 
 def decode_workspace_bytes(nseq, nheads, headdim, dstate, chunk, cmax, dtype) -> int:
