@@ -64,6 +64,30 @@ def parse():
     return p.parse_args()
 
 
+def captured_traffic(kernel: str):
+    """DRAM bytes per launch of `kernel` from profiles/traffic.txt, or None if
+    absent or if its source files changed since the capture."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(path):
+        return None
+    for line in open(path):
+        if line.startswith("#") or "|" not in line:
+            continue
+        name, files, sha, nbytes = [f.strip() for f in line.split("|")[:4]]
+        if name != kernel:
+            continue
+        m = hashlib.sha256()
+        try:
+            for f in files.split(","):
+                with open(os.path.join(ROOT, f), "rb") as fh:
+                    m.update(fh.read())
+        except OSError:
+            return None
+        return float(nbytes) if m.hexdigest()[:16] == sha else None
+    return None
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -351,7 +375,7 @@ def decode_region(args, dist, dart, peaks):
                    "cached_chunks": DEC.ncached, "context": DEC.ncached * DEC.chunk,
                    "l2": "cache 4.3 GB per step >> 126 MB L2"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": captured_traffic("decode_step"),
                      "kernel": "dart_decode_step (decode_partial + decode_combine + decode_advance)",
                      "bytes_per_step": bytes_step},
     }
@@ -472,7 +496,8 @@ def main():
             roof = {"bound": "alu", "achieved": sma_tflops, "peak": alu_peak, "unit": "TFLOP/s",
                     "frac": sma_tflops / alu_peak}
             peak_note = "fp32 FMA peak: 148 SMs x 128 lanes x 2 flop x sm_max_mhz"
-        roof.update({"traffic": None, "kernel": impl, "flop_per_launch": f_sma, "peak_source": peak_note})
+        roof.update({"traffic": captured_traffic(impl), "traffic_unit": "bytes per launch", "kernel": impl,
+                     "flop_per_launch": f_sma, "peak_source": peak_note})
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": dist.world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
