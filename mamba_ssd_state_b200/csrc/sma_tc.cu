@@ -18,13 +18,18 @@
 // Each batch of 4 memories costs two M=128, N=256, K=128 MMAs.  The epilogue
 // warps read U as soon as it lands (scores, online softmax) and hand the U
 // columns back while the V MMA runs, then read V (value accumulation) while
-// the next batch's U MMA runs, so the tensor pipe never waits for them.
+// the next batch's U MMA runs.
 //
-// Roles (192 threads): warp 0 issues TMA, warp 1 allocates TMEM and issues
-// tcgen05.mma, warps 2-5 (one per TMEM lane quadrant) run the softmax and
-// write the output.  The grid is persistent: CTA i takes tiles i, i+G, ...
-// of a list ordered from the most memories to the fewest, so the triangular
-// work spreads evenly.
+// Roles (320 threads): warp 0 issues TMA, warp 1 allocates TMEM and issues
+// tcgen05.mma, warps 2-9 run the epilogue as four pairs, one pair per TMEM
+// lane quadrant (32 token rows); the two warps of a pair split the 64 value
+// columns, exchange partial scores through shared memory, run the same
+// online softmax and each write their half of the output row.  Splitting
+// the columns halves the epilogue's time per batch, which is what keeps the
+// MMA fed.  The grid is persistent: CTA i takes tiles i, i+G, ... of a list
+// ordered from the most memories to the fewest, so the triangular work
+// spreads evenly; each tile prefetches the next tile's E and y_ssd rows into
+// L2.
 #include <cuda_bf16.h>
 #include <string.h>
 
@@ -48,13 +53,19 @@ constexpr uint32_t kOffC = 2 * kHalfA;
 constexpr uint32_t kOffB = 4 * kHalfA;
 constexpr uint32_t kStageBytes = kCB * kMemBytes;
 constexpr uint32_t kOffBar = kOffB + kNB * kStageBytes;
-constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;  // + barriers, + alignment slack
-constexpr int kThreads = 192;
+constexpr uint32_t kOffX = kOffBar + 256;            // partial-score exchange: [2 parity][2 half][128 rows][4]
+constexpr uint32_t kSmemBytes = kOffX + 2 * 2 * 128 * 4 * 4 + 1024;  // + alignment slack
+constexpr int kEpiWarps = 8;                          // four pairs, one pair per TMEM lane quadrant
+constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColV = 256;
+constexpr int kHalfP = kP / 2;                        // value columns per epilogue warp
 
-enum Bar { Q_FULL = 0, Q_FREE, C_FULL, C_FREE, U_FULL, U_EMPTY, V_FULL, V_EMPTY, B_FULL0, B_EMPTY0 = B_FULL0 + kNB,
-           NUM_BARS = B_EMPTY0 + kNB };
+// Barrier slots (explicit; the memory ring takes consecutive slots).
+enum Bar { Q_FULL = 0, Q_FREE = 1, C_FULL = 2, C_FREE = 3, U_FULL = 4, U_EMPTY = 5, V_FULL = 6, V_EMPTY = 7,
+           B_FULL0 = 8, B_EMPTY0 = B_FULL0 + kNB, NUM_BARS = B_EMPTY0 + kNB };
+static_assert(NUM_BARS * 8 + 8 <= 256, "barrier block");
+static_assert(kOffX % 16 == 0 && kSmemBytes <= 232448, "shared memory layout");
 
 struct SmaTcParams {
     CUtensorMap tmap_q;  // Q viewed as dims (N, B*L, H)
@@ -87,16 +98,6 @@ __device__ __forceinline__ Tile decode_tile(const SmaTcParams& p, int i) {
     return t;
 }
 
-__device__ __forceinline__ void load_row_bf16(const __nv_bfloat16* src, float* dst) {
-#pragma unroll
-    for (int i = 0; i < kP / 8; ++i) {
-        float tmp[8];
-        Vec16<__nv_bfloat16>::load(src + 8 * i, tmp);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) dst[8 * i + j] = tmp[j];
-    }
-}
-
 __global__ void __launch_bounds__(kThreads, 1) sma_tc_kernel(const __grid_constant__ SmaTcParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -112,9 +113,9 @@ __global__ void __launch_bounds__(kThreads, 1) sma_tc_kernel(const __grid_consta
         mbar_init(bar(C_FULL), 1);
         mbar_init(bar(C_FREE), 1);
         mbar_init(bar(U_FULL), 1);
-        mbar_init(bar(U_EMPTY), 4);
+        mbar_init(bar(U_EMPTY), kEpiWarps);
         mbar_init(bar(V_FULL), 1);
-        mbar_init(bar(V_EMPTY), 4);
+        mbar_init(bar(V_EMPTY), kEpiWarps);
         for (int s = 0; s < kNB; ++s) {
             mbar_init(bar(B_FULL0 + s), 1);
             mbar_init(bar(B_EMPTY0 + s), 1);
@@ -232,52 +233,101 @@ __global__ void __launch_bounds__(kThreads, 1) sma_tc_kernel(const __grid_consta
         }
     } else {
         // ------------------------------------------------------- epilogue
-        const int quad = warp & 3;                 // TMEM lane quadrant of this warp
+        // Warp pair (w, w+4) shares TMEM lane quadrant w & 3 (32 token rows);
+        // warp half h owns value columns [32h, 32h+32) of every memory.  Both
+        // warps of a pair run the same batches and the same named barrier
+        // per batch, also after a failed wait (they then skip the work).
+        const int quad = warp & 3;
+        const int half = (warp - 2) >> 2;
+        const int col0 = half * kHalfP;
         const int row = quad * 32 + lane;          // token row inside the tile
         const uint32_t t_lane = tmem + ((uint32_t)(quad * 32) << 16);
         const float sscale = kLog2e * rsqrtf((float)kN);
+        float* xbuf = reinterpret_cast<float*>(smem + kOffX);
         int it_u = 0;
+        bool ok = true;
+        auto row_offset = [&](const Tile& t) -> size_t {
+            const size_t tok = (size_t)t.b * p.L + t.t0 + row;
+            return (tok * p.H + t.h) * kP + col0;
+        };
+        // This warp's 32 columns of E for the tile about to run, as packed
+        // bf16; the next tile's are fetched together with the y_ssd rows at
+        // the end of each tile, so that neither latency sits between tiles.
+        uint4 e_raw[kHalfP / 8];
+        auto load_e = [&](int i) {
+#pragma unroll
+            for (int q = 0; q < kHalfP / 8; ++q) e_raw[q] = make_uint4(0u, 0u, 0u, 0u);
+            if (i >= p.total_tiles) return;
+            const Tile t = decode_tile(p, i);
+            if (t.k == 0) return;
+            const uint4* src = reinterpret_cast<const uint4*>(p.E + row_offset(t));
+#pragma unroll
+            for (int q = 0; q < kHalfP / 8; ++q) e_raw[q] = __ldg(src + q);
+        };
+        load_e(blockIdx.x);
         for (int i = blockIdx.x; i < p.total_tiles; i += gridDim.x) {
             const Tile t = decode_tile(p, i);
-            const size_t tok = (size_t)t.b * p.L + t.t0 + row;
-            float* orow = p.out + (tok * p.H + t.h) * kP;
-            const float* yrow = p.y_ssd ? p.y_ssd + (tok * p.H + t.h) * kP : nullptr;
-            float o[kP];
+            const size_t rowoff = row_offset(t);
+            if (i + (int)gridDim.x < p.total_tiles) {  // next tile's rows, on their way to L2
+                const size_t offn = row_offset(decode_tile(p, i + gridDim.x));
+                prefetch_l2(p.E + offn);
+                if (p.y_ssd) prefetch_l2(p.y_ssd + offn);
+            }
+            float2 o2[kHalfP / 2];
 #pragma unroll
-            for (int j = 0; j < kP; ++j) o[j] = 0.f;
+            for (int j = 0; j < kHalfP / 2; ++j) o2[j] = make_float2(0.f, 0.f);
             float l = 0.f;
-            bool ok = true;
             if (t.k > 0) {
-                float e[kP];
-                load_row_bf16(p.E + (tok * p.H + t.h) * kP, e);
+                // E widened to fp32 once per tile (bf16 -> fp32 is a shift)
+                float2 e2[kHalfP / 2];
+                {
+#pragma unroll
+                    for (int q = 0; q < kHalfP / 8; ++q) {
+                        const uint4 v4 = e_raw[q];
+                        const uint32_t w4[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+                        for (int r = 0; r < 4; ++r)
+                            e2[4 * q + r] = make_float2(__uint_as_float(w4[r] << 16), __uint_as_float(w4[r] & 0xffff0000u));
+                    }
+                }
                 float m = -INFINITY;
                 const int nbatch = (t.k + kCB - 1) / kCB;
                 for (int j = 0; j < nbatch; ++j, ++it_u) {
                     const int nv = min(kCB, t.k - kCB * j);
                     const uint32_t ph = (uint32_t)it_u & 1u;
-                    if (!mbar_wait_warp(bar(U_FULL), ph, wc, 9)) { ok = false; break; }
-                    tc_fence_after();
+                    float part[kCB] = {0.f, 0.f, 0.f, 0.f};
+                    if (ok) ok = mbar_wait_warp(bar(U_FULL), ph, wc, 9);
+                    if (ok) {
+                        tc_fence_after();
+#pragma unroll
+                        for (int c = 0; c < kCB; ++c) {
+                            if (c < nv) {
+                                float u[kHalfP];
+                                tmem_ld_32x32b_x32(t_lane + (uint32_t)(c * kP + col0), u);
+                                tmem_ld_wait();
+                                float2 a0 = make_float2(0.f, 0.f), a1 = a0;
+#pragma unroll
+                                for (int q = 0; q < kHalfP / 2; q += 2) {
+                                    a0 = __ffma2_rn(make_float2(u[2 * q], u[2 * q + 1]), e2[q], a0);
+                                    a1 = __ffma2_rn(make_float2(u[2 * q + 2], u[2 * q + 3]), e2[q + 1], a1);
+                                }
+                                part[c] = (a0.x + a1.x) + (a0.y + a1.y);
+                            }
+                        }
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(bar(U_EMPTY));
+                    }
+                    // scores: own partial + partner's partial
+                    float* xs = xbuf + (((it_u & 1) * 2 + half) * 128 + row) * 4;
+                    const float* xp = xbuf + (((it_u & 1) * 2 + (1 - half)) * 128 + row) * 4;
+                    *reinterpret_cast<float4*>(xs) = make_float4(part[0], part[1], part[2], part[3]);
+                    named_bar_sync(2 + quad, 64);
+                    const float4 pp = *reinterpret_cast<const float4*>(xp);
+                    const float other[kCB] = {pp.x, pp.y, pp.z, pp.w};
                     float sc[kCB];
 #pragma unroll
-                    for (int c = 0; c < kCB; ++c) {
-                        sc[c] = -INFINITY;
-                        if (c < nv) {
-                            float u[kP];
-                            tmem_ld_32x32b_x32(t_lane + (uint32_t)(c * kP), u);
-                            tmem_ld_32x32b_x32(t_lane + (uint32_t)(c * kP + 32), u + 32);
-                            tmem_ld_wait();
-                            float acc0 = 0.f, acc1 = 0.f;
-#pragma unroll
-                            for (int q = 0; q < kP; q += 2) {
-                                acc0 = fmaf(u[q], e[q], acc0);
-                                acc1 = fmaf(u[q + 1], e[q + 1], acc1);
-                            }
-                            sc[c] = (acc0 + acc1) * sscale;
-                        }
-                    }
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(bar(U_EMPTY));
+                    for (int c = 0; c < kCB; ++c) sc[c] = c < nv ? (part[c] + other[c]) * sscale : -INFINITY;
                     float mnew = m;
 #pragma unroll
                     for (int c = 0; c < kCB; ++c) mnew = fmaxf(mnew, sc[c]);
@@ -287,37 +337,48 @@ __global__ void __launch_bounds__(kThreads, 1) sma_tc_kernel(const __grid_consta
                     for (int c = 0; c < kCB; ++c) w[c] = c < nv ? exp2f(sc[c] - mnew) : 0.f;
                     l = l * alpha + (w[0] + w[1]) + (w[2] + w[3]);
                     m = mnew;
+                    const float2 alpha2 = make_float2(alpha, alpha);
 #pragma unroll
-                    for (int q = 0; q < kP; ++q) o[q] *= alpha;
-                    if (!mbar_wait_warp(bar(V_FULL), ph, wc, 10)) { ok = false; break; }
-                    tc_fence_after();
+                    for (int q = 0; q < kHalfP / 2; ++q) o2[q] = __fmul2_rn(o2[q], alpha2);
+                    if (ok) ok = mbar_wait_warp(bar(V_FULL), ph, wc, 10);
+                    if (ok) {
+                        tc_fence_after();
 #pragma unroll
-                    for (int c = 0; c < kCB; ++c) {
-                        if (c < nv) {
-                            float v[kP];
-                            tmem_ld_32x32b_x32(t_lane + kColV + (uint32_t)(c * kP), v);
-                            tmem_ld_32x32b_x32(t_lane + kColV + (uint32_t)(c * kP + 32), v + 32);
-                            tmem_ld_wait();
+                        for (int c = 0; c < kCB; ++c) {
+                            if (c < nv) {
+                                float v[kHalfP];
+                                tmem_ld_32x32b_x32(t_lane + kColV + (uint32_t)(c * kP + col0), v);
+                                tmem_ld_wait();
+                                const float2 w2 = make_float2(w[c], w[c]);
 #pragma unroll
-                            for (int q = 0; q < kP; ++q) o[q] = fmaf(w[c], v[q], o[q]);
+                                for (int q = 0; q < kHalfP / 2; ++q)
+                                    o2[q] = __ffma2_rn(w2, make_float2(v[2 * q], v[2 * q + 1]), o2[q]);
+                            }
                         }
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(bar(V_EMPTY));
                     }
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(bar(V_EMPTY));
                 }
             }
-            if (!ok) break;
-            const float inv = t.k > 0 ? 1.f / l : 0.f;
+            const float inv = t.k > 0 && l > 0.f ? 1.f / l : 0.f;
+            float* orow = p.out + rowoff;
+            const float* yrow = p.y_ssd ? p.y_ssd + rowoff : nullptr;
+            // All loads (this tile's y_ssd row, the next tile's E) are issued
+            // before the first store: out may alias y_ssd, so loads placed
+            // after a store would each wait a full memory round trip.
+            float4 yv[kHalfP / 4];
 #pragma unroll
-            for (int q = 0; q < kP; q += 4) {
-                float4 r = make_float4(o[q] * inv, o[q + 1] * inv, o[q + 2] * inv, o[q + 3] * inv);
-                if (yrow) {
-                    const float4 yv = *reinterpret_cast<const float4*>(yrow + q);
-                    r = make_float4(fmaf(p.g, r.x, yv.x), fmaf(p.g, r.y, yv.y), fmaf(p.g, r.z, yv.z),
-                                    fmaf(p.g, r.w, yv.w));
-                }
-                *reinterpret_cast<float4*>(orow + q) = r;
+            for (int q = 0; q < kHalfP / 4; ++q)
+                yv[q] = yrow ? *reinterpret_cast<const float4*>(yrow + 4 * q) : make_float4(0.f, 0.f, 0.f, 0.f);
+            load_e(i + gridDim.x);
+            const float gg = yrow ? p.g : 1.f;
+#pragma unroll
+            for (int q = 0; q < kHalfP / 4; ++q) {
+                const float2 lo = o2[2 * q], hi = o2[2 * q + 1];
+                const float4 r = make_float4(fmaf(gg, lo.x * inv, yv[q].x), fmaf(gg, lo.y * inv, yv[q].y),
+                                             fmaf(gg, hi.x * inv, yv[q].z), fmaf(gg, hi.y * inv, yv[q].w));
+                if (ok) *reinterpret_cast<float4*>(orow + 4 * q) = r;
             }
         }
     }
