@@ -54,7 +54,9 @@ constexpr uint32_t kOffB = 4 * kHalfA;
 constexpr uint32_t kStageBytes = kCB * kMemBytes;
 constexpr uint32_t kOffBar = kOffB + kNB * kStageBytes;
 constexpr uint32_t kOffX = kOffBar + 256;            // partial-score exchange: [2 parity][2 half][128 rows][4]
-constexpr uint32_t kSmemBytes = kOffX + 2 * 2 * 128 * 4 * 4 + 1024;  // + alignment slack
+constexpr uint32_t kOffS = kOffX + 2 * 2 * 128 * 4 * 4;  // per-warp staging for coalesced row traffic
+constexpr uint32_t kStageWarp = 32 * 80;                  // 32 E rows of 64 B (+16 pad) or 16 out rows of 144 B
+constexpr uint32_t kSmemBytes = kOffS + 8 * kStageWarp + 1024;  // + alignment slack
 constexpr int kEpiWarps = 8;                          // four pairs, one pair per TMEM lane quadrant
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr uint32_t kTmemCols = 512;
@@ -65,7 +67,8 @@ constexpr int kHalfP = kP / 2;                        // value columns per epilo
 enum Bar { Q_FULL = 0, Q_FREE = 1, C_FULL = 2, C_FREE = 3, U_FULL = 4, U_EMPTY = 5, V_FULL = 6, V_EMPTY = 7,
            B_FULL0 = 8, B_EMPTY0 = B_FULL0 + kNB, NUM_BARS = B_EMPTY0 + kNB };
 static_assert(NUM_BARS * 8 + 8 <= 256, "barrier block");
-static_assert(kOffX % 16 == 0 && kSmemBytes <= 232448, "shared memory layout");
+static_assert(kOffX % 16 == 0 && kOffS % 16 == 0 && kSmemBytes <= 232448, "shared memory layout");
+static_assert(16 * 36 * 4 <= kStageWarp, "out staging fits the per-warp buffer");
 
 struct SmaTcParams {
     CUtensorMap tmap_q;  // Q viewed as dims (N, B*L, H)
@@ -144,10 +147,28 @@ __global__ void __launch_bounds__(kThreads, 1) sma_tc_kernel(const __grid_consta
         uint32_t q_ph = 0, c_ph = 0;
         int it_b = 0;
         bool ok = true;
+        auto load_b = [&](const Tile& t, int j) -> bool {
+            const int nv = min(kCB, t.k - kCB * j);
+            const int s = it_b % kNB;
+            const uint32_t ph = (uint32_t)(it_b / kNB) & 1u;
+            if (!mbar_wait_warp(bar(B_EMPTY0 + s), ph ^ 1, wc, 3)) return false;
+            if (lane == 0) {
+                mbar_expect_tx(bar(B_FULL0 + s), (uint32_t)nv * kMemBytes);
+                const int mem_row = ((t.b * p.H + t.h) * p.C + kCB * j) * kN;
+                for (int q = 0; q < nv; ++q)
+                    tma_load_2d(sbase + kOffB + (uint32_t)s * kStageBytes + (uint32_t)q * kMemBytes, &p.tmap_h,
+                                bar(B_FULL0 + s), 0, mem_row + q * kN);
+            }
+            ++it_b;
+            return true;
+        };
         for (int i = blockIdx.x; i < p.total_tiles && ok; i += gridDim.x) {
             const Tile t = decode_tile(p, i);
             if (t.k == 0) continue;
             const int row = t.b * p.L + t.t0;
+            // The first memories of this tile go out before its Q and C: their
+            // stage is free long before the previous tile releases Q and C.
+            if (!(ok = load_b(t, 0))) break;
             if (!(ok = mbar_wait_warp(bar(Q_FREE), q_ph ^ 1, wc, 1))) break;
             if (lane == 0) {
                 mbar_expect_tx(bar(Q_FULL), 2 * kHalfA);
@@ -160,22 +181,22 @@ __global__ void __launch_bounds__(kThreads, 1) sma_tc_kernel(const __grid_consta
                 mbar_expect_tx(bar(C_FULL), 2 * kHalfA);
                 tma_load_2d(sbase + kOffC, &p.tmap_c, bar(C_FULL), 0, row);
                 tma_load_2d(sbase + kOffC + kHalfA, &p.tmap_c, bar(C_FULL), 64, row);
+                // the next non-empty tile's Q and C rows start moving into L2 now
+                for (int in = i + gridDim.x; in < p.total_tiles; in += gridDim.x) {
+                    const Tile tn = decode_tile(p, in);
+                    if (tn.k == 0) continue;
+                    const int rown = tn.b * p.L + tn.t0;
+                    tma_prefetch_3d(&p.tmap_q, 0, rown, tn.h);
+                    tma_prefetch_3d(&p.tmap_q, 64, rown, tn.h);
+                    tma_prefetch_2d(&p.tmap_c, 0, rown);
+                    tma_prefetch_2d(&p.tmap_c, 64, rown);
+                    break;
+                }
             }
             c_ph ^= 1;
             const int nbatch = (t.k + kCB - 1) / kCB;
-            for (int j = 0; j < nbatch; ++j, ++it_b) {
-                const int nv = min(kCB, t.k - kCB * j);
-                const int s = it_b % kNB;
-                const uint32_t ph = (uint32_t)(it_b / kNB) & 1u;
-                if (!(ok = mbar_wait_warp(bar(B_EMPTY0 + s), ph ^ 1, wc, 3))) break;
-                if (lane == 0) {
-                    mbar_expect_tx(bar(B_FULL0 + s), (uint32_t)nv * kMemBytes);
-                    const int mem_row = ((t.b * p.H + t.h) * p.C + kCB * j) * kN;
-                    for (int q = 0; q < nv; ++q)
-                        tma_load_2d(sbase + kOffB + (uint32_t)s * kStageBytes + (uint32_t)q * kMemBytes, &p.tmap_h,
-                                    bar(B_FULL0 + s), 0, mem_row + q * kN);
-                }
-            }
+            for (int j = 1; j < nbatch; ++j)
+                if (!(ok = load_b(t, j))) break;
             __syncwarp();
         }
     } else if (warp == 1) {
@@ -244,6 +265,7 @@ __global__ void __launch_bounds__(kThreads, 1) sma_tc_kernel(const __grid_consta
         const uint32_t t_lane = tmem + ((uint32_t)(quad * 32) << 16);
         const float sscale = kLog2e * rsqrtf((float)kN);
         float* xbuf = reinterpret_cast<float*>(smem + kOffX);
+        uint8_t* stage = smem + kOffS + (uint32_t)(warp - 2) * kStageWarp;
         int it_u = 0;
         bool ok = true;
         auto row_offset = [&](const Tile& t) -> size_t {
@@ -265,6 +287,12 @@ __global__ void __launch_bounds__(kThreads, 1) sma_tc_kernel(const __grid_consta
             for (int q = 0; q < kHalfP / 8; ++q) e_raw[q] = __ldg(src + q);
         };
         load_e(blockIdx.x);
+        // Row-contiguous (coalesced) view of the warp's 32 x 32 block: in
+        // step i, lane l covers row (i * 32 + l) / kPerRow, piece l % kPerRow.
+        auto block_row = [&](const Tile& t, int r) -> size_t {
+            const size_t tok = (size_t)t.b * p.L + t.t0 + quad * 32 + r;
+            return (tok * p.H + t.h) * kP + col0;
+        };
         for (int i = blockIdx.x; i < p.total_tiles; i += gridDim.x) {
             const Tile t = decode_tile(p, i);
             const size_t rowoff = row_offset(t);
@@ -362,23 +390,61 @@ __global__ void __launch_bounds__(kThreads, 1) sma_tc_kernel(const __grid_consta
                 }
             }
             const float inv = t.k > 0 && l > 0.f ? 1.f / l : 0.f;
-            float* orow = p.out + rowoff;
-            const float* yrow = p.y_ssd ? p.y_ssd + rowoff : nullptr;
-            // All loads (this tile's y_ssd row, the next tile's E) are issued
-            // before the first store: out may alias y_ssd, so loads placed
-            // after a store would each wait a full memory round trip.
-            float4 yv[kHalfP / 4];
+            // Tile end.  Rows of out, y_ssd and E are 128 B / 64 B pieces 8 KB
+            // apart, so they move through the per-warp staging buffer in a
+            // row-contiguous order (4 or 8 rows per instruction) instead of
+            // one row per lane.  Every load is issued before the first store
+            // (out may alias y_ssd); each lane stores exactly the elements it
+            // loaded.
+            float4 yv[8];  // rows 4i + l/8, columns 4 (l % 8) ..
 #pragma unroll
-            for (int q = 0; q < kHalfP / 4; ++q)
-                yv[q] = yrow ? *reinterpret_cast<const float4*>(yrow + 4 * q) : make_float4(0.f, 0.f, 0.f, 0.f);
-            load_e(i + gridDim.x);
-            const float gg = yrow ? p.g : 1.f;
+            for (int iy = 0; iy < 8; ++iy)
+                yv[iy] = p.y_ssd ? *reinterpret_cast<const float4*>(p.y_ssd + block_row(t, 4 * iy + lane / 8) + 4 * (lane % 8))
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+            const int inext = i + (int)gridDim.x;
+            const bool next_mem = inext < p.total_tiles && decode_tile(p, inext).k > 0;
+            uint4 en[4];   // next tile's E: rows 8i + l/4, columns 8 (l % 4) ..
+            if (next_mem) {
+                const Tile tn = decode_tile(p, inext);
 #pragma unroll
-            for (int q = 0; q < kHalfP / 4; ++q) {
-                const float2 lo = o2[2 * q], hi = o2[2 * q + 1];
-                const float4 r = make_float4(fmaf(gg, lo.x * inv, yv[q].x), fmaf(gg, lo.y * inv, yv[q].y),
-                                             fmaf(gg, hi.x * inv, yv[q].z), fmaf(gg, hi.y * inv, yv[q].w));
-                if (ok) *reinterpret_cast<float4*>(orow + 4 * q) = r;
+                for (int i2 = 0; i2 < 4; ++i2)
+                    en[i2] = __ldg(reinterpret_cast<const uint4*>(p.E + block_row(tn, 8 * i2 + lane / 4)) + (lane % 4));
+            }
+            const float gg = p.y_ssd ? p.g : 1.f;
+            float* st_f = reinterpret_cast<float*>(stage);
+#pragma unroll
+            for (int r2 = 0; r2 < 2; ++r2) {   // rows 16 r2 .. 16 r2 + 15
+                if ((lane >> 4) == r2) {
+                    float* dst = st_f + (lane & 15) * 36;
+#pragma unroll
+                    for (int q = 0; q < kHalfP / 4; ++q) {
+                        const float2 lo = o2[2 * q], hi = o2[2 * q + 1];
+                        *reinterpret_cast<float4*>(dst + 4 * q) =
+                            make_float4(gg * (lo.x * inv), gg * (lo.y * inv), gg * (hi.x * inv), gg * (hi.y * inv));
+                    }
+                }
+                __syncwarp();
+#pragma unroll
+                for (int i2 = 0; i2 < 4; ++i2) {
+                    const int rr = 4 * i2 + lane / 8;
+                    const float4 a = *reinterpret_cast<const float4*>(st_f + rr * 36 + 4 * (lane % 8));
+                    const float4 yy = yv[4 * r2 + i2];
+                    if (ok)
+                        *reinterpret_cast<float4*>(p.out + block_row(t, 16 * r2 + rr) + 4 * (lane % 8)) =
+                            make_float4(a.x + yy.x, a.y + yy.y, a.z + yy.z, a.w + yy.w);
+                }
+                __syncwarp();
+            }
+#pragma unroll
+            for (int q = 0; q < kHalfP / 8; ++q) e_raw[q] = make_uint4(0u, 0u, 0u, 0u);
+            if (next_mem) {
+#pragma unroll
+                for (int i2 = 0; i2 < 4; ++i2)
+                    *reinterpret_cast<uint4*>(stage + (8 * i2 + lane / 4) * 80 + (lane % 4) * 16) = en[i2];
+                __syncwarp();
+#pragma unroll
+                for (int q = 0; q < kHalfP / 8; ++q) e_raw[q] = *reinterpret_cast<const uint4*>(stage + lane * 80 + q * 16);
+                __syncwarp();
             }
         }
     }
