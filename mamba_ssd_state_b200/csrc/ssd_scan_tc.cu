@@ -20,9 +20,10 @@
 //      heads).  G = C B^T for the half's rows (128 x KS, KS = 128 (half+1))
 //      is computed once into TMEM and shared by the heads of the group.  Per
 //      head the worker warps build P[t,s] = G[t,s] exp(Acum_t - Acum_s)
-//      (s <= t, else 0) in bf16 straight from TMEM into shared memory, scale
-//      the x tile by dt, and the tensor core computes
-//        Y_diag = P (dt o x)          (K = KS)
+//      (s <= t, else 0) times dt_s in bf16 straight from TMEM into shared
+//      memory (dt of the source token is folded into P, so the x tile is used
+//      as loaded), and the tensor core computes
+//        Y_diag = P x                 (K = KS)
 //        Y_off  = C hin[c]            (K = N)
 //      y = Y_diag + exp(Acum_t) Y_off.
 //
@@ -327,20 +328,25 @@ __global__ void __launch_bounds__(256) state_pass_tc_kernel(const __grid_constan
 namespace co {
 constexpr int kWorkers = 256;
 constexpr int kThreads = 64 + kWorkers;  // warp 0 TMA, warp 1 MMA, warps 2-9 workers
-// Barrier slots; the two-deep rings take two consecutive slots each.
-enum Bar { IN_FULL = 0, G_FULL = 1, X_FULL0 = 2, X_FREE0 = 4, READY = 6, P_FREE = 7, ACC_FULL0 = 8,
-           ACC_EMPTY0 = 10, NUM_BARS = 12 };
-static_assert(X_FREE0 >= X_FULL0 + 2 && READY >= X_FREE0 + 2 && ACC_EMPTY0 >= ACC_FULL0 + 2 &&
-                  NUM_BARS >= ACC_EMPTY0 + 2 && P_FREE != READY && ACC_FULL0 > P_FREE,
-              "barrier slots overlap");
+// Barrier slots.  The two-deep rings take two consecutive slots; P is built
+// and consumed in 64-column panels (at most four), each with its own
+// ready / free pair, so the tensor core starts on a panel while the workers
+// build the next one.
+constexpr int kPanels = 4;
+enum Bar { IN_FULL = 0, G_FULL = 1, X_FULL0 = 2, X_FREE0 = 4, P_READY0 = 6, P_FREE0 = P_READY0 + kPanels,
+           ACC_FULL0 = P_FREE0 + kPanels, ACC_EMPTY0 = ACC_FULL0 + 2, NUM_BARS = ACC_EMPTY0 + 2 };
+static_assert(X_FREE0 >= X_FULL0 + 2 && P_READY0 >= X_FREE0 + 2 && NUM_BARS == 18, "barrier slots overlap");
 constexpr uint32_t kOffC = 0;                          // C rows: 2 panels x 128 rows (32 KB)
 constexpr uint32_t kOffBP = 2 * kBox;                  // B rows (2 panels x KS rows), later P (KS/64 panels x 128 rows)
 constexpr uint32_t kOffX = kOffBP + 4 * kBox;          // 2 buffers x (256 rows x 128 B)
 constexpr uint32_t kXBytes = 2 * kBox;
 constexpr uint32_t kOffHp = kOffX + 2 * kXBytes;       // 2 buffers x 128 rows (16 KB)
-constexpr uint32_t kOffF = kOffHp + 2 * kBox;          // a2[256], colf[256], dts[256], warp totals[16]
-constexpr uint32_t kOffBar = kOffF + (3 * 256 + 16) * 4;
+constexpr uint32_t kOffF = kOffHp + 2 * kBox;          // a2[256], colf[256], warp totals[16]
+constexpr uint32_t kOffYs = kOffF + (2 * 256 + 16) * 4;  // per-worker-warp y staging: 16 rows x 36 floats
+constexpr uint32_t kYsWarp = 16 * 36 * 4;
+constexpr uint32_t kOffBar = kOffYs + 8 * kYsWarp;
 constexpr uint32_t kBytes = kOffBar + NUM_BARS * 8 + 16 + 1024;
+static_assert(kOffYs % 16 == 0 && kBytes <= 232448, "chunk_output shared memory");
 constexpr uint32_t kColDiag = 256, kColOff = 384;
 
 __global__ void __launch_bounds__(kThreads, 1) chunk_output_tc_kernel(const __grid_constant__ ScanTcParams p) {
@@ -349,8 +355,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_output_tc_kernel(const __gr
     const uint32_t sbase = smem_u32(smem);
     float* a2 = reinterpret_cast<float*>(smem + kOffF);   // log2(e) * Acum over the chunk
     float* colf = a2 + 256;
-    float* dts = colf + 256;
-    float* warp_tot = dts + 256;
+    float* warp_tot = colf + 256;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + kOffBar + NUM_BARS * 8);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
     auto bar = [&](int i) -> uint32_t { return sbase + kOffBar + 8u * (uint32_t)i; };
@@ -380,8 +385,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_output_tc_kernel(const __gr
             mbar_init(bar(ACC_FULL0 + s), 1);
             mbar_init(bar(ACC_EMPTY0 + s), kWorkers / 32);
         }
-        mbar_init(bar(READY), kWorkers / 32);
-        mbar_init(bar(P_FREE), 1);
+        for (int k = 0; k < kPanels; ++k) {
+            mbar_init(bar(P_READY0 + k), kWorkers / 32);
+            mbar_init(bar(P_FREE0 + k), 1);
+        }
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -451,35 +458,47 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_output_tc_kernel(const __gr
             __syncwarp();
         }
         const uint32_t idesc_y = idesc_bf16_f32(128, kP, false, true);
+        const int npanel = KS / 64;
         for (int i = 0; i < p.HG && ok; ++i) {
             const int xs = i & 1, a = i & 1;
             const uint32_t ph = (uint32_t)(i >> 1) & 1u;
-            if (!(ok = mbar_wait_warp(bar(READY), (uint32_t)i & 1u, wc, 3))) break;
+            if (!(ok = mbar_wait_warp(bar(X_FULL0 + xs), ph, wc, 5))) break;
             if (!(ok = mbar_wait_warp(bar(ACC_EMPTY0 + a), ph ^ 1u, wc, 4))) break;
             tc_fence_after();
-            if (lane == 0) {
-                // Y_diag = P (dt o x): A = P (K-major, K = s), B = x (MN-major)
-                const uint32_t xbase = sbase + kOffX + (uint32_t)xs * kXBytes;
-                for (int kk = 0; kk < KS / 16; ++kk) {
-                    const uint64_t ad = smem_desc_sw128(
-                        sbase + kOffBP + (uint32_t)(kk >> 2) * kBox + (uint32_t)(kk & 3) * 32, 16, 1024);
-                    const uint64_t bd = smem_desc_sw128(xbase + (uint32_t)kk * 2048, 8192, 1024);
-                    mma_f16_ss(tmem + kColDiag + (uint32_t)a * 64, ad, bd, idesc_y, kk > 0 ? 1u : 0u);
-                }
-                if (has_off) {
-                    // Y_off = C hin[c]: A = C rows (K-major, K = n), B = hin (MN-major)
-                    const uint32_t hbase = sbase + kOffHp + (uint32_t)xs * kBox;
+            if (has_off && lane == 0) {
+                // Y_off = C hin[c]: A = C rows (K-major, K = n), B = hin (MN-major); needs no P
+                const uint32_t hbase = sbase + kOffHp + (uint32_t)xs * kBox;
 #pragma unroll
-                    for (int kk = 0; kk < kN / 16; ++kk) {
-                        const uint64_t ad = smem_desc_sw128(
-                            sbase + kOffC + (uint32_t)(kk >> 2) * kBox + (uint32_t)(kk & 3) * 32, 16, 1024);
-                        const uint64_t bd = smem_desc_sw128(hbase + (uint32_t)kk * 2048, 8192, 1024);
-                        mma_f16_ss(tmem + kColOff + (uint32_t)a * 64, ad, bd, idesc_y, kk > 0 ? 1u : 0u);
-                    }
+                for (int kk = 0; kk < kN / 16; ++kk) {
+                    const uint64_t ad = smem_desc_sw128(
+                        sbase + kOffC + (uint32_t)(kk >> 2) * kBox + (uint32_t)(kk & 3) * 32, 16, 1024);
+                    const uint64_t bd = smem_desc_sw128(hbase + (uint32_t)kk * 2048, 8192, 1024);
+                    mma_f16_ss(tmem + kColOff + (uint32_t)a * 64, ad, bd, idesc_y, kk > 0 ? 1u : 0u);
                 }
+            }
+            __syncwarp();
+            // Y_diag = P x with dt folded into P: A = P (K-major, K = s), B = x (MN-major),
+            // one 64-column panel of P at a time
+            const uint32_t xbase = sbase + kOffX + (uint32_t)xs * kXBytes;
+            for (int k = 0; k < npanel && ok; ++k) {
+                if (!(ok = mbar_wait_warp(bar(P_READY0 + k), (uint32_t)i & 1u, wc, 3))) break;
+                tc_fence_after();
+                if (lane == 0) {
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4) {
+                        const int kk = 4 * k + k4;
+                        const uint64_t ad = smem_desc_sw128(sbase + kOffBP + (uint32_t)k * kBox + (uint32_t)k4 * 32, 16, 1024);
+                        const uint64_t bd = smem_desc_sw128(xbase + (uint32_t)kk * 2048, 8192, 1024);
+                        mma_f16_ss(tmem + kColDiag + (uint32_t)a * 64, ad, bd, idesc_y, kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(bar(P_FREE0 + k));
+                }
+                __syncwarp();
+            }
+            if (!ok) break;
+            if (lane == 0) {
                 mma_commit(bar(ACC_FULL0 + a));
                 mma_commit(bar(X_FREE0 + xs));
-                mma_commit(bar(P_FREE));
             }
             __syncwarp();
         }
@@ -492,9 +511,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_output_tc_kernel(const __gr
         const int trow = quad * 32 + lane;               // row inside the half (TMEM lane)
         const int t = 128 * half + trow;                 // chunk-local token of this row
         const uint32_t t_lane = tmem + ((uint32_t)(quad * 32) << 16);
-        const int nblk = KS / 32;                        // 32-column blocks of P
-        const int blk0 = colhalf * (nblk / 2), blk1 = blk0 + nblk / 2;
+        const int npanel = KS / 64;                      // 64-column panels of P; this warp builds
+                                                         // block 2k + colhalf of panel k
         float row_scale_prev = 0.f;
+        float* ys = reinterpret_cast<float*>(smem + kOffYs + (uint32_t)wk * kYsWarp);
         auto epilogue = [&](int i, float row_scale) -> bool {
             const int a = i & 1;
             const uint32_t ph = (uint32_t)(i >> 1) & 1u;
@@ -507,102 +527,123 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_output_tc_kernel(const __gr
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(ACC_EMPTY0 + a));
+            // Rows of y are 256 B apart by H * 256 B: the warp's 32 x 32 block
+            // goes out through its staging buffer, 16 rows at a time, four
+            // rows per store instruction.
             const int h = hg * p.HG + i;
-            float* yrow = p.y + (((size_t)row0 + t) * p.H + h) * kP + colhalf * 32;
+            float* ybase = p.y + (((size_t)row0 + 128 * half + 32 * quad + lane / 8) * p.H + h) * kP + colhalf * 32 +
+                           4 * (lane % 8);
+            const size_t ystep = (size_t)4 * p.H * kP;
 #pragma unroll
-            for (int q = 0; q < 32; q += 4) {
-                float4 r = make_float4(yd[q], yd[q + 1], yd[q + 2], yd[q + 3]);
-                if (has_off) {
-                    r.x = fmaf(row_scale, yo[q], r.x);
-                    r.y = fmaf(row_scale, yo[q + 1], r.y);
-                    r.z = fmaf(row_scale, yo[q + 2], r.z);
-                    r.w = fmaf(row_scale, yo[q + 3], r.w);
+            for (int r2 = 0; r2 < 2; ++r2) {
+                if ((lane >> 4) == r2) {
+                    float* dst = ys + (lane & 15) * 36;
+#pragma unroll
+                    for (int q = 0; q < 32; q += 4) {
+                        float4 r = make_float4(yd[q], yd[q + 1], yd[q + 2], yd[q + 3]);
+                        if (has_off) {
+                            r.x = fmaf(row_scale, yo[q], r.x);
+                            r.y = fmaf(row_scale, yo[q + 1], r.y);
+                            r.z = fmaf(row_scale, yo[q + 2], r.z);
+                            r.w = fmaf(row_scale, yo[q + 3], r.w);
+                        }
+                        *reinterpret_cast<float4*>(dst + q) = r;
+                    }
                 }
-                *reinterpret_cast<float4*>(yrow + q) = r;
+                __syncwarp();
+#pragma unroll
+                for (int i2 = 0; i2 < 4; ++i2) {
+                    const int rr = 4 * i2 + lane / 8;
+                    *reinterpret_cast<float4*>(ybase + (4 * r2 + i2) * ystep) =
+                        *reinterpret_cast<const float4*>(ys + rr * 36 + 4 * (lane % 8));
+                }
+                __syncwarp();
             }
             return true;
         };
         // Every worker warp executes the same named barriers for every head,
         // also after a failed wait (it then skips the work).
         bool ok = true;
+        // dt of this thread's token for the next head, loaded one head ahead
+        const float* dt_row = p.dt + ((size_t)row0 + wi) * p.H + hg * p.HG;
+        float dt_next = wi < KS ? dt_row[0] : 0.f;
         for (int i = 0; i < p.HG; ++i) {
             const int h = hg * p.HG + i;
             const float Ah = p.A[h] * kLog2e;
-            if (i > 0) named_bar_sync(1, kWorkers);      // a2 / colf / dts of the previous head consumed
+            const float d0 = dt_next;
+            if (i + 1 < p.HG && wi < KS) dt_next = dt_row[i + 1];
+            if (i > 0) named_bar_sync(1, kWorkers);      // a2 / colf of the previous head consumed
             // log2-domain prefix of the decay over the chunk's first KS tokens
-            float d0 = 0.f, v0 = 0.f, v1 = 0.f;
-            if (wi < KS) {
-                d0 = p.dt[((size_t)row0 + wi) * p.H + h];
-                v0 = d0 * Ah;
-            }
+            float v0 = d0 * Ah, v1 = 0.f;
             block_scan<false>(v0, v1, wi, kWorkers, warp_tot, 2);
-            if (wi < KS) {
-                a2[wi] = v0;
-                dts[wi] = d0;
-            }
+            if (wi < KS) a2[wi] = v0;
             named_bar_sync(1, kWorkers);
-            if (wi < KS) colf[wi] = exp2f(a2[wi & ~31] - a2[wi]);
+            // column factor exp(Acum_r - Acum_s) dt_s: dt of the source token is
+            // folded into P, so the x tile is used as loaded
+            if (wi < KS) colf[wi] = exp2f(a2[wi & ~31] - v0) * d0;
             const float a2t = a2[t];
             const float row_scale = exp2f(a2t);          // exp(Acum_t): decay from the chunk start
             named_bar_sync(1, kWorkers);
-            // scale x rows by dt in place
-            const int xs = i & 1;
-            const uint32_t ph = (uint32_t)(i >> 1) & 1u;
-            if (ok) ok = mbar_wait_warp(bar(X_FULL0 + xs), ph, wc, 5);
-            // P may be written once G (first head) or the previous head's MMA has consumed the buffer
-            if (ok) ok = (i == 0) ? mbar_wait_warp(bar(G_FULL), 0, wc, 6)
-                                  : mbar_wait_warp(bar(P_FREE), (uint32_t)(i - 1) & 1u, wc, 7);
-            if (!ok) continue;
-            uint8_t* xb = smem + kOffX + (uint32_t)xs * kXBytes;
-            for (int k = wi; k < KS * 8; k += kWorkers) {
-                uint4* ptr = reinterpret_cast<uint4*>(xb + (size_t)k * 16);
-                float f[8];
-                Vec16<__nv_bfloat16>::unpack(*ptr, f);
-                const float ds = dts[k >> 3];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) f[j] *= ds;
-                Vec16<__nv_bfloat16>::store(reinterpret_cast<__nv_bfloat16*>(ptr), f);
-            }
-            tc_fence_after();
-            // P[t, s] = G[t, s] * exp(Acum_t - Acum_r) * exp(Acum_r - Acum_s), s <= t
-            const int warp_tmax = 128 * half + 32 * quad + 31;   // last row of this warp
-            for (int j = blk0; j < blk1; ++j) {
+            const int warp_tmin = 128 * half + 32 * quad;        // first row of this warp
+            const int warp_tmax = warp_tmin + 31;                // last row of this warp
+            for (int k = 0; k < npanel; ++k) {
+                // panel k may be written once G (first head) or the previous
+                // head's MMA on that panel has consumed the buffer
+                if (ok) ok = (i == 0) ? mbar_wait_warp(bar(G_FULL), 0, wc, 6)
+                                      : mbar_wait_warp(bar(P_FREE0 + k), (uint32_t)(i - 1) & 1u, wc, 7);
+                if (!ok) break;
+                tc_fence_after();
+                const int j = 2 * k + colhalf;
                 const int s0 = 32 * j;
                 uint32_t packed[16];
-                float g[32];
-                const bool warp_needs = s0 <= warp_tmax;            // warp-uniform
-                if (warp_needs) {
+                if (s0 <= warp_tmax) {                           // warp-uniform
+                    float g[32];
                     tmem_ld_32x32b_x32(t_lane + (uint32_t)s0, g);
-                    tmem_ld_wait();
-                }
-                if (warp_needs && s0 <= t) {
-                    const float rf = exp2f(a2t - a2[s0]);
+                    float2 cf[16];                               // column factors, same for every row
+                    const float4* c4 = reinterpret_cast<const float4*>(colf + s0);
 #pragma unroll
-                    for (int q = 0; q < 16; ++q) {
-                        const int sa = s0 + 2 * q, sb = sa + 1;
-                        const float va = sa <= t ? g[2 * q] * rf * colf[sa] : 0.f;
-                        const float vb = sb <= t ? g[2 * q + 1] * rf * colf[sb] : 0.f;
-                        __nv_bfloat162 pr = __floats2bfloat162_rn(va, vb);
-                        packed[q] = *reinterpret_cast<uint32_t*>(&pr);
+                    for (int q = 0; q < 8; ++q) {
+                        const float4 v = c4[q];
+                        cf[2 * q] = make_float2(v.x, v.y);
+                        cf[2 * q + 1] = make_float2(v.z, v.w);
+                    }
+                    const float rf = exp2f(a2t - a2[s0]);
+                    const float2 rf2 = make_float2(rf, rf);
+                    tmem_ld_wait();
+                    if (s0 + 31 <= warp_tmin) {                  // block below every row's diagonal
+#pragma unroll
+                        for (int q = 0; q < 16; ++q) {
+                            const float2 v = __fmul2_rn(__fmul2_rn(make_float2(g[2 * q], g[2 * q + 1]), cf[q]), rf2);
+                            __nv_bfloat162 pr = __floats2bfloat162_rn(v.x, v.y);
+                            packed[q] = *reinterpret_cast<uint32_t*>(&pr);
+                        }
+                    } else {                                     // the diagonal block: causal mask s <= t
+#pragma unroll
+                        for (int q = 0; q < 16; ++q) {
+                            const int sa = s0 + 2 * q;
+                            const float2 v = __fmul2_rn(__fmul2_rn(make_float2(g[2 * q], g[2 * q + 1]), cf[q]), rf2);
+                            __nv_bfloat162 pr = __floats2bfloat162_rn(sa <= t ? v.x : 0.f, sa + 1 <= t ? v.y : 0.f);
+                            packed[q] = *reinterpret_cast<uint32_t*>(&pr);
+                        }
                     }
                 } else {
 #pragma unroll
                     for (int q = 0; q < 16; ++q) packed[q] = 0u;
                 }
                 // row trow of panel j/2, 16-byte chunks (j%2)*4 .. +3, 128-byte swizzle
-                uint8_t* prow = smem + kOffBP + (uint32_t)(j >> 1) * kBox + (uint32_t)trow * kRowBytes;
+                uint8_t* prow = smem + kOffBP + (uint32_t)k * kBox + (uint32_t)trow * kRowBytes;
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
-                    const int ch = ((j & 1) * 4 + u) ^ (trow & 7);
+                    const int ch = (colhalf * 4 + u) ^ (trow & 7);
                     *reinterpret_cast<uint4*>(prow + ch * 16) =
                         make_uint4(packed[4 * u], packed[4 * u + 1], packed[4 * u + 2], packed[4 * u + 3]);
                 }
+                tc_fence_before();
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(P_READY0 + k));
             }
-            tc_fence_before();
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(READY));
-            if (i > 0) ok = epilogue(i - 1, row_scale_prev);
+            if (ok && i > 0) ok = epilogue(i - 1, row_scale_prev);
             row_scale_prev = row_scale;
         }
         if (ok) epilogue(p.HG - 1, row_scale_prev);
