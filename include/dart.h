@@ -69,8 +69,12 @@ typedef struct {
 } dart_dims;
 
 /*
- * Workspace for dart_ssd_chunk_scan: B*H*C floats (the per-chunk sum of
- * log-decays).  Pass at least this many bytes, 16-byte aligned.
+ * Workspace for dart_ssd_chunk_scan, in bytes: B*H*C floats (the per-chunk
+ * sum of log-decays, padded to 256 bytes); for the bf16 shapes that run on
+ * the tensor cores also the bf16 state entering each chunk (B*H*C*N*P*2
+ * bytes) and three fp32 per-token decay terms (3*B*H*L*4 bytes).  Pass at
+ * least this many bytes, 16-byte aligned.
+ * Its contents on entry do not matter and are not preserved.
  */
 size_t dart_ssd_chunk_scan_workspace_bytes(const dart_dims* dims, dart_dtype dtype);
 

@@ -112,8 +112,10 @@ size_t dart_ssd_chunk_scan_workspace_bytes(const dart_dims* d, dart_dtype dtype)
     const size_t C = (size_t)(d->seqlen / d->chunk);
     const size_t bhc = (size_t)d->batch * (size_t)d->nheads * C;
     size_t bytes = scan_asum_bytes(bhc);
-    if (dart::ssd_scan_tc_applicable(d->dstate, d->headdim, d->chunk, dtype))
+    if (dart::ssd_scan_tc_applicable(d->dstate, d->headdim, d->chunk, dtype)) {
         bytes += bhc * (size_t)d->dstate * (size_t)d->headdim * 2;  // bf16 state entering each chunk
+        bytes += 3 * bhc * (size_t)d->chunk * sizeof(float);         // per-token decay terms
+    }
     return bytes;
 }
 
@@ -134,9 +136,11 @@ dart_status dart_ssd_chunk_scan(const dart_dims* d, dart_dtype dtype, const void
         return fail(DART_ERR_INVALID_ARG, "workspace: %zu bytes, need %zu", workspace_bytes,
                     dart_ssd_chunk_scan_workspace_bytes(d, dtype));
     const size_t bhc = (size_t)d->batch * (size_t)d->nheads * (size_t)(d->seqlen / d->chunk);
+    char* hin = static_cast<char*>(workspace) + scan_asum_bytes(bhc);
+    float* decay = reinterpret_cast<float*>(hin + bhc * (size_t)d->dstate * (size_t)d->headdim * 2);
     dart::ScanArgs a{d->batch, d->seqlen, d->nheads, d->headdim, d->dstate, d->chunk,
                      x, dt, A, Bm, Cm, init_state, y_ssd, dH, states, static_cast<float*>(workspace),
-                     static_cast<char*>(workspace) + scan_asum_bytes(bhc), status_word()};
+                     hin, decay, status_word()};
     if (!a.status) return fail(DART_ERR_CUDA, "dart_ssd_chunk_scan: no device status word");
     cudaError_t e = dart::launch_ssd_scan(a, dtype, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "dart_ssd_chunk_scan launch");

@@ -105,6 +105,7 @@ struct ScanArgs {
     const float* init_state;
     float* y; void* dH; float* states; float* asum;  // asum: [B,H,C] workspace
     void* hin;    // tensor-core path: bf16 state entering each chunk [B,H,C,N,P] (workspace)
+    float* decay; // tensor-core path: per-token decay terms, 3 x [B,H,C,S] fp32 (workspace)
     int* status;  // device status word
 };
 struct SmaArgs {

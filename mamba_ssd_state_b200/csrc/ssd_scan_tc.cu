@@ -60,35 +60,63 @@ struct ScanTcParams {
     float* asum;
     __nv_bfloat16* hin;
     float* y;
+    // per-token decay terms, each [B, H, C, S] fp32 (written by chunk_decay):
+    //   a2   = log2(e) * Acum_s, the inclusive prefix of dt A inside the chunk
+    //   colf = exp(Acum_r - Acum_s) dt_s, r the first token of s's 32-token block
+    //   wst  = exp(Acum_end - Acum_s) dt_s, the weight of token s in dH[c]
+    float* a2;
+    float* colf;
+    float* wst;
     int B, L, H, S, C, HG;
     int* status;
 };
 
-// Inclusive prefix sum over `n` values held one or two per thread by
-// `nthreads` threads (n <= 2 * nthreads, nthreads a multiple of 32).
-// v0/v1 are this thread's values for elements 2*i, 2*i+1 (pair mode) or
-// element i (single mode, v1 ignored).  Returns the inclusive prefix of each.
-template <bool kPair>
-__device__ __forceinline__ void block_scan(float& v0, float& v1, int i, int nthreads, float* warp_tot, int bar_id) {
-    const int lane = i & 31, w = i >> 5;
-    float local = kPair ? v0 + v1 : v0;
-    float incl = local;
+// ===========================================================================
+// chunk_decay: the per-token decay terms of every (b, h, c), one warp each
+// ===========================================================================
+template <int S>
+__global__ void __launch_bounds__(256) chunk_decay_kernel(const __grid_constant__ ScanTcParams p) {
+    constexpr int K = S / 32;        // consecutive tokens per lane
+    constexpr int LPB = 32 / K;      // lanes per 32-token block
+    const int gw = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5);  // (b * H + h) * C + c
+    const int lane = threadIdx.x & 31;
+    if (gw >= p.B * p.H * p.C) return;  // whole warps only
+    const int c = gw % p.C, h = (gw / p.C) % p.H, b = gw / (p.C * p.H);
+    const float Ah = p.A[h];
+    const float* dtp = p.dt + ((size_t)b * p.L + (size_t)c * S + (size_t)lane * K) * p.H + h;
+    float d[K], v[K];
+    float run = 0.f;
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+        d[k] = dtp[(size_t)k * p.H];
+        run += d[k] * Ah;
+        v[k] = run;
+    }
+    float incl = run;  // inclusive prefix of the lane totals
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
         const float up = __shfl_up_sync(0xffffffffu, incl, o);
         if (lane >= o) incl += up;
     }
-    if (lane == 31) warp_tot[w] = incl;
-    named_bar_sync(bar_id, nthreads);
-    float base = 0.f;
-    for (int j = 0; j < w; ++j) base += warp_tot[j];
-    const float excl = base + incl - local;
-    if (kPair) {
-        v0 = excl + v0;
-        v1 = v0 + v1;
-    } else {
-        v0 = excl + v0;
+    const float excl = incl - run;
+    const float aend = __shfl_sync(0xffffffffu, incl, 31);
+    float a2[K], cf[K], ws[K];
+#pragma unroll
+    for (int k = 0; k < K; ++k) a2[k] = (excl + v[k]) * kLog2e;
+    const float a2r = __shfl_sync(0xffffffffu, a2[0], lane & ~(LPB - 1));
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+        cf[k] = exp2f(a2r - a2[k]) * d[k];
+        ws[k] = expf(aend - (excl + v[k])) * d[k];
     }
+    const size_t o = (size_t)gw * S + (size_t)lane * K;
+#pragma unroll
+    for (int k = 0; k < K; k += 4) {
+        *reinterpret_cast<float4*>(p.a2 + o + k) = make_float4(a2[k], a2[k + 1], a2[k + 2], a2[k + 3]);
+        *reinterpret_cast<float4*>(p.colf + o + k) = make_float4(cf[k], cf[k + 1], cf[k + 2], cf[k + 3]);
+        *reinterpret_cast<float4*>(p.wst + o + k) = make_float4(ws[k], ws[k + 1], ws[k + 2], ws[k + 3]);
+    }
+    if (lane == 0) p.asum[gw] = aend;
 }
 
 // ===========================================================================
@@ -104,8 +132,8 @@ struct Layout {
     static constexpr uint32_t kOffB = 0;                        // 2 panels x S rows
     static constexpr uint32_t kOffX = 2 * S * kRowBytes;        // 2 buffers x S rows
     static constexpr uint32_t kXBytes = S * kRowBytes;
-    static constexpr uint32_t kOffF = kOffX + 2 * kXBytes;      // w[S] floats + 8 warp totals
-    static constexpr uint32_t kOffBar = kOffF + (S + 8) * 4;
+    static constexpr uint32_t kOffF = kOffX + 2 * kXBytes;      // 2 buffers x wst[S] floats
+    static constexpr uint32_t kOffBar = kOffF + 2 * S * 4;
     static constexpr uint32_t kBytes = kOffBar + NUM_BARS * 8 + 16 + 1024;
 };
 
@@ -115,8 +143,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_state_tc_kernel(const __gri
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
-    float* w_s = reinterpret_cast<float*>(smem + Ly::kOffF);
-    float* warp_tot = w_s + S;
+    const float* wst_s = reinterpret_cast<const float*>(smem + Ly::kOffF);
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Ly::kOffBar + NUM_BARS * 8);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
     auto bar = [&](int i) -> uint32_t { return sbase + Ly::kOffBar + 8u * (uint32_t)i; };
@@ -167,10 +194,13 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_state_tc_kernel(const __gri
             const uint32_t ph = (uint32_t)(i >> 1) & 1u;
             if (!mbar_wait_warp(bar(X_EMPTY0 + xs), ph ^ 1u, wc, 1)) break;
             if (lane == 0) {
-                mbar_expect_tx(bar(X_FULL0 + xs), Ly::kXBytes);
+                const int h = hg * p.HG + i;
+                mbar_expect_tx(bar(X_FULL0 + xs), Ly::kXBytes + S * 4);
                 for (int r = 0; r < S / 128; ++r)
                     tma_load_3d(sbase + Ly::kOffX + (uint32_t)xs * Ly::kXBytes + (uint32_t)r * kBox, &p.tmap_x,
-                                bar(X_FULL0 + xs), 0, row0 + 128 * r, hg * p.HG + i);
+                                bar(X_FULL0 + xs), 0, row0 + 128 * r, h);
+                bulk_load(sbase + Ly::kOffF + (uint32_t)xs * S * 4, p.wst + (((size_t)b * p.H + h) * p.C + c) * S,
+                          S * 4, bar(X_FULL0 + xs));
             }
             __syncwarp();
         }
@@ -232,46 +262,18 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_state_tc_kernel(const __gri
         };
         bool ok = true;
         for (int i = 0; i < p.HG; ++i) {
-            const int h = hg * p.HG + i;
-            const float Ah = p.A[h];
-            if (i > 0) named_bar_sync(1, 128);  // w_s of the previous head fully consumed
-            // per-token log-decay prefix and the memory weights w_s
-            float d0, d1 = 0.f, a0, a1 = 0.f;
-            const float* dtp = p.dt + ((size_t)row0) * p.H + h;
-            if (S == 256) {
-                d0 = dtp[(size_t)(2 * wi) * p.H];
-                d1 = dtp[(size_t)(2 * wi + 1) * p.H];
-                a0 = d0 * Ah;
-                a1 = d1 * Ah;
-                block_scan<true>(a0, a1, wi, 128, warp_tot, 2);
-            } else {
-                d0 = dtp[(size_t)wi * p.H];
-                a0 = d0 * Ah;
-                block_scan<false>(a0, a1, wi, 128, warp_tot, 2);
-            }
-            // total over the chunk: the last thread's inclusive value
-            if (wi == 127) warp_tot[4] = (S == 256) ? a1 : a0;
-            named_bar_sync(1, 128);
-            const float aend = warp_tot[4];
-            if (S == 256) {
-                w_s[2 * wi] = expf(aend - a0) * d0;
-                w_s[2 * wi + 1] = expf(aend - a1) * d1;
-            } else {
-                w_s[wi] = expf(aend - a0) * d0;
-            }
-            if (wi == 0) p.asum[((size_t)b * p.H + h) * p.C + c] = aend;
-            named_bar_sync(1, 128);
-            // scale the x tile in place: row s of the panel times w_s
+            // scale the x tile in place: row s of the panel times wst_s
             const int xs = i & 1;
             const uint32_t ph = (uint32_t)(i >> 1) & 1u;
             if (ok) ok = mbar_wait_warp(bar(X_FULL0 + xs), ph, wc, 6);
             if (ok) {
                 uint8_t* xb = smem + Ly::kOffX + (uint32_t)xs * Ly::kXBytes;
+                const float* w = wst_s + xs * S;
                 for (int k = wi; k < S * 8; k += 128) {
                     uint4* ptr = reinterpret_cast<uint4*>(xb + (size_t)k * 16);
                     float f[8];
                     Vec16<__nv_bfloat16>::unpack(*ptr, f);
-                    const float ws = w_s[k >> 3];
+                    const float ws = w[k >> 3];
 #pragma unroll
                     for (int j = 0; j < 8; ++j) f[j] *= ws;
                     Vec16<__nv_bfloat16>::store(reinterpret_cast<__nv_bfloat16*>(ptr), f);
@@ -341,8 +343,8 @@ constexpr uint32_t kOffBP = 2 * kBox;                  // B rows (2 panels x KS 
 constexpr uint32_t kOffX = kOffBP + 4 * kBox;          // 2 buffers x (256 rows x 128 B)
 constexpr uint32_t kXBytes = 2 * kBox;
 constexpr uint32_t kOffHp = kOffX + 2 * kXBytes;       // 2 buffers x 128 rows (16 KB)
-constexpr uint32_t kOffF = kOffHp + 2 * kBox;          // a2[256], colf[256], warp totals[16]
-constexpr uint32_t kOffYs = kOffF + (2 * 256 + 16) * 4;  // per-worker-warp y staging: 16 rows x 36 floats
+constexpr uint32_t kOffF = kOffHp + 2 * kBox;          // 2 buffers x (a2[256], colf[256])
+constexpr uint32_t kOffYs = kOffF + 2 * 2 * 256 * 4;   // per-worker-warp y staging: 16 rows x 36 floats
 constexpr uint32_t kYsWarp = 16 * 36 * 4;
 constexpr uint32_t kOffBar = kOffYs + 8 * kYsWarp;
 constexpr uint32_t kBytes = kOffBar + NUM_BARS * 8 + 16 + 1024;
@@ -353,9 +355,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_output_tc_kernel(const __gr
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
-    float* a2 = reinterpret_cast<float*>(smem + kOffF);   // log2(e) * Acum over the chunk
-    float* colf = a2 + 256;
-    float* warp_tot = colf + 256;
+    const float* dec_s = reinterpret_cast<const float*>(smem + kOffF);  // [2][a2[256], colf[256]]
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + kOffBar + NUM_BARS * 8);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
     auto bar = [&](int i) -> uint32_t { return sbase + kOffBar + 8u * (uint32_t)i; };
@@ -426,8 +426,11 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_output_tc_kernel(const __gr
             const int h = hg * p.HG + i;
             if (!mbar_wait_warp(bar(X_FREE0 + xs), ph ^ 1u, wc, 1)) break;
             if (lane == 0) {
-                const uint32_t bytes = (uint32_t)KS * kRowBytes + (has_off ? kBox : 0u);
+                const uint32_t bytes = (uint32_t)KS * kRowBytes + (has_off ? kBox : 0u) + 2u * KS * 4u;
                 mbar_expect_tx(bar(X_FULL0 + xs), bytes);
+                const size_t drow = (((size_t)b * p.H + h) * p.C + c) * S;   // this (b, h, c) in the decay arrays
+                bulk_load(sbase + kOffF + (uint32_t)xs * 2048, p.a2 + drow, KS * 4, bar(X_FULL0 + xs));
+                bulk_load(sbase + kOffF + (uint32_t)xs * 2048 + 1024, p.colf + drow, KS * 4, bar(X_FULL0 + xs));
                 for (int r = 0; r < KS / 128; ++r)
                     tma_load_3d(sbase + kOffX + (uint32_t)xs * kXBytes + (uint32_t)r * kBox, &p.tmap_x,
                                 bar(X_FULL0 + xs), 0, row0 + 128 * r, h);
@@ -504,7 +507,6 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_output_tc_kernel(const __gr
         }
     } else {
         // ---------------------------------------------------------- workers
-        const int wi = threadIdx.x - 64;                 // 0..255
         const int wk = warp - 2;                         // 0..7
         const int quad = warp & 3;                       // TMEM lane quadrant
         const int colhalf = wk >> 2;                     // which half of the columns
@@ -564,26 +566,15 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_output_tc_kernel(const __gr
         // Every worker warp executes the same named barriers for every head,
         // also after a failed wait (it then skips the work).
         bool ok = true;
-        // dt of this thread's token for the next head, loaded one head ahead
-        const float* dt_row = p.dt + ((size_t)row0 + wi) * p.H + hg * p.HG;
-        float dt_next = wi < KS ? dt_row[0] : 0.f;
         for (int i = 0; i < p.HG; ++i) {
-            const int h = hg * p.HG + i;
-            const float Ah = p.A[h] * kLog2e;
-            const float d0 = dt_next;
-            if (i + 1 < p.HG && wi < KS) dt_next = dt_row[i + 1];
-            if (i > 0) named_bar_sync(1, kWorkers);      // a2 / colf of the previous head consumed
-            // log2-domain prefix of the decay over the chunk's first KS tokens
-            float v0 = d0 * Ah, v1 = 0.f;
-            block_scan<false>(v0, v1, wi, kWorkers, warp_tot, 2);
-            if (wi < KS) a2[wi] = v0;
-            named_bar_sync(1, kWorkers);
-            // column factor exp(Acum_r - Acum_s) dt_s: dt of the source token is
-            // folded into P, so the x tile is used as loaded
-            if (wi < KS) colf[wi] = exp2f(a2[wi & ~31] - v0) * d0;
-            const float a2t = a2[t];
+            // decay terms of this head arrive with its x tile
+            const int xs = i & 1;
+            const uint32_t ph = (uint32_t)(i >> 1) & 1u;
+            if (ok) ok = mbar_wait_warp(bar(X_FULL0 + xs), ph, wc, 9);
+            const float* a2 = dec_s + xs * 512;
+            const float* colf = a2 + 256;
+            const float a2t = ok ? a2[t] : 0.f;
             const float row_scale = exp2f(a2t);          // exp(Acum_t): decay from the chunk start
-            named_bar_sync(1, kWorkers);
             const int warp_tmin = 128 * half + 32 * quad;        // first row of this warp
             const int warp_tmax = warp_tmin + 31;                // last row of this warp
             for (int k = 0; k < npanel; ++k) {
@@ -708,8 +699,22 @@ cudaError_t launch_ssd_scan_tc(const ScanArgs& a, cudaStream_t st) {
     p.hin = static_cast<__nv_bfloat16*>(a.hin);
     p.y = a.y;
     p.B = a.B; p.L = a.L; p.H = a.H; p.S = a.S; p.C = a.L / a.S;
+    const size_t bhcs = (size_t)a.B * a.H * a.L;
+    p.a2 = a.decay;
+    p.colf = a.decay + bhcs;
+    p.wst = a.decay + 2 * bhcs;
     p.status = a.status;
     cudaError_t e;
+    // 0. per-token decay terms, one warp per (b, h, c)
+    {
+        const int warps = a.B * a.H * p.C;
+        const int grid = (warps + 7) / 8;
+        if (a.S == 256)
+            chunk_decay_kernel<256><<<grid, 256, 0, st>>>(p);
+        else
+            chunk_decay_kernel<128><<<grid, 256, 0, st>>>(p);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
     // 1. chunk memories
     p.HG = pick_group(a.H, 8);
     {
@@ -742,7 +747,7 @@ cudaError_t launch_ssd_scan_tc(const ScanArgs& a, cudaStream_t st) {
         co::chunk_output_tc_kernel<<<grid, co::kThreads, co::kBytes, st>>>(p);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    count_launches(3);
+    count_launches(4);
     return cudaSuccess;
 }
 

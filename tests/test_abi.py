@@ -84,8 +84,9 @@ def test_scan_rejects_small_workspace(lib):
     d = dart.Dims(2, 512, 4, 64, 128, 256, 1)
     need = lib.dart_ssd_chunk_scan_workspace_bytes(ctypes.byref(d), dart.DART_BF16)
     bhc = 2 * 4 * 2
-    # per-chunk decay sums padded to 256 bytes + the bf16 state entering each chunk
-    assert need == 256 + bhc * 128 * 64 * 2
+    # per-chunk decay sums padded to 256 bytes + the bf16 state entering each
+    # chunk + three fp32 per-token decay terms
+    assert need == 256 + bhc * 128 * 64 * 2 + 3 * bhc * 256 * 4
     assert lib.dart_ssd_chunk_scan_workspace_bytes(ctypes.byref(d), dart.DART_F32) == 256
     assert _scan(lib, d, ws_bytes=need - 1) == dart.DART_ERR_INVALID_ARG
 
