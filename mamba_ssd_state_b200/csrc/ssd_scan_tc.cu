@@ -52,6 +52,8 @@ struct ScanTcParams {
     CUtensorMap tmap_b;    // Bm as (N, B*L),    box (64, 128)
     CUtensorMap tmap_c;    // Cm as (N, B*L),    box (64, 128)
     CUtensorMap tmap_hin;  // hin as (P, B*H*C*N), box (64, 128)
+    CUtensorMap tmap_dh;   // dH as (P, B*H*C*N) bf16, box (64, 128): chunk_state's store
+    CUtensorMap tmap_st;   // states as (P, B*H*C*N) fp32, box (32, 128): chunk_state's store
     const float* dt;
     const float* A;
     const float* init_state;
@@ -133,7 +135,10 @@ struct Layout {
     static constexpr uint32_t kOffX = 2 * S * kRowBytes;        // 2 buffers x S rows
     static constexpr uint32_t kXBytes = S * kRowBytes;
     static constexpr uint32_t kOffF = kOffX + 2 * kXBytes;      // 2 buffers x wst[S] floats
-    static constexpr uint32_t kOffBar = kOffF + 2 * S * 4;
+    // output staging (128-byte swizzle, as the store tensor maps expect):
+    // dH tile 128 rows x 128 B, then the states tile as two 128 x 128 B panels
+    static constexpr uint32_t kOffOut = (kOffF + 2 * S * 4 + 1023) & ~1023u;
+    static constexpr uint32_t kOffBar = kOffOut + 3 * kBox;
     static constexpr uint32_t kBytes = kOffBar + NUM_BARS * 8 + 16 + 1024;
 };
 
@@ -237,28 +242,51 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_state_tc_kernel(const __gri
         const int quad = warp & 3;
         const int nrow = quad * 32 + lane;          // TMEM lane = state row n
         const uint32_t t_lane = tmem + ((uint32_t)(quad * 32) << 16);
-        auto epilogue = [&](int i) -> bool {
+        // The four worker warps run every epilogue's two named barriers
+        // whether or not their own waits succeeded (they then skip the work),
+        // so none of them can be left at a barrier the others never reach.
+        uint8_t* out_s = smem + Ly::kOffOut;
+        auto epilogue = [&](int i, bool live) -> bool {
             const int a = i & 1;
             const uint32_t ph = (uint32_t)(i >> 1) & 1u;
-            if (!mbar_wait_warp(bar(ACC_FULL0 + a), ph, wc, 5)) return false;
-            tc_fence_after();
+            live = live && mbar_wait_warp(bar(ACC_FULL0 + a), ph, wc, 5);
             float v[kP];
-            tmem_ld_32x32b_x32(t_lane + (uint32_t)a * 64, v);
-            tmem_ld_32x32b_x32(t_lane + (uint32_t)a * 64 + 32, v + 32);
-            tmem_ld_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(ACC_EMPTY0 + a));
-            const int h = hg * p.HG + i;
-            const size_t off = ((((size_t)b * p.H + h) * p.C + c) * kN + nrow) * kP;
-#pragma unroll
-            for (int q = 0; q < kP; q += 8) {
-                Vec16<__nv_bfloat16>::store(p.dH + off + q, v + q);
-                *reinterpret_cast<float4*>(p.states + off + q) = make_float4(v[q], v[q + 1], v[q + 2], v[q + 3]);
-                *reinterpret_cast<float4*>(p.states + off + q + 4) =
-                    make_float4(v[q + 4], v[q + 5], v[q + 6], v[q + 7]);
+            if (live) {
+                tc_fence_after();
+                tmem_ld_32x32b_x32(t_lane + (uint32_t)a * 64, v);
+                tmem_ld_32x32b_x32(t_lane + (uint32_t)a * 64 + 32, v + 32);
+                tmem_ld_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(ACC_EMPTY0 + a));
             }
-            return true;
+            if (wi == 0) bulk_wait_read<0>();  // the previous head's tiles have left the staging
+            named_bar_sync(1, 128);
+            if (live) {
+                // row nrow, 16-byte chunk j at position j ^ (nrow & 7) of its 128-byte row
+                uint8_t* drow = out_s + (uint32_t)nrow * kRowBytes;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    Vec16<__nv_bfloat16>::store(reinterpret_cast<__nv_bfloat16*>(drow + ((j ^ (nrow & 7)) << 4)), v + 8 * j);
+                }
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    uint8_t* srow = out_s + (uint32_t)(1 + (j >> 3)) * kBox + (uint32_t)nrow * kRowBytes;
+                    *reinterpret_cast<float4*>(srow + (((j & 7) ^ (nrow & 7)) << 4)) =
+                        make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+                }
+            }
+            fence_proxy_async_smem();
+            named_bar_sync(1, 128);
+            if (wi == 0 && !*abort_flag) {
+                const int h = hg * p.HG + i;
+                const int row = (((b * p.H + h) * p.C + c) * kN);
+                tma_store_2d(&p.tmap_dh, smem_u32(out_s), 0, row);
+                tma_store_2d(&p.tmap_st, smem_u32(out_s + kBox), 0, row);
+                tma_store_2d(&p.tmap_st, smem_u32(out_s + 2 * kBox), 32, row);
+                bulk_commit();
+            }
+            return live;
         };
         bool ok = true;
         for (int i = 0; i < p.HG; ++i) {
@@ -282,9 +310,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_state_tc_kernel(const __gri
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(W_READY0 + xs));
             }
-            if (ok && i > 0) ok = epilogue(i - 1);
+            if (i > 0) ok = epilogue(i - 1, ok);
         }
-        if (ok) epilogue(p.HG - 1);
+        epilogue(p.HG - 1, ok);
+        if (wi == 0) bulk_wait<0>();  // stores complete before the CTA's shared memory goes away
     }
 
     tc_fence_before();
@@ -670,6 +699,13 @@ bool make_maps(const ScanArgs& a, ScanTcParams& p) {
         const uint64_t strides[1] = {(uint64_t)kP * 2};
         const uint32_t box[2] = {64, 128};
         if (!encode_tile_map_bf16(&p.tmap_hin, 2, a.hin, dims, strides, box)) return false;
+        if (!encode_tile_map_bf16(&p.tmap_dh, 2, a.dH, dims, strides, box)) return false;
+    }
+    {
+        const uint64_t dims[2] = {(uint64_t)kP, (uint64_t)a.B * a.H * C * kN};
+        const uint64_t strides[1] = {(uint64_t)kP * 4};
+        const uint32_t box[2] = {32, 128};
+        if (!encode_tile_map_f32(&p.tmap_st, 2, a.states, dims, strides, box)) return false;
     }
     return true;
 }

@@ -20,8 +20,9 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 }  // namespace
 
-bool encode_tile_map_bf16(CUtensorMap* map, int rank, const void* base, const uint64_t* dims,
-                          const uint64_t* strides_bytes, const uint32_t* box) {
+namespace {
+bool encode_tile_map(CUtensorMap* map, CUtensorMapDataType type, int rank, const void* base, const uint64_t* dims,
+                     const uint64_t* strides_bytes, const uint32_t* box) {
     auto fn = encode_fn();
     if (!fn) return false;
     cuuint64_t gd[5];
@@ -33,10 +34,20 @@ bool encode_tile_map_bf16(CUtensorMap* map, int rank, const void* base, const ui
         es[i] = 1;
     }
     for (int i = 0; i + 1 < rank; ++i) gs[i] = strides_bytes[i];
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), gd, gs, bx, es,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    CUresult r = fn(map, type, (cuuint32_t)rank, const_cast<void*>(base), gd, gs, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
+}
+}  // namespace
+
+bool encode_tile_map_bf16(CUtensorMap* map, int rank, const void* base, const uint64_t* dims,
+                          const uint64_t* strides_bytes, const uint32_t* box) {
+    return encode_tile_map(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, base, dims, strides_bytes, box);
+}
+
+bool encode_tile_map_f32(CUtensorMap* map, int rank, const void* base, const uint64_t* dims,
+                         const uint64_t* strides_bytes, const uint32_t* box) {
+    return encode_tile_map(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, rank, base, dims, strides_bytes, box);
 }
 
 int sm_count() {

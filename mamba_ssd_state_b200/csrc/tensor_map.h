@@ -13,6 +13,10 @@ namespace dart {
 bool encode_tile_map_bf16(CUtensorMap* map, int rank, const void* base, const uint64_t* dims,
                           const uint64_t* strides_bytes, const uint32_t* box);
 
+// The same for fp32 elements (box[0] * 4 must not exceed the 128-byte swizzle span).
+bool encode_tile_map_f32(CUtensorMap* map, int rank, const void* base, const uint64_t* dims,
+                         const uint64_t* strides_bytes, const uint32_t* box);
+
 // Number of SMs of the current device (0 on error).
 int sm_count();
 
