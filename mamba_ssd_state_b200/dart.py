@@ -120,6 +120,19 @@ def _dev(t: Optional[torch.Tensor], device, dtype=None) -> Optional[torch.Tensor
     return t.contiguous()
 
 
+def _to_host(*ts):
+    """Copies device tensors back into page-locked host tensors (torch's
+    caching host allocator) with asynchronous copies, then waits for them."""
+    out = []
+    for t in ts:
+        h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+        h.copy_(t, non_blocking=True)
+        out.append(h)
+    if ts:
+        torch.cuda.current_stream(ts[0].device).synchronize()
+    return out
+
+
 def _device_of(*ts) -> torch.device:
     for t in ts:
         if isinstance(t, torch.Tensor) and t.is_cuda:
@@ -192,7 +205,7 @@ def dart_ssd_chunk_scan(x, dt, A, Bm, Cm, chunk: int, init_state=None, *, y_ssd=
                                        _ptr(Cm), _ptr(init_state), _ptr(y_ssd), _ptr(dH), _ptr(states),
                                        _ptr(workspace), workspace.numel(), _stream()))
     if host:
-        return y_ssd.cpu(), dH.cpu(), states.cpu()
+        return tuple(_to_host(y_ssd, dH, states))
     return y_ssd, dH, states
 
 
@@ -218,7 +231,7 @@ def dart_sma_forward(Q, E, Cm, dH, chunk: int, g: float, y_ssd=None, *, out=None
     with torch.cuda.device(dev):
         _check(lib.dart_sma_forward(ctypes.byref(dims), _dtype_code(Q.dtype), _ptr(Q), _ptr(E), _ptr(Cm),
                                     _ptr(dH), float(g), _ptr(y_ssd), _ptr(out), _stream()))
-    return out.cpu() if host else out
+    return _to_host(out)[0] if host else out
 
 
 def layer_forward(x, dt, A, Bm, Cm, Q, E, chunk: int, g: float, init_state=None, *,
@@ -238,7 +251,7 @@ def layer_forward(x, dt, A, Bm, Cm, Q, E, chunk: int, g: float, init_state=None,
     dart_sma_forward(args[5], args[6], args[4], dH, chunk, g, y, out=y)
     res = {"y": y, "dH": dH, "states": states}
     if host:
-        return {k: res[k].cpu() for k in outputs}
+        return dict(zip(outputs, _to_host(*(res[k] for k in outputs))))
     return {k: res[k] for k in outputs}
 
 
@@ -279,7 +292,7 @@ def dart_decode_step(x, dt, A, Bm, Cm, Q, E, g: float, state, dH_cur, cache, nch
                                     _ptr(Q), _ptr(E), float(g), _ptr(state), _ptr(dH_cur), _ptr(cache),
                                     cmax, _ptr(nchunks), _ptr(pos), _ptr(y), _ptr(workspace),
                                     workspace.numel(), _stream()))
-    return y.cpu() if host else y
+    return _to_host(y)[0] if host else y
 
 
 def dart_decode_step_noalloc(x, dt, A, Bm, Cm, Q, E, g: float, state, dH_cur, cache, nchunks, pos,
