@@ -122,7 +122,9 @@ dart_status dart_ssd_chunk_scan(const dart_dims* dims, dart_dtype dtype,
  *   out = y_ssd + g * o   when y_ssd != NULL (the DART layer output), else
  *   out = o               (the raw readout).
  *   Q[B,L,H,N], E[B,L,H,P], Cm[B,L,N], dH[B,H,C,N,P]: dtype inputs.
- *   y_ssd: nullable float [B,L,H,P]; out: float [B,L,H,P] (may alias y_ssd).
+ *   y_ssd: nullable float [B,L,H,P]; out: float [B,L,H,P], either the same
+ *   pointer as y_ssd (updated in place, the fastest form) or not overlapping it
+ *   (y_ssd is then copied into out on the stream first).
  */
 dart_status dart_sma_forward(const dart_dims* dims, dart_dtype dtype,
                              const void* Q, const void* E, const void* Cm, const void* dH,

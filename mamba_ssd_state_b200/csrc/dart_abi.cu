@@ -158,6 +158,12 @@ dart_status dart_sma_forward(const dart_dims* d, dart_dtype dtype, const void* Q
                     d->dstate, d->headdim, d->chunk);
     DART_REQUIRE_PTR(Q); DART_REQUIRE_PTR(E); DART_REQUIRE_PTR(Cm); DART_REQUIRE_PTR(dH);
     DART_OPTIONAL_PTR(y_ssd); DART_REQUIRE_PTR(out);
+    if (y_ssd && y_ssd != out) {
+        const size_t bytes = (size_t)d->batch * d->seqlen * d->nheads * d->headdim * sizeof(float);
+        const uintptr_t ya = reinterpret_cast<uintptr_t>(y_ssd), oa = reinterpret_cast<uintptr_t>(out);
+        if (ya < oa + bytes && oa < ya + bytes)
+            return fail(DART_ERR_INVALID_ARG, "dart_sma_forward: out overlaps y_ssd without being the same pointer");
+    }
     dart::SmaArgs a{d->batch, d->seqlen, d->nheads, d->headdim, d->dstate, d->chunk,
                     Q, E, Cm, dH, g, y_ssd, out, status_word()};
     if (!a.status) return fail(DART_ERR_CUDA, "dart_sma_forward: no device status word");

@@ -52,11 +52,15 @@ constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffC = 2 * kHalfA;
 constexpr uint32_t kOffB = 4 * kHalfA;
 constexpr uint32_t kStageBytes = kCB * kMemBytes;
-constexpr uint32_t kOffBar = kOffB + kNB * kStageBytes;
-constexpr uint32_t kOffX = kOffBar + 256;            // partial-score exchange: [2 parity][2 half][128 rows][4]
-constexpr uint32_t kOffS = kOffX + 2 * 2 * 128 * 4 * 4;  // per-warp staging for coalesced row traffic
-constexpr uint32_t kStageWarp = 32 * 80;                  // 32 E rows of 64 B (+16 pad) or 16 out rows of 144 B
-constexpr uint32_t kSmemBytes = kOffS + 8 * kStageWarp + 1024;  // + alignment slack
+// Output tile: at a tile end the gated attention output g o / l of the 128
+// rows, as two 128-byte-swizzled boxes of 32 fp32 columns (the layout of the
+// out tensor map), added into out (which holds y_ssd) by a TMA reduction.
+// While a tile runs, its first 8 KB hold the partial-score exchange
+// [2 parity][2 half][128 rows][4].
+constexpr uint32_t kOffO = kOffB + kNB * kStageBytes;
+constexpr uint32_t kOBox = 128 * 32 * 4;              // one box: 128 rows x 32 fp32
+constexpr uint32_t kOffBar = kOffO + 2 * kOBox;
+constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;  // + alignment slack
 constexpr int kEpiWarps = 8;                          // four pairs, one pair per TMEM lane quadrant
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr uint32_t kTmemCols = 512;
@@ -67,17 +71,20 @@ constexpr int kHalfP = kP / 2;                        // value columns per epilo
 enum Bar { Q_FULL = 0, Q_FREE = 1, C_FULL = 2, C_FREE = 3, U_FULL = 4, U_EMPTY = 5, V_FULL = 6, V_EMPTY = 7,
            B_FULL0 = 8, B_EMPTY0 = B_FULL0 + kNB, NUM_BARS = B_EMPTY0 + kNB };
 static_assert(NUM_BARS * 8 + 8 <= 256, "barrier block");
-static_assert(kOffX % 16 == 0 && kOffS % 16 == 0 && kSmemBytes <= 232448, "shared memory layout");
-static_assert(16 * 36 * 4 <= kStageWarp, "out staging fits the per-warp buffer");
+static_assert(kOffO % 1024 == 0 && 2 * 2 * 128 * 4 * 4 <= 2 * kOBox && kSmemBytes <= 232448,
+              "shared memory layout");
 
 struct SmaTcParams {
     CUtensorMap tmap_q;  // Q viewed as dims (N, B*L, H)
     CUtensorMap tmap_c;  // Cm viewed as dims (N, B*L)
     CUtensorMap tmap_h;  // dH viewed as dims (P, B*H*C*N)
+    CUtensorMap tmap_e;  // E viewed as dims (P, H, B*L), box (64, 1, 128): L2 prefetch only
+    CUtensorMap tmap_o;  // out viewed as dims (P, H, B*L) fp32, box (32, 1, 128): reduce-add / store
     const __nv_bfloat16* E;
     const float* y_ssd;
     float* out;
     float g;
+    int add_into_out;  // 1: out already holds y_ssd, the tile end adds g o / l; 0: it stores o / l
     int B, L, H, S, C;
     int tiles_per_chunk, total_tiles;
     int* status;
@@ -130,6 +137,8 @@ __global__ void __launch_bounds__(kThreads, 1) sma_tc_kernel(const __grid_consta
         tma_prefetch_desc(&p.tmap_q);
         tma_prefetch_desc(&p.tmap_c);
         tma_prefetch_desc(&p.tmap_h);
+        tma_prefetch_desc(&p.tmap_e);
+        tma_prefetch_desc(&p.tmap_o);
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_holder), kTmemCols);
@@ -181,16 +190,23 @@ __global__ void __launch_bounds__(kThreads, 1) sma_tc_kernel(const __grid_consta
                 mbar_expect_tx(bar(C_FULL), 2 * kHalfA);
                 tma_load_2d(sbase + kOffC, &p.tmap_c, bar(C_FULL), 0, row);
                 tma_load_2d(sbase + kOffC + kHalfA, &p.tmap_c, bar(C_FULL), 64, row);
-                // the next non-empty tile's Q and C rows start moving into L2 now
-                for (int in = i + gridDim.x; in < p.total_tiles; in += gridDim.x) {
-                    const Tile tn = decode_tile(p, in);
-                    if (tn.k == 0) continue;
+                // the next tile's rows start moving into L2 now: its Q and C
+                // (if it has memories), the E rows its epilogue starts from
+                // and the out rows (holding y_ssd) its output is added into
+                if (i + (int)gridDim.x < p.total_tiles) {
+                    const Tile tn = decode_tile(p, i + gridDim.x);
                     const int rown = tn.b * p.L + tn.t0;
-                    tma_prefetch_3d(&p.tmap_q, 0, rown, tn.h);
-                    tma_prefetch_3d(&p.tmap_q, 64, rown, tn.h);
-                    tma_prefetch_2d(&p.tmap_c, 0, rown);
-                    tma_prefetch_2d(&p.tmap_c, 64, rown);
-                    break;
+                    if (tn.k > 0) {
+                        tma_prefetch_3d(&p.tmap_q, 0, rown, tn.h);
+                        tma_prefetch_3d(&p.tmap_q, 64, rown, tn.h);
+                        tma_prefetch_2d(&p.tmap_c, 0, rown);
+                        tma_prefetch_2d(&p.tmap_c, 64, rown);
+                        tma_prefetch_3d(&p.tmap_e, 0, tn.h, rown);
+                    }
+                    if (p.add_into_out && tn.k > 0) {
+                        tma_prefetch_3d(&p.tmap_o, 0, tn.h, rown);
+                        tma_prefetch_3d(&p.tmap_o, 32, tn.h, rown);
+                    }
                 }
             }
             c_ph ^= 1;
@@ -264,8 +280,16 @@ __global__ void __launch_bounds__(kThreads, 1) sma_tc_kernel(const __grid_consta
         const int row = quad * 32 + lane;          // token row inside the tile
         const uint32_t t_lane = tmem + ((uint32_t)(quad * 32) << 16);
         const float sscale = kLog2e * rsqrtf((float)kN);
-        float* xbuf = reinterpret_cast<float*>(smem + kOffX);
-        uint8_t* stage = smem + kOffS + (uint32_t)(warp - 2) * kStageWarp;
+        float* xbuf = reinterpret_cast<float*>(smem + kOffO);
+        // this lane's row of the output tile: box `half`, row `row`, 128-byte swizzle
+        uint8_t* orow_s = smem + kOffO + (uint32_t)half * kOBox + (uint32_t)row * 128u;
+        const bool issuer = warp == 2 && lane == 0;  // issues the output tile's TMA operation
+        // The eight epilogue warps meet at named barrier 1 before the output
+        // tile is written, after it is written, and before the first score
+        // exchange of every tile (after the issuer saw the previous tile's
+        // TMA operation finish reading the tile).  All of them run every
+        // tile and batch, also after a failed wait.
+        auto tile_sync = [&]() { named_bar_sync(1, 32 * kEpiWarps); };
         int it_u = 0;
         bool ok = true;
         auto row_offset = [&](const Tile& t) -> size_t {
@@ -273,8 +297,7 @@ __global__ void __launch_bounds__(kThreads, 1) sma_tc_kernel(const __grid_consta
             return (tok * p.H + t.h) * kP + col0;
         };
         // This warp's 32 columns of E for the tile about to run, as packed
-        // bf16; the next tile's are fetched together with the y_ssd rows at
-        // the end of each tile, so that neither latency sits between tiles.
+        // bf16; the next tile's are fetched at the end of each tile.
         uint4 e_raw[kHalfP / 8];
         auto load_e = [&](int i) {
 #pragma unroll
@@ -287,20 +310,8 @@ __global__ void __launch_bounds__(kThreads, 1) sma_tc_kernel(const __grid_consta
             for (int q = 0; q < kHalfP / 8; ++q) e_raw[q] = __ldg(src + q);
         };
         load_e(blockIdx.x);
-        // Row-contiguous (coalesced) view of the warp's 32 x 32 block: in
-        // step i, lane l covers row (i * 32 + l) / kPerRow, piece l % kPerRow.
-        auto block_row = [&](const Tile& t, int r) -> size_t {
-            const size_t tok = (size_t)t.b * p.L + t.t0 + quad * 32 + r;
-            return (tok * p.H + t.h) * kP + col0;
-        };
         for (int i = blockIdx.x; i < p.total_tiles; i += gridDim.x) {
             const Tile t = decode_tile(p, i);
-            const size_t rowoff = row_offset(t);
-            if (i + (int)gridDim.x < p.total_tiles) {  // next tile's rows, on their way to L2
-                const size_t offn = row_offset(decode_tile(p, i + gridDim.x));
-                prefetch_l2(p.E + offn);
-                if (p.y_ssd) prefetch_l2(p.y_ssd + offn);
-            }
             float2 o2[kHalfP / 2];
 #pragma unroll
             for (int j = 0; j < kHalfP / 2; ++j) o2[j] = make_float2(0.f, 0.f);
@@ -346,6 +357,10 @@ __global__ void __launch_bounds__(kThreads, 1) sma_tc_kernel(const __grid_consta
                         __syncwarp();
                         if (lane == 0) mbar_arrive(bar(U_EMPTY));
                     }
+                    if (j == 0) {  // the exchange area is free once the last tile's output left it
+                        if (issuer) bulk_wait_read<0>();
+                        tile_sync();
+                    }
                     // scores: own partial + partner's partial
                     float* xs = xbuf + (((it_u & 1) * 2 + half) * 128 + row) * 4;
                     const float* xp = xbuf + (((it_u & 1) * 2 + (1 - half)) * 128 + row) * 4;
@@ -390,63 +405,48 @@ __global__ void __launch_bounds__(kThreads, 1) sma_tc_kernel(const __grid_consta
                 }
             }
             const float inv = t.k > 0 && l > 0.f ? 1.f / l : 0.f;
-            // Tile end.  Rows of out, y_ssd and E are 128 B / 64 B pieces 8 KB
-            // apart, so they move through the per-warp staging buffer in a
-            // row-contiguous order (4 or 8 rows per instruction) instead of
-            // one row per lane.  Every load is issued before the first store
-            // (out may alias y_ssd); each lane stores exactly the elements it
-            // loaded.
-            float4 yv[8];  // rows 4i + l/8, columns 4 (l % 8) ..
-#pragma unroll
-            for (int iy = 0; iy < 8; ++iy)
-                yv[iy] = p.y_ssd ? *reinterpret_cast<const float4*>(p.y_ssd + block_row(t, 4 * iy + lane / 8) + 4 * (lane % 8))
-                                : make_float4(0.f, 0.f, 0.f, 0.f);
-            const int inext = i + (int)gridDim.x;
-            const bool next_mem = inext < p.total_tiles && decode_tile(p, inext).k > 0;
-            uint4 en[4];   // next tile's E: rows 8i + l/4, columns 8 (l % 4) ..
+            // Tile end.  The next tile's E row goes out first (its latency
+            // overlaps the rest); then every lane writes g o / l of its row
+            // and 32 columns into the output tile and one thread hands the
+            // tile to the TMA unit, which adds it into out (holding y_ssd)
+            // or stores it.  No lane touches y_ssd or out itself.
+            const bool next_mem = i + (int)gridDim.x < p.total_tiles && decode_tile(p, i + gridDim.x).k > 0;
+            uint4 en[kHalfP / 8];
             if (next_mem) {
-                const Tile tn = decode_tile(p, inext);
+                const uint4* src = reinterpret_cast<const uint4*>(p.E + row_offset(decode_tile(p, i + gridDim.x)));
 #pragma unroll
-                for (int i2 = 0; i2 < 4; ++i2)
-                    en[i2] = __ldg(reinterpret_cast<const uint4*>(p.E + block_row(tn, 8 * i2 + lane / 4)) + (lane % 4));
+                for (int q = 0; q < kHalfP / 8; ++q) en[q] = __ldg(src + q);
+            } else {
+#pragma unroll
+                for (int q = 0; q < kHalfP / 8; ++q) en[q] = make_uint4(0u, 0u, 0u, 0u);
             }
-            const float gg = p.y_ssd ? p.g : 1.f;
-            float* st_f = reinterpret_cast<float*>(stage);
+            if (issuer) bulk_wait_read<0>();   // a tile without memories has no exchange step
+            tile_sync();                        // exchange area no longer read
+            const float gi = (p.add_into_out ? p.g : 1.f) * inv;
 #pragma unroll
-            for (int r2 = 0; r2 < 2; ++r2) {   // rows 16 r2 .. 16 r2 + 15
-                if ((lane >> 4) == r2) {
-                    float* dst = st_f + (lane & 15) * 36;
-#pragma unroll
-                    for (int q = 0; q < kHalfP / 4; ++q) {
-                        const float2 lo = o2[2 * q], hi = o2[2 * q + 1];
-                        *reinterpret_cast<float4*>(dst + 4 * q) =
-                            make_float4(gg * (lo.x * inv), gg * (lo.y * inv), gg * (hi.x * inv), gg * (hi.y * inv));
-                    }
+            for (int q = 0; q < kHalfP / 4; ++q) {
+                const float2 lo = o2[2 * q], hi = o2[2 * q + 1];
+                *reinterpret_cast<float4*>(orow_s + (((uint32_t)q ^ (uint32_t)(row & 7)) << 4)) =
+                    make_float4(gi * lo.x, gi * lo.y, gi * hi.x, gi * hi.y);
+            }
+            fence_proxy_async_smem();
+            tile_sync();
+            // (a tile without memories adds nothing: out already holds y_ssd there)
+            if (issuer && !*abort_flag && (t.k > 0 || !p.add_into_out)) {
+                const int tok0 = t.b * p.L + t.t0;
+                if (p.add_into_out) {
+                    tma_reduce_add_3d(&p.tmap_o, sbase + kOffO, 0, t.h, tok0);
+                    tma_reduce_add_3d(&p.tmap_o, sbase + kOffO + kOBox, 32, t.h, tok0);
+                } else {
+                    tma_store_3d(&p.tmap_o, sbase + kOffO, 0, t.h, tok0);
+                    tma_store_3d(&p.tmap_o, sbase + kOffO + kOBox, 32, t.h, tok0);
                 }
-                __syncwarp();
-#pragma unroll
-                for (int i2 = 0; i2 < 4; ++i2) {
-                    const int rr = 4 * i2 + lane / 8;
-                    const float4 a = *reinterpret_cast<const float4*>(st_f + rr * 36 + 4 * (lane % 8));
-                    const float4 yy = yv[4 * r2 + i2];
-                    if (ok)
-                        *reinterpret_cast<float4*>(p.out + block_row(t, 16 * r2 + rr) + 4 * (lane % 8)) =
-                            make_float4(a.x + yy.x, a.y + yy.y, a.z + yy.z, a.w + yy.w);
-                }
-                __syncwarp();
+                bulk_commit();
             }
 #pragma unroll
-            for (int q = 0; q < kHalfP / 8; ++q) e_raw[q] = make_uint4(0u, 0u, 0u, 0u);
-            if (next_mem) {
-#pragma unroll
-                for (int i2 = 0; i2 < 4; ++i2)
-                    *reinterpret_cast<uint4*>(stage + (8 * i2 + lane / 4) * 80 + (lane % 4) * 16) = en[i2];
-                __syncwarp();
-#pragma unroll
-                for (int q = 0; q < kHalfP / 8; ++q) e_raw[q] = *reinterpret_cast<const uint4*>(stage + lane * 80 + q * 16);
-                __syncwarp();
-            }
+            for (int q = 0; q < kHalfP / 8; ++q) e_raw[q] = en[q];
         }
+        if (issuer) bulk_wait<0>();  // out written before the CTA's shared memory goes away
     }
 
     tc_fence_before();
@@ -485,10 +485,30 @@ cudaError_t launch_sma_tc(const SmaArgs& a, cudaStream_t st) {
         const uint32_t box[2] = {kP, kN};
         if (!encode_tile_map_bf16(&p.tmap_h, 2, a.dH, dims, strides, box)) return cudaErrorInvalidValue;
     }
+    {
+        const uint64_t dims[3] = {(uint64_t)kP, (uint64_t)a.H, (uint64_t)a.B * a.L};
+        const uint64_t strides[2] = {(uint64_t)kP * 2, (uint64_t)a.H * kP * 2};
+        const uint32_t box[3] = {64, 1, kBQ};
+        if (!encode_tile_map_bf16(&p.tmap_e, 3, a.E, dims, strides, box)) return cudaErrorInvalidValue;
+    }
+    {
+        const uint64_t dims[3] = {(uint64_t)kP, (uint64_t)a.H, (uint64_t)a.B * a.L};
+        const uint64_t strides[2] = {(uint64_t)kP * 4, (uint64_t)a.H * kP * 4};
+        const uint32_t box[3] = {32, 1, kBQ};
+        if (!encode_tile_map_f32(&p.tmap_o, 3, a.out, dims, strides, box)) return cudaErrorInvalidValue;
+    }
     p.E = static_cast<const __nv_bfloat16*>(a.E);
     p.y_ssd = a.y_ssd;
     p.out = a.out;
     p.g = a.g;
+    // The kernel adds g o into out, so out must hold y_ssd first; with no
+    // y_ssd it stores o itself.
+    p.add_into_out = a.y_ssd != nullptr;
+    if (a.y_ssd && a.y_ssd != a.out) {
+        const size_t bytes = (size_t)a.B * a.L * a.H * kP * sizeof(float);
+        cudaError_t ce = cudaMemcpyAsync(a.out, a.y_ssd, bytes, cudaMemcpyDeviceToDevice, st);
+        if (ce != cudaSuccess) return ce;
+    }
     p.B = a.B; p.L = a.L; p.H = a.H; p.S = a.S; p.C = C;
     p.tiles_per_chunk = a.S / kBQ;
     p.total_tiles = C * a.B * a.H * p.tiles_per_chunk;

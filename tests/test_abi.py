@@ -107,6 +107,17 @@ def test_sma_rejects_bad_args(lib):
     assert rc == dart.DART_ERR_UNSUPPORTED
 
 
+def test_sma_rejects_partially_overlapping_out(lib):
+    """out must be y_ssd itself or disjoint from it."""
+    d = dart.Dims(1, 512, 2, 64, 128, 256, 1)
+    base = 1 << 32
+    y = ctypes.c_void_p(base)
+    rc = lib.dart_sma_forward(ctypes.byref(d), dart.DART_BF16, FAKE, FAKE, FAKE, FAKE, 0.5, y,
+                              ctypes.c_void_p(base + 4096), None)
+    assert rc == dart.DART_ERR_INVALID_ARG
+    assert b"overlaps" in lib.dart_last_error()
+
+
 def test_decode_rejects_bad_args(lib):
     d = dart.Dims(4, 0, 2, 64, 128, 256, 1)
     ws = lib.dart_decode_step_workspace_bytes(ctypes.byref(d), dart.DART_BF16, 9)

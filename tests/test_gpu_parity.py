@@ -237,6 +237,29 @@ def test_sma_on_shared_memories(orc):
     assert_close("o", o, ref["o"], TOL[torch.bfloat16])
 
 
+def test_sma_output_modes(orc):
+    """out = y_ssd + g o written three ways: in place over y_ssd, into a
+    separate buffer (y_ssd left untouched), and o alone without y_ssd."""
+    shape = LayerShape(2, 6 * 256, 3, 64, 128, 256, "bf16", "loguniform")
+    inp = synth.layer_inputs(shape, seed=21)
+    dH = synth.memory_inputs(2, 3, 6, 128, 64, "bf16", seed=21).cuda()
+    d = to_device(inp)
+    y_ssd = torch.randn(2, 6 * 256, 3, 64, generator=torch.Generator().manual_seed(21)).cuda()
+    oi = oracle_inputs(inp)
+    ref = orc.sma(oi["Q"], oi["E"], oi["Cm"], dH.float().cpu().numpy(), 256, 0.5, y_ssd.cpu().double().numpy())
+    keep = y_ssd.clone()
+    sep = dart.dart_sma_forward(d["Q"], d["E"], d["Cm"], dH, 256, 0.5, y_ssd)
+    assert torch.equal(y_ssd, keep)
+    inplace = y_ssd.clone()
+    dart.dart_sma_forward(d["Q"], d["E"], d["Cm"], dH, 256, 0.5, inplace, out=inplace)
+    o = dart.dart_sma_forward(d["Q"], d["E"], d["Cm"], dH, 256, 0.5)
+    dart.dart_sync_status()
+    assert_close("y (separate out)", sep, ref["y"], TOL[torch.bfloat16])
+    assert_close("y (in place)", inplace, ref["y"], TOL[torch.bfloat16])
+    assert_close("o", o, ref["o"], TOL[torch.bfloat16])
+    assert torch.equal(sep, inplace)
+
+
 def test_deterministic():
     shape = LayerShape(1, 4 * 256, 4, 64, 128, 256, "bf16", "loguniform")
     inp = synth.layer_inputs(shape, seed=13)
