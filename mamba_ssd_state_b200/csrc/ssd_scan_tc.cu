@@ -54,6 +54,7 @@ struct ScanTcParams {
     CUtensorMap tmap_hin;  // hin as (P, B*H*C*N), box (64, 128)
     CUtensorMap tmap_dh;   // dH as (P, B*H*C*N) bf16, box (64, 128): chunk_state's store
     CUtensorMap tmap_st;   // states as (P, B*H*C*N) fp32, box (32, 128): chunk_state's store
+    CUtensorMap tmap_y;    // y as (P, H, B*L) fp32, box (32, 1, 128): chunk_output's store
     const float* dt;
     const float* A;
     const float* init_state;
@@ -357,8 +358,9 @@ __global__ void __launch_bounds__(256) state_pass_tc_kernel(const __grid_constan
 // chunk_output_tc
 // ===========================================================================
 namespace co {
-constexpr int kWorkers = 256;
-constexpr int kThreads = 64 + kWorkers;  // warp 0 TMA, warp 1 MMA, warps 2-9 workers
+constexpr int kWorkers = 256;                  // warps 2-9 build P
+constexpr int kEpi = 128;                      // warps 10-13 write y
+constexpr int kThreads = 64 + kWorkers + kEpi; // warp 0 TMA, warp 1 MMA
 // Barrier slots.  The two-deep rings take two consecutive slots; P is built
 // and consumed in 64-column panels (at most four), each with its own
 // ready / free pair, so the tensor core starts on a panel while the workers
@@ -373,11 +375,11 @@ constexpr uint32_t kOffX = kOffBP + 4 * kBox;          // 2 buffers x (256 rows 
 constexpr uint32_t kXBytes = 2 * kBox;
 constexpr uint32_t kOffHp = kOffX + 2 * kXBytes;       // 2 buffers x 128 rows (16 KB)
 constexpr uint32_t kOffF = kOffHp + 2 * kBox;          // 2 buffers x (a2[256], colf[256])
-constexpr uint32_t kOffYs = kOffF + 2 * 2 * 256 * 4;   // per-worker-warp y staging: 16 rows x 36 floats
-constexpr uint32_t kYsWarp = 16 * 36 * 4;
-constexpr uint32_t kOffBar = kOffYs + 8 * kYsWarp;
+constexpr uint32_t kOffRs = kOffF + 2 * 2 * 256 * 4;  // row scales exp(Acum_t), ring of 4 heads x 256
+constexpr uint32_t kOffYs = kOffRs + 4 * 256 * 4;      // y staging: one box of 128 rows x 32 fp32 (16 KB)
+constexpr uint32_t kOffBar = kOffYs + kBox;
 constexpr uint32_t kBytes = kOffBar + NUM_BARS * 8 + 16 + 1024;
-static_assert(kOffYs % 16 == 0 && kBytes <= 232448, "chunk_output shared memory");
+static_assert(kOffYs % 1024 == 0 && kBytes <= 232448, "chunk_output shared memory");
 constexpr uint32_t kColDiag = 256, kColOff = 384;
 
 __global__ void __launch_bounds__(kThreads, 1) chunk_output_tc_kernel(const __grid_constant__ ScanTcParams p) {
@@ -412,7 +414,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_output_tc_kernel(const __gr
             mbar_init(bar(X_FULL0 + s), 1);
             mbar_init(bar(X_FREE0 + s), 1);
             mbar_init(bar(ACC_FULL0 + s), 1);
-            mbar_init(bar(ACC_EMPTY0 + s), kWorkers / 32);
+            mbar_init(bar(ACC_EMPTY0 + s), kEpi / 32);
         }
         for (int k = 0; k < kPanels; ++k) {
             mbar_init(bar(P_READY0 + k), kWorkers / 32);
@@ -534,8 +536,69 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_output_tc_kernel(const __gr
             }
             __syncwarp();
         }
+    } else if (warp >= 2 + kWorkers / 32) {
+        // --------------------------------------------------------- epilogue
+        // y = Y_diag + exp(Acum_t) Y_off for the head whose accumulators are
+        // ready, one box of 32 columns at a time: written 128-byte-swizzled
+        // into the staging area and stored by TMA.  The four warps run every
+        // box's named barriers, also after a failed wait (they then skip the
+        // work).
+        const int quad = warp & 3;
+        const int trow = quad * 32 + lane;
+        const int t = 128 * half + trow;
+        const uint32_t t_lane = tmem + ((uint32_t)(quad * 32) << 16);
+        const bool issuer = warp == 2 + kWorkers / 32 && lane == 0;
+        uint8_t* yrow = smem + kOffYs + (uint32_t)trow * kRowBytes;
+        const float* rs_s = reinterpret_cast<const float*>(smem + kOffRs);
+        bool ok = true;
+        for (int i = 0; i < p.HG; ++i) {
+            const int a = i & 1;
+            const uint32_t ph = (uint32_t)(i >> 1) & 1u;
+            if (ok) ok = mbar_wait_warp(bar(ACC_FULL0 + a), ph, wc, 8);
+            float yv[64];
+            if (ok) {
+                tc_fence_after();
+                // exp(Acum_t), left by the P builders: the decay terms in the x
+                // buffer may already belong to a later head
+                const float row_scale = rs_s[(i & 3) * 256 + t];
+#pragma unroll
+                for (int ch = 0; ch < 2; ++ch) {
+                    float yo[32];
+                    tmem_ld_32x32b_x32(t_lane + kColDiag + (uint32_t)a * 64 + (uint32_t)ch * 32, yv + 32 * ch);
+                    if (has_off) tmem_ld_32x32b_x32(t_lane + kColOff + (uint32_t)a * 64 + (uint32_t)ch * 32, yo);
+                    tmem_ld_wait();
+                    if (has_off) {
+#pragma unroll
+                        for (int q = 0; q < 32; ++q) yv[32 * ch + q] = fmaf(row_scale, yo[q], yv[32 * ch + q]);
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(ACC_EMPTY0 + a));
+            }
+            const int h = hg * p.HG + i;
+#pragma unroll
+            for (int ch = 0; ch < 2; ++ch) {
+                if (issuer) bulk_wait_read<0>();   // the previous box has left the staging area
+                named_bar_sync(1, kEpi);
+                if (ok) {
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        *reinterpret_cast<float4*>(yrow + ((q ^ (trow & 7)) << 4)) =
+                            make_float4(yv[32 * ch + 4 * q], yv[32 * ch + 4 * q + 1], yv[32 * ch + 4 * q + 2],
+                                        yv[32 * ch + 4 * q + 3]);
+                }
+                fence_proxy_async_smem();
+                named_bar_sync(1, kEpi);
+                if (issuer && !*abort_flag) {
+                    tma_store_3d(&p.tmap_y, sbase + kOffYs, 32 * ch, h, row0 + 128 * half);
+                    bulk_commit();
+                }
+            }
+        }
+        if (issuer) bulk_wait<0>();   // y written before the CTA's shared memory goes away
     } else {
-        // ---------------------------------------------------------- workers
+        // ---------------------------------------------------------- P build
         const int wk = warp - 2;                         // 0..7
         const int quad = warp & 3;                       // TMEM lane quadrant
         const int colhalf = wk >> 2;                     // which half of the columns
@@ -544,56 +607,6 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_output_tc_kernel(const __gr
         const uint32_t t_lane = tmem + ((uint32_t)(quad * 32) << 16);
         const int npanel = KS / 64;                      // 64-column panels of P; this warp builds
                                                          // block 2k + colhalf of panel k
-        float row_scale_prev = 0.f;
-        float* ys = reinterpret_cast<float*>(smem + kOffYs + (uint32_t)wk * kYsWarp);
-        auto epilogue = [&](int i, float row_scale) -> bool {
-            const int a = i & 1;
-            const uint32_t ph = (uint32_t)(i >> 1) & 1u;
-            if (!mbar_wait_warp(bar(ACC_FULL0 + a), ph, wc, 8)) return false;
-            tc_fence_after();
-            float yd[32], yo[32];
-            tmem_ld_32x32b_x32(t_lane + kColDiag + (uint32_t)a * 64 + (uint32_t)colhalf * 32, yd);
-            if (has_off) tmem_ld_32x32b_x32(t_lane + kColOff + (uint32_t)a * 64 + (uint32_t)colhalf * 32, yo);
-            tmem_ld_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(ACC_EMPTY0 + a));
-            // Rows of y are 256 B apart by H * 256 B: the warp's 32 x 32 block
-            // goes out through its staging buffer, 16 rows at a time, four
-            // rows per store instruction.
-            const int h = hg * p.HG + i;
-            float* ybase = p.y + (((size_t)row0 + 128 * half + 32 * quad + lane / 8) * p.H + h) * kP + colhalf * 32 +
-                           4 * (lane % 8);
-            const size_t ystep = (size_t)4 * p.H * kP;
-#pragma unroll
-            for (int r2 = 0; r2 < 2; ++r2) {
-                if ((lane >> 4) == r2) {
-                    float* dst = ys + (lane & 15) * 36;
-#pragma unroll
-                    for (int q = 0; q < 32; q += 4) {
-                        float4 r = make_float4(yd[q], yd[q + 1], yd[q + 2], yd[q + 3]);
-                        if (has_off) {
-                            r.x = fmaf(row_scale, yo[q], r.x);
-                            r.y = fmaf(row_scale, yo[q + 1], r.y);
-                            r.z = fmaf(row_scale, yo[q + 2], r.z);
-                            r.w = fmaf(row_scale, yo[q + 3], r.w);
-                        }
-                        *reinterpret_cast<float4*>(dst + q) = r;
-                    }
-                }
-                __syncwarp();
-#pragma unroll
-                for (int i2 = 0; i2 < 4; ++i2) {
-                    const int rr = 4 * i2 + lane / 8;
-                    *reinterpret_cast<float4*>(ybase + (4 * r2 + i2) * ystep) =
-                        *reinterpret_cast<const float4*>(ys + rr * 36 + 4 * (lane % 8));
-                }
-                __syncwarp();
-            }
-            return true;
-        };
-        // Every worker warp executes the same named barriers for every head,
-        // also after a failed wait (it then skips the work).
         bool ok = true;
         for (int i = 0; i < p.HG; ++i) {
             // decay terms of this head arrive with its x tile
@@ -603,7 +616,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_output_tc_kernel(const __gr
             const float* a2 = dec_s + xs * 512;
             const float* colf = a2 + 256;
             const float a2t = ok ? a2[t] : 0.f;
-            const float row_scale = exp2f(a2t);          // exp(Acum_t): decay from the chunk start
+            // The epilogue reads head i's row scale after head i's MMAs; the
+            // slot is rewritten by head i + 4, whose P build cannot start
+            // before the epilogue has released head i's accumulators.
+            if (colhalf == 0) reinterpret_cast<float*>(smem + kOffRs)[(i & 3) * 256 + t] = exp2f(a2t);
             const int warp_tmin = 128 * half + 32 * quad;        // first row of this warp
             const int warp_tmax = warp_tmin + 31;                // last row of this warp
             for (int k = 0; k < npanel; ++k) {
@@ -663,10 +679,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_output_tc_kernel(const __gr
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(P_READY0 + k));
             }
-            if (ok && i > 0) ok = epilogue(i - 1, row_scale_prev);
-            row_scale_prev = row_scale;
         }
-        if (ok) epilogue(p.HG - 1, row_scale_prev);
     }
 
     tc_fence_before();
@@ -706,6 +719,12 @@ bool make_maps(const ScanArgs& a, ScanTcParams& p) {
         const uint64_t strides[1] = {(uint64_t)kP * 4};
         const uint32_t box[2] = {32, 128};
         if (!encode_tile_map_f32(&p.tmap_st, 2, a.states, dims, strides, box)) return false;
+    }
+    {
+        const uint64_t dims[3] = {(uint64_t)kP, (uint64_t)a.H, BL};
+        const uint64_t strides[2] = {(uint64_t)kP * 4, (uint64_t)a.H * kP * 4};
+        const uint32_t box[3] = {32, 1, 128};
+        if (!encode_tile_map_f32(&p.tmap_y, 3, a.y, dims, strides, box)) return false;
     }
     return true;
 }
