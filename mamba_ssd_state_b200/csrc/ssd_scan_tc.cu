@@ -127,8 +127,24 @@ __global__ void __launch_bounds__(256) chunk_decay_kernel(const __grid_constant_
 // ===========================================================================
 namespace cs {
 constexpr int kThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 workers
-enum Bar { B_FULL = 0, X_FULL0, X_EMPTY0 = X_FULL0 + 2, W_READY0 = X_EMPTY0 + 2, ACC_FULL0 = W_READY0 + 2,
-           ACC_EMPTY0 = ACC_FULL0 + 2, NUM_BARS = ACC_EMPTY0 + 2 };
+enum Bar { B_FULL = 0, B_FREE = 1, X_FULL0 = 2, X_EMPTY0 = X_FULL0 + 2, W_READY0 = X_EMPTY0 + 2,
+           ACC_FULL0 = W_READY0 + 2, ACC_EMPTY0 = ACC_FULL0 + 2, NUM_BARS = ACC_EMPTY0 + 2 };
+static_assert(NUM_BARS == 12, "chunk_state barrier slots");
+
+// Work items (b, c, h) in that order, h fastest; consecutive items of one
+// (b, c) share the chunk's B tile.  CTA r of G takes items
+// [r T / G, (r + 1) T / G): equal shares, and the B tile is reloaded only
+// where the range crosses into the next chunk.
+struct Item {
+    int b, c, h;
+};
+__device__ __forceinline__ Item cs_item(const ScanTcParams& p, int j) {
+    Item it;
+    it.h = j % p.H;
+    it.c = (j / p.H) % p.C;
+    it.b = j / (p.H * p.C);
+    return it;
+}
 
 template <int S>
 struct Layout {
@@ -155,14 +171,14 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_state_tc_kernel(const __gri
     auto bar = [&](int i) -> uint32_t { return sbase + Ly::kOffBar + 8u * (uint32_t)i; };
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    const int ngroups = p.H / p.HG;
-    const int hg = blockIdx.x % ngroups;
-    const int c = (blockIdx.x / ngroups) % p.C;
-    const int b = blockIdx.x / (ngroups * p.C);
-    const int row0 = b * p.L + c * S;  // first token of the chunk in the (B*L) row space
+    const int total = p.B * p.C * p.H;
+    const int j0 = (int)((long long)blockIdx.x * total / gridDim.x);
+    const int j1 = (int)((long long)(blockIdx.x + 1) * total / gridDim.x);
+    const int n_items = j1 - j0;
 
     if (threadIdx.x == 0) {
         mbar_init(bar(B_FULL), 1);
+        mbar_init(bar(B_FREE), 1);
         for (int s = 0; s < 2; ++s) {
             mbar_init(bar(X_FULL0 + s), 1);
             mbar_init(bar(X_EMPTY0 + s), 1);
@@ -188,25 +204,33 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_state_tc_kernel(const __gri
         if (lane == 0) {
             tma_prefetch_desc(&p.tmap_x);
             tma_prefetch_desc(&p.tmap_b);
-            mbar_expect_tx(bar(B_FULL), 2 * S * kRowBytes);
-            for (int pnl = 0; pnl < 2; ++pnl)
-                for (int r = 0; r < S / 128; ++r)
-                    tma_load_2d(sbase + Ly::kOffB + (uint32_t)pnl * S * kRowBytes + (uint32_t)r * kBox, &p.tmap_b,
-                                bar(B_FULL), 64 * pnl, row0 + 128 * r);
         }
-        __syncwarp();
-        for (int i = 0; i < p.HG; ++i) {
+        int b_loads = 0;
+        for (int i = 0; i < n_items; ++i) {
+            const Item it = cs_item(p, j0 + i);
+            const int row0 = it.b * p.L + it.c * S;   // first token of the chunk in the (B*L) row space
+            if (i == 0 || it.h == 0) {
+                // a new chunk: its B tile, once the MMAs on the previous one are done
+                if (b_loads > 0 && !mbar_wait_warp(bar(B_FREE), (uint32_t)(b_loads - 1) & 1u, wc, 7)) break;
+                if (lane == 0) {
+                    mbar_expect_tx(bar(B_FULL), 2 * S * kRowBytes);
+                    for (int pnl = 0; pnl < 2; ++pnl)
+                        for (int r = 0; r < S / 128; ++r)
+                            tma_load_2d(sbase + Ly::kOffB + (uint32_t)pnl * S * kRowBytes + (uint32_t)r * kBox,
+                                        &p.tmap_b, bar(B_FULL), 64 * pnl, row0 + 128 * r);
+                }
+                ++b_loads;
+            }
             const int xs = i & 1;
             const uint32_t ph = (uint32_t)(i >> 1) & 1u;
             if (!mbar_wait_warp(bar(X_EMPTY0 + xs), ph ^ 1u, wc, 1)) break;
             if (lane == 0) {
-                const int h = hg * p.HG + i;
                 mbar_expect_tx(bar(X_FULL0 + xs), Ly::kXBytes + S * 4);
                 for (int r = 0; r < S / 128; ++r)
                     tma_load_3d(sbase + Ly::kOffX + (uint32_t)xs * Ly::kXBytes + (uint32_t)r * kBox, &p.tmap_x,
-                                bar(X_FULL0 + xs), 0, row0 + 128 * r, h);
-                bulk_load(sbase + Ly::kOffF + (uint32_t)xs * S * 4, p.wst + (((size_t)b * p.H + h) * p.C + c) * S,
-                          S * 4, bar(X_FULL0 + xs));
+                                bar(X_FULL0 + xs), 0, row0 + 128 * r, it.h);
+                bulk_load(sbase + Ly::kOffF + (uint32_t)xs * S * 4,
+                          p.wst + (((size_t)it.b * p.H + it.h) * p.C + it.c) * S, S * 4, bar(X_FULL0 + xs));
             }
             __syncwarp();
         }
@@ -214,8 +238,16 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_state_tc_kernel(const __gri
         // MMA: D[n, p] = sum_s B[s, n] W[s, p]: A = B^T (MN-major, M = n over
         // two 64-wide panels), B = W (MN-major), K = s.  Lane 0 issues.
         const uint32_t idesc = idesc_bf16_f32(128, kP, true, true);
-        bool ok = mbar_wait_warp(bar(B_FULL), 0, wc, 2);
-        for (int i = 0; i < p.HG && ok; ++i) {
+        bool ok = true;
+        int b_loads = 0;
+        for (int i = 0; i < n_items && ok; ++i) {
+            const Item it = cs_item(p, j0 + i);
+            if (i == 0 || it.h == 0) {
+                if (!(ok = mbar_wait_warp(bar(B_FULL), (uint32_t)b_loads & 1u, wc, 2))) break;
+                ++b_loads;
+            }
+            // the last item on this B tile releases it after its MMAs
+            const bool last_on_b = i + 1 == n_items || it.h == p.H - 1;
             const int xs = i & 1, a = i & 1;
             const uint32_t ph = (uint32_t)(i >> 1) & 1u;
             if (!(ok = mbar_wait_warp(bar(W_READY0 + xs), ph, wc, 3))) break;
@@ -231,6 +263,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_state_tc_kernel(const __gri
                 }
                 mma_commit(bar(ACC_FULL0 + a));
                 mma_commit(bar(X_EMPTY0 + xs));
+                if (last_on_b) mma_commit(bar(B_FREE));
             }
             __syncwarp();
         }
@@ -280,8 +313,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_state_tc_kernel(const __gri
             fence_proxy_async_smem();
             named_bar_sync(1, 128);
             if (wi == 0 && !*abort_flag) {
-                const int h = hg * p.HG + i;
-                const int row = (((b * p.H + h) * p.C + c) * kN);
+                const Item it = cs_item(p, j0 + i);
+                const int row = (((it.b * p.H + it.h) * p.C + it.c) * kN);
                 tma_store_2d(&p.tmap_dh, smem_u32(out_s), 0, row);
                 tma_store_2d(&p.tmap_st, smem_u32(out_s + kBox), 0, row);
                 tma_store_2d(&p.tmap_st, smem_u32(out_s + 2 * kBox), 32, row);
@@ -290,7 +323,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_state_tc_kernel(const __gri
             return live;
         };
         bool ok = true;
-        for (int i = 0; i < p.HG; ++i) {
+        for (int i = 0; i < n_items; ++i) {
             // scale the x tile in place: row s of the panel times wst_s
             const int xs = i & 1;
             const uint32_t ph = (uint32_t)(i >> 1) & 1u;
@@ -313,7 +346,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_state_tc_kernel(const __gri
             }
             if (i > 0) ok = epilogue(i - 1, ok);
         }
-        epilogue(p.HG - 1, ok);
+        if (n_items > 0) epilogue(n_items - 1, ok);
         if (wi == 0) bulk_wait<0>();  // stores complete before the CTA's shared memory goes away
     }
 
@@ -771,9 +804,12 @@ cudaError_t launch_ssd_scan_tc(const ScanArgs& a, cudaStream_t st) {
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     // 1. chunk memories
-    p.HG = pick_group(a.H, 8);
     {
-        const int grid = a.B * p.C * (a.H / p.HG);
+        // persistent: one CTA per SM, equal shares of the (b, c, h) items
+        const int sms = sm_count();
+        if (sms <= 0) return cudaErrorInvalidDevice;
+        const int items = a.B * p.C * a.H;
+        const int grid = items < sms ? items : sms;
         if (a.S == 256) {
             auto k = cs::chunk_state_tc_kernel<256>;
             const uint32_t smem = cs::Layout<256>::kBytes;
