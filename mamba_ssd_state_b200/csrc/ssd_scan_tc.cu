@@ -46,6 +46,7 @@ using namespace sm100;
 constexpr int kN = 128, kP = 64;
 constexpr uint32_t kRowBytes = 128;                  // one 64-element bf16 row of a swizzle panel
 constexpr uint32_t kBox = 128 * kRowBytes;           // a 128-row TMA box, 16 KB
+constexpr int kScanMaxCtas = 160;                    // largest persistent grid (one CTA per SM)
 
 struct ScanTcParams {
     CUtensorMap tmap_x;    // x  as (P, B*L, H), box (64, 128, 1)
@@ -70,7 +71,8 @@ struct ScanTcParams {
     float* a2;
     float* colf;
     float* wst;
-    int B, L, H, S, C, HG;
+    int B, L, H, S, C;
+    int co_range[kScanMaxCtas + 1];  // chunk_output: CTA r runs items co_range[r] .. co_range[r + 1] - 1
     int* status;
 };
 
@@ -397,23 +399,42 @@ constexpr int kThreads = 64 + kWorkers + kEpi; // warp 0 TMA, warp 1 MMA
 // Barrier slots.  The two-deep rings take two consecutive slots; P is built
 // and consumed in 64-column panels (at most four), each with its own
 // ready / free pair, so the tensor core starts on a panel while the workers
-// build the next one.
+// build the next one.  A group (b, c, half) shares C rows, B rows and G:
+// GRP_FREE releases C, B and P after the group's last MMAs, G_FREE releases
+// G after the P builders' last reads of it.
 constexpr int kPanels = 4;
-enum Bar { IN_FULL = 0, G_FULL = 1, X_FULL0 = 2, X_FREE0 = 4, P_READY0 = 6, P_FREE0 = P_READY0 + kPanels,
-           ACC_FULL0 = P_FREE0 + kPanels, ACC_EMPTY0 = ACC_FULL0 + 2, NUM_BARS = ACC_EMPTY0 + 2 };
-static_assert(X_FREE0 >= X_FULL0 + 2 && P_READY0 >= X_FREE0 + 2 && NUM_BARS == 18, "barrier slots overlap");
+enum Bar { IN_FULL = 0, G_FULL = 1, G_FREE = 2, GRP_FREE = 3, X_FULL0 = 4, X_FREE0 = 6, P_READY0 = 8,
+           P_FREE0 = P_READY0 + kPanels, ACC_FULL0 = P_FREE0 + kPanels, ACC_EMPTY0 = ACC_FULL0 + 2,
+           NUM_BARS = ACC_EMPTY0 + 2 };
+static_assert(NUM_BARS == 20, "barrier slots overlap");
 constexpr uint32_t kOffC = 0;                          // C rows: 2 panels x 128 rows (32 KB)
 constexpr uint32_t kOffBP = 2 * kBox;                  // B rows (2 panels x KS rows), later P (KS/64 panels x 128 rows)
 constexpr uint32_t kOffX = kOffBP + 4 * kBox;          // 2 buffers x (256 rows x 128 B)
 constexpr uint32_t kXBytes = 2 * kBox;
 constexpr uint32_t kOffHp = kOffX + 2 * kXBytes;       // 2 buffers x 128 rows (16 KB)
 constexpr uint32_t kOffF = kOffHp + 2 * kBox;          // 2 buffers x (a2[256], colf[256])
-constexpr uint32_t kOffRs = kOffF + 2 * 2 * 256 * 4;  // row scales exp(Acum_t), ring of 4 heads x 256
+constexpr uint32_t kOffRs = kOffF + 2 * 2 * 256 * 4;  // row scales exp(Acum_t), ring of 4 items x 256
 constexpr uint32_t kOffYs = kOffRs + 4 * 256 * 4;      // y staging: one box of 128 rows x 32 fp32 (16 KB)
 constexpr uint32_t kOffBar = kOffYs + kBox;
 constexpr uint32_t kBytes = kOffBar + NUM_BARS * 8 + 16 + 1024;
 static_assert(kOffYs % 1024 == 0 && kBytes <= 232448, "chunk_output shared memory");
 constexpr uint32_t kColDiag = 256, kColOff = 384;
+
+// Work items (b, c, half, h), h fastest.  The items of one (b, c, half)
+// form a group.  CTA r runs items co_range[r] .. co_range[r + 1] - 1.
+struct Item {
+    int b, c, half, h;
+};
+__device__ __forceinline__ Item co_item(const ScanTcParams& p, int j) {
+    const int R = p.S / 128;
+    const int g = j / p.H;
+    Item it;
+    it.h = j % p.H;
+    it.half = g % R;
+    it.c = (g / R) % p.C;
+    it.b = g / (R * p.C);
+    return it;
+}
 
 __global__ void __launch_bounds__(kThreads, 1) chunk_output_tc_kernel(const __grid_constant__ ScanTcParams p) {
     extern __shared__ uint8_t smem_raw[];
@@ -424,25 +445,17 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_output_tc_kernel(const __gr
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
     auto bar = [&](int i) -> uint32_t { return sbase + kOffBar + 8u * (uint32_t)i; };
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-    // CTA -> (b, c, half, head group); the heavier second halves come first
     const int S = p.S;
-    const int R = S / 128;
-    const int ngroups = p.H / p.HG;
-    int idx = blockIdx.x;
-    const int per_half = p.B * p.C * ngroups;
-    const int half = (R - 1) - idx / per_half;
-    idx %= per_half;
-    const int hg = idx % ngroups;
-    const int c = (idx / ngroups) % p.C;
-    const int b = idx / (ngroups * p.C);
-    const int KS = 128 * (half + 1);               // source tokens this half depends on
-    const int row0 = b * p.L + c * S;              // first token of the chunk
-    const bool has_off = (c > 0) || (p.init_state != nullptr);
+    const int j0 = p.co_range[blockIdx.x];
+    const int n_items = p.co_range[blockIdx.x + 1] - j0;
+    auto group_first = [&](int i, const Item& it) { return i == 0 || it.h == 0; };
+    auto group_last = [&](int i, const Item& it) { return i + 1 == n_items || it.h == p.H - 1; };
 
     if (threadIdx.x == 0) {
         mbar_init(bar(IN_FULL), 1);
         mbar_init(bar(G_FULL), 1);
+        mbar_init(bar(G_FREE), kWorkers / 32);
+        mbar_init(bar(GRP_FREE), 1);
         for (int s = 0; s < 2; ++s) {
             mbar_init(bar(X_FULL0 + s), 1);
             mbar_init(bar(X_FREE0 + s), 1);
@@ -467,66 +480,85 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_output_tc_kernel(const __gr
 
     const WaitCtx wc{abort_flag, p.status, 3};
     if (warp == 0) {
-        // TMA: the whole warp walks the heads, lane 0 issues
+        // TMA: the whole warp walks the items, lane 0 issues
         if (lane == 0) {
             tma_prefetch_desc(&p.tmap_x);
             tma_prefetch_desc(&p.tmap_b);
             tma_prefetch_desc(&p.tmap_c);
             tma_prefetch_desc(&p.tmap_hin);
-            // C rows of this half (A of G and of Y_off) and B rows 0..KS-1 (B of G)
-            mbar_expect_tx(bar(IN_FULL), 2 * kBox + 2 * (uint32_t)KS * kRowBytes);
-            for (int pnl = 0; pnl < 2; ++pnl) {
-                tma_load_2d(sbase + kOffC + (uint32_t)pnl * kBox, &p.tmap_c, bar(IN_FULL), 64 * pnl,
-                            row0 + 128 * half);
-                for (int r = 0; r < KS / 128; ++r)
-                    tma_load_2d(sbase + kOffBP + (uint32_t)pnl * KS * kRowBytes + (uint32_t)r * kBox, &p.tmap_b,
-                                bar(IN_FULL), 64 * pnl, row0 + 128 * r);
-            }
         }
-        __syncwarp();
-        for (int i = 0; i < p.HG; ++i) {
+        int ng = 0;  // groups loaded so far
+        for (int i = 0; i < n_items; ++i) {
+            const Item it = co_item(p, j0 + i);
+            const int KS = 128 * (it.half + 1);            // source tokens this half depends on
+            const int row0 = it.b * p.L + it.c * S;        // first token of the chunk
+            const bool has_off = (it.c > 0) || (p.init_state != nullptr);
+            if (group_first(i, it)) {
+                // C rows of this half (A of G and of Y_off) and B rows 0..KS-1 (B of G),
+                // once the previous group's MMAs are done with C, B and P
+                if (ng > 0 && !mbar_wait_warp(bar(GRP_FREE), (uint32_t)(ng - 1) & 1u, wc, 10)) break;
+                if (lane == 0) {
+                    mbar_expect_tx(bar(IN_FULL), 2 * kBox + 2 * (uint32_t)KS * kRowBytes);
+                    for (int pnl = 0; pnl < 2; ++pnl) {
+                        tma_load_2d(sbase + kOffC + (uint32_t)pnl * kBox, &p.tmap_c, bar(IN_FULL), 64 * pnl,
+                                    row0 + 128 * it.half);
+                        for (int r = 0; r < KS / 128; ++r)
+                            tma_load_2d(sbase + kOffBP + (uint32_t)pnl * KS * kRowBytes + (uint32_t)r * kBox,
+                                        &p.tmap_b, bar(IN_FULL), 64 * pnl, row0 + 128 * r);
+                    }
+                }
+                ++ng;
+            }
             const int xs = i & 1;
             const uint32_t ph = (uint32_t)(i >> 1) & 1u;
-            const int h = hg * p.HG + i;
             if (!mbar_wait_warp(bar(X_FREE0 + xs), ph ^ 1u, wc, 1)) break;
             if (lane == 0) {
                 const uint32_t bytes = (uint32_t)KS * kRowBytes + (has_off ? kBox : 0u) + 2u * KS * 4u;
                 mbar_expect_tx(bar(X_FULL0 + xs), bytes);
-                const size_t drow = (((size_t)b * p.H + h) * p.C + c) * S;   // this (b, h, c) in the decay arrays
+                const size_t drow = (((size_t)it.b * p.H + it.h) * p.C + it.c) * S;   // (b, h, c) in the decay arrays
                 bulk_load(sbase + kOffF + (uint32_t)xs * 2048, p.a2 + drow, KS * 4, bar(X_FULL0 + xs));
                 bulk_load(sbase + kOffF + (uint32_t)xs * 2048 + 1024, p.colf + drow, KS * 4, bar(X_FULL0 + xs));
                 for (int r = 0; r < KS / 128; ++r)
                     tma_load_3d(sbase + kOffX + (uint32_t)xs * kXBytes + (uint32_t)r * kBox, &p.tmap_x,
-                                bar(X_FULL0 + xs), 0, row0 + 128 * r, h);
+                                bar(X_FULL0 + xs), 0, row0 + 128 * r, it.h);
                 if (has_off)
                     tma_load_2d(sbase + kOffHp + (uint32_t)xs * kBox, &p.tmap_hin, bar(X_FULL0 + xs), 0,
-                                ((b * p.H + h) * p.C + c) * kN);
+                                ((it.b * p.H + it.h) * p.C + it.c) * kN);
             }
             __syncwarp();
         }
     } else if (warp == 1) {
-        // MMA: lane 0 issues, the whole warp walks the heads
-        bool ok = mbar_wait_warp(bar(IN_FULL), 0, wc, 2);
-        if (ok) {
-            // G[t, s] = sum_n C[t, n] B[s, n]: both K-major, K = N.
-            tc_fence_after();
-            if (lane == 0) {
-                const uint32_t idesc_g = idesc_bf16_f32(128, KS, false, false);
-#pragma unroll
-                for (int kk = 0; kk < kN / 16; ++kk) {
-                    const uint32_t koff = (uint32_t)(kk & 3) * 32;   // 16 K-elements inside a panel
-                    const uint64_t ad = smem_desc_sw128(sbase + kOffC + (uint32_t)(kk >> 2) * kBox + koff, 16, 1024);
-                    const uint64_t bd = smem_desc_sw128(
-                        sbase + kOffBP + (uint32_t)(kk >> 2) * (uint32_t)KS * kRowBytes + koff, 16, 1024);
-                    mma_f16_ss(tmem, ad, bd, idesc_g, kk > 0 ? 1u : 0u);
-                }
-                mma_commit(bar(G_FULL));
-            }
-            __syncwarp();
-        }
+        // MMA: lane 0 issues, the whole warp walks the items
         const uint32_t idesc_y = idesc_bf16_f32(128, kP, false, true);
-        const int npanel = KS / 64;
-        for (int i = 0; i < p.HG && ok; ++i) {
+        bool ok = true;
+        int ng = 0;
+        uint32_t ready_par = 0;  // bit k: parity of the next P_READY(k) completion
+        for (int i = 0; i < n_items && ok; ++i) {
+            const Item it = co_item(p, j0 + i);
+            const int KS = 128 * (it.half + 1);
+            const int npanel = KS / 64;
+            const bool has_off = (it.c > 0) || (p.init_state != nullptr);
+            if (group_first(i, it)) {
+                // G[t, s] = sum_n C[t, n] B[s, n]: both K-major, K = N; written over the
+                // previous group's G once the P builders are done reading it
+                if (!(ok = mbar_wait_warp(bar(IN_FULL), (uint32_t)ng & 1u, wc, 2))) break;
+                if (ng > 0 && !(ok = mbar_wait_warp(bar(G_FREE), (uint32_t)(ng - 1) & 1u, wc, 11))) break;
+                tc_fence_after();
+                if (lane == 0) {
+                    const uint32_t idesc_g = idesc_bf16_f32(128, KS, false, false);
+#pragma unroll
+                    for (int kk = 0; kk < kN / 16; ++kk) {
+                        const uint32_t koff = (uint32_t)(kk & 3) * 32;   // 16 K-elements inside a panel
+                        const uint64_t ad = smem_desc_sw128(sbase + kOffC + (uint32_t)(kk >> 2) * kBox + koff, 16, 1024);
+                        const uint64_t bd = smem_desc_sw128(
+                            sbase + kOffBP + (uint32_t)(kk >> 2) * (uint32_t)KS * kRowBytes + koff, 16, 1024);
+                        mma_f16_ss(tmem, ad, bd, idesc_g, kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(bar(G_FULL));
+                }
+                __syncwarp();
+                ++ng;
+            }
             const int xs = i & 1, a = i & 1;
             const uint32_t ph = (uint32_t)(i >> 1) & 1u;
             if (!(ok = mbar_wait_warp(bar(X_FULL0 + xs), ph, wc, 5))) break;
@@ -548,7 +580,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_output_tc_kernel(const __gr
             // one 64-column panel of P at a time
             const uint32_t xbase = sbase + kOffX + (uint32_t)xs * kXBytes;
             for (int k = 0; k < npanel && ok; ++k) {
-                if (!(ok = mbar_wait_warp(bar(P_READY0 + k), (uint32_t)i & 1u, wc, 3))) break;
+                if (!(ok = mbar_wait_warp(bar(P_READY0 + k), (ready_par >> k) & 1u, wc, 3))) break;
+                ready_par ^= 1u << k;
                 tc_fence_after();
                 if (lane == 0) {
 #pragma unroll
@@ -566,25 +599,27 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_output_tc_kernel(const __gr
             if (lane == 0) {
                 mma_commit(bar(ACC_FULL0 + a));
                 mma_commit(bar(X_FREE0 + xs));
+                if (group_last(i, it)) mma_commit(bar(GRP_FREE));
             }
             __syncwarp();
         }
     } else if (warp >= 2 + kWorkers / 32) {
         // --------------------------------------------------------- epilogue
-        // y = Y_diag + exp(Acum_t) Y_off for the head whose accumulators are
+        // y = Y_diag + exp(Acum_t) Y_off for the item whose accumulators are
         // ready, one box of 32 columns at a time: written 128-byte-swizzled
         // into the staging area and stored by TMA.  The four warps run every
         // box's named barriers, also after a failed wait (they then skip the
         // work).
         const int quad = warp & 3;
         const int trow = quad * 32 + lane;
-        const int t = 128 * half + trow;
         const uint32_t t_lane = tmem + ((uint32_t)(quad * 32) << 16);
         const bool issuer = warp == 2 + kWorkers / 32 && lane == 0;
         uint8_t* yrow = smem + kOffYs + (uint32_t)trow * kRowBytes;
         const float* rs_s = reinterpret_cast<const float*>(smem + kOffRs);
         bool ok = true;
-        for (int i = 0; i < p.HG; ++i) {
+        for (int i = 0; i < n_items; ++i) {
+            const Item it = co_item(p, j0 + i);
+            const bool has_off = (it.c > 0) || (p.init_state != nullptr);
             const int a = i & 1;
             const uint32_t ph = (uint32_t)(i >> 1) & 1u;
             if (ok) ok = mbar_wait_warp(bar(ACC_FULL0 + a), ph, wc, 8);
@@ -592,8 +627,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_output_tc_kernel(const __gr
             if (ok) {
                 tc_fence_after();
                 // exp(Acum_t), left by the P builders: the decay terms in the x
-                // buffer may already belong to a later head
-                const float row_scale = rs_s[(i & 3) * 256 + t];
+                // buffer may already belong to a later item
+                const float row_scale = rs_s[(i & 3) * 256 + 128 * it.half + trow];
 #pragma unroll
                 for (int ch = 0; ch < 2; ++ch) {
                     float yo[32];
@@ -609,7 +644,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_output_tc_kernel(const __gr
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(ACC_EMPTY0 + a));
             }
-            const int h = hg * p.HG + i;
+            const int row0 = it.b * p.L + it.c * S;
 #pragma unroll
             for (int ch = 0; ch < 2; ++ch) {
                 if (issuer) bulk_wait_read<0>();   // the previous box has left the staging area
@@ -624,7 +659,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_output_tc_kernel(const __gr
                 fence_proxy_async_smem();
                 named_bar_sync(1, kEpi);
                 if (issuer && !*abort_flag) {
-                    tma_store_3d(&p.tmap_y, sbase + kOffYs, 32 * ch, h, row0 + 128 * half);
+                    tma_store_3d(&p.tmap_y, sbase + kOffYs, 32 * ch, it.h, row0 + 128 * it.half);
                     bulk_commit();
                 }
             }
@@ -636,30 +671,41 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_output_tc_kernel(const __gr
         const int quad = warp & 3;                       // TMEM lane quadrant
         const int colhalf = wk >> 2;                     // which half of the columns
         const int trow = quad * 32 + lane;               // row inside the half (TMEM lane)
-        const int t = 128 * half + trow;                 // chunk-local token of this row
         const uint32_t t_lane = tmem + ((uint32_t)(quad * 32) << 16);
-        const int npanel = KS / 64;                      // 64-column panels of P; this warp builds
-                                                         // block 2k + colhalf of panel k
+        float* rs_w = reinterpret_cast<float*>(smem + kOffRs);
         bool ok = true;
-        for (int i = 0; i < p.HG; ++i) {
-            // decay terms of this head arrive with its x tile
+        int ng = 0;
+        uint32_t free_cnt = 0;  // bit k: parity of the P_FREE(k) commits made for earlier items
+        for (int i = 0; i < n_items; ++i) {
+            const Item it = co_item(p, j0 + i);
+            const int KS = 128 * (it.half + 1);
+            const int npanel = KS / 64;                  // 64-column panels of P; this warp builds
+                                                         // block 2k + colhalf of panel k
+            const int t = 128 * it.half + trow;          // chunk-local token of this row
+            const bool first = group_first(i, it);
+            // decay terms of this item arrive with its x tile
             const int xs = i & 1;
             const uint32_t ph = (uint32_t)(i >> 1) & 1u;
             if (ok) ok = mbar_wait_warp(bar(X_FULL0 + xs), ph, wc, 9);
             const float* a2 = dec_s + xs * 512;
             const float* colf = a2 + 256;
             const float a2t = ok ? a2[t] : 0.f;
-            // The epilogue reads head i's row scale after head i's MMAs; the
-            // slot is rewritten by head i + 4, whose P build cannot start
-            // before the epilogue has released head i's accumulators.
-            if (colhalf == 0) reinterpret_cast<float*>(smem + kOffRs)[(i & 3) * 256 + t] = exp2f(a2t);
-            const int warp_tmin = 128 * half + 32 * quad;        // first row of this warp
+            // The epilogue reads item i's row scale after item i's MMAs; the
+            // slot is rewritten by item i + 4, whose P build cannot start
+            // before the epilogue has released item i's accumulators.
+            if (colhalf == 0) rs_w[(i & 3) * 256 + t] = exp2f(a2t);
+            // a new group's P may be written once its G is in TMEM (the P
+            // buffer held its B rows until then)
+            if (first) {
+                if (ok) ok = mbar_wait_warp(bar(G_FULL), (uint32_t)ng & 1u, wc, 6);
+                ++ng;
+            }
+            const int warp_tmin = 128 * it.half + 32 * quad;     // first row of this warp
             const int warp_tmax = warp_tmin + 31;                // last row of this warp
             for (int k = 0; k < npanel; ++k) {
-                // panel k may be written once G (first head) or the previous
-                // head's MMA on that panel has consumed the buffer
-                if (ok) ok = (i == 0) ? mbar_wait_warp(bar(G_FULL), 0, wc, 6)
-                                      : mbar_wait_warp(bar(P_FREE0 + k), (uint32_t)(i - 1) & 1u, wc, 7);
+                // within a group, panel k may be written once the previous
+                // item's MMA on it is done
+                if (ok && !first) ok = mbar_wait_warp(bar(P_FREE0 + k), ((free_cnt >> k) & 1u) ^ 1u, wc, 7);
                 if (!ok) break;
                 tc_fence_after();
                 const int j = 2 * k + colhalf;
@@ -699,7 +745,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_output_tc_kernel(const __gr
 #pragma unroll
                     for (int q = 0; q < 16; ++q) packed[q] = 0u;
                 }
-                // row trow of panel j/2, 16-byte chunks (j%2)*4 .. +3, 128-byte swizzle
+                // row trow of panel k, 16-byte chunks colhalf*4 .. +3, 128-byte swizzle
                 uint8_t* prow = smem + kOffBP + (uint32_t)k * kBox + (uint32_t)trow * kRowBytes;
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
@@ -712,6 +758,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_output_tc_kernel(const __gr
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(P_READY0 + k));
             }
+            free_cnt ^= (1u << npanel) - 1u;   // the MMA commits P_FREE(k) once for this item, k < npanel
+            // after the group's last item the P builders are done with its G
+            if (group_last(i, it) && lane == 0) mbar_arrive(bar(G_FREE));
         }
     }
 
@@ -760,12 +809,6 @@ bool make_maps(const ScanArgs& a, ScanTcParams& p) {
         if (!encode_tile_map_f32(&p.tmap_y, 3, a.y, dims, strides, box)) return false;
     }
     return true;
-}
-
-int pick_group(int H, int want) {
-    int g = want < H ? want : H;
-    while (H % g) --g;
-    return g;
 }
 
 }  // namespace
@@ -829,9 +872,31 @@ cudaError_t launch_ssd_scan_tc(const ScanArgs& a, cudaStream_t st) {
     state_pass_tc_kernel<<<dim3(kN * kP / 4 / 256, a.H, a.B), 256, 0, st>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     // 3. outputs
-    p.HG = pick_group(a.H, 16);
     {
-        const int grid = a.B * p.C * (a.H / p.HG) * (a.S / 128);
+        // persistent: one CTA per SM, contiguous ranges of the (b, c, half, h)
+        // items with equal estimated work.  An item of the second half (256
+        // source tokens) costs about 4/3 of one of the first; a group change
+        // (C and B rows, G) about as much as one item.
+        const int sms = sm_count();
+        if (sms <= 0) return cudaErrorInvalidDevice;
+        const int R = a.S / 128;
+        const int items = a.B * p.C * R * a.H;
+        int grid = sms < kScanMaxCtas ? sms : kScanMaxCtas;
+        if (items < grid) grid = items;
+        auto cost = [&](int j) {
+            const int half = (j / a.H) % R;
+            return (half == 0 ? 3 : 4) + (j % a.H == 0 ? 3 : 0);
+        };
+        long long total = 0;
+        for (int j = 0; j < items; ++j) total += cost(j);
+        long long acc = 0;
+        int r = 1;
+        p.co_range[0] = 0;
+        for (int j = 0; j < items && r < grid; ++j) {
+            acc += cost(j);
+            while (r < grid && acc * grid >= total * r) p.co_range[r++] = j + 1;
+        }
+        while (r <= grid) p.co_range[r++] = items;
         if ((e = cudaFuncSetAttribute(co::chunk_output_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)co::kBytes)) != cudaSuccess)
             return e;
