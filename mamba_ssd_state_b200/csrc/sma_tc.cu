@@ -28,8 +28,16 @@
 // the columns halves the epilogue's time per batch, which is what keeps the
 // MMA fed.  The grid is persistent: CTA i takes tiles i, i+G, ... of a list
 // ordered from the most memories to the fewest, so the triangular work
-// spreads evenly; each tile prefetches the next tile's E and y_ssd rows into
-// L2.
+// spreads evenly.
+//
+// CTA pairs (S a multiple of 256): two CTAs of a cluster run the two
+// 128-token halves of a 256-token tile as one M = 256 MMA (tcgen05 with
+// cta_group::2).  Each CTA loads its own Q and C rows and two of the four
+// memories of a batch (its half of N), so the 128 KB memory ring holds four
+// stages instead of two and each SM streams half the memory bytes; CTA 0
+// issues the MMAs and owns the FULL / EMPTY barriers they wait on, the
+// peer's loads complete on them and its epilogue warps arrive on them
+// remotely; the commits reach both CTAs.  S = 128 runs one CTA per tile.
 #include <cuda_bf16.h>
 #include <string.h>
 
@@ -45,19 +53,29 @@ using namespace sm100;
 constexpr int kN = 128, kP = 64;   // compiled shape
 constexpr int kBQ = 128;           // query tokens per tile (MMA M)
 constexpr int kCB = 4;             // chunk memories per MMA (N = 4 * P = 256)
-constexpr int kNB = 2;             // stages of the memory ring
 constexpr uint32_t kHalfA = 128 * 64 * 2;        // 128 rows x 64 bf16 (one swizzle panel)
 constexpr uint32_t kMemBytes = kN * kP * 2;       // one chunk memory, 16 KB
 constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffC = 2 * kHalfA;
 constexpr uint32_t kOffB = 4 * kHalfA;
-constexpr uint32_t kStageBytes = kCB * kMemBytes;
+constexpr uint32_t kRingBytes = 2 * kCB * kMemBytes;   // the memory ring: 128 KB
+// Ring geometry.  A single CTA holds all four memories of a batch (two
+// stages of 64 KB); in a CTA pair each CTA holds two of them (its half of
+// the MMA's N columns), so the same 128 KB give four stages.
+template <bool kPair>
+struct Ring {
+    static constexpr int kMem = kPair ? 2 : 4;
+    static constexpr int kStages = kPair ? 4 : 2;
+    static constexpr uint32_t kStageBytes = kMem * kMemBytes;
+    static_assert(kStages * kStageBytes == kRingBytes, "ring size");
+};
+constexpr int kMaxStages = 4;
 // Output tile: at a tile end the gated attention output g o / l of the 128
 // rows, as two 128-byte-swizzled boxes of 32 fp32 columns (the layout of the
 // out tensor map), added into out (which holds y_ssd) by a TMA reduction.
 // While a tile runs, its first 8 KB hold the partial-score exchange
 // [2 parity][2 half][128 rows][4].
-constexpr uint32_t kOffO = kOffB + kNB * kStageBytes;
+constexpr uint32_t kOffO = kOffB + kRingBytes;
 constexpr uint32_t kOBox = 128 * 32 * 4;              // one box: 128 rows x 32 fp32
 constexpr uint32_t kOffBar = kOffO + 2 * kOBox;
 constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;  // + alignment slack
@@ -69,7 +87,7 @@ constexpr int kHalfP = kP / 2;                        // value columns per epilo
 
 // Barrier slots (explicit; the memory ring takes consecutive slots).
 enum Bar { Q_FULL = 0, Q_FREE = 1, C_FULL = 2, C_FREE = 3, U_FULL = 4, U_EMPTY = 5, V_FULL = 6, V_EMPTY = 7,
-           B_FULL0 = 8, B_EMPTY0 = B_FULL0 + kNB, NUM_BARS = B_EMPTY0 + kNB };
+           B_FULL0 = 8, B_EMPTY0 = B_FULL0 + kMaxStages, NUM_BARS = B_EMPTY0 + kMaxStages };
 static_assert(NUM_BARS * 8 + 8 <= 256, "barrier block");
 static_assert(kOffO % 1024 == 0 && 2 * 2 * 128 * 4 * 4 <= 2 * kOBox && kSmemBytes <= 232448,
               "shared memory layout");
@@ -86,6 +104,7 @@ struct SmaTcParams {
     float g;
     int add_into_out;  // 1: out already holds y_ssd, the tile end adds g o / l; 0: it stores o / l
     int B, L, H, S, C;
+    int cta_per_tile;  // 1, or 2 for a CTA pair (each CTA 128 of the tile's 256 rows)
     int tiles_per_chunk, total_tiles;
     int* status;
 };
@@ -95,7 +114,8 @@ struct Tile {
 };
 
 // Tile list ordered by decreasing chunk index (most memories first).
-__device__ __forceinline__ Tile decode_tile(const SmaTcParams& p, int i) {
+// `rank` picks this CTA's 128 rows of a pair tile.
+__device__ __forceinline__ Tile decode_tile(const SmaTcParams& p, int i, int rank) {
     const int per_k = p.B * p.H * p.tiles_per_chunk;
     Tile t;
     t.k = p.C - 1 - i / per_k;
@@ -104,11 +124,13 @@ __device__ __forceinline__ Tile decode_tile(const SmaTcParams& p, int i) {
     const int bh = r / p.tiles_per_chunk;
     t.b = bh / p.H;
     t.h = bh % p.H;
-    t.t0 = t.k * p.S + sub * kBQ;
+    t.t0 = t.k * p.S + (sub * p.cta_per_tile + rank) * kBQ;
     return t;
 }
 
+template <bool kPair>
 __global__ void __launch_bounds__(kThreads, 1) sma_tc_kernel(const __grid_constant__ SmaTcParams p) {
+    using Rg = Ring<kPair>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
@@ -116,6 +138,12 @@ __global__ void __launch_bounds__(kThreads, 1) sma_tc_kernel(const __grid_consta
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
     auto bar = [&](int i) -> uint32_t { return sbase + kOffBar + 8u * (uint32_t)i; };
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // A pair tile is run by both CTAs of a cluster; CTA 0 issues the MMAs
+    // and owns the FULL / EMPTY barriers they wait on.
+    const int rank = kPair ? (int)cluster_ctarank() : 0;
+    const int tile0 = kPair ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+    const int tstride = kPair ? (int)(gridDim.x >> 1) : (int)gridDim.x;
+    auto bar_lead = [&](int i) -> uint32_t { return kPair ? mapa_shared(bar(i), 0) : bar(i); };
 
     if (threadIdx.x == 0) {
         mbar_init(bar(Q_FULL), 1);
@@ -123,10 +151,10 @@ __global__ void __launch_bounds__(kThreads, 1) sma_tc_kernel(const __grid_consta
         mbar_init(bar(C_FULL), 1);
         mbar_init(bar(C_FREE), 1);
         mbar_init(bar(U_FULL), 1);
-        mbar_init(bar(U_EMPTY), kEpiWarps);
+        mbar_init(bar(U_EMPTY), kEpiWarps * (kPair ? 2 : 1));
         mbar_init(bar(V_FULL), 1);
-        mbar_init(bar(V_EMPTY), kEpiWarps);
-        for (int s = 0; s < kNB; ++s) {
+        mbar_init(bar(V_EMPTY), kEpiWarps * (kPair ? 2 : 1));
+        for (int s = 0; s < Rg::kStages; ++s) {
             mbar_init(bar(B_FULL0 + s), 1);
             mbar_init(bar(B_EMPTY0 + s), 1);
         }
@@ -141,11 +169,19 @@ __global__ void __launch_bounds__(kThreads, 1) sma_tc_kernel(const __grid_consta
         tma_prefetch_desc(&p.tmap_o);
     }
     if (warp == 1) {
-        tmem_alloc(smem_u32(tmem_holder), kTmemCols);
-        tmem_relinquish();
+        if (kPair) {
+            tmem_alloc_pair(smem_u32(tmem_holder), kTmemCols);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(smem_u32(tmem_holder), kTmemCols);
+            tmem_relinquish();
+        }
     }
     tc_fence_before();
-    __syncthreads();
+    if (kPair)
+        cluster_sync();  // both CTAs' barriers exist before any remote arrive or copy
+    else
+        __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
 
@@ -158,21 +194,29 @@ __global__ void __launch_bounds__(kThreads, 1) sma_tc_kernel(const __grid_consta
         bool ok = true;
         auto load_b = [&](const Tile& t, int j) -> bool {
             const int nv = min(kCB, t.k - kCB * j);
-            const int s = it_b % kNB;
-            const uint32_t ph = (uint32_t)(it_b / kNB) & 1u;
+            const int s = it_b % Rg::kStages;
+            const uint32_t ph = (uint32_t)(it_b / Rg::kStages) & 1u;
             if (!mbar_wait_warp(bar(B_EMPTY0 + s), ph ^ 1, wc, 3)) return false;
             if (lane == 0) {
-                mbar_expect_tx(bar(B_FULL0 + s), (uint32_t)nv * kMemBytes);
-                const int mem_row = ((t.b * p.H + t.h) * p.C + kCB * j) * kN;
-                for (int q = 0; q < nv; ++q)
-                    tma_load_2d(sbase + kOffB + (uint32_t)s * kStageBytes + (uint32_t)q * kMemBytes, &p.tmap_h,
-                                bar(B_FULL0 + s), 0, mem_row + q * kN);
+                // this CTA's memories of the batch: all four, or its two of a pair
+                const int q0 = Rg::kMem * rank;
+                const int mine = max(0, min(Rg::kMem, nv - q0));
+                if (rank == 0) mbar_expect_tx(bar(B_FULL0 + s), (uint32_t)nv * kMemBytes);
+                const int mem_row = ((t.b * p.H + t.h) * p.C + kCB * j + q0) * kN;
+                const uint32_t dst = sbase + kOffB + (uint32_t)s * Rg::kStageBytes;
+                for (int q = 0; q < mine; ++q) {
+                    if (kPair)
+                        tma_load_2d_pair(dst + (uint32_t)q * kMemBytes, &p.tmap_h, bar_lead(B_FULL0 + s), 0,
+                                         mem_row + q * kN);
+                    else
+                        tma_load_2d(dst + (uint32_t)q * kMemBytes, &p.tmap_h, bar(B_FULL0 + s), 0, mem_row + q * kN);
+                }
             }
             ++it_b;
             return true;
         };
-        for (int i = blockIdx.x; i < p.total_tiles && ok; i += gridDim.x) {
-            const Tile t = decode_tile(p, i);
+        for (int i = tile0; i < p.total_tiles && ok; i += tstride) {
+            const Tile t = decode_tile(p, i, rank);
             if (t.k == 0) continue;
             const int row = t.b * p.L + t.t0;
             // The first memories of this tile go out before its Q and C: their
@@ -180,21 +224,31 @@ __global__ void __launch_bounds__(kThreads, 1) sma_tc_kernel(const __grid_consta
             if (!(ok = load_b(t, 0))) break;
             if (!(ok = mbar_wait_warp(bar(Q_FREE), q_ph ^ 1, wc, 1))) break;
             if (lane == 0) {
-                mbar_expect_tx(bar(Q_FULL), 2 * kHalfA);
-                tma_load_3d(sbase + kOffQ, &p.tmap_q, bar(Q_FULL), 0, row, t.h);
-                tma_load_3d(sbase + kOffQ + kHalfA, &p.tmap_q, bar(Q_FULL), 64, row, t.h);
+                if (rank == 0) mbar_expect_tx(bar(Q_FULL), 2 * kHalfA * (kPair ? 2 : 1));
+                if (kPair) {
+                    tma_load_3d_pair(sbase + kOffQ, &p.tmap_q, bar_lead(Q_FULL), 0, row, t.h);
+                    tma_load_3d_pair(sbase + kOffQ + kHalfA, &p.tmap_q, bar_lead(Q_FULL), 64, row, t.h);
+                } else {
+                    tma_load_3d(sbase + kOffQ, &p.tmap_q, bar(Q_FULL), 0, row, t.h);
+                    tma_load_3d(sbase + kOffQ + kHalfA, &p.tmap_q, bar(Q_FULL), 64, row, t.h);
+                }
             }
             q_ph ^= 1;
             if (!(ok = mbar_wait_warp(bar(C_FREE), c_ph ^ 1, wc, 2))) break;
             if (lane == 0) {
-                mbar_expect_tx(bar(C_FULL), 2 * kHalfA);
-                tma_load_2d(sbase + kOffC, &p.tmap_c, bar(C_FULL), 0, row);
-                tma_load_2d(sbase + kOffC + kHalfA, &p.tmap_c, bar(C_FULL), 64, row);
+                if (rank == 0) mbar_expect_tx(bar(C_FULL), 2 * kHalfA * (kPair ? 2 : 1));
+                if (kPair) {
+                    tma_load_2d_pair(sbase + kOffC, &p.tmap_c, bar_lead(C_FULL), 0, row);
+                    tma_load_2d_pair(sbase + kOffC + kHalfA, &p.tmap_c, bar_lead(C_FULL), 64, row);
+                } else {
+                    tma_load_2d(sbase + kOffC, &p.tmap_c, bar(C_FULL), 0, row);
+                    tma_load_2d(sbase + kOffC + kHalfA, &p.tmap_c, bar(C_FULL), 64, row);
+                }
                 // the next tile's rows start moving into L2 now: its Q and C
                 // (if it has memories), the E rows its epilogue starts from
                 // and the out rows (holding y_ssd) its output is added into
-                if (i + (int)gridDim.x < p.total_tiles) {
-                    const Tile tn = decode_tile(p, i + gridDim.x);
+                if (i + tstride < p.total_tiles) {
+                    const Tile tn = decode_tile(p, i + tstride, rank);
                     const int rown = tn.b * p.L + tn.t0;
                     if (tn.k > 0) {
                         tma_prefetch_3d(&p.tmap_q, 0, rown, tn.h);
@@ -215,14 +269,28 @@ __global__ void __launch_bounds__(kThreads, 1) sma_tc_kernel(const __grid_consta
                 if (!(ok = load_b(t, j))) break;
             __syncwarp();
         }
-    } else if (warp == 1) {
+    } else if (warp == 1 && rank == 0) {
         // ------------------------------------------------------------ MMA
-        // The whole warp walks the schedule; lane 0 issues the MMAs.
+        // The whole warp walks the schedule; lane 0 issues the MMAs (in a
+        // pair, the leader's for both CTAs: M = 256, N = 256 with each CTA
+        // supplying its two memories, commits reaching both CTAs).
         uint32_t q_ph = 0, c_ph = 0;
         int it_b = 0, it_u = 0;
         bool ok = true;
-        for (int i = blockIdx.x; i < p.total_tiles && ok; i += gridDim.x) {
-            const Tile t = decode_tile(p, i);
+        auto mma = [&](uint32_t d, uint64_t ad, uint64_t bd, uint32_t idesc, uint32_t acc) {
+            if (kPair)
+                mma_f16_ss_pair(d, ad, bd, idesc, acc);
+            else
+                mma_f16_ss(d, ad, bd, idesc, acc);
+        };
+        auto commit = [&](int b) {
+            if (kPair)
+                mma_commit_pair(bar(b));
+            else
+                mma_commit(bar(b));
+        };
+        for (int i = tile0; i < p.total_tiles && ok; i += tstride) {
+            const Tile t = decode_tile(p, i, rank);
             if (t.k == 0) continue;
             if (!(ok = mbar_wait_warp(bar(Q_FULL), q_ph, wc, 4))) break;
             q_ph ^= 1;
@@ -230,10 +298,13 @@ __global__ void __launch_bounds__(kThreads, 1) sma_tc_kernel(const __grid_consta
             const int nbatch = (t.k + kCB - 1) / kCB;
             for (int j = 0; j < nbatch; ++j, ++it_b, ++it_u) {
                 const int nv = min(kCB, t.k - kCB * j);
-                const int s = it_b % kNB;
-                const uint32_t ph = (uint32_t)(it_b / kNB) & 1u;
-                const uint32_t idesc = idesc_bf16_f32(kBQ, kP * nv, false, true);
-                const uint32_t b_base = sbase + kOffB + (uint32_t)s * kStageBytes;
+                const int s = it_b % Rg::kStages;
+                const uint32_t ph = (uint32_t)(it_b / Rg::kStages) & 1u;
+                // a pair always multiplies all four column blocks (the epilogue
+                // reads only the nv valid ones); N splits evenly over the CTAs
+                const uint32_t idesc = kPair ? idesc_bf16_f32(2 * kBQ, kP * kCB, false, true)
+                                             : idesc_bf16_f32(kBQ, kP * nv, false, true);
+                const uint32_t b_base = sbase + kOffB + (uint32_t)s * Rg::kStageBytes;
                 if (!(ok = mbar_wait_warp(bar(B_FULL0 + s), ph, wc, 5))) break;
                 if (!(ok = mbar_wait_warp(bar(U_EMPTY), ((uint32_t)it_u & 1u) ^ 1u, wc, 6))) break;
                 tc_fence_after();
@@ -242,10 +313,10 @@ __global__ void __launch_bounds__(kThreads, 1) sma_tc_kernel(const __grid_consta
                     for (int kk = 0; kk < kN / 16; ++kk) {
                         const uint64_t ad = smem_desc_sw128(sbase + kOffQ + (uint32_t)(kk >> 2) * kHalfA + (uint32_t)(kk & 3) * 32, 16, 1024);
                         const uint64_t bd = smem_desc_sw128(b_base + (uint32_t)kk * 2048, kMemBytes, 1024);
-                        mma_f16_ss(tmem, ad, bd, idesc, kk > 0 ? 1u : 0u);
+                        mma(tmem, ad, bd, idesc, kk > 0 ? 1u : 0u);
                     }
-                    mma_commit(bar(U_FULL));
-                    if (j == nbatch - 1) mma_commit(bar(Q_FREE));
+                    commit(U_FULL);
+                    if (j == nbatch - 1) commit(Q_FREE);
                 }
                 __syncwarp();
                 if (j == 0) {
@@ -259,16 +330,16 @@ __global__ void __launch_bounds__(kThreads, 1) sma_tc_kernel(const __grid_consta
                     for (int kk = 0; kk < kN / 16; ++kk) {
                         const uint64_t ad = smem_desc_sw128(sbase + kOffC + (uint32_t)(kk >> 2) * kHalfA + (uint32_t)(kk & 3) * 32, 16, 1024);
                         const uint64_t bd = smem_desc_sw128(b_base + (uint32_t)kk * 2048, kMemBytes, 1024);
-                        mma_f16_ss(tmem + kColV, ad, bd, idesc, kk > 0 ? 1u : 0u);
+                        mma(tmem + kColV, ad, bd, idesc, kk > 0 ? 1u : 0u);
                     }
-                    mma_commit(bar(V_FULL));
-                    mma_commit(bar(B_EMPTY0 + s));
-                    if (j == nbatch - 1) mma_commit(bar(C_FREE));
+                    commit(V_FULL);
+                    commit(B_EMPTY0 + s);
+                    if (j == nbatch - 1) commit(C_FREE);
                 }
                 __syncwarp();
             }
         }
-    } else {
+    } else if (warp >= 2) {
         // ------------------------------------------------------- epilogue
         // Warp pair (w, w+4) shares TMEM lane quadrant w & 3 (32 token rows);
         // warp half h owns value columns [32h, 32h+32) of every memory.  Both
@@ -303,15 +374,15 @@ __global__ void __launch_bounds__(kThreads, 1) sma_tc_kernel(const __grid_consta
 #pragma unroll
             for (int q = 0; q < kHalfP / 8; ++q) e_raw[q] = make_uint4(0u, 0u, 0u, 0u);
             if (i >= p.total_tiles) return;
-            const Tile t = decode_tile(p, i);
+            const Tile t = decode_tile(p, i, rank);
             if (t.k == 0) return;
             const uint4* src = reinterpret_cast<const uint4*>(p.E + row_offset(t));
 #pragma unroll
             for (int q = 0; q < kHalfP / 8; ++q) e_raw[q] = __ldg(src + q);
         };
-        load_e(blockIdx.x);
-        for (int i = blockIdx.x; i < p.total_tiles; i += gridDim.x) {
-            const Tile t = decode_tile(p, i);
+        load_e(tile0);
+        for (int i = tile0; i < p.total_tiles; i += tstride) {
+            const Tile t = decode_tile(p, i, rank);
             float2 o2[kHalfP / 2];
 #pragma unroll
             for (int j = 0; j < kHalfP / 2; ++j) o2[j] = make_float2(0.f, 0.f);
@@ -355,7 +426,12 @@ __global__ void __launch_bounds__(kThreads, 1) sma_tc_kernel(const __grid_consta
                         }
                         tc_fence_before();
                         __syncwarp();
-                        if (lane == 0) mbar_arrive(bar(U_EMPTY));
+                        if (lane == 0) {
+                            if (kPair)
+                                mbar_arrive_cluster(bar_lead(U_EMPTY));
+                            else
+                                mbar_arrive(bar(U_EMPTY));
+                        }
                     }
                     if (j == 0) {  // the exchange area is free once the last tile's output left it
                         if (issuer) bulk_wait_read<0>();
@@ -400,7 +476,12 @@ __global__ void __launch_bounds__(kThreads, 1) sma_tc_kernel(const __grid_consta
                         }
                         tc_fence_before();
                         __syncwarp();
-                        if (lane == 0) mbar_arrive(bar(V_EMPTY));
+                        if (lane == 0) {
+                            if (kPair)
+                                mbar_arrive_cluster(bar_lead(V_EMPTY));
+                            else
+                                mbar_arrive(bar(V_EMPTY));
+                        }
                     }
                 }
             }
@@ -410,10 +491,10 @@ __global__ void __launch_bounds__(kThreads, 1) sma_tc_kernel(const __grid_consta
             // and 32 columns into the output tile and one thread hands the
             // tile to the TMA unit, which adds it into out (holding y_ssd)
             // or stores it.  No lane touches y_ssd or out itself.
-            const bool next_mem = i + (int)gridDim.x < p.total_tiles && decode_tile(p, i + gridDim.x).k > 0;
+            const bool next_mem = i + tstride < p.total_tiles && decode_tile(p, i + tstride, rank).k > 0;
             uint4 en[kHalfP / 8];
             if (next_mem) {
-                const uint4* src = reinterpret_cast<const uint4*>(p.E + row_offset(decode_tile(p, i + gridDim.x)));
+                const uint4* src = reinterpret_cast<const uint4*>(p.E + row_offset(decode_tile(p, i + tstride, rank)));
 #pragma unroll
                 for (int q = 0; q < kHalfP / 8; ++q) en[q] = __ldg(src + q);
             } else {
@@ -450,10 +531,16 @@ __global__ void __launch_bounds__(kThreads, 1) sma_tc_kernel(const __grid_consta
     }
 
     tc_fence_before();
-    __syncthreads();
+    if (kPair)
+        cluster_sync();  // neither CTA leaves while the other may still reach its memory
+    else
+        __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, kTmemCols);
+        if (kPair)
+            tmem_dealloc_pair(tmem, kTmemCols);
+        else
+            tmem_dealloc(tmem, kTmemCols);
     }
 }
 
@@ -510,15 +597,48 @@ cudaError_t launch_sma_tc(const SmaArgs& a, cudaStream_t st) {
         if (ce != cudaSuccess) return ce;
     }
     p.B = a.B; p.L = a.L; p.H = a.H; p.S = a.S; p.C = C;
-    p.tiles_per_chunk = a.S / kBQ;
-    p.total_tiles = C * a.B * a.H * p.tiles_per_chunk;
     p.status = a.status;
     const int sms = sm_count();
     if (sms <= 0) return cudaErrorInvalidDevice;
-    const int grid = p.total_tiles < sms ? p.total_tiles : sms;
-    cudaError_t e = cudaFuncSetAttribute(sma_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
-    if (e != cudaSuccess) return e;
-    sma_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(p);
+    cudaError_t e;
+    if (a.S % (2 * kBQ) == 0) {
+        // CTA pairs: each pair tile covers 256 query rows of one (b, h, chunk)
+        p.cta_per_tile = 2;
+        p.tiles_per_chunk = a.S / (2 * kBQ);
+        p.total_tiles = C * a.B * a.H * p.tiles_per_chunk;
+        auto kern = sma_tc_kernel<true>;
+        if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes)) != cudaSuccess)
+            return e;
+        cudaLaunchConfig_t cfg;
+        memset(&cfg, 0, sizeof(cfg));
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.blockDim = dim3(kThreads, 1, 1);
+        cfg.dynamicSmemBytes = kSmemBytes;
+        cfg.stream = st;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        // as many pairs as can be resident at once (not every SM need pair up)
+        cfg.gridDim = dim3(2 * (unsigned)(sms / 2), 1, 1);
+        int clusters = 0;
+        if ((e = cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg)) != cudaSuccess) return e;
+        if (clusters <= 0) return cudaErrorInvalidConfiguration;
+        if (clusters > p.total_tiles) clusters = p.total_tiles;
+        cfg.gridDim = dim3(2 * (unsigned)clusters, 1, 1);
+        if ((e = cudaLaunchKernelEx(&cfg, kern, p)) != cudaSuccess) return e;
+    } else {
+        p.cta_per_tile = 1;
+        p.tiles_per_chunk = a.S / kBQ;
+        p.total_tiles = C * a.B * a.H * p.tiles_per_chunk;
+        const int grid = p.total_tiles < sms ? p.total_tiles : sms;
+        auto kern = sma_tc_kernel<false>;
+        if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes)) != cudaSuccess)
+            return e;
+        kern<<<grid, kThreads, kSmemBytes, st>>>(p);
+    }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     count_launches(1);
     return cudaSuccess;
