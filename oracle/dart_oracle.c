@@ -47,7 +47,10 @@
  *
  * Readings where the pages are silent: mask c < k(t) (strict), scale 1/sqrt(N),
  * exp(dt*A) discretisation with input dt*B x^T, no D skip, ngroups = 1 (B and C
- * shared by all heads), o_t = 0 with no memory.
+ * shared by all heads), o_t = 0 with no memory.  A sequence length that is not
+ * a multiple of S ends in a partial chunk: C = ceil(L / S) chunks, the last
+ * one closing at token L-1 (its dH and state are what a decode would carry
+ * on from); no token attends to it, since its own tokens have k(t) = C-1.
  *
  * Layouts (row-major, last index fastest):
  *   x[B,L,H,P] dt[B,L,H] A[H] Bm[B,L,N] Cm[B,L,N] Q[B,L,H,N] E[B,L,H,P]
@@ -118,7 +121,7 @@ static void scan_unit(void* vctx, int unit) {
     scan_ctx* c = (scan_ctx*)vctx;
     const oracle_dims* d = c->d;
     const int L = d->seqlen, H = d->nheads, P = d->headdim, N = d->dstate, S = d->chunk;
-    const int nchunks = L / S;
+    const int nchunks = (L + S - 1) / S; /* the last chunk may be partial */
     const int b = unit / H, h = unit % H;
     double* Hs = (double*)calloc((size_t)N * P, sizeof(double)); /* recurrent state  */
     double* D = (double*)calloc((size_t)N * P, sizeof(double));  /* chunk contribution */
@@ -147,7 +150,7 @@ static void scan_unit(void* vctx, int unit) {
             for (int n = 0; n < N; ++n) acc += (double)Ct[n] * Hs[n * P + p];
             yt[p] = acc;
         }
-        if (t % S == S - 1) {
+        if (t % S == S - 1 || t == L - 1) { /* the chunk's last token (a partial chunk ends at L-1) */
             const int ck = t / S;
             const size_t off = (((size_t)b * H + h) * nchunks + ck) * (size_t)N * P;
             if (c->dH) memcpy(c->dH + off, D, sizeof(double) * (size_t)N * P);
@@ -162,7 +165,7 @@ static void scan_unit(void* vctx, int unit) {
 int oracle_ssd_scan(const oracle_dims* d, const float* x, const float* dt, const float* A,
                     const float* Bm, const float* Cm, const double* init_state,
                     double* y_ssd, double* dH, double* states, int nthreads) {
-    if (!d || d->chunk <= 0 || d->seqlen % d->chunk != 0) return -1;
+    if (!d || d->chunk <= 0 || d->seqlen <= 0) return -1;
     scan_ctx c = {d, x, dt, A, Bm, Cm, init_state, y_ssd, dH, states};
     run_units(scan_unit, &c, d->batch * d->nheads, nthreads);
     return 0;
@@ -188,7 +191,7 @@ static void sma_unit(void* vctx, int unit) {
     sma_ctx* c = (sma_ctx*)vctx;
     const oracle_dims* d = c->d;
     const int L = d->seqlen, H = d->nheads, P = d->headdim, N = d->dstate, S = d->chunk;
-    const int nchunks = L / S;
+    const int nchunks = (L + S - 1) / S;
     const int b = unit / H, h = unit % H;
     const int nrows = c->tokens ? c->ntok : L;
     double* key = (double*)malloc(sizeof(double) * (size_t)N);
@@ -261,7 +264,7 @@ static void sma_unit(void* vctx, int unit) {
 int oracle_sma(const oracle_dims* d, const float* Q, const float* E, const float* Cm,
                const double* dH, double g, const double* y_ssd, double* o, double* y,
                double* scores, const int* tokens, int ntok, int nthreads) {
-    if (!d || d->chunk <= 0 || d->seqlen % d->chunk != 0) return -1;
+    if (!d || d->chunk <= 0 || d->seqlen <= 0) return -1;
     if (tokens) {
         for (int i = 0; i < ntok; ++i)
             if (tokens[i] < 0 || tokens[i] >= d->seqlen) return -1;

@@ -79,13 +79,12 @@ class Oracle:
     # ------------------------------------------------------------------
     def ssd_scan(self, x, dt, A, Bm, Cm, chunk: int, init_state=None):
         """Token-by-token recurrence.  Returns (y_ssd[B,L,H,P], dH[B,H,C,N,P],
-        states[B,H,C,N,P]) in float64."""
+        states[B,H,C,N,P]) in float64, C = ceil(L / chunk) (a partial last
+        chunk closes at token L-1)."""
         x, dt, A, Bm, Cm = (self._f32(v) for v in (x, dt, A, Bm, Cm))
         Bsz, L, H, P = x.shape
         N = Bm.shape[-1]
-        if L % chunk:
-            raise ValueError("seqlen must be a multiple of chunk")
-        C = L // chunk
+        C = -(-L // chunk)
         d = _Dims(Bsz, L, H, P, N, chunk)
         y = np.empty((Bsz, L, H, P), np.float64)
         dH = np.empty((Bsz, H, C, N, P), np.float64)
@@ -108,9 +107,7 @@ class Oracle:
         dH = self._f64(dH)
         Bsz, L, H, N = Q.shape
         P = E.shape[-1]
-        C = L // chunk
-        if L % chunk:
-            raise ValueError("seqlen must be a multiple of chunk")
+        C = -(-L // chunk)
         d = _Dims(Bsz, L, H, P, N, chunk)
         tok = None if tokens is None else np.ascontiguousarray(np.asarray(tokens, np.int32))
         rows = L if tok is None else len(tok)

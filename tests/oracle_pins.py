@@ -309,6 +309,71 @@ def pin_decode_matches_prefill(orc):
     _close(state, full["states"][:, :, -1], 1e-12, "decode state")
 
 
+def pin_partial_last_chunk(orc):
+    """A sequence that is not a multiple of S ends in a partial chunk, which
+    closes at token L-1: its dH and state follow the same definitions with
+    e(C-1) = L-1 (brute force below), the full chunks are those of the
+    length-32 prefix, and every output row (y_ssd and the layer output) is
+    the same row of a longer sequence with the same leading inputs
+    (causality: row t reads only tokens <= t and chunk memories c < k(t))."""
+    Bz, L, H, P, N, S = 1, 37, 2, 3, 4, 8
+    T = 48
+    inp = _rand_layer(21, Bz, T, H, P, N)
+    cut = {k: (v[:, :L] if k != "A" else v) for k, v in inp.items()}
+    y, dH, st = orc.ssd_scan(cut["x"], cut["dt"], cut["A"], cut["Bm"], cut["Cm"], S)
+    C = -(-L // S)
+    assert dH.shape[2] == C == 5
+    a = _log_decay(cut["dt"], cut["A"])[0]
+    Bm, x, dt = cut["Bm"][0].astype(np.float64), cut["x"][0].astype(np.float64), cut["dt"][0]
+    c0 = (C - 1) * S
+    for h in range(H):
+        m = np.zeros((N, P))
+        for s_ in range(c0, L):
+            m += np.exp(a[s_ + 1:L, h].sum()) * dt[s_, h] * np.outer(Bm[s_], x[s_, h])
+        _close(dH[0, h, C - 1], m, 1e-12, f"partial dH[h={h}]")
+        _close(st[0, h, C - 1], np.exp(a[c0:L, h].sum()) * st[0, h, C - 2] + m, 1e-12, "partial state")
+    y32, dH32, st32 = orc.ssd_scan(*(cut[k][:, :32] if k != "A" else cut[k]
+                                     for k in ("x", "dt", "A", "Bm", "Cm")), S)
+    _close(dH[:, :, :4], dH32, 1e-12, "full chunks of the ragged scan")
+    _close(st[:, :, :4], st32, 1e-12, "full-chunk states of the ragged scan")
+    g = 0.7
+    ragged = orc.layer_forward(*(cut[k] for k in ("x", "dt", "A", "Bm", "Cm", "Q", "E")), S, g)
+    longer = orc.layer_forward(*(inp[k] for k in ("x", "dt", "A", "Bm", "Cm", "Q", "E")), S, g)
+    _close(ragged["y_ssd"], longer["y_ssd"][:, :L], 1e-12, "ragged y_ssd = prefix rows")
+    _close(ragged["y"], longer["y"][:, :L], 1e-12, "ragged layer output = prefix rows")
+
+
+def pin_ragged_prefill_then_decode(orc):
+    """A prefill that stops inside a chunk hands its partial chunk to decode:
+    state = states[C-1], running contribution = dH[C-1], C-1 cached memories,
+    position L mod S.  Decoding the remaining tokens of a longer sequence
+    reproduces the full forward's outputs, its appended memory and its final
+    state (the decode rule and the chunked scan are separate code paths)."""
+    Bz, L, H, P, N, S = 2, 21, 2, 3, 5, 8
+    T = 40
+    inp = _rand_layer(22, Bz, T, H, P, N)
+    g = 0.4
+    full = orc.layer_forward(*(inp[k] for k in ("x", "dt", "A", "Bm", "Cm", "Q", "E")), S, g)
+    pre = orc.layer_forward(*(inp[k][:, :L] if k != "A" else inp[k]
+                              for k in ("x", "dt", "A", "Bm", "Cm", "Q", "E")), S, g)
+    Cfull = L // S
+    cmax = T // S + 1
+    cache = np.zeros((Bz, H, cmax, N, P))
+    cache[:, :, :Cfull] = pre["dH"][:, :, :Cfull]
+    state = np.ascontiguousarray(pre["states"][:, :, -1])
+    dcur = np.ascontiguousarray(pre["dH"][:, :, -1])
+    nch = np.full((Bz,), Cfull, np.int32)
+    pos = np.full((Bz,), L % S, np.int32)
+    for t in range(L, T):
+        y = orc.decode_step(inp["x"][:, t], inp["dt"][:, t], inp["A"], inp["Bm"][:, t],
+                            inp["Cm"][:, t], inp["Q"][:, t], inp["E"][:, t], g, state, dcur,
+                            cache, nch, pos, S)
+        _close(y, full["y"][:, t], 1e-12, f"decode y at t={t}")
+    assert np.all(nch == T // S) and np.all(pos == 0)
+    _close(cache[:, :, :T // S], full["dH"], 1e-12, "memories after the handoff")
+    _close(state, full["states"][:, :, -1], 1e-12, "decode state")
+
+
 def pin_cache_ratio(orc):
     """Eq. (14) (Pith review, circularity check): per head the DART cache is
     M N P elements (M = L/S chunk memories) against 2 L P for a token-level
@@ -333,5 +398,7 @@ ALL_PINS = [
     pin_one_hot_mask,
     pin_sampled_rows,
     pin_decode_matches_prefill,
+    pin_partial_last_chunk,
+    pin_ragged_prefill_then_decode,
     pin_cache_ratio,
 ]

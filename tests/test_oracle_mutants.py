@@ -44,6 +44,9 @@ MUTATIONS = [
     ("decode_no_reset_after_append", "memset(D, 0, sizeof(double) * (size_t)N * P);\n    }\n}",
      "}\n}", 0),
     ("decode_gate_dropped", "yt[p] += c->g * acc;", "yt[p] += acc;", 0),
+    ("partial_chunk_not_closed", "if (t % S == S - 1 || t == L - 1) {", "if (t % S == S - 1) {", 0),
+    ("sma_memory_stride_floor", "const int nchunks = (L + S - 1) / S;\n    const int b = unit / H, h = unit % H;\n    const int nrows",
+     "const int nchunks = L / S;\n    const int b = unit / H, h = unit % H;\n    const int nrows", 0),
 ]
 
 
