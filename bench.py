@@ -58,6 +58,8 @@ def parse():
     p.add_argument("--no-decode", action="store_true", help="skip the decode region")
     p.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end region")
     p.add_argument("--no-cpu-baseline", action="store_true", help="skip timing the oracle")
+    p.add_argument("--no-partial", action="store_true",
+                   help="skip the forward with a partial last chunk (L = 8092)")
     p.add_argument("--decode-steps", type=int, default=DEC.nsteps)
     p.add_argument("--reference-heads", type=int, default=0,
                    help="heads per reference-arm step (default: one per host core, at most 32)")
@@ -102,9 +104,10 @@ def load_peaks():
 # ---------------------------------------------------------------------------
 def sma_flops(s: synth.LayerShape) -> float:
     """4*N*P per valid (token, earlier chunk) pair per head: 2NP for Q^T dH and
-    2NP for C^T dH.  Pairs per (b, h): S * C(C-1)/2."""
-    C = s.nchunks
-    return 4.0 * s.dstate * s.headdim * s.chunk * C * (C - 1) / 2 * s.batch * s.nheads
+    2NP for C^T dH.  A token of chunk k pairs with k memories (S C(C-1)/2
+    pairs per (b, h) when L = C S)."""
+    pairs = sum(min(s.chunk, s.seqlen - k * s.chunk) * k for k in range(s.nchunks))
+    return 4.0 * s.dstate * s.headdim * pairs * s.batch * s.nheads
 
 
 def ssd_flops(s: synth.LayerShape) -> float:
@@ -219,12 +222,12 @@ class Dist:
 # ---------------------------------------------------------------------------
 # GPU regions
 # ---------------------------------------------------------------------------
-def forward_region(args, dist, dart):
+def forward_region(args, dist, dart, shape=FWD):
     dev = torch.device("cuda", torch.cuda.current_device())
-    inp = synth.layer_inputs(FWD, seed=dist.rank)
+    inp = synth.layer_inputs(shape, seed=dist.rank)
     d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
-    B, L, H, P, N, S = FWD.batch, FWD.seqlen, FWD.nheads, FWD.headdim, FWD.dstate, FWD.chunk
-    C = L // S
+    B, L, H, P, N, S = shape.batch, shape.seqlen, shape.nheads, shape.headdim, shape.dstate, shape.chunk
+    C = -(-L // S)
     y = torch.empty((B, L, H, P), device=dev, dtype=torch.float32)
     dH = torch.empty((B, H, C, N, P), device=dev, dtype=torch.bfloat16)
     states = torch.empty((B, H, C, N, P), device=dev, dtype=torch.float32)
@@ -515,6 +518,19 @@ def main():
                               "layer_frac_bf16_peak": (f_sma + f_ssd) / (ms / args.steps / 1e3) / 1e12
                               / peaks["bf16_tflops"]},
         }
+        if not args.no_partial:
+            # the same layer when the sequence ends inside its last chunk
+            ps = synth.TRAIN_L8K_PARTIAL
+            part = forward_region(args, dist, dart, ps)
+            pms = dist.max(part["ms_total"])
+            line["partial_last_chunk"] = {
+                "value": dist.world * ps.batch * ps.seqlen * args.steps / (pms / 1e3), "unit": "tokens/s",
+                "ms_per_step": pms / args.steps, "scan_ms": part["scan_ms"], "sma_ms": part["sma_ms"],
+                "sma_tflops": sma_flops(ps) / (part["sma_ms"] / 1e3) / 1e12,
+                "config": {"workload": "dart_layer_fwd_L8092_partial_last_chunk", "batch": ps.batch,
+                           "seqlen": ps.seqlen, "nheads": ps.nheads, "chunk": ps.chunk,
+                           "last_chunk_tokens": ps.seqlen - (ps.nchunks - 1) * ps.chunk}}
+            line["gpu_launches"] += part["launches"]
         if not args.no_e2e:
             line["e2e"] = e2e_region(args, dist, dart, fwd["inputs"])
         if not args.no_decode:

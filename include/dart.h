@@ -60,7 +60,7 @@ typedef enum { DART_F32 = 0, DART_BF16 = 1 } dart_dtype;
 
 typedef struct {
     int batch;    /* B (decode: number of sequences) */
-    int seqlen;   /* L, a multiple of chunk (ignored by dart_decode_step) */
+    int seqlen;   /* L >= 1 (ignored by dart_decode_step); C = ceil(L / chunk) chunks */
     int nheads;   /* H */
     int headdim;  /* P, the value axis */
     int dstate;   /* N, the key axis */
@@ -72,7 +72,7 @@ typedef struct {
  * Workspace for dart_ssd_chunk_scan, in bytes: B*H*C floats (the per-chunk
  * sum of log-decays, padded to 256 bytes); for the bf16 shapes that run on
  * the tensor cores also the bf16 state entering each chunk (B*H*C*N*P*2
- * bytes) and three fp32 per-token decay terms (3*B*H*L*4 bytes).  Pass at
+ * bytes) and three fp32 per-token decay terms (3*B*H*C*S*4 bytes).  Pass at
  * least this many bytes, 16-byte aligned.
  * Its contents on entry do not matter and are not preserved.
  */
@@ -91,7 +91,10 @@ size_t dart_ssd_chunk_scan_workspace_bytes(const dart_dims* dims, dart_dtype dty
  *                         its last token e(c); no decay beyond e(c))
  *   boundary     states[c] = H_{e(c)}
  * evaluated chunk-wise (intra-chunk quadratic block + inter-chunk state
- * passing), not token by token.
+ * passing), not token by token.  C = ceil(L / S): when L is not a multiple
+ * of S the last chunk is partial and closes at e(C-1) = L-1, so its dH and
+ * state are what a decode carries on from (dH_cur = dH[C-1], state =
+ * states[C-1], C-1 cached memories, position L mod S).
  *
  *   x, Bm, Cm     dtype inputs; dt, A float inputs (dt > 0 after softplus,
  *                 A < 0 per head).
@@ -100,8 +103,8 @@ size_t dart_ssd_chunk_scan_workspace_bytes(const dart_dims* dims, dart_dtype dty
  *   dH            dtype [B,H,C,N,P] output (rounded to nearest-even for bf16).
  *   states        float [B,H,C,N,P] output.
  *   workspace     device scratch of dart_ssd_chunk_scan_workspace_bytes().
- * Requires L % S == 0, ngroups == 1, and (N, P, S, dtype) in the compiled set
- * (see dart_supported()).
+ * Requires ngroups == 1 and (N, P, S, dtype) in the compiled set (see
+ * dart_supported()).
  */
 dart_status dart_ssd_chunk_scan(const dart_dims* dims, dart_dtype dtype,
                                 const void* x, const float* dt, const float* A,
@@ -118,7 +121,8 @@ dart_status dart_ssd_chunk_scan(const dart_dims* dims, dart_dtype dtype,
  *   score  s_{t,c} = Q_t . k_{t,c} / sqrt(N)
  *   o_t = sum_c softmax_c(s_{t,c}) v_{t,c};   o_t = 0 when k(t) == 0.
  * Memories are used as stored, without inter-chunk decay (referee comment 3
- * on Eq. (8)).
+ * on Eq. (8)).  With a partial last chunk (L not a multiple of S) dH has
+ * C = ceil(L / S) memories and no token attends to the last one.
  *   out = y_ssd + g * o   when y_ssd != NULL (the DART layer output), else
  *   out = o               (the raw readout).
  *   Q[B,L,H,N], E[B,L,H,P], Cm[B,L,N], dH[B,H,C,N,P]: dtype inputs.

@@ -76,8 +76,6 @@ dart_status check_common(const dart_dims* d, dart_dtype dt, bool need_seqlen) {
     if (d->ngroups != 1) return fail(DART_ERR_UNSUPPORTED, "ngroups = %d: only 1 (B, C shared by all heads)", d->ngroups);
     if (need_seqlen) {
         if (d->seqlen < 1) return fail(DART_ERR_INVALID_ARG, "dims: seqlen must be >= 1");
-        if (d->seqlen % d->chunk != 0)
-            return fail(DART_ERR_UNSUPPORTED, "seqlen %d is not a multiple of chunk %d", d->seqlen, d->chunk);
     }
     if (d->batch > 65535 || d->nheads > 65535)
         return fail(DART_ERR_UNSUPPORTED, "batch and nheads must be <= 65535");
@@ -109,7 +107,7 @@ const char* dart_sma_impl(int dstate, int headdim, int chunk, dart_dtype dtype) 
 
 size_t dart_ssd_chunk_scan_workspace_bytes(const dart_dims* d, dart_dtype dtype) {
     if (!d || d->chunk < 1) return 0;
-    const size_t C = (size_t)(d->seqlen / d->chunk);
+    const size_t C = (size_t)((d->seqlen + d->chunk - 1) / d->chunk);
     const size_t bhc = (size_t)d->batch * (size_t)d->nheads * C;
     size_t bytes = scan_asum_bytes(bhc);
     if (dart::ssd_scan_tc_applicable(d->dstate, d->headdim, d->chunk, dtype)) {
@@ -135,7 +133,7 @@ dart_status dart_ssd_chunk_scan(const dart_dims* d, dart_dtype dtype, const void
     if (workspace_bytes < dart_ssd_chunk_scan_workspace_bytes(d, dtype))
         return fail(DART_ERR_INVALID_ARG, "workspace: %zu bytes, need %zu", workspace_bytes,
                     dart_ssd_chunk_scan_workspace_bytes(d, dtype));
-    const size_t bhc = (size_t)d->batch * (size_t)d->nheads * (size_t)(d->seqlen / d->chunk);
+    const size_t bhc = (size_t)d->batch * (size_t)d->nheads * (size_t)((d->seqlen + d->chunk - 1) / d->chunk);
     char* hin = static_cast<char*>(workspace) + scan_asum_bytes(bhc);
     float* decay = reinterpret_cast<float*>(hin + bhc * (size_t)d->dstate * (size_t)d->headdim * 2);
     dart::ScanArgs a{d->batch, d->seqlen, d->nheads, d->headdim, d->dstate, d->chunk,

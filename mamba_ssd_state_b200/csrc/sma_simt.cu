@@ -23,7 +23,7 @@ template <typename T, int N, int P>
 __global__ void __launch_bounds__(kThreads) sma_simt_kernel(SmaArgs a) {
     constexpr int PT = P / 4;
     constexpr int NS = N + 4;          // padded row stride, keeps float4 alignment
-    const int S = a.S, C = a.L / S;
+    const int S = a.S, C = (a.L + S - 1) / S;
     const int t0 = blockIdx.x * kTQ;   // first token of the tile
     const int h = blockIdx.y, b = blockIdx.z;
     const int k = t0 / S;              // chunk of every token in the tile
@@ -39,20 +39,22 @@ __global__ void __launch_bounds__(kThreads) sma_simt_kernel(SmaArgs a) {
 
     const int tl = threadIdx.x / 4, pg = threadIdx.x % 4;
     const int t = t0 + tl;
+    const bool live = t < a.L;         // rows past the end of a partial last chunk only help load tiles
     float o[PT], e[PT];
 #pragma unroll
     for (int j = 0; j < PT; ++j) {
         o[j] = 0.f;
-        e[j] = ldf(E + (((size_t)b * a.L + t) * a.H + h) * P + pg * PT + j);
+        e[j] = live ? ldf(E + (((size_t)b * a.L + t) * a.H + h) * P + pg * PT + j) : 0.f;
     }
     float mrun = -INFINITY, lrun = 0.f;
 
     if (k > 0) {
         for (int i = threadIdx.x; i < kTQ * N; i += blockDim.x) {
             const int r = i / N, n = i % N;
+            const bool in = t0 + r < a.L;
             const size_t tok = (size_t)b * a.L + t0 + r;
-            Qs[r * NS + n] = qscale * ldf(Q + (tok * a.H + h) * N + n);
-            Cs[r * NS + n] = ldf(Cm + tok * N + n);
+            Qs[r * NS + n] = in ? qscale * ldf(Q + (tok * a.H + h) * N + n) : 0.f;
+            Cs[r * NS + n] = in ? ldf(Cm + tok * N + n) : 0.f;
         }
         const T* mem = dH + ((size_t)b * a.H + h) * (size_t)C * N * P;
         for (int c = 0; c < k; ++c) {
@@ -91,6 +93,7 @@ __global__ void __launch_bounds__(kThreads) sma_simt_kernel(SmaArgs a) {
             mrun = mnew;
         }
     }
+    if (!live) return;
     const float inv = k > 0 ? 1.f / lrun : 0.f;
     const size_t row = (((size_t)b * a.L + t) * a.H + h) * P + pg * PT;
 #pragma unroll
@@ -106,7 +109,7 @@ cudaError_t run(const SmaArgs& a, cudaStream_t st) {
     auto k = sma_simt_kernel<T, N, P>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    k<<<dim3(a.L / kTQ, a.H, a.B), kThreads, smem, st>>>(a);
+    k<<<dim3((a.L + kTQ - 1) / kTQ, a.H, a.B), kThreads, smem, st>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     count_launches(1);
     return cudaSuccess;

@@ -93,11 +93,14 @@ static_assert(kOffO % 1024 == 0 && 2 * 2 * 128 * 4 * 4 <= 2 * kOBox && kSmemByte
               "shared memory layout");
 
 struct SmaTcParams {
-    CUtensorMap tmap_q;  // Q viewed as dims (N, B*L, H)
-    CUtensorMap tmap_c;  // Cm viewed as dims (N, B*L)
+    // Token-indexed tensors keep the sequence and batch axes apart, so a tile
+    // that runs past the end of a partial last chunk reads zeros and writes
+    // nothing there.
+    CUtensorMap tmap_q;  // Q viewed as dims (N, H, L, B), box (64, 1, 128, 1)
+    CUtensorMap tmap_c;  // Cm viewed as dims (N, L, B)
     CUtensorMap tmap_h;  // dH viewed as dims (P, B*H*C*N)
-    CUtensorMap tmap_e;  // E viewed as dims (P, H, B*L), box (64, 1, 128): L2 prefetch only
-    CUtensorMap tmap_o;  // out viewed as dims (P, H, B*L) fp32, box (32, 1, 128): reduce-add / store
+    CUtensorMap tmap_e;  // E viewed as dims (P, H, L, B), box (64, 1, 128, 1): L2 prefetch only
+    CUtensorMap tmap_o;  // out viewed as dims (P, H, L, B) fp32, box (32, 1, 128, 1): reduce-add / store
     const __nv_bfloat16* E;
     const float* y_ssd;
     float* out;
@@ -218,7 +221,7 @@ __global__ void __launch_bounds__(kThreads, 1) sma_tc_kernel(const __grid_consta
         for (int i = tile0; i < p.total_tiles && ok; i += tstride) {
             const Tile t = decode_tile(p, i, rank);
             if (t.k == 0) continue;
-            const int row = t.b * p.L + t.t0;
+            const int row = t.t0;   // first token of the tile within sequence t.b
             // The first memories of this tile go out before its Q and C: their
             // stage is free long before the previous tile releases Q and C.
             if (!(ok = load_b(t, 0))) break;
@@ -226,11 +229,11 @@ __global__ void __launch_bounds__(kThreads, 1) sma_tc_kernel(const __grid_consta
             if (lane == 0) {
                 if (rank == 0) mbar_expect_tx(bar(Q_FULL), 2 * kHalfA * (kPair ? 2 : 1));
                 if (kPair) {
-                    tma_load_3d_pair(sbase + kOffQ, &p.tmap_q, bar_lead(Q_FULL), 0, row, t.h);
-                    tma_load_3d_pair(sbase + kOffQ + kHalfA, &p.tmap_q, bar_lead(Q_FULL), 64, row, t.h);
+                    tma_load_4d_pair(sbase + kOffQ, &p.tmap_q, bar_lead(Q_FULL), 0, t.h, row, t.b);
+                    tma_load_4d_pair(sbase + kOffQ + kHalfA, &p.tmap_q, bar_lead(Q_FULL), 64, t.h, row, t.b);
                 } else {
-                    tma_load_3d(sbase + kOffQ, &p.tmap_q, bar(Q_FULL), 0, row, t.h);
-                    tma_load_3d(sbase + kOffQ + kHalfA, &p.tmap_q, bar(Q_FULL), 64, row, t.h);
+                    tma_load_4d(sbase + kOffQ, &p.tmap_q, bar(Q_FULL), 0, t.h, row, t.b);
+                    tma_load_4d(sbase + kOffQ + kHalfA, &p.tmap_q, bar(Q_FULL), 64, t.h, row, t.b);
                 }
             }
             q_ph ^= 1;
@@ -238,28 +241,28 @@ __global__ void __launch_bounds__(kThreads, 1) sma_tc_kernel(const __grid_consta
             if (lane == 0) {
                 if (rank == 0) mbar_expect_tx(bar(C_FULL), 2 * kHalfA * (kPair ? 2 : 1));
                 if (kPair) {
-                    tma_load_2d_pair(sbase + kOffC, &p.tmap_c, bar_lead(C_FULL), 0, row);
-                    tma_load_2d_pair(sbase + kOffC + kHalfA, &p.tmap_c, bar_lead(C_FULL), 64, row);
+                    tma_load_3d_pair(sbase + kOffC, &p.tmap_c, bar_lead(C_FULL), 0, row, t.b);
+                    tma_load_3d_pair(sbase + kOffC + kHalfA, &p.tmap_c, bar_lead(C_FULL), 64, row, t.b);
                 } else {
-                    tma_load_2d(sbase + kOffC, &p.tmap_c, bar(C_FULL), 0, row);
-                    tma_load_2d(sbase + kOffC + kHalfA, &p.tmap_c, bar(C_FULL), 64, row);
+                    tma_load_3d(sbase + kOffC, &p.tmap_c, bar(C_FULL), 0, row, t.b);
+                    tma_load_3d(sbase + kOffC + kHalfA, &p.tmap_c, bar(C_FULL), 64, row, t.b);
                 }
                 // the next tile's rows start moving into L2 now: its Q and C
                 // (if it has memories), the E rows its epilogue starts from
                 // and the out rows (holding y_ssd) its output is added into
                 if (i + tstride < p.total_tiles) {
                     const Tile tn = decode_tile(p, i + tstride, rank);
-                    const int rown = tn.b * p.L + tn.t0;
+                    const int rown = tn.t0;
                     if (tn.k > 0) {
-                        tma_prefetch_3d(&p.tmap_q, 0, rown, tn.h);
-                        tma_prefetch_3d(&p.tmap_q, 64, rown, tn.h);
-                        tma_prefetch_2d(&p.tmap_c, 0, rown);
-                        tma_prefetch_2d(&p.tmap_c, 64, rown);
-                        tma_prefetch_3d(&p.tmap_e, 0, tn.h, rown);
+                        tma_prefetch_4d(&p.tmap_q, 0, tn.h, rown, tn.b);
+                        tma_prefetch_4d(&p.tmap_q, 64, tn.h, rown, tn.b);
+                        tma_prefetch_3d(&p.tmap_c, 0, rown, tn.b);
+                        tma_prefetch_3d(&p.tmap_c, 64, rown, tn.b);
+                        tma_prefetch_4d(&p.tmap_e, 0, tn.h, rown, tn.b);
                     }
                     if (p.add_into_out && tn.k > 0) {
-                        tma_prefetch_3d(&p.tmap_o, 0, tn.h, rown);
-                        tma_prefetch_3d(&p.tmap_o, 32, tn.h, rown);
+                        tma_prefetch_4d(&p.tmap_o, 0, tn.h, rown, tn.b);
+                        tma_prefetch_4d(&p.tmap_o, 32, tn.h, rown, tn.b);
                     }
                 }
             }
@@ -375,7 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1) sma_tc_kernel(const __grid_consta
             for (int q = 0; q < kHalfP / 8; ++q) e_raw[q] = make_uint4(0u, 0u, 0u, 0u);
             if (i >= p.total_tiles) return;
             const Tile t = decode_tile(p, i, rank);
-            if (t.k == 0) return;
+            if (t.k == 0 || t.t0 + row >= p.L) return;   // no memories, or a row past the end of the sequence
             const uint4* src = reinterpret_cast<const uint4*>(p.E + row_offset(t));
 #pragma unroll
             for (int q = 0; q < kHalfP / 8; ++q) e_raw[q] = __ldg(src + q);
@@ -491,7 +494,8 @@ __global__ void __launch_bounds__(kThreads, 1) sma_tc_kernel(const __grid_consta
             // and 32 columns into the output tile and one thread hands the
             // tile to the TMA unit, which adds it into out (holding y_ssd)
             // or stores it.  No lane touches y_ssd or out itself.
-            const bool next_mem = i + tstride < p.total_tiles && decode_tile(p, i + tstride, rank).k > 0;
+            const bool next_mem = i + tstride < p.total_tiles && decode_tile(p, i + tstride, rank).k > 0 &&
+                                  decode_tile(p, i + tstride, rank).t0 + row < p.L;
             uint4 en[kHalfP / 8];
             if (next_mem) {
                 const uint4* src = reinterpret_cast<const uint4*>(p.E + row_offset(decode_tile(p, i + tstride, rank)));
@@ -512,15 +516,15 @@ __global__ void __launch_bounds__(kThreads, 1) sma_tc_kernel(const __grid_consta
             }
             fence_proxy_async_smem();
             tile_sync();
-            // (a tile without memories adds nothing: out already holds y_ssd there)
-            if (issuer && !*abort_flag && (t.k > 0 || !p.add_into_out)) {
-                const int tok0 = t.b * p.L + t.t0;
+            // (a tile without memories adds nothing: out already holds y_ssd there;
+            // a tile that starts past the end of the sequence has no rows to write)
+            if (issuer && !*abort_flag && (t.k > 0 || !p.add_into_out) && t.t0 < p.L) {
                 if (p.add_into_out) {
-                    tma_reduce_add_3d(&p.tmap_o, sbase + kOffO, 0, t.h, tok0);
-                    tma_reduce_add_3d(&p.tmap_o, sbase + kOffO + kOBox, 32, t.h, tok0);
+                    tma_reduce_add_4d(&p.tmap_o, sbase + kOffO, 0, t.h, t.t0, t.b);
+                    tma_reduce_add_4d(&p.tmap_o, sbase + kOffO + kOBox, 32, t.h, t.t0, t.b);
                 } else {
-                    tma_store_3d(&p.tmap_o, sbase + kOffO, 0, t.h, tok0);
-                    tma_store_3d(&p.tmap_o, sbase + kOffO + kOBox, 32, t.h, tok0);
+                    tma_store_4d(&p.tmap_o, sbase + kOffO, 0, t.h, t.t0, t.b);
+                    tma_store_4d(&p.tmap_o, sbase + kOffO + kOBox, 32, t.h, t.t0, t.b);
                 }
                 bulk_commit();
             }
@@ -553,18 +557,18 @@ bool sma_tc_applicable(int N, int P, int S, dart_dtype dt) {
 cudaError_t launch_sma_tc(const SmaArgs& a, cudaStream_t st) {
     SmaTcParams p;
     memset(&p, 0, sizeof(p));
-    const int C = a.L / a.S;
+    const int C = (a.L + a.S - 1) / a.S;   // a partial last chunk counts
     {
-        const uint64_t dims[3] = {(uint64_t)kN, (uint64_t)a.B * a.L, (uint64_t)a.H};
-        const uint64_t strides[2] = {(uint64_t)a.H * kN * 2, (uint64_t)kN * 2};
-        const uint32_t box[3] = {64, kBQ, 1};
-        if (!encode_tile_map_bf16(&p.tmap_q, 3, a.Q, dims, strides, box)) return cudaErrorInvalidValue;
+        const uint64_t dims[4] = {(uint64_t)kN, (uint64_t)a.H, (uint64_t)a.L, (uint64_t)a.B};
+        const uint64_t strides[3] = {(uint64_t)kN * 2, (uint64_t)a.H * kN * 2, (uint64_t)a.L * a.H * kN * 2};
+        const uint32_t box[4] = {64, 1, kBQ, 1};
+        if (!encode_tile_map_bf16(&p.tmap_q, 4, a.Q, dims, strides, box)) return cudaErrorInvalidValue;
     }
     {
-        const uint64_t dims[2] = {(uint64_t)kN, (uint64_t)a.B * a.L};
-        const uint64_t strides[1] = {(uint64_t)kN * 2};
-        const uint32_t box[2] = {64, kBQ};
-        if (!encode_tile_map_bf16(&p.tmap_c, 2, a.Cm, dims, strides, box)) return cudaErrorInvalidValue;
+        const uint64_t dims[3] = {(uint64_t)kN, (uint64_t)a.L, (uint64_t)a.B};
+        const uint64_t strides[2] = {(uint64_t)kN * 2, (uint64_t)a.L * kN * 2};
+        const uint32_t box[3] = {64, kBQ, 1};
+        if (!encode_tile_map_bf16(&p.tmap_c, 3, a.Cm, dims, strides, box)) return cudaErrorInvalidValue;
     }
     {
         const uint64_t dims[2] = {(uint64_t)kP, (uint64_t)a.B * a.H * C * kN};
@@ -573,16 +577,16 @@ cudaError_t launch_sma_tc(const SmaArgs& a, cudaStream_t st) {
         if (!encode_tile_map_bf16(&p.tmap_h, 2, a.dH, dims, strides, box)) return cudaErrorInvalidValue;
     }
     {
-        const uint64_t dims[3] = {(uint64_t)kP, (uint64_t)a.H, (uint64_t)a.B * a.L};
-        const uint64_t strides[2] = {(uint64_t)kP * 2, (uint64_t)a.H * kP * 2};
-        const uint32_t box[3] = {64, 1, kBQ};
-        if (!encode_tile_map_bf16(&p.tmap_e, 3, a.E, dims, strides, box)) return cudaErrorInvalidValue;
+        const uint64_t dims[4] = {(uint64_t)kP, (uint64_t)a.H, (uint64_t)a.L, (uint64_t)a.B};
+        const uint64_t strides[3] = {(uint64_t)kP * 2, (uint64_t)a.H * kP * 2, (uint64_t)a.L * a.H * kP * 2};
+        const uint32_t box[4] = {64, 1, kBQ, 1};
+        if (!encode_tile_map_bf16(&p.tmap_e, 4, a.E, dims, strides, box)) return cudaErrorInvalidValue;
     }
     {
-        const uint64_t dims[3] = {(uint64_t)kP, (uint64_t)a.H, (uint64_t)a.B * a.L};
-        const uint64_t strides[2] = {(uint64_t)kP * 4, (uint64_t)a.H * kP * 4};
-        const uint32_t box[3] = {32, 1, kBQ};
-        if (!encode_tile_map_f32(&p.tmap_o, 3, a.out, dims, strides, box)) return cudaErrorInvalidValue;
+        const uint64_t dims[4] = {(uint64_t)kP, (uint64_t)a.H, (uint64_t)a.L, (uint64_t)a.B};
+        const uint64_t strides[3] = {(uint64_t)kP * 4, (uint64_t)a.H * kP * 4, (uint64_t)a.L * a.H * kP * 4};
+        const uint32_t box[4] = {32, 1, kBQ, 1};
+        if (!encode_tile_map_f32(&p.tmap_o, 4, a.out, dims, strides, box)) return cudaErrorInvalidValue;
     }
     p.E = static_cast<const __nv_bfloat16*>(a.E);
     p.y_ssd = a.y_ssd;

@@ -36,11 +36,17 @@ __device__ void block_inclusive_scan(float* v, int n) {
     }
 }
 
+// dt of token t of batch b, head h; 0 past the end of a partial last chunk
+// (no decay, no input), so the chunk's sums stop at token L-1.
+__device__ __forceinline__ float dt_at(const ScanArgs& a, int b, int t, int h) {
+    return t < a.L ? a.dt[((size_t)b * a.L + t) * a.H + h] : 0.f;
+}
+
 // Acum[s] for the chunk starting at token t0 of (b, h).
 __device__ void load_chunk_cumsum(const ScanArgs& a, int b, int h, int t0, float* acum) {
     const float Ah = a.A[h];
     for (int s = threadIdx.x; s < a.S; s += blockDim.x)
-        acum[s] = a.dt[((size_t)b * a.L + t0 + s) * a.H + h] * Ah;
+        acum[s] = dt_at(a, b, t0 + s, h) * Ah;
     __syncthreads();
     block_inclusive_scan(acum, a.S);
 }
@@ -51,7 +57,7 @@ __global__ void __launch_bounds__(kThreads) chunk_state_kernel(ScanArgs a) {
     constexpr int TS = 32;             // tokens per smem tile
     constexpr int RN = N / 16, RP = P / 16;
     const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    const int S = a.S, C = a.L / S, t0 = c * S;
+    const int S = a.S, C = (a.L + S - 1) / S, t0 = c * S;
     extern __shared__ float sm[];
     float* acum = sm;                  // [S]
     float* w = acum + S;               // [S]
@@ -60,7 +66,7 @@ __global__ void __launch_bounds__(kThreads) chunk_state_kernel(ScanArgs a) {
     load_chunk_cumsum(a, b, h, t0, acum);
     const float aend = acum[S - 1];
     for (int s = threadIdx.x; s < S; s += blockDim.x)
-        w[s] = expf(aend - acum[s]) * a.dt[((size_t)b * a.L + t0 + s) * a.H + h];
+        w[s] = expf(aend - acum[s]) * dt_at(a, b, t0 + s, h);
     __syncthreads();
 
     const T* x = static_cast<const T*>(a.x);
@@ -75,11 +81,13 @@ __global__ void __launch_bounds__(kThreads) chunk_state_kernel(ScanArgs a) {
     for (int s0 = 0; s0 < S; s0 += TS) {
         for (int e = threadIdx.x; e < TS * N; e += blockDim.x) {
             const int s = e / N, n = e % N;
-            Bs[e] = ldf(Bm + ((size_t)b * a.L + t0 + s0 + s) * N + n);
+            const int t = t0 + s0 + s;
+            Bs[e] = t < a.L ? ldf(Bm + ((size_t)b * a.L + t) * N + n) : 0.f;
         }
         for (int e = threadIdx.x; e < TS * P; e += blockDim.x) {
             const int s = e / P, p = e % P;
-            Xs[e] = w[s0 + s] * ldf(x + (((size_t)b * a.L + t0 + s0 + s) * a.H + h) * P + p);
+            const int t = t0 + s0 + s;
+            Xs[e] = t < a.L ? w[s0 + s] * ldf(x + (((size_t)b * a.L + t) * a.H + h) * P + p) : 0.f;
         }
         __syncthreads();
 #pragma unroll 4
@@ -114,7 +122,7 @@ __global__ void __launch_bounds__(kThreads) state_pass_kernel(ScanArgs a) {
     const int h = blockIdx.y, b = blockIdx.z;
     const int idx = blockIdx.x * blockDim.x + threadIdx.x;
     if (idx >= N * P) return;
-    const int C = a.L / a.S;
+    const int C = (a.L + a.S - 1) / a.S;
     const size_t bh = (size_t)b * a.H + h;
     float prev = a.init_state ? a.init_state[bh * N * P + idx] : 0.f;
     float* st = a.states + bh * (size_t)C * N * P + idx;
@@ -132,7 +140,7 @@ __global__ void __launch_bounds__(kThreads) chunk_output_kernel(ScanArgs a) {
     constexpr int TS = 32;             // source tokens per smem tile
     constexpr int NP = N + 1;          // padded row stride (bank spread)
     constexpr int PT = P / 4;          // outputs per thread (4 threads per token)
-    const int S = a.S, C = a.L / S;
+    const int S = a.S, C = (a.L + S - 1) / S;
     const int tiles_per_chunk = S / TQ;
     const int c = blockIdx.x / tiles_per_chunk;
     const int q0 = (blockIdx.x % tiles_per_chunk) * TQ;  // first query, chunk-local
@@ -152,7 +160,8 @@ __global__ void __launch_bounds__(kThreads) chunk_output_kernel(ScanArgs a) {
     load_chunk_cumsum(a, b, h, t0, acum);
     for (int e = threadIdx.x; e < TQ * N; e += blockDim.x) {
         const int t = e / N, n = e % N;
-        Cs[t * NP + n] = ldf(Cm + ((size_t)b * a.L + t0 + q0 + t) * N + n);
+        const int tok = t0 + q0 + t;
+        Cs[t * NP + n] = tok < a.L ? ldf(Cm + ((size_t)b * a.L + tok) * N + n) : 0.f;
     }
     const int tl = threadIdx.x / 4, pg = threadIdx.x % 4;
     const int tq = q0 + tl;            // chunk-local query index
@@ -164,12 +173,14 @@ __global__ void __launch_bounds__(kThreads) chunk_output_kernel(ScanArgs a) {
         __syncthreads();
         for (int e = threadIdx.x; e < TS * N; e += blockDim.x) {
             const int s = e / N, n = e % N;
-            Bs[s * NP + n] = ldf(Bm + ((size_t)b * a.L + t0 + s0 + s) * N + n);
+            const int t = t0 + s0 + s;
+            Bs[s * NP + n] = t < a.L ? ldf(Bm + ((size_t)b * a.L + t) * N + n) : 0.f;
         }
         for (int e = threadIdx.x; e < TS * P; e += blockDim.x) {
             const int s = e / P, p = e % P;
-            const size_t tok = (size_t)b * a.L + t0 + s0 + s;
-            Xs[e] = a.dt[tok * a.H + h] * ldf(x + (tok * a.H + h) * P + p);
+            const int t = t0 + s0 + s;
+            const size_t tok = (size_t)b * a.L + t;
+            Xs[e] = t < a.L ? a.dt[tok * a.H + h] * ldf(x + (tok * a.H + h) * P + p) : 0.f;
         }
         __syncthreads();
         // masked, decayed C.B for TQ x TS pairs: 8 per thread
@@ -212,6 +223,7 @@ __global__ void __launch_bounds__(kThreads) chunk_output_kernel(ScanArgs a) {
 #pragma unroll
         for (int j = 0; j < PT; ++j) acc[j] = fmaf(scale, off[j], acc[j]);
     }
+    if (t0 + tq >= a.L) return;   // a row past the end of a partial last chunk
     float* y = a.y + (((size_t)b * a.L + t0 + tq) * a.H + h) * P + pg * PT;
 #pragma unroll
     for (int j = 0; j < PT; ++j) y[j] = acc[j];
@@ -219,7 +231,7 @@ __global__ void __launch_bounds__(kThreads) chunk_output_kernel(ScanArgs a) {
 
 template <typename T, int N, int P>
 cudaError_t run(const ScanArgs& a, cudaStream_t st) {
-    const int C = a.L / a.S;
+    const int C = (a.L + a.S - 1) / a.S;
     {
         const size_t smem = sizeof(float) * (2 * a.S + 32 * N + 32 * P);
         auto k = chunk_state_kernel<T, N, P>;

@@ -88,12 +88,13 @@ __global__ void __launch_bounds__(256) chunk_decay_kernel(const __grid_constant_
     if (gw >= p.B * p.H * p.C) return;  // whole warps only
     const int c = gw % p.C, h = (gw / p.C) % p.H, b = gw / (p.C * p.H);
     const float Ah = p.A[h];
-    const float* dtp = p.dt + ((size_t)b * p.L + (size_t)c * S + (size_t)lane * K) * p.H + h;
+    const int tl = c * S + lane * K;   // this lane's first token
     float d[K], v[K];
     float run = 0.f;
 #pragma unroll
     for (int k = 0; k < K; ++k) {
-        d[k] = dtp[(size_t)k * p.H];
+        // past the end of a partial last chunk: no decay, no input
+        d[k] = tl + k < p.L ? p.dt[((size_t)b * p.L + tl + k) * p.H + h] : 0.f;
         run += d[k] * Ah;
         v[k] = run;
     }
@@ -210,7 +211,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_state_tc_kernel(const __gri
         int b_loads = 0;
         for (int i = 0; i < n_items; ++i) {
             const Item it = cs_item(p, j0 + i);
-            const int row0 = it.b * p.L + it.c * S;   // first token of the chunk in the (B*L) row space
+            const int t0 = it.c * S;                  // first token of the chunk
             if (i == 0 || it.h == 0) {
                 // a new chunk: its B tile, once the MMAs on the previous one are done
                 if (b_loads > 0 && !mbar_wait_warp(bar(B_FREE), (uint32_t)(b_loads - 1) & 1u, wc, 7)) break;
@@ -218,8 +219,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_state_tc_kernel(const __gri
                     mbar_expect_tx(bar(B_FULL), 2 * S * kRowBytes);
                     for (int pnl = 0; pnl < 2; ++pnl)
                         for (int r = 0; r < S / 128; ++r)
-                            tma_load_2d(sbase + Ly::kOffB + (uint32_t)pnl * S * kRowBytes + (uint32_t)r * kBox,
-                                        &p.tmap_b, bar(B_FULL), 64 * pnl, row0 + 128 * r);
+                            tma_load_3d(sbase + Ly::kOffB + (uint32_t)pnl * S * kRowBytes + (uint32_t)r * kBox,
+                                        &p.tmap_b, bar(B_FULL), 64 * pnl, t0 + 128 * r, it.b);
                 }
                 ++b_loads;
             }
@@ -229,8 +230,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_state_tc_kernel(const __gri
             if (lane == 0) {
                 mbar_expect_tx(bar(X_FULL0 + xs), Ly::kXBytes + S * 4);
                 for (int r = 0; r < S / 128; ++r)
-                    tma_load_3d(sbase + Ly::kOffX + (uint32_t)xs * Ly::kXBytes + (uint32_t)r * kBox, &p.tmap_x,
-                                bar(X_FULL0 + xs), 0, row0 + 128 * r, it.h);
+                    tma_load_4d(sbase + Ly::kOffX + (uint32_t)xs * Ly::kXBytes + (uint32_t)r * kBox, &p.tmap_x,
+                                bar(X_FULL0 + xs), 0, it.h, t0 + 128 * r, it.b);
                 bulk_load(sbase + Ly::kOffF + (uint32_t)xs * S * 4,
                           p.wst + (((size_t)it.b * p.H + it.h) * p.C + it.c) * S, S * 4, bar(X_FULL0 + xs));
             }
@@ -491,7 +492,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_output_tc_kernel(const __gr
         for (int i = 0; i < n_items; ++i) {
             const Item it = co_item(p, j0 + i);
             const int KS = 128 * (it.half + 1);            // source tokens this half depends on
-            const int row0 = it.b * p.L + it.c * S;        // first token of the chunk
+            const int t0 = it.c * S;                       // first token of the chunk
             const bool has_off = (it.c > 0) || (p.init_state != nullptr);
             if (group_first(i, it)) {
                 // C rows of this half (A of G and of Y_off) and B rows 0..KS-1 (B of G),
@@ -500,11 +501,11 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_output_tc_kernel(const __gr
                 if (lane == 0) {
                     mbar_expect_tx(bar(IN_FULL), 2 * kBox + 2 * (uint32_t)KS * kRowBytes);
                     for (int pnl = 0; pnl < 2; ++pnl) {
-                        tma_load_2d(sbase + kOffC + (uint32_t)pnl * kBox, &p.tmap_c, bar(IN_FULL), 64 * pnl,
-                                    row0 + 128 * it.half);
+                        tma_load_3d(sbase + kOffC + (uint32_t)pnl * kBox, &p.tmap_c, bar(IN_FULL), 64 * pnl,
+                                    t0 + 128 * it.half, it.b);
                         for (int r = 0; r < KS / 128; ++r)
-                            tma_load_2d(sbase + kOffBP + (uint32_t)pnl * KS * kRowBytes + (uint32_t)r * kBox,
-                                        &p.tmap_b, bar(IN_FULL), 64 * pnl, row0 + 128 * r);
+                            tma_load_3d(sbase + kOffBP + (uint32_t)pnl * KS * kRowBytes + (uint32_t)r * kBox,
+                                        &p.tmap_b, bar(IN_FULL), 64 * pnl, t0 + 128 * r, it.b);
                     }
                 }
                 ++ng;
@@ -519,8 +520,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_output_tc_kernel(const __gr
                 bulk_load(sbase + kOffF + (uint32_t)xs * 2048, p.a2 + drow, KS * 4, bar(X_FULL0 + xs));
                 bulk_load(sbase + kOffF + (uint32_t)xs * 2048 + 1024, p.colf + drow, KS * 4, bar(X_FULL0 + xs));
                 for (int r = 0; r < KS / 128; ++r)
-                    tma_load_3d(sbase + kOffX + (uint32_t)xs * kXBytes + (uint32_t)r * kBox, &p.tmap_x,
-                                bar(X_FULL0 + xs), 0, row0 + 128 * r, it.h);
+                    tma_load_4d(sbase + kOffX + (uint32_t)xs * kXBytes + (uint32_t)r * kBox, &p.tmap_x,
+                                bar(X_FULL0 + xs), 0, it.h, t0 + 128 * r, it.b);
                 if (has_off)
                     tma_load_2d(sbase + kOffHp + (uint32_t)xs * kBox, &p.tmap_hin, bar(X_FULL0 + xs), 0,
                                 ((it.b * p.H + it.h) * p.C + it.c) * kN);
@@ -644,7 +645,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_output_tc_kernel(const __gr
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(ACC_EMPTY0 + a));
             }
-            const int row0 = it.b * p.L + it.c * S;
+            const int t0 = it.c * S;
 #pragma unroll
             for (int ch = 0; ch < 2; ++ch) {
                 if (issuer) bulk_wait_read<0>();   // the previous box has left the staging area
@@ -658,8 +659,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_output_tc_kernel(const __gr
                 }
                 fence_proxy_async_smem();
                 named_bar_sync(1, kEpi);
-                if (issuer && !*abort_flag) {
-                    tma_store_3d(&p.tmap_y, sbase + kOffYs, 32 * ch, it.h, row0 + 128 * it.half);
+                if (issuer && !*abort_flag && t0 + 128 * it.half < p.L) {   // rows past the end are not written
+                    tma_store_4d(&p.tmap_y, sbase + kOffYs, 32 * ch, it.h, t0 + 128 * it.half, it.b);
                     bulk_commit();
                 }
             }
@@ -773,21 +774,23 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_output_tc_kernel(const __gr
 }
 }  // namespace co
 
+// Token-indexed tensors are described with the sequence and batch axes
+// apart, so a box that runs past the end of a partial last chunk reads
+// zeros and writes nothing there (instead of reaching the next sequence).
 bool make_maps(const ScanArgs& a, ScanTcParams& p) {
-    const uint64_t BL = (uint64_t)a.B * a.L;
-    const int C = a.L / a.S;
+    const int C = (a.L + a.S - 1) / a.S;
     {
-        const uint64_t dims[3] = {(uint64_t)kP, BL, (uint64_t)a.H};
-        const uint64_t strides[2] = {(uint64_t)a.H * kP * 2, (uint64_t)kP * 2};
-        const uint32_t box[3] = {64, 128, 1};
-        if (!encode_tile_map_bf16(&p.tmap_x, 3, a.x, dims, strides, box)) return false;
+        const uint64_t dims[4] = {(uint64_t)kP, (uint64_t)a.H, (uint64_t)a.L, (uint64_t)a.B};
+        const uint64_t strides[3] = {(uint64_t)kP * 2, (uint64_t)a.H * kP * 2, (uint64_t)a.L * a.H * kP * 2};
+        const uint32_t box[4] = {64, 1, 128, 1};
+        if (!encode_tile_map_bf16(&p.tmap_x, 4, a.x, dims, strides, box)) return false;
     }
     {
-        const uint64_t dims[2] = {(uint64_t)kN, BL};
-        const uint64_t strides[1] = {(uint64_t)kN * 2};
-        const uint32_t box[2] = {64, 128};
-        if (!encode_tile_map_bf16(&p.tmap_b, 2, a.Bm, dims, strides, box)) return false;
-        if (!encode_tile_map_bf16(&p.tmap_c, 2, a.Cm, dims, strides, box)) return false;
+        const uint64_t dims[3] = {(uint64_t)kN, (uint64_t)a.L, (uint64_t)a.B};
+        const uint64_t strides[2] = {(uint64_t)kN * 2, (uint64_t)a.L * kN * 2};
+        const uint32_t box[3] = {64, 128, 1};
+        if (!encode_tile_map_bf16(&p.tmap_b, 3, a.Bm, dims, strides, box)) return false;
+        if (!encode_tile_map_bf16(&p.tmap_c, 3, a.Cm, dims, strides, box)) return false;
     }
     {
         const uint64_t dims[2] = {(uint64_t)kP, (uint64_t)a.B * a.H * C * kN};
@@ -803,10 +806,10 @@ bool make_maps(const ScanArgs& a, ScanTcParams& p) {
         if (!encode_tile_map_f32(&p.tmap_st, 2, a.states, dims, strides, box)) return false;
     }
     {
-        const uint64_t dims[3] = {(uint64_t)kP, (uint64_t)a.H, BL};
-        const uint64_t strides[2] = {(uint64_t)kP * 4, (uint64_t)a.H * kP * 4};
-        const uint32_t box[3] = {32, 1, 128};
-        if (!encode_tile_map_f32(&p.tmap_y, 3, a.y, dims, strides, box)) return false;
+        const uint64_t dims[4] = {(uint64_t)kP, (uint64_t)a.H, (uint64_t)a.L, (uint64_t)a.B};
+        const uint64_t strides[3] = {(uint64_t)kP * 4, (uint64_t)a.H * kP * 4, (uint64_t)a.L * a.H * kP * 4};
+        const uint32_t box[4] = {32, 1, 128, 1};
+        if (!encode_tile_map_f32(&p.tmap_y, 4, a.y, dims, strides, box)) return false;
     }
     return true;
 }
@@ -829,8 +832,8 @@ cudaError_t launch_ssd_scan_tc(const ScanArgs& a, cudaStream_t st) {
     p.asum = a.asum;
     p.hin = static_cast<__nv_bfloat16*>(a.hin);
     p.y = a.y;
-    p.B = a.B; p.L = a.L; p.H = a.H; p.S = a.S; p.C = a.L / a.S;
-    const size_t bhcs = (size_t)a.B * a.H * a.L;
+    p.B = a.B; p.L = a.L; p.H = a.H; p.S = a.S; p.C = (a.L + a.S - 1) / a.S;
+    const size_t bhcs = (size_t)a.B * a.H * p.C * a.S;   // decay arrays are [B, H, C, S]
     p.a2 = a.decay;
     p.colf = a.decay + bhcs;
     p.wst = a.decay + 2 * bhcs;

@@ -186,9 +186,7 @@ def dart_ssd_chunk_scan(x, dt, A, Bm, Cm, chunk: int, init_state=None, *, y_ssd=
     _shape("Cm", Cm, (Bsz, L, N))
     if init_state is not None:
         _shape("init_state", init_state, (Bsz, H, N, P))
-    if L % chunk:
-        raise ValueError(f"seqlen {L} is not a multiple of chunk {chunk}")
-    C = L // chunk
+    C = -(-L // chunk)   # a partial last chunk counts
     dims = Dims(Bsz, L, H, P, N, chunk, 1)
     code = _dtype_code(x.dtype)
     if y_ssd is None:
@@ -219,9 +217,7 @@ def dart_sma_forward(Q, E, Cm, dH, chunk: int, g: float, y_ssd=None, *, out=None
     y_ssd = _dev(y_ssd, dev, torch.float32)
     Bsz, L, H, N = Q.shape
     P = E.shape[-1]
-    if L % chunk:
-        raise ValueError(f"seqlen {L} is not a multiple of chunk {chunk}")
-    C = L // chunk
+    C = -(-L // chunk)   # a partial last chunk counts
     _shape("E", E, (Bsz, L, H, P)); _shape("Cm", Cm, (Bsz, L, N)); _shape("dH", dH, (Bsz, H, C, N, P))
     if y_ssd is not None:
         _shape("y_ssd", y_ssd, (Bsz, L, H, P))

@@ -39,7 +39,7 @@ class LayerShape:
 
     @property
     def nchunks(self) -> int:
-        return self.seqlen // self.chunk
+        return -(-self.seqlen // self.chunk)   # a partial last chunk counts
 
     def asdict(self):
         return asdict(self)
@@ -63,6 +63,8 @@ class DecodeShape:
 TINY_FP32 = LayerShape(1, 512, 2, 16, 16, 64, "f32", "softplus")
 LAYER_L2K = LayerShape(4, 2048, 32, 64, 128, 256, "bf16", "loguniform")
 TRAIN_L8K = LayerShape(2, 8192, 32, 64, 128, 256, "bf16", "loguniform")
+# the training-length layer with a sequence that ends 100 tokens into its last chunk
+TRAIN_L8K_PARTIAL = LayerShape(2, 8192 - 100, 32, 64, 128, 256, "bf16", "loguniform")
 LONG_L64K = LayerShape(1, 65536, 32, 64, 128, 256, "bf16", "loguniform")
 DECODE_64x32K = DecodeShape(64, 32, 64, 128, 256, 128, 129, 256)
 

@@ -58,10 +58,15 @@ def _scan(lib, dims, dtype=dart.DART_BF16, x=FAKE, ws_bytes=1 << 20):
                                    FAKE, FAKE, ws_bytes, None)
 
 
-def test_scan_rejects_ragged_seqlen(lib):
-    rc = _scan(lib, dart.Dims(1, 300, 2, 64, 128, 256, 1))
-    assert rc == dart.DART_ERR_UNSUPPORTED
-    assert b"multiple of chunk" in lib.dart_last_error()
+def test_ragged_seqlen_counts_the_partial_chunk(lib):
+    """L = 300, S = 256: two chunks, the second one partial.  The workspace
+    is sized for ceil(L / S) chunks and a smaller one is rejected before any
+    launch."""
+    d = dart.Dims(1, 300, 2, 64, 128, 256, 1)
+    need = lib.dart_ssd_chunk_scan_workspace_bytes(ctypes.byref(d), dart.DART_BF16)
+    bhc = 1 * 2 * 2
+    assert need == 256 + bhc * 128 * 64 * 2 + 3 * bhc * 256 * 4
+    assert _scan(lib, d, ws_bytes=need - 16) == dart.DART_ERR_INVALID_ARG
 
 
 def test_scan_rejects_ngroups(lib):
@@ -102,7 +107,7 @@ def test_sma_rejects_bad_args(lib):
     d = dart.Dims(1, 512, 2, 64, 128, 256, 1)
     rc = lib.dart_sma_forward(ctypes.byref(d), dart.DART_BF16, FAKE, None, FAKE, FAKE, 0.5, None, FAKE, None)
     assert rc == dart.DART_ERR_INVALID_ARG
-    d.seqlen = 500
+    d.chunk = 96   # not a compiled chunk length (a seqlen that is not a multiple of chunk is accepted)
     rc = lib.dart_sma_forward(ctypes.byref(d), dart.DART_BF16, FAKE, FAKE, FAKE, FAKE, 0.5, None, FAKE, None)
     assert rc == dart.DART_ERR_UNSUPPORTED
 

@@ -136,6 +136,39 @@ def test_prefill_then_decode_matches_longer_prefill():
     assert_close("state", state, full["states"][:, :, -1].cpu().numpy(), 2e-2)
 
 
+def test_ragged_prefill_then_decode_matches_longer_prefill():
+    """A prefill that ends inside a chunk (L = 2 S + 100) hands its partial
+    chunk to decode (dH_cur = dH[C-1], state = states[C-1], C-1 memories,
+    position L mod S); decoding to 4 S reproduces the longer prefill."""
+    S = 256
+    shape = LayerShape(2, 4 * S, 3, 64, 128, S, "bf16", "loguniform")
+    inp = synth.layer_inputs(shape, seed=23)
+    d = to_device(inp)
+    L = 2 * S + 100
+    full = dart.layer_forward(d["x"], d["dt"], d["A"], d["Bm"], d["Cm"], d["Q"], d["E"], S, d["g"])
+    pre = dart.layer_forward(*(d[k][:, :L] if k != "A" else d[k] for k in ("x", "dt", "A", "Bm", "Cm", "Q", "E")),
+                             S, d["g"])
+    assert pre["dH"].shape[2] == 3
+    B, H, N, P = 2, 3, 128, 64
+    cmax = 5
+    cache = torch.zeros(B, H, cmax, N, P, dtype=torch.bfloat16, device="cuda")
+    cache[:, :, :2] = pre["dH"][:, :, :2]
+    state = pre["states"][:, :, -1].contiguous()
+    dcur = pre["dH"][:, :, -1].float().contiguous()
+    nch = torch.full((B,), 2, dtype=torch.int32, device="cuda")
+    pos = torch.full((B,), L % S, dtype=torch.int32, device="cuda")
+    ys = []
+    for t in range(L, 4 * S):
+        ys.append(dart.dart_decode_step(d["x"][:, t], d["dt"][:, t], d["A"], d["Bm"][:, t], d["Cm"][:, t],
+                                        d["Q"][:, t], d["E"][:, t], d["g"], state, dcur, cache, nch, pos, S))
+    dart.dart_sync_status()
+    y_dec = torch.stack(ys, 1)
+    assert_close("decode vs prefill y", y_dec, full["y"][:, L:].cpu().numpy(), 2e-2)
+    assert torch.all(nch == 4) and torch.all(pos == 0)
+    assert_close("memories", cache[:, :, :4].float(), full["dH"].float().cpu().numpy(), 2e-2)
+    assert_close("state", state, full["states"][:, :, -1].cpu().numpy(), 2e-2)
+
+
 def test_decode_bad_counters_are_flagged():
     """A sequence with pos outside [0, S) or a full cache is skipped and the
     device status reports DART_ERR_DEVICE; the other sequences advance."""

@@ -96,6 +96,31 @@ def test_bf16_N64_P64_cuda_core_path(orc):
     check_full(orc, shape, synth.layer_inputs(shape, seed=31), TOL[torch.bfloat16])
 
 
+# ---------------------------------------------------------------------------
+# sequences that end inside a chunk (C = ceil(L / S), the last chunk partial)
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("tail", [200, 100, 37])
+def test_bf16_partial_last_chunk(orc, tail):
+    """3 full chunks of 256 and a partial one: 200 tokens (its second 128-row
+    half partly past the end), 100 (second half entirely past the end) and 37;
+    two sequences, so a box past the end of the first must not reach the
+    second."""
+    shape = LayerShape(2, 3 * 256 + tail, 3, 64, 128, 256, "bf16", "loguniform")
+    check_full(orc, shape, synth.layer_inputs(shape, seed=50 + tail), TOL[torch.bfloat16])
+
+
+def test_bf16_partial_last_chunk_S128(orc):
+    """S = 128 (one-CTA attention kernel), 4 full chunks and 60 tokens."""
+    shape = LayerShape(2, 4 * 128 + 60, 2, 64, 128, 128, "bf16", "loguniform")
+    check_full(orc, shape, synth.layer_inputs(shape, seed=53), TOL[torch.bfloat16])
+
+
+def test_fp32_partial_last_chunk(orc):
+    """The CUDA-core kernels: fp32, S = 64, 7 full chunks and 27 tokens."""
+    shape = LayerShape(2, 7 * 64 + 27, 2, 16, 16, 64, "f32", "softplus")
+    check_full(orc, shape, synth.layer_inputs(shape, seed=54), TOL[torch.float32])
+
+
 def test_dispatch_uses_tensor_cores_for_the_layer_shape():
     assert dart.sma_impl(128, 64, 256, torch.bfloat16) == "sma_tcgen05"
     assert dart.sma_impl(128, 64, 128, torch.bfloat16) == "sma_tcgen05"
