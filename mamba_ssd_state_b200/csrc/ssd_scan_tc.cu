@@ -77,52 +77,56 @@ struct ScanTcParams {
 };
 
 // ===========================================================================
-// chunk_decay: the per-token decay terms of every (b, h, c), one warp each
+// chunk_decay: the per-token decay terms of every (b, h, c).  One CTA per
+// (b, c, group of 8 heads): the group's dt block [S tokens][8 heads] is read
+// once (8 consecutive floats per token) into shared memory, head-major with
+// one padding word per row; warp w then scans head w of the group in rounds
+// of 32 tokens, one token per lane.
 // ===========================================================================
 template <int S>
 __global__ void __launch_bounds__(256) chunk_decay_kernel(const __grid_constant__ ScanTcParams p) {
-    constexpr int K = S / 32;        // consecutive tokens per lane
-    constexpr int LPB = 32 / K;      // lanes per 32-token block
-    const int gw = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5);  // (b * H + h) * C + c
-    const int lane = threadIdx.x & 31;
-    if (gw >= p.B * p.H * p.C) return;  // whole warps only
-    const int c = gw % p.C, h = (gw / p.C) % p.H, b = gw / (p.C * p.H);
+    constexpr int K = S / 32;             // rounds of 32 tokens
+    __shared__ float dts[8 * (S + 1)];    // [head of the group][S + 1]
+    const int ngh = (p.H + 7) / 8;
+    const int hgi = blockIdx.x % ngh;
+    const int c = (blockIdx.x / ngh) % p.C, b = blockIdx.x / (ngh * p.C);
+    const int nh = min(8, p.H - 8 * hgi);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t0 = c * S;
+    for (int i = threadIdx.x; i < 8 * S; i += blockDim.x) {
+        const int t = i >> 3, hh = i & 7;
+        // past the end of a partial last chunk (or of the heads): no decay, no input
+        dts[hh * (S + 1) + t] =
+            (t0 + t < p.L && hh < nh) ? p.dt[((size_t)b * p.L + t0 + t) * p.H + 8 * hgi + hh] : 0.f;
+    }
+    __syncthreads();
+    if (warp >= nh) return;
+    const int h = 8 * hgi + warp;
     const float Ah = p.A[h];
-    const int tl = c * S + lane * K;   // this lane's first token
-    float d[K], v[K];
-    float run = 0.f;
+    const float* d = dts + warp * (S + 1);
+    const size_t o = (((size_t)b * p.H + h) * p.C + c) * S;   // this (b, h, c) in the decay arrays
+    float carry = 0.f;      // prefix of dt A over the previous rounds
+    float v[K];
 #pragma unroll
-    for (int k = 0; k < K; ++k) {
-        // past the end of a partial last chunk: no decay, no input
-        d[k] = tl + k < p.L ? p.dt[((size_t)b * p.L + tl + k) * p.H + h] : 0.f;
-        run += d[k] * Ah;
-        v[k] = run;
+    for (int r = 0; r < K; ++r) {
+        const float dv = d[32 * r + lane];
+        float incl = dv * Ah;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const float up = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += up;
+        }
+        v[r] = carry + incl;                                  // Acum at token 32 r + lane
+        const float a2 = v[r] * kLog2e;
+        const float a2r = __shfl_sync(0xffffffffu, a2, 0);    // the round's first token
+        p.a2[o + 32 * r + lane] = a2;
+        p.colf[o + 32 * r + lane] = exp2f(a2r - a2) * dv;
+        carry = __shfl_sync(0xffffffffu, v[r], 31);
     }
-    float incl = run;  // inclusive prefix of the lane totals
+    const float aend = carry;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const float up = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += up;
-    }
-    const float excl = incl - run;
-    const float aend = __shfl_sync(0xffffffffu, incl, 31);
-    float a2[K], cf[K], ws[K];
-#pragma unroll
-    for (int k = 0; k < K; ++k) a2[k] = (excl + v[k]) * kLog2e;
-    const float a2r = __shfl_sync(0xffffffffu, a2[0], lane & ~(LPB - 1));
-#pragma unroll
-    for (int k = 0; k < K; ++k) {
-        cf[k] = exp2f(a2r - a2[k]) * d[k];
-        ws[k] = expf(aend - (excl + v[k])) * d[k];
-    }
-    const size_t o = (size_t)gw * S + (size_t)lane * K;
-#pragma unroll
-    for (int k = 0; k < K; k += 4) {
-        *reinterpret_cast<float4*>(p.a2 + o + k) = make_float4(a2[k], a2[k + 1], a2[k + 2], a2[k + 3]);
-        *reinterpret_cast<float4*>(p.colf + o + k) = make_float4(cf[k], cf[k + 1], cf[k + 2], cf[k + 3]);
-        *reinterpret_cast<float4*>(p.wst + o + k) = make_float4(ws[k], ws[k + 1], ws[k + 2], ws[k + 3]);
-    }
-    if (lane == 0) p.asum[gw] = aend;
+    for (int r = 0; r < K; ++r) p.wst[o + 32 * r + lane] = expf(aend - v[r]) * d[32 * r + lane];
+    if (lane == 0) p.asum[((size_t)b * p.H + h) * p.C + c] = aend;
 }
 
 // ===========================================================================
@@ -839,10 +843,9 @@ cudaError_t launch_ssd_scan_tc(const ScanArgs& a, cudaStream_t st) {
     p.wst = a.decay + 2 * bhcs;
     p.status = a.status;
     cudaError_t e;
-    // 0. per-token decay terms, one warp per (b, h, c)
+    // 0. per-token decay terms, one CTA per (b, c, group of 8 heads)
     {
-        const int warps = a.B * a.H * p.C;
-        const int grid = (warps + 7) / 8;
+        const int grid = a.B * p.C * ((a.H + 7) / 8);
         if (a.S == 256)
             chunk_decay_kernel<256><<<grid, 256, 0, st>>>(p);
         else
