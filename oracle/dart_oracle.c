@@ -35,6 +35,14 @@
  *    raw dH[c] with no inter-chunk decay (referee major comment 3).  A token
  *    in chunk 0 has no memory and gets o_t = 0.
  *
+ *  - The decayed-memory variant that the same referee comment asks to
+ *    compare against: every memory is first carried from its chunk's last
+ *    token e(c) to t by the recurrence's own decay,
+ *        dH[c] -> exp(A_h * sum_{r=e(c)+1}^{t} dt_r) * dH[c],
+ *    i.e. the amount of dH[c] still present in the state H_t, and then used
+ *    as above for both the key and the value.  The exponent is summed here
+ *    token by token from dt, straight from that definition.
+ *
  *  - The gated residual y_t = y_ssd_t + g * o_t with one scalar g (Pith
  *    review, "Core claim": a zero-initialised scalar gate added to the SSM
  *    output).
@@ -178,6 +186,7 @@ typedef struct {
     const oracle_dims* d;
     const float *Q, *E, *Cm;
     const double* dH;
+    const float *dt, *A; /* both NULL: raw memories; both set: decayed  */
     double g;
     const double* y_ssd; /* nullable; indexed like the output rows */
     double* o;           /* nullable: raw readout o_t              */
@@ -207,17 +216,26 @@ static void sma_unit(void* vctx, int unit) {
         const float* Ct = c->Cm + ((size_t)b * L + t) * N;
         for (int cc = 0; cc < k; ++cc) {
             const double* M = c->dH + (((size_t)b * H + h) * nchunks + cc) * (size_t)N * P;
+            /* decayed variant: the factor that carries dH[c] from e(c) to t */
+            double wdec = 1.0;
+            if (c->dt) {
+                const int ec = cc * S + S - 1; /* last token of memory chunk cc */
+                double logdec = 0.0;
+                for (int r = ec + 1; r <= t; ++r)
+                    logdec += (double)c->dt[((size_t)b * L + r) * H + h] * (double)c->A[h];
+                wdec = exp(logdec);
+            }
             /* key = dH[c] E_t */
             for (int n = 0; n < N; ++n) {
                 double acc = 0.0;
                 for (int p = 0; p < P; ++p) acc += M[n * P + p] * (double)Et[p];
-                key[n] = acc;
+                key[n] = wdec * acc;
             }
             /* value = C_t^T dH[c] */
             for (int p = 0; p < P; ++p) {
                 double acc = 0.0;
                 for (int n = 0; n < N; ++n) acc += (double)Ct[n] * M[n * P + p];
-                val[(size_t)cc * P + p] = acc;
+                val[(size_t)cc * P + p] = wdec * acc;
             }
             /* score = Q_t . key / sqrt(N) */
             double s = 0.0;
@@ -257,19 +275,23 @@ static void sma_unit(void* vctx, int unit) {
 
 /*
  * Q[B,L,H,N], E[B,L,H,P], Cm[B,L,N] float; dH[B,H,C,N,P] double.
+ * dt[B,L,H] and A[H] float, both NULL for raw memories or both given for the
+ * decayed-memory variant.
  * With tokens == NULL every position is computed and the outputs are
  * [B,L,H,P]; otherwise only the ntok listed positions, outputs [B,ntok,H,P]
  * (and y_ssd, when given, is read with that same compact indexing).
  */
 int oracle_sma(const oracle_dims* d, const float* Q, const float* E, const float* Cm,
-               const double* dH, double g, const double* y_ssd, double* o, double* y,
-               double* scores, const int* tokens, int ntok, int nthreads) {
+               const double* dH, const float* dt, const float* A, double g,
+               const double* y_ssd, double* o, double* y, double* scores,
+               const int* tokens, int ntok, int nthreads) {
     if (!d || d->chunk <= 0 || d->seqlen <= 0) return -1;
+    if ((dt == NULL) != (A == NULL)) return -1;
     if (tokens) {
         for (int i = 0; i < ntok; ++i)
             if (tokens[i] < 0 || tokens[i] >= d->seqlen) return -1;
     }
-    sma_ctx c = {d, Q, E, Cm, dH, g, y_ssd, o, y, scores, tokens, ntok};
+    sma_ctx c = {d, Q, E, Cm, dH, dt, A, g, y_ssd, o, y, scores, tokens, ntok};
     run_units(sma_unit, &c, d->batch * d->nheads, nthreads);
     return 0;
 }

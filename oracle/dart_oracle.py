@@ -56,7 +56,7 @@ class Oracle:
         self.lib.oracle_ssd_scan.restype = ctypes.c_int
         self.lib.oracle_ssd_scan.argtypes = [ctypes.POINTER(_Dims)] + [_P] * 9 + [ctypes.c_int]
         self.lib.oracle_sma.restype = ctypes.c_int
-        self.lib.oracle_sma.argtypes = ([ctypes.POINTER(_Dims)] + [_P] * 4 + [ctypes.c_double]
+        self.lib.oracle_sma.argtypes = ([ctypes.POINTER(_Dims)] + [_P] * 6 + [ctypes.c_double]
                                         + [_P] * 5 + [ctypes.c_int, ctypes.c_int])
         self.lib.oracle_decode_step.restype = ctypes.c_int
         self.lib.oracle_decode_step.argtypes = (
@@ -98,12 +98,18 @@ class Oracle:
         return y, dH, st
 
     def sma(self, Q, E, Cm, dH, chunk: int, g: float = 1.0, y_ssd=None,
-            tokens=None, want_scores: bool = False):
+            tokens=None, want_scores: bool = False, dt=None, A=None):
         """Naive state-memory attention.  Returns dict with 'o' (raw readout),
         'y' (y_ssd + g*o; y_ssd = 0 when not given) and optionally 'scores'
         ([B,H,rows,C], NaN where masked).  With ``tokens`` only those
-        positions are computed and rows are compacted to [B,len(tokens),H,P]."""
+        positions are computed and rows are compacted to [B,len(tokens),H,P].
+        With ``dt`` [B,L,H] and ``A`` [H] every memory is decayed from its
+        chunk's last token to t before use (the decayed-memory variant)."""
+        if (dt is None) != (A is None):
+            raise ValueError("dt and A go together")
         Q, E, Cm = (self._f32(v) for v in (Q, E, Cm))
+        dtv = None if dt is None else self._f32(dt)
+        Av = None if A is None else self._f32(A)
         dH = self._f64(dH)
         Bsz, L, H, N = Q.shape
         P = E.shape[-1]
@@ -118,7 +124,8 @@ class Oracle:
             raise ValueError("y_ssd must have the output row shape")
         sc = np.empty((Bsz, H, rows, C), np.float64) if want_scores else None
         rc = self.lib.oracle_sma(ctypes.byref(d), self._ptr(Q), self._ptr(E), self._ptr(Cm),
-                                 self._ptr(dH), float(g), self._ptr(ys), self._ptr(o),
+                                 self._ptr(dH), self._ptr(dtv), self._ptr(Av), float(g),
+                                 self._ptr(ys), self._ptr(o),
                                  self._ptr(y), self._ptr(sc), self._ptr(tok),
                                  0 if tok is None else len(tok), self.nthreads)
         if rc:
@@ -129,12 +136,14 @@ class Oracle:
         return out
 
     def layer_forward(self, x, dt, A, Bm, Cm, Q, E, chunk: int, g: float, init_state=None,
-                      tokens=None):
+                      tokens=None, decayed: bool = False):
         """Full DART layer forward: scan, SMA over the scan's own fp64 dH,
-        gated residual.  Returns dict(y, y_ssd, o, dH, states)."""
+        gated residual.  Returns dict(y, y_ssd, o, dH, states).  ``decayed``
+        selects the decayed-memory SMA."""
         y_ssd, dH, st = self.ssd_scan(x, dt, A, Bm, Cm, chunk, init_state)
         ys = y_ssd if tokens is None else y_ssd[:, np.asarray(tokens)]
-        r = self.sma(Q, E, Cm, dH, chunk, g, ys, tokens)
+        r = self.sma(Q, E, Cm, dH, chunk, g, ys, tokens,
+                     dt=dt if decayed else None, A=A if decayed else None)
         return {"y": r["y"], "o": r["o"], "y_ssd": y_ssd, "dH": dH, "states": st}
 
     def decode_step(self, x, dt, A, Bm, Cm, Q, E, g, state, dH_cur, cache, nchunks, pos,

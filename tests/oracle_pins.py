@@ -386,6 +386,94 @@ def pin_cache_ratio(orc):
     assert dart / attn == N / (2 * S) == 0.25
 
 
+# ----------------------------------------------------------------------------
+# decayed-memory variant (referee major comment 3 on Eq. (8): the memories
+# carried to t by the recurrence's decay, exp(sum_{r=e(c)+1..t} a_r) dH[c])
+# ----------------------------------------------------------------------------
+def _recurrence_states(inp, b, h, start, stop, reset_at=None):
+    """Plain token-by-token recurrence H_t = exp(dt_t A) H_{t-1} + dt_t B_t x_t^T
+    for one (b, h) from zero at ``start``; with ``reset_at`` (a set of
+    positions) the state restarts from zero before those tokens.  Returns
+    {t: H_t}."""
+    N = inp["Bm"].shape[-1]
+    P = inp["x"].shape[-1]
+    Hs = np.zeros((N, P))
+    out = {}
+    for t in range(start, stop):
+        if reset_at is not None and t in reset_at:
+            Hs = np.zeros((N, P))
+        dtt = float(inp["dt"][b, t, h])
+        Hs = np.exp(dtt * float(inp["A"][h])) * Hs + dtt * np.outer(
+            inp["Bm"][b, t].astype(np.float64), inp["x"][b, t, h].astype(np.float64))
+        out[t] = Hs
+    return out
+
+
+def pin_decayed_memories_sum_to_state(orc):
+    """With decayed memories, sum_{c < k(t)} of the carried dH[c] is exactly
+    the part of the SSM state H_t that tokens before chunk k(t) left behind:
+    H_t minus the state the tokens of chunk k(t) up to t build from zero.
+    With Q = 0 every score is 0, the softmax is uniform over the k(t)
+    memories and o_t = C_t^T (H_t - H_t^in) / k(t).  Both states come from a
+    token-by-token recurrence written here; L is not a multiple of S."""
+    Bz, L, H, P, N, S = 2, 44, 2, 3, 4, 8
+    inp = _rand_layer(13, Bz, L, H, P, N, dt_scale=0.5)
+    Q = np.zeros_like(inp["Q"])
+    r = orc.layer_forward(inp["x"], inp["dt"], inp["A"], inp["Bm"], inp["Cm"], Q, inp["E"], S,
+                          g=1.0, decayed=True)
+    chunk_starts = set(range(0, L, S))
+    for b in range(Bz):
+        for h in range(H):
+            full = _recurrence_states(inp, b, h, 0, L)
+            inner = _recurrence_states(inp, b, h, 0, L, reset_at=chunk_starts)
+            for t in range(L):
+                k = t // S
+                if k == 0:
+                    assert np.all(r["o"][b, t, h] == 0.0)
+                    continue
+                expect = inp["Cm"][b, t].astype(np.float64) @ (full[t] - inner[t]) / k
+                _close(r["o"][b, t, h], expect, 1e-11, f"decayed o[b={b},t={t},h={h}]")
+
+
+def pin_decayed_bruteforce_attention(orc):
+    """Decayed keys and values materialised per token and fed to torch's
+    scaled-dot-product attention.  The factor for memory c at token t is the
+    fraction of a unit placed in the state at e(c) that survives to t, taken
+    from a scalar run of the recurrence with no further input.  With A = 0
+    nothing decays and the variant equals the raw-memory SMA."""
+    Bz, L, H, P, N, S = 1, 40, 2, 5, 6, 8
+    inp = _rand_layer(14, Bz, L, H, P, N, dt_scale=0.6)
+    C = L // S
+    dH = np.random.default_rng(144).standard_normal((Bz, H, C, N, P))
+    ys = np.random.default_rng(145).standard_normal((Bz, L, H, P))
+    g = 0.5
+    r = orc.sma(inp["Q"], inp["E"], inp["Cm"], dH, S, g=g, y_ssd=ys, dt=inp["dt"], A=inp["A"])
+    Q, E, Cm, M = (torch.from_numpy(v.astype(np.float64)) for v in
+                   (inp["Q"], inp["E"], inp["Cm"], dH))
+    for h in range(H):
+        surv = np.zeros((C, L))   # surv[c, t]: what is left at t of a unit held at e(c)
+        for c in range(C):
+            z = 1.0
+            for t in range(c * S + S, L):
+                z = np.exp(float(inp["dt"][0, t, h]) * float(inp["A"][h])) * z
+                surv[c, t] = z
+        for t in range(L):
+            k = t // S
+            if k == 0:
+                continue
+            w = torch.from_numpy(surv[:k, t])[:, None]
+            Kt = w * torch.einsum("cnp,p->cn", M[0, h, :k], E[0, t, h])
+            Vt = w * torch.einsum("n,cnp->cp", Cm[0, t], M[0, h, :k])
+            expect = torch.nn.functional.scaled_dot_product_attention(
+                Q[0, t, h][None, None, None, :], Kt[None, None], Vt[None, None])[0, 0, 0].numpy()
+            _close(r["o"][0, t, h], expect, 1e-12, f"decayed o[t={t},h={h}]")
+            _close(r["y"][0, t, h], ys[0, t, h] + g * expect, 1e-12, "decayed gated y")
+    zeroA = np.zeros_like(inp["A"])
+    r0 = orc.sma(inp["Q"], inp["E"], inp["Cm"], dH, S, g=g, y_ssd=ys, dt=inp["dt"], A=zeroA)
+    raw = orc.sma(inp["Q"], inp["E"], inp["Cm"], dH, S, g=g, y_ssd=ys)
+    assert np.array_equal(r0["y"], raw["y"]), "A = 0: decayed and raw memories differ"
+
+
 ALL_PINS = [
     pin_closed_form_single_token,
     pin_quadratic_form,
@@ -401,4 +489,6 @@ ALL_PINS = [
     pin_partial_last_chunk,
     pin_ragged_prefill_then_decode,
     pin_cache_ratio,
+    pin_decayed_memories_sum_to_state,
+    pin_decayed_bruteforce_attention,
 ]

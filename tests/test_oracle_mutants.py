@@ -47,6 +47,13 @@ MUTATIONS = [
     ("partial_chunk_not_closed", "if (t % S == S - 1 || t == L - 1) {", "if (t % S == S - 1) {", 0),
     ("sma_memory_stride_floor", "const int nchunks = (L + S - 1) / S;\n    const int b = unit / H, h = unit % H;\n    const int nrows",
      "const int nchunks = L / S;\n    const int b = unit / H, h = unit % H;\n    const int nrows", 0),
+    ("decay_window_from_e", "for (int r = ec + 1; r <= t; ++r)", "for (int r = ec; r <= t; ++r)", 0),
+    ("decay_window_before_t", "for (int r = ec + 1; r <= t; ++r)", "for (int r = ec + 1; r < t; ++r)", 0),
+    ("decay_value_only", "key[n] = wdec * acc;", "key[n] = acc;", 0),
+    ("decay_key_only", "val[(size_t)cc * P + p] = wdec * acc;", "val[(size_t)cc * P + p] = acc;", 0),
+    ("decay_wrong_head", "(double)c->dt[((size_t)b * L + r) * H + h] * (double)c->A[h];",
+     "(double)c->dt[((size_t)b * L + r) * H + h] * (double)c->A[0];", 0),
+    ("decay_sign_flipped", "wdec = exp(logdec);", "wdec = exp(-logdec);", 0),
 ]
 
 
