@@ -135,6 +135,33 @@ dart_status dart_sma_forward(const dart_dims* dims, dart_dtype dtype,
                              float g, const float* y_ssd, float* out, void* stream);
 
 /*
+ * Workspace for dart_sma_forward_decayed, in bytes: the per-token in-chunk
+ * log-decay prefix (B*H*C*S floats, padded to 256 bytes) and the per-chunk
+ * prefix of chunk log-decays (B*H*C doubles).  0 for invalid dims.
+ */
+size_t dart_sma_decayed_workspace_bytes(const dart_dims* dims);
+
+/*
+ * Decayed-memory variant of dart_sma_forward (referee major comment 3 on SMA
+ * Eq. (8), Pith review of DART: the memories carried to the query token by
+ * the recurrence's decay instead of used raw).  For token t in chunk k(t)
+ * and each c < k(t) memory c is first scaled by
+ *   w_{t,c} = exp( A_h * sum_{r=e(c)+1}^{t} dt_r ),   e(c) = (c+1) S - 1,
+ * the share of dH[c] still present in the SSM state at t, and then used as
+ * in dart_sma_forward for both the key and the value:
+ *   s_{t,c} = w_{t,c} Q_t . (dH[c] E_t) / sqrt(N),  v_{t,c} = w_{t,c} C_t^T dH[c].
+ *   dt [B,L,H], A [H]: float, the same tensors the scan was given.
+ *   workspace: device scratch of dart_sma_decayed_workspace_bytes(), 16-byte
+ *   aligned; contents on entry do not matter and are not preserved.
+ * Other arguments, layouts, output modes and errors as dart_sma_forward.
+ * Enqueues the two decay-prefix kernels before the attention kernel.
+ */
+dart_status dart_sma_forward_decayed(const dart_dims* dims, dart_dtype dtype,
+                                     const void* Q, const void* E, const void* Cm, const void* dH,
+                                     const float* dt, const float* A, float g, const float* y_ssd,
+                                     float* out, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Workspace for dart_decode_step: per (sequence, head, split) partial softmax
  * statistics and partial outputs.  Pass at least this many bytes.
  */

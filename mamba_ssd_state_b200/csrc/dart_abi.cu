@@ -170,6 +170,51 @@ dart_status dart_sma_forward(const dart_dims* d, dart_dtype dtype, const void* Q
     return DART_OK;
 }
 
+size_t dart_sma_decayed_workspace_bytes(const dart_dims* d) {
+    if (!d) return 0;
+    return dart::sma_decay_workspace_bytes(d->batch, d->seqlen, d->nheads, d->chunk);
+}
+
+dart_status dart_sma_forward_decayed(const dart_dims* d, dart_dtype dtype, const void* Q, const void* E,
+                                     const void* Cm, const void* dH, const float* dt, const float* A, float g,
+                                     const float* y_ssd, float* out, void* workspace, size_t workspace_bytes,
+                                     void* stream) {
+    t_err[0] = 0;
+    dart_status st = check_common(d, dtype, true);
+    if (st != DART_OK) return st;
+    if (!dart::sma_supported(d->dstate, d->headdim, d->chunk, dtype))
+        return fail(DART_ERR_UNSUPPORTED, "dart_sma_forward_decayed: (N=%d, P=%d, S=%d) not compiled",
+                    d->dstate, d->headdim, d->chunk);
+    DART_REQUIRE_PTR(Q); DART_REQUIRE_PTR(E); DART_REQUIRE_PTR(Cm); DART_REQUIRE_PTR(dH);
+    DART_REQUIRE_PTR(dt); DART_REQUIRE_PTR(A);
+    DART_OPTIONAL_PTR(y_ssd); DART_REQUIRE_PTR(out); DART_REQUIRE_PTR(workspace);
+    if (reinterpret_cast<uintptr_t>(workspace) % 16 != 0)
+        return fail(DART_ERR_INVALID_ARG, "dart_sma_forward_decayed: workspace not 16-byte aligned");
+    const size_t need = dart_sma_decayed_workspace_bytes(d);
+    if (workspace_bytes < need)
+        return fail(DART_ERR_INVALID_ARG, "workspace: %zu bytes, need %zu", workspace_bytes, need);
+    if (y_ssd && y_ssd != out) {
+        const size_t bytes = (size_t)d->batch * d->seqlen * d->nheads * d->headdim * sizeof(float);
+        const uintptr_t ya = reinterpret_cast<uintptr_t>(y_ssd), oa = reinterpret_cast<uintptr_t>(out);
+        if (ya < oa + bytes && oa < ya + bytes)
+            return fail(DART_ERR_INVALID_ARG,
+                        "dart_sma_forward_decayed: out overlaps y_ssd without being the same pointer");
+    }
+    const int C = (d->seqlen + d->chunk - 1) / d->chunk;
+    float* la2 = static_cast<float*>(workspace);
+    const size_t la2_bytes = ((sizeof(float) * (size_t)d->batch * d->nheads * C * d->chunk) + 255) & ~size_t(255);
+    double* gpre = reinterpret_cast<double*>(static_cast<uint8_t*>(workspace) + la2_bytes);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = dart::launch_sma_decay_terms(d->batch, d->seqlen, d->nheads, d->chunk, dt, A, la2, gpre, s);
+    if (e != cudaSuccess) return cuda_fail(e, "dart_sma_forward_decayed: decay terms");
+    dart::SmaArgs a{d->batch, d->seqlen, d->nheads, d->headdim, d->dstate, d->chunk,
+                    Q, E, Cm, dH, g, y_ssd, out, status_word(), la2, gpre};
+    if (!a.status) return fail(DART_ERR_CUDA, "dart_sma_forward_decayed: no device status word");
+    e = dart::launch_sma(a, dtype, s);
+    if (e != cudaSuccess) return cuda_fail(e, "dart_sma_forward_decayed launch");
+    return DART_OK;
+}
+
 size_t dart_decode_step_workspace_bytes(const dart_dims* d, dart_dtype, int cmax) {
     if (!d || cmax < 0) return 0;
     const size_t ns = (size_t)dart::decode_num_splits(d->batch, d->nheads, cmax);

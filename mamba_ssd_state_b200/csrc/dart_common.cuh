@@ -113,6 +113,11 @@ struct SmaArgs {
     const void* Q; const void* E; const void* Cm; const void* dH;
     float g; const float* y_ssd; float* out;
     int* status;  // device status word
+    // Decayed-memory variant (both set) or raw memories (both null): the
+    // base-2 exponent of memory c's decay at token t of chunk k is
+    // la2[b,h,t] + gpre[b,h,k] - gpre[b,h,c+1] (see sma_decay.cu).
+    const float* la2;     // [B,H,C*S] fp32
+    const double* gpre;   // [B,H,C] fp64
 };
 struct DecodeArgs {
     int B, H, P, N, S, cmax, nsplit;
@@ -135,6 +140,11 @@ cudaError_t launch_ssd_scan_tc(const ScanArgs& a, cudaStream_t st);
 bool sma_supported(int N, int P, int S, dart_dtype dt);
 bool sma_tc_applicable(int N, int P, int S, dart_dtype dt);
 cudaError_t launch_sma_tc(const SmaArgs& a, cudaStream_t st);
+// Decay terms of the decayed-memory SMA from dt [B,L,H] and A [H] into la2 and
+// gpre (layouts as in SmaArgs); two launches.
+cudaError_t launch_sma_decay_terms(int B, int L, int H, int S, const float* dt, const float* A,
+                                   float* la2, double* gpre, cudaStream_t st);
+size_t sma_decay_workspace_bytes(int B, int L, int H, int S);
 const char* sma_impl_name(int N, int P, int S, dart_dtype dt);
 bool decode_supported(int N, int P, int S, dart_dtype dt);
 int decode_num_splits(int B, int H, int cmax);

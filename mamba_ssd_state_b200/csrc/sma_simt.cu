@@ -7,6 +7,9 @@
 // which equals Q_t . (dH[c] E_t) / sqrt(N) -- the key read out of the memory by
 // contracting its value axis -- by associativity.  An online softmax over c
 // accumulates o_t; the epilogue writes y_ssd + g * o_t (or o_t alone).
+// In the decayed-memory variant (referee comment 3 on Eq. (8)) memory c is
+// scaled by w = exp(sum_{r=e(c)+1}^{t} dt_r A_h) before use: the score becomes
+// w s and the value w v (terms from sma_decay.cu).
 //
 // One block = 64 query tokens of one (b, h), all in the same chunk; 4 threads
 // per token, each owning P/4 output columns.  The memory dH[c] is staged in
@@ -47,6 +50,11 @@ __global__ void __launch_bounds__(kThreads) sma_simt_kernel(SmaArgs a) {
         e[j] = live ? ldf(E + (((size_t)b * a.L + t) * a.H + h) * P + pg * PT + j) : 0.f;
     }
     float mrun = -INFINITY, lrun = 0.f;
+    const bool decayed = a.la2 != nullptr;
+    const size_t bh = (size_t)b * a.H + h;
+    // decayed variant: t's in-chunk log2 prefix and the chunk prefix at k
+    const float la_t = decayed && live ? a.la2[bh * C * S + t] : 0.f;
+    const double g_k = decayed && k > 0 ? a.gpre[bh * C + k] : 0.0;
 
     if (k > 0) {
         for (int i = threadIdx.x; i < kTQ * N; i += blockDim.x) {
@@ -84,12 +92,18 @@ __global__ void __launch_bounds__(kThreads) sma_simt_kernel(SmaArgs a) {
             for (int j = 0; j < PT; ++j) s = fmaf(u[j], e[j], s);
             s += __shfl_xor_sync(0xffffffffu, s, 1);
             s += __shfl_xor_sync(0xffffffffu, s, 2);
+            float wd = 1.f;   // decay of memory c at token t (1 for raw memories)
+            if (decayed) {
+                wd = exp2f(la_t + (float)(g_k - a.gpre[bh * C + c + 1]));
+                s *= wd;
+            }
             const float mnew = fmaxf(mrun, s);
             const float alpha = exp2f(mrun - mnew);
             const float w = exp2f(s - mnew);
             lrun = lrun * alpha + w;
+            const float wv = w * wd;
 #pragma unroll
-            for (int j = 0; j < PT; ++j) o[j] = fmaf(o[j], alpha, w * v[j]);
+            for (int j = 0; j < PT; ++j) o[j] = fmaf(o[j], alpha, wv * v[j]);
             mrun = mnew;
         }
     }

@@ -38,6 +38,12 @@
 // issues the MMAs and owns the FULL / EMPTY barriers they wait on, the
 // peer's loads complete on them and its epilogue warps arrive on them
 // remotely; the commits reach both CTAs.  S = 128 runs one CTA per tile.
+//
+// Decayed memories (kDecay; referee comment 3 on Eq. (8)): memory c reaches
+// token t scaled by w = exp(sum_{r=e(c)+1}^{t} dt_r A_h), and since U and V are
+// linear in the memory the scale is applied in the epilogue: score w s, value
+// weight p w (the softmax normaliser keeps p).  The base-2 exponent comes from
+// the per-token and per-chunk prefixes of sma_decay.cu.
 #include <cuda_bf16.h>
 #include <string.h>
 
@@ -104,6 +110,8 @@ struct SmaTcParams {
     const __nv_bfloat16* E;
     const float* y_ssd;
     float* out;
+    const float* la2;     // decayed memories: [B,H,C*S] in-chunk log2-decay prefix
+    const double* gpre;   // decayed memories: [B,H,C] chunk-level prefix
     float g;
     int add_into_out;  // 1: out already holds y_ssd, the tile end adds g o / l; 0: it stores o / l
     int B, L, H, S, C;
@@ -131,7 +139,7 @@ __device__ __forceinline__ Tile decode_tile(const SmaTcParams& p, int i, int ran
     return t;
 }
 
-template <bool kPair>
+template <bool kPair, bool kDecay>
 __global__ void __launch_bounds__(kThreads, 1) sma_tc_kernel(const __grid_constant__ SmaTcParams p) {
     using Rg = Ring<kPair>;
     extern __shared__ uint8_t smem_raw[];
@@ -405,10 +413,25 @@ __global__ void __launch_bounds__(kThreads, 1) sma_tc_kernel(const __grid_consta
                 }
                 float m = -INFINITY;
                 const int nbatch = (t.k + kCB - 1) / kCB;
+                // decayed memories: this row's in-chunk prefix and the chunk prefix at k
+                const size_t bh = (size_t)t.b * p.H + t.h;
+                float la_row = 0.f;
+                double g_k = 0.0;
+                if (kDecay) {
+                    la_row = p.la2[bh * p.C * p.S + t.t0 + row];   // t0 + row < C * S
+                    g_k = p.gpre[bh * p.C + t.k];
+                }
                 for (int j = 0; j < nbatch; ++j, ++it_u) {
                     const int nv = min(kCB, t.k - kCB * j);
                     const uint32_t ph = (uint32_t)it_u & 1u;
                     float part[kCB] = {0.f, 0.f, 0.f, 0.f};
+                    float wd[kCB] = {1.f, 1.f, 1.f, 1.f};   // decay of each memory at this row
+                    if (kDecay) {
+#pragma unroll
+                        for (int c = 0; c < kCB; ++c)
+                            if (c < nv)   // memory kCB j + c < k, so its index + 1 <= k < C
+                                wd[c] = exp2f(la_row + (float)(g_k - __ldg(p.gpre + bh * p.C + kCB * j + c + 1)));
+                    }
                     if (ok) ok = mbar_wait_warp(bar(U_FULL), ph, wc, 9);
                     if (ok) {
                         tc_fence_after();
@@ -449,7 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1) sma_tc_kernel(const __grid_consta
                     const float other[kCB] = {pp.x, pp.y, pp.z, pp.w};
                     float sc[kCB];
 #pragma unroll
-                    for (int c = 0; c < kCB; ++c) sc[c] = c < nv ? (part[c] + other[c]) * sscale : -INFINITY;
+                    for (int c = 0; c < kCB; ++c) sc[c] = c < nv ? (part[c] + other[c]) * sscale * wd[c] : -INFINITY;
                     float mnew = m;
 #pragma unroll
                     for (int c = 0; c < kCB; ++c) mnew = fmaxf(mnew, sc[c]);
@@ -471,7 +494,8 @@ __global__ void __launch_bounds__(kThreads, 1) sma_tc_kernel(const __grid_consta
                                 float v[kHalfP];
                                 tmem_ld_32x32b_x32(t_lane + kColV + (uint32_t)(c * kP + col0), v);
                                 tmem_ld_wait();
-                                const float2 w2 = make_float2(w[c], w[c]);
+                                const float wv = kDecay ? w[c] * wd[c] : w[c];
+                                const float2 w2 = make_float2(wv, wv);
 #pragma unroll
                                 for (int q = 0; q < kHalfP / 2; ++q)
                                     o2[q] = __ffma2_rn(w2, make_float2(v[2 * q], v[2 * q + 1]), o2[q]);
@@ -589,6 +613,9 @@ cudaError_t launch_sma_tc(const SmaArgs& a, cudaStream_t st) {
         if (!encode_tile_map_f32(&p.tmap_o, 4, a.out, dims, strides, box)) return cudaErrorInvalidValue;
     }
     p.E = static_cast<const __nv_bfloat16*>(a.E);
+    p.la2 = a.la2;
+    p.gpre = a.gpre;
+    const bool decayed = a.la2 != nullptr;
     p.y_ssd = a.y_ssd;
     p.out = a.out;
     p.g = a.g;
@@ -610,7 +637,7 @@ cudaError_t launch_sma_tc(const SmaArgs& a, cudaStream_t st) {
         p.cta_per_tile = 2;
         p.tiles_per_chunk = a.S / (2 * kBQ);
         p.total_tiles = C * a.B * a.H * p.tiles_per_chunk;
-        auto kern = sma_tc_kernel<true>;
+        auto kern = decayed ? sma_tc_kernel<true, true> : sma_tc_kernel<true, false>;
         if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes)) != cudaSuccess)
             return e;
         cudaLaunchConfig_t cfg;
@@ -638,7 +665,7 @@ cudaError_t launch_sma_tc(const SmaArgs& a, cudaStream_t st) {
         p.tiles_per_chunk = a.S / kBQ;
         p.total_tiles = C * a.B * a.H * p.tiles_per_chunk;
         const int grid = p.total_tiles < sms ? p.total_tiles : sms;
-        auto kern = sma_tc_kernel<false>;
+        auto kern = decayed ? sma_tc_kernel<false, true> : sma_tc_kernel<false, false>;
         if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes)) != cudaSuccess)
             return e;
         kern<<<grid, kThreads, kSmemBytes, st>>>(p);

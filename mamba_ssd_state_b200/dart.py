@@ -31,7 +31,8 @@ _STATUS = {0: "DART_OK", 1: "DART_ERR_INVALID_ARG", 2: "DART_ERR_UNSUPPORTED", 3
 EXPORTS = ("dart_ssd_chunk_scan_workspace_bytes", "dart_ssd_chunk_scan", "dart_sma_forward",
            "dart_decode_step_workspace_bytes", "dart_decode_step", "dart_supported",
            "dart_sync_status", "dart_last_error", "dart_abi_version", "dart_launch_count",
-           "dart_sma_impl", "dart_decode_step_noalloc")
+           "dart_sma_impl", "dart_decode_step_noalloc", "dart_sma_decayed_workspace_bytes",
+           "dart_sma_forward_decayed")
 
 
 class DartError(RuntimeError):
@@ -64,6 +65,11 @@ def load(path: str = LIBRARY) -> ctypes.CDLL:
     lib.dart_ssd_chunk_scan.argtypes = [D, ctypes.c_int] + [_P] * 10 + [ctypes.c_size_t, _P]
     lib.dart_sma_forward.restype = ctypes.c_int
     lib.dart_sma_forward.argtypes = [D, ctypes.c_int] + [_P] * 4 + [ctypes.c_float, _P, _P, _P]
+    lib.dart_sma_decayed_workspace_bytes.restype = ctypes.c_size_t
+    lib.dart_sma_decayed_workspace_bytes.argtypes = [D]
+    lib.dart_sma_forward_decayed.restype = ctypes.c_int
+    lib.dart_sma_forward_decayed.argtypes = ([D, ctypes.c_int] + [_P] * 6 + [ctypes.c_float, _P, _P, _P,
+                                             ctypes.c_size_t, _P])
     lib.dart_decode_step_workspace_bytes.restype = ctypes.c_size_t
     lib.dart_decode_step_workspace_bytes.argtypes = [D, ctypes.c_int, ctypes.c_int]
     lib.dart_decode_step.restype = ctypes.c_int
@@ -230,13 +236,52 @@ def dart_sma_forward(Q, E, Cm, dH, chunk: int, g: float, y_ssd=None, *, out=None
     return _to_host(out)[0] if host else out
 
 
+def dart_sma_forward_decayed(Q, E, Cm, dH, dt, A, chunk: int, g: float, y_ssd=None, *, out=None,
+                             workspace=None):
+    """The decayed-memory variant of dart_sma_forward: memory c reaches token
+    t scaled by exp(A_h sum_{r=e(c)+1..t} dt_r).  dt [B,L,H] and A [H] are
+    float32, as given to the scan.  Returns float32 [B,L,H,P]."""
+    lib = load()
+    host = not Q.is_cuda
+    dev = _device_of(Q, E, Cm, dH, dt, A)
+    Q, E, Cm, dH = (_dev(v, dev, Q.dtype) for v in (Q, E, Cm, dH))
+    dt, A = _dev(dt, dev, torch.float32), _dev(A, dev, torch.float32)
+    y_ssd = _dev(y_ssd, dev, torch.float32)
+    Bsz, L, H, N = Q.shape
+    P = E.shape[-1]
+    C = -(-L // chunk)
+    _shape("E", E, (Bsz, L, H, P)); _shape("Cm", Cm, (Bsz, L, N)); _shape("dH", dH, (Bsz, H, C, N, P))
+    _shape("dt", dt, (Bsz, L, H)); _shape("A", A, (H,))
+    if y_ssd is not None:
+        _shape("y_ssd", y_ssd, (Bsz, L, H, P))
+    if out is None:
+        out = torch.empty((Bsz, L, H, P), device=dev, dtype=torch.float32)
+    dims = Dims(Bsz, L, H, P, N, chunk, 1)
+    wsb = lib.dart_sma_decayed_workspace_bytes(ctypes.byref(dims))
+    if workspace is None:
+        workspace = torch.empty(max(16, wsb), device=dev, dtype=torch.uint8)
+    with torch.cuda.device(dev):
+        _check(lib.dart_sma_forward_decayed(ctypes.byref(dims), _dtype_code(Q.dtype), _ptr(Q), _ptr(E),
+                                            _ptr(Cm), _ptr(dH), _ptr(dt), _ptr(A), float(g), _ptr(y_ssd),
+                                            _ptr(out), _ptr(workspace), workspace.numel(), _stream()))
+    return _to_host(out)[0] if host else out
+
+
+def sma_decayed_workspace_bytes(batch, seqlen, nheads, headdim, dstate, chunk) -> int:
+    return int(load().dart_sma_decayed_workspace_bytes(
+        ctypes.byref(Dims(batch, seqlen, nheads, headdim, dstate, chunk, 1))))
+
+
 def layer_forward(x, dt, A, Bm, Cm, Q, E, chunk: int, g: float, init_state=None, *,
-                  outputs=("y", "dH", "states"), buffers: Optional[dict] = None):
+                  outputs=("y", "dH", "states"), buffers: Optional[dict] = None,
+                  decayed: bool = False):
     """The DART layer forward: scan, then SMA with the gated residual written
     in place over y_ssd.  Returns a dict with the requested `outputs` among
     y, dH, states.  With host (CPU) inputs the inputs are copied to the
     current device and only the requested outputs are copied back.
-    `buffers` may hold preallocated device tensors y, dH, states, workspace."""
+    `buffers` may hold preallocated device tensors y, dH, states, workspace
+    (and sma_workspace for the decayed variant).  ``decayed`` selects the
+    decayed-memory SMA."""
     host = not x.is_cuda
     dev = _device_of(x)
     args = [_dev(v, dev) for v in (x, dt, A, Bm, Cm, Q, E)]
@@ -244,7 +289,11 @@ def layer_forward(x, dt, A, Bm, Cm, Q, E, chunk: int, g: float, init_state=None,
     b = buffers or {}
     y, dH, states = dart_ssd_chunk_scan(*args[:5], chunk, init_state, y_ssd=b.get("y"), dH=b.get("dH"),
                                         states=b.get("states"), workspace=b.get("workspace"))
-    dart_sma_forward(args[5], args[6], args[4], dH, chunk, g, y, out=y)
+    if decayed:
+        dart_sma_forward_decayed(args[5], args[6], args[4], dH, args[1], args[2], chunk, g, y, out=y,
+                                 workspace=b.get("sma_workspace"))
+    else:
+        dart_sma_forward(args[5], args[6], args[4], dH, chunk, g, y, out=y)
     res = {"y": y, "dH": dH, "states": states}
     if host:
         return dict(zip(outputs, _to_host(*(res[k] for k in outputs))))

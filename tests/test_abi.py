@@ -123,6 +123,34 @@ def test_sma_rejects_partially_overlapping_out(lib):
     assert b"overlaps" in lib.dart_last_error()
 
 
+def test_sma_decayed_workspace_and_validation(lib):
+    """Workspace = B*H*C*S floats (padded to 256 bytes) + B*H*C doubles, C =
+    ceil(L/S); missing dt/A, a small or misaligned workspace and uncompiled
+    shapes are rejected on the host."""
+    d = dart.Dims(2, 500, 3, 64, 128, 256, 1)
+    C = 2
+    la2 = (2 * 3 * C * 256 * 4 + 255) // 256 * 256
+    assert lib.dart_sma_decayed_workspace_bytes(ctypes.byref(d)) == la2 + 2 * 3 * C * 8
+    assert lib.dart_sma_decayed_workspace_bytes(None) == 0
+    ws = lib.dart_sma_decayed_workspace_bytes(ctypes.byref(d))
+    f = lib.dart_sma_forward_decayed
+    assert f(ctypes.byref(d), dart.DART_BF16, FAKE, FAKE, FAKE, FAKE, None, FAKE, 0.5, None, FAKE,
+             FAKE, ws, None) == dart.DART_ERR_INVALID_ARG
+    assert f(ctypes.byref(d), dart.DART_BF16, FAKE, FAKE, FAKE, FAKE, FAKE, None, 0.5, None, FAKE,
+             FAKE, ws, None) == dart.DART_ERR_INVALID_ARG
+    assert f(ctypes.byref(d), dart.DART_BF16, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0.5, None, FAKE,
+             FAKE, ws - 1, None) == dart.DART_ERR_INVALID_ARG
+    assert b"workspace" in lib.dart_last_error()
+    assert f(ctypes.byref(d), dart.DART_BF16, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0.5, None, FAKE,
+             ctypes.c_void_p((1 << 32) + 8), ws, None) == dart.DART_ERR_INVALID_ARG
+    base = 1 << 32
+    assert f(ctypes.byref(d), dart.DART_BF16, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0.5,
+             ctypes.c_void_p(base), ctypes.c_void_p(base + 4096), FAKE, ws, None) == dart.DART_ERR_INVALID_ARG
+    d.chunk = 96
+    assert f(ctypes.byref(d), dart.DART_BF16, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0.5, None, FAKE,
+             FAKE, 1 << 30, None) == dart.DART_ERR_UNSUPPORTED
+
+
 def test_decode_rejects_bad_args(lib):
     d = dart.Dims(4, 0, 2, 64, 128, 256, 1)
     ws = lib.dart_decode_step_workspace_bytes(ctypes.byref(d), dart.DART_BF16, 9)
