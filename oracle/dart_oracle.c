@@ -51,7 +51,11 @@
  *    a cache of completed chunk memories; when the token closes its chunk the
  *    running contribution is appended to the cache after the token's output
  *    is formed (DART abstract; Pith review "If this is right": the
- *    length-dependent inference cache is the set of chunk memories).
+ *    length-dependent inference cache is the set of chunk memories).  In the
+ *    decayed variant each cached memory carries the log-decay accumulated
+ *    since its chunk closed, sum_{r=e(c)+1}^{t-1} dt_r A_h; the step adds the
+ *    new token's dt_t A_h to it, uses exp of the result as the memory's
+ *    factor, and a memory appended at t starts from zero.
  *
  * Readings where the pages are silent: mask c < k(t) (strict), scale 1/sqrt(N),
  * exp(dt*A) discretisation with input dt*B x^T, no D skip, ngroups = 1 (B and C
@@ -305,6 +309,7 @@ typedef struct {
     const float *x, *dt, *A, *Bm, *Cm, *Q, *E;
     double g;
     double *state, *dHcur, *cache;
+    double* memlog; /* nullable: [Bs,H,cmax] log-decay of each cached memory */
     const int *nchunks, *pos;
     double* y;
 } dec_ctx;
@@ -346,15 +351,21 @@ static void decode_unit(void* vctx, int unit) {
         double* key = (double*)malloc(sizeof(double) * (size_t)N);
         for (int cc = 0; cc < nmem; ++cc) {
             const double* M = c->cache + (bh * (size_t)c->cmax + cc) * (size_t)N * P;
+            double wdec = 1.0;
+            if (c->memlog) {
+                double* lw = c->memlog + bh * (size_t)c->cmax + cc;
+                *lw += dtt * (double)c->A[h]; /* now sum_{r=e(c)+1}^{t} dt_r A_h */
+                wdec = exp(*lw);
+            }
             for (int n = 0; n < N; ++n) {
                 double acc = 0.0;
                 for (int p = 0; p < P; ++p) acc += M[n * P + p] * (double)Et[p];
-                key[n] = acc;
+                key[n] = wdec * acc;
             }
             for (int p = 0; p < P; ++p) {
                 double acc = 0.0;
                 for (int n = 0; n < N; ++n) acc += (double)Ct[n] * M[n * P + p];
-                val[(size_t)cc * P + p] = acc;
+                val[(size_t)cc * P + p] = wdec * acc;
             }
             double s = 0.0;
             for (int n = 0; n < N; ++n) s += (double)Qt[n] * key[n];
@@ -378,26 +389,29 @@ static void decode_unit(void* vctx, int unit) {
         double* slot = c->cache + (bh * (size_t)c->cmax + nmem) * (size_t)N * P;
         memcpy(slot, D, sizeof(double) * (size_t)N * P);
         memset(D, 0, sizeof(double) * (size_t)N * P);
+        if (c->memlog) c->memlog[bh * (size_t)c->cmax + nmem] = 0.0; /* closes at this token */
     }
 }
 
 /*
  * x[Bs,H,P] dt[Bs,H] A[H] Bm[Bs,N] Cm[Bs,N] Q[Bs,H,N] E[Bs,H,P] (float);
  * state, dH_cur [Bs,H,N,P], cache [Bs,H,cmax,N,P], y [Bs,H,P] (double);
- * nchunks[Bs], pos[Bs] in/out.  Returns -1 (and changes nothing) when an
- * append would overflow the cache or a counter is out of range.
+ * nchunks[Bs], pos[Bs] in/out; memlog [Bs,H,cmax] (double, in/out) selects
+ * the decayed-memory variant when not NULL.  Returns -1 (and changes
+ * nothing) when an append would overflow the cache or a counter is out of
+ * range.
  */
 int oracle_decode_step(const oracle_dims* d, int cmax, const float* x, const float* dt,
                        const float* A, const float* Bm, const float* Cm, const float* Q,
                        const float* E, double g, double* state, double* dH_cur, double* cache,
-                       int* nchunks, int* pos, double* y, int nthreads) {
+                       int* nchunks, int* pos, double* memlog, double* y, int nthreads) {
     if (!d || d->chunk <= 0) return -1;
     for (int b = 0; b < d->batch; ++b) {
         if (nchunks[b] < 0 || nchunks[b] > cmax) return -1;
         if (pos[b] < 0 || pos[b] >= d->chunk) return -1;
         if (pos[b] == d->chunk - 1 && nchunks[b] >= cmax) return -1;
     }
-    dec_ctx c = {d, cmax, x, dt, A, Bm, Cm, Q, E, g, state, dH_cur, cache, nchunks, pos, y};
+    dec_ctx c = {d, cmax, x, dt, A, Bm, Cm, Q, E, g, state, dH_cur, cache, memlog, nchunks, pos, y};
     run_units(decode_unit, &c, d->batch * d->nheads, nthreads);
     for (int b = 0; b < d->batch; ++b) {
         if (pos[b] == d->chunk - 1) {

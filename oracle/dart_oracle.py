@@ -61,7 +61,7 @@ class Oracle:
         self.lib.oracle_decode_step.restype = ctypes.c_int
         self.lib.oracle_decode_step.argtypes = (
             [ctypes.POINTER(_Dims), ctypes.c_int] + [_P] * 7 + [ctypes.c_double]
-            + [_P] * 6 + [ctypes.c_int])
+            + [_P] * 7 + [ctypes.c_int])
 
     # ------------------------------------------------------------------
     @staticmethod
@@ -147,12 +147,18 @@ class Oracle:
         return {"y": r["y"], "o": r["o"], "y_ssd": y_ssd, "dH": dH, "states": st}
 
     def decode_step(self, x, dt, A, Bm, Cm, Q, E, g, state, dH_cur, cache, nchunks, pos,
-                    chunk: int):
+                    chunk: int, memlog=None):
         """One decode step.  state, dH_cur, cache (float64, C-contiguous) and
-        nchunks, pos (int32) are updated in place.  Returns y[Bs,H,P]."""
+        nchunks, pos (int32) are updated in place.  With ``memlog`` (float64
+        [Bs,H,cmax], updated in place: the log-decay each cached memory has
+        accumulated since its chunk closed) the memories are decayed to the
+        new token before use.  Returns y[Bs,H,P]."""
         x, dt, A, Bm, Cm, Q, E = (self._f32(v) for v in (x, dt, A, Bm, Cm, Q, E))
-        for arr, dtp in ((state, np.float64), (dH_cur, np.float64), (cache, np.float64),
-                         (nchunks, np.int32), (pos, np.int32)):
+        bufs = [(state, np.float64), (dH_cur, np.float64), (cache, np.float64),
+                (nchunks, np.int32), (pos, np.int32)]
+        if memlog is not None:
+            bufs.append((memlog, np.float64))
+        for arr, dtp in bufs:
             if arr.dtype != dtp or not arr.flags.c_contiguous:
                 raise ValueError("decode buffers must be contiguous with the documented dtype")
         Bs, H, P = x.shape
@@ -164,7 +170,7 @@ class Oracle:
                                          self._ptr(A), self._ptr(Bm), self._ptr(Cm),
                                          self._ptr(Q), self._ptr(E), float(g), self._ptr(state),
                                          self._ptr(dH_cur), self._ptr(cache), self._ptr(nchunks),
-                                         self._ptr(pos), self._ptr(y), self.nthreads)
+                                         self._ptr(pos), self._ptr(memlog), self._ptr(y), self.nthreads)
         if rc:
             raise ValueError("oracle_decode_step rejected its arguments")
         return y

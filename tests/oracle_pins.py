@@ -474,6 +474,56 @@ def pin_decayed_bruteforce_attention(orc):
     assert np.array_equal(r0["y"], raw["y"]), "A = 0: decayed and raw memories differ"
 
 
+def pin_decayed_decode_matches_prefill(orc):
+    """Decayed memories in decode: each cached memory carries the log-decay
+    accumulated since its chunk closed (the slot of a memory not yet appended
+    holds junk until the append sets it).  (1) Decoding a whole sequence from an
+    empty cache, and (2) decoding on from a prefill that stops inside a chunk,
+    with every cached memory's log-decay set to sum_{r=e(c)+1}^{L-1} dt_r A_h
+    (summed here from dt), both reproduce the decayed-memory layer forward
+    token by token, which the recurrence pins above."""
+    Bz, H, P, N, S = 2, 2, 3, 4, 8
+    T = 4 * S + 3
+    inp = _rand_layer(23, Bz, T, H, P, N, dt_scale=0.4)
+    g = 0.8
+    keys = ("x", "dt", "A", "Bm", "Cm", "Q", "E")
+    full = orc.layer_forward(*(inp[k] for k in keys), S, g, decayed=True)
+    cmax = T // S + 1
+    # (1) from an empty cache
+    cache = np.zeros((Bz, H, cmax, N, P))
+    state = np.zeros((Bz, H, N, P))
+    dcur = np.zeros((Bz, H, N, P))
+    memlog = np.full((Bz, H, cmax), 7.0)   # slots of memories not yet appended hold junk
+    nch = np.zeros((Bz,), np.int32)
+    pos = np.zeros((Bz,), np.int32)
+    for t in range(T):
+        y = orc.decode_step(inp["x"][:, t], inp["dt"][:, t], inp["A"], inp["Bm"][:, t],
+                            inp["Cm"][:, t], inp["Q"][:, t], inp["E"][:, t], g, state, dcur,
+                            cache, nch, pos, S, memlog=memlog)
+        _close(y, full["y"][:, t], 1e-12, f"decayed decode y at t={t}")
+    a = _log_decay(inp["dt"], inp["A"])
+    for c in range(T // S):
+        _close(memlog[:, :, c], a[:, (c + 1) * S:T].sum(1), 1e-12, f"memlog[{c}]")
+    # (2) from a ragged prefill
+    L = 2 * S + 5
+    pre = orc.layer_forward(*(inp[k][:, :L] if k != "A" else inp[k] for k in keys), S, g, decayed=True)
+    Cfull = L // S
+    cache = np.zeros((Bz, H, cmax, N, P))
+    cache[:, :, :Cfull] = pre["dH"][:, :, :Cfull]
+    state = np.ascontiguousarray(pre["states"][:, :, -1])
+    dcur = np.ascontiguousarray(pre["dH"][:, :, -1])
+    memlog = np.full((Bz, H, cmax), 7.0)
+    for c in range(Cfull):
+        memlog[:, :, c] = a[:, (c + 1) * S:L].sum(1)
+    nch = np.full((Bz,), Cfull, np.int32)
+    pos = np.full((Bz,), L % S, np.int32)
+    for t in range(L, T):
+        y = orc.decode_step(inp["x"][:, t], inp["dt"][:, t], inp["A"], inp["Bm"][:, t],
+                            inp["Cm"][:, t], inp["Q"][:, t], inp["E"][:, t], g, state, dcur,
+                            cache, nch, pos, S, memlog=memlog)
+        _close(y, full["y"][:, t], 1e-12, f"decayed decode after prefill, y at t={t}")
+
+
 ALL_PINS = [
     pin_closed_form_single_token,
     pin_quadratic_form,
@@ -491,4 +541,5 @@ ALL_PINS = [
     pin_cache_ratio,
     pin_decayed_memories_sum_to_state,
     pin_decayed_bruteforce_attention,
+    pin_decayed_decode_matches_prefill,
 ]

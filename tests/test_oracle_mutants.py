@@ -41,8 +41,8 @@ MUTATIONS = [
      "D[n * P + p] = D[n * P + p] + inp;", 1),
     ("decode_sees_open_chunk", "const int nmem = c->nchunks[b];",
      "const int nmem = c->nchunks[b] + (c->pos[b] == S - 1);", 0),
-    ("decode_no_reset_after_append", "memset(D, 0, sizeof(double) * (size_t)N * P);\n    }\n}",
-     "}\n}", 0),
+    ("decode_no_reset_after_append", "memset(D, 0, sizeof(double) * (size_t)N * P);\n        if (c->memlog)",
+     "if (c->memlog)", 0),
     ("decode_gate_dropped", "yt[p] += c->g * acc;", "yt[p] += acc;", 0),
     ("partial_chunk_not_closed", "if (t % S == S - 1 || t == L - 1) {", "if (t % S == S - 1) {", 0),
     ("sma_memory_stride_floor", "const int nchunks = (L + S - 1) / S;\n    const int b = unit / H, h = unit % H;\n    const int nrows",
@@ -54,6 +54,10 @@ MUTATIONS = [
     ("decay_wrong_head", "(double)c->dt[((size_t)b * L + r) * H + h] * (double)c->A[h];",
      "(double)c->dt[((size_t)b * L + r) * H + h] * (double)c->A[0];", 0),
     ("decay_sign_flipped", "wdec = exp(logdec);", "wdec = exp(-logdec);", 0),
+    ("decode_memlog_after_use", "*lw += dtt * (double)c->A[h]; /* now sum_{r=e(c)+1}^{t} dt_r A_h */\n                wdec = exp(*lw);",
+     "wdec = exp(*lw);\n                *lw += dtt * (double)c->A[h];", 0),
+    ("decode_memlog_not_reset", "if (c->memlog) c->memlog[bh * (size_t)c->cmax + nmem] = 0.0;", "", 0),
+    ("decode_decay_value_only", "key[n] = wdec * acc;", "key[n] = acc;", 1),
 ]
 
 
