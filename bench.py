@@ -60,6 +60,8 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true", help="skip timing the oracle")
     p.add_argument("--no-partial", action="store_true",
                    help="skip the forward with a partial last chunk (L = 8092)")
+    p.add_argument("--no-decayed", action="store_true",
+                   help="skip the forward with decayed memories (dart_sma_forward_decayed)")
     p.add_argument("--decode-steps", type=int, default=DEC.nsteps)
     p.add_argument("--reference-heads", type=int, default=0,
                    help="heads per reference-arm step (default: one per host core, at most 32)")
@@ -222,7 +224,7 @@ class Dist:
 # ---------------------------------------------------------------------------
 # GPU regions
 # ---------------------------------------------------------------------------
-def forward_region(args, dist, dart, shape=FWD):
+def forward_region(args, dist, dart, shape=FWD, decayed=False):
     dev = torch.device("cuda", torch.cuda.current_device())
     inp = synth.layer_inputs(shape, seed=dist.rank)
     d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
@@ -233,6 +235,8 @@ def forward_region(args, dist, dart, shape=FWD):
     states = torch.empty((B, H, C, N, P), device=dev, dtype=torch.float32)
     ws = torch.empty(max(16, dart.scan_workspace_bytes(B, L, H, P, N, S, torch.bfloat16)), device=dev,
                      dtype=torch.uint8)
+    sma_ws = torch.empty(max(16, dart.sma_decayed_workspace_bytes(B, L, H, P, N, S)), device=dev,
+                         dtype=torch.uint8) if decayed else None
     stream = torch.cuda.current_stream()
 
     def step(ev=None):
@@ -242,7 +246,11 @@ def forward_region(args, dist, dart, shape=FWD):
                                  workspace=ws)
         if ev:
             ev[1].record(stream)
-        dart.dart_sma_forward(d["Q"], d["E"], d["Cm"], dH, S, d["g"], y, out=y)
+        if decayed:
+            dart.dart_sma_forward_decayed(d["Q"], d["E"], d["Cm"], dH, d["dt"], d["A"], S, d["g"], y, out=y,
+                                          workspace=sma_ws)
+        else:
+            dart.dart_sma_forward(d["Q"], d["E"], d["Cm"], dH, S, d["g"], y, out=y)
         if ev:
             ev[2].record(stream)
 
@@ -313,10 +321,14 @@ def e2e_region(args, dist, dart, inp):
             "path": "dart.layer_forward on pinned host inputs, y returned to host"}
 
 
-def decode_region(args, dist, dart, peaks):
+def decode_region(args, dist, dart, peaks, decayed=False):
     dev = torch.device("cuda", torch.cuda.current_device())
     init = synth.decode_initial(DEC, seed=dist.rank)
     work = {k: v.to(dev) for k, v in init.items()}
+    if decayed:
+        # log-decays of the cached memories (dart_decode_step_decayed), -U(0, 3)
+        g = torch.Generator().manual_seed(1000 + dist.rank)
+        work["memlog"] = (-3.0 * torch.rand((DEC.nseq, DEC.nheads, DEC.cmax), generator=g)).to(dev)
     saved = {k: v.clone() for k, v in work.items()}
     A = synth.decode_A(DEC, seed=dist.rank).to(dev)
     # the cache holds one free slot: at most S steps (one append) per run
@@ -335,7 +347,7 @@ def decode_region(args, dist, dart, peaks):
             ev[0].record(stream)
         dart.dart_decode_step(t["x"], t["dt"], A, t["Bm"], t["Cm"], t["Q"], t["E"], DEC.g, work["state"],
                               work["dH_cur"], work["cache"], work["nchunks"], work["pos"], DEC.chunk, y=y,
-                              workspace=ws)
+                              workspace=ws, memlog=work.get("memlog"))
         if ev:
             ev[1].record(stream)
 
@@ -367,6 +379,8 @@ def decode_region(args, dist, dart, peaks):
     # step s starts at pos = s % S with ncached + s // S memories; pos = S-1 appends
     total_bytes = sum(decode_bytes(DEC, DEC.ncached + s // DEC.chunk, s % DEC.chunk == DEC.chunk - 1)
                       for s in range(nsteps))
+    if decayed:   # each cached memory's log-decay is read and written once per step
+        total_bytes += sum(8 * DEC.nseq * DEC.nheads * (DEC.ncached + s // DEC.chunk) for s in range(nsteps))
     bytes_step = total_bytes / nsteps
     step_ms = statistics.mean(per)
     achieved = bytes_step / (step_ms / 1e3) / 1e9
@@ -531,12 +545,31 @@ def main():
                            "seqlen": ps.seqlen, "nheads": ps.nheads, "chunk": ps.chunk,
                            "last_chunk_tokens": ps.seqlen - (ps.nchunks - 1) * ps.chunk}}
             line["gpu_launches"] += part["launches"]
+        if not args.no_decayed:
+            # the same layer with the decayed-memory SMA (two decay-prefix kernels + SMA)
+            dec_f = forward_region(args, dist, dart, FWD, decayed=True)
+            dms = dist.max(dec_f["ms_total"])
+            line["decayed_memories"] = {
+                "value": dist.world * FWD.batch * FWD.seqlen * args.steps / (dms / 1e3), "unit": "tokens/s",
+                "ms_per_step": dms / args.steps, "scan_ms": dec_f["scan_ms"], "sma_ms": dec_f["sma_ms"],
+                "sma_tflops": f_sma / (dec_f["sma_ms"] / 1e3) / 1e12,
+                "sma_ms_raw_memories": fwd["sma_ms"],
+                "config": {"workload": "dart_layer_fwd_L8k_decayed_memories", "batch": FWD.batch,
+                           "seqlen": FWD.seqlen, "nheads": FWD.nheads, "chunk": FWD.chunk}}
+            line["gpu_launches"] += dec_f["launches"]
         if not args.no_e2e:
             line["e2e"] = e2e_region(args, dist, dart, fwd["inputs"])
         if not args.no_decode:
             dec = decode_region(args, dist, dart, peaks)
             line["decode"] = dec
             line["gpu_launches"] += dec["launches"]
+            if not args.no_decayed:
+                dd = decode_region(args, dist, dart, peaks, decayed=True)
+                line["decode"]["decayed_memories"] = {
+                    "value": dd["value"], "unit": "tokens/s", "ms_per_step": dd["ms_per_step"],
+                    "roofline_frac": dd["roofline"]["frac"], "bytes_per_step": dd["roofline"]["bytes_per_step"],
+                    "kernel": "dart_decode_step_decayed"}
+                line["gpu_launches"] += dd["launches"]
         if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(fwd["inputs"])
         if dist.rank == 0:

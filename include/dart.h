@@ -195,6 +195,38 @@ dart_status dart_decode_step(const dart_dims* dims, dart_dtype dtype,
                              void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * dart_decode_step with decayed memories (referee major comment 3 on SMA
+ * Eq. (8), Pith review of DART; the decode form of dart_sma_forward_decayed).
+ * mem_logdecay: float [B,H,cmax], in/out.  Slot c < n_chunks[b] holds the
+ * log-decay memory c has accumulated since its chunk closed,
+ *   lw_c = sum_{r=e(c)+1}^{t-1} dt_r A_h   (t the incoming token).
+ * The step sets lw_c += dt_t A_h, scales the memory's score and value by
+ * exp(lw_c) exactly as dart_sma_forward_decayed does, and when the token
+ * closes its chunk sets the appended memory's slot to 0.  Slots >= n_chunks
+ * are not read.  Everything else -- arguments, layouts, counters, errors --
+ * as dart_decode_step.
+ */
+dart_status dart_decode_step_decayed(const dart_dims* dims, dart_dtype dtype,
+                                     const void* x_t, const float* dt_t, const float* A,
+                                     const void* B_t, const void* C_t, const void* Q_t,
+                                     const void* E_t, float g, float* state, float* dH_cur,
+                                     void* dH_cache, int cmax, int* n_chunks, int* pos,
+                                     float* mem_logdecay, float* y,
+                                     void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * mem_logdecay for decode after a prefill of dims->seqlen = L tokens (the
+ * handoff of dart_ssd_chunk_scan: L / S completed memories are cached):
+ *   mem_logdecay[b,h,c] = sum_{r=(c+1)S}^{L-1} dt[b,r,h] A[h]   for c < L / S,
+ * summed with an fp64 carry; other slots are left as they are.
+ *   dt: float [B,L,H] (the prefill's), A: float [H], mem_logdecay: float
+ *   [B,H,cmax] with L / S <= cmax.  Uses batch, seqlen, nheads and chunk of
+ *   dims.  One kernel on `stream`.
+ */
+dart_status dart_decode_memlog_init(const dart_dims* dims, const float* dt, const float* A,
+                                    float* mem_logdecay, int cmax, void* stream);
+
+/*
  * dart_decode_step for callers that cannot allocate device memory.  The
  * paper has no counterpart: this is an interface for embedding the decode
  * step where cudaMalloc is not available to the caller -- for example a host

@@ -249,6 +249,51 @@ dart_status dart_decode_step(const dart_dims* d, dart_dtype dtype, const void* x
     return DART_OK;
 }
 
+dart_status dart_decode_step_decayed(const dart_dims* d, dart_dtype dtype, const void* x_t, const float* dt_t,
+                                     const float* A, const void* B_t, const void* C_t, const void* Q_t,
+                                     const void* E_t, float g, float* state, float* dH_cur, void* dH_cache,
+                                     int cmax, int* n_chunks, int* pos, float* mem_logdecay, float* y,
+                                     void* workspace, size_t workspace_bytes, void* stream) {
+    t_err[0] = 0;
+    dart_status st = check_common(d, dtype, false);
+    if (st != DART_OK) return st;
+    if (!dart::decode_supported(d->dstate, d->headdim, d->chunk, dtype))
+        return fail(DART_ERR_UNSUPPORTED, "dart_decode_step_decayed: (N=%d, P=%d) not compiled", d->dstate,
+                    d->headdim);
+    if (cmax < 1) return fail(DART_ERR_INVALID_ARG, "cmax must be >= 1");
+    DART_REQUIRE_PTR(x_t); DART_REQUIRE_PTR(dt_t); DART_REQUIRE_PTR(A); DART_REQUIRE_PTR(B_t);
+    DART_REQUIRE_PTR(C_t); DART_REQUIRE_PTR(Q_t); DART_REQUIRE_PTR(E_t); DART_REQUIRE_PTR(state);
+    DART_REQUIRE_PTR(dH_cur); DART_REQUIRE_PTR(dH_cache); DART_REQUIRE_PTR(n_chunks);
+    DART_REQUIRE_PTR(pos); DART_REQUIRE_PTR(mem_logdecay); DART_REQUIRE_PTR(y); DART_REQUIRE_PTR(workspace);
+    if (workspace_bytes < dart_decode_step_workspace_bytes(d, dtype, cmax))
+        return fail(DART_ERR_INVALID_ARG, "workspace: %zu bytes, need %zu", workspace_bytes,
+                    dart_decode_step_workspace_bytes(d, dtype, cmax));
+    dart::DecodeArgs a{d->batch, d->nheads, d->headdim, d->dstate, d->chunk, cmax,
+                       dart::decode_num_splits(d->batch, d->nheads, cmax),
+                       x_t, dt_t, A, B_t, C_t, Q_t, E_t, g, state, dH_cur, dH_cache,
+                       n_chunks, pos, y, static_cast<float*>(workspace), status_word(), mem_logdecay};
+    if (!a.status) return fail(DART_ERR_CUDA, "dart_decode_step_decayed: no device status word");
+    cudaError_t e = dart::launch_decode(a, dtype, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "dart_decode_step_decayed launch");
+    return DART_OK;
+}
+
+dart_status dart_decode_memlog_init(const dart_dims* d, const float* dt, const float* A, float* mem_logdecay,
+                                    int cmax, void* stream) {
+    t_err[0] = 0;
+    if (!d) return fail(DART_ERR_INVALID_ARG, "dims is NULL");
+    if (d->batch < 1 || d->seqlen < 1 || d->nheads < 1 || d->chunk < 1)
+        return fail(DART_ERR_INVALID_ARG, "dart_decode_memlog_init: batch, seqlen, nheads and chunk must be >= 1");
+    if (cmax < 1 || d->seqlen / d->chunk > cmax)
+        return fail(DART_ERR_INVALID_ARG, "dart_decode_memlog_init: %d completed chunks do not fit cmax = %d",
+                    d->seqlen / d->chunk, cmax);
+    DART_REQUIRE_PTR(dt); DART_REQUIRE_PTR(A); DART_REQUIRE_PTR(mem_logdecay);
+    cudaError_t e = dart::launch_decode_memlog_init(d->batch, d->seqlen, d->nheads, d->chunk, cmax, dt, A,
+                                                    mem_logdecay, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "dart_decode_memlog_init launch");
+    return DART_OK;
+}
+
 // The decode step for callers that cannot allocate device memory: the split
 // partials go to the library's fixed static scratch (decode.cu) instead of a
 // caller workspace.  Validation matches dart_decode_step, plus the scratch

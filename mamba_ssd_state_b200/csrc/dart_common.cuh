@@ -126,6 +126,9 @@ struct DecodeArgs {
     float* state; float* dHcur; void* cache; int* nchunks; int* pos; float* y;
     float* part;  // [B,H,nsplit,2+2P] workspace
     int* status;  // device status word
+    // Decayed-memory variant (null: raw memories): [B,H,cmax] fp32, the
+    // log-decay sum_{r=e(c)+1}^{t-1} dt_r A_h each cached memory carries.
+    float* memlog;
 };
 
 // Counts one kernel launch (see dart_launch_count).
@@ -148,6 +151,9 @@ size_t sma_decay_workspace_bytes(int B, int L, int H, int S);
 const char* sma_impl_name(int N, int P, int S, dart_dtype dt);
 bool decode_supported(int N, int P, int S, dart_dtype dt);
 int decode_num_splits(int B, int H, int cmax);
+// memlog[b,h,c] = sum_{r=(c+1)S}^{L-1} dt[b,r,h] A[h] for c < L / S (one launch).
+cudaError_t launch_decode_memlog_init(int B, int L, int H, int S, int cmax, const float* dt, const float* A,
+                                      float* memlog, cudaStream_t st);
 
 // dart_decode_step_noalloc: size of the library-owned static scratch, and its
 // device address on the current device (set up on the first call per device).

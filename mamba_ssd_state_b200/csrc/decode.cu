@@ -19,6 +19,12 @@
 // decode_combine  grid (h, b): merges the splits, y = y_ssd + g * o.
 // decode_advance  one thread per sequence: advances (n_chunks, pos) after
 //   every block of the step has read them.
+//
+// Decayed memories (memlog set; referee comment 3 on SMA Eq. (8)): memory c
+// carries lw = sum_{r=e(c)+1}^{t-1} dt_r A_h.  The warp that reads memory c
+// adds this token's dt_t A_h, scales the score by w = exp(lw) and the value
+// weight by w, and stores the new lw; a memory appended by this token starts
+// at 0 (written by split 0).
 #include "dart_common.cuh"
 
 namespace dart {
@@ -43,7 +49,7 @@ __device__ __forceinline__ SeqCounters read_counters(const DecodeArgs& a, int b)
     return s;
 }
 
-template <typename T, int N, int P>
+template <typename T, int N, int P, bool kDecay>
 __global__ void __launch_bounds__(kThreads) decode_partial_kernel(DecodeArgs a) {
     constexpr int VEC = Vec16<T>::kN;        // elements per 16-byte load
     constexpr int LPR = P / VEC;             // lanes per memory row
@@ -118,10 +124,23 @@ __global__ void __launch_bounds__(kThreads) decode_partial_kernel(DecodeArgs a) 
     float m = -INFINITY, l = 0.f, o[VEC];
 #pragma unroll
     for (int j = 0; j < VEC; ++j) o[j] = 0.f;
+    float* memlog = kDecay ? a.memlog + bh * a.cmax : nullptr;
+    const float a_t = kDecay ? a.dt[bh] * a.A[h] : 0.f;   // this token's log-decay
+    if (kDecay && sc.append && split == 0 && tid == 0) memlog[sc.n] = 0.f;   // closes at this token
     const int c_begin = split * kChunksPerSplit;
     const int c_end = min(sc.n, c_begin + kChunksPerSplit);
     const T* cache = static_cast<const T*>(a.cache) + bh * a.cmax * (size_t)N * P;
-    for (int c = c_begin + warp; c < c_end; c += kWarps) {
+    // decayed memories: lane i holds the log-decay of this warp's i-th memory
+    // (memory c_begin + warp + i kWarps), read before and written after the
+    // streaming loop so that the loop itself touches only the cache
+    static_assert(kChunksPerSplit / kWarps <= 32, "one lane per memory of a warp");
+    float lw_mine = 0.f;
+    if (kDecay && lane < kChunksPerSplit / kWarps) {
+        const int c = c_begin + warp + kWarps * lane;
+        if (c < c_end) lw_mine = memlog[c] + a_t;   // now sum_{r=e(c)+1}^{t} dt_r A_h
+    }
+    int it = 0;   // this warp's memory counter
+    for (int c = c_begin + warp; c < c_end; c += kWarps, ++it) {
         const T* mem = cache + (size_t)c * N * P + (size_t)lrow * P + pcol;
         float v[VEC], s = 0.f;
 #pragma unroll
@@ -158,13 +177,23 @@ __global__ void __launch_bounds__(kThreads) decode_partial_kernel(DecodeArgs a) 
 #pragma unroll
             for (int j = 0; j < VEC; ++j) v[j] += __shfl_xor_sync(0xffffffffu, v[j], off);
         s = warp_sum(s);
+        float wd = 1.f;   // decay of memory c at this token (1 for raw memories)
+        if (kDecay) {
+            wd = exp2f(kLog2e * __shfl_sync(0xffffffffu, lw_mine, it));
+            s *= wd;
+        }
         const float mnew = fmaxf(m, s);
         const float alpha = exp2f(m - mnew);
         const float w = exp2f(s - mnew);
         l = l * alpha + w;
+        const float wv = kDecay ? w * wd : w;
 #pragma unroll
-        for (int j = 0; j < VEC; ++j) o[j] = fmaf(o[j], alpha, w * v[j]);
+        for (int j = 0; j < VEC; ++j) o[j] = fmaf(o[j], alpha, wv * v[j]);
         m = mnew;
+    }
+    if (kDecay && lane < kChunksPerSplit / kWarps) {
+        const int c = c_begin + warp + kWarps * lane;
+        if (c < c_end) memlog[c] = lw_mine;
     }
     if (lane == 0) { red_m[warp] = m; red_l[warp] = l; }
     if (lrow == 0) {
@@ -229,9 +258,40 @@ __global__ void decode_advance_kernel(DecodeArgs a) {
     }
 }
 
+// One warp per (b, h): suffix sums of dt A over the prefill, walked from the
+// last token down 32 tokens at a time with an fp64 carry; the suffix that
+// starts at a chunk boundary (c+1) S is memory c's log-decay.
+__global__ void __launch_bounds__(256) memlog_init_kernel(int BH, int L, int H, int S, int cmax,
+                                                           const float* __restrict__ dt,
+                                                           const float* __restrict__ A, float* __restrict__ memlog) {
+    const int bh = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (bh >= BH) return;
+    const int b = bh / H, h = bh % H;
+    const int ncached = L / S;            // complete chunks of the prefill
+    float* out = memlog + (size_t)bh * cmax;
+    if (lane == 0 && ncached > 0 && ncached * S == L) out[ncached - 1] = 0.f;   // closed at the last token
+    const float Ah = A[h];
+    double carry = 0.0;
+    for (int base = L - 1; base >= S; base -= 32) {
+        const int t = base - lane;
+        float v = t >= 0 ? dt[((size_t)b * L + t) * H + h] * Ah : 0.f;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float u = __shfl_up_sync(0xffffffffu, v, o);
+            if (lane >= o) v += u;
+        }
+        if (t >= S && t % S == 0) out[t / S - 1] = (float)(carry + (double)v);
+        carry += (double)__shfl_sync(0xffffffffu, v, 31);
+    }
+}
+
 template <typename T, int N, int P>
 cudaError_t run(const DecodeArgs& a, cudaStream_t st) {
-    decode_partial_kernel<T, N, P><<<dim3(a.nsplit, a.H, a.B), kThreads, 0, st>>>(a);
+    if (a.memlog)
+        decode_partial_kernel<T, N, P, true><<<dim3(a.nsplit, a.H, a.B), kThreads, 0, st>>>(a);
+    else
+        decode_partial_kernel<T, N, P, false><<<dim3(a.nsplit, a.H, a.B), kThreads, 0, st>>>(a);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     decode_combine_kernel<P><<<dim3(a.H, a.B), P, 0, st>>>(a);
@@ -243,6 +303,16 @@ cudaError_t run(const DecodeArgs& a, cudaStream_t st) {
 }
 
 }  // namespace
+
+cudaError_t launch_decode_memlog_init(int B, int L, int H, int S, int cmax, const float* dt, const float* A,
+                                      float* memlog, cudaStream_t st) {
+    const int BH = B * H;
+    memlog_init_kernel<<<(BH + 7) / 8, 256, 0, st>>>(BH, L, H, S, cmax, dt, A, memlog);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    count_launches(1);
+    return cudaSuccess;
+}
 
 int decode_num_splits(int, int, int cmax) {
     const int ns = (cmax + kChunksPerSplit - 1) / kChunksPerSplit;

@@ -32,7 +32,7 @@ EXPORTS = ("dart_ssd_chunk_scan_workspace_bytes", "dart_ssd_chunk_scan", "dart_s
            "dart_decode_step_workspace_bytes", "dart_decode_step", "dart_supported",
            "dart_sync_status", "dart_last_error", "dart_abi_version", "dart_launch_count",
            "dart_sma_impl", "dart_decode_step_noalloc", "dart_sma_decayed_workspace_bytes",
-           "dart_sma_forward_decayed")
+           "dart_sma_forward_decayed", "dart_decode_step_decayed", "dart_decode_memlog_init")
 
 
 class DartError(RuntimeError):
@@ -65,6 +65,11 @@ def load(path: str = LIBRARY) -> ctypes.CDLL:
     lib.dart_ssd_chunk_scan.argtypes = [D, ctypes.c_int] + [_P] * 10 + [ctypes.c_size_t, _P]
     lib.dart_sma_forward.restype = ctypes.c_int
     lib.dart_sma_forward.argtypes = [D, ctypes.c_int] + [_P] * 4 + [ctypes.c_float, _P, _P, _P]
+    lib.dart_decode_step_decayed.restype = ctypes.c_int
+    lib.dart_decode_step_decayed.argtypes = ([D, ctypes.c_int] + [_P] * 7 + [ctypes.c_float] + [_P] * 3
+                                             + [ctypes.c_int] + [_P] * 5 + [ctypes.c_size_t, _P])
+    lib.dart_decode_memlog_init.restype = ctypes.c_int
+    lib.dart_decode_memlog_init.argtypes = [D, _P, _P, _P, ctypes.c_int, _P]
     lib.dart_sma_decayed_workspace_bytes.restype = ctypes.c_size_t
     lib.dart_sma_decayed_workspace_bytes.argtypes = [D]
     lib.dart_sma_forward_decayed.restype = ctypes.c_int
@@ -301,14 +306,18 @@ def layer_forward(x, dt, A, Bm, Cm, Q, E, chunk: int, g: float, init_state=None,
 
 
 def dart_decode_step(x, dt, A, Bm, Cm, Q, E, g: float, state, dH_cur, cache, nchunks, pos,
-                     chunk: int, *, y=None, workspace=None):
+                     chunk: int, *, y=None, workspace=None, memlog=None):
     """One decode step for every sequence.  x[Bs,H,P], Bm/Cm[Bs,N],
     Q[Bs,H,N], E[Bs,H,P] (cache dtype), dt[Bs,H], A[H] float32; state and
     dH_cur float32 [Bs,H,N,P], cache [Bs,H,cmax,N,P], nchunks/pos int32 [Bs]
-    are device tensors updated in place.  Returns y float32 [Bs,H,P]."""
+    are device tensors updated in place.  With ``memlog`` (float32
+    [Bs,H,cmax] device tensor, updated in place) the memories are decayed to
+    the new token (dart_decode_step_decayed).  Returns y float32 [Bs,H,P]."""
     lib = load()
-    for name, t in (("state", state), ("dH_cur", dH_cur), ("cache", cache), ("nchunks", nchunks),
-                    ("pos", pos)):
+    bufs = [("state", state), ("dH_cur", dH_cur), ("cache", cache), ("nchunks", nchunks), ("pos", pos)]
+    if memlog is not None:
+        bufs.append(("memlog", memlog))
+    for name, t in bufs:
         if not t.is_cuda or not t.is_contiguous():
             raise ValueError(f"{name} must be a contiguous CUDA tensor (updated in place)")
     dev = cache.device
@@ -325,6 +334,10 @@ def dart_decode_step(x, dt, A, Bm, Cm, Q, E, g: float, state, dH_cur, cache, nch
         raise TypeError("state and dH_cur must be float32")
     if nchunks.dtype != torch.int32 or pos.dtype != torch.int32:
         raise TypeError("nchunks and pos must be int32")
+    if memlog is not None:
+        _shape("memlog", memlog, (Bs, H, cmax))
+        if memlog.dtype != torch.float32:
+            raise TypeError("memlog must be float32")
     dims = Dims(Bs, 0, H, P, N, chunk, 1)
     code = _dtype_code(cache.dtype)
     if y is None:
@@ -333,11 +346,36 @@ def dart_decode_step(x, dt, A, Bm, Cm, Q, E, g: float, state, dH_cur, cache, nch
     if workspace is None:
         workspace = torch.empty(max(16, wsb), device=dev, dtype=torch.uint8)
     with torch.cuda.device(dev):
-        _check(lib.dart_decode_step(ctypes.byref(dims), code, _ptr(x), _ptr(dt), _ptr(A), _ptr(Bm), _ptr(Cm),
-                                    _ptr(Q), _ptr(E), float(g), _ptr(state), _ptr(dH_cur), _ptr(cache),
-                                    cmax, _ptr(nchunks), _ptr(pos), _ptr(y), _ptr(workspace),
-                                    workspace.numel(), _stream()))
+        if memlog is None:
+            _check(lib.dart_decode_step(ctypes.byref(dims), code, _ptr(x), _ptr(dt), _ptr(A), _ptr(Bm),
+                                        _ptr(Cm), _ptr(Q), _ptr(E), float(g), _ptr(state), _ptr(dH_cur),
+                                        _ptr(cache), cmax, _ptr(nchunks), _ptr(pos), _ptr(y), _ptr(workspace),
+                                        workspace.numel(), _stream()))
+        else:
+            _check(lib.dart_decode_step_decayed(ctypes.byref(dims), code, _ptr(x), _ptr(dt), _ptr(A), _ptr(Bm),
+                                                _ptr(Cm), _ptr(Q), _ptr(E), float(g), _ptr(state),
+                                                _ptr(dH_cur), _ptr(cache), cmax, _ptr(nchunks), _ptr(pos),
+                                                _ptr(memlog), _ptr(y), _ptr(workspace), workspace.numel(),
+                                                _stream()))
     return _to_host(y)[0] if host else y
+
+
+def decode_memlog_init(dt, A, chunk: int, memlog):
+    """Fill memlog[b,h,c] (float32 [B,H,cmax] device tensor) for decode after
+    a prefill whose dt [B,L,H] is given: the log-decay of each of the L //
+    chunk completed memories, sum_{r=(c+1)S..L-1} dt A_h."""
+    lib = load()
+    if not memlog.is_cuda or not memlog.is_contiguous() or memlog.dtype != torch.float32:
+        raise ValueError("memlog must be a contiguous float32 CUDA tensor")
+    dev = memlog.device
+    dt, A = _dev(dt, dev, torch.float32), _dev(A, dev, torch.float32)
+    Bsz, L, H = dt.shape
+    _shape("A", A, (H,)); _shape("memlog", memlog, (Bsz, H, memlog.shape[2]))
+    dims = Dims(Bsz, L, H, 0, 0, chunk, 1)
+    with torch.cuda.device(dev):
+        _check(lib.dart_decode_memlog_init(ctypes.byref(dims), _ptr(dt), _ptr(A), _ptr(memlog),
+                                           memlog.shape[2], _stream()))
+    return memlog
 
 
 def dart_decode_step_noalloc(x, dt, A, Bm, Cm, Q, E, g: float, state, dH_cur, cache, nchunks, pos,

@@ -151,6 +151,20 @@ def test_sma_decayed_workspace_and_validation(lib):
              FAKE, 1 << 30, None) == dart.DART_ERR_UNSUPPORTED
 
 
+def test_decayed_decode_validation(lib):
+    """The decayed decode step needs mem_logdecay on top of dart_decode_step's
+    arguments; the memlog initialiser rejects prefills that overflow cmax."""
+    d = dart.Dims(4, 0, 2, 64, 128, 256, 1)
+    ws = lib.dart_decode_step_workspace_bytes(ctypes.byref(d), dart.DART_BF16, 9)
+    args = [FAKE] * 7 + [0.5] + [FAKE] * 3 + [9] + [FAKE, FAKE, None, FAKE, FAKE, ws, None]
+    assert lib.dart_decode_step_decayed(ctypes.byref(d), dart.DART_BF16, *args) == dart.DART_ERR_INVALID_ARG
+    assert b"mem_logdecay" in lib.dart_last_error()
+    p = dart.Dims(2, 10 * 256 + 7, 2, 64, 128, 256, 1)
+    assert lib.dart_decode_memlog_init(ctypes.byref(p), FAKE, FAKE, FAKE, 9, None) == dart.DART_ERR_INVALID_ARG
+    assert lib.dart_decode_memlog_init(ctypes.byref(p), FAKE, None, FAKE, 16, None) == dart.DART_ERR_INVALID_ARG
+    assert lib.dart_decode_memlog_init(None, FAKE, FAKE, FAKE, 16, None) == dart.DART_ERR_INVALID_ARG
+
+
 def test_decode_rejects_bad_args(lib):
     d = dart.Dims(4, 0, 2, 64, 128, 256, 1)
     ws = lib.dart_decode_step_workspace_bytes(ctypes.byref(d), dart.DART_BF16, 9)
