@@ -64,6 +64,16 @@
  * one closing at token L-1 (its dH and state are what a decode would carry
  * on from); no token attends to it, since its own tokens have k(t) = C-1.
  *
+ *  - An fp8 decode cache (the cache quantization the pages list as an
+ *    extension; DART abstract and Pith review "If this is right" for the cache
+ *    itself).  Each row of P values of a memory is stored as OCP FP8 E4M3
+ *    codes (1 sign, 4 exponent bits with bias 7, 3 mantissa bits; largest
+ *    finite 448, subnormals down to 2^-9) times a power of two 2^k, k the
+ *    smallest integer with max|row| * 2^-k <= 448, clamped to [-126, 60].
+ *    Codes round to nearest, ties to even, and saturate at 448.  The decode
+ *    step then reads the dequantized memories and quantizes the memory it
+ *    appends.  Written from the format's definition, not from any library.
+ *
  * Layouts (row-major, last index fastest):
  *   x[B,L,H,P] dt[B,L,H] A[H] Bm[B,L,N] Cm[B,L,N] Q[B,L,H,N] E[B,L,H,P]
  *   y[B,L,H,P] dH[B,H,C,N,P] states[B,H,C,N,P] init_state[B,H,N,P]
@@ -301,6 +311,71 @@ int oracle_sma(const oracle_dims* d, const float* Q, const float* E, const float
 }
 
 /* ------------------------------------------------------------------ */
+/* fp8 (E4M3) cache rows                                                */
+/* ------------------------------------------------------------------ */
+/* The row exponent: smallest k with amax * 2^-k <= 448 = 0.875 * 2^9.  With
+ * amax = f 2^e, f in [0.5, 1): f 2^(e-k) <= 0.875 2^9 holds for k = e - 9
+ * when f <= 0.875, else first for k = e - 8. */
+static int e4m3_row_exponent(double amax) {
+    int e = 0;
+    const double f = frexp(amax, &e); /* amax = 0 gives f = 0, e = 0 */
+    int k = f <= 0.875 ? e - 9 : e - 8;
+    if (k < -126) k = -126;
+    if (k > 60) k = 60;
+    return k;
+}
+
+/* Nearest E4M3 code of v (already scaled), ties to even, saturating. */
+static uint8_t e4m3_encode(double v) {
+    const uint8_t sign = signbit(v) ? 0x80 : 0x00;
+    double a = fabs(v);
+    if (a >= 448.0) return sign | 0x7E;
+    if (a < 0.015625) { /* below 2^-6: subnormal grid, step 2^-9 */
+        const double q = nearbyint(a * 512.0); /* 0..8; 8 is the code of 2^-6 */
+        return sign | (uint8_t)q;
+    }
+    int e = 0;
+    frexp(a, &e);              /* a = f 2^e, f in [0.5, 1): a in [2^(e-1), 2^e) */
+    int E = e - 1;             /* unbiased exponent, -6 .. 8 */
+    double q = nearbyint(ldexp(a, 3 - E)); /* 8 .. 16 mantissa steps of 2^(E-3) */
+    if (q >= 16.0) {
+        q = 8.0;
+        E += 1;
+    }
+    const int code = ((E + 7) << 3) | ((int)q - 8);
+    return sign | (uint8_t)(code > 0x7E ? 0x7E : code);
+}
+
+static double e4m3_decode(uint8_t c) {
+    const int e = (c >> 3) & 0xF, m = c & 0x7;
+    const double mag = e == 0 ? ldexp((double)m, -9) : ldexp(8.0 + m, e - 10);
+    return (c & 0x80) ? -mag : mag;
+}
+
+/* Quantize one row of P values: codes[P], its exponent, and (nullable) the
+ * dequantized values codes * 2^k. */
+static void e4m3_quantize_row(const double* x, int P, uint8_t* codes, int8_t* kout, double* deq) {
+    double amax = 0.0;
+    for (int p = 0; p < P; ++p) if (fabs(x[p]) > amax) amax = fabs(x[p]);
+    const int k = e4m3_row_exponent(amax);
+    for (int p = 0; p < P; ++p) {
+        codes[p] = e4m3_encode(ldexp(x[p], -k));
+        if (deq) deq[p] = ldexp(e4m3_decode(codes[p]), k);
+    }
+    *kout = (int8_t)k;
+}
+
+/*
+ * x[rows,P] double -> codes[rows,P], exps[rows], deq[rows,P] (nullable).
+ */
+int oracle_quantize_e4m3(const double* x, long rows, int P, uint8_t* codes, int8_t* exps, double* deq) {
+    if (!x || !codes || !exps || rows < 0 || P <= 0) return -1;
+    for (long r = 0; r < rows; ++r)
+        e4m3_quantize_row(x + r * P, P, codes + r * P, exps + r, deq ? deq + r * P : NULL);
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
 /* 5: one decode step against the cache of completed chunk memories     */
 /* ------------------------------------------------------------------ */
 typedef struct {
@@ -310,6 +385,7 @@ typedef struct {
     double g;
     double *state, *dHcur, *cache;
     double* memlog; /* nullable: [Bs,H,cmax] log-decay of each cached memory */
+    int cache_e4m3; /* the cache holds dequantized E4M3 rows; appends quantize */
     const int *nchunks, *pos;
     double* y;
 } dec_ctx;
@@ -387,7 +463,16 @@ static void decode_unit(void* vctx, int unit) {
     /* the token that closes its chunk appends the finished contribution */
     if (c->pos[b] == S - 1) {
         double* slot = c->cache + (bh * (size_t)c->cmax + nmem) * (size_t)N * P;
-        memcpy(slot, D, sizeof(double) * (size_t)N * P);
+        if (c->cache_e4m3) {
+            uint8_t* codes = (uint8_t*)malloc((size_t)P);
+            for (int n = 0; n < N; ++n) {
+                int8_t k;
+                e4m3_quantize_row(D + (size_t)n * P, P, codes, &k, slot + (size_t)n * P);
+            }
+            free(codes);
+        } else {
+            memcpy(slot, D, sizeof(double) * (size_t)N * P);
+        }
         memset(D, 0, sizeof(double) * (size_t)N * P);
         if (c->memlog) c->memlog[bh * (size_t)c->cmax + nmem] = 0.0; /* closes at this token */
     }
@@ -397,21 +482,24 @@ static void decode_unit(void* vctx, int unit) {
  * x[Bs,H,P] dt[Bs,H] A[H] Bm[Bs,N] Cm[Bs,N] Q[Bs,H,N] E[Bs,H,P] (float);
  * state, dH_cur [Bs,H,N,P], cache [Bs,H,cmax,N,P], y [Bs,H,P] (double);
  * nchunks[Bs], pos[Bs] in/out; memlog [Bs,H,cmax] (double, in/out) selects
- * the decayed-memory variant when not NULL.  Returns -1 (and changes
- * nothing) when an append would overflow the cache or a counter is out of
- * range.
+ * the decayed-memory variant when not NULL; cache_e4m3 != 0 makes an append
+ * store the E4M3-quantized (then dequantized) memory, for a cache that holds
+ * dequantized E4M3 rows.  Returns -1 (and changes nothing) when an append
+ * would overflow the cache or a counter is out of range.
  */
 int oracle_decode_step(const oracle_dims* d, int cmax, const float* x, const float* dt,
                        const float* A, const float* Bm, const float* Cm, const float* Q,
                        const float* E, double g, double* state, double* dH_cur, double* cache,
-                       int* nchunks, int* pos, double* memlog, double* y, int nthreads) {
+                       int* nchunks, int* pos, double* memlog, int cache_e4m3, double* y,
+                       int nthreads) {
     if (!d || d->chunk <= 0) return -1;
     for (int b = 0; b < d->batch; ++b) {
         if (nchunks[b] < 0 || nchunks[b] > cmax) return -1;
         if (pos[b] < 0 || pos[b] >= d->chunk) return -1;
         if (pos[b] == d->chunk - 1 && nchunks[b] >= cmax) return -1;
     }
-    dec_ctx c = {d, cmax, x, dt, A, Bm, Cm, Q, E, g, state, dH_cur, cache, memlog, nchunks, pos, y};
+    dec_ctx c = {d, cmax, x, dt, A, Bm, Cm, Q, E, g, state, dH_cur, cache, memlog, cache_e4m3,
+                 nchunks, pos, y};
     run_units(decode_unit, &c, d->batch * d->nheads, nthreads);
     for (int b = 0; b < d->batch; ++b) {
         if (pos[b] == d->chunk - 1) {

@@ -61,7 +61,9 @@ class Oracle:
         self.lib.oracle_decode_step.restype = ctypes.c_int
         self.lib.oracle_decode_step.argtypes = (
             [ctypes.POINTER(_Dims), ctypes.c_int] + [_P] * 7 + [ctypes.c_double]
-            + [_P] * 7 + [ctypes.c_int])
+            + [_P] * 6 + [ctypes.c_int, _P, ctypes.c_int])
+        self.lib.oracle_quantize_e4m3.restype = ctypes.c_int
+        self.lib.oracle_quantize_e4m3.argtypes = [_P, ctypes.c_long, ctypes.c_int, _P, _P, _P]
 
     # ------------------------------------------------------------------
     @staticmethod
@@ -146,13 +148,29 @@ class Oracle:
                      dt=dt if decayed else None, A=A if decayed else None)
         return {"y": r["y"], "o": r["o"], "y_ssd": y_ssd, "dH": dH, "states": st}
 
+    def quantize_e4m3(self, x):
+        """E4M3 cache rows: x[..., P] (float64) -> (codes uint8 [..., P],
+        exponents int8 [...], dequantized float64 [..., P])."""
+        x = self._f64(x)
+        P = x.shape[-1]
+        rows = x.size // P
+        codes = np.empty(x.shape, np.uint8)
+        exps = np.empty(x.shape[:-1], np.int8)
+        deq = np.empty(x.shape, np.float64)
+        if self.lib.oracle_quantize_e4m3(self._ptr(x), rows, P, self._ptr(codes), self._ptr(exps),
+                                         self._ptr(deq)):
+            raise ValueError("oracle_quantize_e4m3 rejected its arguments")
+        return codes, exps, deq
+
     def decode_step(self, x, dt, A, Bm, Cm, Q, E, g, state, dH_cur, cache, nchunks, pos,
-                    chunk: int, memlog=None):
+                    chunk: int, memlog=None, cache_e4m3: bool = False):
         """One decode step.  state, dH_cur, cache (float64, C-contiguous) and
         nchunks, pos (int32) are updated in place.  With ``memlog`` (float64
         [Bs,H,cmax], updated in place: the log-decay each cached memory has
         accumulated since its chunk closed) the memories are decayed to the
-        new token before use.  Returns y[Bs,H,P]."""
+        new token before use.  With ``cache_e4m3`` the cache holds dequantized
+        E4M3 rows and an append stores the quantized memory.  Returns
+        y[Bs,H,P]."""
         x, dt, A, Bm, Cm, Q, E = (self._f32(v) for v in (x, dt, A, Bm, Cm, Q, E))
         bufs = [(state, np.float64), (dH_cur, np.float64), (cache, np.float64),
                 (nchunks, np.int32), (pos, np.int32)]
@@ -170,7 +188,8 @@ class Oracle:
                                          self._ptr(A), self._ptr(Bm), self._ptr(Cm),
                                          self._ptr(Q), self._ptr(E), float(g), self._ptr(state),
                                          self._ptr(dH_cur), self._ptr(cache), self._ptr(nchunks),
-                                         self._ptr(pos), self._ptr(memlog), self._ptr(y), self.nthreads)
+                                         self._ptr(pos), self._ptr(memlog), int(bool(cache_e4m3)),
+                                         self._ptr(y), self.nthreads)
         if rc:
             raise ValueError("oracle_decode_step rejected its arguments")
         return y

@@ -524,6 +524,100 @@ def pin_decayed_decode_matches_prefill(orc):
         _close(y, full["y"][:, t], 1e-12, f"decayed decode after prefill, y at t={t}")
 
 
+# ----------------------------------------------------------------------------
+# fp8 (OCP E4M3) decode cache: rows of P values as codes times 2^k
+# ----------------------------------------------------------------------------
+def _torch_e4m3_codes(v):
+    """Library rounding of float32-exact values to float8_e4m3fn codes."""
+    t = torch.from_numpy(np.ascontiguousarray(v, np.float32))
+    return t.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def _torch_e4m3_values(codes):
+    return torch.from_numpy(np.ascontiguousarray(codes, np.uint8)).view(torch.float8_e4m3fn).to(
+        torch.float64).numpy()
+
+
+def pin_e4m3_rows_match_library(orc):
+    """Codes equal torch's float8_e4m3fn cast of x 2^-k (round to nearest even)
+    for rows of every magnitude, exact ties and subnormals included; the row
+    exponent is the smallest k with max|row| 2^-k <= 448 (so the scaled max
+    lies in (224, 448]); dequantized values are the library's code values
+    times 2^k exactly; every finite code survives a round trip."""
+    r = np.random.default_rng(31)
+    P = 64
+    rows = []
+    for amax in np.exp(r.uniform(np.log(1e-7), np.log(1e3), 200)):
+        row = (r.standard_normal(P) * amax / 3).astype(np.float32)
+        row[r.integers(0, P)] = np.float32(amax) * (1 if r.random() < 0.5 else -1)
+        rows.append(row)
+    rows.append(np.zeros(P, np.float32))
+    one = np.zeros(P, np.float32)
+    one[5] = -3.0e-3
+    rows.append(one)
+    # exact midpoints between neighbouring codes (ties), in a row whose max is 448
+    vals = _torch_e4m3_values(np.arange(0, 0x7E, dtype=np.uint8))
+    mids = ((vals[:-1] + vals[1:]) / 2).astype(np.float32)
+    for i in range(0, len(mids), P - 1):
+        row = np.zeros(P, np.float32)
+        chunk = mids[i:i + P - 1]
+        row[:len(chunk)] = chunk
+        row[-1] = 448.0
+        rows.append(row)
+    X = np.stack(rows).astype(np.float64)
+    codes, exps, deq = orc.quantize_e4m3(X)
+    amax = np.abs(X).max(1)
+    nz = amax > 0
+    scaled_max = amax[nz] * np.exp2(-exps[nz].astype(np.float64))
+    assert np.all(scaled_max <= 448.0) and np.all(scaled_max > 224.0), "row exponent"
+    want = _torch_e4m3_codes(X * np.exp2(-exps.astype(np.float64))[:, None])
+    assert np.array_equal(codes, want), f"{np.count_nonzero(codes != want)} codes differ from the library"
+    assert np.array_equal(deq, _torch_e4m3_values(codes) * np.exp2(exps.astype(np.float64))[:, None])
+    # round trip of every finite code (0x7F / 0xFF are NaN in E4M3FN)
+    fin = np.array([c for c in range(256) if c & 0x7F != 0x7F], np.uint8)
+    v = _torch_e4m3_values(fin)
+    row = np.zeros((1, 4 * P))
+    row[0, :len(v)] = v
+    row[0, -1] = 448.0
+    c2, e2, _ = orc.quantize_e4m3(row)
+    assert e2[0] == 0 and np.array_equal(c2[0, :len(v)], fin)
+
+
+def pin_e4m3_decode_append(orc):
+    """With an E4M3 cache the decode step reads the dequantized memories and
+    quantizes the memory it appends: run side by side with the plain-cache
+    decode from the same cache, the outputs agree exactly until the append,
+    the appended slot is the quantizer's output for the plain slot, and the
+    next outputs equal the plain decode run with that slot quantized."""
+    Bz, H, P, N, S = 2, 2, 8, 4, 4
+    T = 6
+    inp = _rand_layer(32, Bz, T, H, P, N)
+    cmax = 3
+    r = np.random.default_rng(33)
+    _, _, cache0 = orc.quantize_e4m3(r.standard_normal((Bz, H, cmax, N, P)) * 0.3)
+    st = [dict(cache=cache0.copy(), state=r.standard_normal((Bz, H, N, P)) * 0.1,
+               dcur=r.standard_normal((Bz, H, N, P)) * 0.05, nch=np.full((Bz,), 1, np.int32),
+               pos=np.full((Bz,), 1, np.int32)) for _ in range(2)]
+    st[1] = {k: v.copy() for k, v in st[0].items()}
+    g = 0.9
+
+    def step(sd, t, e4m3):
+        return orc.decode_step(inp["x"][:, t], inp["dt"][:, t], inp["A"], inp["Bm"][:, t], inp["Cm"][:, t],
+                               inp["Q"][:, t], inp["E"][:, t], g, sd["state"], sd["dcur"], sd["cache"],
+                               sd["nch"], sd["pos"], S, cache_e4m3=e4m3)
+    for t in range(3):   # positions 1, 2, 3: the third step appends memory 1
+        ya, yb = step(st[0], t, True), step(st[1], t, False)
+        assert np.array_equal(ya, yb), f"step {t}"
+    assert np.all(st[0]["nch"] == 2)
+    _, _, q = orc.quantize_e4m3(st[1]["cache"][:, :, 1])
+    assert np.array_equal(st[0]["cache"][:, :, 1], q), "appended slot = quantized memory"
+    assert not np.array_equal(q, st[1]["cache"][:, :, 1])
+    st[1]["cache"][:, :, 1] = q
+    for t in range(3, T):
+        ya, yb = step(st[0], t, True), step(st[1], t, False)
+        assert np.array_equal(ya, yb), f"step {t}"
+
+
 ALL_PINS = [
     pin_closed_form_single_token,
     pin_quadratic_form,
@@ -542,4 +636,6 @@ ALL_PINS = [
     pin_decayed_memories_sum_to_state,
     pin_decayed_bruteforce_attention,
     pin_decayed_decode_matches_prefill,
+    pin_e4m3_rows_match_library,
+    pin_e4m3_decode_append,
 ]

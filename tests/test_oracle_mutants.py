@@ -58,6 +58,13 @@ MUTATIONS = [
      "wdec = exp(*lw);\n                *lw += dtt * (double)c->A[h];", 0),
     ("decode_memlog_not_reset", "if (c->memlog) c->memlog[bh * (size_t)c->cmax + nmem] = 0.0;", "", 0),
     ("decode_decay_value_only", "key[n] = wdec * acc;", "key[n] = acc;", 1),
+    ("e4m3_truncates", "double q = nearbyint(ldexp(a, 3 - E));", "double q = floor(ldexp(a, 3 - E));", 0),
+    ("e4m3_row_exponent_too_big", "int k = f <= 0.875 ? e - 9 : e - 8;", "int k = e - 8;", 0),
+    ("e4m3_sign_dropped", "return sign | (uint8_t)(code > 0x7E ? 0x7E : code);",
+     "return (uint8_t)(code > 0x7E ? 0x7E : code);", 0),
+    ("e4m3_subnormal_step", "const double q = nearbyint(a * 512.0);", "const double q = nearbyint(a * 256.0);", 0),
+    ("e4m3_decode_bias", "ldexp(8.0 + m, e - 10)", "ldexp(8.0 + m, e - 11)", 0),
+    ("decode_append_not_quantized", "if (c->cache_e4m3) {", "if (0) {", 0),
 ]
 
 
