@@ -62,6 +62,7 @@ def parse():
                    help="skip the forward with a partial last chunk (L = 8092)")
     p.add_argument("--no-decayed", action="store_true",
                    help="skip the forward with decayed memories (dart_sma_forward_decayed)")
+    p.add_argument("--no-e4m3", action="store_true", help="skip the decode with an E4M3 cache")
     p.add_argument("--decode-steps", type=int, default=DEC.nsteps)
     p.add_argument("--reference-heads", type=int, default=0,
                    help="heads per reference-arm step (default: one per host core, at most 32)")
@@ -121,17 +122,19 @@ def ssd_flops(s: synth.LayerShape) -> float:
     return float(B * per_b)
 
 
-def decode_bytes(d: synth.DecodeShape, n: int, append: bool) -> float:
+def decode_bytes(d: synth.DecodeShape, n: int, append: bool, e4m3: bool = False) -> float:
     """Bytes one decode step must move: every cached memory once, the float32
     state and running contribution read and written, the token inputs, the
-    output, and the appended memory when the step closes a chunk."""
+    output, and the appended memory when the step closes a chunk.  An E4M3
+    cache holds 1 byte per element plus 1 exponent byte per row."""
     esz = 2 if d.dtype == "bf16" else 4
-    per_sh = n * d.dstate * d.headdim * esz + 4 * d.dstate * d.headdim * 4
+    mem = d.dstate * d.headdim * esz if not e4m3 else d.dstate * (d.headdim + 1)
+    per_sh = n * mem + 4 * d.dstate * d.headdim * 4
     per_sh += (2 * d.headdim + d.dstate) * esz + 4 + d.headdim * 4
     per_seq = d.nheads * per_sh + 2 * d.dstate * esz
     total = d.nseq * per_seq
     if append:
-        total += d.nseq * d.nheads * d.dstate * d.headdim * esz
+        total += d.nseq * d.nheads * mem
     return float(total)
 
 
@@ -321,10 +324,17 @@ def e2e_region(args, dist, dart, inp):
             "path": "dart.layer_forward on pinned host inputs, y returned to host"}
 
 
-def decode_region(args, dist, dart, peaks, decayed=False):
+def decode_region(args, dist, dart, peaks, decayed=False, e4m3=False):
     dev = torch.device("cuda", torch.cuda.current_device())
     init = synth.decode_initial(DEC, seed=dist.rank)
     work = {k: v.to(dev) for k, v in init.items()}
+    if e4m3:
+        # the same memories in an E4M3 cache (codes + row exponents)
+        cache8 = torch.empty(work["cache"].shape, device=dev, dtype=torch.uint8)
+        cexp = torch.empty(work["cache"].shape[:-1], device=dev, dtype=torch.int8)
+        dart.cache_quantize_e4m3(work["cache"], DEC.ncached, cache8, cexp)
+        del work["cache"]
+        work["cache"], work["cache_exp"] = cache8, cexp
     if decayed:
         # log-decays of the cached memories (dart_decode_step_decayed), -U(0, 3)
         g = torch.Generator().manual_seed(1000 + dist.rank)
@@ -347,7 +357,7 @@ def decode_region(args, dist, dart, peaks, decayed=False):
             ev[0].record(stream)
         dart.dart_decode_step(t["x"], t["dt"], A, t["Bm"], t["Cm"], t["Q"], t["E"], DEC.g, work["state"],
                               work["dH_cur"], work["cache"], work["nchunks"], work["pos"], DEC.chunk, y=y,
-                              workspace=ws, memlog=work.get("memlog"))
+                              workspace=ws, memlog=work.get("memlog"), cache_exp=work.get("cache_exp"))
         if ev:
             ev[1].record(stream)
 
@@ -377,7 +387,7 @@ def decode_region(args, dist, dart, peaks, decayed=False):
     ms = dist.max(start.elapsed_time(end))
     per = [e[0].elapsed_time(e[1]) for e in evs]
     # step s starts at pos = s % S with ncached + s // S memories; pos = S-1 appends
-    total_bytes = sum(decode_bytes(DEC, DEC.ncached + s // DEC.chunk, s % DEC.chunk == DEC.chunk - 1)
+    total_bytes = sum(decode_bytes(DEC, DEC.ncached + s // DEC.chunk, s % DEC.chunk == DEC.chunk - 1, e4m3)
                       for s in range(nsteps))
     if decayed:   # each cached memory's log-decay is read and written once per step
         total_bytes += sum(8 * DEC.nseq * DEC.nheads * (DEC.ncached + s // DEC.chunk) for s in range(nsteps))
@@ -570,6 +580,14 @@ def main():
                     "roofline_frac": dd["roofline"]["frac"], "bytes_per_step": dd["roofline"]["bytes_per_step"],
                     "kernel": "dart_decode_step_decayed"}
                 line["gpu_launches"] += dd["launches"]
+            if not args.no_e4m3:
+                de = decode_region(args, dist, dart, peaks, e4m3=True)
+                line["decode"]["e4m3_cache"] = {
+                    "value": de["value"], "unit": "tokens/s", "ms_per_step": de["ms_per_step"],
+                    "roofline_frac": de["roofline"]["frac"], "bytes_per_step": de["roofline"]["bytes_per_step"],
+                    "achieved_gbs": de["roofline"]["achieved"], "kernel": "dart_decode_step_e4m3",
+                    "cache": "E4M3 codes + one int8 exponent per row (1.016 B per element)"}
+                line["gpu_launches"] += de["launches"]
         if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(fwd["inputs"])
         if dist.rank == 0:

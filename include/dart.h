@@ -227,6 +227,44 @@ dart_status dart_decode_memlog_init(const dart_dims* dims, const float* dt, cons
                                     float* mem_logdecay, int cmax, void* stream);
 
 /*
+ * dart_decode_step with an fp8 cache: each row of P values of a cached
+ * memory is stored as OCP FP8 E4M3 codes times 2^k, one signed exponent k
+ * per row -- half the bytes of a bf16 cache, and the decode step streams the
+ * cache, so about half the time (the cache quantization the pages list as
+ * an extension; the cache itself is the DART abstract's and the Pith
+ * review's "If this is right").
+ *   cache:     uint8 [B,H,cmax,N,P] E4M3 codes, in/out;
+ *   cache_exp: int8  [B,H,cmax,N] row exponents, in/out; memory row value =
+ *              code_value * 2^k.
+ * The step reads memories 0..n-1 dequantized.  When the token closes its
+ * chunk the finished contribution is quantized row by row into slot n:
+ * k = the smallest integer with max|row| * 2^-k <= 448, clamped to
+ * [-126, 60], codes = E4M3(row * 2^-k) rounded to nearest even and
+ * saturating at 448.  mem_logdecay: NULL for raw memories, else as in
+ * dart_decode_step_decayed.  Inputs x_t .. E_t in dtype (bf16 or f32); the
+ * remaining arguments, counters and errors as dart_decode_step.  Compiled
+ * for P = 64 with N = 64 or 128.  Contributions to the value readout below
+ * 2^-89 in magnitude underflow to zero.
+ */
+dart_status dart_decode_step_e4m3(const dart_dims* dims, dart_dtype dtype,
+                                  const void* x_t, const float* dt_t, const float* A,
+                                  const void* B_t, const void* C_t, const void* Q_t, const void* E_t,
+                                  float g, float* state, float* dH_cur, unsigned char* cache,
+                                  signed char* cache_exp, int cmax, int* n_chunks, int* pos,
+                                  float* mem_logdecay, float* y,
+                                  void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * The prefill -> fp8 decode handoff: memories 0..nmem-1 of dH (dtype
+ * [B,H,C,N,P] as written by dart_ssd_chunk_scan, C = ceil(seqlen / chunk))
+ * quantized into cache slots 0..nmem-1 of an E4M3 cache (layouts and
+ * rounding as dart_decode_step_e4m3).  Uses batch, seqlen, nheads, headdim,
+ * dstate and chunk of dims; nmem <= min(C, cmax).  One kernel on `stream`.
+ */
+dart_status dart_cache_quantize_e4m3(const dart_dims* dims, dart_dtype dtype, const void* dH, int nmem,
+                                     unsigned char* cache, signed char* cache_exp, int cmax, void* stream);
+
+/*
  * dart_decode_step for callers that cannot allocate device memory.  The
  * paper has no counterpart: this is an interface for embedding the decode
  * step where cudaMalloc is not available to the caller -- for example a host

@@ -278,6 +278,54 @@ dart_status dart_decode_step_decayed(const dart_dims* d, dart_dtype dtype, const
     return DART_OK;
 }
 
+dart_status dart_decode_step_e4m3(const dart_dims* d, dart_dtype dtype, const void* x_t, const float* dt_t,
+                                  const float* A, const void* B_t, const void* C_t, const void* Q_t,
+                                  const void* E_t, float g, float* state, float* dH_cur, unsigned char* cache,
+                                  signed char* cache_exp, int cmax, int* n_chunks, int* pos, float* mem_logdecay,
+                                  float* y, void* workspace, size_t workspace_bytes, void* stream) {
+    t_err[0] = 0;
+    dart_status st = check_common(d, dtype, false);
+    if (st != DART_OK) return st;
+    if (!dart::decode_e4m3_supported(d->dstate, d->headdim))
+        return fail(DART_ERR_UNSUPPORTED, "dart_decode_step_e4m3: (N=%d, P=%d) not compiled (P = 64, N = 64 or 128)",
+                    d->dstate, d->headdim);
+    if (cmax < 1) return fail(DART_ERR_INVALID_ARG, "cmax must be >= 1");
+    DART_REQUIRE_PTR(x_t); DART_REQUIRE_PTR(dt_t); DART_REQUIRE_PTR(A); DART_REQUIRE_PTR(B_t);
+    DART_REQUIRE_PTR(C_t); DART_REQUIRE_PTR(Q_t); DART_REQUIRE_PTR(E_t); DART_REQUIRE_PTR(state);
+    DART_REQUIRE_PTR(dH_cur); DART_REQUIRE_PTR(cache); DART_REQUIRE_PTR(cache_exp); DART_REQUIRE_PTR(n_chunks);
+    DART_REQUIRE_PTR(pos); DART_OPTIONAL_PTR(mem_logdecay); DART_REQUIRE_PTR(y); DART_REQUIRE_PTR(workspace);
+    if (workspace_bytes < dart_decode_step_workspace_bytes(d, dtype, cmax))
+        return fail(DART_ERR_INVALID_ARG, "workspace: %zu bytes, need %zu", workspace_bytes,
+                    dart_decode_step_workspace_bytes(d, dtype, cmax));
+    dart::DecodeArgs a{d->batch, d->nheads, d->headdim, d->dstate, d->chunk, cmax,
+                       dart::decode_num_splits(d->batch, d->nheads, cmax),
+                       x_t, dt_t, A, B_t, C_t, Q_t, E_t, g, state, dH_cur, cache,
+                       n_chunks, pos, y, static_cast<float*>(workspace), status_word(), mem_logdecay, cache_exp};
+    if (!a.status) return fail(DART_ERR_CUDA, "dart_decode_step_e4m3: no device status word");
+    cudaError_t e = dart::launch_decode_e4m3(a, dtype, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "dart_decode_step_e4m3 launch");
+    return DART_OK;
+}
+
+dart_status dart_cache_quantize_e4m3(const dart_dims* d, dart_dtype dtype, const void* dH, int nmem,
+                                     unsigned char* cache, signed char* cache_exp, int cmax, void* stream) {
+    t_err[0] = 0;
+    dart_status st = check_common(d, dtype, true);
+    if (st != DART_OK) return st;
+    if (!dart::decode_e4m3_supported(d->dstate, d->headdim))
+        return fail(DART_ERR_UNSUPPORTED, "dart_cache_quantize_e4m3: (N=%d, P=%d) not compiled", d->dstate,
+                    d->headdim);
+    const int C = (d->seqlen + d->chunk - 1) / d->chunk;
+    if (nmem < 0 || nmem > C || nmem > cmax)
+        return fail(DART_ERR_INVALID_ARG, "dart_cache_quantize_e4m3: nmem = %d outside [0, min(C = %d, cmax = %d)]",
+                    nmem, C, cmax);
+    DART_REQUIRE_PTR(dH); DART_REQUIRE_PTR(cache); DART_REQUIRE_PTR(cache_exp);
+    cudaError_t e = dart::launch_cache_quantize_e4m3(d->batch, d->nheads, C, d->dstate, d->headdim, nmem, cmax, dH,
+                                                     dtype, cache, cache_exp, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "dart_cache_quantize_e4m3 launch");
+    return DART_OK;
+}
+
 dart_status dart_decode_memlog_init(const dart_dims* d, const float* dt, const float* A, float* mem_logdecay,
                                     int cmax, void* stream) {
     t_err[0] = 0;

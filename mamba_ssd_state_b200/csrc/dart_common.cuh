@@ -129,6 +129,9 @@ struct DecodeArgs {
     // Decayed-memory variant (null: raw memories): [B,H,cmax] fp32, the
     // log-decay sum_{r=e(c)+1}^{t-1} dt_r A_h each cached memory carries.
     float* memlog;
+    // E4M3 cache (null: the cache holds dtype values): cache holds E4M3 codes
+    // [B,H,cmax,N,P] and cexp the row exponents [B,H,cmax,N] (value = code 2^k).
+    signed char* cexp;
 };
 
 // Counts one kernel launch (see dart_launch_count).
@@ -151,6 +154,12 @@ size_t sma_decay_workspace_bytes(int B, int L, int H, int S);
 const char* sma_impl_name(int N, int P, int S, dart_dtype dt);
 bool decode_supported(int N, int P, int S, dart_dtype dt);
 int decode_num_splits(int B, int H, int cmax);
+bool decode_e4m3_supported(int N, int P);
+cudaError_t launch_decode_e4m3(const DecodeArgs& a, dart_dtype dt, cudaStream_t st);
+// dH [B,H,C,N,P] (dtype) memories 0..nmem-1 -> E4M3 codes and row exponents
+// in cache slots 0..nmem-1 ([B,H,cmax,N,P] / [B,H,cmax,N]); one launch.
+cudaError_t launch_cache_quantize_e4m3(int B, int H, int C, int N, int P, int nmem, int cmax, const void* dH,
+                                       dart_dtype dt, unsigned char* cache, signed char* cexp, cudaStream_t st);
 // memlog[b,h,c] = sum_{r=(c+1)S}^{L-1} dt[b,r,h] A[h] for c < L / S (one launch).
 cudaError_t launch_decode_memlog_init(int B, int L, int H, int S, int cmax, const float* dt, const float* A,
                                       float* memlog, cudaStream_t st);

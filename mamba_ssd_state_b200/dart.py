@@ -32,7 +32,8 @@ EXPORTS = ("dart_ssd_chunk_scan_workspace_bytes", "dart_ssd_chunk_scan", "dart_s
            "dart_decode_step_workspace_bytes", "dart_decode_step", "dart_supported",
            "dart_sync_status", "dart_last_error", "dart_abi_version", "dart_launch_count",
            "dart_sma_impl", "dart_decode_step_noalloc", "dart_sma_decayed_workspace_bytes",
-           "dart_sma_forward_decayed", "dart_decode_step_decayed", "dart_decode_memlog_init")
+           "dart_sma_forward_decayed", "dart_decode_step_decayed", "dart_decode_memlog_init",
+           "dart_decode_step_e4m3", "dart_cache_quantize_e4m3")
 
 
 class DartError(RuntimeError):
@@ -68,6 +69,11 @@ def load(path: str = LIBRARY) -> ctypes.CDLL:
     lib.dart_decode_step_decayed.restype = ctypes.c_int
     lib.dart_decode_step_decayed.argtypes = ([D, ctypes.c_int] + [_P] * 7 + [ctypes.c_float] + [_P] * 3
                                              + [ctypes.c_int] + [_P] * 5 + [ctypes.c_size_t, _P])
+    lib.dart_decode_step_e4m3.restype = ctypes.c_int
+    lib.dart_decode_step_e4m3.argtypes = ([D, ctypes.c_int] + [_P] * 7 + [ctypes.c_float] + [_P] * 4
+                                          + [ctypes.c_int] + [_P] * 5 + [ctypes.c_size_t, _P])
+    lib.dart_cache_quantize_e4m3.restype = ctypes.c_int
+    lib.dart_cache_quantize_e4m3.argtypes = [D, ctypes.c_int, _P, ctypes.c_int, _P, _P, ctypes.c_int, _P]
     lib.dart_decode_memlog_init.restype = ctypes.c_int
     lib.dart_decode_memlog_init.argtypes = [D, _P, _P, _P, ctypes.c_int, _P]
     lib.dart_sma_decayed_workspace_bytes.restype = ctypes.c_size_t
@@ -306,23 +312,32 @@ def layer_forward(x, dt, A, Bm, Cm, Q, E, chunk: int, g: float, init_state=None,
 
 
 def dart_decode_step(x, dt, A, Bm, Cm, Q, E, g: float, state, dH_cur, cache, nchunks, pos,
-                     chunk: int, *, y=None, workspace=None, memlog=None):
+                     chunk: int, *, y=None, workspace=None, memlog=None, cache_exp=None):
     """One decode step for every sequence.  x[Bs,H,P], Bm/Cm[Bs,N],
     Q[Bs,H,N], E[Bs,H,P] (cache dtype), dt[Bs,H], A[H] float32; state and
     dH_cur float32 [Bs,H,N,P], cache [Bs,H,cmax,N,P], nchunks/pos int32 [Bs]
     are device tensors updated in place.  With ``memlog`` (float32
     [Bs,H,cmax] device tensor, updated in place) the memories are decayed to
-    the new token (dart_decode_step_decayed).  Returns y float32 [Bs,H,P]."""
+    the new token (dart_decode_step_decayed).  A uint8 ``cache`` is an E4M3
+    cache with row exponents ``cache_exp`` (int8 [Bs,H,cmax,N], in place);
+    the token inputs then keep their own dtype (dart_decode_step_e4m3).
+    Returns y float32 [Bs,H,P]."""
     lib = load()
+    e4m3 = cache.dtype == torch.uint8
+    if e4m3 and (cache_exp is None or cache_exp.dtype != torch.int8):
+        raise ValueError("an E4M3 (uint8) cache needs its int8 row exponents cache_exp")
     bufs = [("state", state), ("dH_cur", dH_cur), ("cache", cache), ("nchunks", nchunks), ("pos", pos)]
     if memlog is not None:
         bufs.append(("memlog", memlog))
+    if e4m3:
+        bufs.append(("cache_exp", cache_exp))
     for name, t in bufs:
         if not t.is_cuda or not t.is_contiguous():
             raise ValueError(f"{name} must be a contiguous CUDA tensor (updated in place)")
     dev = cache.device
     host = not x.is_cuda
-    x, Bm, Cm, Q, E = (_dev(v, dev, cache.dtype) for v in (x, Bm, Cm, Q, E))
+    in_dtype = x.dtype if e4m3 else cache.dtype
+    x, Bm, Cm, Q, E = (_dev(v, dev, in_dtype) for v in (x, Bm, Cm, Q, E))
     dt, A = _dev(dt, dev, torch.float32), _dev(A, dev, torch.float32)
     Bs, H, P = x.shape
     N = Bm.shape[-1]
@@ -338,15 +353,23 @@ def dart_decode_step(x, dt, A, Bm, Cm, Q, E, g: float, state, dH_cur, cache, nch
         _shape("memlog", memlog, (Bs, H, cmax))
         if memlog.dtype != torch.float32:
             raise TypeError("memlog must be float32")
+    if e4m3:
+        _shape("cache_exp", cache_exp, (Bs, H, cmax, N))
     dims = Dims(Bs, 0, H, P, N, chunk, 1)
-    code = _dtype_code(cache.dtype)
+    code = _dtype_code(in_dtype)
     if y is None:
         y = torch.empty((Bs, H, P), device=dev, dtype=torch.float32)
     wsb = lib.dart_decode_step_workspace_bytes(ctypes.byref(dims), code, cmax)
     if workspace is None:
         workspace = torch.empty(max(16, wsb), device=dev, dtype=torch.uint8)
     with torch.cuda.device(dev):
-        if memlog is None:
+        if e4m3:
+            _check(lib.dart_decode_step_e4m3(ctypes.byref(dims), code, _ptr(x), _ptr(dt), _ptr(A), _ptr(Bm),
+                                             _ptr(Cm), _ptr(Q), _ptr(E), float(g), _ptr(state), _ptr(dH_cur),
+                                             _ptr(cache), _ptr(cache_exp), cmax, _ptr(nchunks), _ptr(pos),
+                                             _ptr(memlog), _ptr(y), _ptr(workspace), workspace.numel(),
+                                             _stream()))
+        elif memlog is None:
             _check(lib.dart_decode_step(ctypes.byref(dims), code, _ptr(x), _ptr(dt), _ptr(A), _ptr(Bm),
                                         _ptr(Cm), _ptr(Q), _ptr(E), float(g), _ptr(state), _ptr(dH_cur),
                                         _ptr(cache), cmax, _ptr(nchunks), _ptr(pos), _ptr(y), _ptr(workspace),
@@ -358,6 +381,26 @@ def dart_decode_step(x, dt, A, Bm, Cm, Q, E, g: float, state, dH_cur, cache, nch
                                                 _ptr(memlog), _ptr(y), _ptr(workspace), workspace.numel(),
                                                 _stream()))
     return _to_host(y)[0] if host else y
+
+
+def cache_quantize_e4m3(dH, nmem: int, cache, cache_exp):
+    """Quantize memories 0..nmem-1 of a prefill's dH [B,H,C,N,P] (float32 or
+    bfloat16, on the device) into slots 0..nmem-1 of an E4M3 cache (uint8
+    [B,H,cmax,N,P] codes, int8 [B,H,cmax,N] row exponents), in place."""
+    lib = load()
+    for name, t in (("dH", dH), ("cache", cache), ("cache_exp", cache_exp)):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    if cache.dtype != torch.uint8 or cache_exp.dtype != torch.int8:
+        raise TypeError("cache must be uint8 and cache_exp int8")
+    Bsz, H, C, N, P = dH.shape
+    cmax = cache.shape[2]
+    _shape("cache", cache, (Bsz, H, cmax, N, P)); _shape("cache_exp", cache_exp, (Bsz, H, cmax, N))
+    dims = Dims(Bsz, C, H, P, N, 1, 1)   # C memories: seqlen C at chunk 1
+    with torch.cuda.device(dH.device):
+        _check(lib.dart_cache_quantize_e4m3(ctypes.byref(dims), _dtype_code(dH.dtype), _ptr(dH), int(nmem),
+                                            _ptr(cache), _ptr(cache_exp), cmax, _stream()))
+    return cache, cache_exp
 
 
 def decode_memlog_init(dt, A, chunk: int, memlog):

@@ -165,6 +165,25 @@ def test_decayed_decode_validation(lib):
     assert lib.dart_decode_memlog_init(None, FAKE, FAKE, FAKE, 16, None) == dart.DART_ERR_INVALID_ARG
 
 
+def test_e4m3_decode_validation(lib):
+    """The fp8-cache decode needs the code cache and the row exponents; only
+    P = 64 (N = 64 or 128) is compiled; the handoff quantizer checks nmem."""
+    d = dart.Dims(4, 0, 2, 64, 128, 256, 1)
+    ws = lib.dart_decode_step_workspace_bytes(ctypes.byref(d), dart.DART_BF16, 9)
+    f = lib.dart_decode_step_e4m3
+    args = [FAKE] * 7 + [0.5] + [FAKE, FAKE, FAKE, None] + [9] + [FAKE, FAKE, None, FAKE, FAKE, ws, None]
+    assert f(ctypes.byref(d), dart.DART_BF16, *args) == dart.DART_ERR_INVALID_ARG
+    assert b"cache_exp" in lib.dart_last_error()
+    d16 = dart.Dims(4, 0, 2, 16, 16, 64, 1)
+    args[3 + 8] = FAKE
+    assert f(ctypes.byref(d16), dart.DART_F32, *args) == dart.DART_ERR_UNSUPPORTED
+    p = dart.Dims(2, 5 * 256, 2, 64, 128, 256, 1)
+    q = lib.dart_cache_quantize_e4m3
+    assert q(ctypes.byref(p), dart.DART_BF16, FAKE, 6, FAKE, FAKE, 9, None) == dart.DART_ERR_INVALID_ARG
+    assert q(ctypes.byref(p), dart.DART_BF16, FAKE, 5, FAKE, FAKE, 4, None) == dart.DART_ERR_INVALID_ARG
+    assert q(ctypes.byref(p), dart.DART_BF16, FAKE, 2, FAKE, None, 4, None) == dart.DART_ERR_INVALID_ARG
+
+
 def test_decode_rejects_bad_args(lib):
     d = dart.Dims(4, 0, 2, 64, 128, 256, 1)
     ws = lib.dart_decode_step_workspace_bytes(ctypes.byref(d), dart.DART_BF16, 9)
