@@ -58,8 +58,9 @@
  *    factor, and a memory appended at t starts from zero.
  *
  * Readings where the pages are silent: mask c < k(t) (strict), scale 1/sqrt(N),
- * exp(dt*A) discretisation with input dt*B x^T, no D skip, ngroups = 1 (B and C
- * shared by all heads), o_t = 0 with no memory.  A sequence length that is not
+ * exp(dt*A) discretisation with input dt*B x^T, no D skip, o_t = 0 with no
+ * memory.  B and C are shared by groups of heads as in Mamba-2: with G groups
+ * (G divides H) head h reads group h / (H / G); G = 1 shares them by all.  A sequence length that is not
  * a multiple of S ends in a partial chunk: C = ceil(L / S) chunks, the last
  * one closing at token L-1 (its dH and state are what a decode would carry
  * on from); no token attends to it, since its own tokens have k(t) = C-1.
@@ -75,7 +76,7 @@
  *    appends.  Written from the format's definition, not from any library.
  *
  * Layouts (row-major, last index fastest):
- *   x[B,L,H,P] dt[B,L,H] A[H] Bm[B,L,N] Cm[B,L,N] Q[B,L,H,N] E[B,L,H,P]
+ *   x[B,L,H,P] dt[B,L,H] A[H] Bm[B,L,G,N] Cm[B,L,G,N] Q[B,L,H,N] E[B,L,H,P]
  *   y[B,L,H,P] dH[B,H,C,N,P] states[B,H,C,N,P] init_state[B,H,N,P]
  * Inputs are float (bf16 inputs are exact in float); all arithmetic and every
  * output is double.
@@ -91,7 +92,15 @@
 
 typedef struct {
     int batch, seqlen, nheads, headdim, dstate, chunk;
+    int ngroups; /* G >= 1 dividing nheads (0 is read as 1) */
 } oracle_dims;
+
+static int ngroups_of(const oracle_dims* d) { return d->ngroups > 0 ? d->ngroups : 1; }
+/* the B/C group that head h reads */
+static int group_of(const oracle_dims* d, int h) { return h / (d->nheads / ngroups_of(d)); }
+static int dims_ok(const oracle_dims* d) {
+    return d && d->chunk > 0 && d->nheads > 0 && d->nheads % ngroups_of(d) == 0;
+}
 
 /* ------------------------------------------------------------------ */
 /* a tiny work splitter over (batch, head) problems                    */
@@ -155,8 +164,9 @@ static void scan_unit(void* vctx, int unit) {
     for (int t = 0; t < L; ++t) {
         const double dtt = (double)c->dt[((size_t)b * L + t) * H + h];
         const double decay = exp(dtt * Ah);
-        const float* Bt = c->Bm + ((size_t)b * L + t) * N;
-        const float* Ct = c->Cm + ((size_t)b * L + t) * N;
+        const size_t bc = (((size_t)b * L + t) * ngroups_of(d) + group_of(d, h)) * N;
+        const float* Bt = c->Bm + bc;
+        const float* Ct = c->Cm + bc;
         const float* xt = c->x + (((size_t)b * L + t) * H + h) * P;
         if (t % S == 0) memset(D, 0, sizeof(double) * (size_t)N * P);
         for (int n = 0; n < N; ++n) {
@@ -187,7 +197,7 @@ static void scan_unit(void* vctx, int unit) {
 int oracle_ssd_scan(const oracle_dims* d, const float* x, const float* dt, const float* A,
                     const float* Bm, const float* Cm, const double* init_state,
                     double* y_ssd, double* dH, double* states, int nthreads) {
-    if (!d || d->chunk <= 0 || d->seqlen <= 0) return -1;
+    if (!dims_ok(d) || d->seqlen <= 0) return -1;
     scan_ctx c = {d, x, dt, A, Bm, Cm, init_state, y_ssd, dH, states};
     run_units(scan_unit, &c, d->batch * d->nheads, nthreads);
     return 0;
@@ -227,7 +237,7 @@ static void sma_unit(void* vctx, int unit) {
         const int k = t / S; /* chunk holding t; memories are c < k */
         const float* Qt = c->Q + (((size_t)b * L + t) * H + h) * N;
         const float* Et = c->E + (((size_t)b * L + t) * H + h) * P;
-        const float* Ct = c->Cm + ((size_t)b * L + t) * N;
+        const float* Ct = c->Cm + (((size_t)b * L + t) * ngroups_of(d) + group_of(d, h)) * N;
         for (int cc = 0; cc < k; ++cc) {
             const double* M = c->dH + (((size_t)b * H + h) * nchunks + cc) * (size_t)N * P;
             /* decayed variant: the factor that carries dH[c] from e(c) to t */
@@ -288,7 +298,7 @@ static void sma_unit(void* vctx, int unit) {
 }
 
 /*
- * Q[B,L,H,N], E[B,L,H,P], Cm[B,L,N] float; dH[B,H,C,N,P] double.
+ * Q[B,L,H,N], E[B,L,H,P], Cm[B,L,G,N] float; dH[B,H,C,N,P] double.
  * dt[B,L,H] and A[H] float, both NULL for raw memories or both given for the
  * decayed-memory variant.
  * With tokens == NULL every position is computed and the outputs are
@@ -299,7 +309,7 @@ int oracle_sma(const oracle_dims* d, const float* Q, const float* E, const float
                const double* dH, const float* dt, const float* A, double g,
                const double* y_ssd, double* o, double* y, double* scores,
                const int* tokens, int ntok, int nthreads) {
-    if (!d || d->chunk <= 0 || d->seqlen <= 0) return -1;
+    if (!dims_ok(d) || d->seqlen <= 0) return -1;
     if ((dt == NULL) != (A == NULL)) return -1;
     if (tokens) {
         for (int i = 0; i < ntok; ++i)
@@ -400,8 +410,8 @@ static void decode_unit(void* vctx, int unit) {
     double* Hs = c->state + bh * N * P;
     double* D = c->dHcur + bh * N * P;
     const float* xt = c->x + bh * P;
-    const float* Bt = c->Bm + (size_t)b * N;
-    const float* Ct = c->Cm + (size_t)b * N;
+    const float* Bt = c->Bm + ((size_t)b * ngroups_of(d) + group_of(d, h)) * N;
+    const float* Ct = c->Cm + ((size_t)b * ngroups_of(d) + group_of(d, h)) * N;
     const float* Qt = c->Q + bh * N;
     const float* Et = c->E + bh * P;
     const double dtt = (double)c->dt[bh];
@@ -479,7 +489,7 @@ static void decode_unit(void* vctx, int unit) {
 }
 
 /*
- * x[Bs,H,P] dt[Bs,H] A[H] Bm[Bs,N] Cm[Bs,N] Q[Bs,H,N] E[Bs,H,P] (float);
+ * x[Bs,H,P] dt[Bs,H] A[H] Bm[Bs,G,N] Cm[Bs,G,N] Q[Bs,H,N] E[Bs,H,P] (float);
  * state, dH_cur [Bs,H,N,P], cache [Bs,H,cmax,N,P], y [Bs,H,P] (double);
  * nchunks[Bs], pos[Bs] in/out; memlog [Bs,H,cmax] (double, in/out) selects
  * the decayed-memory variant when not NULL; cache_e4m3 != 0 makes an append
@@ -492,7 +502,7 @@ int oracle_decode_step(const oracle_dims* d, int cmax, const float* x, const flo
                        const float* E, double g, double* state, double* dH_cur, double* cache,
                        int* nchunks, int* pos, double* memlog, int cache_e4m3, double* y,
                        int nthreads) {
-    if (!d || d->chunk <= 0) return -1;
+    if (!dims_ok(d)) return -1;
     for (int b = 0; b < d->batch; ++b) {
         if (nchunks[b] < 0 || nchunks[b] > cmax) return -1;
         if (pos[b] < 0 || pos[b] >= d->chunk) return -1;

@@ -23,7 +23,13 @@ LIBRARY = os.path.join(_HERE, "libdart_oracle.so")
 
 class _Dims(ctypes.Structure):
     _fields_ = [(name, ctypes.c_int) for name in
-                ("batch", "seqlen", "nheads", "headdim", "dstate", "chunk")]
+                ("batch", "seqlen", "nheads", "headdim", "dstate", "chunk", "ngroups")]
+
+
+def _groups(a, ndim_shared: int) -> int:
+    """Number of B/C groups of an array: ndim_shared dims means one group
+    shared by all heads; one more dim is the group axis (second to last)."""
+    return 1 if a.ndim == ndim_shared else a.shape[-2]
 
 
 def build(source: str = SOURCE, library: str = LIBRARY, extra_flags=()) -> str:
@@ -87,7 +93,7 @@ class Oracle:
         Bsz, L, H, P = x.shape
         N = Bm.shape[-1]
         C = -(-L // chunk)
-        d = _Dims(Bsz, L, H, P, N, chunk)
+        d = _Dims(Bsz, L, H, P, N, chunk, _groups(Bm, 3))
         y = np.empty((Bsz, L, H, P), np.float64)
         dH = np.empty((Bsz, H, C, N, P), np.float64)
         st = np.empty((Bsz, H, C, N, P), np.float64)
@@ -116,7 +122,7 @@ class Oracle:
         Bsz, L, H, N = Q.shape
         P = E.shape[-1]
         C = -(-L // chunk)
-        d = _Dims(Bsz, L, H, P, N, chunk)
+        d = _Dims(Bsz, L, H, P, N, chunk, _groups(Cm, 3))
         tok = None if tokens is None else np.ascontiguousarray(np.asarray(tokens, np.int32))
         rows = L if tok is None else len(tok)
         o = np.empty((Bsz, rows, H, P), np.float64)
@@ -182,7 +188,7 @@ class Oracle:
         Bs, H, P = x.shape
         N = Bm.shape[-1]
         cmax = cache.shape[2]
-        d = _Dims(Bs, 0, H, P, N, chunk)
+        d = _Dims(Bs, 0, H, P, N, chunk, _groups(Bm, 2))
         y = np.empty((Bs, H, P), np.float64)
         rc = self.lib.oracle_decode_step(ctypes.byref(d), cmax, self._ptr(x), self._ptr(dt),
                                          self._ptr(A), self._ptr(Bm), self._ptr(Cm),

@@ -618,6 +618,55 @@ def pin_e4m3_decode_append(orc):
         assert np.array_equal(ya, yb), f"step {t}"
 
 
+# ----------------------------------------------------------------------------
+# B and C shared by groups of heads (Mamba-2 ngroups)
+# ----------------------------------------------------------------------------
+def pin_ngroups_split_into_independent_problems(orc):
+    """With G groups head h reads B and C of group h // (H / G).  A layer with
+    H = 4 heads in G = 2 groups (and G = 4: every head its own B, C) equals G
+    separate layers of H / G heads each fed its own group's B and C through
+    the single-group path pinned above: scan outputs, SMA and layer output,
+    and a decode step."""
+    Bz, L, H, P, N, S = 2, 20, 4, 3, 4, 8
+    r = np.random.default_rng(41)
+    for G in (2, 4):
+        inp = _rand_layer(41 + G, Bz, L, H, P, N)
+        Bg = (r.standard_normal((Bz, L, G, N)) / np.sqrt(N)).astype(np.float32)
+        Cg = (r.standard_normal((Bz, L, G, N)) / np.sqrt(N)).astype(np.float32)
+        full = orc.layer_forward(inp["x"], inp["dt"], inp["A"], Bg, Cg, inp["Q"], inp["E"], S, 0.6)
+        hg = H // G
+        for g in range(G):
+            hs = slice(g * hg, (g + 1) * hg)
+            part = orc.layer_forward(inp["x"][:, :, hs], inp["dt"][:, :, hs], inp["A"][hs], Bg[:, :, g],
+                                     Cg[:, :, g], inp["Q"][:, :, hs], inp["E"][:, :, hs], S, 0.6)
+            for k in ("y", "y_ssd", "o"):
+                assert np.array_equal(full[k][:, :, hs], part[k]), (G, g, k)
+            for k in ("dH", "states"):
+                assert np.array_equal(full[k][:, hs], part[k]), (G, g, k)
+        # one decode step from the prefill's last boundary
+        cmax = L // S + 1
+        nc = L // S
+        t = L - 1
+        rr = np.random.default_rng(42)
+        cache = np.zeros((Bz, H, cmax, N, P))
+        cache[:, :, :nc] = full["dH"][:, :, :nc]
+        state = rr.standard_normal((Bz, H, N, P))
+        dcur = rr.standard_normal((Bz, H, N, P)) * 0.1
+        nch = np.full((Bz,), nc, np.int32)
+        pos = np.full((Bz,), 3, np.int32)
+        ys = {}
+        for g in [None] + list(range(G)):
+            hs = slice(None) if g is None else slice(g * hg, (g + 1) * hg)
+            Bt = Bg[:, t] if g is None else Bg[:, t, g]
+            Ct = Cg[:, t] if g is None else Cg[:, t, g]
+            st, dc, ca = (np.array(a[:, hs], copy=True, order="C") for a in (state, dcur, cache))
+            ys[g] = orc.decode_step(inp["x"][:, t, hs], inp["dt"][:, t, hs], inp["A"][hs], Bt, Ct,
+                                    inp["Q"][:, t, hs], inp["E"][:, t, hs], 0.6, st, dc, ca,
+                                    nch.copy(), pos.copy(), S)
+        for g in range(G):
+            assert np.array_equal(ys[None][:, g * hg:(g + 1) * hg], ys[g]), (G, g, "decode")
+
+
 ALL_PINS = [
     pin_closed_form_single_token,
     pin_quadratic_form,
@@ -638,4 +687,5 @@ ALL_PINS = [
     pin_decayed_decode_matches_prefill,
     pin_e4m3_rows_match_library,
     pin_e4m3_decode_append,
+    pin_ngroups_split_into_independent_problems,
 ]

@@ -65,6 +65,7 @@ MUTATIONS = [
     ("e4m3_subnormal_step", "const double q = nearbyint(a * 512.0);", "const double q = nearbyint(a * 256.0);", 0),
     ("e4m3_decode_bias", "ldexp(8.0 + m, e - 10)", "ldexp(8.0 + m, e - 11)", 0),
     ("decode_append_not_quantized", "if (c->cache_e4m3) {", "if (0) {", 0),
+    ("group_by_modulo", "return h / (d->nheads / ngroups_of(d));", "return h % ngroups_of(d);", 0),
 ]
 
 
