@@ -162,6 +162,39 @@ dart_status dart_sma_forward_decayed(const dart_dims* dims, dart_dtype dtype,
                                      float* out, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Workspace for dart_sma_backward, in bytes: the softmax weights and score
+ * gradients of every (token, memory) pair (2 * B*H*L*C floats), the per-head
+ * dC (B*L*H*N floats) and per-tile dg partials, each padded to 256 bytes.
+ * 0 for invalid dims.
+ */
+size_t dart_sma_backward_workspace_bytes(const dart_dims* dims);
+
+/*
+ * Gradients of state-memory attention with the gated residual (the training
+ * pass, DART abstract "DART supports practical training"; the forward of
+ * dart_sma_forward with raw memories).  Given dy = dLoss/dy for
+ * y = y_ssd + g o, with do = g dy_t, p the softmax over the memories c < k(t),
+ * v_c = C_t^T dH[c], w1 = dH[c] E_t, w2 = dH[c] do and D_t = do . o_t:
+ *   ds_c = p_c (C_t . w2 - D_t)
+ *   dQ_t = sum_c ds_c w1 / sqrt(N)         dE_t = sum_c ds_c dH[c]^T Q_t / sqrt(N)
+ *   dC_t = sum_h sum_c p_c w2              dg = sum dy . o
+ *   ddH[c] = sum_{t: k(t) > c} (ds_tc / sqrt(N) Q_t E_t^T + p_tc C_t do_t^T)
+ * (dy also flows unchanged to y_ssd; that part is the caller's.)
+ *   Q[B,L,H,N], E[B,L,H,P], Cm[B,L,N], dH[B,H,C,N,P]: dtype inputs (as given
+ *   to the forward); dy: float [B,L,H,P].
+ *   dQ float [B,L,H,N], dE float [B,L,H,P], dCm float [B,L,N],
+ *   ddH float [B,H,C,N,P], dg float [1]: outputs, every element written.
+ *   workspace: device scratch of dart_sma_backward_workspace_bytes().
+ * CUDA-core kernels; sums run in a fixed order (deterministic).  Shapes and
+ * errors as dart_sma_forward.
+ */
+dart_status dart_sma_backward(const dart_dims* dims, dart_dtype dtype,
+                              const void* Q, const void* E, const void* Cm, const void* dH,
+                              float g, const float* dy, float* dQ, float* dE, float* dCm,
+                              float* ddH, float* dg, void* workspace, size_t workspace_bytes,
+                              void* stream);
+
+/*
  * Workspace for dart_decode_step: per (sequence, head, split) partial softmax
  * statistics and partial outputs.  Pass at least this many bytes.
  */

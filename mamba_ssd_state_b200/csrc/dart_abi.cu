@@ -215,6 +215,34 @@ dart_status dart_sma_forward_decayed(const dart_dims* d, dart_dtype dtype, const
     return DART_OK;
 }
 
+size_t dart_sma_backward_workspace_bytes(const dart_dims* d) {
+    if (!d) return 0;
+    return dart::sma_bwd_workspace_bytes(d->batch, d->seqlen, d->nheads, d->dstate, d->chunk);
+}
+
+dart_status dart_sma_backward(const dart_dims* d, dart_dtype dtype, const void* Q, const void* E, const void* Cm,
+                              const void* dH, float g, const float* dy, float* dQ, float* dE, float* dCm,
+                              float* ddH, float* dg, void* workspace, size_t workspace_bytes, void* stream) {
+    t_err[0] = 0;
+    dart_status st = check_common(d, dtype, true);
+    if (st != DART_OK) return st;
+    if (!dart::sma_supported(d->dstate, d->headdim, d->chunk, dtype))
+        return fail(DART_ERR_UNSUPPORTED, "dart_sma_backward: (N=%d, P=%d, S=%d) not compiled", d->dstate,
+                    d->headdim, d->chunk);
+    DART_REQUIRE_PTR(Q); DART_REQUIRE_PTR(E); DART_REQUIRE_PTR(Cm); DART_REQUIRE_PTR(dH); DART_REQUIRE_PTR(dy);
+    DART_REQUIRE_PTR(dQ); DART_REQUIRE_PTR(dE); DART_REQUIRE_PTR(dCm); DART_REQUIRE_PTR(ddH); DART_REQUIRE_PTR(dg);
+    DART_REQUIRE_PTR(workspace);
+    const size_t need = dart_sma_backward_workspace_bytes(d);
+    if (workspace_bytes < need)
+        return fail(DART_ERR_INVALID_ARG, "workspace: %zu bytes, need %zu", workspace_bytes, need);
+    dart::SmaBwdArgs a{d->batch, d->seqlen, d->nheads, d->headdim, d->dstate, d->chunk, Q, E, Cm, dH, g, dy,
+                       dQ, dE, dCm, ddH, dg, status_word()};
+    if (!a.status) return fail(DART_ERR_CUDA, "dart_sma_backward: no device status word");
+    cudaError_t e = dart::launch_sma_bwd(a, workspace, dtype, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "dart_sma_backward launch");
+    return DART_OK;
+}
+
 size_t dart_decode_step_workspace_bytes(const dart_dims* d, dart_dtype, int cmax) {
     if (!d || cmax < 0) return 0;
     const size_t ns = (size_t)dart::decode_num_splits(d->batch, d->nheads, cmax);

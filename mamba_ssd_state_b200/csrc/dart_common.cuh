@@ -119,6 +119,17 @@ struct SmaArgs {
     const float* la2;     // [B,H,C*S] fp32
     const double* gpre;   // [B,H,C] fp64
 };
+struct SmaBwdArgs {
+    int B, L, H, P, N, S;
+    const void* Q; const void* E; const void* Cm; const void* dH;
+    float g; const float* dy;               // dy: [B,L,H,P] gradient of the layer output
+    float* dQ; float* dE; float* dCm; float* ddH; float* dg;   // outputs (fp32)
+    int* status;
+    // workspace views (set by launch_sma_bwd)
+    float* pbuf; float* dsbuf;              // [B,H,L,C] softmax weights and score gradients
+    float* dCh;                             // [B,L,H,N] per-head dC
+    float* gpart;                           // [B,H,tiles] per-tile dg
+};
 struct DecodeArgs {
     int B, H, P, N, S, cmax, nsplit;
     const void* x; const float* dt; const float* A; const void* Bm; const void* Cm;
@@ -153,6 +164,8 @@ cudaError_t launch_sma_decay_terms(int B, int L, int H, int S, const float* dt, 
 size_t sma_decay_workspace_bytes(int B, int L, int H, int S);
 const char* sma_impl_name(int N, int P, int S, dart_dtype dt);
 bool decode_supported(int N, int P, int S, dart_dtype dt);
+size_t sma_bwd_workspace_bytes(int B, int L, int H, int N, int S);
+cudaError_t launch_sma_bwd(SmaBwdArgs a, void* workspace, dart_dtype dt, cudaStream_t st);
 int decode_num_splits(int B, int H, int cmax);
 bool decode_e4m3_supported(int N, int P);
 cudaError_t launch_decode_e4m3(const DecodeArgs& a, dart_dtype dt, cudaStream_t st);

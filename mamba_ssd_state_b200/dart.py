@@ -33,7 +33,8 @@ EXPORTS = ("dart_ssd_chunk_scan_workspace_bytes", "dart_ssd_chunk_scan", "dart_s
            "dart_sync_status", "dart_last_error", "dart_abi_version", "dart_launch_count",
            "dart_sma_impl", "dart_decode_step_noalloc", "dart_sma_decayed_workspace_bytes",
            "dart_sma_forward_decayed", "dart_decode_step_decayed", "dart_decode_memlog_init",
-           "dart_decode_step_e4m3", "dart_cache_quantize_e4m3")
+           "dart_decode_step_e4m3", "dart_cache_quantize_e4m3", "dart_sma_backward_workspace_bytes",
+           "dart_sma_backward")
 
 
 class DartError(RuntimeError):
@@ -69,6 +70,11 @@ def load(path: str = LIBRARY) -> ctypes.CDLL:
     lib.dart_decode_step_decayed.restype = ctypes.c_int
     lib.dart_decode_step_decayed.argtypes = ([D, ctypes.c_int] + [_P] * 7 + [ctypes.c_float] + [_P] * 3
                                              + [ctypes.c_int] + [_P] * 5 + [ctypes.c_size_t, _P])
+    lib.dart_sma_backward_workspace_bytes.restype = ctypes.c_size_t
+    lib.dart_sma_backward_workspace_bytes.argtypes = [D]
+    lib.dart_sma_backward.restype = ctypes.c_int
+    lib.dart_sma_backward.argtypes = ([D, ctypes.c_int] + [_P] * 4 + [ctypes.c_float] + [_P] * 7
+                                      + [ctypes.c_size_t, _P])
     lib.dart_decode_step_e4m3.restype = ctypes.c_int
     lib.dart_decode_step_e4m3.argtypes = ([D, ctypes.c_int] + [_P] * 7 + [ctypes.c_float] + [_P] * 4
                                           + [ctypes.c_int] + [_P] * 5 + [ctypes.c_size_t, _P])
@@ -276,6 +282,35 @@ def dart_sma_forward_decayed(Q, E, Cm, dH, dt, A, chunk: int, g: float, y_ssd=No
                                             _ptr(Cm), _ptr(dH), _ptr(dt), _ptr(A), float(g), _ptr(y_ssd),
                                             _ptr(out), _ptr(workspace), workspace.numel(), _stream()))
     return _to_host(out)[0] if host else out
+
+
+def dart_sma_backward(Q, E, Cm, dH, chunk: int, g: float, dy, *, workspace=None) -> dict:
+    """Gradients of sum(dy * y) for y = y_ssd + g * SMA(Q, E, Cm; dH) (raw
+    memories): a dict of float32 device tensors dQ [B,L,H,N], dE [B,L,H,P],
+    dCm [B,L,N], ddH [B,H,C,N,P] and dg (shape [1]).  Inputs as for
+    dart_sma_forward, on the device; dy float32 [B,L,H,P]."""
+    lib = load()
+    dev = _device_of(Q, E, Cm, dH, dy)
+    Q, E, Cm, dH = (_dev(v, dev, Q.dtype) for v in (Q, E, Cm, dH))
+    dy = _dev(dy, dev, torch.float32)
+    Bsz, L, H, N = Q.shape
+    P = E.shape[-1]
+    C = -(-L // chunk)
+    _shape("E", E, (Bsz, L, H, P)); _shape("Cm", Cm, (Bsz, L, N)); _shape("dH", dH, (Bsz, H, C, N, P))
+    _shape("dy", dy, (Bsz, L, H, P))
+    dims = Dims(Bsz, L, H, P, N, chunk, 1)
+    out = {"dQ": torch.empty((Bsz, L, H, N), device=dev), "dE": torch.empty((Bsz, L, H, P), device=dev),
+           "dCm": torch.empty((Bsz, L, N), device=dev), "ddH": torch.empty((Bsz, H, C, N, P), device=dev),
+           "dg": torch.empty((1,), device=dev)}
+    wsb = lib.dart_sma_backward_workspace_bytes(ctypes.byref(dims))
+    if workspace is None:
+        workspace = torch.empty(max(16, wsb), device=dev, dtype=torch.uint8)
+    with torch.cuda.device(dev):
+        _check(lib.dart_sma_backward(ctypes.byref(dims), _dtype_code(Q.dtype), _ptr(Q), _ptr(E), _ptr(Cm), _ptr(dH),
+                                     float(g), _ptr(dy), _ptr(out["dQ"]), _ptr(out["dE"]), _ptr(out["dCm"]),
+                                     _ptr(out["ddH"]), _ptr(out["dg"]), _ptr(workspace), workspace.numel(),
+                                     _stream()))
+    return out
 
 
 def sma_decayed_workspace_bytes(batch, seqlen, nheads, headdim, dstate, chunk) -> int:

@@ -184,6 +184,23 @@ def test_e4m3_decode_validation(lib):
     assert q(ctypes.byref(p), dart.DART_BF16, FAKE, 2, FAKE, None, 4, None) == dart.DART_ERR_INVALID_ARG
 
 
+def test_sma_backward_workspace_and_validation(lib):
+    d = dart.Dims(2, 500, 3, 64, 128, 256, 1)
+    C, tiles = 2, 16
+    pad = lambda b: (b + 255) // 256 * 256
+    want = 2 * pad(4 * 2 * 3 * 500 * C) + pad(4 * 2 * 500 * 3 * 128) + pad(4 * 2 * 3 * tiles)
+    assert lib.dart_sma_backward_workspace_bytes(ctypes.byref(d)) == want
+    ws = want
+    f = lib.dart_sma_backward
+    assert f(ctypes.byref(d), dart.DART_BF16, FAKE, FAKE, FAKE, FAKE, 0.5, None, FAKE, FAKE, FAKE, FAKE, FAKE,
+             FAKE, ws, None) == dart.DART_ERR_INVALID_ARG
+    assert f(ctypes.byref(d), dart.DART_BF16, FAKE, FAKE, FAKE, FAKE, 0.5, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+             FAKE, ws - 1, None) == dart.DART_ERR_INVALID_ARG
+    d.chunk = 96
+    assert f(ctypes.byref(d), dart.DART_BF16, FAKE, FAKE, FAKE, FAKE, 0.5, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+             FAKE, 1 << 30, None) == dart.DART_ERR_UNSUPPORTED
+
+
 def test_decode_rejects_bad_args(lib):
     d = dart.Dims(4, 0, 2, 64, 128, 256, 1)
     ws = lib.dart_decode_step_workspace_bytes(ctypes.byref(d), dart.DART_BF16, 9)
