@@ -153,3 +153,21 @@ def sma_grads(Q, E, Cm, dH, chunk: int, g: float, dy, dt=None, A=None) -> dict:
     for n, gr in zip(names, grads):
         res["d" + n] = (gr if gr is not None else torch.zeros_like(ts[n])).detach().numpy()
     return res
+
+
+def scan_grads(x, dt, A, Bm, Cm, chunk: int, dy, gdH, init_state=None) -> dict:
+    """Gradients of sum(dy * y_ssd) + sum(gdH * dH) through the scan alone
+    (gdH is what the SMA backward hands back for the memories): dx, ddt, dA,
+    dBm, dCm (and dinit_state when an initial state is given), plus the
+    forward outputs y_ssd, dH, states."""
+    names = ["x", "dt", "A", "Bm", "Cm"]
+    ts = {n: _t(v, True) for n, v in zip(names, (x, dt, A, Bm, Cm))}
+    h0 = None if init_state is None else _t(init_state, True)
+    y_ssd, dH, st = ssd_scan(ts["x"], ts["dt"], ts["A"], ts["Bm"], ts["Cm"], chunk, h0)
+    loss = (y_ssd * _t(dy)).sum() + (dH * _t(gdH)).sum()
+    want = [ts[n] for n in names] + ([h0] if h0 is not None else [])
+    grads = torch.autograd.grad(loss, want, allow_unused=True)
+    res = {"y_ssd": y_ssd.detach().numpy(), "dH": dH.detach().numpy(), "states": st.detach().numpy()}
+    for n, gr, src in zip(names + ["init_state"], grads, want):
+        res["d" + n] = (gr if gr is not None else torch.zeros_like(src)).detach().numpy()
+    return res

@@ -152,3 +152,50 @@ def test_sma_gradients_match_finite_differences(orc, decayed):
             m_[name][idx] -= hstep
             fd = (loss(**p_) - loss(**m_)) / (2 * hstep)
             assert abs(gr[key][idx] - fd) <= 1e-6 * max(1.0, abs(fd)), (name, idx, gr[key][idx], fd)
+
+
+def test_layer_gradients_compose_from_scan_and_sma():
+    """The chain rule across the two steps: layer gradients = the scan's
+    gradients driven by (dy, ddH from the SMA backward) plus the SMA's own
+    gradients of Q, E and C (B and C of the scan and of SMA are one tensor)."""
+    Bz, L, H, P, N, S = 1, 21, 2, 3, 4, 8
+    g = 0.6
+    inp = _inputs(21, Bz, L, H, P, N)
+    h0 = np.random.default_rng(22).standard_normal((Bz, H, N, P)) * 0.2
+    dy = np.random.default_rng(23).standard_normal((Bz, L, H, P))
+    full = dart_backward.layer_grads(*(inp[k] for k in KEYS), S, g, dy, init_state=h0)
+    sm = dart_backward.sma_grads(inp["Q"], inp["E"], inp["Cm"], full["dH"], S, g, dy)
+    sc = dart_backward.scan_grads(inp["x"], inp["dt"], inp["A"], inp["Bm"], inp["Cm"], S, dy, sm["ddH"],
+                                  init_state=h0)
+    for k in ("dx", "ddt", "dA", "dBm", "dinit_state"):
+        np.testing.assert_allclose(sc[k], full[k], rtol=1e-11, atol=1e-12, err_msg=k)
+    np.testing.assert_allclose(sc["dCm"] + sm["dCm"], full["dCm"], rtol=1e-11, atol=1e-12)
+    for k in ("dQ", "dE"):
+        np.testing.assert_allclose(sm[k], full[k], rtol=1e-11, atol=1e-12, err_msg=k)
+
+
+def test_scan_gradients_match_finite_differences(orc):
+    """dx, ddt, dA, dB, dC of sum(dy * y_ssd) + sum(gdH * dH) against central
+    differences of the C oracle's scan (ragged length, initial state)."""
+    Bz, L, H, P, N, S = 1, 19, 2, 3, 4, 8
+    inp = _inputs(24, Bz, L, H, P, N)
+    C = -(-L // S)
+    r = np.random.default_rng(25)
+    h0 = r.standard_normal((Bz, H, N, P)) * 0.3
+    dy = r.standard_normal((Bz, L, H, P))
+    gdH = r.standard_normal((Bz, H, C, N, P))
+    gr = dart_backward.scan_grads(inp["x"], inp["dt"], inp["A"], inp["Bm"], inp["Cm"], S, dy, gdH, init_state=h0)
+
+    def loss(d):
+        y, dH, _ = orc.ssd_scan(d["x"], d["dt"], d["A"], d["Bm"], d["Cm"], S, init_state=h0)
+        return float(np.sum(dy * y) + np.sum(gdH * dH))
+    for name in ("x", "dt", "A", "Bm", "Cm"):
+        a = inp[name]
+        for idx in [tuple(r.integers(0, s_) for s_ in a.shape) for _ in range(4)]:
+            hstep = _step(a[idx])
+            plus, minus = dict(inp), dict(inp)
+            plus[name], minus[name] = a.copy(), a.copy()
+            plus[name][idx] += hstep
+            minus[name][idx] -= hstep
+            fd = (loss(plus) - loss(minus)) / (2 * hstep)
+            assert abs(gr["d" + name][idx] - fd) <= 1e-6 * max(1.0, abs(fd)), (name, idx, gr["d" + name][idx], fd)
