@@ -162,6 +162,45 @@ dart_status dart_sma_forward_decayed(const dart_dims* dims, dart_dtype dtype,
                                      float* out, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Workspace for dart_ssd_scan_backward, in bytes: the recomputed states of
+ * one chunk per (b, h) (2 * B*H*S*N*P floats), per-head dB and dC
+ * (2 * B*L*H*N floats) and per-(b, h) dA, each padded to 256 bytes.
+ */
+size_t dart_ssd_scan_backward_workspace_bytes(const dart_dims* dims);
+
+/*
+ * Gradients through dart_ssd_chunk_scan (the training pass, DART abstract
+ * "DART supports practical training"; the recurrence of Eq. (4) of the SSD
+ * view).  For loss = sum(dy * y_ssd) + sum(ddH * dH), with a_t = exp(dt_t A_h)
+ * and the adjoints run from the last token,
+ *   G_t = C_t dy_t^T + a_{t+1} G_{t+1}                     (dLoss/dH_t)
+ *   K_t = ddH[c] at the chunk's last token, a_{t+1} K_{t+1} inside the chunk
+ *   dx_t = dt_t (G_t + K_t)^T B_t,  dB_t = sum_h dt_t (G_t + K_t) x_t,
+ *   dC_t = sum_h H_t dy_t,
+ *   ddt_t = sum((G_t + K_t) o B_t x_t^T) + A_h a_t (sum(G_t o H_{t-1}) + sum(K_t o D_{t-1})),
+ *   dA_h = sum over b, t of dt_t a_t (sum(G_t o H_{t-1}) + sum(K_t o D_{t-1})),
+ *   dinit_state = a_0 G_0,
+ * D the chunk-restarted accumulator whose value at a chunk's last token is
+ * dH[c].  The forward's H_{t-1} are recomputed chunk by chunk from `states`.
+ *   x, Bm, Cm: dtype, dt, A, init_state (nullable): float -- the forward's inputs;
+ *   states: float [B,H,C,N,P] the forward's boundary states;
+ *   dy: float [B,L,H,P]; ddH: nullable float [B,H,C,N,P] (NULL = zero), e.g.
+ *   dart_sma_backward's memory gradient;
+ *   dx float [B,L,H,P], ddt float [B,L,H], dA float [H], dBm, dCm float [B,L,N]
+ *   (dCm is the scan's part: add dart_sma_backward's for the layer);
+ *   dinit_state: nullable float [B,H,N,P].
+ * CUDA cores, one CTA per (b, h); sums in a fixed order (deterministic).
+ * Compiled for (N, P) = (128, 64), (64, 64), (16, 16).
+ */
+dart_status dart_ssd_scan_backward(const dart_dims* dims, dart_dtype dtype,
+                                   const void* x, const float* dt, const float* A,
+                                   const void* Bm, const void* Cm, const float* init_state,
+                                   const float* states, const float* dy, const float* ddH,
+                                   float* dx, float* ddt, float* dA, float* dBm, float* dCm,
+                                   float* dinit_state, void* workspace, size_t workspace_bytes,
+                                   void* stream);
+
+/*
  * Workspace for dart_sma_backward, in bytes: the softmax weights and score
  * gradients of every (token, memory) pair (2 * B*H*L*C floats), the per-head
  * dC (B*L*H*N floats) and per-tile dg partials, each padded to 256 bytes.

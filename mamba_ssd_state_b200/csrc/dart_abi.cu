@@ -215,6 +215,36 @@ dart_status dart_sma_forward_decayed(const dart_dims* d, dart_dtype dtype, const
     return DART_OK;
 }
 
+size_t dart_ssd_scan_backward_workspace_bytes(const dart_dims* d) {
+    if (!d) return 0;
+    return dart::scan_bwd_workspace_bytes(d->batch, d->seqlen, d->nheads, d->dstate, d->headdim, d->chunk);
+}
+
+dart_status dart_ssd_scan_backward(const dart_dims* d, dart_dtype dtype, const void* x, const float* dt,
+                                   const float* A, const void* Bm, const void* Cm, const float* init_state,
+                                   const float* states, const float* dy, const float* ddH, float* dx, float* ddt,
+                                   float* dA, float* dBm, float* dCm, float* dinit_state, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
+    t_err[0] = 0;
+    dart_status st = check_common(d, dtype, true);
+    if (st != DART_OK) return st;
+    if (!dart::scan_bwd_supported(d->dstate, d->headdim))
+        return fail(DART_ERR_UNSUPPORTED, "dart_ssd_scan_backward: (N=%d, P=%d) not compiled", d->dstate, d->headdim);
+    DART_REQUIRE_PTR(x); DART_REQUIRE_PTR(dt); DART_REQUIRE_PTR(A); DART_REQUIRE_PTR(Bm); DART_REQUIRE_PTR(Cm);
+    DART_OPTIONAL_PTR(init_state); DART_REQUIRE_PTR(states); DART_REQUIRE_PTR(dy); DART_OPTIONAL_PTR(ddH);
+    DART_REQUIRE_PTR(dx); DART_REQUIRE_PTR(ddt); DART_REQUIRE_PTR(dA); DART_REQUIRE_PTR(dBm); DART_REQUIRE_PTR(dCm);
+    DART_OPTIONAL_PTR(dinit_state); DART_REQUIRE_PTR(workspace);
+    const size_t need = dart_ssd_scan_backward_workspace_bytes(d);
+    if (workspace_bytes < need)
+        return fail(DART_ERR_INVALID_ARG, "workspace: %zu bytes, need %zu", workspace_bytes, need);
+    dart::ScanBwdArgs a{d->batch, d->seqlen, d->nheads, d->headdim, d->dstate, d->chunk, x, dt, A, Bm, Cm,
+                        init_state, states, dy, ddH, dx, ddt, dA, dBm, dCm, dinit_state, status_word()};
+    if (!a.status) return fail(DART_ERR_CUDA, "dart_ssd_scan_backward: no device status word");
+    cudaError_t e = dart::launch_ssd_scan_bwd(a, workspace, dtype, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "dart_ssd_scan_backward launch");
+    return DART_OK;
+}
+
 size_t dart_sma_backward_workspace_bytes(const dart_dims* d) {
     if (!d) return 0;
     return dart::sma_bwd_workspace_bytes(d->batch, d->seqlen, d->nheads, d->dstate, d->chunk);

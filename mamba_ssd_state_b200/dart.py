@@ -34,7 +34,7 @@ EXPORTS = ("dart_ssd_chunk_scan_workspace_bytes", "dart_ssd_chunk_scan", "dart_s
            "dart_sma_impl", "dart_decode_step_noalloc", "dart_sma_decayed_workspace_bytes",
            "dart_sma_forward_decayed", "dart_decode_step_decayed", "dart_decode_memlog_init",
            "dart_decode_step_e4m3", "dart_cache_quantize_e4m3", "dart_sma_backward_workspace_bytes",
-           "dart_sma_backward")
+           "dart_sma_backward", "dart_ssd_scan_backward_workspace_bytes", "dart_ssd_scan_backward")
 
 
 class DartError(RuntimeError):
@@ -70,6 +70,10 @@ def load(path: str = LIBRARY) -> ctypes.CDLL:
     lib.dart_decode_step_decayed.restype = ctypes.c_int
     lib.dart_decode_step_decayed.argtypes = ([D, ctypes.c_int] + [_P] * 7 + [ctypes.c_float] + [_P] * 3
                                              + [ctypes.c_int] + [_P] * 5 + [ctypes.c_size_t, _P])
+    lib.dart_ssd_scan_backward_workspace_bytes.restype = ctypes.c_size_t
+    lib.dart_ssd_scan_backward_workspace_bytes.argtypes = [D]
+    lib.dart_ssd_scan_backward.restype = ctypes.c_int
+    lib.dart_ssd_scan_backward.argtypes = [D, ctypes.c_int] + [_P] * 16 + [ctypes.c_size_t, _P]
     lib.dart_sma_backward_workspace_bytes.restype = ctypes.c_size_t
     lib.dart_sma_backward_workspace_bytes.argtypes = [D]
     lib.dart_sma_backward.restype = ctypes.c_int
@@ -310,6 +314,58 @@ def dart_sma_backward(Q, E, Cm, dH, chunk: int, g: float, dy, *, workspace=None)
                                      float(g), _ptr(dy), _ptr(out["dQ"]), _ptr(out["dE"]), _ptr(out["dCm"]),
                                      _ptr(out["ddH"]), _ptr(out["dg"]), _ptr(workspace), workspace.numel(),
                                      _stream()))
+    return out
+
+
+def dart_ssd_scan_backward(x, dt, A, Bm, Cm, chunk: int, states, dy, ddH=None, init_state=None, *,
+                           workspace=None) -> dict:
+    """Gradients of sum(dy * y_ssd) + sum(ddH * dH) through the scan: a dict
+    of float32 device tensors dx, ddt, dA, dBm, dCm (the scan's part) and,
+    with an initial state, dinit_state.  x/Bm/Cm as given to the forward
+    (dtype), dt/A/init_state float32, states = the forward's boundary states,
+    dy float32 [B,L,H,P], ddH float32 [B,H,C,N,P] or None."""
+    lib = load()
+    dev = _device_of(x, dt, A, Bm, Cm, states, dy)
+    x, Bm, Cm = (_dev(v, dev, x.dtype) for v in (x, Bm, Cm))
+    dt, A, states, dy = (_dev(v, dev, torch.float32) for v in (dt, A, states, dy))
+    ddH = _dev(ddH, dev, torch.float32)
+    init_state = _dev(init_state, dev, torch.float32)
+    Bsz, L, H, P = x.shape
+    N = Bm.shape[-1]
+    C = -(-L // chunk)
+    _shape("states", states, (Bsz, H, C, N, P)); _shape("dy", dy, (Bsz, L, H, P))
+    if ddH is not None:
+        _shape("ddH", ddH, (Bsz, H, C, N, P))
+    dims = Dims(Bsz, L, H, P, N, chunk, 1)
+    out = {"dx": torch.empty((Bsz, L, H, P), device=dev), "ddt": torch.empty((Bsz, L, H), device=dev),
+           "dA": torch.empty((H,), device=dev), "dBm": torch.empty((Bsz, L, N), device=dev),
+           "dCm": torch.empty((Bsz, L, N), device=dev)}
+    if init_state is not None:
+        out["dinit_state"] = torch.empty((Bsz, H, N, P), device=dev)
+    wsb = lib.dart_ssd_scan_backward_workspace_bytes(ctypes.byref(dims))
+    if workspace is None:
+        workspace = torch.empty(max(16, wsb), device=dev, dtype=torch.uint8)
+    with torch.cuda.device(dev):
+        _check(lib.dart_ssd_scan_backward(ctypes.byref(dims), _dtype_code(x.dtype), _ptr(x), _ptr(dt), _ptr(A),
+                                          _ptr(Bm), _ptr(Cm), _ptr(init_state), _ptr(states), _ptr(dy), _ptr(ddH),
+                                          _ptr(out["dx"]), _ptr(out["ddt"]), _ptr(out["dA"]), _ptr(out["dBm"]),
+                                          _ptr(out["dCm"]), _ptr(out.get("dinit_state")), _ptr(workspace),
+                                          workspace.numel(), _stream()))
+    return out
+
+
+def layer_backward(x, dt, A, Bm, Cm, Q, E, chunk: int, g: float, dy, init_state=None) -> dict:
+    """Gradients of sum(dy * y) for the DART layer forward (raw memories):
+    runs the forward scan for its memories and boundary states, the SMA
+    backward, then the scan backward driven by dy and the memory gradients.
+    Returns float32 device tensors dx, ddt, dA, dBm, dCm, dQ, dE, dg (and
+    dinit_state with an initial state)."""
+    y_ssd, dH, states = dart_ssd_chunk_scan(x, dt, A, Bm, Cm, chunk, init_state)
+    sm = dart_sma_backward(Q, E, Cm, dH, chunk, g, dy)
+    sc = dart_ssd_scan_backward(x, dt, A, Bm, Cm, chunk, states, dy, sm["ddH"], init_state)
+    out = dict(sc)
+    out["dCm"] = sc["dCm"] + sm["dCm"]
+    out.update(dQ=sm["dQ"], dE=sm["dE"], dg=sm["dg"])
     return out
 
 

@@ -201,6 +201,20 @@ def test_sma_backward_workspace_and_validation(lib):
              FAKE, 1 << 30, None) == dart.DART_ERR_UNSUPPORTED
 
 
+def test_scan_backward_workspace_and_validation(lib):
+    d = dart.Dims(2, 500, 3, 64, 128, 256, 1)
+    pad = lambda b: (b + 255) // 256 * 256
+    want = 2 * pad(4 * 2 * 3 * 256 * 128 * 64) + 2 * pad(4 * 2 * 500 * 3 * 128) + pad(4 * 2 * 3)
+    assert lib.dart_ssd_scan_backward_workspace_bytes(ctypes.byref(d)) == want
+    f = lib.dart_ssd_scan_backward
+    ok = [FAKE] * 5 + [None, FAKE, FAKE, None] + [FAKE] * 5 + [None, FAKE]
+    assert f(ctypes.byref(d), dart.DART_BF16, *ok[:6], None, *ok[7:], want, None) == dart.DART_ERR_INVALID_ARG
+    assert b"states" in lib.dart_last_error()
+    assert f(ctypes.byref(d), dart.DART_BF16, *ok, want - 1, None) == dart.DART_ERR_INVALID_ARG
+    d.headdim, d.dstate = 32, 32
+    assert f(ctypes.byref(d), dart.DART_BF16, *ok, 1 << 40, None) == dart.DART_ERR_UNSUPPORTED
+
+
 def test_decode_rejects_bad_args(lib):
     d = dart.Dims(4, 0, 2, 64, 128, 256, 1)
     ws = lib.dart_decode_step_workspace_bytes(ctypes.byref(d), dart.DART_BF16, 9)

@@ -61,3 +61,66 @@ def test_sma_backward_deterministic():
     b = dart.dart_sma_backward(*args, 256, 0.5, dy.cuda())
     for k in a:
         assert torch.equal(a[k], b[k]), k
+
+
+# ---------------------------------------------------------------------------
+# scan backward and the whole layer backward
+# ---------------------------------------------------------------------------
+SCAN_CASES = [
+    ((1, 3 * 64 + 17, 2, 16, 16, 64), "f32", True),
+    ((2, 3 * 128 + 40, 2, 64, 64, 128), "f32", False),
+    ((1, 3 * 256, 2, 64, 128, 256), "bf16", False),
+    ((1, 2 * 256 + 77, 3, 64, 128, 256), "bf16", True),
+]
+SCAN_IDS = ["f32_N16_ragged_init", "f32_N64_B2_ragged", "bf16_N128", "bf16_N128_ragged_init"]
+TOL_FWD_INPUTS = {"f32": 1e-4, "bf16": 2e-2}   # bf16: the tensor-core forward's states carry bf16 rounding
+
+
+def _layer_case(shape, dt_name, seed):
+    Bz, L, H, P, N, S = shape
+    inp = synth.layer_inputs(synth.LayerShape(Bz, L, H, P, N, S, dt_name, "loguniform"), seed=seed)
+    r = np.random.default_rng(seed)
+    C = -(-L // S)
+    dy = torch.from_numpy(r.standard_normal((Bz, L, H, P)).astype(np.float32))
+    gdH = torch.from_numpy((r.standard_normal((Bz, H, C, N, P)) * 0.5).astype(np.float32))
+    h0 = torch.from_numpy((r.standard_normal((Bz, H, N, P)) * 0.2).astype(np.float32))
+    return inp, dy, gdH, h0
+
+
+@pytest.mark.parametrize("shape,dt_name,with_init", SCAN_CASES, ids=SCAN_IDS)
+def test_scan_backward_matches_oracle(shape, dt_name, with_init):
+    Bz, L, H, P, N, S = shape
+    inp, dy, gdH, h0 = _layer_case(shape, dt_name, seed=L + 1)
+    h0 = h0 if with_init else None
+    d = {k: inp[k].cuda() for k in ("x", "dt", "A", "Bm", "Cm")}
+    _, _, states = dart.dart_ssd_chunk_scan(d["x"], d["dt"], d["A"], d["Bm"], d["Cm"], S,
+                                            None if h0 is None else h0.cuda())
+    got = dart.dart_ssd_scan_backward(d["x"], d["dt"], d["A"], d["Bm"], d["Cm"], S, states, dy.cuda(), gdH.cuda(),
+                                      None if h0 is None else h0.cuda())
+    dart.dart_sync_status()
+    ref = dart_backward.scan_grads(*(inp[k].double().numpy() for k in ("x", "dt", "A", "Bm", "Cm")), S,
+                                   dy.double().numpy(), gdH.double().numpy(),
+                                   init_state=None if h0 is None else h0.double().numpy())
+    tol = TOL_FWD_INPUTS[dt_name]
+    for k in ("dx", "ddt", "dA", "dBm", "dCm") + (("dinit_state",) if h0 is not None else ()):
+        assert_close(k, got[k], ref[k], tol)
+
+
+@pytest.mark.parametrize("shape,dt_name,with_init", [SCAN_CASES[0], SCAN_CASES[3]], ids=[SCAN_IDS[0], SCAN_IDS[3]])
+def test_layer_backward_matches_oracle(shape, dt_name, with_init):
+    """dart.layer_backward (forward scan, SMA backward, scan backward driven
+    by dy and the memory gradients) against autograd over the whole layer."""
+    Bz, L, H, P, N, S = shape
+    inp, dy, _, h0 = _layer_case(shape, dt_name, seed=L + 2)
+    h0 = h0 if with_init else None
+    g = 0.6
+    keys = ("x", "dt", "A", "Bm", "Cm", "Q", "E")
+    got = dart.layer_backward(*(inp[k].cuda() for k in keys), S, g, dy.cuda(),
+                              None if h0 is None else h0.cuda())
+    dart.dart_sync_status()
+    ref = dart_backward.layer_grads(*(inp[k].double().numpy() for k in keys), S, g, dy.double().numpy(),
+                                    init_state=None if h0 is None else h0.double().numpy())
+    tol = TOL_FWD_INPUTS[dt_name]
+    for k in ("dx", "ddt", "dA", "dBm", "dCm", "dQ", "dE") + (("dinit_state",) if h0 is not None else ()):
+        assert_close(k, got[k], ref[k], tol)
+    assert abs(float(got["dg"][0]) - float(ref["dg"])) <= tol * max(1.0, abs(float(ref["dg"])))
