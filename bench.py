@@ -290,7 +290,7 @@ def e2e_region(args, dist, dart, inp):
     dev = torch.device("cuda", torch.cuda.current_device())
     host = {k: (v.pin_memory() if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
     B, L, H, P, N, S = FWD.batch, FWD.seqlen, FWD.nheads, FWD.headdim, FWD.dstate, FWD.chunk
-    C = L // S
+    C = -(-L // S)   # a partial last chunk counts
     bufs = {"y": torch.empty((B, L, H, P), device=dev, dtype=torch.float32),
             "dH": torch.empty((B, H, C, N, P), device=dev, dtype=torch.bfloat16),
             "states": torch.empty((B, H, C, N, P), device=dev, dtype=torch.float32),
