@@ -388,7 +388,8 @@ dart_status dart_sync_status(void* stream);
 /* Message describing the last failure on the calling host thread ("" if none). */
 const char* dart_last_error(void);
 
-/* ABI version, bumped on any signature change. */
+/* ABI version, bumped on any signature change or addition (2: the decayed-memory,
+ * E4M3-cache and backward entry points). */
 int dart_abi_version(void);
 
 /*

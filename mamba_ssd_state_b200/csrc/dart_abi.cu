@@ -86,7 +86,7 @@ dart_status check_common(const dart_dims* d, dart_dtype dt, bool need_seqlen) {
 
 extern "C" {
 
-int dart_abi_version(void) { return 1; }
+int dart_abi_version(void) { return 2; }
 
 unsigned long long dart_launch_count(void) { return dart::g_launches.load(std::memory_order_relaxed); }
 
