@@ -6,7 +6,7 @@
 #include <stdio.h>
 #include <string.h>
 
-#include "dart_common.cuh"
+#include "dart_backward.cuh"
 
 namespace dart {
 // [0]: status flags; [1]: (kernel id << 8 | wait site) of the first bounded

@@ -1,0 +1,43 @@
+// dart_backward.cuh -- argument blocks and launchers of the backward kernels
+// (sma_bwd.cu, ssd_scan_bwd.cu), used by the C ABI in dart_abi.cu.
+#pragma once
+
+#include "dart_common.cuh"
+
+namespace dart {
+
+struct SmaBwdArgs {
+    int B, L, H, P, N, S;
+    const void* Q; const void* E; const void* Cm; const void* dH;
+    float g; const float* dy;               // dy: [B,L,H,P] gradient of the layer output
+    float* dQ; float* dE; float* dCm; float* ddH; float* dg;   // outputs (fp32)
+    int* status;
+    // workspace views (set by launch_sma_bwd)
+    float* pbuf; float* dsbuf;              // [B,H,L,C] softmax weights and score gradients
+    float* dCh;                             // [B,L,H,N] per-head dC
+    float* gpart;                           // [B,H,tiles] per-tile dg
+};
+
+struct ScanBwdArgs {
+    int B, L, H, P, N, S;
+    const void* x; const float* dt; const float* A; const void* Bm; const void* Cm;
+    const float* init;      // nullable [B,H,N,P] initial state of the forward
+    const float* states;    // [B,H,C,N,P] boundary states written by the forward
+    const float* dy;        // [B,L,H,P] gradient of y_ssd
+    const float* ddH;       // nullable [B,H,C,N,P] gradient of the chunk memories
+    float* dx; float* ddt; float* dA; float* dB; float* dC;   // outputs (fp32)
+    float* dinit;           // nullable [B,H,N,P] output
+    int* status;
+    // workspace views (set by launch_ssd_scan_bwd)
+    float* hist;            // [2][B,H,S,N,P] H_{t-1}, D_{t-1} of the chunk being walked
+    float* dBh; float* dCh; // [B,L,H,N] per-head dB, dC
+    float* dApart;          // [B,H]
+};
+
+size_t sma_bwd_workspace_bytes(int B, int L, int H, int N, int S);
+cudaError_t launch_sma_bwd(SmaBwdArgs a, void* workspace, dart_dtype dt, cudaStream_t st);
+size_t scan_bwd_workspace_bytes(int B, int L, int H, int N, int P, int S);
+bool scan_bwd_supported(int N, int P);
+cudaError_t launch_ssd_scan_bwd(ScanBwdArgs a, void* workspace, dart_dtype dt, cudaStream_t st);
+
+}  // namespace dart

@@ -23,7 +23,7 @@
 //   tiles of dg, in a fixed order (deterministic).
 // Memories are staged in shared memory once per (tile, memory) and shared by
 // the tile's 32 tokens.
-#include "dart_common.cuh"
+#include "dart_backward.cuh"
 
 namespace dart {
 namespace {

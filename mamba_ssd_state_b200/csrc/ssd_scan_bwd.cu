@@ -25,7 +25,7 @@
 // the ddt terms (sums over the whole state) are reduced with warp shuffles and
 // one shared-memory exchange; dB and dC (sums over columns) with shuffles
 // among the lanes of a row, written per head and summed over heads after.
-#include "dart_common.cuh"
+#include "dart_backward.cuh"
 
 namespace dart {
 namespace {
