@@ -26,7 +26,9 @@ pin the restatement to the C oracle's forward and the gradients to central
 finite differences and to closed forms.
 
 Layouts as in ``dart_oracle.c``: x[B,L,H,P] dt[B,L,H] A[H] Bm[B,L,N] Cm[B,L,N]
-Q[B,L,H,N] E[B,L,H,P] y[B,L,H,P] dH[B,H,C,N,P] init_state[B,H,N,P].
+Q[B,L,H,N] E[B,L,H,P] y[B,L,H,P] dH[B,H,C,N,P] init_state[B,H,N,P].  B and C
+may also carry a group axis, Bm/Cm[B,L,G,N] with G dividing H: head h then
+reads group h // (H / G) (Mamba-2 ngroups).
 """
 from __future__ import annotations
 
@@ -37,6 +39,13 @@ import numpy as np
 import torch
 
 _F64 = torch.float64
+
+
+def _bc(M, b, t, h, H):
+    """Row of B or C that head h reads at token t: [N]."""
+    if M.dim() == 3:
+        return M[b, t]
+    return M[b, t, h // (H // M.shape[2])]
 
 
 def _t(a, requires_grad=False):
@@ -63,10 +72,10 @@ def ssd_scan(x, dt, A, Bm, Cm, chunk: int, init_state=None):
                 if t % S == 0:
                     D = torch.zeros(N, P, dtype=_F64)   # a new chunk's own contribution
                 decay = torch.exp(dt[b, t, h] * A[h])
-                inp = dt[b, t, h] * torch.outer(Bm[b, t], x[b, t, h])
+                inp = dt[b, t, h] * torch.outer(_bc(Bm, b, t, h, H), x[b, t, h])
                 Hs = decay * Hs + inp
                 D = decay * D + inp
-                yh.append(Hs.transpose(0, 1) @ Cm[b, t])
+                yh.append(Hs.transpose(0, 1) @ _bc(Cm, b, t, h, H))
                 if t % S == S - 1 or t == L - 1:        # the chunk closes at its last token
                     dHh.append(D)
                     sth.append(Hs)
@@ -103,7 +112,7 @@ def sma(Q, E, Cm, dH, chunk: int, dt=None, A=None):
                     if dt is not None:
                         M = torch.exp(A[h] * dt[b, c * S + S:t + 1, h].sum()) * M
                     key = M @ E[b, t, h]                  # [N]
-                    values.append(Cm[b, t] @ M)           # [P]
+                    values.append(_bc(Cm, b, t, h, H) @ M)  # [P]
                     scores.append((Q[b, t, h] @ key) * inv_sqrt_n)
                 p = torch.softmax(torch.stack(scores), 0)
                 oh.append((p[:, None] * torch.stack(values)).sum(0))

@@ -199,3 +199,33 @@ def test_scan_gradients_match_finite_differences(orc):
             minus[name][idx] -= hstep
             fd = (loss(plus) - loss(minus)) / (2 * hstep)
             assert abs(gr["d" + name][idx] - fd) <= 1e-6 * max(1.0, abs(fd)), (name, idx, gr["d" + name][idx], fd)
+
+
+def test_grouped_B_C_restatement_and_split(orc):
+    """B and C per group of heads (H = 4, G = 2): the restatement equals the C
+    oracle's grouped forward, and the layer gradients equal those of two
+    single-group problems (heads of group g with group g's B and C), with dB
+    and dC landing on the group's slice."""
+    Bz, L, H, P, N, S, G = 1, 18, 4, 3, 4, 8, 2
+    inp = _inputs(41, Bz, L, H, P, N)
+    r = np.random.default_rng(42)
+    f = lambda a: np.asarray(a, np.float32).astype(np.float64)
+    Bg = f(r.standard_normal((Bz, L, G, N)) / np.sqrt(N))
+    Cg = f(r.standard_normal((Bz, L, G, N)) / np.sqrt(N))
+    dy = r.standard_normal((Bz, L, H, P))
+    g = 0.7
+    grouped = dict(inp, Bm=Bg, Cm=Cg)
+    ref = orc.layer_forward(*(grouped[k] for k in KEYS), S, g)
+    full = dart_backward.layer_grads(*(grouped[k] for k in KEYS), S, g, dy)
+    np.testing.assert_allclose(full["y"], ref["y"], rtol=1e-12, atol=1e-12)
+    hg = H // G
+    for gi in range(G):
+        hs = slice(gi * hg, (gi + 1) * hg)
+        part_in = dict(x=inp["x"][:, :, hs], dt=inp["dt"][:, :, hs], A=inp["A"][hs], Bm=Bg[:, :, gi],
+                       Cm=Cg[:, :, gi], Q=inp["Q"][:, :, hs], E=inp["E"][:, :, hs])
+        part = dart_backward.layer_grads(*(part_in[k] for k in KEYS), S, g, dy[:, :, hs])
+        for k in ("dx", "ddt", "dQ", "dE"):
+            np.testing.assert_allclose(full[k][:, :, hs], part[k], rtol=1e-11, atol=1e-12, err_msg=k)
+        np.testing.assert_allclose(full["dA"][hs], part["dA"], rtol=1e-11, atol=1e-12)
+        np.testing.assert_allclose(full["dBm"][:, :, gi], part["dBm"], rtol=1e-11, atol=1e-12)
+        np.testing.assert_allclose(full["dCm"][:, :, gi], part["dCm"], rtol=1e-11, atol=1e-12)

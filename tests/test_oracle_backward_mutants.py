@@ -21,12 +21,13 @@ MUTATIONS = [
      "                    pass\n"),
     ("decay_after_input", "                Hs = decay * Hs + inp\n", "                Hs = decay * (Hs + inp)\n"),
     ("memory_not_decayed", "                D = decay * D + inp\n", "                D = D + inp\n"),
-    ("readout_before_update", "                yh.append(Hs.transpose(0, 1) @ Cm[b, t])\n                if t % S",
-     "                yh.append((Hs - inp).transpose(0, 1) @ Cm[b, t])\n                if t % S"),
+    ("readout_before_update", "                yh.append(Hs.transpose(0, 1) @ _bc(Cm, b, t, h, H))\n",
+     "                yh.append((Hs - inp).transpose(0, 1) @ _bc(Cm, b, t, h, H))\n"),
+    ("group_by_modulo", "    return M[b, t, h // (H // M.shape[2])]\n", "    return M[b, t, h % M.shape[2]]\n"),
     ("scale_by_P", "    inv_sqrt_n = 1.0 / math.sqrt(N)\n", "    inv_sqrt_n = 1.0 / math.sqrt(P)\n"),
     ("mask_off_by_one", "            k = t // S\n", "            k = (t + 1) // S\n"),
-    ("value_read_with_Q", "                    values.append(Cm[b, t] @ M)           # [P]\n",
-     "                    values.append(Q[b, t, h] @ M)         # [P]\n"),
+    ("value_read_with_Q", "                    values.append(_bc(Cm, b, t, h, H) @ M)  # [P]\n",
+     "                    values.append(Q[b, t, h] @ M)  # [P]\n"),
     ("decay_window_from_e", "dt[b, c * S + S:t + 1, h].sum()", "dt[b, c * S + S - 1:t + 1, h].sum()"),
     ("gate_ignored", "    return y_ssd + g * o, y_ssd, o, dH, st\n", "    return y_ssd + o, y_ssd, o, dH, st\n"),
     ("scan_loss_drops_memories", "    loss = (y_ssd * _t(dy)).sum() + (dH * _t(gdH)).sum()\n",
@@ -65,6 +66,16 @@ def _pins_hold(mod, orc) -> bool:
             for name, got in zip(("y", "y_ssd", "o", "dH", "states"), out):
                 if not np.allclose(got.detach().numpy(), ref[name], rtol=1e-10, atol=1e-10):
                     return False
+        # B and C per group of heads (H = 4, G = 2) against the C oracle
+        gin = _inputs(33, 1, 17, 4, 3, 4)
+        rg = np.random.default_rng(34)
+        gin["Bm"] = np.asarray(rg.standard_normal((1, 17, 2, 4)) / 2, np.float32).astype(np.float64)
+        gin["Cm"] = np.asarray(rg.standard_normal((1, 17, 2, 4)) / 2, np.float32).astype(np.float64)
+        gref = orc.layer_forward(*(gin[k] for k in KEYS), S, g)
+        gts = {k: mod._t(v) for k, v in gin.items()}
+        gout = mod.layer_forward(*(gts[k] for k in KEYS), S, g)
+        if not np.allclose(gout[0].detach().numpy(), gref["y"], rtol=1e-10, atol=1e-10):
+            return False
         # layer gradients against finite differences of the C oracle
         gr = mod.layer_grads(*(inp[k] for k in KEYS), S, g, dy, init_state=h0)
 
