@@ -1,31 +1,31 @@
 // ssd_scan_tc.cu -- the SSD chunked scan with retained chunk memories on the
 // 5th-generation tensor cores (bf16 inputs, N = 128, P = 64, S in {128, 256}).
 //
-// Same three stages as the CUDA-core scan (Mamba-2 SSD chunked scan as used by
-// DART: "Transformers are SSMs" SSD view, Eq. (4); Pith review of DART, "What
-// carries the argument" for the retained chunk contribution dH[c]):
+// Mamba-2 SSD chunked scan as used by DART ("Transformers are SSMs" SSD view,
+// Eq. (4); Pith review of DART, "What carries the argument" for the retained
+// chunk contribution dH[c]), in four launches:
 //
-//  chunk_state_tc  one CTA per (b, c, group of heads).  The chunk's B tile
-//      (S x N) is loaded once and shared by every head of the group (B is the
-//      same for all heads, ngroups = 1).  Per head the x tile (S x P) is
-//      scaled in shared memory by w_s = exp(Acum_e - Acum_s) dt_s and
+//  chunk_decay     per (b, h, c): the in-chunk prefix Acum of dt A, Asum[c]
+//      and three per-token decay terms the other kernels bulk-copy.
+//  chunk_state_tc  persistent, one CTA per SM over equal shares of the
+//      (b, c, h) items.  The chunk's B tile (S x N) is loaded once and shared
+//      by the heads that follow (B is the same for all heads, ngroups = 1).
+//      Per head the x tile (S x P) is scaled in shared memory by
+//      w_s = exp(Acum_e - Acum_s) dt_s and
 //        dH[c] = B^T (w o x)      (M = N = 128, N_mma = P = 64, K = S)
-//      runs on the tensor core.  Writes dH (bf16), its fp32 value into
-//      `states` (consumed in place by state_pass) and Asum[c] = Acum_e.
-//  state_pass_tc   states[c] = exp(Asum[c]) states[c-1] + dH[c] in place,
-//      sequential in c; also writes the bf16 state entering each chunk,
-//      hin[c] = bf16(states[c-1]) (hin[0] = init_state or 0), the operand of
-//      the inter-chunk output product.
-//  chunk_output_tc one CTA per (b, c, half of the chunk's rows, group of
-//      heads).  G = C B^T for the half's rows (128 x KS, KS = 128 (half+1))
-//      is computed once into TMEM and shared by the heads of the group.  Per
-//      head the worker warps build P[t,s] = G[t,s] exp(Acum_t - Acum_s)
-//      (s <= t, else 0) times dt_s in bf16 straight from TMEM into shared
-//      memory (dt of the source token is folded into P, so the x tile is used
-//      as loaded), and the tensor core computes
-//        Y_diag = P x                 (K = KS)
-//        Y_off  = C hin[c]            (K = N)
-//      y = Y_diag + exp(Acum_t) Y_off.
+//      runs on the tensor core; dH (bf16) leaves by TMA tensor store.
+//  state_pass_tc   states[c] = exp(Asum[c]) states[c-1] + dH[c] from the
+//      stored bf16 memories, sequential in c; also writes the bf16 state
+//      entering each chunk, hin[c] = bf16(states[c-1]) (hin[0] = init_state
+//      or 0), the operand of the inter-chunk output product.
+//  chunk_output    y = Y_diag + exp(Acum_t) Y_off with
+//        G = C B^T,  P[t,s] = G[t,s] exp(Acum_t - Acum_s) dt_s (s <= t),
+//        Y_diag = P x,  Y_off = C hin[c].
+//      Persistent, one CTA per SM over cost-balanced ranges of the
+//      (b, c, 128-row half, h) items.  G is computed once per (b, c, half)
+//      into TMEM and shared by the heads; the P builders read it from TMEM
+//      and write P (bf16) in 64-column panels, each handed to the MMA by its
+//      own barrier pair.
 //
 // Decay factors: exp(Acum_t - Acum_s) = exp(Acum_t - Acum_r) exp(Acum_r -
 // Acum_s) with r the first token of the 32-token column block holding s; both
@@ -54,8 +54,7 @@ struct ScanTcParams {
     CUtensorMap tmap_c;    // Cm as (N, B*L),    box (64, 128)
     CUtensorMap tmap_hin;  // hin as (P, B*H*C*N), box (64, 128)
     CUtensorMap tmap_dh;   // dH as (P, B*H*C*N) bf16, box (64, 128): chunk_state's store
-    CUtensorMap tmap_st;   // states as (P, B*H*C*N) fp32, box (32, 128): chunk_state's store
-    CUtensorMap tmap_y;    // y as (P, H, B*L) fp32, box (32, 1, 128): chunk_output's store
+    CUtensorMap tmap_y;    // y as (P, H, L, B) fp32, box (32, 1, 128, 1): chunk_output's store
     const float* dt;
     const float* A;
     const float* init_state;
@@ -133,10 +132,13 @@ __global__ void __launch_bounds__(256) chunk_decay_kernel(const __grid_constant_
 // chunk_state_tc
 // ===========================================================================
 namespace cs {
-constexpr int kThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 workers
-enum Bar { B_FULL = 0, B_FREE = 1, X_FULL0 = 2, X_EMPTY0 = X_FULL0 + 2, W_READY0 = X_EMPTY0 + 2,
-           ACC_FULL0 = W_READY0 + 2, ACC_EMPTY0 = ACC_FULL0 + 2, NUM_BARS = ACC_EMPTY0 + 2 };
-static_assert(NUM_BARS == 12, "chunk_state barrier slots");
+// warp 0 TMA, warp 1 MMA, warps 2-5 scale the x tiles, warps 6-9 write dH
+constexpr int kThreads = 320;
+constexpr int kScalers = 128, kEpi = 128;
+constexpr int kMaxStages = 6;
+enum Bar { B_FULL = 0, B_FREE = 1, X_FULL0 = 2, X_EMPTY0 = X_FULL0 + kMaxStages, W_READY0 = X_EMPTY0 + kMaxStages,
+           ACC_FULL0 = W_READY0 + kMaxStages, ACC_EMPTY0 = ACC_FULL0 + 2, NUM_BARS = ACC_EMPTY0 + 2 };
+static_assert(NUM_BARS == 24, "chunk_state barrier slots");
 
 // Work items (b, c, h) in that order, h fastest; consecutive items of one
 // (b, c) share the chunk's B tile.  CTA r of G takes items
@@ -153,22 +155,28 @@ __device__ __forceinline__ Item cs_item(const ScanTcParams& p, int j) {
     return it;
 }
 
+// x tiles (S rows x 128 B) move through a ring of kStages buffers: loaded by
+// TMA, scaled in place (row s times wst_s) by the scaler warps, consumed by
+// the MMA.  The finished dH (bf16, 128 rows x 128 B) leaves through one of
+// two swizzled staging tiles by TMA tensor store.
 template <int S>
 struct Layout {
+    static constexpr int kStages = S == 256 ? 3 : 6;
+    static_assert(kStages <= kMaxStages, "x ring depth");
     static constexpr uint32_t kOffB = 0;                        // 2 panels x S rows
-    static constexpr uint32_t kOffX = 2 * S * kRowBytes;        // 2 buffers x S rows
+    static constexpr uint32_t kOffX = 2 * S * kRowBytes;        // kStages buffers x S rows
     static constexpr uint32_t kXBytes = S * kRowBytes;
-    static constexpr uint32_t kOffF = kOffX + 2 * kXBytes;      // 2 buffers x wst[S] floats
-    // output staging (128-byte swizzle, as the store tensor maps expect):
-    // dH tile 128 rows x 128 B, then the states tile as two 128 x 128 B panels
-    static constexpr uint32_t kOffOut = (kOffF + 2 * S * 4 + 1023) & ~1023u;
-    static constexpr uint32_t kOffBar = kOffOut + 3 * kBox;
+    static constexpr uint32_t kOffF = kOffX + kStages * kXBytes; // kStages buffers x wst[S] floats
+    static constexpr uint32_t kOffOut = (kOffF + kStages * S * 4 + 1023) & ~1023u;   // 2 dH staging tiles
+    static constexpr uint32_t kOffBar = kOffOut + 2 * kBox;
     static constexpr uint32_t kBytes = kOffBar + NUM_BARS * 8 + 16 + 1024;
+    static_assert(kBytes <= 232448, "chunk_state shared memory");
 };
 
 template <int S>
 __global__ void __launch_bounds__(kThreads, 1) chunk_state_tc_kernel(const __grid_constant__ ScanTcParams p) {
     using Ly = Layout<S>;
+    constexpr int kSt = Ly::kStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
@@ -186,12 +194,14 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_state_tc_kernel(const __gri
     if (threadIdx.x == 0) {
         mbar_init(bar(B_FULL), 1);
         mbar_init(bar(B_FREE), 1);
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < kSt; ++s) {
             mbar_init(bar(X_FULL0 + s), 1);
             mbar_init(bar(X_EMPTY0 + s), 1);
-            mbar_init(bar(W_READY0 + s), 4);
-            mbar_init(bar(ACC_FULL0 + s), 1);
-            mbar_init(bar(ACC_EMPTY0 + s), 4);
+            mbar_init(bar(W_READY0 + s), kScalers / 32);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(bar(ACC_FULL0 + a), 1);
+            mbar_init(bar(ACC_EMPTY0 + a), kEpi / 32);
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -207,7 +217,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_state_tc_kernel(const __gri
 
     const WaitCtx wc{abort_flag, p.status, 2};
     if (warp == 0) {
-        // TMA: the whole warp walks the heads, lane 0 issues
+        // TMA: the whole warp walks the items, lane 0 issues
         if (lane == 0) {
             tma_prefetch_desc(&p.tmap_x);
             tma_prefetch_desc(&p.tmap_b);
@@ -228,8 +238,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_state_tc_kernel(const __gri
                 }
                 ++b_loads;
             }
-            const int xs = i & 1;
-            const uint32_t ph = (uint32_t)(i >> 1) & 1u;
+            const int xs = i % kSt;
+            const uint32_t ph = (uint32_t)(i / kSt) & 1u;
             if (!mbar_wait_warp(bar(X_EMPTY0 + xs), ph ^ 1u, wc, 1)) break;
             if (lane == 0) {
                 mbar_expect_tx(bar(X_FULL0 + xs), Ly::kXBytes + S * 4);
@@ -255,10 +265,11 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_state_tc_kernel(const __gri
             }
             // the last item on this B tile releases it after its MMAs
             const bool last_on_b = i + 1 == n_items || it.h == p.H - 1;
-            const int xs = i & 1, a = i & 1;
-            const uint32_t ph = (uint32_t)(i >> 1) & 1u;
+            const int xs = i % kSt, a = i & 1;
+            const uint32_t ph = (uint32_t)(i / kSt) & 1u;
+            const uint32_t aph = (uint32_t)(i >> 1) & 1u;
             if (!(ok = mbar_wait_warp(bar(W_READY0 + xs), ph, wc, 3))) break;
-            if (!(ok = mbar_wait_warp(bar(ACC_EMPTY0 + a), ph ^ 1u, wc, 4))) break;
+            if (!(ok = mbar_wait_warp(bar(ACC_EMPTY0 + a), aph ^ 1u, wc, 4))) break;
             tc_fence_after();
             if (lane == 0) {
                 const uint32_t xbase = sbase + Ly::kOffX + (uint32_t)xs * Ly::kXBytes;
@@ -274,25 +285,47 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_state_tc_kernel(const __gri
             }
             __syncwarp();
         }
-    } else {
-        // ---------------------------------------------------------- workers
-        // Every worker warp executes the same sequence of named barriers for
-        // every head, also after a failed wait (it then skips the work), so
-        // no warp can be left waiting at a barrier the others never reach.
+    } else if (warp < 2 + kScalers / 32) {
+        // ---------------------------------------------------------- scalers
+        // row s of the x tile times wst_s, in place (bf16 -> fp32 -> bf16)
         const int wi = threadIdx.x - 64;            // 0..127
+        bool ok = true;
+        for (int i = 0; i < n_items && ok; ++i) {
+            const int xs = i % kSt;
+            const uint32_t ph = (uint32_t)(i / kSt) & 1u;
+            if (!(ok = mbar_wait_warp(bar(X_FULL0 + xs), ph, wc, 6))) break;
+            uint8_t* xb = smem + Ly::kOffX + (uint32_t)xs * Ly::kXBytes;
+            const float* w = wst_s + xs * S;
+#pragma unroll 4
+            for (int k = wi; k < S * 8; k += kScalers) {
+                uint4* ptr = reinterpret_cast<uint4*>(xb + (size_t)k * 16);
+                float f[8];
+                Vec16<__nv_bfloat16>::unpack(*ptr, f);
+                const float ws = w[k >> 3];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) f[j] *= ws;
+                Vec16<__nv_bfloat16>::store(reinterpret_cast<__nv_bfloat16*>(ptr), f);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(W_READY0 + xs));
+        }
+    } else {
+        // --------------------------------------------------------- epilogue
+        // The four warps run every item's two named barriers whether or not
+        // their own waits succeeded (they then skip the work), so none of
+        // them can be left at a barrier the others never reach.
+        const int wi = threadIdx.x - 64 - kScalers;  // 0..127
         const int quad = warp & 3;
         const int nrow = quad * 32 + lane;          // TMEM lane = state row n
         const uint32_t t_lane = tmem + ((uint32_t)(quad * 32) << 16);
-        // The four worker warps run every epilogue's two named barriers
-        // whether or not their own waits succeeded (they then skip the work),
-        // so none of them can be left at a barrier the others never reach.
-        uint8_t* out_s = smem + Ly::kOffOut;
-        auto epilogue = [&](int i, bool live) -> bool {
+        bool ok = true;
+        for (int i = 0; i < n_items; ++i) {
             const int a = i & 1;
-            const uint32_t ph = (uint32_t)(i >> 1) & 1u;
-            live = live && mbar_wait_warp(bar(ACC_FULL0 + a), ph, wc, 5);
+            const uint32_t aph = (uint32_t)(i >> 1) & 1u;
+            if (ok) ok = mbar_wait_warp(bar(ACC_FULL0 + a), aph, wc, 5);
             float v[kP];
-            if (live) {
+            if (ok) {
                 tc_fence_after();
                 tmem_ld_32x32b_x32(t_lane + (uint32_t)a * 64, v);
                 tmem_ld_32x32b_x32(t_lane + (uint32_t)a * 64 + 32, v + 32);
@@ -301,59 +334,27 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_state_tc_kernel(const __gri
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(ACC_EMPTY0 + a));
             }
-            if (wi == 0) bulk_wait_read<0>();  // the previous head's tiles have left the staging
-            named_bar_sync(1, 128);
-            if (live) {
+            // staging tile i & 1 was last used by item i - 2: its store must
+            // have finished reading it
+            uint8_t* out_s = smem + Ly::kOffOut + (uint32_t)(i & 1) * kBox;
+            if (wi == 0) bulk_wait_read<1>();
+            named_bar_sync(1, kEpi);
+            if (ok) {
                 // row nrow, 16-byte chunk j at position j ^ (nrow & 7) of its 128-byte row
                 uint8_t* drow = out_s + (uint32_t)nrow * kRowBytes;
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
+                for (int j = 0; j < 8; ++j)
                     Vec16<__nv_bfloat16>::store(reinterpret_cast<__nv_bfloat16*>(drow + ((j ^ (nrow & 7)) << 4)), v + 8 * j);
-                }
-#pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    uint8_t* srow = out_s + (uint32_t)(1 + (j >> 3)) * kBox + (uint32_t)nrow * kRowBytes;
-                    *reinterpret_cast<float4*>(srow + (((j & 7) ^ (nrow & 7)) << 4)) =
-                        make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-                }
             }
             fence_proxy_async_smem();
-            named_bar_sync(1, 128);
+            named_bar_sync(1, kEpi);
             if (wi == 0 && !*abort_flag) {
                 const Item it = cs_item(p, j0 + i);
                 const int row = (((it.b * p.H + it.h) * p.C + it.c) * kN);
                 tma_store_2d(&p.tmap_dh, smem_u32(out_s), 0, row);
-                tma_store_2d(&p.tmap_st, smem_u32(out_s + kBox), 0, row);
-                tma_store_2d(&p.tmap_st, smem_u32(out_s + 2 * kBox), 32, row);
                 bulk_commit();
             }
-            return live;
-        };
-        bool ok = true;
-        for (int i = 0; i < n_items; ++i) {
-            // scale the x tile in place: row s of the panel times wst_s
-            const int xs = i & 1;
-            const uint32_t ph = (uint32_t)(i >> 1) & 1u;
-            if (ok) ok = mbar_wait_warp(bar(X_FULL0 + xs), ph, wc, 6);
-            if (ok) {
-                uint8_t* xb = smem + Ly::kOffX + (uint32_t)xs * Ly::kXBytes;
-                const float* w = wst_s + xs * S;
-                for (int k = wi; k < S * 8; k += 128) {
-                    uint4* ptr = reinterpret_cast<uint4*>(xb + (size_t)k * 16);
-                    float f[8];
-                    Vec16<__nv_bfloat16>::unpack(*ptr, f);
-                    const float ws = w[k >> 3];
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) f[j] *= ws;
-                    Vec16<__nv_bfloat16>::store(reinterpret_cast<__nv_bfloat16*>(ptr), f);
-                }
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar(W_READY0 + xs));
-            }
-            if (i > 0) ok = epilogue(i - 1, ok);
         }
-        if (n_items > 0) epilogue(n_items - 1, ok);
         if (wi == 0) bulk_wait<0>();  // stores complete before the CTA's shared memory goes away
     }
 
@@ -369,28 +370,48 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_state_tc_kernel(const __gri
 // ===========================================================================
 // state_pass_tc (CUDA cores; memory-bound)
 // ===========================================================================
+// states[c] = exp(Asum[c]) states[c-1] + dH[c] from the bf16 chunk memories
+// chunk_state wrote, sequential in c, and hin[c] = bf16(states[c-1]).  Each
+// thread owns 4 consecutive elements of one (b, h) state; the memories of the
+// next kPre chunks are in flight while the current one is folded in, so the
+// loads never wait on the dependent chain of FMAs.
+constexpr int kPassPre = 8;
 __global__ void __launch_bounds__(256) state_pass_tc_kernel(const __grid_constant__ ScanTcParams p) {
     constexpr int NP = kN * kP;
     const int h = blockIdx.y, b = blockIdx.z;
     const int e4 = (blockIdx.x * blockDim.x + threadIdx.x) * 4;  // 4 consecutive elements
     if (e4 >= NP) return;
     const size_t bh = (size_t)b * p.H + h;
+    const int C = p.C;
     float4 prev = p.init_state ? *reinterpret_cast<const float4*>(p.init_state + bh * NP + e4)
                                : make_float4(0.f, 0.f, 0.f, 0.f);
-    float* st = p.states + bh * (size_t)p.C * NP + e4;
-    __nv_bfloat16* hin = p.hin + bh * (size_t)p.C * NP + e4;
-    const float* asum = p.asum + bh * p.C;
-    for (int c = 0; c < p.C; ++c) {
-        __nv_bfloat162 lo = __floats2bfloat162_rn(prev.x, prev.y), hi = __floats2bfloat162_rn(prev.z, prev.w);
-        uint2 pk;
-        pk.x = *reinterpret_cast<uint32_t*>(&lo);
-        pk.y = *reinterpret_cast<uint32_t*>(&hi);
-        *reinterpret_cast<uint2*>(hin + (size_t)c * NP) = pk;
-        const float dec = expf(asum[c]);
-        const float4 d = *reinterpret_cast<const float4*>(st + (size_t)c * NP);
-        prev = make_float4(fmaf(dec, prev.x, d.x), fmaf(dec, prev.y, d.y), fmaf(dec, prev.z, d.z),
-                           fmaf(dec, prev.w, d.w));
-        *reinterpret_cast<float4*>(st + (size_t)c * NP) = prev;
+    float* st = p.states + bh * (size_t)C * NP + e4;
+    __nv_bfloat16* hin = p.hin + bh * (size_t)C * NP + e4;
+    const uint2* dh = reinterpret_cast<const uint2*>(p.dH + bh * (size_t)C * NP + e4);
+    const float* asum = p.asum + bh * C;
+    uint2 pre[kPassPre];
+#pragma unroll
+    for (int q = 0; q < kPassPre; ++q) pre[q] = q < C ? __ldg(dh + (size_t)q * (NP / 4)) : make_uint2(0u, 0u);
+    for (int c0 = 0; c0 < C; c0 += kPassPre) {
+#pragma unroll
+        for (int q = 0; q < kPassPre; ++q) {
+            const int c = c0 + q;
+            if (c < C) {
+                const uint2 d = pre[q];
+                if (c + kPassPre < C) pre[q] = __ldg(dh + (size_t)(c + kPassPre) * (NP / 4));
+                __nv_bfloat162 lo = __floats2bfloat162_rn(prev.x, prev.y), hi = __floats2bfloat162_rn(prev.z, prev.w);
+                uint2 pk;
+                pk.x = *reinterpret_cast<uint32_t*>(&lo);
+                pk.y = *reinterpret_cast<uint32_t*>(&hi);
+                *reinterpret_cast<uint2*>(hin + (size_t)c * NP) = pk;
+                const float dec = expf(__ldg(asum + c));
+                prev = make_float4(fmaf(dec, prev.x, __uint_as_float(d.x << 16)),
+                                   fmaf(dec, prev.y, __uint_as_float(d.x & 0xffff0000u)),
+                                   fmaf(dec, prev.z, __uint_as_float(d.y << 16)),
+                                   fmaf(dec, prev.w, __uint_as_float(d.y & 0xffff0000u)));
+                *reinterpret_cast<float4*>(st + (size_t)c * NP) = prev;
+            }
+        }
     }
 }
 
@@ -804,12 +825,6 @@ bool make_maps(const ScanArgs& a, ScanTcParams& p) {
         if (!encode_tile_map_bf16(&p.tmap_dh, 2, a.dH, dims, strides, box)) return false;
     }
     {
-        const uint64_t dims[2] = {(uint64_t)kP, (uint64_t)a.B * a.H * C * kN};
-        const uint64_t strides[1] = {(uint64_t)kP * 4};
-        const uint32_t box[2] = {32, 128};
-        if (!encode_tile_map_f32(&p.tmap_st, 2, a.states, dims, strides, box)) return false;
-    }
-    {
         const uint64_t dims[4] = {(uint64_t)kP, (uint64_t)a.H, (uint64_t)a.L, (uint64_t)a.B};
         const uint64_t strides[3] = {(uint64_t)kP * 4, (uint64_t)a.H * kP * 4, (uint64_t)a.L * a.H * kP * 4};
         const uint32_t box[4] = {32, 1, 128, 1};
@@ -880,9 +895,10 @@ cudaError_t launch_ssd_scan_tc(const ScanArgs& a, cudaStream_t st) {
     // 3. outputs
     {
         // persistent: one CTA per SM, contiguous ranges of the (b, c, half, h)
-        // items with equal estimated work.  An item of the second half (256
-        // source tokens) costs about 4/3 of one of the first; a group change
-        // (C and B rows, G) about as much as one item.
+        // items with equal estimated work.  Building P bounds an item, and on
+        // the busiest TMEM lane quadrant an item of the second half (256
+        // source tokens) has twice the blocks of one of the first; a group
+        // change (C and B rows, G) costs about one first-half item.
         const int sms = sm_count();
         if (sms <= 0) return cudaErrorInvalidDevice;
         const int R = a.S / 128;
@@ -891,7 +907,7 @@ cudaError_t launch_ssd_scan_tc(const ScanArgs& a, cudaStream_t st) {
         if (items < grid) grid = items;
         auto cost = [&](int j) {
             const int half = (j / a.H) % R;
-            return (half == 0 ? 3 : 4) + (j % a.H == 0 ? 3 : 0);
+            return (half == 0 ? 2 : 4) + (j % a.H == 0 ? 2 : 0);
         };
         long long total = 0;
         for (int j = 0; j < items; ++j) total += cost(j);
