@@ -64,6 +64,9 @@ def parse():
                    help="skip the forward with decayed memories (dart_sma_forward_decayed)")
     p.add_argument("--no-e4m3", action="store_true", help="skip the decode with an E4M3 cache")
     p.add_argument("--decode-steps", type=int, default=DEC.nsteps)
+    p.add_argument("--no-configs", action="store_true",
+                   help="skip the other forward workloads (B=4, L=2048 and B=1, L=65536)")
+    p.add_argument("--no-backward", action="store_true", help="skip the backward region")
     p.add_argument("--reference-heads", type=int, default=0,
                    help="heads per reference-arm step (default: one per host core, at most 32)")
     return p.parse_args()
@@ -282,6 +285,72 @@ def forward_region(args, dist, dart, shape=FWD, decayed=False):
     sma_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
     return {"ms_total": ms, "scan_ms": scan_ms, "sma_ms": sma_ms, "launches": n1 - n0, "clocks": clk,
             "inputs": inp}
+
+
+def backward_region(args, dist, dart, shape=FWD):
+    """The training pass of the layer at the headline shape: SMA backward
+    (dQ, dE, dC, memory and gate gradients) and scan backward (dx, ddt, dA,
+    dB, dC) from the forward's memories and boundary states, timed per call
+    with CUDA events.  Both run on CUDA cores."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    inp = synth.layer_inputs(shape, seed=dist.rank)
+    d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    S = shape.chunk
+    y, dH, states = dart.dart_ssd_chunk_scan(d["x"], d["dt"], d["A"], d["Bm"], d["Cm"], S)
+    g = torch.Generator(device="cpu").manual_seed(7 + dist.rank)
+    dy = torch.randn(y.shape, generator=g).to(dev)
+    B, L, H, P, N = shape.batch, shape.seqlen, shape.nheads, shape.headdim, shape.dstate
+    sma_ws = torch.empty(max(16, dart.sma_backward_workspace_bytes(B, L, H, P, N, S)), device=dev,
+                         dtype=torch.uint8)
+    scan_ws = torch.empty(max(16, dart.scan_backward_workspace_bytes(B, L, H, P, N, S)), device=dev,
+                          dtype=torch.uint8)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        sm = dart.dart_sma_backward(d["Q"], d["E"], d["Cm"], dH, S, d["g"], dy, workspace=sma_ws)
+        if ev:
+            ev[1].record(stream)
+        dart.dart_ssd_scan_backward(d["x"], d["dt"], d["A"], d["Bm"], d["Cm"], S, states, dy, sm["ddH"],
+                                    dCm_add=sm["dCm"], workspace=scan_ws)
+        if ev:
+            ev[2].record(stream)
+
+    warm, steps = max(1, min(args.warmup, 2)), max(1, min(args.steps, 3))
+    for _ in range(warm):
+        step()
+    dart.dart_sync_status()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    dist.barrier()
+    torch.cuda.synchronize()
+    n0 = dart.launch_count()
+    for i in range(steps):
+        step(evs[i])
+    torch.cuda.synchronize()
+    n1 = dart.launch_count()
+    dist.barrier()
+    dart.dart_sync_status()
+    sma_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    scan_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    ms = dist.max(sma_ms + scan_ms)
+    # algorithmic work of the SMA backward (CUDA cores): per valid (t, c) pair
+    # and head, 4 N P to recompute U = Q dH and V = C dH, 5 N P for the row
+    # gradients (dQ, dE, dC and the score gradient) and 4 N P for the memory
+    # gradient sum_t ds Q E^T + p C do^T
+    pairs = sum(min(S, L - k * S) * k for k in range(shape.nchunks)) * B * H
+    sma_flop = 13.0 * N * P * pairs
+    fp32_peak = SMS * FP32_LANES_PER_SM * 2 * 1965e6 / 1e12
+    return {"value": dist.world * B * L / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms, "steps": steps,
+            "warmup": warm, "sma_backward_ms": sma_ms, "scan_backward_ms": scan_ms, "launches": n1 - n0,
+            "sma_backward_roofline": {"bound": "alu", "achieved": sma_flop / (sma_ms / 1e3) / 1e12,
+                                      "peak": fp32_peak, "unit": "TFLOP/s",
+                                      "frac": sma_flop / (sma_ms / 1e3) / 1e12 / fp32_peak,
+                                      "flop_per_launch": sma_flop,
+                                      "peak_source": "fp32 FMA: 148 SMs x 128 lanes x 2 flop x 1965 MHz"},
+            "config": {"workload": "dart_layer_bwd_L8k", "batch": B, "seqlen": L, "nheads": H, "headdim": P,
+                       "dstate": N, "chunk": S},
+            "path": "dart_sma_backward + dart_ssd_scan_backward (CUDA cores) from the forward's memories"}
 
 
 def e2e_region(args, dist, dart, inp):
@@ -523,8 +592,11 @@ def main():
             roof = {"bound": "alu", "achieved": sma_tflops, "peak": alu_peak, "unit": "TFLOP/s",
                     "frac": sma_tflops / alu_peak}
             peak_note = "fp32 FMA peak: 148 SMs x 128 lanes x 2 flop x sm_max_mhz"
-        roof.update({"traffic": captured_traffic(impl), "traffic_unit": "bytes per launch", "kernel": impl,
+        roof.update({"traffic": captured_traffic(impl), "traffic_unit": "bytes per launch",
+                     "kernel": f"{impl} (the dominant kernel, state-memory attention alone; "
+                               "the whole layer is under layer_roofline)",
                      "flop_per_launch": f_sma, "peak_source": peak_note})
+        layer_tflops = (f_sma + f_ssd) / (ms / args.steps / 1e3) / 1e12
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": dist.world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
@@ -536,6 +608,12 @@ def main():
             "gpu_launches": fwd["launches"],
             "clocks": fwd["clocks"],
             "roofline": roof,
+            "layer_roofline": {"bound": "tensor", "achieved": layer_tflops, "peak": peaks["bf16_tflops"],
+                               "unit": "TFLOP/s", "frac": layer_tflops / peaks["bf16_tflops"],
+                               "flop_per_step": f_sma + f_ssd,
+                               "what": "scan + state-memory attention per step (all algorithmic flops) "
+                                       "over the measured dense bf16 peak",
+                               "peak_source": peak_note},
             "fwd_breakdown": {"scan_ms": fwd["scan_ms"], "sma_ms": fwd["sma_ms"],
                               "sma_gflop": f_sma / 1e9, "ssd_gflop": f_ssd / 1e9,
                               "layer_tflops": (f_sma + f_ssd) / (ms / args.steps / 1e3) / 1e12,
@@ -567,6 +645,35 @@ def main():
                 "config": {"workload": "dart_layer_fwd_L8k_decayed_memories", "batch": FWD.batch,
                            "seqlen": FWD.seqlen, "nheads": FWD.nheads, "chunk": FWD.chunk}}
             line["gpu_launches"] += dec_f["launches"]
+        if not args.no_configs:
+            # the other forward workloads at their own sizes: the 370M layer shape
+            # and the long-context one (256 chunk memories per head)
+            line["configs"] = {}
+            sub = argparse.Namespace(**vars(args))
+            sub.warmup, sub.steps = max(3, min(args.warmup, 3)), max(1, min(args.steps, 5))
+            for name, shp in (("layer_L2k", synth.LAYER_L2K), ("long_L64k", synth.LONG_L64K)):
+                r = forward_region(sub, dist, dart, shp)
+                rms = dist.max(r["ms_total"])
+                fs, fd = sma_flops(shp), ssd_flops(shp)
+                lt = (fs + fd) / (rms / sub.steps / 1e3) / 1e12
+                st = fs / (r["sma_ms"] / 1e3) / 1e12
+                line["configs"][name] = {
+                    "value": dist.world * shp.batch * shp.seqlen * sub.steps / (rms / 1e3), "unit": "tokens/s",
+                    "ms_per_step": rms / sub.steps, "steps": sub.steps, "warmup": sub.warmup,
+                    "scan_ms": r["scan_ms"], "sma_ms": r["sma_ms"], "sma_gflop": fs / 1e9, "ssd_gflop": fd / 1e9,
+                    "roofline": {"bound": "tensor", "kernel": "sma_tcgen05", "achieved": st,
+                                 "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                                 "frac": st / peaks["bf16_tflops"]},
+                    "layer_tflops": lt, "layer_frac_bf16_peak": lt / peaks["bf16_tflops"],
+                    "config": {"workload": f"dart_layer_fwd_{name}", "batch": shp.batch, "seqlen": shp.seqlen,
+                               "nheads": shp.nheads, "headdim": shp.headdim, "dstate": shp.dstate,
+                               "chunk": shp.chunk}}
+                line["gpu_launches"] += r["launches"]
+                del r
+        if not args.no_backward:
+            bwd = backward_region(args, dist, dart)
+            line["backward"] = bwd
+            line["gpu_launches"] += bwd.pop("launches")
         if not args.no_e2e:
             line["e2e"] = e2e_region(args, dist, dart, fwd["inputs"])
         if not args.no_decode:

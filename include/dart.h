@@ -14,8 +14,9 @@
  * Conventions shared by every call
  * --------------------------------
  * - Notation: B batch, L sequence length, H heads, P head dimension (value
- *   axis), N state size (key axis), S chunk size, C = L / S chunks.  B and C
- *   projections are shared by all heads (ngroups = 1).
+ *   axis), N state size (key axis), S chunk size, C = ceil(L / S) chunks (a
+ *   partial last chunk counts).  B and C projections are shared by all heads
+ *   (ngroups = 1).
  * - Every tensor is dense, row-major (last index fastest), on the CUDA device
  *   that is current for the calling thread, and 16-byte aligned.  Layouts:
  *     x[B,L,H,P]  dt[B,L,H]  A[H]  Bm[B,L,N]  Cm[B,L,N]  Q[B,L,H,N]
@@ -25,8 +26,10 @@
  *   (__nv_bfloat16).  dt, A, y, states, the decode state and dH_cur are
  *   always float.  Accumulation is always float.
  * - Ownership: the caller allocates and owns every buffer, including the
- *   optional workspace; the library keeps no device memory of its own apart
- *   from one status word per device.
+ *   workspaces.  The library's own device memory is a status word per device
+ *   and the fixed 16 MiB scratch array of dart_decode_step_noalloc; both are
+ *   statically sized, exist on every device where the library's module is
+ *   loaded, and live until the process exits.
  * - Execution: calls enqueue kernels on `stream` (a cudaStream_t; NULL is the
  *   legacy default stream) and return without synchronising.  Arguments are
  *   validated on the host before anything is enqueued; a rejected call
@@ -186,8 +189,10 @@ size_t dart_ssd_scan_backward_workspace_bytes(const dart_dims* dims);
  *   states: float [B,H,C,N,P] the forward's boundary states;
  *   dy: float [B,L,H,P]; ddH: nullable float [B,H,C,N,P] (NULL = zero), e.g.
  *   dart_sma_backward's memory gradient;
- *   dx float [B,L,H,P], ddt float [B,L,H], dA float [H], dBm, dCm float [B,L,N]
- *   (dCm is the scan's part: add dart_sma_backward's for the layer);
+ *   dCm_add: nullable float [B,L,N], added to dCm (NULL = nothing); passing
+ *   dart_sma_backward's dCm gives the layer's C gradient.  It may be dCm
+ *   itself (each element is read before it is written);
+ *   dx float [B,L,H,P], ddt float [B,L,H], dA float [H], dBm, dCm float [B,L,N];
  *   dinit_state: nullable float [B,H,N,P].
  * CUDA cores, one CTA per (b, h); sums in a fixed order (deterministic).
  * Compiled for (N, P) = (128, 64), (64, 64), (16, 16).
@@ -196,6 +201,7 @@ dart_status dart_ssd_scan_backward(const dart_dims* dims, dart_dtype dtype,
                                    const void* x, const float* dt, const float* A,
                                    const void* Bm, const void* Cm, const float* init_state,
                                    const float* states, const float* dy, const float* ddH,
+                                   const float* dCm_add,
                                    float* dx, float* ddt, float* dA, float* dBm, float* dCm,
                                    float* dinit_state, void* workspace, size_t workspace_bytes,
                                    void* stream);
@@ -235,7 +241,9 @@ dart_status dart_sma_backward(const dart_dims* dims, dart_dtype dtype,
 
 /*
  * Workspace for dart_decode_step: per (sequence, head, split) partial softmax
- * statistics and partial outputs.  Pass at least this many bytes.
+ * statistics and partial outputs.  Pass at least this many bytes.  Every
+ * decode entry takes 1 <= cmax <= 2^20 (memories per sequence) and rejects
+ * other values with DART_ERR_INVALID_ARG; this query returns 0 for them.
  */
 size_t dart_decode_step_workspace_bytes(const dart_dims* dims, dart_dtype dtype, int cmax);
 

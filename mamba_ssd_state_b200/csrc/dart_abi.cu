@@ -22,18 +22,20 @@ void count_launches(int n) { g_launches.fetch_add((unsigned long long)n, std::me
 
 namespace {
 
-// Device address of the status word on the current device (looked up once
-// per device; the lookup is idempotent, so a race only repeats it).
+// Device address of the status word on the current device, looked up once
+// per device.  Threads that race on the first lookup store the same value.
 int* status_word() {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-    static int* cache[64] = {};
-    if (!cache[dev]) {
+    static std::atomic<int*> cache[64];
+    int* w = cache[dev].load(std::memory_order_relaxed);
+    if (!w) {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, dart::g_status) != cudaSuccess) return nullptr;
-        cache[dev] = static_cast<int*>(p);
+        w = static_cast<int*>(p);
+        cache[dev].store(w, std::memory_order_relaxed);
     }
-    return cache[dev];
+    return w;
 }
 
 thread_local char t_err[512] = "";
@@ -86,7 +88,7 @@ dart_status check_common(const dart_dims* d, dart_dtype dt, bool need_seqlen) {
 
 extern "C" {
 
-int dart_abi_version(void) { return 2; }
+int dart_abi_version(void) { return 3; }
 
 unsigned long long dart_launch_count(void) { return dart::g_launches.load(std::memory_order_relaxed); }
 
@@ -222,9 +224,9 @@ size_t dart_ssd_scan_backward_workspace_bytes(const dart_dims* d) {
 
 dart_status dart_ssd_scan_backward(const dart_dims* d, dart_dtype dtype, const void* x, const float* dt,
                                    const float* A, const void* Bm, const void* Cm, const float* init_state,
-                                   const float* states, const float* dy, const float* ddH, float* dx, float* ddt,
-                                   float* dA, float* dBm, float* dCm, float* dinit_state, void* workspace,
-                                   size_t workspace_bytes, void* stream) {
+                                   const float* states, const float* dy, const float* ddH, const float* dCm_add,
+                                   float* dx, float* ddt, float* dA, float* dBm, float* dCm, float* dinit_state,
+                                   void* workspace, size_t workspace_bytes, void* stream) {
     t_err[0] = 0;
     dart_status st = check_common(d, dtype, true);
     if (st != DART_OK) return st;
@@ -232,13 +234,13 @@ dart_status dart_ssd_scan_backward(const dart_dims* d, dart_dtype dtype, const v
         return fail(DART_ERR_UNSUPPORTED, "dart_ssd_scan_backward: (N=%d, P=%d) not compiled", d->dstate, d->headdim);
     DART_REQUIRE_PTR(x); DART_REQUIRE_PTR(dt); DART_REQUIRE_PTR(A); DART_REQUIRE_PTR(Bm); DART_REQUIRE_PTR(Cm);
     DART_OPTIONAL_PTR(init_state); DART_REQUIRE_PTR(states); DART_REQUIRE_PTR(dy); DART_OPTIONAL_PTR(ddH);
-    DART_REQUIRE_PTR(dx); DART_REQUIRE_PTR(ddt); DART_REQUIRE_PTR(dA); DART_REQUIRE_PTR(dBm); DART_REQUIRE_PTR(dCm);
+    DART_OPTIONAL_PTR(dCm_add); DART_REQUIRE_PTR(dx); DART_REQUIRE_PTR(ddt); DART_REQUIRE_PTR(dA); DART_REQUIRE_PTR(dBm); DART_REQUIRE_PTR(dCm);
     DART_OPTIONAL_PTR(dinit_state); DART_REQUIRE_PTR(workspace);
     const size_t need = dart_ssd_scan_backward_workspace_bytes(d);
     if (workspace_bytes < need)
         return fail(DART_ERR_INVALID_ARG, "workspace: %zu bytes, need %zu", workspace_bytes, need);
     dart::ScanBwdArgs a{d->batch, d->seqlen, d->nheads, d->headdim, d->dstate, d->chunk, x, dt, A, Bm, Cm,
-                        init_state, states, dy, ddH, dx, ddt, dA, dBm, dCm, dinit_state, status_word()};
+                        init_state, states, dy, ddH, dCm_add, dx, ddt, dA, dBm, dCm, dinit_state, status_word()};
     if (!a.status) return fail(DART_ERR_CUDA, "dart_ssd_scan_backward: no device status word");
     cudaError_t e = dart::launch_ssd_scan_bwd(a, workspace, dtype, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "dart_ssd_scan_backward launch");
@@ -274,7 +276,7 @@ dart_status dart_sma_backward(const dart_dims* d, dart_dtype dtype, const void* 
 }
 
 size_t dart_decode_step_workspace_bytes(const dart_dims* d, dart_dtype, int cmax) {
-    if (!d || cmax < 0) return 0;
+    if (!d || cmax < 0 || cmax > dart::kDecodeMaxCmax) return 0;
     const size_t ns = (size_t)dart::decode_num_splits(d->batch, d->nheads, cmax);
     return sizeof(float) * (size_t)d->batch * (size_t)d->nheads * ns * (2 + 2 * (size_t)d->headdim);
 }
@@ -289,7 +291,8 @@ dart_status dart_decode_step(const dart_dims* d, dart_dtype dtype, const void* x
     if (st != DART_OK) return st;
     if (!dart::decode_supported(d->dstate, d->headdim, d->chunk, dtype))
         return fail(DART_ERR_UNSUPPORTED, "dart_decode_step: (N=%d, P=%d) not compiled", d->dstate, d->headdim);
-    if (cmax < 1) return fail(DART_ERR_INVALID_ARG, "cmax must be >= 1");
+    if (cmax < 1 || cmax > dart::kDecodeMaxCmax)
+        return fail(DART_ERR_INVALID_ARG, "cmax = %d outside [1, %d]", cmax, dart::kDecodeMaxCmax);
     DART_REQUIRE_PTR(x_t); DART_REQUIRE_PTR(dt_t); DART_REQUIRE_PTR(A); DART_REQUIRE_PTR(B_t);
     DART_REQUIRE_PTR(C_t); DART_REQUIRE_PTR(Q_t); DART_REQUIRE_PTR(E_t); DART_REQUIRE_PTR(state);
     DART_REQUIRE_PTR(dH_cur); DART_REQUIRE_PTR(dH_cache); DART_REQUIRE_PTR(n_chunks);
@@ -318,7 +321,8 @@ dart_status dart_decode_step_decayed(const dart_dims* d, dart_dtype dtype, const
     if (!dart::decode_supported(d->dstate, d->headdim, d->chunk, dtype))
         return fail(DART_ERR_UNSUPPORTED, "dart_decode_step_decayed: (N=%d, P=%d) not compiled", d->dstate,
                     d->headdim);
-    if (cmax < 1) return fail(DART_ERR_INVALID_ARG, "cmax must be >= 1");
+    if (cmax < 1 || cmax > dart::kDecodeMaxCmax)
+        return fail(DART_ERR_INVALID_ARG, "cmax = %d outside [1, %d]", cmax, dart::kDecodeMaxCmax);
     DART_REQUIRE_PTR(x_t); DART_REQUIRE_PTR(dt_t); DART_REQUIRE_PTR(A); DART_REQUIRE_PTR(B_t);
     DART_REQUIRE_PTR(C_t); DART_REQUIRE_PTR(Q_t); DART_REQUIRE_PTR(E_t); DART_REQUIRE_PTR(state);
     DART_REQUIRE_PTR(dH_cur); DART_REQUIRE_PTR(dH_cache); DART_REQUIRE_PTR(n_chunks);
@@ -347,7 +351,8 @@ dart_status dart_decode_step_e4m3(const dart_dims* d, dart_dtype dtype, const vo
     if (!dart::decode_e4m3_supported(d->dstate, d->headdim))
         return fail(DART_ERR_UNSUPPORTED, "dart_decode_step_e4m3: (N=%d, P=%d) not compiled (P = 64, N = 64 or 128)",
                     d->dstate, d->headdim);
-    if (cmax < 1) return fail(DART_ERR_INVALID_ARG, "cmax must be >= 1");
+    if (cmax < 1 || cmax > dart::kDecodeMaxCmax)
+        return fail(DART_ERR_INVALID_ARG, "cmax = %d outside [1, %d]", cmax, dart::kDecodeMaxCmax);
     DART_REQUIRE_PTR(x_t); DART_REQUIRE_PTR(dt_t); DART_REQUIRE_PTR(A); DART_REQUIRE_PTR(B_t);
     DART_REQUIRE_PTR(C_t); DART_REQUIRE_PTR(Q_t); DART_REQUIRE_PTR(E_t); DART_REQUIRE_PTR(state);
     DART_REQUIRE_PTR(dH_cur); DART_REQUIRE_PTR(cache); DART_REQUIRE_PTR(cache_exp); DART_REQUIRE_PTR(n_chunks);
@@ -414,7 +419,8 @@ dart_status dart_decode_step_noalloc(const dart_dims* d, dart_dtype dtype, const
     if (!dart::decode_supported(d->dstate, d->headdim, d->chunk, dtype))
         return fail(DART_ERR_UNSUPPORTED, "dart_decode_step_noalloc: (N=%d, P=%d) not compiled", d->dstate,
                     d->headdim);
-    if (cmax < 1) return fail(DART_ERR_INVALID_ARG, "cmax must be >= 1");
+    if (cmax < 1 || cmax > dart::kDecodeMaxCmax)
+        return fail(DART_ERR_INVALID_ARG, "cmax = %d outside [1, %d]", cmax, dart::kDecodeMaxCmax);
     DART_REQUIRE_PTR(x_t); DART_REQUIRE_PTR(dt_t); DART_REQUIRE_PTR(A); DART_REQUIRE_PTR(B_t);
     DART_REQUIRE_PTR(C_t); DART_REQUIRE_PTR(Q_t); DART_REQUIRE_PTR(E_t); DART_REQUIRE_PTR(state);
     DART_REQUIRE_PTR(dH_cur); DART_REQUIRE_PTR(dH_cache); DART_REQUIRE_PTR(n_chunks);

@@ -25,6 +25,7 @@ struct ScanBwdArgs {
     const float* states;    // [B,H,C,N,P] boundary states written by the forward
     const float* dy;        // [B,L,H,P] gradient of y_ssd
     const float* ddH;       // nullable [B,H,C,N,P] gradient of the chunk memories
+    const float* dC_add;    // nullable [B,L,N]: added to dC (e.g. the SMA backward's part; may be dC)
     float* dx; float* ddt; float* dA; float* dB; float* dC;   // outputs (fp32)
     float* dinit;           // nullable [B,H,N,P] output
     int* status;

@@ -154,6 +154,9 @@ size_t sma_decay_workspace_bytes(int B, int L, int H, int S);
 const char* sma_impl_name(int N, int P, int S, dart_dtype dt);
 bool decode_supported(int N, int P, int S, dart_dtype dt);
 int decode_num_splits(int B, int H, int cmax);
+// Largest cache capacity the decode entries accept (memories per sequence):
+// 2^20 memories is 2^28 tokens of context at S = 256.
+constexpr int kDecodeMaxCmax = 1 << 20;
 bool decode_e4m3_supported(int N, int P);
 cudaError_t launch_decode_e4m3(const DecodeArgs& a, dart_dtype dt, cudaStream_t st);
 // dH [B,H,C,N,P] (dtype) memories 0..nmem-1 -> E4M3 codes and row exponents

@@ -43,6 +43,8 @@
 // at 0 (written by split 0).
 #include <cuda_fp8.h>
 
+#include <atomic>
+
 #include "dart_common.cuh"
 
 namespace dart {
@@ -663,8 +665,8 @@ cudaError_t launch_cache_quantize_e4m3(int B, int H, int C, int N, int P, int nm
 }
 
 int decode_num_splits(int, int, int cmax) {
-    const int ns = (cmax + kChunksPerSplit - 1) / kChunksPerSplit;
-    return ns < 1 ? 1 : ns;
+    const long long ns = ((long long)cmax + kChunksPerSplit - 1) / kChunksPerSplit;
+    return ns < 1 ? 1 : (int)ns;
 }
 
 bool decode_supported(int N, int P, int S, dart_dtype) {
@@ -705,14 +707,15 @@ cudaError_t noalloc_scratch(void** out) {
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    static void* cache[64] = {};  // looked up once per device; a racing lookup only repeats it
-    if (!cache[dev]) {
-        void* p = nullptr;
+    // looked up once per device; threads that race on the first lookup store the same value
+    static std::atomic<void*> cache[64];
+    void* p = cache[dev].load(std::memory_order_relaxed);
+    if (!p) {
         e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
         if (e != cudaSuccess) return e;
-        cache[dev] = p;
+        cache[dev].store(p, std::memory_order_relaxed);
     }
-    *out = cache[dev];
+    *out = p;
     return cudaSuccess;
 }
 

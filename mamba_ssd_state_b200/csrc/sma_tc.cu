@@ -47,6 +47,8 @@
 #include <cuda_bf16.h>
 #include <string.h>
 
+#include <atomic>
+
 #include "dart_common.cuh"
 #include "sm100.cuh"
 #include "tensor_map.h"
@@ -652,11 +654,19 @@ cudaError_t launch_sma_tc(const SmaArgs& a, cudaStream_t st) {
         cfg.stream = st;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        // as many pairs as can be resident at once (not every SM need pair up)
-        cfg.gridDim = dim3(2 * (unsigned)(sms / 2), 1, 1);
-        int clusters = 0;
-        if ((e = cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg)) != cudaSuccess) return e;
-        if (clusters <= 0) return cudaErrorInvalidConfiguration;
+        // as many pairs as can be resident at once (not every SM need pair
+        // up), queried once per device and variant; threads that race on the
+        // first query store the same value
+        static std::atomic<int> pairs_cache[2][64];
+        int dev = 0;
+        if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+        int clusters = dev >= 0 && dev < 64 ? pairs_cache[decayed][dev].load(std::memory_order_relaxed) : 0;
+        if (clusters <= 0) {
+            cfg.gridDim = dim3(2 * (unsigned)(sms / 2), 1, 1);
+            if ((e = cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg)) != cudaSuccess) return e;
+            if (clusters <= 0) return cudaErrorInvalidConfiguration;
+            if (dev >= 0 && dev < 64) pairs_cache[decayed][dev].store(clusters, std::memory_order_relaxed);
+        }
         if (clusters > p.total_tiles) clusters = p.total_tiles;
         cfg.gridDim = dim3(2 * (unsigned)clusters, 1, 1);
         if ((e = cudaLaunchKernelEx(&cfg, kern, p)) != cudaSuccess) return e;

@@ -205,7 +205,8 @@ __global__ void __launch_bounds__(N * P / kCols) ssd_scan_bwd_kernel(ScanBwdArgs
     if (tid == 0) a.dApart[bh] = dA_acc;
 }
 
-// dB, dC summed over heads; dA summed over the batch (fixed order).
+// dB, dC summed over heads (dC plus dC_add when given); dA summed over the
+// batch (fixed order).
 __global__ void scan_bwd_reduce(ScanBwdArgs a, int N) {
     const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
     const size_t nbc = (size_t)a.B * a.L * N;
@@ -216,6 +217,7 @@ __global__ void scan_bwd_reduce(ScanBwdArgs a, int N) {
             sb += a.dBh[(tok * a.H + h) * N + nn];
             sc += a.dCh[(tok * a.H + h) * N + nn];
         }
+        if (a.dC_add) sc += a.dC_add[i];   // read before the write: dC_add may be dC itself
         a.dB[i] = sb;
         a.dC[i] = sc;
     }

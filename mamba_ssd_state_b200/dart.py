@@ -73,7 +73,7 @@ def load(path: str = LIBRARY) -> ctypes.CDLL:
     lib.dart_ssd_scan_backward_workspace_bytes.restype = ctypes.c_size_t
     lib.dart_ssd_scan_backward_workspace_bytes.argtypes = [D]
     lib.dart_ssd_scan_backward.restype = ctypes.c_int
-    lib.dart_ssd_scan_backward.argtypes = [D, ctypes.c_int] + [_P] * 16 + [ctypes.c_size_t, _P]
+    lib.dart_ssd_scan_backward.argtypes = [D, ctypes.c_int] + [_P] * 17 + [ctypes.c_size_t, _P]
     lib.dart_sma_backward_workspace_bytes.restype = ctypes.c_size_t
     lib.dart_sma_backward_workspace_bytes.argtypes = [D]
     lib.dart_sma_backward.restype = ctypes.c_int
@@ -318,17 +318,19 @@ def dart_sma_backward(Q, E, Cm, dH, chunk: int, g: float, dy, *, workspace=None)
 
 
 def dart_ssd_scan_backward(x, dt, A, Bm, Cm, chunk: int, states, dy, ddH=None, init_state=None, *,
-                           workspace=None) -> dict:
+                           dCm_add=None, workspace=None) -> dict:
     """Gradients of sum(dy * y_ssd) + sum(ddH * dH) through the scan: a dict
-    of float32 device tensors dx, ddt, dA, dBm, dCm (the scan's part) and,
-    with an initial state, dinit_state.  x/Bm/Cm as given to the forward
-    (dtype), dt/A/init_state float32, states = the forward's boundary states,
-    dy float32 [B,L,H,P], ddH float32 [B,H,C,N,P] or None."""
+    of float32 device tensors dx, ddt, dA, dBm, dCm and, with an initial
+    state, dinit_state.  x/Bm/Cm as given to the forward (dtype),
+    dt/A/init_state float32, states = the forward's boundary states, dy
+    float32 [B,L,H,P], ddH float32 [B,H,C,N,P] or None.  The library adds
+    dCm_add (float32 [B,L,N], e.g. dart_sma_backward's dCm) into dCm."""
     lib = load()
     dev = _device_of(x, dt, A, Bm, Cm, states, dy)
     x, Bm, Cm = (_dev(v, dev, x.dtype) for v in (x, Bm, Cm))
     dt, A, states, dy = (_dev(v, dev, torch.float32) for v in (dt, A, states, dy))
     ddH = _dev(ddH, dev, torch.float32)
+    dCm_add = _dev(dCm_add, dev, torch.float32)
     init_state = _dev(init_state, dev, torch.float32)
     Bsz, L, H, P = x.shape
     N = Bm.shape[-1]
@@ -336,6 +338,8 @@ def dart_ssd_scan_backward(x, dt, A, Bm, Cm, chunk: int, states, dy, ddH=None, i
     _shape("states", states, (Bsz, H, C, N, P)); _shape("dy", dy, (Bsz, L, H, P))
     if ddH is not None:
         _shape("ddH", ddH, (Bsz, H, C, N, P))
+    if dCm_add is not None:
+        _shape("dCm_add", dCm_add, (Bsz, L, N))
     dims = Dims(Bsz, L, H, P, N, chunk, 1)
     out = {"dx": torch.empty((Bsz, L, H, P), device=dev), "ddt": torch.empty((Bsz, L, H), device=dev),
            "dA": torch.empty((H,), device=dev), "dBm": torch.empty((Bsz, L, N), device=dev),
@@ -348,7 +352,7 @@ def dart_ssd_scan_backward(x, dt, A, Bm, Cm, chunk: int, states, dy, ddH=None, i
     with torch.cuda.device(dev):
         _check(lib.dart_ssd_scan_backward(ctypes.byref(dims), _dtype_code(x.dtype), _ptr(x), _ptr(dt), _ptr(A),
                                           _ptr(Bm), _ptr(Cm), _ptr(init_state), _ptr(states), _ptr(dy), _ptr(ddH),
-                                          _ptr(out["dx"]), _ptr(out["ddt"]), _ptr(out["dA"]), _ptr(out["dBm"]),
+                                          _ptr(dCm_add), _ptr(out["dx"]), _ptr(out["ddt"]), _ptr(out["dA"]), _ptr(out["dBm"]),
                                           _ptr(out["dCm"]), _ptr(out.get("dinit_state")), _ptr(workspace),
                                           workspace.numel(), _stream()))
     return out
@@ -362,9 +366,8 @@ def layer_backward(x, dt, A, Bm, Cm, Q, E, chunk: int, g: float, dy, init_state=
     dinit_state with an initial state)."""
     y_ssd, dH, states = dart_ssd_chunk_scan(x, dt, A, Bm, Cm, chunk, init_state)
     sm = dart_sma_backward(Q, E, Cm, dH, chunk, g, dy)
-    sc = dart_ssd_scan_backward(x, dt, A, Bm, Cm, chunk, states, dy, sm["ddH"], init_state)
-    out = dict(sc)
-    out["dCm"] = sc["dCm"] + sm["dCm"]
+    # the scan backward adds the SMA's C gradient into its own (in the library)
+    out = dart_ssd_scan_backward(x, dt, A, Bm, Cm, chunk, states, dy, sm["ddH"], init_state, dCm_add=sm["dCm"])
     out.update(dQ=sm["dQ"], dE=sm["dE"], dg=sm["dg"])
     return out
 
@@ -544,6 +547,16 @@ def dart_decode_step_noalloc(x, dt, A, Bm, Cm, Q, E, g: float, state, dH_cur, ca
 def decode_workspace_bytes(nseq, nheads, headdim, dstate, chunk, cmax, dtype) -> int:
     dims = Dims(nseq, 0, nheads, headdim, dstate, chunk, 1)
     return load().dart_decode_step_workspace_bytes(ctypes.byref(dims), _dtype_code(dtype), cmax)
+
+
+def sma_backward_workspace_bytes(batch, seqlen, nheads, headdim, dstate, chunk) -> int:
+    dims = Dims(batch, seqlen, nheads, headdim, dstate, chunk, 1)
+    return int(load().dart_sma_backward_workspace_bytes(ctypes.byref(dims)))
+
+
+def scan_backward_workspace_bytes(batch, seqlen, nheads, headdim, dstate, chunk) -> int:
+    dims = Dims(batch, seqlen, nheads, headdim, dstate, chunk, 1)
+    return int(load().dart_ssd_scan_backward_workspace_bytes(ctypes.byref(dims)))
 
 
 def scan_workspace_bytes(batch, seqlen, nheads, headdim, dstate, chunk, dtype) -> int:

@@ -39,7 +39,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version(lib):
-    assert lib.dart_abi_version() == 2
+    assert lib.dart_abi_version() == 3
 
 
 def test_supported_set(lib):
@@ -207,7 +207,7 @@ def test_scan_backward_workspace_and_validation(lib):
     want = 2 * pad(4 * 2 * 3 * 256 * 128 * 64) + 2 * pad(4 * 2 * 500 * 3 * 128) + pad(4 * 2 * 3)
     assert lib.dart_ssd_scan_backward_workspace_bytes(ctypes.byref(d)) == want
     f = lib.dart_ssd_scan_backward
-    ok = [FAKE] * 5 + [None, FAKE, FAKE, None] + [FAKE] * 5 + [None, FAKE]
+    ok = [FAKE] * 5 + [None, FAKE, FAKE, None, None] + [FAKE] * 5 + [None, FAKE]
     assert f(ctypes.byref(d), dart.DART_BF16, *ok[:6], None, *ok[7:], want, None) == dart.DART_ERR_INVALID_ARG
     assert b"states" in lib.dart_last_error()
     assert f(ctypes.byref(d), dart.DART_BF16, *ok, want - 1, None) == dart.DART_ERR_INVALID_ARG
@@ -227,6 +227,30 @@ def test_decode_rejects_bad_args(lib):
     assert call(cmax=0) == dart.DART_ERR_INVALID_ARG
     assert call(state=None) == dart.DART_ERR_INVALID_ARG
     assert call(ws_bytes=ws - 4) == dart.DART_ERR_INVALID_ARG
+
+
+def test_decode_cmax_bound(lib):
+    """Every decode entry takes 1 <= cmax <= 2^20; a cmax near INT_MAX (whose
+    split count would overflow 32-bit arithmetic) is rejected on the host,
+    and the workspace query answers 0 for it instead of a one-split size."""
+    d = dart.Dims(4, 0, 2, 64, 128, 256, 1)
+    big = (1 << 31) - 10
+    assert lib.dart_decode_step_workspace_bytes(ctypes.byref(d), dart.DART_BF16, big) == 0
+    assert lib.dart_decode_step_workspace_bytes(ctypes.byref(d), dart.DART_BF16, (1 << 20) + 1) == 0
+    assert lib.dart_decode_step_workspace_bytes(ctypes.byref(d), dart.DART_BF16, 1 << 20) > 0
+    tok = [FAKE] * 7 + [0.5]          # x, dt, A, B, C, Q, E and g
+    mem = [FAKE] * 3                  # state, dH_cur, cache
+    for cmax in ((1 << 20) + 1, big):
+        assert lib.dart_decode_step(ctypes.byref(d), dart.DART_BF16, *tok, *mem, cmax, *[FAKE] * 4, 1 << 40,
+                                    None) == dart.DART_ERR_INVALID_ARG
+        assert b"cmax" in lib.dart_last_error()
+        assert lib.dart_decode_step_decayed(ctypes.byref(d), dart.DART_BF16, *tok, *mem, cmax, *[FAKE] * 5,
+                                            1 << 40, None) == dart.DART_ERR_INVALID_ARG
+        assert lib.dart_decode_step_e4m3(ctypes.byref(d), dart.DART_BF16, *tok, *mem, FAKE, cmax, FAKE, FAKE,
+                                         None, FAKE, FAKE, 1 << 40, None) == dart.DART_ERR_INVALID_ARG
+        assert lib.dart_decode_step_noalloc(ctypes.byref(d), dart.DART_BF16, *tok, *mem, cmax, FAKE, FAKE, FAKE,
+                                            None) == dart.DART_ERR_INVALID_ARG
+        assert b"cmax" in lib.dart_last_error()
 
 
 def test_binding_fails_loudly_without_cuda(lib):

@@ -104,6 +104,14 @@ def test_scan_backward_matches_oracle(shape, dt_name, with_init):
     tol = TOL_FWD_INPUTS[dt_name]
     for k in ("dx", "ddt", "dA", "dBm", "dCm") + (("dinit_state",) if h0 is not None else ()):
         assert_close(k, got[k], ref[k], tol)
+    # dCm_add is added into dCm inside the library: the same float sum as
+    # adding it afterwards, so the two agree bit for bit
+    add = torch.from_numpy(np.random.default_rng(L + 3).standard_normal((Bz, L, N)).astype(np.float32)).cuda()
+    got2 = dart.dart_ssd_scan_backward(d["x"], d["dt"], d["A"], d["Bm"], d["Cm"], S, states, dy.cuda(),
+                                       gdH.cuda(), None if h0 is None else h0.cuda(), dCm_add=add)
+    dart.dart_sync_status()
+    assert torch.equal(got2["dCm"], got["dCm"] + add)
+    assert torch.equal(got2["dx"], got["dx"])
 
 
 @pytest.mark.parametrize("shape,dt_name,with_init", [SCAN_CASES[0], SCAN_CASES[3]], ids=[SCAN_IDS[0], SCAN_IDS[3]])
