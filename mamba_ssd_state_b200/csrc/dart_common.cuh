@@ -137,6 +137,35 @@ struct DecodeArgs {
 // Counts one kernel launch (see dart_launch_count).
 void count_launches(int n);
 
+// Launches `kernel` so that it may start while the previous launch on the
+// stream finishes (programmatic dependent launch); the kernel must call
+// sm100::griddep_wait() before touching global memory.  cluster_x > 1
+// launches clusters of that many CTAs along x.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                             int cluster_x, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[2];
+    int na = 0;
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+    if (cluster_x > 1) {
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = (unsigned)cluster_x;
+        attr[na].val.clusterDim.y = 1;
+        attr[na].val.clusterDim.z = 1;
+        ++na;
+    }
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = (unsigned)na;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
+}
+
 cudaError_t launch_ssd_scan(const ScanArgs& a, dart_dtype dt, cudaStream_t st);
 cudaError_t launch_sma(const SmaArgs& a, dart_dtype dt, cudaStream_t st);
 cudaError_t launch_decode(const DecodeArgs& a, dart_dtype dt, cudaStream_t st);

@@ -114,6 +114,12 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// Programmatic dependent launch: waits until the kernels this grid depends
+// on (the previous launches on the stream) have completed and their memory
+// is visible.  Kernels launched with launch_dependent() do their shared
+// memory and TMEM set-up first and call this before any global memory access.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // Hint that a global line will be read soon (fetched into L2).
 __device__ __forceinline__ void prefetch_l2(const void* p) {
     asm volatile("prefetch.global.L2 [%0];" ::"l"(p));

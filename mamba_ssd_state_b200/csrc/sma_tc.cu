@@ -197,6 +197,7 @@ __global__ void __launch_bounds__(kThreads, 1) sma_tc_kernel(const __grid_consta
         __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
+    griddep_wait();
 
     const WaitCtx wc{abort_flag, p.status, 1};
     if (warp == 0) {
@@ -644,11 +645,15 @@ cudaError_t launch_sma_tc(const SmaArgs& a, cudaStream_t st) {
             return e;
         cudaLaunchConfig_t cfg;
         memset(&cfg, 0, sizeof(cfg));
-        cudaLaunchAttribute attr[1];
+        cudaLaunchAttribute attr[2];
         attr[0].id = cudaLaunchAttributeClusterDimension;
         attr[0].val.clusterDim.x = 2;
         attr[0].val.clusterDim.y = 1;
         attr[0].val.clusterDim.z = 1;
+        // it may start while the previous launch on the stream finishes; the
+        // kernel waits for it before touching global memory
+        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[1].val.programmaticStreamSerializationAllowed = 1;
         cfg.blockDim = dim3(kThreads, 1, 1);
         cfg.dynamicSmemBytes = kSmemBytes;
         cfg.stream = st;
@@ -669,6 +674,7 @@ cudaError_t launch_sma_tc(const SmaArgs& a, cudaStream_t st) {
         }
         if (clusters > p.total_tiles) clusters = p.total_tiles;
         cfg.gridDim = dim3(2 * (unsigned)clusters, 1, 1);
+        cfg.numAttrs = 2;
         if ((e = cudaLaunchKernelEx(&cfg, kern, p)) != cudaSuccess) return e;
     } else {
         p.cta_per_tile = 1;
@@ -678,7 +684,7 @@ cudaError_t launch_sma_tc(const SmaArgs& a, cudaStream_t st) {
         auto kern = decayed ? sma_tc_kernel<false, true> : sma_tc_kernel<false, false>;
         if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes)) != cudaSuccess)
             return e;
-        kern<<<grid, kThreads, kSmemBytes, st>>>(p);
+        if ((e = launch_dependent(kern, dim3(grid), dim3(kThreads), kSmemBytes, st, 1, p)) != cudaSuccess) return e;
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     count_launches(1);

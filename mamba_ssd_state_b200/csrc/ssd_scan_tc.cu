@@ -86,6 +86,7 @@ template <int S>
 __global__ void __launch_bounds__(256) chunk_decay_kernel(const __grid_constant__ ScanTcParams p) {
     constexpr int K = S / 32;             // rounds of 32 tokens
     __shared__ float dts[8 * (S + 1)];    // [head of the group][S + 1]
+    griddep_wait();
     const int ngh = (p.H + 7) / 8;
     const int hgi = blockIdx.x % ngh;
     const int c = (blockIdx.x / ngh) % p.C, b = blockIdx.x / (ngh * p.C);
@@ -214,6 +215,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_state_tc_kernel(const __gri
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
+    griddep_wait();
 
     const WaitCtx wc{abort_flag, p.status, 2};
     if (warp == 0) {
@@ -378,6 +380,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_state_tc_kernel(const __gri
 constexpr int kPassPre = 8;
 __global__ void __launch_bounds__(256) state_pass_tc_kernel(const __grid_constant__ ScanTcParams p) {
     constexpr int NP = kN * kP;
+    griddep_wait();
     const int h = blockIdx.y, b = blockIdx.z;
     const int e4 = (blockIdx.x * blockDim.x + threadIdx.x) * 4;  // 4 consecutive elements
     if (e4 >= NP) return;
@@ -503,6 +506,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_output_tc_kernel(const __gr
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
+    griddep_wait();
 
     const WaitCtx wc{abort_flag, p.status, 3};
     if (warp == 0) {
@@ -861,11 +865,9 @@ cudaError_t launch_ssd_scan_tc(const ScanArgs& a, cudaStream_t st) {
     // 0. per-token decay terms, one CTA per (b, c, group of 8 heads)
     {
         const int grid = a.B * p.C * ((a.H + 7) / 8);
-        if (a.S == 256)
-            chunk_decay_kernel<256><<<grid, 256, 0, st>>>(p);
-        else
-            chunk_decay_kernel<128><<<grid, 256, 0, st>>>(p);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        e = a.S == 256 ? launch_dependent(chunk_decay_kernel<256>, dim3(grid), dim3(256), 0, st, 1, p)
+                       : launch_dependent(chunk_decay_kernel<128>, dim3(grid), dim3(256), 0, st, 1, p);
+        if (e != cudaSuccess) return e;
     }
     // 1. chunk memories
     {
@@ -879,19 +881,20 @@ cudaError_t launch_ssd_scan_tc(const ScanArgs& a, cudaStream_t st) {
             const uint32_t smem = cs::Layout<256>::kBytes;
             if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
                 return e;
-            k<<<grid, cs::kThreads, smem, st>>>(p);
+            if ((e = launch_dependent(k, dim3(grid), dim3(cs::kThreads), smem, st, 1, p)) != cudaSuccess) return e;
         } else {
             auto k = cs::chunk_state_tc_kernel<128>;
             const uint32_t smem = cs::Layout<128>::kBytes;
             if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
                 return e;
-            k<<<grid, cs::kThreads, smem, st>>>(p);
+            if ((e = launch_dependent(k, dim3(grid), dim3(cs::kThreads), smem, st, 1, p)) != cudaSuccess) return e;
         }
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     // 2. state passing
-    state_pass_tc_kernel<<<dim3(kN * kP / 4 / 256, a.H, a.B), 256, 0, st>>>(p);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_dependent(state_pass_tc_kernel, dim3(kN * kP / 4 / 256, a.H, a.B), dim3(256), 0, st, 1, p)) !=
+        cudaSuccess)
+        return e;
     // 3. outputs
     {
         // persistent: one CTA per SM, contiguous ranges of the (b, c, half, h)
@@ -922,7 +925,9 @@ cudaError_t launch_ssd_scan_tc(const ScanArgs& a, cudaStream_t st) {
         if ((e = cudaFuncSetAttribute(co::chunk_output_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)co::kBytes)) != cudaSuccess)
             return e;
-        co::chunk_output_tc_kernel<<<grid, co::kThreads, co::kBytes, st>>>(p);
+        if ((e = launch_dependent(co::chunk_output_tc_kernel, dim3(grid), dim3(co::kThreads), co::kBytes, st, 1, p)) !=
+            cudaSuccess)
+            return e;
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     count_launches(4);
