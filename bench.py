@@ -23,6 +23,7 @@ a bounded sample of the same workload, on this host's cores.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import datetime
 import json
 import os
@@ -64,6 +65,8 @@ def parse():
                    help="skip the forward with decayed memories (dart_sma_forward_decayed)")
     p.add_argument("--no-e4m3", action="store_true", help="skip the decode with an E4M3 cache")
     p.add_argument("--decode-steps", type=int, default=DEC.nsteps)
+    p.add_argument("--decode-nseq", type=int, default=DEC.nseq,
+                   help="sequences in the decode batch (a smaller cache for profiling)")
     p.add_argument("--no-configs", action="store_true",
                    help="skip the other forward workloads (B=4, L=2048 and B=1, L=65536)")
     p.add_argument("--no-backward", action="store_true", help="skip the backward region")
@@ -394,29 +397,30 @@ def e2e_region(args, dist, dart, inp):
 
 
 def decode_region(args, dist, dart, peaks, decayed=False, e4m3=False):
+    dec = dataclasses.replace(DEC, nseq=args.decode_nseq)
     dev = torch.device("cuda", torch.cuda.current_device())
-    init = synth.decode_initial(DEC, seed=dist.rank)
+    init = synth.decode_initial(dec, seed=dist.rank)
     work = {k: v.to(dev) for k, v in init.items()}
     if e4m3:
         # the same memories in an E4M3 cache (codes + row exponents)
         cache8 = torch.empty(work["cache"].shape, device=dev, dtype=torch.uint8)
         cexp = torch.empty(work["cache"].shape[:-1], device=dev, dtype=torch.int8)
-        dart.cache_quantize_e4m3(work["cache"], DEC.ncached, cache8, cexp)
+        dart.cache_quantize_e4m3(work["cache"], dec.ncached, cache8, cexp)
         del work["cache"]
         work["cache"], work["cache_exp"] = cache8, cexp
     if decayed:
         # log-decays of the cached memories (dart_decode_step_decayed), -U(0, 3)
         g = torch.Generator().manual_seed(1000 + dist.rank)
-        work["memlog"] = (-3.0 * torch.rand((DEC.nseq, DEC.nheads, DEC.cmax), generator=g)).to(dev)
+        work["memlog"] = (-3.0 * torch.rand((dec.nseq, dec.nheads, dec.cmax), generator=g)).to(dev)
     saved = {k: v.clone() for k, v in work.items()}
-    A = synth.decode_A(DEC, seed=dist.rank).to(dev)
+    A = synth.decode_A(dec, seed=dist.rank).to(dev)
     # the cache holds one free slot: at most S steps (one append) per run
-    nsteps = max(1, min(args.decode_steps, DEC.chunk * (DEC.cmax - DEC.ncached)))
-    toks = [synth.decode_tokens(DEC, s, seed=dist.rank) for s in range(nsteps)]
+    nsteps = max(1, min(args.decode_steps, dec.chunk * (dec.cmax - dec.ncached)))
+    toks = [synth.decode_tokens(dec, s, seed=dist.rank) for s in range(nsteps)]
     toks = [{k: v.to(dev) for k, v in t.items()} for t in toks]
-    y = torch.empty((DEC.nseq, DEC.nheads, DEC.headdim), device=dev, dtype=torch.float32)
-    ws = torch.empty(max(16, dart.decode_workspace_bytes(DEC.nseq, DEC.nheads, DEC.headdim, DEC.dstate,
-                                                         DEC.chunk, DEC.cmax, torch.bfloat16)),
+    y = torch.empty((dec.nseq, dec.nheads, dec.headdim), device=dev, dtype=torch.float32)
+    ws = torch.empty(max(16, dart.decode_workspace_bytes(dec.nseq, dec.nheads, dec.headdim, dec.dstate,
+                                                         dec.chunk, dec.cmax, torch.bfloat16)),
                      device=dev, dtype=torch.uint8)
     stream = torch.cuda.current_stream()
 
@@ -424,8 +428,8 @@ def decode_region(args, dist, dart, peaks, decayed=False, e4m3=False):
         t = toks[s]
         if ev:
             ev[0].record(stream)
-        dart.dart_decode_step(t["x"], t["dt"], A, t["Bm"], t["Cm"], t["Q"], t["E"], DEC.g, work["state"],
-                              work["dH_cur"], work["cache"], work["nchunks"], work["pos"], DEC.chunk, y=y,
+        dart.dart_decode_step(t["x"], t["dt"], A, t["Bm"], t["Cm"], t["Q"], t["E"], dec.g, work["state"],
+                              work["dH_cur"], work["cache"], work["nchunks"], work["pos"], dec.chunk, y=y,
                               workspace=ws, memlog=work.get("memlog"), cache_exp=work.get("cache_exp"))
         if ev:
             ev[1].record(stream)
@@ -456,19 +460,19 @@ def decode_region(args, dist, dart, peaks, decayed=False, e4m3=False):
     ms = dist.max(start.elapsed_time(end))
     per = [e[0].elapsed_time(e[1]) for e in evs]
     # step s starts at pos = s % S with ncached + s // S memories; pos = S-1 appends
-    total_bytes = sum(decode_bytes(DEC, DEC.ncached + s // DEC.chunk, s % DEC.chunk == DEC.chunk - 1, e4m3)
+    total_bytes = sum(decode_bytes(dec, dec.ncached + s // dec.chunk, s % dec.chunk == dec.chunk - 1, e4m3)
                       for s in range(nsteps))
     if decayed:   # each cached memory's log-decay is read and written once per step
-        total_bytes += sum(8 * DEC.nseq * DEC.nheads * (DEC.ncached + s // DEC.chunk) for s in range(nsteps))
+        total_bytes += sum(8 * dec.nseq * dec.nheads * (dec.ncached + s // dec.chunk) for s in range(nsteps))
     bytes_step = total_bytes / nsteps
     step_ms = statistics.mean(per)
     achieved = bytes_step / (step_ms / 1e3) / 1e9
     return {
-        "value": dist.world * DEC.nseq * nsteps / (ms / 1e3), "unit": "tokens/s",
+        "value": dist.world * dec.nseq * nsteps / (ms / 1e3), "unit": "tokens/s",
         "ms_per_step": ms / nsteps, "steps": nsteps, "launches": n1 - n0, "clocks": clk,
-        "config": {"workload": "decode_64seq_128mem", "nseq": DEC.nseq, "nheads": DEC.nheads,
-                   "headdim": DEC.headdim, "dstate": DEC.dstate, "chunk": DEC.chunk,
-                   "cached_chunks": DEC.ncached, "context": DEC.ncached * DEC.chunk,
+        "config": {"workload": f"decode_{dec.nseq}seq_128mem", "nseq": dec.nseq, "nheads": dec.nheads,
+                   "headdim": dec.headdim, "dstate": dec.dstate, "chunk": dec.chunk,
+                   "cached_chunks": dec.ncached, "context": dec.ncached * dec.chunk,
                    "l2": "cache 4.3 GB per step >> 126 MB L2"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": achieved / peaks["hbm_gbs"], "traffic": captured_traffic("decode_step"),
