@@ -15,11 +15,12 @@
  * --------------------------------
  * - Notation: B batch, L sequence length, H heads, P head dimension (value
  *   axis), N state size (key axis), S chunk size, C = ceil(L / S) chunks (a
- *   partial last chunk counts).  B and C projections are shared by all heads
- *   (ngroups = 1).
+ *   partial last chunk counts), G = ngroups groups of heads sharing one B
+ *   and one C projection (Mamba-2's grouped B/C): G divides H and head h
+ *   reads group h / (H / G).  G = 1 is one B and C for all heads.
  * - Every tensor is dense, row-major (last index fastest), on the CUDA device
  *   that is current for the calling thread, and 16-byte aligned.  Layouts:
- *     x[B,L,H,P]  dt[B,L,H]  A[H]  Bm[B,L,N]  Cm[B,L,N]  Q[B,L,H,N]
+ *     x[B,L,H,P]  dt[B,L,H]  A[H]  Bm[B,L,G,N]  Cm[B,L,G,N]  Q[B,L,H,N]
  *     E[B,L,H,P]  y[B,L,H,P]  dH[B,H,C,N,P]  states[B,H,C,N,P]
  * - dtype selects the element type of x, Bm, Cm, Q, E and of the chunk
  *   memories dH / the decode cache: DART_F32 (float) or DART_BF16
@@ -68,7 +69,8 @@ typedef struct {
     int headdim;  /* P, the value axis */
     int dstate;   /* N, the key axis */
     int chunk;    /* S */
-    int ngroups;  /* must be 1: B and C shared by all heads */
+    int ngroups;  /* G >= 1, dividing nheads: B and C groups of heads; an
+                     invalid count returns DART_ERR_INVALID_ARG */
 } dart_dims;
 
 /*
@@ -106,7 +108,7 @@ size_t dart_ssd_chunk_scan_workspace_bytes(const dart_dims* dims, dart_dtype dty
  *   dH            dtype [B,H,C,N,P] output (rounded to nearest-even for bf16).
  *   states        float [B,H,C,N,P] output.
  *   workspace     device scratch of dart_ssd_chunk_scan_workspace_bytes().
- * Requires ngroups == 1 and (N, P, S, dtype) in the compiled set (see
+ * Requires (N, P, S, dtype) in the compiled set (see
  * dart_supported()).
  */
 dart_status dart_ssd_chunk_scan(const dart_dims* dims, dart_dtype dtype,
@@ -128,7 +130,7 @@ dart_status dart_ssd_chunk_scan(const dart_dims* dims, dart_dtype dtype,
  * C = ceil(L / S) memories and no token attends to the last one.
  *   out = y_ssd + g * o   when y_ssd != NULL (the DART layer output), else
  *   out = o               (the raw readout).
- *   Q[B,L,H,N], E[B,L,H,P], Cm[B,L,N], dH[B,H,C,N,P]: dtype inputs.
+ *   Q[B,L,H,N], E[B,L,H,P], Cm[B,L,G,N], dH[B,H,C,N,P]: dtype inputs.
  *   y_ssd: nullable float [B,L,H,P]; out: float [B,L,H,P], either the same
  *   pointer as y_ssd (updated in place, the fastest form) or not overlapping it
  *   (y_ssd is then copied into out on the stream first).
@@ -189,10 +191,10 @@ size_t dart_ssd_scan_backward_workspace_bytes(const dart_dims* dims);
  *   states: float [B,H,C,N,P] the forward's boundary states;
  *   dy: float [B,L,H,P]; ddH: nullable float [B,H,C,N,P] (NULL = zero), e.g.
  *   dart_sma_backward's memory gradient;
- *   dCm_add: nullable float [B,L,N], added to dCm (NULL = nothing); passing
+ *   dCm_add: nullable float [B,L,G,N], added to dCm (NULL = nothing); passing
  *   dart_sma_backward's dCm gives the layer's C gradient.  It may be dCm
  *   itself (each element is read before it is written);
- *   dx float [B,L,H,P], ddt float [B,L,H], dA float [H], dBm, dCm float [B,L,N];
+ *   dx float [B,L,H,P], ddt float [B,L,H], dA float [H], dBm, dCm float [B,L,G,N] (summed over the heads of each group);
  *   dinit_state: nullable float [B,H,N,P].
  * CUDA cores, one CTA per (b, h); sums in a fixed order (deterministic).
  * Compiled for (N, P) = (128, 64), (64, 64), (16, 16).
@@ -225,9 +227,9 @@ size_t dart_sma_backward_workspace_bytes(const dart_dims* dims);
  *   dC_t = sum_h sum_c p_c w2              dg = sum dy . o
  *   ddH[c] = sum_{t: k(t) > c} (ds_tc / sqrt(N) Q_t E_t^T + p_tc C_t do_t^T)
  * (dy also flows unchanged to y_ssd; that part is the caller's.)
- *   Q[B,L,H,N], E[B,L,H,P], Cm[B,L,N], dH[B,H,C,N,P]: dtype inputs (as given
+ *   Q[B,L,H,N], E[B,L,H,P], Cm[B,L,G,N], dH[B,H,C,N,P]: dtype inputs (as given
  *   to the forward); dy: float [B,L,H,P].
- *   dQ float [B,L,H,N], dE float [B,L,H,P], dCm float [B,L,N],
+ *   dQ float [B,L,H,N], dE float [B,L,H,P], dCm float [B,L,G,N],
  *   ddH float [B,H,C,N,P], dg float [1]: outputs, every element written.
  *   workspace: device scratch of dart_sma_backward_workspace_bytes().
  * CUDA-core kernels; sums run in a fixed order (deterministic).  Shapes and
@@ -257,7 +259,7 @@ size_t dart_decode_step_workspace_bytes(const dart_dims* dims, dart_dtype dtype,
  *   if pos == S-1:  dH_cache[b,h,n] = dH_cur (rounded to dtype);
  *                   dH_cur = 0;  n_chunks[b] = n + 1;  pos[b] = 0
  *   else            pos[b] = pos + 1
- *   x_t[B,H,P], B_t[B,N], C_t[B,N], Q_t[B,H,N], E_t[B,H,P]: dtype inputs;
+ *   x_t[B,H,P], B_t[B,G,N], C_t[B,G,N], Q_t[B,H,N], E_t[B,H,P]: dtype inputs;
  *   dt_t[B,H], A[H]: float inputs.
  *   state, dH_cur: float [B,H,N,P], in/out.
  *   dH_cache: dtype [B,H,cmax,N,P], in/out (slots >= n are not read).

@@ -75,7 +75,8 @@ dart_status check_common(const dart_dims* d, dart_dtype dt, bool need_seqlen) {
     if (dt != DART_F32 && dt != DART_BF16) return fail(DART_ERR_INVALID_ARG, "dtype: unknown value %d", (int)dt);
     if (d->batch < 1 || d->nheads < 1 || d->headdim < 1 || d->dstate < 1 || d->chunk < 1)
         return fail(DART_ERR_INVALID_ARG, "dims: batch, nheads, headdim, dstate and chunk must be >= 1");
-    if (d->ngroups != 1) return fail(DART_ERR_UNSUPPORTED, "ngroups = %d: only 1 (B, C shared by all heads)", d->ngroups);
+    if (d->ngroups < 1 || d->nheads % d->ngroups != 0)
+        return fail(DART_ERR_INVALID_ARG, "ngroups = %d: must be >= 1 and divide nheads = %d", d->ngroups, d->nheads);
     if (need_seqlen) {
         if (d->seqlen < 1) return fail(DART_ERR_INVALID_ARG, "dims: seqlen must be >= 1");
     }
@@ -138,7 +139,7 @@ dart_status dart_ssd_chunk_scan(const dart_dims* d, dart_dtype dtype, const void
     const size_t bhc = (size_t)d->batch * (size_t)d->nheads * (size_t)((d->seqlen + d->chunk - 1) / d->chunk);
     char* hin = static_cast<char*>(workspace) + scan_asum_bytes(bhc);
     float* decay = reinterpret_cast<float*>(hin + bhc * (size_t)d->dstate * (size_t)d->headdim * 2);
-    dart::ScanArgs a{d->batch, d->seqlen, d->nheads, d->headdim, d->dstate, d->chunk,
+    dart::ScanArgs a{d->batch, d->seqlen, d->nheads, d->headdim, d->dstate, d->chunk, d->ngroups,
                      x, dt, A, Bm, Cm, init_state, y_ssd, dH, states, static_cast<float*>(workspace),
                      hin, decay, status_word()};
     if (!a.status) return fail(DART_ERR_CUDA, "dart_ssd_chunk_scan: no device status word");
@@ -164,7 +165,7 @@ dart_status dart_sma_forward(const dart_dims* d, dart_dtype dtype, const void* Q
         if (ya < oa + bytes && oa < ya + bytes)
             return fail(DART_ERR_INVALID_ARG, "dart_sma_forward: out overlaps y_ssd without being the same pointer");
     }
-    dart::SmaArgs a{d->batch, d->seqlen, d->nheads, d->headdim, d->dstate, d->chunk,
+    dart::SmaArgs a{d->batch, d->seqlen, d->nheads, d->headdim, d->dstate, d->chunk, d->ngroups,
                     Q, E, Cm, dH, g, y_ssd, out, status_word()};
     if (!a.status) return fail(DART_ERR_CUDA, "dart_sma_forward: no device status word");
     cudaError_t e = dart::launch_sma(a, dtype, static_cast<cudaStream_t>(stream));
@@ -209,7 +210,7 @@ dart_status dart_sma_forward_decayed(const dart_dims* d, dart_dtype dtype, const
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e = dart::launch_sma_decay_terms(d->batch, d->seqlen, d->nheads, d->chunk, dt, A, la2, gpre, s);
     if (e != cudaSuccess) return cuda_fail(e, "dart_sma_forward_decayed: decay terms");
-    dart::SmaArgs a{d->batch, d->seqlen, d->nheads, d->headdim, d->dstate, d->chunk,
+    dart::SmaArgs a{d->batch, d->seqlen, d->nheads, d->headdim, d->dstate, d->chunk, d->ngroups,
                     Q, E, Cm, dH, g, y_ssd, out, status_word(), la2, gpre};
     if (!a.status) return fail(DART_ERR_CUDA, "dart_sma_forward_decayed: no device status word");
     e = dart::launch_sma(a, dtype, s);
@@ -239,7 +240,7 @@ dart_status dart_ssd_scan_backward(const dart_dims* d, dart_dtype dtype, const v
     const size_t need = dart_ssd_scan_backward_workspace_bytes(d);
     if (workspace_bytes < need)
         return fail(DART_ERR_INVALID_ARG, "workspace: %zu bytes, need %zu", workspace_bytes, need);
-    dart::ScanBwdArgs a{d->batch, d->seqlen, d->nheads, d->headdim, d->dstate, d->chunk, x, dt, A, Bm, Cm,
+    dart::ScanBwdArgs a{d->batch, d->seqlen, d->nheads, d->headdim, d->dstate, d->chunk, d->ngroups, x, dt, A, Bm, Cm,
                         init_state, states, dy, ddH, dCm_add, dx, ddt, dA, dBm, dCm, dinit_state, status_word()};
     if (!a.status) return fail(DART_ERR_CUDA, "dart_ssd_scan_backward: no device status word");
     cudaError_t e = dart::launch_ssd_scan_bwd(a, workspace, dtype, static_cast<cudaStream_t>(stream));
@@ -267,7 +268,7 @@ dart_status dart_sma_backward(const dart_dims* d, dart_dtype dtype, const void* 
     const size_t need = dart_sma_backward_workspace_bytes(d);
     if (workspace_bytes < need)
         return fail(DART_ERR_INVALID_ARG, "workspace: %zu bytes, need %zu", workspace_bytes, need);
-    dart::SmaBwdArgs a{d->batch, d->seqlen, d->nheads, d->headdim, d->dstate, d->chunk, Q, E, Cm, dH, g, dy,
+    dart::SmaBwdArgs a{d->batch, d->seqlen, d->nheads, d->headdim, d->dstate, d->chunk, d->ngroups, Q, E, Cm, dH, g, dy,
                        dQ, dE, dCm, ddH, dg, status_word()};
     if (!a.status) return fail(DART_ERR_CUDA, "dart_sma_backward: no device status word");
     cudaError_t e = dart::launch_sma_bwd(a, workspace, dtype, static_cast<cudaStream_t>(stream));
@@ -300,7 +301,7 @@ dart_status dart_decode_step(const dart_dims* d, dart_dtype dtype, const void* x
     if (workspace_bytes < dart_decode_step_workspace_bytes(d, dtype, cmax))
         return fail(DART_ERR_INVALID_ARG, "workspace: %zu bytes, need %zu", workspace_bytes,
                     dart_decode_step_workspace_bytes(d, dtype, cmax));
-    dart::DecodeArgs a{d->batch, d->nheads, d->headdim, d->dstate, d->chunk, cmax,
+    dart::DecodeArgs a{d->batch, d->nheads, d->headdim, d->dstate, d->chunk, d->ngroups, cmax,
                        dart::decode_num_splits(d->batch, d->nheads, cmax),
                        x_t, dt_t, A, B_t, C_t, Q_t, E_t, g, state, dH_cur, dH_cache,
                        n_chunks, pos, y, static_cast<float*>(workspace), status_word()};
@@ -330,7 +331,7 @@ dart_status dart_decode_step_decayed(const dart_dims* d, dart_dtype dtype, const
     if (workspace_bytes < dart_decode_step_workspace_bytes(d, dtype, cmax))
         return fail(DART_ERR_INVALID_ARG, "workspace: %zu bytes, need %zu", workspace_bytes,
                     dart_decode_step_workspace_bytes(d, dtype, cmax));
-    dart::DecodeArgs a{d->batch, d->nheads, d->headdim, d->dstate, d->chunk, cmax,
+    dart::DecodeArgs a{d->batch, d->nheads, d->headdim, d->dstate, d->chunk, d->ngroups, cmax,
                        dart::decode_num_splits(d->batch, d->nheads, cmax),
                        x_t, dt_t, A, B_t, C_t, Q_t, E_t, g, state, dH_cur, dH_cache,
                        n_chunks, pos, y, static_cast<float*>(workspace), status_word(), mem_logdecay};
@@ -360,7 +361,7 @@ dart_status dart_decode_step_e4m3(const dart_dims* d, dart_dtype dtype, const vo
     if (workspace_bytes < dart_decode_step_workspace_bytes(d, dtype, cmax))
         return fail(DART_ERR_INVALID_ARG, "workspace: %zu bytes, need %zu", workspace_bytes,
                     dart_decode_step_workspace_bytes(d, dtype, cmax));
-    dart::DecodeArgs a{d->batch, d->nheads, d->headdim, d->dstate, d->chunk, cmax,
+    dart::DecodeArgs a{d->batch, d->nheads, d->headdim, d->dstate, d->chunk, d->ngroups, cmax,
                        dart::decode_num_splits(d->batch, d->nheads, cmax),
                        x_t, dt_t, A, B_t, C_t, Q_t, E_t, g, state, dH_cur, cache,
                        n_chunks, pos, y, static_cast<float*>(workspace), status_word(), mem_logdecay, cache_exp};
@@ -434,7 +435,7 @@ dart_status dart_decode_step_noalloc(const dart_dims* d, dart_dtype dtype, const
     void* scratch = nullptr;
     cudaError_t e = dart::noalloc_scratch(&scratch);
     if (e != cudaSuccess) return cuda_fail(e, "dart_decode_step_noalloc: static scratch address");
-    dart::DecodeArgs a{d->batch, d->nheads, d->headdim, d->dstate, d->chunk, cmax,
+    dart::DecodeArgs a{d->batch, d->nheads, d->headdim, d->dstate, d->chunk, d->ngroups, cmax,
                        dart::decode_num_splits(d->batch, d->nheads, cmax),
                        x_t, dt_t, A, B_t, C_t, Q_t, E_t, g, state, dH_cur, dH_cache,
                        n_chunks, pos, y, static_cast<float*>(scratch), status_word()};

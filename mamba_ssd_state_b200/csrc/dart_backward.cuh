@@ -7,10 +7,10 @@
 namespace dart {
 
 struct SmaBwdArgs {
-    int B, L, H, P, N, S;
+    int B, L, H, P, N, S, G;
     const void* Q; const void* E; const void* Cm; const void* dH;
     float g; const float* dy;               // dy: [B,L,H,P] gradient of the layer output
-    float* dQ; float* dE; float* dCm; float* ddH; float* dg;   // outputs (fp32)
+    float* dQ; float* dE; float* dCm; float* ddH; float* dg;   // outputs (fp32); dCm [B,L,G,N]
     int* status;
     // workspace views (set by launch_sma_bwd)
     float* pbuf; float* dsbuf;              // [B,H,L,C] softmax weights and score gradients
@@ -19,14 +19,14 @@ struct SmaBwdArgs {
 };
 
 struct ScanBwdArgs {
-    int B, L, H, P, N, S;
+    int B, L, H, P, N, S, G;
     const void* x; const float* dt; const float* A; const void* Bm; const void* Cm;
     const float* init;      // nullable [B,H,N,P] initial state of the forward
     const float* states;    // [B,H,C,N,P] boundary states written by the forward
     const float* dy;        // [B,L,H,P] gradient of y_ssd
     const float* ddH;       // nullable [B,H,C,N,P] gradient of the chunk memories
-    const float* dC_add;    // nullable [B,L,N]: added to dC (e.g. the SMA backward's part; may be dC)
-    float* dx; float* ddt; float* dA; float* dB; float* dC;   // outputs (fp32)
+    const float* dC_add;    // nullable [B,L,G,N]: added to dC (e.g. the SMA backward's part; may be dC)
+    float* dx; float* ddt; float* dA; float* dB; float* dC;   // outputs (fp32); dB, dC [B,L,G,N]
     float* dinit;           // nullable [B,H,N,P] output
     int* status;
     // workspace views (set by launch_ssd_scan_bwd)

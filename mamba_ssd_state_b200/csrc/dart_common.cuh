@@ -99,8 +99,13 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 // Host-side launch helpers implemented per kernel family.
 namespace dart {
+// B and C are shared by groups of heads (Mamba-2 ngroups): with G groups
+// (G divides H) they are [B, L, G, N] and head h reads group h / (H / G);
+// G = 1 is the [B, L, N] layout shared by all heads.
+__host__ __device__ __forceinline__ int group_of(int h, int H, int G) { return h / (H / G); }
+
 struct ScanArgs {
-    int B, L, H, P, N, S;
+    int B, L, H, P, N, S, G;
     const void* x; const float* dt; const float* A; const void* Bm; const void* Cm;
     const float* init_state;
     float* y; void* dH; float* states; float* asum;  // asum: [B,H,C] workspace
@@ -109,7 +114,7 @@ struct ScanArgs {
     int* status;  // device status word
 };
 struct SmaArgs {
-    int B, L, H, P, N, S;
+    int B, L, H, P, N, S, G;
     const void* Q; const void* E; const void* Cm; const void* dH;
     float g; const float* y_ssd; float* out;
     int* status;  // device status word
@@ -120,7 +125,7 @@ struct SmaArgs {
     const double* gpre;   // [B,H,C] fp64
 };
 struct DecodeArgs {
-    int B, H, P, N, S, cmax, nsplit;
+    int B, H, P, N, S, G, cmax, nsplit;
     const void* x; const float* dt; const float* A; const void* Bm; const void* Cm;
     const void* Q; const void* E; float g;
     float* state; float* dHcur; void* cache; int* nchunks; int* pos; float* y;

@@ -92,8 +92,9 @@ __global__ void __launch_bounds__(kThreads) decode_partial_kernel(DecodeArgs a) 
 
     const size_t bh = (size_t)b * a.H + h;
     const T* xt = static_cast<const T*>(a.x) + bh * P;
-    const T* Bt = static_cast<const T*>(a.Bm) + (size_t)b * N;
-    const T* Ct = static_cast<const T*>(a.Cm) + (size_t)b * N;
+    const size_t bg = (size_t)b * a.G + group_of(h, a.H, a.G);   // B_t, C_t are [B, G, N]
+    const T* Bt = static_cast<const T*>(a.Bm) + bg * N;
+    const T* Ct = static_cast<const T*>(a.Cm) + bg * N;
     const T* Qt = static_cast<const T*>(a.Q) + bh * N;
     const T* Et = static_cast<const T*>(a.E) + bh * P;
     const float qscale = kLog2e * rsqrtf((float)N);
@@ -335,8 +336,9 @@ __global__ void __launch_bounds__(kThreads) decode_partial_e4m3_kernel(DecodeArg
 
     const size_t bh = (size_t)b * a.H + h;
     const T* xt = static_cast<const T*>(a.x) + bh * P;
-    const T* Bt = static_cast<const T*>(a.Bm) + (size_t)b * N;
-    const T* Ct = static_cast<const T*>(a.Cm) + (size_t)b * N;
+    const size_t bg = (size_t)b * a.G + group_of(h, a.H, a.G);   // B_t, C_t are [B, G, N]
+    const T* Bt = static_cast<const T*>(a.Bm) + bg * N;
+    const T* Ct = static_cast<const T*>(a.Cm) + bg * N;
     const T* Qt = static_cast<const T*>(a.Q) + bh * N;
     const T* Et = static_cast<const T*>(a.E) + bh * P;
     const float qscale = kLog2e * rsqrtf((float)N);

@@ -59,7 +59,7 @@ __global__ void __launch_bounds__(kRowThreads) sma_bwd_rows(SmaBwdArgs a) {
         const bool in = t0 + r < L;
         const size_t tok = (size_t)b * L + t0 + r;
         Qs[r * NS + n] = in ? ldf(Q + (tok * H + h) * N + n) : 0.f;
-        Cs[r * NS + n] = in ? ldf(Cm + tok * N + n) : 0.f;
+        Cs[r * NS + n] = in ? ldf(Cm + (tok * a.G + group_of(h, H, a.G)) * N + n) : 0.f;
     }
     for (int i = threadIdx.x; i < kTQ * P; i += blockDim.x) {
         const int r = i / P, p = i % P;
@@ -237,7 +237,7 @@ __global__ void __launch_bounds__(256) sma_bwd_memories(SmaBwdArgs a) {
             const bool in = tb + r < L;
             const size_t tok = (size_t)b * L + tb + r;
             Qs[i] = in ? ldf(Q + (tok * H + h) * N + nn) : 0.f;
-            Cs[i] = in ? ldf(Cm + tok * N + nn) : 0.f;
+            Cs[i] = in ? ldf(Cm + (tok * a.G + group_of(h, H, a.G)) * N + nn) : 0.f;
         }
         for (int i = threadIdx.x; i < TT * P; i += blockDim.x) {
             const int r = i / P, pp = i % P;
@@ -264,12 +264,14 @@ __global__ void __launch_bounds__(256) sma_bwd_memories(SmaBwdArgs a) {
     for (int j = 0; j < CPT; ++j) out[j] = acc[j];
 }
 
+// dC [B,L,G,N]: the per-head parts summed over the heads of each group
 __global__ void sma_bwd_reduce_dc(SmaBwdArgs a, int N) {
-    const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;   // over B * L * N
-    if (i >= (size_t)a.B * a.L * N) return;
-    const size_t tok = i / N, n = i % N;
+    const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;   // over B * L * G * N
+    if (i >= (size_t)a.B * a.L * a.G * N) return;
+    const size_t tok = i / ((size_t)a.G * N), n = i % N;
+    const int g = (int)((i / N) % a.G), hg = a.H / a.G;
     float sum = 0.f;
-    for (int h = 0; h < a.H; ++h) sum += a.dCh[(tok * a.H + h) * N + n];
+    for (int h = g * hg; h < (g + 1) * hg; ++h) sum += a.dCh[(tok * a.H + h) * N + n];
     a.dCm[i] = sum;
 }
 
@@ -296,7 +298,7 @@ cudaError_t run(const SmaBwdArgs& a, cudaStream_t st) {
         return e;
     k2<<<dim3(C, a.H, a.B), 256, smem_mem, st>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    const size_t ndc = (size_t)a.B * a.L * N;
+    const size_t ndc = (size_t)a.B * a.L * a.G * N;
     sma_bwd_reduce_dc<<<(unsigned)((ndc + 255) / 256), 256, 0, st>>>(a, N);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     sma_bwd_reduce_dg<<<1, 32, 0, st>>>(a, a.B * a.H * tiles);

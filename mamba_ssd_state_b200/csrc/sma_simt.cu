@@ -62,7 +62,7 @@ __global__ void __launch_bounds__(kThreads) sma_simt_kernel(SmaArgs a) {
             const bool in = t0 + r < a.L;
             const size_t tok = (size_t)b * a.L + t0 + r;
             Qs[r * NS + n] = in ? qscale * ldf(Q + (tok * a.H + h) * N + n) : 0.f;
-            Cs[r * NS + n] = in ? ldf(Cm + tok * N + n) : 0.f;
+            Cs[r * NS + n] = in ? ldf(Cm + (tok * a.G + group_of(h, a.H, a.G)) * N + n) : 0.f;
         }
         const T* mem = dH + ((size_t)b * a.H + h) * (size_t)C * N * P;
         for (int c = 0; c < k; ++c) {

@@ -105,7 +105,7 @@ struct SmaTcParams {
     // that runs past the end of a partial last chunk reads zeros and writes
     // nothing there.
     CUtensorMap tmap_q;  // Q viewed as dims (N, H, L, B), box (64, 1, 128, 1)
-    CUtensorMap tmap_c;  // Cm viewed as dims (N, L, B)
+    CUtensorMap tmap_c;  // Cm viewed as dims (N, G, L, B), box (64, 1, 128, 1)
     CUtensorMap tmap_h;  // dH viewed as dims (P, B*H*C*N)
     CUtensorMap tmap_e;  // E viewed as dims (P, H, L, B), box (64, 1, 128, 1): L2 prefetch only
     CUtensorMap tmap_o;  // out viewed as dims (P, H, L, B) fp32, box (32, 1, 128, 1): reduce-add / store
@@ -117,6 +117,7 @@ struct SmaTcParams {
     float g;
     int add_into_out;  // 1: out already holds y_ssd, the tile end adds g o / l; 0: it stores o / l
     int B, L, H, S, C;
+    int HG;            // heads per group sharing C (head h reads group h / HG)
     int cta_per_tile;  // 1, or 2 for a CTA pair (each CTA 128 of the tile's 256 rows)
     int tiles_per_chunk, total_tiles;
     int* status;
@@ -252,11 +253,11 @@ __global__ void __launch_bounds__(kThreads, 1) sma_tc_kernel(const __grid_consta
             if (lane == 0) {
                 if (rank == 0) mbar_expect_tx(bar(C_FULL), 2 * kHalfA * (kPair ? 2 : 1));
                 if (kPair) {
-                    tma_load_3d_pair(sbase + kOffC, &p.tmap_c, bar_lead(C_FULL), 0, row, t.b);
-                    tma_load_3d_pair(sbase + kOffC + kHalfA, &p.tmap_c, bar_lead(C_FULL), 64, row, t.b);
+                    tma_load_4d_pair(sbase + kOffC, &p.tmap_c, bar_lead(C_FULL), 0, t.h / p.HG, row, t.b);
+                    tma_load_4d_pair(sbase + kOffC + kHalfA, &p.tmap_c, bar_lead(C_FULL), 64, t.h / p.HG, row, t.b);
                 } else {
-                    tma_load_3d(sbase + kOffC, &p.tmap_c, bar(C_FULL), 0, row, t.b);
-                    tma_load_3d(sbase + kOffC + kHalfA, &p.tmap_c, bar(C_FULL), 64, row, t.b);
+                    tma_load_4d(sbase + kOffC, &p.tmap_c, bar(C_FULL), 0, t.h / p.HG, row, t.b);
+                    tma_load_4d(sbase + kOffC + kHalfA, &p.tmap_c, bar(C_FULL), 64, t.h / p.HG, row, t.b);
                 }
                 // the next tile's rows start moving into L2 now: its Q and C
                 // (if it has memories), the E rows its epilogue starts from
@@ -267,8 +268,8 @@ __global__ void __launch_bounds__(kThreads, 1) sma_tc_kernel(const __grid_consta
                     if (tn.k > 0) {
                         tma_prefetch_4d(&p.tmap_q, 0, tn.h, rown, tn.b);
                         tma_prefetch_4d(&p.tmap_q, 64, tn.h, rown, tn.b);
-                        tma_prefetch_3d(&p.tmap_c, 0, rown, tn.b);
-                        tma_prefetch_3d(&p.tmap_c, 64, rown, tn.b);
+                        tma_prefetch_4d(&p.tmap_c, 0, tn.h / p.HG, rown, tn.b);
+                        tma_prefetch_4d(&p.tmap_c, 64, tn.h / p.HG, rown, tn.b);
                         tma_prefetch_4d(&p.tmap_e, 0, tn.h, rown, tn.b);
                     }
                     if (p.add_into_out && tn.k > 0) {
@@ -592,10 +593,10 @@ cudaError_t launch_sma_tc(const SmaArgs& a, cudaStream_t st) {
         if (!encode_tile_map_bf16(&p.tmap_q, 4, a.Q, dims, strides, box)) return cudaErrorInvalidValue;
     }
     {
-        const uint64_t dims[3] = {(uint64_t)kN, (uint64_t)a.L, (uint64_t)a.B};
-        const uint64_t strides[2] = {(uint64_t)kN * 2, (uint64_t)a.L * kN * 2};
-        const uint32_t box[3] = {64, kBQ, 1};
-        if (!encode_tile_map_bf16(&p.tmap_c, 3, a.Cm, dims, strides, box)) return cudaErrorInvalidValue;
+        const uint64_t dims[4] = {(uint64_t)kN, (uint64_t)a.G, (uint64_t)a.L, (uint64_t)a.B};
+        const uint64_t strides[3] = {(uint64_t)kN * 2, (uint64_t)a.G * kN * 2, (uint64_t)a.L * a.G * kN * 2};
+        const uint32_t box[4] = {64, 1, kBQ, 1};
+        if (!encode_tile_map_bf16(&p.tmap_c, 4, a.Cm, dims, strides, box)) return cudaErrorInvalidValue;
     }
     {
         const uint64_t dims[2] = {(uint64_t)kP, (uint64_t)a.B * a.H * C * kN};
@@ -631,6 +632,7 @@ cudaError_t launch_sma_tc(const SmaArgs& a, cudaStream_t st) {
         if (ce != cudaSuccess) return ce;
     }
     p.B = a.B; p.L = a.L; p.H = a.H; p.S = a.S; p.C = C;
+    p.HG = a.H / a.G;
     p.status = a.status;
     const int sms = sm_count();
     if (sms <= 0) return cudaErrorInvalidDevice;

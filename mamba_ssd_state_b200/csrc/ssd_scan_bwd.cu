@@ -64,8 +64,9 @@ __global__ void __launch_bounds__(N * P / kCols) ssd_scan_bwd_kernel(ScanBwdArgs
             const int r = i / N, nn = i % N;
             const bool in = tb + r < L;
             const size_t tok = (size_t)b * L + tb + r;
-            Bs[i] = in ? ldf(Bm + tok * N + nn) : 0.f;
-            Cs[i] = in ? ldf(Cm + tok * N + nn) : 0.f;
+            const size_t tg = tok * a.G + group_of(h, H, a.G);   // B and C of this head's group
+            Bs[i] = in ? ldf(Bm + tg * N + nn) : 0.f;
+            Cs[i] = in ? ldf(Cm + tg * N + nn) : 0.f;
         }
         for (int i = tid; i < kTT * P; i += NT) {
             const int r = i / P, pp = i % P;
@@ -205,15 +206,16 @@ __global__ void __launch_bounds__(N * P / kCols) ssd_scan_bwd_kernel(ScanBwdArgs
     if (tid == 0) a.dApart[bh] = dA_acc;
 }
 
-// dB, dC summed over heads (dC plus dC_add when given); dA summed over the
-// batch (fixed order).
+// dB, dC [B,L,G,N] summed over the heads of each group (dC plus dC_add when
+// given); dA summed over the batch (fixed order).
 __global__ void scan_bwd_reduce(ScanBwdArgs a, int N) {
     const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const size_t nbc = (size_t)a.B * a.L * N;
+    const size_t nbc = (size_t)a.B * a.L * a.G * N;
     if (i < nbc) {
-        const size_t tok = i / N, nn = i % N;
+        const size_t tok = i / ((size_t)a.G * N), nn = i % N;
+        const int g = (int)((i / N) % a.G), hg = a.H / a.G;
         float sb = 0.f, sc = 0.f;
-        for (int h = 0; h < a.H; ++h) {
+        for (int h = g * hg; h < (g + 1) * hg; ++h) {
             sb += a.dBh[(tok * a.H + h) * N + nn];
             sc += a.dCh[(tok * a.H + h) * N + nn];
         }
@@ -237,7 +239,7 @@ cudaError_t run(const ScanBwdArgs& a, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     k<<<dim3(a.H, a.B), NT, smem, st>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    const size_t n = (size_t)a.B * a.L * N;
+    const size_t n = (size_t)a.B * a.L * a.G * N;
     const size_t m = n > (size_t)a.H ? n : (size_t)a.H;
     scan_bwd_reduce<<<(unsigned)((m + 255) / 256), 256, 0, st>>>(a, N);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;

@@ -82,7 +82,7 @@ __global__ void __launch_bounds__(kThreads) chunk_state_kernel(ScanArgs a) {
         for (int e = threadIdx.x; e < TS * N; e += blockDim.x) {
             const int s = e / N, n = e % N;
             const int t = t0 + s0 + s;
-            Bs[e] = t < a.L ? ldf(Bm + ((size_t)b * a.L + t) * N + n) : 0.f;
+            Bs[e] = t < a.L ? ldf(Bm + (((size_t)b * a.L + t) * a.G + group_of(h, a.H, a.G)) * N + n) : 0.f;
         }
         for (int e = threadIdx.x; e < TS * P; e += blockDim.x) {
             const int s = e / P, p = e % P;
@@ -161,7 +161,7 @@ __global__ void __launch_bounds__(kThreads) chunk_output_kernel(ScanArgs a) {
     for (int e = threadIdx.x; e < TQ * N; e += blockDim.x) {
         const int t = e / N, n = e % N;
         const int tok = t0 + q0 + t;
-        Cs[t * NP + n] = tok < a.L ? ldf(Cm + ((size_t)b * a.L + tok) * N + n) : 0.f;
+        Cs[t * NP + n] = tok < a.L ? ldf(Cm + (((size_t)b * a.L + tok) * a.G + group_of(h, a.H, a.G)) * N + n) : 0.f;
     }
     const int tl = threadIdx.x / 4, pg = threadIdx.x % 4;
     const int tq = q0 + tl;            // chunk-local query index
@@ -174,7 +174,7 @@ __global__ void __launch_bounds__(kThreads) chunk_output_kernel(ScanArgs a) {
         for (int e = threadIdx.x; e < TS * N; e += blockDim.x) {
             const int s = e / N, n = e % N;
             const int t = t0 + s0 + s;
-            Bs[s * NP + n] = t < a.L ? ldf(Bm + ((size_t)b * a.L + t) * N + n) : 0.f;
+            Bs[s * NP + n] = t < a.L ? ldf(Bm + (((size_t)b * a.L + t) * a.G + group_of(h, a.H, a.G)) * N + n) : 0.f;
         }
         for (int e = threadIdx.x; e < TS * P; e += blockDim.x) {
             const int s = e / P, p = e % P;

@@ -9,7 +9,7 @@
 //      and three per-token decay terms the other kernels bulk-copy.
 //  chunk_state_tc  persistent, one CTA per SM over equal shares of the
 //      (b, c, h) items.  The chunk's B tile (S x N) is loaded once and shared
-//      by the heads that follow (B is the same for all heads, ngroups = 1).
+//      by the heads that follow (B is the same for the heads of a group).
 //      Per head the x tile (S x P) is scaled in shared memory by
 //      w_s = exp(Acum_e - Acum_s) dt_s and
 //        dH[c] = B^T (w o x)      (M = N = 128, N_mma = P = 64, K = S)
@@ -22,8 +22,8 @@
 //        G = C B^T,  P[t,s] = G[t,s] exp(Acum_t - Acum_s) dt_s (s <= t),
 //        Y_diag = P x,  Y_off = C hin[c].
 //      Persistent, one CTA per SM over cost-balanced ranges of the
-//      (b, c, 128-row half, h) items.  G is computed once per (b, c, half)
-//      into TMEM and shared by the heads; the P builders read it from TMEM
+//      (b, c, 128-row half, h) items.  G is computed once per (b, c, half,
+//      group) into TMEM and shared by its heads; the P builders read it from TMEM
 //      and write P (bf16) in 64-column panels, each handed to the MMA by its
 //      own barrier pair.
 //
@@ -50,8 +50,8 @@ constexpr int kScanMaxCtas = 160;                    // largest persistent grid 
 
 struct ScanTcParams {
     CUtensorMap tmap_x;    // x  as (P, B*L, H), box (64, 128, 1)
-    CUtensorMap tmap_b;    // Bm as (N, B*L),    box (64, 128)
-    CUtensorMap tmap_c;    // Cm as (N, B*L),    box (64, 128)
+    CUtensorMap tmap_b;    // Bm as (N, G, L, B), box (64, 1, 128, 1)
+    CUtensorMap tmap_c;    // Cm as (N, G, L, B), box (64, 1, 128, 1)
     CUtensorMap tmap_hin;  // hin as (P, B*H*C*N), box (64, 128)
     CUtensorMap tmap_dh;   // dH as (P, B*H*C*N) bf16, box (64, 128): chunk_state's store
     CUtensorMap tmap_y;    // y as (P, H, L, B) fp32, box (32, 1, 128, 1): chunk_output's store
@@ -71,6 +71,7 @@ struct ScanTcParams {
     float* colf;
     float* wst;
     int B, L, H, S, C;
+    int G, HG;             // groups of heads sharing B and C, heads per group
     int co_range[kScanMaxCtas + 1];  // chunk_output: CTA r runs items co_range[r] .. co_range[r + 1] - 1
     int* status;
 };
@@ -228,15 +229,15 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_state_tc_kernel(const __gri
         for (int i = 0; i < n_items; ++i) {
             const Item it = cs_item(p, j0 + i);
             const int t0 = it.c * S;                  // first token of the chunk
-            if (i == 0 || it.h == 0) {
-                // a new chunk: its B tile, once the MMAs on the previous one are done
+            if (i == 0 || it.h % p.HG == 0) {
+                // a new chunk or group: its B tile, once the MMAs on the previous one are done
                 if (b_loads > 0 && !mbar_wait_warp(bar(B_FREE), (uint32_t)(b_loads - 1) & 1u, wc, 7)) break;
                 if (lane == 0) {
                     mbar_expect_tx(bar(B_FULL), 2 * S * kRowBytes);
                     for (int pnl = 0; pnl < 2; ++pnl)
                         for (int r = 0; r < S / 128; ++r)
-                            tma_load_3d(sbase + Ly::kOffB + (uint32_t)pnl * S * kRowBytes + (uint32_t)r * kBox,
-                                        &p.tmap_b, bar(B_FULL), 64 * pnl, t0 + 128 * r, it.b);
+                            tma_load_4d(sbase + Ly::kOffB + (uint32_t)pnl * S * kRowBytes + (uint32_t)r * kBox,
+                                        &p.tmap_b, bar(B_FULL), 64 * pnl, it.h / p.HG, t0 + 128 * r, it.b);
                 }
                 ++b_loads;
             }
@@ -261,12 +262,12 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_state_tc_kernel(const __gri
         int b_loads = 0;
         for (int i = 0; i < n_items && ok; ++i) {
             const Item it = cs_item(p, j0 + i);
-            if (i == 0 || it.h == 0) {
+            if (i == 0 || it.h % p.HG == 0) {
                 if (!(ok = mbar_wait_warp(bar(B_FULL), (uint32_t)b_loads & 1u, wc, 2))) break;
                 ++b_loads;
             }
             // the last item on this B tile releases it after its MMAs
-            const bool last_on_b = i + 1 == n_items || it.h == p.H - 1;
+            const bool last_on_b = i + 1 == n_items || (it.h + 1) % p.HG == 0;
             const int xs = i % kSt, a = i & 1;
             const uint32_t ph = (uint32_t)(i / kSt) & 1u;
             const uint32_t aph = (uint32_t)(i >> 1) & 1u;
@@ -477,8 +478,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_output_tc_kernel(const __gr
     const int S = p.S;
     const int j0 = p.co_range[blockIdx.x];
     const int n_items = p.co_range[blockIdx.x + 1] - j0;
-    auto group_first = [&](int i, const Item& it) { return i == 0 || it.h == 0; };
-    auto group_last = [&](int i, const Item& it) { return i + 1 == n_items || it.h == p.H - 1; };
+    // a group shares C rows, B rows and G: one (b, c, half) and one group of heads
+    auto group_first = [&](int i, const Item& it) { return i == 0 || it.h % p.HG == 0; };
+    auto group_last = [&](int i, const Item& it) { return i + 1 == n_items || (it.h + 1) % p.HG == 0; };
 
     if (threadIdx.x == 0) {
         mbar_init(bar(IN_FULL), 1);
@@ -530,11 +532,11 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_output_tc_kernel(const __gr
                 if (lane == 0) {
                     mbar_expect_tx(bar(IN_FULL), 2 * kBox + 2 * (uint32_t)KS * kRowBytes);
                     for (int pnl = 0; pnl < 2; ++pnl) {
-                        tma_load_3d(sbase + kOffC + (uint32_t)pnl * kBox, &p.tmap_c, bar(IN_FULL), 64 * pnl,
-                                    t0 + 128 * it.half, it.b);
+                        tma_load_4d(sbase + kOffC + (uint32_t)pnl * kBox, &p.tmap_c, bar(IN_FULL), 64 * pnl,
+                                    it.h / p.HG, t0 + 128 * it.half, it.b);
                         for (int r = 0; r < KS / 128; ++r)
-                            tma_load_3d(sbase + kOffBP + (uint32_t)pnl * KS * kRowBytes + (uint32_t)r * kBox,
-                                        &p.tmap_b, bar(IN_FULL), 64 * pnl, t0 + 128 * r, it.b);
+                            tma_load_4d(sbase + kOffBP + (uint32_t)pnl * KS * kRowBytes + (uint32_t)r * kBox,
+                                        &p.tmap_b, bar(IN_FULL), 64 * pnl, it.h / p.HG, t0 + 128 * r, it.b);
                     }
                 }
                 ++ng;
@@ -815,11 +817,11 @@ bool make_maps(const ScanArgs& a, ScanTcParams& p) {
         if (!encode_tile_map_bf16(&p.tmap_x, 4, a.x, dims, strides, box)) return false;
     }
     {
-        const uint64_t dims[3] = {(uint64_t)kN, (uint64_t)a.L, (uint64_t)a.B};
-        const uint64_t strides[2] = {(uint64_t)kN * 2, (uint64_t)a.L * kN * 2};
-        const uint32_t box[3] = {64, 128, 1};
-        if (!encode_tile_map_bf16(&p.tmap_b, 3, a.Bm, dims, strides, box)) return false;
-        if (!encode_tile_map_bf16(&p.tmap_c, 3, a.Cm, dims, strides, box)) return false;
+        const uint64_t dims[4] = {(uint64_t)kN, (uint64_t)a.G, (uint64_t)a.L, (uint64_t)a.B};
+        const uint64_t strides[3] = {(uint64_t)kN * 2, (uint64_t)a.G * kN * 2, (uint64_t)a.L * a.G * kN * 2};
+        const uint32_t box[4] = {64, 1, 128, 1};
+        if (!encode_tile_map_bf16(&p.tmap_b, 4, a.Bm, dims, strides, box)) return false;
+        if (!encode_tile_map_bf16(&p.tmap_c, 4, a.Cm, dims, strides, box)) return false;
     }
     {
         const uint64_t dims[2] = {(uint64_t)kP, (uint64_t)a.B * a.H * C * kN};
@@ -856,6 +858,7 @@ cudaError_t launch_ssd_scan_tc(const ScanArgs& a, cudaStream_t st) {
     p.hin = static_cast<__nv_bfloat16*>(a.hin);
     p.y = a.y;
     p.B = a.B; p.L = a.L; p.H = a.H; p.S = a.S; p.C = (a.L + a.S - 1) / a.S;
+    p.G = a.G; p.HG = a.H / a.G;
     const size_t bhcs = (size_t)a.B * a.H * p.C * a.S;   // decay arrays are [B, H, C, S]
     p.a2 = a.decay;
     p.colf = a.decay + bhcs;
@@ -910,7 +913,7 @@ cudaError_t launch_ssd_scan_tc(const ScanArgs& a, cudaStream_t st) {
         if (items < grid) grid = items;
         auto cost = [&](int j) {
             const int half = (j / a.H) % R;
-            return (half == 0 ? 2 : 4) + (j % a.H == 0 ? 2 : 0);
+            return (half == 0 ? 2 : 4) + ((j % a.H) % (a.H / a.G) == 0 ? 2 : 0);
         };
         long long total = 0;
         for (int j = 0; j < items; ++j) total += cost(j);

@@ -174,6 +174,22 @@ def _shape(name, t, shape):
         raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
 
 
+def _bc_groups(name, t, lead, H) -> int:
+    """Number of B/C groups of a B or C tensor: shape lead + (N,) is one group
+    shared by all heads, lead + (G, N) is G groups (G divides H, head h reads
+    group h // (H // G))."""
+    if t.dim() == len(lead) + 1:
+        _shape(name, t, (*lead, t.shape[-1]))
+        return 1
+    if t.dim() == len(lead) + 2:
+        G = t.shape[-2]
+        _shape(name, t, (*lead, G, t.shape[-1]))
+        if G < 1 or H % G:
+            raise ValueError(f"{name}: {G} groups do not divide {H} heads")
+        return G
+    raise ValueError(f"{name}: expected shape {tuple(lead)} + ([G,] N), got {tuple(t.shape)}")
+
+
 def supported(dstate: int, headdim: int, chunk: int, dtype: torch.dtype) -> bool:
     return bool(load().dart_supported(dstate, headdim, chunk, _dtype_code(dtype)))
 
@@ -197,7 +213,8 @@ def dart_ssd_chunk_scan(x, dt, A, Bm, Cm, chunk: int, init_state=None, *, y_ssd=
                         states=None, workspace=None):
     """SSD chunked scan keeping the chunk memories.
 
-    x[B,L,H,P], Bm/Cm[B,L,N] (float32 or bfloat16), dt[B,L,H] and A[H] float32,
+    x[B,L,H,P], Bm/Cm[B,L,N] or [B,L,G,N] with G groups of heads (head h
+    reads group h // (H // G)) (float32 or bfloat16), dt[B,L,H] and A[H] float32,
     init_state optional float32 [B,H,N,P].  Returns (y_ssd float32 [B,L,H,P],
     dH [B,H,C,N,P] in x's dtype, states float32 [B,H,C,N,P]).  Optional
     preallocated outputs/workspace avoid allocation in timed loops."""
@@ -209,12 +226,14 @@ def dart_ssd_chunk_scan(x, dt, A, Bm, Cm, chunk: int, init_state=None, *, y_ssd=
     init_state = _dev(init_state, dev, torch.float32)
     Bsz, L, H, P = x.shape
     N = Bm.shape[-1]
-    _shape("dt", dt, (Bsz, L, H)); _shape("A", A, (H,)); _shape("Bm", Bm, (Bsz, L, N))
-    _shape("Cm", Cm, (Bsz, L, N))
+    _shape("dt", dt, (Bsz, L, H)); _shape("A", A, (H,))
+    G = _bc_groups("Bm", Bm, (Bsz, L), H)
+    if _bc_groups("Cm", Cm, (Bsz, L), H) != G or Cm.shape != Bm.shape:
+        raise ValueError("Bm and Cm must have the same shape")
     if init_state is not None:
         _shape("init_state", init_state, (Bsz, H, N, P))
     C = -(-L // chunk)   # a partial last chunk counts
-    dims = Dims(Bsz, L, H, P, N, chunk, 1)
+    dims = Dims(Bsz, L, H, P, N, chunk, G)
     code = _dtype_code(x.dtype)
     if y_ssd is None:
         y_ssd = torch.empty((Bsz, L, H, P), device=dev, dtype=torch.float32)
@@ -245,12 +264,13 @@ def dart_sma_forward(Q, E, Cm, dH, chunk: int, g: float, y_ssd=None, *, out=None
     Bsz, L, H, N = Q.shape
     P = E.shape[-1]
     C = -(-L // chunk)   # a partial last chunk counts
-    _shape("E", E, (Bsz, L, H, P)); _shape("Cm", Cm, (Bsz, L, N)); _shape("dH", dH, (Bsz, H, C, N, P))
+    _shape("E", E, (Bsz, L, H, P)); _shape("dH", dH, (Bsz, H, C, N, P))
+    G = _bc_groups("Cm", Cm, (Bsz, L), H)
     if y_ssd is not None:
         _shape("y_ssd", y_ssd, (Bsz, L, H, P))
     if out is None:
         out = torch.empty((Bsz, L, H, P), device=dev, dtype=torch.float32)
-    dims = Dims(Bsz, L, H, P, N, chunk, 1)
+    dims = Dims(Bsz, L, H, P, N, chunk, G)
     with torch.cuda.device(dev):
         _check(lib.dart_sma_forward(ctypes.byref(dims), _dtype_code(Q.dtype), _ptr(Q), _ptr(E), _ptr(Cm),
                                     _ptr(dH), float(g), _ptr(y_ssd), _ptr(out), _stream()))
@@ -271,13 +291,14 @@ def dart_sma_forward_decayed(Q, E, Cm, dH, dt, A, chunk: int, g: float, y_ssd=No
     Bsz, L, H, N = Q.shape
     P = E.shape[-1]
     C = -(-L // chunk)
-    _shape("E", E, (Bsz, L, H, P)); _shape("Cm", Cm, (Bsz, L, N)); _shape("dH", dH, (Bsz, H, C, N, P))
+    _shape("E", E, (Bsz, L, H, P)); _shape("dH", dH, (Bsz, H, C, N, P))
+    G = _bc_groups("Cm", Cm, (Bsz, L), H)
     _shape("dt", dt, (Bsz, L, H)); _shape("A", A, (H,))
     if y_ssd is not None:
         _shape("y_ssd", y_ssd, (Bsz, L, H, P))
     if out is None:
         out = torch.empty((Bsz, L, H, P), device=dev, dtype=torch.float32)
-    dims = Dims(Bsz, L, H, P, N, chunk, 1)
+    dims = Dims(Bsz, L, H, P, N, chunk, G)
     wsb = lib.dart_sma_decayed_workspace_bytes(ctypes.byref(dims))
     if workspace is None:
         workspace = torch.empty(max(16, wsb), device=dev, dtype=torch.uint8)
@@ -300,11 +321,12 @@ def dart_sma_backward(Q, E, Cm, dH, chunk: int, g: float, dy, *, workspace=None)
     Bsz, L, H, N = Q.shape
     P = E.shape[-1]
     C = -(-L // chunk)
-    _shape("E", E, (Bsz, L, H, P)); _shape("Cm", Cm, (Bsz, L, N)); _shape("dH", dH, (Bsz, H, C, N, P))
+    _shape("E", E, (Bsz, L, H, P)); _shape("dH", dH, (Bsz, H, C, N, P))
+    G = _bc_groups("Cm", Cm, (Bsz, L), H)
     _shape("dy", dy, (Bsz, L, H, P))
-    dims = Dims(Bsz, L, H, P, N, chunk, 1)
+    dims = Dims(Bsz, L, H, P, N, chunk, G)
     out = {"dQ": torch.empty((Bsz, L, H, N), device=dev), "dE": torch.empty((Bsz, L, H, P), device=dev),
-           "dCm": torch.empty((Bsz, L, N), device=dev), "ddH": torch.empty((Bsz, H, C, N, P), device=dev),
+           "dCm": torch.empty(tuple(Cm.shape), device=dev), "ddH": torch.empty((Bsz, H, C, N, P), device=dev),
            "dg": torch.empty((1,), device=dev)}
     wsb = lib.dart_sma_backward_workspace_bytes(ctypes.byref(dims))
     if workspace is None:
@@ -338,12 +360,15 @@ def dart_ssd_scan_backward(x, dt, A, Bm, Cm, chunk: int, states, dy, ddH=None, i
     _shape("states", states, (Bsz, H, C, N, P)); _shape("dy", dy, (Bsz, L, H, P))
     if ddH is not None:
         _shape("ddH", ddH, (Bsz, H, C, N, P))
+    G = _bc_groups("Bm", Bm, (Bsz, L), H)
+    if Cm.shape != Bm.shape:
+        raise ValueError("Bm and Cm must have the same shape")
     if dCm_add is not None:
-        _shape("dCm_add", dCm_add, (Bsz, L, N))
-    dims = Dims(Bsz, L, H, P, N, chunk, 1)
+        _shape("dCm_add", dCm_add, tuple(Cm.shape))
+    dims = Dims(Bsz, L, H, P, N, chunk, G)
     out = {"dx": torch.empty((Bsz, L, H, P), device=dev), "ddt": torch.empty((Bsz, L, H), device=dev),
-           "dA": torch.empty((H,), device=dev), "dBm": torch.empty((Bsz, L, N), device=dev),
-           "dCm": torch.empty((Bsz, L, N), device=dev)}
+           "dA": torch.empty((H,), device=dev), "dBm": torch.empty(tuple(Bm.shape), device=dev),
+           "dCm": torch.empty(tuple(Cm.shape), device=dev)}
     if init_state is not None:
         out["dinit_state"] = torch.empty((Bsz, H, N, P), device=dev)
     wsb = lib.dart_ssd_scan_backward_workspace_bytes(ctypes.byref(dims))
@@ -407,7 +432,8 @@ def layer_forward(x, dt, A, Bm, Cm, Q, E, chunk: int, g: float, init_state=None,
 
 def dart_decode_step(x, dt, A, Bm, Cm, Q, E, g: float, state, dH_cur, cache, nchunks, pos,
                      chunk: int, *, y=None, workspace=None, memlog=None, cache_exp=None):
-    """One decode step for every sequence.  x[Bs,H,P], Bm/Cm[Bs,N],
+    """One decode step for every sequence.  x[Bs,H,P], Bm/Cm[Bs,N] (or
+    [Bs,G,N] with G groups of heads),
     Q[Bs,H,N], E[Bs,H,P] (cache dtype), dt[Bs,H], A[H] float32; state and
     dH_cur float32 [Bs,H,N,P], cache [Bs,H,cmax,N,P], nchunks/pos int32 [Bs]
     are device tensors updated in place.  With ``memlog`` (float32
@@ -438,7 +464,10 @@ def dart_decode_step(x, dt, A, Bm, Cm, Q, E, g: float, state, dH_cur, cache, nch
     cmax = cache.shape[2]
     _shape("state", state, (Bs, H, N, P)); _shape("dH_cur", dH_cur, (Bs, H, N, P))
     _shape("cache", cache, (Bs, H, cmax, N, P)); _shape("Q", Q, (Bs, H, N)); _shape("E", E, (Bs, H, P))
-    _shape("dt", dt, (Bs, H)); _shape("Cm", Cm, (Bs, N))
+    _shape("dt", dt, (Bs, H))
+    G = _bc_groups("Bm", Bm, (Bs,), H)
+    if Cm.shape != Bm.shape:
+        raise ValueError("Bm and Cm must have the same shape")
     if state.dtype != torch.float32 or dH_cur.dtype != torch.float32:
         raise TypeError("state and dH_cur must be float32")
     if nchunks.dtype != torch.int32 or pos.dtype != torch.int32:
@@ -449,7 +478,7 @@ def dart_decode_step(x, dt, A, Bm, Cm, Q, E, g: float, state, dH_cur, cache, nch
             raise TypeError("memlog must be float32")
     if e4m3:
         _shape("cache_exp", cache_exp, (Bs, H, cmax, N))
-    dims = Dims(Bs, 0, H, P, N, chunk, 1)
+    dims = Dims(Bs, 0, H, P, N, chunk, G)
     code = _dtype_code(in_dtype)
     if y is None:
         y = torch.empty((Bs, H, P), device=dev, dtype=torch.float32)
@@ -533,9 +562,12 @@ def dart_decode_step_noalloc(x, dt, A, Bm, Cm, Q, E, g: float, state, dH_cur, ca
     cmax = cache.shape[2]
     _shape("state", state, (Bs, H, N, P)); _shape("dH_cur", dH_cur, (Bs, H, N, P))
     _shape("cache", cache, (Bs, H, cmax, N, P))
+    G = _bc_groups("Bm", Bm, (Bs,), H)
+    if Cm.shape != Bm.shape:
+        raise ValueError("Bm and Cm must have the same shape")
     if y is None:
         y = torch.empty((Bs, H, P), device=cache.device, dtype=torch.float32)
-    dims = Dims(Bs, 0, H, P, N, chunk, 1)
+    dims = Dims(Bs, 0, H, P, N, chunk, G)
     with torch.cuda.device(cache.device):
         _check(lib.dart_decode_step_noalloc(ctypes.byref(dims), _dtype_code(cache.dtype), _ptr(x), _ptr(dt),
                                             _ptr(A), _ptr(Bm), _ptr(Cm), _ptr(Q), _ptr(E), float(g), _ptr(state),

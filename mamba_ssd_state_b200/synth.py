@@ -110,16 +110,18 @@ def _cast(a: np.ndarray, dtype: str) -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(a)).to(torch_dtype(dtype))
 
 
-def layer_inputs(shape: LayerShape, seed: int = 0) -> dict:
+def layer_inputs(shape: LayerShape, seed: int = 0, ngroups: int = 1) -> dict:
     """CPU tensors x, dt, A, Bm, Cm, Q, E (x/Bm/Cm/Q/E in the shape's dtype,
-    dt and A always float32) and the gate g."""
+    dt and A always float32) and the gate g.  With ngroups > 1, Bm and Cm are
+    [B, L, ngroups, N] (one row per group of heads), else [B, L, N]."""
     Bz, L, H, P, N = shape.batch, shape.seqlen, shape.nheads, shape.headdim, shape.dstate
+    bc = (Bz, L, N) if ngroups == 1 else (Bz, L, ngroups, N)
     out = {
         "A": torch.from_numpy(_A(seed, H)),
         "dt": torch.from_numpy(_dt(seed, "dt", (Bz, L, H), shape.dt_dist)),
         "x": _cast(_normal(seed, "x", (Bz, L, H, P)), shape.dtype),
-        "Bm": _cast(_normal(seed, "B", (Bz, L, N), 1.0 / np.sqrt(N)), shape.dtype),
-        "Cm": _cast(_normal(seed, "C", (Bz, L, N), 1.0 / np.sqrt(N)), shape.dtype),
+        "Bm": _cast(_normal(seed, "B", bc, 1.0 / np.sqrt(N)), shape.dtype),
+        "Cm": _cast(_normal(seed, "C", bc, 1.0 / np.sqrt(N)), shape.dtype),
         "Q": _cast(_normal(seed, "Q", (Bz, L, H, N)), shape.dtype),
         "E": _cast(_normal(seed, "E", (Bz, L, H, P), 1.0 / np.sqrt(P)), shape.dtype),
     }
@@ -174,19 +176,21 @@ def decode_initial(shape: DecodeShape, seed: int = 0, sequences=None, threads: i
     }
 
 
-def decode_tokens(shape: DecodeShape, step: int, seed: int = 0, sequences=None) -> dict:
+def decode_tokens(shape: DecodeShape, step: int, seed: int = 0, sequences=None, ngroups: int = 1) -> dict:
     """Token inputs of one decode step for every sequence (or a subset):
     x[Bs,H,P], dt[Bs,H], Bm[Bs,N], Cm[Bs,N], Q[Bs,H,N], E[Bs,H,P]; drawn per
-    (step, sequence) as in the 370M-shape layer case."""
+    (step, sequence) as in the 370M-shape layer case.  With ngroups > 1, Bm
+    and Cm are [Bs, ngroups, N]."""
     seqs = list(range(shape.nseq)) if sequences is None else list(sequences)
     H, N, P = shape.nheads, shape.dstate, shape.headdim
+    bc = (N,) if ngroups == 1 else (ngroups, N)
     cols = {k: [] for k in ("x", "dt", "Bm", "Cm", "Q", "E")}
     for b in seqs:
         r = _rng(seed, "token", step, b)
         cols["x"].append(r.standard_normal((H, P), dtype=np.float32))
         cols["dt"].append(np.exp(r.uniform(np.log(1e-3), np.log(1e-1), size=(H,))).astype(np.float32))
-        cols["Bm"].append(r.standard_normal((N,), dtype=np.float32) / np.float32(np.sqrt(N)))
-        cols["Cm"].append(r.standard_normal((N,), dtype=np.float32) / np.float32(np.sqrt(N)))
+        cols["Bm"].append(r.standard_normal(bc, dtype=np.float32) / np.float32(np.sqrt(N)))
+        cols["Cm"].append(r.standard_normal(bc, dtype=np.float32) / np.float32(np.sqrt(N)))
         cols["Q"].append(r.standard_normal((H, N), dtype=np.float32))
         cols["E"].append(r.standard_normal((H, P), dtype=np.float32) / np.float32(np.sqrt(P)))
     out = {k: np.stack(v) for k, v in cols.items()}

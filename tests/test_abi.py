@@ -69,8 +69,13 @@ def test_ragged_seqlen_counts_the_partial_chunk(lib):
     assert _scan(lib, d, ws_bytes=need - 16) == dart.DART_ERR_INVALID_ARG
 
 
-def test_scan_rejects_ngroups(lib):
-    assert _scan(lib, dart.Dims(1, 256, 2, 64, 128, 256, 2)) == dart.DART_ERR_UNSUPPORTED
+def test_scan_rejects_ngroups_not_dividing_heads(lib):
+    """B and C come in ngroups groups, head h reading group h / (nheads /
+    ngroups); a count that does not divide nheads, or is below 1, is rejected
+    before any launch."""
+    assert _scan(lib, dart.Dims(1, 256, 4, 64, 128, 256, 3)) == dart.DART_ERR_INVALID_ARG
+    assert _scan(lib, dart.Dims(1, 256, 4, 64, 128, 256, 0)) == dart.DART_ERR_INVALID_ARG
+    assert _scan(lib, dart.Dims(1, 256, 4, 64, 128, 256, 8)) == dart.DART_ERR_INVALID_ARG
 
 
 def test_scan_rejects_uncompiled_shape(lib):
