@@ -75,6 +75,11 @@
  *    step then reads the dequantized memories and quantizes the memory it
  *    appends.  Written from the format's definition, not from any library.
  *
+ *  - Gradients through the scan (the training pass the DART abstract claims):
+ *    reverse-mode differentiation of the token recurrence above for the loss
+ *    sum(dy * y_ssd) + sum(gD * dH), taken token by token from the last
+ *    token (section 6).
+ *
  * Layouts (row-major, last index fastest):
  *   x[B,L,H,P] dt[B,L,H] A[H] Bm[B,L,G,N] Cm[B,L,G,N] Q[B,L,H,N] E[B,L,H,P]
  *   y[B,L,H,P] dH[B,H,C,N,P] states[B,H,C,N,P] init_state[B,H,N,P]
@@ -519,5 +524,172 @@ int oracle_decode_step(const oracle_dims* d, int cmax, const float* x, const flo
             pos[b] += 1;
         }
     }
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* 6: gradients through the scan, by reverse-mode differentiation of    */
+/*    the token recurrence of section 1 + 2                             */
+/* ------------------------------------------------------------------ */
+/*
+ * Loss = sum(dy * y_ssd) + sum(gD * dH) for given dy [B,L,H,P] and gD
+ * [B,H,C,N,P] (nullable: 0).  Walking the tokens from the last to the first
+ * with the adjoints
+ *     Gt = dLoss/dH_t = C_t dy_t^T + a_{t+1} G_{t+1}
+ *     Kt = dLoss/dD_t = gD[c] at the chunk's last token, else a_{t+1} K_{t+1}
+ * (D restarts at each chunk's first token, so no K flows into the chunk
+ * before), u_t = dt_t B_t x_t^T feeds both H_t and D_t, so with Z = Gt + Kt:
+ *     dx_t = dt_t Z^T B_t,  dB_t += dt_t Z x_t,  dC_t += H_t dy_t,
+ *     da_t = sum(Gt o H_{t-1}) + sum(Kt o D_{t-1}),  a_t = exp(dt_t A_h),
+ *     ddt_t = sum(Z o B_t x_t^T) + da_t a_t A_h,  dA_h += da_t a_t dt_t,
+ *     dinit = a_0 G_0.
+ * The states H_{t-1} and D_{t-1} of one chunk are recomputed from the state
+ * entering the chunk (kept from a first forward pass) before the chunk is
+ * walked backwards: the same fp64 operations in the same order as the
+ * forward pass, so the values are those of a stored history.
+ */
+typedef struct {
+    const oracle_dims* d;
+    const float *x, *dt, *A, *Bm, *Cm;
+    const double *init_state, *dy, *gD;
+    double *dx, *ddt, *dBh, *dCh, *dApart, *dinit; /* dBh, dCh [B,L,H,N]; dApart [B,H] */
+} scan_bwd_ctx;
+
+static void scan_bwd_unit(void* vctx, int unit) {
+    scan_bwd_ctx* c = (scan_bwd_ctx*)vctx;
+    const oracle_dims* d = c->d;
+    const int L = d->seqlen, H = d->nheads, P = d->headdim, N = d->dstate, S = d->chunk;
+    const int NP = N * P, nchunks = (L + S - 1) / S;
+    const int b = unit / H, h = unit % H;
+    const double Ah = (double)c->A[h];
+    double* enter = (double*)calloc((size_t)nchunks * NP, sizeof(double)); /* H before each chunk */
+    double* Hh = (double*)malloc(sizeof(double) * (size_t)(S + 1) * NP);    /* H_{s0-1} .. H_e     */
+    double* Dh = (double*)malloc(sizeof(double) * (size_t)(S + 1) * NP);    /* D_{s0-1} .. D_e     */
+    double* G = (double*)calloc((size_t)NP, sizeof(double));
+    double* K = (double*)calloc((size_t)NP, sizeof(double));
+    double* Hs = (double*)calloc((size_t)NP, sizeof(double));
+    if (c->init_state)
+        for (int i = 0; i < NP; ++i) Hs[i] = c->init_state[((size_t)b * H + h) * NP + i];
+#define TOK(t) ((size_t)b * L + (t))
+#define BROW(M, t) ((M) + (TOK(t) * ngroups_of(d) + group_of(d, h)) * N)
+    /* forward pass: the state entering every chunk */
+    for (int t = 0; t < L; ++t) {
+        if (t % S == 0) memcpy(enter + (size_t)(t / S) * NP, Hs, sizeof(double) * NP);
+        const double dtt = (double)c->dt[TOK(t) * H + h], a = exp(dtt * Ah);
+        const float* Bt = BROW(c->Bm, t);
+        const float* xt = c->x + (TOK(t) * H + h) * P;
+        for (int n = 0; n < N; ++n)
+            for (int p = 0; p < P; ++p) Hs[n * P + p] = a * Hs[n * P + p] + dtt * (double)Bt[n] * (double)xt[p];
+    }
+    double dA = 0.0;
+    for (int ck = nchunks - 1; ck >= 0; --ck) {
+        const int s0 = ck * S, e = (s0 + S < L ? s0 + S : L) - 1;
+        /* recompute H_{t-1}, D_{t-1} for t = s0 .. e: slot t - s0 holds the values before token t */
+        memcpy(Hh, enter + (size_t)ck * NP, sizeof(double) * NP);
+        memset(Dh, 0, sizeof(double) * NP);
+        for (int t = s0; t <= e; ++t) {
+            const double dtt = (double)c->dt[TOK(t) * H + h], a = exp(dtt * Ah);
+            const float* Bt = BROW(c->Bm, t);
+            const float* xt = c->x + (TOK(t) * H + h) * P;
+            const double* hp = Hh + (size_t)(t - s0) * NP;
+            const double* dp = Dh + (size_t)(t - s0) * NP;
+            double* hn = Hh + (size_t)(t - s0 + 1) * NP;
+            double* dn = Dh + (size_t)(t - s0 + 1) * NP;
+            for (int n = 0; n < N; ++n)
+                for (int p = 0; p < P; ++p) {
+                    const double u = dtt * (double)Bt[n] * (double)xt[p];
+                    hn[n * P + p] = a * hp[n * P + p] + u;
+                    dn[n * P + p] = a * dp[n * P + p] + u;
+                }
+        }
+        /* the memory gradient enters at the chunk's last token */
+        for (int i = 0; i < NP; ++i)
+            K[i] = c->gD ? c->gD[(((size_t)b * H + h) * nchunks + ck) * NP + i] : 0.0;
+        for (int t = e; t >= s0; --t) {
+            const double dtt = (double)c->dt[TOK(t) * H + h], a = exp(dtt * Ah);
+            const float* Bt = BROW(c->Bm, t);
+            const float* Ct = BROW(c->Cm, t);
+            const float* xt = c->x + (TOK(t) * H + h) * P;
+            const double* dyt = c->dy + (TOK(t) * H + h) * P;
+            const double* hprev = Hh + (size_t)(t - s0) * NP;
+            const double* dprev = Dh + (size_t)(t - s0) * NP;
+            const double* hcur = Hh + (size_t)(t - s0 + 1) * NP;
+            /* G_t = C_t dy_t^T + (a_{t+1} G_{t+1}, carried in G) */
+            for (int n = 0; n < N; ++n)
+                for (int p = 0; p < P; ++p) G[n * P + p] += (double)Ct[n] * dyt[p];
+            double zbx = 0.0, da = 0.0;
+            for (int p = 0; p < P; ++p) {
+                double s = 0.0;
+                for (int n = 0; n < N; ++n) s += (G[n * P + p] + K[n * P + p]) * (double)Bt[n];
+                c->dx[(TOK(t) * H + h) * P + p] = dtt * s;
+            }
+            for (int n = 0; n < N; ++n) {
+                double sb = 0.0, sc = 0.0;
+                for (int p = 0; p < P; ++p) {
+                    const double z = G[n * P + p] + K[n * P + p];
+                    sb += z * (double)xt[p];
+                    sc += hcur[n * P + p] * dyt[p];
+                    zbx += z * (double)Bt[n] * (double)xt[p];
+                    da += G[n * P + p] * hprev[n * P + p] + K[n * P + p] * dprev[n * P + p];
+                }
+                c->dBh[(TOK(t) * H + h) * N + n] = dtt * sb;
+                c->dCh[(TOK(t) * H + h) * N + n] = sc;
+            }
+            c->ddt[TOK(t) * H + h] = zbx + da * a * Ah;
+            dA += da * a * dtt;
+            /* carry to token t - 1: H_{t-1} feeds H_t through a_t; D_{t-1} only inside the chunk */
+            for (int i = 0; i < NP; ++i) {
+                G[i] *= a;
+                K[i] = t == s0 ? 0.0 : K[i] * a;
+            }
+        }
+    }
+    c->dApart[(size_t)b * H + h] = dA;
+    if (c->dinit)
+        for (int i = 0; i < NP; ++i) c->dinit[((size_t)b * H + h) * NP + i] = G[i];
+#undef TOK
+#undef BROW
+    free(enter); free(Hh); free(Dh); free(G); free(K); free(Hs);
+}
+
+/*
+ * Gradients through the scan: dx [B,L,H,P], ddt [B,L,H], dA [H], dB and dC
+ * [B,L,G,N] (summed over the heads of each group), dinit [B,H,N,P]
+ * (nullable).  dy [B,L,H,P], gD [B,H,C,N,P] (nullable) and init_state
+ * (nullable) are double.  Returns 0, or -1 on a shape it does not accept.
+ */
+int oracle_ssd_scan_backward(const oracle_dims* d, const float* x, const float* dt, const float* A,
+                             const float* Bm, const float* Cm, const double* init_state, const double* dy,
+                             const double* gD, double* dx, double* ddt, double* dA, double* dB, double* dC,
+                             double* dinit, int nthreads) {
+    if (!dims_ok(d) || d->seqlen <= 0) return -1;
+    const int B = d->batch, L = d->seqlen, H = d->nheads, N = d->dstate, G = ngroups_of(d);
+    double* dBh = (double*)malloc(sizeof(double) * (size_t)B * L * H * N);
+    double* dCh = (double*)malloc(sizeof(double) * (size_t)B * L * H * N);
+    double* dAp = (double*)malloc(sizeof(double) * (size_t)B * H);
+    if (!dBh || !dCh || !dAp) {
+        free(dBh); free(dCh); free(dAp);
+        return -1;
+    }
+    scan_bwd_ctx c = {d, x, dt, A, Bm, Cm, init_state, dy, gD, dx, ddt, dBh, dCh, dAp, dinit};
+    run_units(scan_bwd_unit, &c, B * H, nthreads);
+    for (size_t tok = 0; tok < (size_t)B * L; ++tok)
+        for (int g = 0; g < G; ++g)
+            for (int n = 0; n < N; ++n) {
+                double sb = 0.0, sc = 0.0;
+                for (int h = 0; h < H; ++h) {
+                    if (group_of(d, h) != g) continue;
+                    sb += dBh[(tok * H + h) * N + n];
+                    sc += dCh[(tok * H + h) * N + n];
+                }
+                dB[(tok * G + g) * N + n] = sb;
+                dC[(tok * G + g) * N + n] = sc;
+            }
+    for (int h = 0; h < H; ++h) {
+        double s = 0.0;
+        for (int b = 0; b < B; ++b) s += dAp[(size_t)b * H + h];
+        dA[h] = s;
+    }
+    free(dBh); free(dCh); free(dAp);
     return 0;
 }

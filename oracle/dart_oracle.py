@@ -68,6 +68,8 @@ class Oracle:
         self.lib.oracle_decode_step.argtypes = (
             [ctypes.POINTER(_Dims), ctypes.c_int] + [_P] * 7 + [ctypes.c_double]
             + [_P] * 6 + [ctypes.c_int, _P, ctypes.c_int])
+        self.lib.oracle_ssd_scan_backward.restype = ctypes.c_int
+        self.lib.oracle_ssd_scan_backward.argtypes = [ctypes.POINTER(_Dims)] + [_P] * 14 + [ctypes.c_int]
         self.lib.oracle_quantize_e4m3.restype = ctypes.c_int
         self.lib.oracle_quantize_e4m3.argtypes = [_P, ctypes.c_long, ctypes.c_int, _P, _P, _P]
 
@@ -104,6 +106,32 @@ class Oracle:
         if rc:
             raise ValueError("oracle_ssd_scan rejected its arguments")
         return y, dH, st
+
+    def scan_backward(self, x, dt, A, Bm, Cm, chunk: int, dy, gD=None, init_state=None):
+        """Gradients of sum(dy * y_ssd) + sum(gD * dH) through the token
+        recurrence (reverse mode, token by token).  Returns a dict of float64
+        arrays dx, ddt, dA, dBm, dCm (shaped like Bm / Cm: summed over the
+        heads of each group) and, with an initial state, dinit_state."""
+        x, dt, A, Bm, Cm = (self._f32(v) for v in (x, dt, A, Bm, Cm))
+        Bsz, L, H, P = x.shape
+        N = Bm.shape[-1]
+        d = _Dims(Bsz, L, H, P, N, chunk, _groups(Bm, 3))
+        dy = self._f64(dy)
+        gD = None if gD is None else self._f64(gD)
+        h0 = None if init_state is None else self._f64(init_state)
+        out = {"dx": np.empty((Bsz, L, H, P), np.float64), "ddt": np.empty((Bsz, L, H), np.float64),
+               "dA": np.empty((H,), np.float64), "dBm": np.empty(Bm.shape, np.float64),
+               "dCm": np.empty(Cm.shape, np.float64)}
+        dinit = None if h0 is None else np.empty((Bsz, H, N, P), np.float64)
+        rc = self.lib.oracle_ssd_scan_backward(
+            ctypes.byref(d), self._ptr(x), self._ptr(dt), self._ptr(A), self._ptr(Bm), self._ptr(Cm),
+            self._ptr(h0), self._ptr(dy), self._ptr(gD), self._ptr(out["dx"]), self._ptr(out["ddt"]),
+            self._ptr(out["dA"]), self._ptr(out["dBm"]), self._ptr(out["dCm"]), self._ptr(dinit), self.nthreads)
+        if rc:
+            raise ValueError("oracle_ssd_scan_backward rejected its arguments")
+        if dinit is not None:
+            out["dinit_state"] = dinit
+        return out
 
     def sma(self, Q, E, Cm, dH, chunk: int, g: float = 1.0, y_ssd=None,
             tokens=None, want_scores: bool = False, dt=None, A=None):

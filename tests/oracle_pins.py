@@ -667,6 +667,39 @@ def pin_ngroups_split_into_independent_problems(orc):
             assert np.array_equal(ys[None][:, g * hg:(g + 1) * hg], ys[g]), (G, g, "decode")
 
 
+# ----------------------------------------------------------------------------
+# gradients through the scan (the training pass of the DART abstract)
+# ----------------------------------------------------------------------------
+def pin_scan_backward_matches_autograd(orc):
+    """The C oracle's reverse-mode walk of the token recurrence equals
+    autograd over the float64 torch restatement of the same recurrence
+    (``oracle/dart_backward.py``, itself pinned to central finite differences
+    of the C forward in ``test_oracle_backward.py``), to 1e-10 relative: one
+    group and two groups of heads, with and without an initial state and a
+    memory gradient, ragged last chunk."""
+    from oracle import dart_backward
+    for seed, (Bz, L, H, P, N, S, G, init, gmem) in enumerate([
+            (1, 3 * 8 + 5, 2, 3, 4, 8, 1, True, True),
+            (2, 2 * 4 + 3, 4, 2, 3, 4, 2, False, True),
+            (1, 17, 2, 3, 2, 8, 1, True, False)]):
+        inp = _rand_layer(60 + seed, Bz, L, H, P, N)
+        r = np.random.default_rng(70 + seed)
+        if G > 1:
+            inp["Bm"] = (r.standard_normal((Bz, L, G, N)) / np.sqrt(N)).astype(np.float32)
+            inp["Cm"] = (r.standard_normal((Bz, L, G, N)) / np.sqrt(N)).astype(np.float32)
+        C = -(-L // S)
+        dy = r.standard_normal((Bz, L, H, P))
+        gD = r.standard_normal((Bz, H, C, N, P)) if gmem else None
+        h0 = r.standard_normal((Bz, H, N, P)) * 0.3 if init else None
+        args = [inp[k].astype(np.float64) for k in ("x", "dt", "A", "Bm", "Cm")]
+        got = orc.scan_backward(*args, S, dy, gD, init_state=h0)
+        ref = dart_backward.scan_grads(*args, S, dy, np.zeros((Bz, H, C, N, P)) if gD is None else gD,
+                                       init_state=h0)
+        for k, v in got.items():
+            err = np.max(np.abs(v - ref[k])) / max(np.max(np.abs(ref[k])), 1e-300)
+            assert err <= 1e-10, (seed, k, err)
+
+
 ALL_PINS = [
     pin_closed_form_single_token,
     pin_quadratic_form,
@@ -688,4 +721,5 @@ ALL_PINS = [
     pin_e4m3_rows_match_library,
     pin_e4m3_decode_append,
     pin_ngroups_split_into_independent_problems,
+    pin_scan_backward_matches_autograd,
 ]

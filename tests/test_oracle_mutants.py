@@ -66,6 +66,17 @@ MUTATIONS = [
     ("e4m3_decode_bias", "ldexp(8.0 + m, e - 10)", "ldexp(8.0 + m, e - 11)", 0),
     ("decode_append_not_quantized", "if (c->cache_e4m3) {", "if (0) {", 0),
     ("group_by_modulo", "return h / (d->nheads / ngroups_of(d));", "return h % ngroups_of(d);", 0),
+    ("bwd_memory_gradient_ignored", "K[i] = c->gD ? c->gD[(((size_t)b * H + h) * nchunks + ck) * NP + i] : 0.0;",
+     "K[i] = 0.0;", 0),
+    ("bwd_memory_gradient_wrong_chunk", "c->gD[(((size_t)b * H + h) * nchunks + ck) * NP + i]",
+     "c->gD[(((size_t)b * H + h) * nchunks + (ck + 1) % nchunks) * NP + i]", 0),
+    ("bwd_dC_from_previous_state", "sc += hcur[n * P + p] * dyt[p];", "sc += hprev[n * P + p] * dyt[p];", 0),
+    ("bwd_decay_grad_drops_memory_term",
+     "da += G[n * P + p] * hprev[n * P + p] + K[n * P + p] * dprev[n * P + p];",
+     "da += G[n * P + p] * hprev[n * P + p];", 0),
+    ("bwd_dx_without_dt", "c->dx[(TOK(t) * H + h) * P + p] = dtt * s;", "c->dx[(TOK(t) * H + h) * P + p] = s;", 0),
+    ("bwd_dinit_one_decay_short", "for (int i = 0; i < NP; ++i) {\n                G[i] *= a;",
+     "for (int i = 0; i < NP; ++i) {\n                if (t > 0) G[i] *= a;", 0),
 ]
 
 
