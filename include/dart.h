@@ -395,11 +395,23 @@ const char* dart_sma_impl(int dstate, int headdim, int chunk, dart_dtype dtype);
  */
 dart_status dart_sync_status(void* stream);
 
+/*
+ * Failure-detection drill: launches one warp that waits, through the bounded
+ * mbarrier wait every tensor-core kernel uses, on an mbarrier nothing
+ * arrives on.  After limit_us microseconds (1 .. 2e6) the wait gives up and
+ * latches the timeout in the status word (kernel 9, wait site 1); nothing
+ * else is in flight, so the next dart_sync_status(stream) returns
+ * DART_ERR_TIMEOUT, clears the word, and later calls run clean.  Returns
+ * DART_OK once launched, DART_ERR_INVALID_ARG for a limit out of range.
+ */
+dart_status dart_selftest_wait_timeout(unsigned int limit_us, void* stream);
+
 /* Message describing the last failure on the calling host thread ("" if none). */
 const char* dart_last_error(void);
 
 /* ABI version, bumped on any signature change or addition (2: the decayed-memory,
- * E4M3-cache and backward entry points). */
+ * E4M3-cache and backward entry points; 3: dCm_add of the scan backward and
+ * ngroups; 4: dart_selftest_wait_timeout). */
 int dart_abi_version(void);
 
 /*

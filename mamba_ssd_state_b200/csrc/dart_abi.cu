@@ -89,7 +89,7 @@ dart_status check_common(const dart_dims* d, dart_dtype dt, bool need_seqlen) {
 
 extern "C" {
 
-int dart_abi_version(void) { return 3; }
+int dart_abi_version(void) { return 4; }
 
 unsigned long long dart_launch_count(void) { return dart::g_launches.load(std::memory_order_relaxed); }
 
@@ -231,8 +231,9 @@ dart_status dart_ssd_scan_backward(const dart_dims* d, dart_dtype dtype, const v
     t_err[0] = 0;
     dart_status st = check_common(d, dtype, true);
     if (st != DART_OK) return st;
-    if (!dart::scan_bwd_supported(d->dstate, d->headdim))
-        return fail(DART_ERR_UNSUPPORTED, "dart_ssd_scan_backward: (N=%d, P=%d) not compiled", d->dstate, d->headdim);
+    if (!dart::scan_bwd_supported(d->dstate, d->headdim, d->chunk))
+        return fail(DART_ERR_UNSUPPORTED, "dart_ssd_scan_backward: (N=%d, P=%d, S=%d) not compiled", d->dstate,
+                    d->headdim, d->chunk);
     DART_REQUIRE_PTR(x); DART_REQUIRE_PTR(dt); DART_REQUIRE_PTR(A); DART_REQUIRE_PTR(Bm); DART_REQUIRE_PTR(Cm);
     DART_OPTIONAL_PTR(init_state); DART_REQUIRE_PTR(states); DART_REQUIRE_PTR(dy); DART_OPTIONAL_PTR(ddH);
     DART_OPTIONAL_PTR(dCm_add); DART_REQUIRE_PTR(dx); DART_REQUIRE_PTR(ddt); DART_REQUIRE_PTR(dA); DART_REQUIRE_PTR(dBm); DART_REQUIRE_PTR(dCm);
@@ -442,6 +443,18 @@ dart_status dart_decode_step_noalloc(const dart_dims* d, dart_dtype dtype, const
     if (!a.status) return fail(DART_ERR_CUDA, "dart_decode_step_noalloc: no device status word");
     e = dart::launch_decode(a, dtype, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "dart_decode_step_noalloc launch");
+    return DART_OK;
+}
+
+dart_status dart_selftest_wait_timeout(unsigned int limit_us, void* stream) {
+    t_err[0] = 0;
+    if (limit_us < 1 || limit_us > 2000000)
+        return fail(DART_ERR_INVALID_ARG, "dart_selftest_wait_timeout: limit_us = %u outside [1, 2000000]", limit_us);
+    int* status = status_word();
+    if (!status) return fail(DART_ERR_CUDA, "dart_selftest_wait_timeout: no device status word");
+    cudaError_t e = dart::launch_wait_drill(status, 1000ull * limit_us, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "dart_selftest_wait_timeout launch");
+    dart::count_launches(1);
     return DART_OK;
 }
 

@@ -30,15 +30,17 @@ struct ScanBwdArgs {
     float* dinit;           // nullable [B,H,N,P] output
     int* status;
     // workspace views (set by launch_ssd_scan_bwd)
-    float* hist;            // [2][B,H,S,N,P] H_{t-1}, D_{t-1} of the chunk being walked
+    float* gin;             // [B,H,C,N,P] dS[c], then the adjoint entering chunk c from later chunks
+    float* asum;            // [B,H,C] chunk decay sums
+    float* rect;            // [B,H,C,S] the chunk-local decay-gradient term per token
     float* dBh; float* dCh; // [B,L,H,N] per-head dB, dC
-    float* dApart;          // [B,H]
+    float* dApart;          // [B,H,C]
 };
 
 size_t sma_bwd_workspace_bytes(int B, int L, int H, int N, int S);
 cudaError_t launch_sma_bwd(SmaBwdArgs a, void* workspace, dart_dtype dt, cudaStream_t st);
 size_t scan_bwd_workspace_bytes(int B, int L, int H, int N, int P, int S);
-bool scan_bwd_supported(int N, int P);
+bool scan_bwd_supported(int N, int P, int S);
 cudaError_t launch_ssd_scan_bwd(ScanBwdArgs a, void* workspace, dart_dtype dt, cudaStream_t st);
 
 }  // namespace dart

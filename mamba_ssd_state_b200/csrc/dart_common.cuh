@@ -193,6 +193,8 @@ int decode_num_splits(int B, int H, int cmax);
 constexpr int kDecodeMaxCmax = 1 << 20;
 bool decode_e4m3_supported(int N, int P);
 cudaError_t launch_decode_e4m3(const DecodeArgs& a, dart_dtype dt, cudaStream_t st);
+// selftest.cu: one bounded wait on an mbarrier nothing arrives on.
+cudaError_t launch_wait_drill(int* status, unsigned long long limit_ns, cudaStream_t st);
 // dH [B,H,C,N,P] (dtype) memories 0..nmem-1 -> E4M3 codes and row exponents
 // in cache slots 0..nmem-1 ([B,H,cmax,N,P] / [B,H,cmax,N]); one launch.
 cudaError_t launch_cache_quantize_e4m3(int B, int H, int C, int N, int P, int nmem, int cmax, const void* dH,

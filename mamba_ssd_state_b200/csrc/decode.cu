@@ -24,14 +24,13 @@
 // OCP FP8 E4M3 codes times 2^k (k an int8 per row; the cache quantization
 // the pages list as an extension), half the bytes of bf16.  Each lane loads
 // 8 codes of a row (8 bytes; four lanes per 32-byte row segment keep the
-// warp's loads contiguous) and widens each code to fp32 by placing its 7
-// magnitude bits under the fp32 exponent field, which gives
-// code_value * 2^-120 exactly (E4M3 subnormals become fp32 subnormals) at
-// integer-ALU rate; the products run as packed fp32x2 FMAs.  The row's 2^k
-// and the 2^-120 are folded into per-row factors kept in shared memory per
-// warp: E is pre-scaled by 2^60 for the score, (q, C) by 2^(k+60), and the
-// value sum is scaled back by 2^60, so no intermediate overflows for
-// contributions up to 2^68 and only contributions below 2^-89 underflow.  An append
+// warp's loads contiguous) and widens each pair of codes exactly with the
+// hardware E4M3x2 -> f16x2 conversion, then to fp32 (every E4M3 value,
+// subnormals included, is an f16 value); the products run as packed fp32x2
+// FMAs.  The row's 2^k is folded into per-row factors kept in shared memory
+// per warp: (q, C) by 2^(k+60), E pre-scaled by 2^-60 for the score and the
+// value sum scaled back by 2^-60, so no intermediate overflows for
+// contributions up to 2^68 and only contributions below 2^-66 lose bits.  An append
 // quantizes the finished memory row by row (one warp per row): the row
 // exponent is the smallest k with max|row| 2^-k <= 448 (clamped to
 // [-126, 60]) and the codes round to nearest even with saturation.
@@ -255,10 +254,12 @@ __device__ __forceinline__ int e4m3_row_exponent(float amax) {
 // 2^j as an fp32 for j in [-126, 127].
 __device__ __forceinline__ float exp2i(int j) { return __int_as_float((j + 127) << 23); }
 
-// Code i (byte i of w) as fp32 bits equal to code_value * 2^-120: the sign to
-// bit 31, the 4 exponent and 3 mantissa bits to bits 26..20.
-__device__ __forceinline__ float e4m3_scaled(uint32_t w, int i) {
-    return __int_as_float((int)((int)(w << (24 - 8 * i)) >> 4) & (int)0x87F00000);
+// Codes 2j and 2j+1 (bytes 2j, 2j+1 of w) as their exact values (x, y).
+__device__ __forceinline__ float2 e4m3_pair(uint32_t w, int j) {
+    const unsigned short two = (unsigned short)(w >> (16 * j));
+    uint32_t h2;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(two));
+    return __half22float2(*reinterpret_cast<const __half2*>(&h2));
 }
 
 // Quantize rows [r0, r1) of a memory from fp32 `src` (row stride P) into
@@ -381,11 +382,11 @@ __global__ void __launch_bounds__(kThreads) decode_partial_e4m3_kernel(DecodeArg
     // ---- state-memory attention over this split's cached chunks ----------
     const int lrow = lane / LPR;             // row inside a warp load
     const int pcol = (lane % LPR) * VEC;     // first column of this lane
-    constexpr float kTwo60 = 1152921504606846976.0f;   // 2^60
+    constexpr float kTwoM60 = 8.67361737988403547e-19f;   // 2^-60
     float2 ev2[VEC / 2];
 #pragma unroll
     for (int j = 0; j < VEC / 2; ++j)
-        ev2[j] = make_float2(kTwo60 * ldf(Et + pcol + 2 * j), kTwo60 * ldf(Et + pcol + 2 * j + 1));
+        ev2[j] = make_float2(kTwoM60 * ldf(Et + pcol + 2 * j), kTwoM60 * ldf(Et + pcol + 2 * j + 1));
     float m = -INFINITY, l = 0.f;
     float2 o2[VEC / 2];
 #pragma unroll
@@ -433,7 +434,7 @@ __global__ void __launch_bounds__(kThreads) decode_partial_e4m3_kernel(DecodeArg
                 for (int q = 0; q < NW; ++q) {
 #pragma unroll
                     for (int i = 0; i < 4; i += 2) {
-                        const float2 f = make_float2(e4m3_scaled(raw[u][q], i), e4m3_scaled(raw[u][q], i + 1));
+                        const float2 f = e4m3_pair(raw[u][q], i / 2);
                         v2[2 * q + i / 2] = __ffma2_rn(cs2, f, v2[2 * q + i / 2]);
                         rd2 = __ffma2_rn(f, ev2[2 * q + i / 2], rd2);
                     }
@@ -458,7 +459,7 @@ __global__ void __launch_bounds__(kThreads) decode_partial_e4m3_kernel(DecodeArg
         const float alpha = exp2f(m - mnew);
         const float w = exp2f(s - mnew);
         l = l * alpha + w;
-        const float wv = (kDecay ? w * wd : w) * kTwo60;   // the value sum carries 2^-60
+        const float wv = (kDecay ? w * wd : w) * kTwoM60;   // the value sum carries 2^60
         const float2 al2 = make_float2(alpha, alpha), wv2 = make_float2(wv, wv);
 #pragma unroll
         for (int j = 0; j < VEC / 2; ++j)

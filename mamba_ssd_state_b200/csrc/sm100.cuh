@@ -74,7 +74,8 @@ constexpr uint32_t kWaitIterCap = 1u << 26;  // second bound, independent of the
 // Waits until the phase with the given parity has completed.  Returns false
 // at once if the CTA already aborted; returns false after flagging (timeout
 // bit, first timeout site, CTA abort flag) if the wait passed its limit.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCtx& w, int site) {
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCtx& w, int site,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
     if (*w.abort_flag) return false;
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = global_ns();
@@ -82,7 +83,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
         if (mbar_try_wait(bar, parity)) return true;
         if ((i & 63u) == 0) {
             if (*w.abort_flag) return false;
-            if (global_ns() - t0 > kWaitLimitNs || i >= kWaitIterCap) {
+            if (global_ns() - t0 > limit_ns || i >= kWaitIterCap) {
                 *w.abort_flag = 1;
                 flag_status(w.status, kStatusTimeout);
                 atomicCAS(w.status + 1, 0, (w.kernel_id << 8) | site);
@@ -95,9 +96,10 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
 // Warp-uniform wait: lane 0 polls, the verdict is broadcast, and the warp
 // reconverges, so that the .sync.aligned tcgen05 instructions that follow
 // are always reached by all 32 lanes together.
-__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, const WaitCtx& w, int site) {
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, const WaitCtx& w, int site,
+                                               unsigned long long limit_ns = kWaitLimitNs) {
     int ok = 0;
-    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, w, site) ? 1 : 0;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, w, site, limit_ns) ? 1 : 0;
     ok = __shfl_sync(0xffffffffu, ok, 0);
     __syncwarp();
     return ok != 0;

@@ -34,7 +34,8 @@ EXPORTS = ("dart_ssd_chunk_scan_workspace_bytes", "dart_ssd_chunk_scan", "dart_s
            "dart_sma_impl", "dart_decode_step_noalloc", "dart_sma_decayed_workspace_bytes",
            "dart_sma_forward_decayed", "dart_decode_step_decayed", "dart_decode_memlog_init",
            "dart_decode_step_e4m3", "dart_cache_quantize_e4m3", "dart_sma_backward_workspace_bytes",
-           "dart_sma_backward", "dart_ssd_scan_backward_workspace_bytes", "dart_ssd_scan_backward")
+           "dart_sma_backward", "dart_ssd_scan_backward_workspace_bytes", "dart_ssd_scan_backward",
+           "dart_selftest_wait_timeout")
 
 
 class DartError(RuntimeError):
@@ -100,6 +101,8 @@ def load(path: str = LIBRARY) -> ctypes.CDLL:
     lib.dart_supported.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int]
     lib.dart_sync_status.restype = ctypes.c_int
     lib.dart_sync_status.argtypes = [_P]
+    lib.dart_selftest_wait_timeout.restype = ctypes.c_int
+    lib.dart_selftest_wait_timeout.argtypes = [ctypes.c_uint, _P]
     lib.dart_last_error.restype = ctypes.c_char_p
     lib.dart_last_error.argtypes = []
     lib.dart_abi_version.restype = ctypes.c_int
@@ -594,6 +597,14 @@ def scan_backward_workspace_bytes(batch, seqlen, nheads, headdim, dstate, chunk)
 def scan_workspace_bytes(batch, seqlen, nheads, headdim, dstate, chunk, dtype) -> int:
     dims = Dims(batch, seqlen, nheads, headdim, dstate, chunk, 1)
     return load().dart_ssd_chunk_scan_workspace_bytes(ctypes.byref(dims), _dtype_code(dtype))
+
+
+def dart_selftest_wait_timeout(limit_us: int, stream: Optional[torch.cuda.Stream] = None):
+    """Launch the failure-detection drill: one bounded wait on an mbarrier
+    nothing arrives on, giving up after limit_us; the next dart_sync_status
+    raises DartError(DART_ERR_TIMEOUT) and clears the status word."""
+    s = stream or torch.cuda.current_stream()
+    _check(load().dart_selftest_wait_timeout(int(limit_us), ctypes.c_void_p(s.cuda_stream)))
 
 
 def dart_sync_status(stream: Optional[torch.cuda.Stream] = None):

@@ -39,7 +39,13 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version(lib):
-    assert lib.dart_abi_version() == 3
+    assert lib.dart_abi_version() == 4
+
+
+def test_wait_drill_rejects_limits_out_of_range(lib):
+    """Host-side validation only: no launch happens for these."""
+    assert lib.dart_selftest_wait_timeout(0, None) == dart.DART_ERR_INVALID_ARG
+    assert lib.dart_selftest_wait_timeout(2000001, None) == dart.DART_ERR_INVALID_ARG
 
 
 def test_supported_set(lib):
@@ -209,13 +215,19 @@ def test_sma_backward_workspace_and_validation(lib):
 def test_scan_backward_workspace_and_validation(lib):
     d = dart.Dims(2, 500, 3, 64, 128, 256, 1)
     pad = lambda b: (b + 255) // 256 * 256
-    want = 2 * pad(4 * 2 * 3 * 256 * 128 * 64) + 2 * pad(4 * 2 * 500 * 3 * 128) + pad(4 * 2 * 3)
+    C = 2   # ceil(500 / 256)
+    # chunk adjoints, chunk decay sums, per-token decay term, per-head dB and dC, per-chunk dA
+    want = (pad(4 * 2 * 3 * C * 128 * 64) + pad(4 * 2 * 3 * C) + pad(4 * 2 * 3 * C * 256)
+            + 2 * pad(4 * 2 * 500 * 3 * 128) + pad(4 * 2 * 3 * C))
     assert lib.dart_ssd_scan_backward_workspace_bytes(ctypes.byref(d)) == want
     f = lib.dart_ssd_scan_backward
     ok = [FAKE] * 5 + [None, FAKE, FAKE, None, None] + [FAKE] * 5 + [None, FAKE]
     assert f(ctypes.byref(d), dart.DART_BF16, *ok[:6], None, *ok[7:], want, None) == dart.DART_ERR_INVALID_ARG
     assert b"states" in lib.dart_last_error()
     assert f(ctypes.byref(d), dart.DART_BF16, *ok, want - 1, None) == dart.DART_ERR_INVALID_ARG
+    d.chunk = 512
+    assert f(ctypes.byref(d), dart.DART_BF16, *ok, 1 << 40, None) == dart.DART_ERR_UNSUPPORTED
+    d.chunk = 256
     d.headdim, d.dstate = 32, 32
     assert f(ctypes.byref(d), dart.DART_BF16, *ok, 1 << 40, None) == dart.DART_ERR_UNSUPPORTED
 

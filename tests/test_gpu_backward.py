@@ -10,7 +10,7 @@ import pytest
 import torch
 
 from mamba_ssd_state_b200 import build, dart, synth
-from oracle import dart_backward
+from oracle import dart_backward, dart_oracle
 from tests.parity import assert_close
 
 pytestmark = pytest.mark.gpu
@@ -132,3 +132,28 @@ def test_layer_backward_matches_oracle(shape, dt_name, with_init):
     for k in ("dx", "ddt", "dA", "dBm", "dCm", "dQ", "dE") + (("dinit_state",) if h0 is not None else ()):
         assert_close(k, got[k], ref[k], tol)
     assert abs(float(got["dg"][0]) - float(ref["dg"])) <= tol * max(1.0, abs(float(ref["dg"])))
+
+
+def test_scan_backward_train_L8k_every_output():
+    """The training-length layer (B=2, L=8192, H=32, P=64, N=128, S=256,
+    bf16): the chunk-parallel scan backward against the C oracle's
+    token-by-token reverse-mode walk on every output element, driven by
+    random dy and memory gradients and an initial state."""
+    shape = synth.TRAIN_L8K
+    S = shape.chunk
+    inp = synth.layer_inputs(shape, seed=9)
+    r = np.random.default_rng(9)
+    Bz, L, H, P, N = shape.batch, shape.seqlen, shape.nheads, shape.headdim, shape.dstate
+    C = L // S
+    dy = torch.from_numpy(r.standard_normal((Bz, L, H, P)).astype(np.float32))
+    gdH = torch.from_numpy((r.standard_normal((Bz, H, C, N, P)) * 0.5).astype(np.float32))
+    h0 = torch.from_numpy((r.standard_normal((Bz, H, N, P)) * 0.2).astype(np.float32))
+    d = {k: inp[k].cuda() for k in ("x", "dt", "A", "Bm", "Cm")}
+    _, _, states = dart.dart_ssd_chunk_scan(d["x"], d["dt"], d["A"], d["Bm"], d["Cm"], S, h0.cuda())
+    got = dart.dart_ssd_scan_backward(d["x"], d["dt"], d["A"], d["Bm"], d["Cm"], S, states, dy.cuda(),
+                                      gdH.cuda(), h0.cuda())
+    dart.dart_sync_status()
+    ref = dart_oracle.get().scan_backward(*(inp[k].float().numpy() for k in ("x", "dt", "A", "Bm", "Cm")), S,
+                                          dy.numpy(), gdH.numpy(), init_state=h0.numpy())
+    for k in ("dx", "ddt", "dA", "dBm", "dCm", "dinit_state"):
+        assert_close(k, got[k], ref[k], TOL_FWD_INPUTS["bf16"])

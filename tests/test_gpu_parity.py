@@ -152,17 +152,25 @@ def test_train_L8k_config_full(orc):
     check_full(orc, synth.TRAIN_L8K, inp, TOL[torch.bfloat16])
 
 
-@pytest.mark.parametrize("shape,heads,nrand", [(synth.LONG_L64K, [3, 30], 64)], ids=["long_L64k"])
+@pytest.mark.parametrize("shape,heads,nrand", [(synth.LONG_L64K, [0, 3, 9, 15, 16, 22, 30, 31], 64)],
+                         ids=["long_L64k"])
 def test_large_config_sampled(orc, shape, heads, nrand):
+    """L = 65536 (256 chunks, 32 heads): the scan compared on every head and
+    every element, so every persistent CTA's first and last work item is
+    checked whatever the split; SMA on sampled token rows (first and last of
+    every chunk plus random ones) of eight heads spread over the range."""
     inp = synth.layer_inputs(shape, seed=0)
     got = gpu_layer(inp, shape)
-    sub = heads_slice(inp, heads)
-    o = oracle_inputs(sub)
+    o = oracle_inputs(inp)
     y_ssd, dH, st = orc.ssd_scan(o["x"], o["dt"], o["A"], o["Bm"], o["Cm"], shape.chunk)
     tol = TOL[torch.bfloat16]
-    assert_close("y_ssd", got["y_ssd"][:, :, heads], y_ssd, tol)
-    assert_close("dH", got["dH"][:, heads], dH, tol)
-    assert_close("states", got["states"][:, heads], st, tol)
+    for h0 in range(0, shape.nheads, 8):    # per head block, so a bad head is named
+        hs = slice(h0, h0 + 8)
+        assert_close(f"y_ssd heads {h0}..", got["y_ssd"][:, :, hs], y_ssd[:, :, hs], tol)
+        assert_close(f"dH heads {h0}..", got["dH"][:, hs], dH[:, hs], tol)
+        assert_close(f"states heads {h0}..", got["states"][:, hs], st[:, hs], tol)
+    o = oracle_inputs(heads_slice(inp, heads))
+    y_ssd, dH = y_ssd[:, :, heads], dH[:, heads]
     tok = _sample_tokens(shape.seqlen, shape.chunk, nrand, seed=5)
     r = orc.sma(o["Q"], o["E"], o["Cm"], dH, shape.chunk, inp["g"], y_ssd[:, tok], tokens=tok)
     assert_close("o (sampled)", got["o"][:, tok][:, :, heads], r["o"], tol)
