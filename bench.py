@@ -294,7 +294,7 @@ def backward_region(args, dist, dart, shape=FWD):
     """The training pass of the layer at the headline shape: SMA backward
     (dQ, dE, dC, memory and gate gradients) and scan backward (dx, ddt, dA,
     dB, dC) from the forward's memories and boundary states, timed per call
-    with CUDA events.  Both run on CUDA cores."""
+    with CUDA events."""
     dev = torch.device("cuda", torch.cuda.current_device())
     inp = synth.layer_inputs(shape, seed=dist.rank)
     d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
@@ -337,23 +337,30 @@ def backward_region(args, dist, dart, shape=FWD):
     sma_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     scan_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
     ms = dist.max(sma_ms + scan_ms)
-    # algorithmic work of the SMA backward (CUDA cores): per valid (t, c) pair
-    # and head, 4 N P to recompute U = Q dH and V = C dH, 5 N P for the row
-    # gradients (dQ, dE, dC and the score gradient) and 4 N P for the memory
-    # gradient sum_t ds Q E^T + p C do^T
+    # algorithmic work of the SMA backward: per valid (t, c) pair and head,
+    # 4 N P for U = Q dH and V = C dH, 5 N P for the row gradients (dQ, dE,
+    # dC and the score gradient) and 4 N P for the memory gradient
+    # sum_t ds Q E^T + p C do^T
     pairs = sum(min(S, L - k * S) * k for k in range(shape.nchunks)) * B * H
     sma_flop = 13.0 * N * P * pairs
-    fp32_peak = SMS * FP32_LANES_PER_SM * 2 * 1965e6 / 1e12
+    achieved = sma_flop / (sma_ms / 1e3) / 1e12
+    # bf16 with N = 128, P = 64 and S a multiple of 128 runs on the tensor cores
+    tc = shape.dtype == "bf16" and N == 128 and P == 64 and S % 128 == 0
+    if tc:
+        peaks, which = load_peaks()
+        peak, bound, src = peaks["bf16_tflops"], "tensor", f"bf16_tflops ({which})"
+    else:
+        peak, bound = SMS * FP32_LANES_PER_SM * 2 * 1965e6 / 1e12, "alu"
+        src = "fp32 FMA: 148 SMs x 128 lanes x 2 flop x 1965 MHz"
     return {"value": dist.world * B * L / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms, "steps": steps,
             "warmup": warm, "sma_backward_ms": sma_ms, "scan_backward_ms": scan_ms, "launches": n1 - n0,
-            "sma_backward_roofline": {"bound": "alu", "achieved": sma_flop / (sma_ms / 1e3) / 1e12,
-                                      "peak": fp32_peak, "unit": "TFLOP/s",
-                                      "frac": sma_flop / (sma_ms / 1e3) / 1e12 / fp32_peak,
-                                      "flop_per_launch": sma_flop,
-                                      "peak_source": "fp32 FMA: 148 SMs x 128 lanes x 2 flop x 1965 MHz"},
+            "sma_backward_roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                                      "frac": achieved / peak, "flop_per_launch": sma_flop, "peak_source": src},
             "config": {"workload": "dart_layer_bwd_L8k", "batch": B, "seqlen": L, "nheads": H, "headdim": P,
                        "dstate": N, "chunk": S},
-            "path": "dart_sma_backward + dart_ssd_scan_backward (CUDA cores) from the forward's memories"}
+            "path": ("dart_sma_backward (tcgen05: sma_bwd_q_tc, sma_bwd_dh_tc)" if tc else
+                     "dart_sma_backward (CUDA cores)")
+                    + " + dart_ssd_scan_backward (chunk-parallel, CUDA cores) from the forward's memories"}
 
 
 def e2e_region(args, dist, dart, inp):

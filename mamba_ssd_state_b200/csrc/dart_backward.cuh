@@ -13,7 +13,8 @@ struct SmaBwdArgs {
     float* dQ; float* dE; float* dCm; float* ddH; float* dg;   // outputs (fp32); dCm [B,L,G,N]
     int* status;
     // workspace views (set by launch_sma_bwd)
-    float* pbuf; float* dsbuf;              // [B,H,L,C] softmax weights and score gradients
+    float* pbuf; float* dsbuf;              // softmax weights and score gradients: [B,H,L,C] on CUDA
+                                            // cores, [B,H,C,L] on the tensor cores
     float* dCh;                             // [B,L,H,N] per-head dC
     float* gpart;                           // [B,H,tiles] per-tile dg
 };
@@ -38,6 +39,10 @@ struct ScanBwdArgs {
 };
 
 size_t sma_bwd_workspace_bytes(int B, int L, int H, int N, int S);
+// sma_bwd_tc.cu: the tensor-core SMA backward (bf16, N = 128, P = 64, S a multiple of 128)
+bool sma_bwd_tc_applicable(int N, int P, int S, dart_dtype dt);
+int sma_bwd_tc_tiles(int B, int L, int H, int S);
+cudaError_t launch_sma_bwd_tc(const SmaBwdArgs& a, cudaStream_t st);
 cudaError_t launch_sma_bwd(SmaBwdArgs a, void* workspace, dart_dtype dt, cudaStream_t st);
 size_t scan_bwd_workspace_bytes(int B, int L, int H, int N, int P, int S);
 bool scan_bwd_supported(int N, int P, int S);

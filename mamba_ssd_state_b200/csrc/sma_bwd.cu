@@ -312,7 +312,9 @@ cudaError_t run(const SmaBwdArgs& a, cudaStream_t st) {
 size_t sma_bwd_workspace_bytes(int B, int L, int H, int N, int S) {
     if (B <= 0 || L <= 0 || H <= 0 || N <= 0 || S <= 0) return 0;
     const size_t C = (size_t)(L + S - 1) / S;
-    const size_t tiles = (size_t)(L + kTQ - 1) / kTQ;
+    // dg partials: one per 32-token tile (CUDA cores) or per 128-token tile of every chunk (tensor cores)
+    size_t tiles = (size_t)(L + kTQ - 1) / kTQ;
+    if (S % 128 == 0 && C * (size_t)(S / 128) > tiles) tiles = C * (size_t)(S / 128);
     auto pad = [](size_t bytes) { return (bytes + 255) & ~size_t(255); };
     return 2 * pad(sizeof(float) * B * H * L * C)          // p, ds per (token, memory)
            + pad(sizeof(float) * B * L * H * N)            // dC per head
@@ -330,6 +332,18 @@ cudaError_t launch_sma_bwd(SmaBwdArgs a, void* workspace, dart_dtype dt, cudaStr
     a.dCh = reinterpret_cast<float*>(w);
     w += pad(sizeof(float) * a.B * a.L * a.H * a.N);
     a.gpart = reinterpret_cast<float*>(w);
+    if (sma_bwd_tc_applicable(a.N, a.P, a.S, dt)) {
+        // tensor cores: p and ds in [B,H,C,L]; dC per head and dg per tile reduced as below
+        cudaError_t e = launch_sma_bwd_tc(a, st);
+        if (e != cudaSuccess) return e;
+        const size_t ndc = (size_t)a.B * a.L * a.G * a.N;
+        sma_bwd_reduce_dc<<<(unsigned)((ndc + 255) / 256), 256, 0, st>>>(a, a.N);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        sma_bwd_reduce_dg<<<1, 32, 0, st>>>(a, sma_bwd_tc_tiles(a.B, a.L, a.H, a.S));
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        count_launches(2);
+        return cudaSuccess;
+    }
 #define DART_SMA_BWD_CASE(NN, PP)                                                    \
     if (a.N == NN && a.P == PP)                                                      \
         return dt == DART_F32 ? run<float, NN, PP>(a, st) : run<__nv_bfloat16, NN, PP>(a, st);

@@ -2,9 +2,10 @@
 backward oracle (``oracle/dart_backward.py``, autograd over the pinned
 forward restatement), on the same seeded inputs.  Both sides read the same
 float32-exact inputs, so the only differences are fp32 accumulation:
-max|err| / max|ref| <= 1e-4 for float32 inputs and <= 1e-3 for bf16 inputs
-(each value exactly representable; the kernels accumulate in fp32 over up to
-N * P terms per output, twice as deep as the forward)."""
+max|err| / max|ref| <= 1e-4 for float32 inputs (CUDA cores, fp32 throughout)
+and <= 1e-2 for bf16 inputs: the tensor-core path rounds the scaled operand
+rows (ds / sqrt(N)) E and p do to bf16 (2^-9 relative) before its products,
+which accumulate in fp32, as the forward's bf16 memories do."""
 import numpy as np
 import pytest
 import torch
@@ -38,9 +39,12 @@ def _case(Bz, L, H, P, N, S, dtype, seed):
 @pytest.mark.parametrize("shape,dtype,tol", [
     ((1, 3 * 64 + 17, 2, 16, 16, 64), torch.float32, 1e-4),
     ((2, 3 * 128 + 40, 2, 64, 64, 128), torch.float32, 1e-4),
-    ((1, 3 * 256, 2, 64, 128, 256), torch.bfloat16, 1e-3),
-    ((1, 2 * 256 + 77, 3, 64, 128, 256), torch.bfloat16, 1e-3),
-], ids=["f32_N16_ragged", "f32_N64_B2_ragged", "bf16_N128", "bf16_N128_ragged"])
+    ((1, 3 * 256, 2, 64, 128, 256), torch.bfloat16, 1e-2),
+    ((1, 2 * 256 + 77, 3, 64, 128, 256), torch.bfloat16, 1e-2),
+    ((2, 3 * 128 + 50, 2, 64, 128, 128), torch.bfloat16, 1e-2),
+    ((1, 100, 2, 64, 128, 256), torch.bfloat16, 1e-2),
+], ids=["f32_N16_ragged", "f32_N64_B2_ragged", "bf16_N128", "bf16_N128_ragged", "bf16_S128_B2_ragged",
+        "bf16_single_partial_chunk"])
 def test_sma_backward_matches_oracle(shape, dtype, tol):
     Bz, L, H, P, N, S = shape
     g = 0.7
@@ -50,7 +54,7 @@ def test_sma_backward_matches_oracle(shape, dtype, tol):
     ref = dart_backward.sma_grads(*(inp[k].double().numpy() for k in ("Q", "E", "Cm", "dH")), S, g,
                                   dy.double().numpy())
     for k in ("dQ", "dE", "dCm", "ddH"):
-        assert_close(k, got[k], ref[k], tol)
+        print(k, assert_close(k, got[k], ref[k], tol))
     assert abs(float(got["dg"][0]) - float(ref["dg"])) <= tol * max(1.0, abs(float(ref["dg"])))
 
 
