@@ -70,6 +70,8 @@ def parse():
     p.add_argument("--no-configs", action="store_true",
                    help="skip the other forward workloads (B=4, L=2048 and B=1, L=65536)")
     p.add_argument("--no-backward", action="store_true", help="skip the backward region")
+    p.add_argument("--backward-heads", type=int, default=0,
+                   help="heads of the backward region (0: the forward's); a smaller case for profiling")
     p.add_argument("--reference-heads", type=int, default=0,
                    help="heads per reference-arm step (default: one per host core, at most 32)")
     return p.parse_args()
@@ -682,7 +684,8 @@ def main():
                 line["gpu_launches"] += r["launches"]
                 del r
         if not args.no_backward:
-            bwd = backward_region(args, dist, dart)
+            bshape = FWD if args.backward_heads <= 0 else dataclasses.replace(FWD, nheads=args.backward_heads)
+            bwd = backward_region(args, dist, dart, bshape)
             line["backward"] = bwd
             line["gpu_launches"] += bwd.pop("launches")
         if not args.no_e2e:
