@@ -362,7 +362,8 @@ def backward_region(args, dist, dart, shape=FWD):
                        "dstate": N, "chunk": S},
             "path": ("dart_sma_backward (tcgen05: sma_bwd_q_tc, sma_bwd_dh_tc)" if tc else
                      "dart_sma_backward (CUDA cores)")
-                    + " + dart_ssd_scan_backward (chunk-parallel, CUDA cores) from the forward's memories"}
+                    + " + dart_ssd_scan_backward (chunk-parallel; intra-chunk products on tcgen05"
+                      " for bf16, N = 128, P = 64) from the forward's memories"}
 
 
 def e2e_region(args, dist, dart, inp):

@@ -33,7 +33,10 @@ struct ScanBwdArgs {
     // workspace views (set by launch_ssd_scan_bwd)
     float* gin;             // [B,H,C,N,P] dS[c], then the adjoint entering chunk c from later chunks
     float* asum;            // [B,H,C] chunk decay sums
-    float* rect;            // [B,H,C,S] the chunk-local decay-gradient term per token
+    float* rect;            // [B,H,C,S] the chunk-local decay-gradient term per token (CUDA cores);
+                            // [6][B,H,C,S] the per-token scalars u, v, q1, colsum and the rowsum
+                            // parts of row blocks 0 and 1 (tensor cores)
+    float* c0;              // [B,H,C] sum(Gin o h_in) (tensor cores)
     float* dBh; float* dCh; // [B,L,H,N] per-head dB, dC
     float* dApart;          // [B,H,C]
 };
@@ -47,5 +50,8 @@ cudaError_t launch_sma_bwd(SmaBwdArgs a, void* workspace, dart_dtype dt, cudaStr
 size_t scan_bwd_workspace_bytes(int B, int L, int H, int N, int P, int S);
 bool scan_bwd_supported(int N, int P, int S);
 cudaError_t launch_ssd_scan_bwd(ScanBwdArgs a, void* workspace, dart_dtype dt, cudaStream_t st);
+// ssd_scan_bwd_tc.cu: the intra-chunk products of the scan backward on the tensor cores
+bool scan_bwd_tc_applicable(int N, int P, int S, dart_dtype dt);
+cudaError_t launch_scan_bwd_quad_tc(const ScanBwdArgs& a, cudaStream_t st);
 
 }  // namespace dart

@@ -42,6 +42,8 @@
 //                           row n and 8 consecutive value columns.
 //   scan_bwd_reduce         dB, dC summed over the heads of each group, dA
 //                           over (b, c), in a fixed order.
+#include <type_traits>
+
 #include "dart_backward.cuh"
 
 namespace dart {
@@ -150,17 +152,32 @@ __global__ void __launch_bounds__(N * P / kCols) scan_bwd_chunk_adjoint(ScanBwdA
 // ---------------------------------------------------------------------------
 // Gin[c] in place of dS[c], last chunk to first; dinit = Gin[-1].
 // ---------------------------------------------------------------------------
+// Eight chunks' dS are loaded before any of them is used, so the loads of a
+// group are in flight together instead of one after another.
 __global__ void scan_bwd_gin_pass(ScanBwdArgs a, int C) {
+    constexpr int kG = 8;
     const size_t NP = (size_t)a.N * a.P;
     const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= (size_t)a.B * a.H * NP) return;
     const size_t bh = i / NP, e = i % NP;
+    float* __restrict__ gin = a.gin + bh * C * NP + e;
+    const float* __restrict__ asum = a.asum + bh * C;
     float g = 0.f;
-    for (int c = C - 1; c >= 0; --c) {
-        float* p = a.gin + (bh * C + c) * NP + e;
-        const float ds = *p;
-        *p = g;
-        g = fmaf(expf(a.asum[bh * C + c]), g, ds);
+    for (int top = C - 1; top >= 0; top -= kG) {
+        float ds[kG], dec[kG];
+#pragma unroll
+        for (int j = 0; j < kG; ++j) {
+            const int c = top - j;
+            ds[j] = c >= 0 ? gin[(size_t)c * NP] : 0.f;
+            dec[j] = c >= 0 ? expf(asum[c]) : 0.f;
+        }
+#pragma unroll
+        for (int j = 0; j < kG; ++j) {
+            const int c = top - j;
+            if (c < 0) break;
+            gin[(size_t)c * NP] = g;
+            g = fmaf(dec[j], g, ds[j]);
+        }
     }
     if (a.dinit) a.dinit[bh * NP + e] = g;
 }
@@ -461,6 +478,60 @@ __global__ void __launch_bounds__(N * P / kCols) scan_bwd_walk(ScanBwdArgs a) {
     if (tid == 0) a.dApart[bhc] = dA_acc;
 }
 
+// The decay gradient of every token of (b, h, c) from the per-token scalars
+// the tensor-core kernel leaves (u, v, q1, colsum and the row blocks' parts of
+// rowsum; ssd_scan_bwd_tc.cu):
+//   Rect_t = Rect_{t+1} + rowsum_t - colsum_t,   gh_t = v_t + a_{t+1} gh_{t+1},
+//   rd_t = E_{t-1},  E_t = a_t E_{t-1} + dt_t u_t,
+//   dl_t = exp(Acum_t) gh_t + Rect_t + exp(Ae) c0 + exp(Ae - Acum_{t-1}) rd_t,
+//   ddt_t = q1_t + A_h dl_t,  dA += dt_t dl_t.
+// One warp per chunk: the lanes stage the chunk's scalars in shared memory,
+// lane 0 runs the three recursions.
+__global__ void __launch_bounds__(32) scan_bwd_scalars(ScanBwdArgs a, int C) {
+    __shared__ float sdt[256], sacum[256], su[256], sv[256], sq[256], srw[256], scl[256];
+    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z, lane = threadIdx.x;
+    const size_t bhc = ((size_t)b * a.H + h) * C + c;
+    const ChunkSpan cs(c, a.S, a.L);
+    const size_t plane = (size_t)a.B * a.H * C * a.S;
+    const float* sc = a.rect + bhc * a.S;
+    for (int t = lane; t < cs.n; t += 32) {
+        sdt[t] = a.dt[((size_t)b * a.L + cs.s0 + t) * a.H + h];
+        su[t] = sc[t];
+        sv[t] = sc[plane + t];
+        sq[t] = sc[2 * plane + t];
+        scl[t] = sc[3 * plane + t];
+        // rowsum of t: the parts of the row blocks up to t's own (block 0 covers every t)
+        srw[t] = sc[4 * plane + t] + (t >= 128 ? sc[5 * plane + t] : 0.f);
+    }
+    __syncwarp();
+    if (lane != 0) return;
+    const float Ah = a.A[h];
+    float run = 0.f;
+    for (int t = 0; t < cs.n; ++t) {
+        run += sdt[t] * Ah;
+        sacum[t] = run;
+    }
+    const float Ae = run, eAc0 = expf(Ae) * a.c0[bhc];
+    // backward: gh (into sv) and Rect (into srw)
+    float gh = 0.f, rect = 0.f;
+    for (int t = cs.n - 1; t >= 0; --t) {
+        gh = t + 1 < cs.n ? fmaf(expf(sdt[t + 1] * Ah), gh, sv[t]) : sv[t];
+        rect += srw[t] - scl[t];
+        sv[t] = gh;
+        srw[t] = rect;
+    }
+    // forward: rd, dl, ddt, dA
+    float E = 0.f, dA = 0.f;
+    for (int t = 0; t < cs.n; ++t) {
+        const float am1 = t > 0 ? sacum[t - 1] : 0.f;
+        const float dl = expf(sacum[t]) * sv[t] + srw[t] + eAc0 + expf(Ae - am1) * E;
+        a.ddt[((size_t)b * a.L + cs.s0 + t) * a.H + h] = sq[t] + Ah * dl;
+        dA = fmaf(sdt[t], dl, dA);
+        E = fmaf(expf(sdt[t] * Ah), E, sdt[t] * su[t]);
+    }
+    a.dApart[bhc] = dA;
+}
+
 // dB, dC [B,L,G,N] summed over the heads of each group (dC plus dC_add when
 // given); dA summed over (b, c) in a fixed order.
 __global__ void scan_bwd_reduce(ScanBwdArgs a, int N, int C) {
@@ -508,6 +579,12 @@ cudaError_t run(const ScanBwdArgs& a, cudaStream_t st) {
         scan_bwd_gin_pass<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(a, C);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
+    if (scan_bwd_tc_applicable(N, P, a.S, std::is_same<T, __nv_bfloat16>::value ? DART_BF16 : DART_F32)) {
+        // the intra-chunk products on the tensor cores, then the per-token recursions
+        if ((e = launch_scan_bwd_quad_tc(a, st)) != cudaSuccess) return e;
+        scan_bwd_scalars<<<grid, 32, 0, st>>>(a, C);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    } else {
     {
         const size_t smem = sizeof(float) * RectSmem<N, P>::floats;
         auto k = scan_bwd_rect<T, N, P>;
@@ -523,6 +600,7 @@ cudaError_t run(const ScanBwdArgs& a, cudaStream_t st) {
             return e;
         k<<<grid, NT, smem, st>>>(a);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
     }
     const size_t n = (size_t)a.B * a.L * a.G * N;
     const size_t m = n > (size_t)a.H ? n : (size_t)a.H;
@@ -541,7 +619,8 @@ size_t scan_bwd_workspace_bytes(int B, int L, int H, int N, int P, int S) {
     const size_t C = ((size_t)L + S - 1) / S;
     return pad256(sizeof(float) * B * H * C * N * P)    // dS, then Gin, per chunk
            + pad256(sizeof(float) * B * H * C)          // Ae per chunk
-           + pad256(sizeof(float) * B * H * C * S)      // Rect per token slot
+           + pad256(sizeof(float) * 6 * B * H * C * S)  // per-token scalars (Rect alone on CUDA cores)
+           + pad256(sizeof(float) * B * H * C)          // sum(Gin o h_in) per chunk
            + 2 * pad256(sizeof(float) * B * L * H * N)  // dB, dC per head
            + pad256(sizeof(float) * B * H * C);         // dA per (b, h, c)
 }
@@ -559,7 +638,9 @@ cudaError_t launch_ssd_scan_bwd(ScanBwdArgs a, void* workspace, dart_dtype dt, c
     a.asum = reinterpret_cast<float*>(w);
     w += pad256(sizeof(float) * a.B * a.H * C);
     a.rect = reinterpret_cast<float*>(w);
-    w += pad256(sizeof(float) * a.B * a.H * C * a.S);
+    w += pad256(sizeof(float) * 6 * a.B * a.H * C * a.S);
+    a.c0 = reinterpret_cast<float*>(w);
+    w += pad256(sizeof(float) * a.B * a.H * C);
     a.dBh = reinterpret_cast<float*>(w);
     w += pad256(sizeof(float) * a.B * a.L * a.H * a.N);
     a.dCh = reinterpret_cast<float*>(w);

@@ -216,8 +216,9 @@ def test_scan_backward_workspace_and_validation(lib):
     d = dart.Dims(2, 500, 3, 64, 128, 256, 1)
     pad = lambda b: (b + 255) // 256 * 256
     C = 2   # ceil(500 / 256)
-    # chunk adjoints, chunk decay sums, per-token decay term, per-head dB and dC, per-chunk dA
-    want = (pad(4 * 2 * 3 * C * 128 * 64) + pad(4 * 2 * 3 * C) + pad(4 * 2 * 3 * C * 256)
+    # chunk adjoints, chunk decay sums, five per-token scalars, one scalar per chunk,
+    # per-head dB and dC, per-chunk dA
+    want = (pad(4 * 2 * 3 * C * 128 * 64) + pad(4 * 2 * 3 * C) + pad(4 * 6 * 2 * 3 * C * 256) + pad(4 * 2 * 3 * C)
             + 2 * pad(4 * 2 * 500 * 3 * 128) + pad(4 * 2 * 3 * C))
     assert lib.dart_ssd_scan_backward_workspace_bytes(ctypes.byref(d)) == want
     f = lib.dart_ssd_scan_backward

@@ -75,8 +75,11 @@ SCAN_CASES = [
     ((2, 3 * 128 + 40, 2, 64, 64, 128), "f32", False),
     ((1, 3 * 256, 2, 64, 128, 256), "bf16", False),
     ((1, 2 * 256 + 77, 3, 64, 128, 256), "bf16", True),
+    ((2, 3 * 128 + 50, 2, 64, 128, 128), "bf16", True),
+    ((1, 256 + 100, 2, 64, 128, 256), "bf16", False),
 ]
-SCAN_IDS = ["f32_N16_ragged_init", "f32_N64_B2_ragged", "bf16_N128", "bf16_N128_ragged_init"]
+SCAN_IDS = ["f32_N16_ragged_init", "f32_N64_B2_ragged", "bf16_N128", "bf16_N128_ragged_init", "bf16_S128_B2_ragged_init",
+            "bf16_second_block_past_the_end"]
 TOL_FWD_INPUTS = {"f32": 1e-4, "bf16": 2e-2}   # bf16: the tensor-core forward's states carry bf16 rounding
 
 
