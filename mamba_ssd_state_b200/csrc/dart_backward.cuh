@@ -53,5 +53,6 @@ cudaError_t launch_ssd_scan_bwd(ScanBwdArgs a, void* workspace, dart_dtype dt, c
 // ssd_scan_bwd_tc.cu: the intra-chunk products of the scan backward on the tensor cores
 bool scan_bwd_tc_applicable(int N, int P, int S, dart_dtype dt);
 cudaError_t launch_scan_bwd_quad_tc(const ScanBwdArgs& a, cudaStream_t st);
+cudaError_t launch_scan_bwd_dS_tc(const ScanBwdArgs& a, cudaStream_t st);
 
 }  // namespace dart

@@ -568,8 +568,11 @@ cudaError_t run(const ScanBwdArgs& a, cudaStream_t st) {
     constexpr int NT = N * P / kCols;
     const int C = (a.L + a.S - 1) / a.S;
     const dim3 grid(C, a.H, a.B);
+    const bool tc = scan_bwd_tc_applicable(N, P, a.S, std::is_same<T, __nv_bfloat16>::value ? DART_BF16 : DART_F32);
     cudaError_t e;
-    {
+    if (tc) {
+        if ((e = launch_scan_bwd_dS_tc(a, st)) != cudaSuccess) return e;
+    } else {
         const size_t smem = sizeof(float) * (kTT * (N + P) + kTT);
         scan_bwd_chunk_adjoint<T, N, P><<<grid, NT, smem, st>>>(a);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -579,7 +582,7 @@ cudaError_t run(const ScanBwdArgs& a, cudaStream_t st) {
         scan_bwd_gin_pass<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(a, C);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    if (scan_bwd_tc_applicable(N, P, a.S, std::is_same<T, __nv_bfloat16>::value ? DART_BF16 : DART_F32)) {
+    if (tc) {
         // the intra-chunk products on the tensor cores, then the per-token recursions
         if ((e = launch_scan_bwd_quad_tc(a, st)) != cudaSuccess) return e;
         scan_bwd_scalars<<<grid, 32, 0, st>>>(a, C);

@@ -66,9 +66,11 @@ struct ScanBwdTcParams {
     CUtensorMap tmap_b, tmap_c;   // (N, G, L, B), box (64, 1, 128, 1)
     CUtensorMap tmap_x;           // (P, H, L, B), box (64, 1, 128, 1)
     const float* dt; const float* A; const float* dy;
-    const float* gin; const float* ddH; const float* states; const float* init;
+    float* gin;    // the chunk adjoints: dS written by scan_bwd_dS_tc, Gin read by scan_bwd_quad_tc
+    const float* ddH; const float* states; const float* init;
     float* dx; float* dBh; float* dCh;
     float* scal;   // [6][B,H,C,S]: u, v, q1, colsum, rowsum parts of row blocks 0 and 1
+    float* asum;   // [B,H,C] chunk decay sums (written by scan_bwd_dS_tc)
     float* c0;     // [B,H,C]: sum(Gin o h_in)
     int B, L, H, S, C, HG, R;
     int* status;
@@ -294,17 +296,24 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_quad_tc(const __grid_con
             const float* hi = c > 0 ? p.states + (((size_t)bh * p.C + (c - 1)) * kN + n) * kP
                                     : (p.init ? p.init + ((size_t)bh * kN + n) * kP : nullptr);
             float c0p = 0.f;
+            auto ld8 = [](const float* src, int q, float* f) {   // 8 floats at 8 q (rows are 256-byte aligned)
+                const float4 a = __ldg(reinterpret_cast<const float4*>(src) + 2 * q);
+                const float4 d = __ldg(reinterpret_cast<const float4*>(src) + 2 * q + 1);
+                f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = d.x; f[5] = d.y; f[6] = d.z; f[7] = d.w;
+            };
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
-                float g8[8], r8[8], h8[8];
+                float g8[8], d8[8], h8[8];
+                ld8(gi, q, g8);
+                if (gd) ld8(gd, q, d8);
+                if (hi) ld8(hi, q, h8);
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
-                    g8[k] = __ldg(gi + 8 * q + k);
-                    r8[k] = g8[k] + (gd ? __ldg(gd + 8 * q + k) : 0.f);
-                    h8[k] = hi ? __ldg(hi + 8 * q + k) : 0.f;
+                    if (!hi) h8[k] = 0.f;
                     c0p = fmaf(g8[k], h8[k], c0p);
+                    g8[k] += gd ? d8[k] : 0.f;   // R = Gin + gD
                 }
-                st_v4(chunk_addr(sb + kOffR, n, q), pack8(r8));
+                st_v4(chunk_addr(sb + kOffR, n, q), pack8(g8));
                 st_v4(chunk_addr(sb + kOffH, n, q), pack8(h8));
             }
             c0p = warp_sum(c0p);
@@ -532,40 +541,209 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_quad_tc(const __grid_con
     }
 }
 
-}  // namespace
 
-bool scan_bwd_tc_applicable(int N, int P, int S, dart_dtype dt) {
-    return dt == DART_BF16 && N == kN && P == kP && (S == 128 || S == 256);
+// ===========================================================================
+// dS[c] = sum_s exp(Acum_s) C_s dy_s^T  (N x P) and the chunk's decay sum
+// ===========================================================================
+// One CTA per (b, h, c): C_T (S x N, TMA) is the MN-major A operand (M = N),
+// the rows exp(Acum_s) dy_s are built by four warps as two bf16 MN-major B
+// operands, the rounded value and the remainder (together ~16 bits of the
+// fp32 value, so dS and the adjoints built from it keep fp32-like accuracy),
+// and the product accumulates in TMEM over the S tokens.
+constexpr uint32_t ds_kOffC = 0;                 // 2 n-panels x S rows (S * 256 B)
+constexpr uint32_t ds_kOffHi = 4 * kPanel;       // S rows x 128 B
+constexpr uint32_t ds_kOffLo = 6 * kPanel;
+constexpr uint32_t ds_kOffF = 8 * kPanel;        // acum2[256]
+constexpr uint32_t ds_kOffBar = ds_kOffF + 256 * 4;
+constexpr uint32_t ds_kSmemBytes = ds_kOffBar + 64 + 1024;
+enum DsBar { DS_LD = 0, DS_OPS = 1, DS_DONE = 2, ds_NUM_BARS = 3 };
+static_assert(ds_kSmemBytes <= 232448, "shared memory layout");
+
+__global__ void __launch_bounds__(kThreads, 1) scan_bwd_dS_tc(const __grid_constant__ ScanBwdTcParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sb = smem_u32(smem);
+    float* acum2 = reinterpret_cast<float*>(smem + ds_kOffF);
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + ds_kOffBar + ds_NUM_BARS * 8);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+    auto bar = [&](int i) -> uint32_t { return sb + ds_kOffBar + 8u * (uint32_t)i; };
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int c = blockIdx.x % p.C, bh = blockIdx.x / p.C;
+    const int b = bh / p.H, h = bh % p.H, grp = h / p.HG;
+    const size_t bhc = (size_t)bh * p.C + c;
+    const int s0 = c * p.S, n_chunk = min(p.L, s0 + p.S) - s0;
+    const uint32_t rowblk = (uint32_t)kRB * 128u;    // 128 rows of one panel
+    const uint32_t cpanel = (uint32_t)p.R * rowblk;  // one n-panel over all S rows
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar(DS_LD), 1);
+        mbar_init(bar(DS_OPS), 4);
+        mbar_init(bar(DS_DONE), 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_holder), 64);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+    const WaitCtx wc{abort_flag, p.status, 7};
+
+    if (warp == 0) {
+        if (lane == 0) {
+            tma_prefetch_desc(&p.tmap_c);
+            mbar_expect_tx(bar(DS_LD), (uint32_t)p.R * 2u * kPanel);
+            for (int r = 0; r < p.R; ++r)
+                for (int nb = 0; nb < 2; ++nb)
+                    tma_load_4d(sb + ds_kOffC + (uint32_t)nb * cpanel + (uint32_t)r * rowblk, &p.tmap_c, bar(DS_LD), 64 * nb,
+                                grp, s0 + r * kRB, b);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        bool ok = mbar_wait_warp(bar(DS_LD), 0, wc, 1);
+        if (ok) ok = mbar_wait_warp(bar(DS_OPS), 0, wc, 2);
+        tc_fence_after();
+        if (ok && lane == 0) {
+            const uint32_t idesc = idesc_bf16_f32(kN, kP, true, true);   // A = C_T^T (MN-major), B MN-major
+            const int ksteps = p.S / 16;
+            for (int kk = 0; kk < ksteps; ++kk) {
+                const uint64_t ad = smem_desc_sw128(sb + ds_kOffC + (uint32_t)kk * 2048, cpanel, 1024);
+                mma_f16_ss(tmem, ad, smem_desc_sw128(sb + ds_kOffHi + (uint32_t)kk * 2048, kPanel, 1024), idesc,
+                           kk > 0 ? 1u : 0u);
+                mma_f16_ss(tmem, ad, smem_desc_sw128(sb + ds_kOffLo + (uint32_t)kk * 2048, kPanel, 1024), idesc, 1u);
+            }
+            mma_commit(bar(DS_DONE));
+        }
+        __syncwarp();
+    } else {
+        const int quad = warp & 3, row = quad * 32 + lane;
+        const float Ah = p.A[h];
+        if (warp == 2) {   // the chunk's log2 decay prefix and its sum
+            const int per = (p.S + 31) / 32, a0 = lane * per;
+            float run = 0.f;
+            for (int k = 0; k < per && a0 + k < p.S; ++k) {
+                const int t = a0 + k;
+                run += (t < n_chunk ? p.dt[((size_t)b * p.L + s0 + t) * p.H + h] : 0.f) * Ah * kLog2e;
+                acum2[t] = run;
+            }
+            float off = run;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float v = __shfl_up_sync(0xffffffffu, off, o);
+                if (lane >= o) off += v;
+            }
+            off -= run;
+            for (int k = 0; k < per && a0 + k < p.S; ++k) acum2[a0 + k] += off;
+            if (lane == 31) p.asum[bhc] = (off + run) * (1.f / kLog2e);   // Ae = sum of dt A over the chunk
+        }
+        named_bar_sync(1, 128);
+        for (int r = 0; r < p.R; ++r) {
+            const int t = r * kRB + row;
+            const bool valid = t < n_chunk;
+            const float w = valid ? exp2f(acum2[t]) : 0.f;
+            const float* src = p.dy + (((size_t)b * p.L + s0 + t) * p.H + h) * kP;
+            const uint32_t hi = sb + ds_kOffHi + (uint32_t)r * rowblk, lo = sb + ds_kOffLo + (uint32_t)r * rowblk;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                float f[8], g[8];
+                if (valid) {
+                    const float4 a = __ldg(reinterpret_cast<const float4*>(src) + 2 * q);
+                    const float4 d = __ldg(reinterpret_cast<const float4*>(src) + 2 * q + 1);
+                    f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = d.x; f[5] = d.y; f[6] = d.z; f[7] = d.w;
+                } else {
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) f[k] = 0.f;
+                }
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    f[k] *= w;
+                    g[k] = f[k] - __bfloat162float(__float2bfloat16_rn(f[k]));
+                }
+                st_v4(chunk_addr(hi, row, q), pack8(f));
+                st_v4(chunk_addr(lo, row, q), pack8(g));
+            }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(DS_OPS));
+        bool ok = mbar_wait_warp(bar(DS_DONE), 0, wc, 3);
+        if (ok) {
+            tc_fence_after();
+            float v[32];
+            float* dst = p.gin + (bhc * kN + row) * kP;   // TMEM lane = state row n
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {
+                tmem_ld_32x32b_x32(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(32 * part), v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    reinterpret_cast<float4*>(dst + 32 * part)[k] =
+                        make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 64);
+    }
 }
 
-cudaError_t launch_scan_bwd_quad_tc(const ScanBwdArgs& a, cudaStream_t st) {
-    ScanBwdTcParams p;
+bool make_params(const ScanBwdArgs& a, ScanBwdTcParams& p) {
     memset(&p, 0, sizeof(p));
     const int C = (a.L + a.S - 1) / a.S;
     {
         const uint64_t dims[4] = {(uint64_t)kN, (uint64_t)a.G, (uint64_t)a.L, (uint64_t)a.B};
         const uint64_t strides[3] = {(uint64_t)kN * 2, (uint64_t)a.G * kN * 2, (uint64_t)a.L * a.G * kN * 2};
         const uint32_t box[4] = {64, 1, kRB, 1};
-        if (!encode_tile_map_bf16(&p.tmap_b, 4, a.Bm, dims, strides, box)) return cudaErrorInvalidValue;
-        if (!encode_tile_map_bf16(&p.tmap_c, 4, a.Cm, dims, strides, box)) return cudaErrorInvalidValue;
+        if (!encode_tile_map_bf16(&p.tmap_b, 4, a.Bm, dims, strides, box)) return false;
+        if (!encode_tile_map_bf16(&p.tmap_c, 4, a.Cm, dims, strides, box)) return false;
     }
     {
         const uint64_t dims[4] = {(uint64_t)kP, (uint64_t)a.H, (uint64_t)a.L, (uint64_t)a.B};
         const uint64_t strides[3] = {(uint64_t)kP * 2, (uint64_t)a.H * kP * 2, (uint64_t)a.L * a.H * kP * 2};
         const uint32_t box[4] = {64, 1, kRB, 1};
-        if (!encode_tile_map_bf16(&p.tmap_x, 4, a.x, dims, strides, box)) return cudaErrorInvalidValue;
+        if (!encode_tile_map_bf16(&p.tmap_x, 4, a.x, dims, strides, box)) return false;
     }
     p.dt = a.dt; p.A = a.A; p.dy = a.dy;
     p.gin = a.gin; p.ddH = a.ddH; p.states = a.states; p.init = a.init;
     p.dx = a.dx; p.dBh = a.dBh; p.dCh = a.dCh;
-    p.scal = a.rect; p.c0 = a.c0;
+    p.scal = a.rect; p.c0 = a.c0; p.asum = a.asum;
     p.B = a.B; p.L = a.L; p.H = a.H; p.S = a.S; p.C = C; p.HG = a.H / a.G; p.R = a.S / kRB;
     p.status = a.status;
+    return true;
+}
+
+}  // namespace
+
+bool scan_bwd_tc_applicable(int N, int P, int S, dart_dtype dt) {
+    return dt == DART_BF16 && N == kN && P == kP && (S == 128 || S == 256);
+}
+
+cudaError_t launch_scan_bwd_dS_tc(const ScanBwdArgs& a, cudaStream_t st) {
+    ScanBwdTcParams p;
+    if (!make_params(a, p)) return cudaErrorInvalidValue;
+    cudaError_t e;
+    if ((e = cudaFuncSetAttribute(scan_bwd_dS_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ds_kSmemBytes)) !=
+        cudaSuccess)
+        return e;
+    scan_bwd_dS_tc<<<a.B * a.H * p.C, kThreads, ds_kSmemBytes, st>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_scan_bwd_quad_tc(const ScanBwdArgs& a, cudaStream_t st) {
+    ScanBwdTcParams p;
+    if (!make_params(a, p)) return cudaErrorInvalidValue;
     cudaError_t e;
     if ((e = cudaFuncSetAttribute(scan_bwd_quad_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes)) !=
         cudaSuccess)
         return e;
-    scan_bwd_quad_tc<<<a.B * a.H * C * p.R, kThreads, kSmemBytes, st>>>(p);
+    scan_bwd_quad_tc<<<a.B * a.H * p.C * p.R, kThreads, kSmemBytes, st>>>(p);
     return cudaGetLastError();
 }
 
