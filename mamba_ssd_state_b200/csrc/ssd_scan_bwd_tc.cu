@@ -54,10 +54,10 @@ constexpr uint32_t kOffR = 6 * kPanel;        // R [n][p]
 constexpr uint32_t kOffH = 7 * kPanel;        // h_in [n][p]
 constexpr uint32_t kOffO = 8 * kPanel;        // the other block: C_1 and dy_1 (block 0) or B_0 and x_0 (block 1)
 constexpr uint32_t kOffOp = 11 * kPanel;      // operand rows built by the threads (2 panels)
-constexpr uint32_t kOffF = 13 * kPanel;       // acum2[256], dtv[256], red[16], colred[4][128]
-constexpr uint32_t kOffBar = kOffF + 2 * 256 * 4 + 64 + 4 * 128 * 4;
+constexpr uint32_t kOffF = 13 * kPanel;       // acum2[256], dtv[256], red[16], colred[4][128], xch[2][2][128] float2
+constexpr uint32_t kOffBar = kOffF + 2 * 256 * 4 + 64 + 4 * 128 * 4 + 2 * 2 * 128 * 8;
 constexpr uint32_t kSmemBytes = kOffBar + 64 + 1024;
-constexpr int kThreads = 64 + 128;
+constexpr int kThreads = 64 + 256;   // TMA, MMA, two warps per TMEM lane quadrant
 constexpr uint32_t kColDX = 0, kColDB = 64, kColDC = 192, kColG = 320;
 enum Bar { LD = 0, PREP = 1, MMA_DONE = 2, OP_READY = 3, NUM_BARS = 4 };
 static_assert(kSmemBytes <= 232448 && NUM_BARS * 8 + 8 <= 64, "shared memory layout");
@@ -134,7 +134,7 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_quad_tc(const __grid_con
     const uint32_t sb = smem_u32(smem);
     float* acum2 = reinterpret_cast<float*>(smem + kOffF);   // log2(e) Acum over the chunk
     float* dtv = acum2 + 256;
-    float* red = dtv + 256;                                  // [4] c0 partials
+    float* red = dtv + 256;                                  // [8] c0 partials
     float* colred = red + 16;                                // [4 warps][128 columns] W sums
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + kOffBar + NUM_BARS * 8);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
@@ -151,9 +151,9 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_quad_tc(const __grid_con
 
     if (threadIdx.x == 0) {
         mbar_init(bar(LD), 1);
-        mbar_init(bar(PREP), 4);
+        mbar_init(bar(PREP), 8);
         mbar_init(bar(MMA_DONE), 1);
-        mbar_init(bar(OP_READY), 4);
+        mbar_init(bar(OP_READY), 8);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -255,13 +255,27 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_quad_tc(const __grid_con
         }
     } else {
         // ------------------------------------------------------- the rows
-        const int quad = warp & 3;
+        // Two warps per TMEM lane quadrant: warp half h owns the value columns
+        // [32h, 32h+32), the state columns [64h, 64h+64) and the token columns
+        // [64h, 64h+64) of every 128-column block; the row sums of the two
+        // halves are exchanged in shared memory.
+        const int quad = warp & 3, half = (warp - 2) >> 2;
         const int row = quad * 32 + lane;
         const int tl = i * kRB + row;            // token index within the chunk
         const bool valid = tl < n_chunk;
         const size_t tok = (size_t)b * p.L + s0 + tl;
         const uint32_t t_lane = tmem + ((uint32_t)(quad * 32) << 16);
         const float Ah = p.A[h];
+        float2* xch = reinterpret_cast<float2*>(colred + 4 * 128);   // [2 parity][2 half][128 rows]
+        int xi = 0;
+        // (a, b) of this row plus the other half's
+        auto exchange = [&](float a, float bb) -> float2 {
+            xch[((xi & 1) * 2 + half) * 128 + row] = make_float2(a, bb);
+            named_bar_sync(2 + quad, 64);
+            const float2 o = xch[((xi & 1) * 2 + (1 - half)) * 128 + row];
+            ++xi;
+            return make_float2(a + o.x, bb + o.y);
+        };
         // the chunk's log2 decay prefix (warp 2), then everyone
         if (warp == 2) {
             const int per = (p.S + 31) / 32, a0 = lane * per;
@@ -282,27 +296,42 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_quad_tc(const __grid_con
             off -= run;
             for (int k = 0; k < per && a0 + k < p.S; ++k) acum2[a0 + k] += off;
         }
-        // dy of block i (and of block 1 for block 0), R and h_in as bf16 operands; c0
-        row_to_bf16(sb + kOffDI, row, p.dy + (tok * p.H + h) * kP, valid);
-        if (other && i == 0) {
-            const int tl1 = kRB + row;
-            row_to_bf16(sb + kOffO + 2 * kPanel, row, p.dy + (((size_t)b * p.L + s0 + tl1) * p.H + h) * kP,
-                        tl1 < n_chunk);
-        }
+        // 8 floats of a 256-byte-aligned row at 8 q
+        auto ld8 = [](const float* src, int q, float* f) {
+            const float4 a = __ldg(reinterpret_cast<const float4*>(src) + 2 * q);
+            const float4 d = __ldg(reinterpret_cast<const float4*>(src) + 2 * q + 1);
+            f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = d.x; f[5] = d.y; f[6] = d.z; f[7] = d.w;
+        };
+        // this half's columns of dy (block i, and block 1 for block 0), R and h_in as bf16; c0
         {
+            auto dy_half = [&](uint32_t panel, int r, const float* src, bool ok_row) {
+#pragma unroll
+                for (int qq = 0; qq < 4; ++qq) {
+                    const int q = 4 * half + qq;
+                    float f[8];
+                    if (ok_row) ld8(src, q, f);
+                    else {
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) f[k] = 0.f;
+                    }
+                    st_v4(chunk_addr(panel, r, q), pack8(f));
+                }
+            };
+            dy_half(sb + kOffDI, row, p.dy + (tok * p.H + h) * kP, valid);
+            if (other && i == 0) {
+                const int tl1 = kRB + row;
+                dy_half(sb + kOffO + 2 * kPanel, row, p.dy + (((size_t)b * p.L + s0 + tl1) * p.H + h) * kP,
+                        tl1 < n_chunk);
+            }
             const int n = row;
             const float* gi = p.gin + (bhc * kN + n) * kP;
             const float* gd = p.ddH ? p.ddH + (bhc * kN + n) * kP : nullptr;
             const float* hi = c > 0 ? p.states + (((size_t)bh * p.C + (c - 1)) * kN + n) * kP
                                     : (p.init ? p.init + ((size_t)bh * kN + n) * kP : nullptr);
             float c0p = 0.f;
-            auto ld8 = [](const float* src, int q, float* f) {   // 8 floats at 8 q (rows are 256-byte aligned)
-                const float4 a = __ldg(reinterpret_cast<const float4*>(src) + 2 * q);
-                const float4 d = __ldg(reinterpret_cast<const float4*>(src) + 2 * q + 1);
-                f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = d.x; f[5] = d.y; f[6] = d.z; f[7] = d.w;
-            };
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
+            for (int qq = 0; qq < 4; ++qq) {
+                const int q = 4 * half + qq;
                 float g8[8], d8[8], h8[8];
                 ld8(gi, q, g8);
                 if (gd) ld8(gd, q, d8);
@@ -317,11 +346,12 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_quad_tc(const __grid_con
                 st_v4(chunk_addr(sb + kOffH, n, q), pack8(h8));
             }
             c0p = warp_sum(c0p);
-            if (lane == 0) red[quad] = c0p;
+            if (lane == 0) red[warp - 2] = c0p;
         }
         fence_proxy_async_smem();
-        named_bar_sync(1, 128);                  // acum2, dtv and red visible to all row threads
-        if (threadIdx.x == 64 && i == 0) p.c0[bhc] = (red[0] + red[1]) + (red[2] + red[3]);
+        named_bar_sync(1, 256);                  // acum2, dtv and red visible to all row threads
+        if (threadIdx.x == 64 && i == 0)
+            p.c0[bhc] = ((red[0] + red[1]) + (red[2] + red[3])) + ((red[4] + red[5]) + (red[6] + red[7]));
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(PREP));
         bool ok = mbar_wait_warp(bar(LD), 0, wc, 4);   // the TMA rows are read below
@@ -347,33 +377,39 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_quad_tc(const __grid_con
         // ---- round 0: u, v; operand f B_i -----------------------------------
         wait_round();
         {
-            float rb[64], hc[64];
+            float rb[32], hc[32];
             if (ok) {
-                tmem_ld_32x32b_x32(t_lane + kColG, rb);
-                tmem_ld_32x32b_x32(t_lane + kColG + 32, rb + 32);
-                tmem_ld_32x32b_x32(t_lane + kColG + 64, hc);
-                tmem_ld_32x32b_x32(t_lane + kColG + 96, hc + 32);
+                tmem_ld_32x32b_x32(t_lane + kColG + (uint32_t)(32 * half), rb);
+                tmem_ld_32x32b_x32(t_lane + kColG + 64 + (uint32_t)(32 * half), hc);
                 tmem_ld_wait();
             }
             float u = 0.f, v = 0.f;
             const float* dyr = p.dy + (tok * p.H + h) * kP;
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                float xv[8];
+            for (int qq = 0; qq < 4; ++qq) {
+                const int q = 4 * half + qq;
+                float xv[8], dv[8];
                 ld_row8(sb + kOffXI, row, q, xv);
+                if (valid) ld8(dyr, q, dv);
+                else {
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) dv[k] = 0.f;
+                }
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
-                    u = fmaf(xv[k], rb[8 * q + k], u);
-                    v = fmaf(valid ? __ldg(dyr + 8 * q + k) : 0.f, hc[8 * q + k], v);
+                    u = fmaf(xv[k], rb[8 * qq + k], u);
+                    v = fmaf(dv[k], hc[8 * qq + k], v);
                 }
             }
-            if (valid) {
+            const float2 uv = exchange(u, v);
+            if (valid && half == 0) {
                 const size_t o = bhc * p.S + tl, plane = (size_t)p.B * p.H * p.C * p.S;
-                p.scal[o] = u;
-                p.scal[plane + o] = v;
+                p.scal[o] = uv.x;
+                p.scal[plane + o] = uv.y;
             }
 #pragma unroll
-            for (int q = 0; q < 16; ++q) {
+            for (int qq = 0; qq < 8; ++qq) {
+                const int q = 8 * half + qq;
                 float bv[8];
                 ld_row8(sb + kOffBI, row, q, bv);
 #pragma unroll
@@ -385,7 +421,8 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_quad_tc(const __grid_con
         // ---- round 1: operands f x_i and exp(Acum) dy_i -----------------------
         wait_round();
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
+        for (int qq = 0; qq < 4; ++qq) {
+            const int q = 4 * half + qq;
             float xv[8], dv[8];
             ld_row8(sb + kOffXI, row, q, xv);
             ld_row8(sb + kOffDI, row, q, dv);
@@ -405,7 +442,9 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_quad_tc(const __grid_con
         for (int j = i; j < p.R; ++j) {
             // B_i C_j^T -> M_x
             wait_round();
-            for (int part = 0; part < 4; ++part) {
+#pragma unroll 1
+            for (int pp = 0; pp < 2; ++pp) {
+                const int part = 2 * half + pp;
                 float g[32];
                 if (ok) {
                     tmem_ld_32x32b_x32(t_lane + kColG + (uint32_t)(32 * part), g);
@@ -423,7 +462,9 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_quad_tc(const __grid_con
             // x_i dy_j^T -> W = dt_t M_x o G (s > t) summed over s (colsum of t)
             // and over t (this block's part of rowsum of s); M_b
             wait_round();
-            for (int part = 0; part < 4; ++part) {
+#pragma unroll 1
+            for (int pp = 0; pp < 2; ++pp) {
+                const int part = 2 * half + pp;
                 float g[32], mx[32], w[32];
                 if (ok) {
                     tmem_ld_32x32b_x32(t_lane + kColG + (uint32_t)(32 * part), g);
@@ -453,8 +494,8 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_quad_tc(const __grid_con
                 }
                 colred[quad * 128 + 32 * part + lane] = w[0];
             }
-            named_bar_sync(1, 128);
-            {   // column `row` of block j: the four warps' sums in order
+            named_bar_sync(1, 256);
+            if (half == 0) {   // column `row` of block j: the four quadrants' sums in order
                 const float rs = (colred[row] + colred[128 + row]) + (colred[256 + row] + colred[384 + row]);
                 const size_t plane = (size_t)p.B * p.H * p.C * p.S;
                 p.scal[(size_t)(4 + i) * plane + bhc * p.S + j * kRB + row] = rs;
@@ -468,7 +509,9 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_quad_tc(const __grid_con
         for (int j = 0; j <= i; ++j) {
             // dy_i x_j^T -> M_c
             wait_round();
-            for (int part = 0; part < 4; ++part) {
+#pragma unroll 1
+            for (int pp = 0; pp < 2; ++pp) {
+                const int part = 2 * half + pp;
                 float g[32];
                 if (ok) {
                     tmem_ld_32x32b_x32(t_lane + kColG + (uint32_t)(32 * part), g);
@@ -488,47 +531,47 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_quad_tc(const __grid_con
             if (j < i) done_round();   // the last round hands nothing back
         }
         // ---- outputs -----------------------------------------------------------
-        if (ok) {
+        {
             float q1 = 0.f;
-            float v[32];
-#pragma unroll
-            for (int part = 0; part < 2; ++part) {
-                tmem_ld_32x32b_x32(t_lane + kColDX + (uint32_t)(32 * part), v);
+            if (ok) {
+                float v[32], xv[32];
+                tmem_ld_32x32b_x32(t_lane + kColDX + (uint32_t)(32 * half), v);
                 tmem_ld_wait();
-                float xv[32];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) ld_row8(sb + kOffXI, row, 4 * part + q, xv + 8 * q);
+                for (int q = 0; q < 4; ++q) ld_row8(sb + kOffXI, row, 4 * half + q, xv + 8 * q);
 #pragma unroll
                 for (int k = 0; k < 32; ++k) q1 = fmaf(xv[k], v[k], q1);
                 if (valid) {
-                    float4* d4 = reinterpret_cast<float4*>(p.dx + (tok * p.H + h) * kP + 32 * part);
+                    float4* d4 = reinterpret_cast<float4*>(p.dx + (tok * p.H + h) * kP + 32 * half);
 #pragma unroll
                     for (int k = 0; k < 8; ++k)
                         d4[k] = make_float4(dtt * v[4 * k], dtt * v[4 * k + 1], dtt * v[4 * k + 2], dtt * v[4 * k + 3]);
                 }
-            }
+#pragma unroll 1
+                for (int pp = 0; pp < 2; ++pp) {
+                    const int part = 2 * half + pp;
+                    tmem_ld_32x32b_x32(t_lane + kColDB + (uint32_t)(32 * part), v);
+                    tmem_ld_wait();
+                    if (valid) {
+                        float4* d4 = reinterpret_cast<float4*>(p.dBh + (tok * p.H + h) * kN + 32 * part);
 #pragma unroll
-            for (int part = 0; part < 4; ++part) {
-                tmem_ld_32x32b_x32(t_lane + kColDB + (uint32_t)(32 * part), v);
-                tmem_ld_wait();
-                if (valid) {
-                    float4* d4 = reinterpret_cast<float4*>(p.dBh + (tok * p.H + h) * kN + 32 * part);
+                        for (int k = 0; k < 8; ++k)
+                            d4[k] = make_float4(dtt * v[4 * k], dtt * v[4 * k + 1], dtt * v[4 * k + 2], dtt * v[4 * k + 3]);
+                    }
+                    tmem_ld_32x32b_x32(t_lane + kColDC + (uint32_t)(32 * part), v);
+                    tmem_ld_wait();
+                    if (valid) {
+                        float4* d4 = reinterpret_cast<float4*>(p.dCh + (tok * p.H + h) * kN + 32 * part);
 #pragma unroll
-                    for (int k = 0; k < 8; ++k)
-                        d4[k] = make_float4(dtt * v[4 * k], dtt * v[4 * k + 1], dtt * v[4 * k + 2], dtt * v[4 * k + 3]);
+                        for (int k = 0; k < 8; ++k) d4[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+                    }
                 }
-                tmem_ld_32x32b_x32(t_lane + kColDC + (uint32_t)(32 * part), v);
-                tmem_ld_wait();
-                if (valid) {
-                    float4* d4 = reinterpret_cast<float4*>(p.dCh + (tok * p.H + h) * kN + 32 * part);
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) d4[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
-                }
             }
-            if (valid) {
+            const float2 qc = exchange(q1, colsum);    // both halves take part, also after a failed wait
+            if (ok && valid && half == 0) {
                 const size_t o = bhc * p.S + tl, plane = (size_t)p.B * p.H * p.C * p.S;
-                p.scal[2 * plane + o] = q1;
-                p.scal[3 * plane + o] = colsum;
+                p.scal[2 * plane + o] = qc.x;
+                p.scal[3 * plane + o] = qc.y;
             }
         }
     }
@@ -559,7 +602,9 @@ constexpr uint32_t ds_kSmemBytes = ds_kOffBar + 64 + 1024;
 enum DsBar { DS_LD = 0, DS_OPS = 1, DS_DONE = 2, ds_NUM_BARS = 3 };
 static_assert(ds_kSmemBytes <= 232448, "shared memory layout");
 
-__global__ void __launch_bounds__(kThreads, 1) scan_bwd_dS_tc(const __grid_constant__ ScanBwdTcParams p) {
+constexpr int kThreadsDS = 64 + 128;   // TMA, MMA, four row warps
+
+__global__ void __launch_bounds__(kThreadsDS, 1) scan_bwd_dS_tc(const __grid_constant__ ScanBwdTcParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sb = smem_u32(smem);
@@ -732,7 +777,7 @@ cudaError_t launch_scan_bwd_dS_tc(const ScanBwdArgs& a, cudaStream_t st) {
     if ((e = cudaFuncSetAttribute(scan_bwd_dS_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ds_kSmemBytes)) !=
         cudaSuccess)
         return e;
-    scan_bwd_dS_tc<<<a.B * a.H * p.C, kThreads, ds_kSmemBytes, st>>>(p);
+    scan_bwd_dS_tc<<<a.B * a.H * p.C, kThreadsDS, ds_kSmemBytes, st>>>(p);
     return cudaGetLastError();
 }
 
