@@ -20,7 +20,7 @@
 // recursions over the chunk's tokens.
 //
 // One CTA per (b, h, c, 128-token row block i) computes those for its rows:
-//   rounds 0-2   B_i R and C_i h_in (for u, v); dx += (f B_i) R,
+//   steps 0-2    B_i R and C_i h_in (for u, v); dx += (f B_i) R,
 //                dB += (f x_i) R^T, dC += (exp(Acum) dy_i) h_in^T;
 //   upper blocks j >= i:   G = B_i C_j^T -> M_x = mask o decay o G (bf16)
 //                dx += M_x dy_j;  G = x_i dy_j^T -> W = dt M_x o G: its sums over
@@ -28,7 +28,7 @@
 //                warps in order); M_b -> dB += M_b C_j;
 //   lower blocks j <= i:   G = dy_i x_j^T -> M_c -> dC += M_c B_j;
 // then dx, dB, dC leave TMEM and the scalars go to the workspace.  The
-// rounds run one after another (an MMA round, then the row threads).
+// steps run one after another (an MMA step, then the row threads).
 // TMEM: dx (64 columns), dB (128), dC (128), one 128-column scratch block.
 // Operands are bf16: B, C, x as given, dy, R, h_in and the M tiles rounded
 // once (2^-9 relative); products accumulate in fp32.
@@ -166,8 +166,8 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_quad_tc(const __grid_con
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
     const WaitCtx wc{abort_flag, p.status, 6};
-    // rounds: 0-2, then 3 per upper block (j = i .. R-1) and 2 per lower block (j = 0 .. i)
-    const int nrounds = 3 + 3 * (p.R - i) + 2 * (i + 1);
+    // steps: 0-2, then 3 per upper block (j = i .. R-1) and 2 per lower block (j = 0 .. i)
+    const int nsteps = 3 + 3 * (p.R - i) + 2 * (i + 1);
 
     if (warp == 0) {
         // ---------------------------------------------------------------- TMA
@@ -211,7 +211,7 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_quad_tc(const __grid_con
                 mma_f16_ss(d, ad, bd, idesc, (acc0 || kk > 0) ? 1u : 0u);
             }
         };
-        for (int r = 0; r < nrounds && ok; ++r) {
+        for (int r = 0; r < nsteps && ok; ++r) {
             if (r > 0 && !(ok = mbar_wait_warp(bar(OP_READY), (uint32_t)(r - 1) & 1u, wc, 3))) break;
             tc_fence_after();
             if (lane == 0) {
@@ -361,21 +361,21 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_quad_tc(const __grid_con
         const float e_t = exp2f(a2t);                  // exp(Acum_t)
         const float dtt = valid ? dtv[tl] : 0.f;
         float colsum = 0.f;
-        int rd = 0;                                    // MMA rounds completed
-        auto wait_round = [&]() {
+        int rd = 0;                                    // MMA steps completed
+        auto wait_step = [&]() {
             if (ok) ok = mbar_wait_warp(bar(MMA_DONE), (uint32_t)rd & 1u, wc, 5);
             ++rd;
             tc_fence_after();
         };
-        auto done_round = [&]() {
+        auto done_step = [&]() {
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(OP_READY));
         };
         const uint32_t op = sb + kOffOp;
-        // ---- round 0: u, v; operand f B_i -----------------------------------
-        wait_round();
+        // ---- step 0: u, v; operand f B_i -----------------------------------
+        wait_step();
         {
             float rb[32], hc[32];
             if (ok) {
@@ -417,9 +417,9 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_quad_tc(const __grid_con
                 st_row8(op, row, q, bv);
             }
         }
-        done_round();
-        // ---- round 1: operands f x_i and exp(Acum) dy_i -----------------------
-        wait_round();
+        done_step();
+        // ---- step 1: operands f x_i and exp(Acum) dy_i -----------------------
+        wait_step();
 #pragma unroll
         for (int qq = 0; qq < 4; ++qq) {
             const int q = 4 * half + qq;
@@ -434,14 +434,14 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_quad_tc(const __grid_con
             st_row8(op, row, q, xv);
             st_row8(op + kPanel, row, q, dv);
         }
-        done_round();
-        // ---- round 2: nothing to build --------------------------------------
-        wait_round();
-        done_round();
+        done_step();
+        // ---- step 2: nothing to build --------------------------------------
+        wait_step();
+        done_step();
         // ---- upper blocks -----------------------------------------------------
         for (int j = i; j < p.R; ++j) {
             // B_i C_j^T -> M_x
-            wait_round();
+            wait_step();
 #pragma unroll 1
             for (int pp = 0; pp < 2; ++pp) {
                 const int part = 2 * half + pp;
@@ -458,10 +458,10 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_quad_tc(const __grid_con
 #pragma unroll
                 for (int q = 0; q < 4; ++q) st_row8(op, row, 4 * part + q, g + 8 * q);
             }
-            done_round();
+            done_step();
             // x_i dy_j^T -> W = dt_t M_x o G (s > t) summed over s (colsum of t)
             // and over t (this block's part of rowsum of s); M_b
-            wait_round();
+            wait_step();
 #pragma unroll 1
             for (int pp = 0; pp < 2; ++pp) {
                 const int part = 2 * half + pp;
@@ -500,15 +500,15 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_quad_tc(const __grid_con
                 const size_t plane = (size_t)p.B * p.H * p.C * p.S;
                 p.scal[(size_t)(4 + i) * plane + bhc * p.S + j * kRB + row] = rs;
             }
-            done_round();
+            done_step();
             // dB += M_b C_j
-            wait_round();
-            done_round();
+            wait_step();
+            done_step();
         }
         // ---- lower blocks -----------------------------------------------------
         for (int j = 0; j <= i; ++j) {
             // dy_i x_j^T -> M_c
-            wait_round();
+            wait_step();
 #pragma unroll 1
             for (int pp = 0; pp < 2; ++pp) {
                 const int part = 2 * half + pp;
@@ -525,10 +525,10 @@ __global__ void __launch_bounds__(kThreads, 1) scan_bwd_quad_tc(const __grid_con
 #pragma unroll
                 for (int q = 0; q < 4; ++q) st_row8(op, row, 4 * part + q, g + 8 * q);
             }
-            done_round();
+            done_step();
             // dC += M_c B_j
-            wait_round();
-            if (j < i) done_round();   // the last round hands nothing back
+            wait_step();
+            if (j < i) done_step();   // the last step hands nothing back
         }
         // ---- outputs -----------------------------------------------------------
         {
