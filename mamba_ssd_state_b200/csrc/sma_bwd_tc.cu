@@ -25,8 +25,8 @@
 //   as four pairs (one per TMEM lane quadrant), each warp of a pair 32 of
 //   the 64 value columns, partial dot products exchanged in shared memory.
 //   TMEM: U, V double-buffered (2 x 128 columns), dQ (128), dC (128).
-// sma_bwd_dh_tc  one CTA per chunk memory of one (b, h): over the query
-//   tiles of the later chunks, ddH[c] (TMEM, 128 lanes n x 64 columns p) +=
+// sma_bwd_dh_tc  one CTA per pair of chunk memories of one (b, h): over the
+//   query tiles of the later chunks, ddH[c] (TMEM, 128 lanes n x 64 columns p) +=
 //   Q_T^T x [(ds / sqrt(N)) E_T] + C_T^T x [p do_T], with Q_T and C_T loaded
 //   by TMA and used as MN-major A operands, the scaled rows built by four
 //   warps as MN-major B operands.
@@ -433,15 +433,19 @@ __global__ void __launch_bounds__(qs::kThreads, 1) sma_bwd_q_tc(const __grid_con
 // memory side
 // ===========================================================================
 namespace ms {
-constexpr uint32_t kOffQ = 0;                   // 2 buffers x 2 panels
-constexpr uint32_t kOffC = 4 * kPanel;          // 2 buffers x 2 panels
-constexpr uint32_t kOffBE = 8 * kPanel;         // 2 buffers of (ds / sqrt(N)) E rows
-constexpr uint32_t kOffBD = 10 * kPanel;        // 2 buffers of p do rows
-constexpr uint32_t kOffBar = 12 * kPanel;
+// One CTA per pair of consecutive memories (c0 = 2m, c1 = 2m + 1) of one
+// (b, h): the query tiles of chunk c0 + 1 feed c0 alone, every later tile
+// feeds both, so each E and dy row a builder loads serves two memories and
+// each Q and C tile two products.
+constexpr uint32_t kOffQ = 0;                   // 2 panels (one buffer)
+constexpr uint32_t kOffC = 2 * kPanel;          // 2 panels (one buffer)
+constexpr uint32_t kOffOps = 4 * kPanel;        // 2 buffers x [E0, D0, E1, D1] operand rows
+constexpr uint32_t kOpsBuf = 4 * kPanel;
+constexpr uint32_t kOffBar = kOffOps + 2 * kOpsBuf;
 constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;
 constexpr int kBuilders = 4;
 constexpr int kThreads = 64 + 32 * kBuilders;
-enum Bar { QC_FULL0 = 0, QC_EMPTY0 = 2, OP_FULL0 = 4, OP_EMPTY0 = 6, D_FULL = 8, NUM_BARS = 9 };
+enum Bar { QC_FULL = 0, QC_EMPTY = 1, OP_FULL0 = 2, OP_EMPTY0 = 4, D_FULL = 6, NUM_BARS = 7 };
 static_assert(NUM_BARS * 8 + 8 <= 256 && kSmemBytes <= 232448, "shared memory layout");
 }  // namespace ms
 
@@ -454,20 +458,24 @@ __global__ void __launch_bounds__(ms::kThreads, 1) sma_bwd_dh_tc(const __grid_co
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
     auto bar = [&](int i) -> uint32_t { return sbase + kOffBar + 8u * (uint32_t)i; };
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // memory c of (b, h), in order of increasing c (most attending tokens first)
-    const int per_c = p.B * p.H;
-    const int c = blockIdx.x / per_c, bhi = blockIdx.x % per_c;
+    // memory pair m of (b, h), in order of increasing m (most attending tokens first)
+    const int per_m = p.B * p.H;
+    const int m = blockIdx.x / per_m, bhi = blockIdx.x % per_m;
     const int b = bhi / p.H, h = bhi % p.H;
     const size_t bh = (size_t)b * p.H + h;
-    // query tiles of chunks c+1 .. C-1 that start before L
-    int ntiles = (p.C - 1 - c) * p.tpc;
-    while (ntiles > 0 && (c + 1 + (ntiles - 1) / p.tpc) * p.S + ((ntiles - 1) % p.tpc) * kBQ >= p.L) --ntiles;
-    auto tile_t0 = [&](int j) { return (c + 1 + j / p.tpc) * p.S + (j % p.tpc) * kBQ; };
+    const int c0 = 2 * m, c1 = 2 * m + 1;
+    // query tiles of chunks c0+1 .. C-1 that start before L; tiles j >= tpc also attend c1
+    int ntiles = (p.C - 1 - c0) * p.tpc;
+    while (ntiles > 0 && (c0 + 1 + (ntiles - 1) / p.tpc) * p.S + ((ntiles - 1) % p.tpc) * kBQ >= p.L) --ntiles;
+    auto tile_t0 = [&](int j) { return (c0 + 1 + j / p.tpc) * p.S + (j % p.tpc) * kBQ; };
+    auto both = [&](int j) { return j >= p.tpc; };
+    const bool has_c1 = c1 < p.C;
+    const bool c1_tiles = has_c1 && ntiles > p.tpc;
 
     if (threadIdx.x == 0) {
+        mbar_init(bar(QC_FULL), 1);
+        mbar_init(bar(QC_EMPTY), 1);
         for (int i = 0; i < 2; ++i) {
-            mbar_init(bar(QC_FULL0 + i), 1);
-            mbar_init(bar(QC_EMPTY0 + i), 1);
             mbar_init(bar(OP_FULL0 + i), kBuilders);
             mbar_init(bar(OP_EMPTY0 + i), 1);
         }
@@ -480,7 +488,7 @@ __global__ void __launch_bounds__(ms::kThreads, 1) sma_bwd_dh_tc(const __grid_co
         tma_prefetch_desc(&p.tmap_c);
     }
     if (warp == 1) {
-        tmem_alloc(smem_u32(tmem_holder), 64);
+        tmem_alloc(smem_u32(tmem_holder), 128);   // ddH[c0] in columns 0-63, ddH[c1] in 64-127
         tmem_relinquish();
     }
     tc_fence_before();
@@ -492,16 +500,14 @@ __global__ void __launch_bounds__(ms::kThreads, 1) sma_bwd_dh_tc(const __grid_co
     if (warp == 0) {
         bool ok = true;
         for (int j = 0; j < ntiles && ok; ++j) {
-            const int buf = j & 1, t0 = tile_t0(j);
-            if (!(ok = mbar_wait_warp(bar(QC_EMPTY0 + buf), ((uint32_t)(j >> 1) & 1u) ^ 1u, wc, 1))) break;
+            const int t0 = tile_t0(j);
+            if (!(ok = mbar_wait_warp(bar(QC_EMPTY), ((uint32_t)j & 1u) ^ 1u, wc, 1))) break;
             if (lane == 0) {
-                const uint32_t qd = sbase + kOffQ + (uint32_t)buf * 2 * kPanel;
-                const uint32_t cd = sbase + kOffC + (uint32_t)buf * 2 * kPanel;
-                mbar_expect_tx(bar(QC_FULL0 + buf), 4 * kPanel);
-                tma_load_4d(qd, &p.tmap_q, bar(QC_FULL0 + buf), 0, h, t0, b);
-                tma_load_4d(qd + kPanel, &p.tmap_q, bar(QC_FULL0 + buf), 64, h, t0, b);
-                tma_load_4d(cd, &p.tmap_c, bar(QC_FULL0 + buf), 0, h / p.HG, t0, b);
-                tma_load_4d(cd + kPanel, &p.tmap_c, bar(QC_FULL0 + buf), 64, h / p.HG, t0, b);
+                mbar_expect_tx(bar(QC_FULL), 4 * kPanel);
+                tma_load_4d(sbase + kOffQ, &p.tmap_q, bar(QC_FULL), 0, h, t0, b);
+                tma_load_4d(sbase + kOffQ + kPanel, &p.tmap_q, bar(QC_FULL), 64, h, t0, b);
+                tma_load_4d(sbase + kOffC, &p.tmap_c, bar(QC_FULL), 0, h / p.HG, t0, b);
+                tma_load_4d(sbase + kOffC + kPanel, &p.tmap_c, bar(QC_FULL), 64, h / p.HG, t0, b);
             }
             __syncwarp();
         }
@@ -510,24 +516,26 @@ __global__ void __launch_bounds__(ms::kThreads, 1) sma_bwd_dh_tc(const __grid_co
         const uint32_t idesc = idesc_bf16_f32(kN, kP, true, true);   // A = Q^T, C^T (MN-major), B MN-major
         for (int j = 0; j < ntiles && ok; ++j) {
             const int buf = j & 1;
-            const uint32_t ph = (uint32_t)(j >> 1) & 1u;
-            if (!(ok = mbar_wait_warp(bar(QC_FULL0 + buf), ph, wc, 2))) break;
-            if (!(ok = mbar_wait_warp(bar(OP_FULL0 + buf), ph, wc, 3))) break;
+            if (!(ok = mbar_wait_warp(bar(QC_FULL), (uint32_t)j & 1u, wc, 2))) break;
+            if (!(ok = mbar_wait_warp(bar(OP_FULL0 + buf), (uint32_t)(j >> 1) & 1u, wc, 3))) break;
             tc_fence_after();
             if (lane == 0) {
-                const uint32_t qa = sbase + kOffQ + (uint32_t)buf * 2 * kPanel;
-                const uint32_t ca = sbase + kOffC + (uint32_t)buf * 2 * kPanel;
-                const uint32_t be = sbase + kOffBE + (uint32_t)buf * kPanel;
-                const uint32_t bdo = sbase + kOffBD + (uint32_t)buf * kPanel;
-#pragma unroll
-                for (int kk = 0; kk < kBQ / 16; ++kk) {
-                    const uint32_t ko = (uint32_t)kk * 2048;   // 16 token rows
-                    mma_f16_ss(tmem, smem_desc_sw128(qa + ko, kPanel, 1024), smem_desc_sw128(be + ko, kPanel, 1024),
-                               idesc, (j > 0 || kk > 0) ? 1u : 0u);
-                    mma_f16_ss(tmem, smem_desc_sw128(ca + ko, kPanel, 1024), smem_desc_sw128(bdo + ko, kPanel, 1024),
-                               idesc, 1u);
+                const uint32_t ops = sbase + kOffOps + (uint32_t)buf * kOpsBuf;
+                const int nmem = both(j) ? 2 : 1;
+                for (int mm = 0; mm < nmem; ++mm) {
+                    const uint32_t d = tmem + (uint32_t)(64 * mm);
+                    const bool first = mm == 0 ? j == 0 : j == p.tpc;
+                    const uint32_t be = ops + (uint32_t)(2 * mm) * kPanel, bdo = be + kPanel;
+#pragma unroll 1
+                    for (int kk = 0; kk < kBQ / 16; ++kk) {
+                        const uint32_t ko = (uint32_t)kk * 2048;   // 16 token rows
+                        mma_f16_ss(d, smem_desc_sw128(sbase + kOffQ + ko, kPanel, 1024),
+                                   smem_desc_sw128(be + ko, kPanel, 1024), idesc, (!first || kk > 0) ? 1u : 0u);
+                        mma_f16_ss(d, smem_desc_sw128(sbase + kOffC + ko, kPanel, 1024),
+                                   smem_desc_sw128(bdo + ko, kPanel, 1024), idesc, 1u);
+                    }
                 }
-                mma_commit(bar(QC_EMPTY0 + buf));
+                mma_commit(bar(QC_EMPTY));
                 mma_commit(bar(OP_EMPTY0 + buf));
                 if (j == ntiles - 1) mma_commit(bar(D_FULL));
             }
@@ -543,11 +551,20 @@ __global__ void __launch_bounds__(ms::kThreads, 1) sma_bwd_dh_tc(const __grid_co
             const int buf = j & 1, tok = tile_t0(j) + r;
             if (ok) ok = mbar_wait_warp(bar(OP_EMPTY0 + buf), ((uint32_t)(j >> 1) & 1u) ^ 1u, wc, 4);
             if (!ok) continue;
-            const uint32_t be = sbase + kOffBE + (uint32_t)buf * kPanel;
-            const uint32_t bdo = sbase + kOffBD + (uint32_t)buf * kPanel;
+            const uint32_t ops = sbase + kOffOps + (uint32_t)buf * kOpsBuf;
+            const int nmem = both(j) ? 2 : 1;
             if (tok < p.L) {
-                const size_t w = (bh * p.C + c) * p.L + tok;
-                const float dsn = __ldg(p.dsbuf + w) * inv_sqrt_n, pg = __ldg(p.pbuf + w) * p.g;
+                float dsn[2], pg[2];
+#pragma unroll
+                for (int mm = 0; mm < 2; ++mm) {
+                    if (mm < nmem) {
+                        const size_t w = (bh * p.C + c0 + mm) * p.L + tok;
+                        dsn[mm] = __ldg(p.dsbuf + w) * inv_sqrt_n;
+                        pg[mm] = __ldg(p.pbuf + w) * p.g;
+                    } else {
+                        dsn[mm] = pg[mm] = 0.f;
+                    }
+                }
                 const size_t orow = ((size_t)b * p.L + tok) * p.H + h;
                 const uint4* es = reinterpret_cast<const uint4*>(p.E + orow * kP);
                 const float4* dys = reinterpret_cast<const float4*>(p.dy + orow * kP);
@@ -556,39 +573,49 @@ __global__ void __launch_bounds__(ms::kThreads, 1) sma_bwd_dh_tc(const __grid_co
                     float ev[8];
                     widen8(__ldg(es + q), ev);
                     const float4 y0 = __ldg(dys + 2 * q), y1 = __ldg(dys + 2 * q + 1);
-                    st_shared_v4(sw128_chunk(be, r, q),
-                                 make_uint4(pack_bf16(dsn * ev[0], dsn * ev[1]), pack_bf16(dsn * ev[2], dsn * ev[3]),
-                                            pack_bf16(dsn * ev[4], dsn * ev[5]), pack_bf16(dsn * ev[6], dsn * ev[7])));
-                    st_shared_v4(sw128_chunk(bdo, r, q),
-                                 make_uint4(pack_bf16(pg * y0.x, pg * y0.y), pack_bf16(pg * y0.z, pg * y0.w),
-                                            pack_bf16(pg * y1.x, pg * y1.y), pack_bf16(pg * y1.z, pg * y1.w)));
+#pragma unroll
+                    for (int mm = 0; mm < 2; ++mm) {
+                        if (mm < nmem) {
+                            const float a = dsn[mm], g = pg[mm];
+                            st_shared_v4(sw128_chunk(ops + (uint32_t)(2 * mm) * kPanel, r, q),
+                                         make_uint4(pack_bf16(a * ev[0], a * ev[1]), pack_bf16(a * ev[2], a * ev[3]),
+                                                    pack_bf16(a * ev[4], a * ev[5]), pack_bf16(a * ev[6], a * ev[7])));
+                            st_shared_v4(sw128_chunk(ops + (uint32_t)(2 * mm + 1) * kPanel, r, q),
+                                         make_uint4(pack_bf16(g * y0.x, g * y0.y), pack_bf16(g * y0.z, g * y0.w),
+                                                    pack_bf16(g * y1.x, g * y1.y), pack_bf16(g * y1.z, g * y1.w)));
+                        }
+                    }
                 }
             } else {
                 const uint4 z = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    st_shared_v4(sw128_chunk(be, r, q), z);
-                    st_shared_v4(sw128_chunk(bdo, r, q), z);
-                }
+                for (int q = 0; q < 8; ++q)
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        if (k < 2 * nmem) st_shared_v4(sw128_chunk(ops + (uint32_t)k * kPanel, r, q), z);
             }
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(OP_FULL0 + buf));
         }
-        float* out = p.ddH + ((bh * p.C + c) * kN + r) * (size_t)kP;
-        if (ntiles == 0) {
-            const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+        // ddH[c0] and ddH[c1]: row r = state row n
+        const uint32_t t_lane = tmem + ((uint32_t)(quad * 32) << 16);
+        if (ntiles > 0 && ok) ok = mbar_wait_warp(bar(D_FULL), 0, wc, 5);
+        if (ok) tc_fence_after();
+#pragma unroll 1
+        for (int mm = 0; mm < 2; ++mm) {
+            if (mm == 1 && !has_c1) break;
+            float* out = p.ddH + ((bh * p.C + c0 + mm) * kN + r) * (size_t)kP;
+            const bool any = mm == 0 ? ntiles > 0 : c1_tiles;
+            if (!any) {
+                const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-            for (int q = 0; q < 16; ++q) reinterpret_cast<float4*>(out)[q] = z;
-        } else {
-            if (ok) ok = mbar_wait_warp(bar(D_FULL), 0, wc, 5);
-            if (ok) {
-                tc_fence_after();
-                const uint32_t t_lane = tmem + ((uint32_t)(quad * 32) << 16);
+                for (int q = 0; q < 16; ++q) reinterpret_cast<float4*>(out)[q] = z;
+            } else if (ok) {
 #pragma unroll
                 for (int part = 0; part < 2; ++part) {
                     float a[32];
-                    tmem_ld_32x32b_x32(t_lane + (uint32_t)(part * 32), a);
+                    tmem_ld_32x32b_x32(t_lane + (uint32_t)(64 * mm + 32 * part), a);
                     tmem_ld_wait();
 #pragma unroll
                     for (int q = 0; q < 8; ++q)
@@ -603,7 +630,7 @@ __global__ void __launch_bounds__(ms::kThreads, 1) sma_bwd_dh_tc(const __grid_co
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, 64);
+        tmem_dealloc(tmem, 128);
     }
 }
 
@@ -661,7 +688,7 @@ cudaError_t launch_sma_bwd_tc(const SmaBwdArgs& a, cudaStream_t st) {
         auto k = sma_bwd_dh_tc;
         if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ms::kSmemBytes)) != cudaSuccess)
             return e;
-        k<<<a.B * a.H * C, ms::kThreads, ms::kSmemBytes, st>>>(p);
+        k<<<a.B * a.H * ((C + 1) / 2), ms::kThreads, ms::kSmemBytes, st>>>(p);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     count_launches(2);
