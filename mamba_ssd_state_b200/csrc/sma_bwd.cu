@@ -275,11 +275,19 @@ __global__ void sma_bwd_reduce_dc(SmaBwdArgs a, int N) {
     a.dCm[i] = sum;
 }
 
-__global__ void sma_bwd_reduce_dg(SmaBwdArgs a, int nparts) {
-    if (threadIdx.x != 0 || blockIdx.x != 0) return;
+// dg = the sum of the tile partials: 256 threads each sum a fixed strided
+// subset, then a fixed tree (the same order on every run).
+__global__ void __launch_bounds__(256) sma_bwd_reduce_dg(SmaBwdArgs a, int nparts) {
+    __shared__ float part[256];
     float sum = 0.f;
-    for (int i = 0; i < nparts; ++i) sum += a.gpart[i];
-    a.dg[0] = sum;
+    for (int i = threadIdx.x; i < nparts; i += 256) sum += a.gpart[i];
+    part[threadIdx.x] = sum;
+    __syncthreads();
+    for (int w = 128; w > 0; w >>= 1) {
+        if (threadIdx.x < w) part[threadIdx.x] += part[threadIdx.x + w];
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) a.dg[0] = part[0];
 }
 
 template <typename T, int N, int P>
@@ -301,7 +309,7 @@ cudaError_t run(const SmaBwdArgs& a, cudaStream_t st) {
     const size_t ndc = (size_t)a.B * a.L * a.G * N;
     sma_bwd_reduce_dc<<<(unsigned)((ndc + 255) / 256), 256, 0, st>>>(a, N);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    sma_bwd_reduce_dg<<<1, 32, 0, st>>>(a, a.B * a.H * tiles);
+    sma_bwd_reduce_dg<<<1, 256, 0, st>>>(a, a.B * a.H * tiles);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     count_launches(4);
     return cudaSuccess;
@@ -339,7 +347,7 @@ cudaError_t launch_sma_bwd(SmaBwdArgs a, void* workspace, dart_dtype dt, cudaStr
         const size_t ndc = (size_t)a.B * a.L * a.G * a.N;
         sma_bwd_reduce_dc<<<(unsigned)((ndc + 255) / 256), 256, 0, st>>>(a, a.N);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        sma_bwd_reduce_dg<<<1, 32, 0, st>>>(a, sma_bwd_tc_tiles(a.B, a.L, a.H, a.S));
+        sma_bwd_reduce_dg<<<1, 256, 0, st>>>(a, sma_bwd_tc_tiles(a.B, a.L, a.H, a.S));
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         count_launches(2);
         return cudaSuccess;
