@@ -44,6 +44,13 @@ from mamba_ssd_state_b200 import synth  # noqa: E402
 FWD = synth.TRAIN_L8K
 DEC = synth.DECODE_64x32K
 METRIC = "DART layer fwd tokens/s at L=8K (% BF16 peak); decode tokens/s (% HBM BW)"
+
+
+def fwd_config(world: int) -> dict:
+    """The headline workload's `config`, the same object on both arms."""
+    return {"workload": "dart_layer_fwd_L8k", "batch": FWD.batch, "seqlen": FWD.seqlen, "nheads": FWD.nheads,
+            "headdim": FWD.headdim, "dstate": FWD.dstate, "chunk": FWD.chunk, "ngroups": 1,
+            "parallelism": f"dp{world}", "l2": "inputs larger than L2 (272 MiB per step)"}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
                   "sm_max_mhz": 1965.0}
 SMS = 148
@@ -561,9 +568,7 @@ def run_reference(args):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": "dart_layer_fwd_L8k", "batch": FWD.batch,
-                                            "seqlen": FWD.seqlen, "nheads": FWD.nheads,
-                                            "headdim": FWD.headdim, "dstate": FWD.dstate, "chunk": FWD.chunk},
+            "data": "synthetic", "config": fwd_config(args.gpus),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": min(nthreads, len(heads)),
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -615,10 +620,7 @@ def main():
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": dist.world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": "dart_layer_fwd_L8k", "batch": FWD.batch, "seqlen": FWD.seqlen,
-                       "nheads": FWD.nheads, "headdim": FWD.headdim, "dstate": FWD.dstate, "chunk": FWD.chunk,
-                       "ngroups": 1, "parallelism": f"dp{dist.world}",
-                       "l2": "inputs larger than L2 (272 MiB per step)"},
+            "config": fwd_config(dist.world),
             "gpu_launches": fwd["launches"],
             "clocks": fwd["clocks"],
             "roofline": roof,

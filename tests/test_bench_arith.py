@@ -8,6 +8,7 @@ that `roofline.achieved` divides by the measured kernel time.
   (P + 1) / (2 P) of a bf16 one.
 * The workload figures quoted in the design notes (266.29 and 26.07 GFLOP,
   4.565 GB per decode step on average) are what the functions return.
+* Both arms (kernels and oracle) name the headline workload with one config.
 """
 import os
 import sys
@@ -46,3 +47,15 @@ def test_decode_bytes_structure():
     # the average over the 256 timed steps (the last one appends), as quoted
     steps = [bench.decode_bytes(d, d.ncached + s // d.chunk, s % d.chunk == d.chunk - 1) for s in range(256)]
     assert sum(steps) / 256 == pytest.approx(4.565147648e9, rel=1e-12)
+
+
+def test_both_arms_share_the_headline_config():
+    """The reference arm and the kernel arm report the same `config` object,
+    so a driver comparing them sees the same workload."""
+    import inspect
+    cfg = bench.fwd_config(4)
+    assert cfg["workload"] == "dart_layer_fwd_L8k" and cfg["parallelism"] == "dp4" and cfg["ngroups"] == 1
+    assert (cfg["batch"], cfg["seqlen"], cfg["nheads"], cfg["headdim"], cfg["dstate"], cfg["chunk"]) == \
+        (2, 8192, 32, 64, 128, 256)
+    assert "fwd_config(args.gpus)" in inspect.getsource(bench.run_reference)
+    assert "fwd_config(dist.world)" in inspect.getsource(bench.main)
