@@ -157,49 +157,129 @@ def decode_bytes(d: synth.DecodeShape, n: int, append: bool, e4m3: bool = False)
 # clocks during the timed region
 # ---------------------------------------------------------------------------
 class ClockSampler:
+    """SM clock, power and clock-event reasons of one GPU.
+
+    Two sources: `nvidia-smi -lms 100` over the whole window (start .. stop),
+    and an NVML poll every millisecond from a thread that keeps only the
+    samples taken between begin() and end(), the timed region (a region of
+    a few milliseconds falls between two nvidia-smi samples).  The median
+    clock is taken from the in-region NVML samples when there are any; the
+    reasons are the union of both sources.  The GPU is found by its UUID."""
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits, in the order of the names reported
+    REASON_BITS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+                   ("sw_power_cap", 0x4))
 
-    def __init__(self, index: int):
+    def __init__(self, index: int, uuid: str | None = None, nvml=None):
         self.index = index
+        self.uuid = uuid
         self.proc = None
         self.path = None
+        self.nvml = nvml
+        self.handle = None
+        self.thread = None
+        self.active = False
+        self.running = False
+        self.samples = []     # (sm MHz, reason bits, power W) inside the region
+
+    @staticmethod
+    def device_uuid(dev: torch.device) -> str | None:
+        try:
+            u = str(torch.cuda.get_device_properties(dev).uuid)
+            return u if u.startswith("GPU-") else "GPU-" + u
+        except (AttributeError, RuntimeError):
+            return None
+
+    def _open_nvml(self):
+        try:
+            if self.nvml is None:
+                import pynvml
+                self.nvml = pynvml
+            self.nvml.nvmlInit()
+            try:
+                self.handle = self.nvml.nvmlDeviceGetHandleByUUID(self.uuid) if self.uuid else None
+            except Exception:
+                self.handle = None
+            if self.handle is None:
+                self.uuid = None
+                self.handle = self.nvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = float(self.nvml.nvmlDeviceGetMaxClockInfo(self.handle, self.nvml.NVML_CLOCK_SM))
+        except Exception:   # no NVML: nvidia-smi alone
+            self.handle = None
+
+    def _poll(self):
+        nv, h = self.nvml, self.handle
+        while self.running:
+            if self.active:
+                try:
+                    self.samples.append((float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)),
+                                         int(nv.nvmlDeviceGetCurrentClocksEventReasons(h)),
+                                         nv.nvmlDeviceGetPowerUsage(h) / 1000.0))
+                except Exception:
+                    self.running = False
+                    break
+            time.sleep(0.001)
 
     def start(self):
+        self._open_nvml()
+        # the UUID names the GPU for nvidia-smi too, once NVML has accepted it
+        target = self.uuid if (self.handle is not None and self.uuid) else str(self.index)
         try:
             fd, self.path = tempfile.mkstemp(suffix=".csv")
             os.close(fd)
             self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                ["nvidia-smi", "-i", target, f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
                  "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
+        if self.handle is not None:
+            import threading
+            self.running = True
+            self.thread = threading.Thread(target=self._poll, daemon=True)
+            self.thread.start()
+
+    def begin(self):
+        self.active = True
+
+    def end(self):
+        self.active = False
 
     def stop(self) -> dict:
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
+        self.active = False
+        if self.thread is not None:
+            self.running = False
+            self.thread.join(timeout=5)
         rows = []
-        with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) >= 9:
-                    rows.append(parts)
-        os.unlink(self.path)
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            with open(self.path) as f:
+                for line in f:
+                    parts = [p.strip() for p in line.split(",")]
+                    if len(parts) >= 9:
+                        rows.append(parts)
+            os.unlink(self.path)
+        if not rows and not self.samples:
+            why = "nvidia-smi unavailable" if self.proc is None else "no samples"
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [why]}
+        names = [n for n, _ in self.REASON_BITS]
+        reasons = {names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"}
+        reasons |= {n for (_, bits, _) in self.samples for n, b in self.REASON_BITS if bits & b}
+        sm_smi = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        sm_in = [c for c, _, _ in self.samples]
         mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        if self.handle is not None:
+            mx.append(self.max_mhz)
+        power = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()] + [w for _, _, w in self.samples]
+        sm = sm_in or sm_smi
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows),
-                "power_w_max": max((float(r[3]) for r in rows if r[3].replace(".", "").isdigit()), default=None)}
+                "reasons": sorted(reasons), "samples": len(rows) + len(self.samples),
+                "region_samples": len(self.samples), "power_w_max": max(power, default=None)}
 
 
 # ---------------------------------------------------------------------------
@@ -277,17 +357,19 @@ def forward_region(args, dist, dart, shape=FWD, decayed=False):
     dart.dart_sync_status()
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    clocks = ClockSampler(dev.index)
+    clocks = ClockSampler(dev.index, ClockSampler.device_uuid(dev))
     clocks.start()
     time.sleep(0.25)
     dist.barrier()
     torch.cuda.synchronize()
     n0 = dart.launch_count()
+    clocks.begin()
     start.record(stream)
     for i in range(args.steps):
         step(evs[i])
     end.record(stream)
     torch.cuda.synchronize()
+    clocks.end()
     n1 = dart.launch_count()
     dist.barrier()
     clk = clocks.stop()
@@ -459,17 +541,19 @@ def decode_region(args, dist, dart, peaks, decayed=False, e4m3=False):
     del saved
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(nsteps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    clocks = ClockSampler(dev.index)
+    clocks = ClockSampler(dev.index, ClockSampler.device_uuid(dev))
     clocks.start()
     time.sleep(0.25)
     dist.barrier()
     torch.cuda.synchronize()
     n0 = dart.launch_count()
+    clocks.begin()
     start.record(stream)
     for s in range(nsteps):
         step(s, evs[s])
     end.record(stream)
     torch.cuda.synchronize()
+    clocks.end()
     n1 = dart.launch_count()
     dist.barrier()
     clk = clocks.stop()
