@@ -484,11 +484,17 @@ __global__ void __launch_bounds__(N * P / kCols) scan_bwd_walk(ScanBwdArgs a) {
 //   Rect_t = Rect_{t+1} + rowsum_t - colsum_t,   gh_t = v_t + a_{t+1} gh_{t+1},
 //   rd_t = E_{t-1},  E_t = a_t E_{t-1} + dt_t u_t,
 //   dl_t = exp(Acum_t) gh_t + Rect_t + exp(Ae) c0 + exp(Ae - Acum_{t-1}) rd_t,
-//   ddt_t = q1_t + A_h dl_t,  dA += dt_t dl_t.
-// One warp per chunk: the lanes stage the chunk's scalars in shared memory,
-// lane 0 runs the three recursions.
+//   ddt_t = q1_t + A_h dl_t,  dA += dt_t dl_t,
+// with a_t = exp(dt_t A_h) (a_S = 0: nothing follows the chunk's last token).
+// One warp per chunk; the lanes stage the chunk's scalars in shared memory and
+// lane l then owns tokens 8l .. 8l+7.  Each recursion is linear, so each is a
+// warp scan: the prefix of dt A and the suffix of rowsum - colsum are sums;
+// gh (backward) and E (forward) compose per-lane affine maps x -> K + M x, so
+// every lane learns the value entering its tokens and finishes them itself.
 __global__ void __launch_bounds__(32) scan_bwd_scalars(ScanBwdArgs a, int C) {
-    __shared__ float sdt[256], sacum[256], su[256], sv[256], sq[256], srw[256], scl[256];
+    constexpr int K = 8;        // tokens per lane; the chunk has at most 256
+    constexpr unsigned kAll = 0xffffffffu;
+    __shared__ float sdt[256], su[256], sv[256], sq[256], srw[256], scl[256];
     const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z, lane = threadIdx.x;
     const size_t bhc = ((size_t)b * a.H + h) * C + c;
     const ChunkSpan cs(c, a.S, a.L);
@@ -504,32 +510,117 @@ __global__ void __launch_bounds__(32) scan_bwd_scalars(ScanBwdArgs a, int C) {
         srw[t] = sc[4 * plane + t] + (t >= 128 ? sc[5 * plane + t] : 0.f);
     }
     __syncwarp();
-    if (lane != 0) return;
     const float Ah = a.A[h];
-    float run = 0.f;
-    for (int t = 0; t < cs.n; ++t) {
-        run += sdt[t] * Ah;
-        sacum[t] = run;
+    const int t0 = K * lane;
+    const int nt = max(0, min(K, cs.n - t0));   // this lane's tokens
+    float dtv[K], av[K], acum[K];
+    float loc = 0.f;
+#pragma unroll
+    for (int j = 0; j < K; ++j) {
+        dtv[j] = j < nt ? sdt[t0 + j] : 0.f;
+        av[j] = expf(dtv[j] * Ah);
+        loc += dtv[j] * Ah;
+        acum[j] = loc;
     }
-    const float Ae = run, eAc0 = expf(Ae) * a.c0[bhc];
-    // backward: gh (into sv) and Rect (into srw)
-    float gh = 0.f, rect = 0.f;
-    for (int t = cs.n - 1; t >= 0; --t) {
-        gh = t + 1 < cs.n ? fmaf(expf(sdt[t + 1] * Ah), gh, sv[t]) : sv[t];
-        rect += srw[t] - scl[t];
-        sv[t] = gh;
-        srw[t] = rect;
+    // Acum: inclusive prefix of the lanes' sums, then the exclusive part
+    float incl = loc;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const float up = __shfl_up_sync(kAll, incl, d);
+        if (lane >= d) incl += up;
     }
-    // forward: rd, dl, ddt, dA
-    float E = 0.f, dA = 0.f;
-    for (int t = 0; t < cs.n; ++t) {
-        const float am1 = t > 0 ? sacum[t - 1] : 0.f;
-        const float dl = expf(sacum[t]) * sv[t] + srw[t] + eAc0 + expf(Ae - am1) * E;
-        a.ddt[((size_t)b * a.L + cs.s0 + t) * a.H + h] = sq[t] + Ah * dl;
-        dA = fmaf(sdt[t], dl, dA);
-        E = fmaf(expf(sdt[t] * Ah), E, sdt[t] * su[t]);
+    float before = __shfl_up_sync(kAll, incl, 1);   // Acum of the token before this lane's first
+    if (lane == 0) before = 0.f;
+#pragma unroll
+    for (int j = 0; j < K; ++j) acum[j] += before;
+    const float Ae = __shfl_sync(kAll, incl, 31);
+    const float eAc0 = expf(Ae) * a.c0[bhc];
+    // a_{t+1} of each of this lane's tokens: the next lane's first for the last
+    const float a_first_next = __shfl_down_sync(kAll, av[0], 1);
+    auto a_next = [&](int j) -> float {
+        if (t0 + j + 1 >= cs.n) return 0.f;
+        return j + 1 < K ? av[j + 1] : a_first_next;
+    };
+    // gh, backward: this lane's map from gh entering from the right to gh at
+    // its first token, composed with the maps of the later lanes
+    float M = 1.f, Kc = 0.f;
+#pragma unroll
+    for (int j = K - 1; j >= 0; --j) {
+        if (j < nt) {
+            const float an = a_next(j);
+            Kc = fmaf(an, Kc, sv[t0 + j]);
+            M *= an;
+        }
     }
-    a.dApart[bhc] = dA;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const float M2 = __shfl_down_sync(kAll, M, d), K2 = __shfl_down_sync(kAll, Kc, d);
+        if (lane + d < 32) {
+            Kc = fmaf(M, K2, Kc);
+            M *= M2;
+        }
+    }
+    float x = __shfl_down_sync(kAll, Kc, 1);   // gh at the next lane's first token
+    if (lane == 31) x = 0.f;
+    float gh[K];
+#pragma unroll
+    for (int j = K - 1; j >= 0; --j) {
+        if (j < nt) x = fmaf(a_next(j), x, sv[t0 + j]);
+        gh[j] = x;
+    }
+    // Rect, backward: suffix sums
+    float seg = 0.f;
+#pragma unroll
+    for (int j = 0; j < K; ++j)
+        if (j < nt) seg += srw[t0 + j] - scl[t0 + j];
+    float suf = seg;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const float dn = __shfl_down_sync(kAll, suf, d);
+        if (lane + d < 32) suf += dn;
+    }
+    float r = __shfl_down_sync(kAll, suf, 1);   // the later lanes' sum
+    if (lane == 31) r = 0.f;
+    float rect[K];
+#pragma unroll
+    for (int j = K - 1; j >= 0; --j) {
+        if (j < nt) r += srw[t0 + j] - scl[t0 + j];
+        rect[j] = r;
+    }
+    // E, forward: this lane's map from E before its first token to E after
+    // its last, composed with the maps of the earlier lanes
+    float Nm = 1.f, Pm = 0.f;
+#pragma unroll
+    for (int j = 0; j < K; ++j) {
+        if (j < nt) {
+            Pm = fmaf(av[j], Pm, dtv[j] * su[t0 + j]);
+            Nm *= av[j];
+        }
+    }
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const float N2 = __shfl_up_sync(kAll, Nm, d), P2 = __shfl_up_sync(kAll, Pm, d);
+        if (lane >= d) {
+            Pm = fmaf(Nm, P2, Pm);
+            Nm *= N2;
+        }
+    }
+    float E = __shfl_up_sync(kAll, Pm, 1);   // E before this lane's first token
+    if (lane == 0) E = 0.f;
+    float dA = 0.f;
+#pragma unroll
+    for (int j = 0; j < K; ++j) {
+        if (j < nt) {
+            const int t = t0 + j;
+            const float am1 = j > 0 ? acum[j - 1] : before;
+            const float dl = expf(acum[j]) * gh[j] + rect[j] + eAc0 + expf(Ae - am1) * E;
+            a.ddt[((size_t)b * a.L + cs.s0 + t) * a.H + h] = sq[t] + Ah * dl;
+            dA = fmaf(dtv[j], dl, dA);
+            E = fmaf(av[j], E, dtv[j] * su[t]);
+        }
+    }
+    dA = warp_sum(dA);
+    if (lane == 0) a.dApart[bhc] = dA;
 }
 
 // dB, dC [B,L,G,N] summed over the heads of each group (dC plus dC_add when
