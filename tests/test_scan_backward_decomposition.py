@@ -8,8 +8,10 @@ crossing sum Rect_t = sum_{r<t<=s} W_{s,r} and the running sums of u and v).
 This test writes that decomposition out in float64 numpy and compares it with
 the C oracle's reverse-mode walk of the token recurrence: the two must agree
 to rounding (1e-10), on grouped B and C, a ragged last chunk, an initial
-state and a memory gradient.  It uses only the seeded input generator and
-the oracle; no compiled library is loaded."""
+state and a memory gradient.  A second test checks the scalar kernel's
+warp-scan form of the decay-gradient recursions against the recursions.  It
+uses only the seeded input generator and the oracle; no compiled library is
+loaded."""
 import numpy as np
 import pytest
 
@@ -107,3 +109,122 @@ def test_chunked_scan_backward_equals_token_walk(Bz, L, H, P, N, S, G, init, mem
     for k in ("dx", "ddt", "dA", "dBm", "dCm") + (("dinit_state",) if init else ()):
         err = np.max(np.abs(got[k] - ref[k])) / max(np.max(np.abs(ref[k])), 1e-300)
         assert err <= 1e-10, (k, err)
+
+
+# ---------------------------------------------------------------------------
+# The per-chunk decay-gradient recursions, sequential and as warp scans.
+# The scalar kernel of the scan backward runs these recursions over a chunk's
+# tokens, eight per lane of one warp:
+#   Rect_t = Rect_{t+1} + rowsum_t - colsum_t,
+#   gh_t = v_t + a_{t+1} gh_{t+1},
+#   E_t = a_t E_{t-1} + dt_t u_t,
+# each as a scan of per-lane sums or affine maps.  The two functions below
+# are that decomposition, written out lane by lane with Hillis-Steele steps,
+# and the recursions themselves; they must agree to rounding for any chunk
+# length.
+# ---------------------------------------------------------------------------
+def _recursions_sequential(dt, A, u, v, q, rw, cl, c0):
+    n = len(dt)
+    acum = np.cumsum(dt * A)
+    Ae = acum[-1]
+    gh, rect = np.zeros(n), np.zeros(n)
+    g = r = 0.0
+    for t in range(n - 1, -1, -1):
+        g = v[t] + (np.exp(dt[t + 1] * A) * g if t + 1 < n else 0.0)
+        r += rw[t] - cl[t]
+        gh[t], rect[t] = g, r
+    E = dA = 0.0
+    ddt = np.zeros(n)
+    for t in range(n):
+        am1 = acum[t - 1] if t > 0 else 0.0
+        dl = np.exp(acum[t]) * gh[t] + rect[t] + np.exp(Ae) * c0 + np.exp(Ae - am1) * E
+        ddt[t] = q[t] + A * dl
+        dA += dt[t] * dl
+        E = np.exp(dt[t] * A) * E + dt[t] * u[t]
+    return ddt, dA
+
+
+def _scan(vals, combine, reverse):
+    """Inclusive Hillis-Steele scan over 32 lanes (toward lower lanes when
+    reverse), combine(mine, other) with `other` the farther lanes' partial."""
+    vals = list(vals)
+    d = 1
+    while d < 32:
+        nxt = list(vals)
+        for l in range(32):
+            o = l + d if reverse else l - d
+            if 0 <= o < 32:
+                nxt[l] = combine(vals[l], vals[o])
+        vals, d = nxt, 2 * d
+    return vals
+
+
+def _recursions_warp(dt, A, u, v, q, rw, cl, c0, K=8):
+    n = len(dt)
+    tok = [[t for t in range(K * l, K * l + K) if t < n] for l in range(32)]
+    a = lambda t: np.exp(dt[t] * A) if t < n else 0.0   # nothing follows the chunk
+    # prefix of dt A
+    tot = [sum(dt[t] * A for t in ts) for ts in tok]
+    incl = _scan(tot, lambda m, o: m + o, reverse=False)
+    acum = np.zeros(n)
+    for l, ts in enumerate(tok):
+        run = incl[l - 1] if l > 0 else 0.0
+        for t in ts:
+            run += dt[t] * A
+            acum[t] = run
+    Ae = incl[31]
+    # gh: map x -> K + M x from gh after the lane to gh at its first token
+    maps = []
+    for ts in tok:
+        M, Kc = 1.0, 0.0
+        for t in reversed(ts):
+            Kc, M = v[t] + a(t + 1) * Kc, a(t + 1) * M
+        maps.append((M, Kc))
+    suf = _scan(maps, lambda m, o: (m[0] * o[0], m[1] + m[0] * o[1]), reverse=True)
+    gh = np.zeros(n)
+    for l, ts in enumerate(tok):
+        x = suf[l + 1][1] if l < 31 else 0.0
+        for t in reversed(ts):
+            x = v[t] + a(t + 1) * x
+            gh[t] = x
+    # Rect: suffix sums
+    seg = [sum(rw[t] - cl[t] for t in ts) for ts in tok]
+    ssum = _scan(seg, lambda m, o: m + o, reverse=True)
+    rect = np.zeros(n)
+    for l, ts in enumerate(tok):
+        r = ssum[l + 1] if l < 31 else 0.0
+        for t in reversed(ts):
+            r += rw[t] - cl[t]
+            rect[t] = r
+    # E: map y -> P + N y from E before the lane to E after it
+    maps = []
+    for ts in tok:
+        N_, P_ = 1.0, 0.0
+        for t in ts:
+            P_, N_ = a(t) * P_ + dt[t] * u[t], a(t) * N_
+        maps.append((N_, P_))
+    pre = _scan(maps, lambda m, o: (m[0] * o[0], m[1] + m[0] * o[1]), reverse=False)
+    ddt, dA = np.zeros(n), 0.0
+    for l, ts in enumerate(tok):
+        E = pre[l - 1][1] if l > 0 else 0.0
+        for t in ts:
+            am1 = acum[t - 1] if t > 0 else 0.0
+            dl = np.exp(acum[t]) * gh[t] + rect[t] + np.exp(Ae) * c0 + np.exp(Ae - am1) * E
+            ddt[t] = q[t] + A * dl
+            dA += dt[t] * dl
+            E = a(t) * E + dt[t] * u[t]
+    return ddt, dA
+
+
+@pytest.mark.parametrize("n", [1, 8, 9, 33, 128, 129, 255, 256])
+@pytest.mark.parametrize("heavy", [False, True])
+def test_decay_gradient_recursions_as_warp_scans(n, heavy):
+    r = np.random.default_rng(n + 7 * heavy)
+    A = -16.0 if heavy else -1.0
+    dt = np.full(n, 0.1) if heavy else np.exp(r.uniform(np.log(1e-3), np.log(1e-1), n))
+    u, v, q, rw, cl = (r.standard_normal(n) for _ in range(5))
+    c0 = r.standard_normal()
+    d1, a1 = _recursions_sequential(dt, A, u, v, q, rw, cl, c0)
+    d2, a2 = _recursions_warp(dt, A, u, v, q, rw, cl, c0)
+    assert np.max(np.abs(d1 - d2)) <= 1e-12 * np.max(np.abs(d1))
+    assert abs(a1 - a2) <= 1e-12 * abs(a1)
