@@ -279,3 +279,17 @@ def test_binding_fails_loudly_without_cuda(lib):
         dart.dart_ssd_chunk_scan(x, torch.zeros(1, 256, 1), torch.zeros(1),
                                  torch.zeros(1, 256, 128, dtype=torch.bfloat16),
                                  torch.zeros(1, 256, 128, dtype=torch.bfloat16), 256)
+
+
+def test_backward_rejects_groups_that_do_not_divide_heads(lib):
+    """ngroups must divide nheads in the backward calls too (B, C and their
+    gradients are [B, L, G, N], head h reading group h / (H / G))."""
+    d = dart.Dims(2, 500, 3, 64, 128, 256, 2)
+    f = lib.dart_sma_backward
+    assert f(ctypes.byref(d), dart.DART_BF16, FAKE, FAKE, FAKE, FAKE, 0.5, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+             FAKE, 1 << 40, None) == dart.DART_ERR_INVALID_ARG
+    assert b"ngroups" in lib.dart_last_error()
+    ok = [FAKE] * 5 + [None, FAKE, FAKE, None, None] + [FAKE] * 5 + [None, FAKE]
+    assert lib.dart_ssd_scan_backward(ctypes.byref(d), dart.DART_BF16, *ok, 1 << 40, None) == \
+        dart.DART_ERR_INVALID_ARG
+    assert b"ngroups" in lib.dart_last_error()
