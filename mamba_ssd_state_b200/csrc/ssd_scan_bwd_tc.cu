@@ -17,7 +17,7 @@
 // column sums, so both sums are taken from the same W values (each pair once,
 // in the upper blocks): a W rounded two different ways cancels badly there.
 // scan_bwd_scalars (ssd_scan_bwd.cu) turns them into ddt and dA by three
-// recursions over the chunk's tokens.
+// recursions over the chunk's tokens, each run as a warp scan.
 //
 // One CTA per (b, h, c, 128-token row block i) computes those for its rows:
 //   steps 0-2    B_i R and C_i h_in (for u, v); dx += (f B_i) R,
