@@ -28,9 +28,11 @@
 //      own barrier pair.
 //
 // Decay factors: exp(Acum_t - Acum_s) = exp(Acum_t - Acum_r) exp(Acum_r -
-// Acum_s) with r the first token of the 32-token column block holding s; both
-// factors stay inside float range (the second is at most exp(32 |a|max)), so
-// only one exponential per (row, block) and one per column are needed.
+// Acum_s) with r the first token of the 32-token column block holding s.  The
+// column factor is at most exp(32 |a|max) dt_s, inside float range; the row
+// factor is at most 1 and underflows only where the term is below about 2^-75
+// of the diagonal's, which then counts as 0.  So one exponential per (row,
+// block) and one per column are needed.
 #include <cuda_bf16.h>
 #include <string.h>
 
